@@ -1,0 +1,68 @@
+"""Oracle pins on the synthetic workloads (CPU only).
+
+* Planted needles (the 2k-context needle workload): with envelope scoring and
+  the group max, every needle page of every KV head is among the top 16.
+* The budget is page_size x top_k tokens ("The comparison", Offline Replay
+  Records card): top-16 of 16-token pages attends to 256 tokens.
+* The chunk generator honours the 16-256 token range of structure-aligned
+  chunks (only the final chunk may be shorter).
+"""
+import math
+
+import numpy as np
+import torch
+
+import datagen as DG
+import oracle as O
+
+
+def _np(x):
+    return x.float().numpy().astype(np.float64)
+
+
+def test_needles_selected_envelope():
+    lay = DG.workload1_layer("cpu")
+    w = DG.WORKLOADS[1]
+    G = w.Hq // w.Hkv
+    for g in range(w.Hkv):
+        r = O.decode_unit(_np(lay.q[0, g * G:(g + 1) * G]), _np(lay.k[0, g]), _np(lay.v[0, g]),
+                          w.N, rule="envelope", page_size=16,
+                          budget={"kind": "topk", "k": 16}, scale=1 / math.sqrt(128))
+        assert set(lay.extra["needle_pages"][g]) <= set(r.selected.tolist())
+        assert r.n_tokens == 16 * 16
+
+
+def test_chunk_generator_ranges():
+    for lens in DG.workload3_chunks(4, 29504):
+        assert lens.sum() == 29504
+        assert lens[:-1].min() >= 16 and lens.max() <= 256
+        assert 150 <= len(lens) <= 300
+
+
+def test_token_budget_fills_without_overflow():
+    """Greedy token budget on a chunked workload: never above the budget, and
+    the first chunk in rank order that was not taken would overflow it."""
+    lay = DG.workload3_layer(0, "cpu", N=4096, B=1)
+    off = lay.chunk_off[0, :int(lay.n_chunks[0]) + 1].numpy()
+    w = DG.WORKLOADS[3]
+    G = w.Hq // w.Hkv
+    for budget in (512, 1024, 4096):
+        r = O.decode_unit(_np(lay.q[0, 0:G]), _np(lay.k[0, 0]), _np(lay.v[0, 0]), 4096,
+                          rule="envelope", chunk_off=off,
+                          budget={"kind": "tokens", "budget": budget}, scale=1 / math.sqrt(128))
+        lens = np.diff(off)
+        assert r.n_tokens == lens[r.selected].sum() <= budget
+        order = O.rank_order(r.scores)
+        rest = [p for p in order if p not in set(r.selected.tolist())]
+        if rest:
+            assert r.n_tokens + lens[rest[0]] > budget
+        if budget >= 4096:
+            assert r.n_tokens == 4096
+
+
+def test_datagen_is_seeded():
+    a = DG.workload2_layer(3, "cpu", N=64)
+    b = DG.workload2_layer(3, "cpu", N=64)
+    assert torch.equal(a.k, b.k) and torch.equal(a.q, b.q) and torch.equal(a.v, b.v)
+    c = DG.workload2_layer(4, "cpu", N=64)
+    assert not torch.equal(a.k, c.k)
