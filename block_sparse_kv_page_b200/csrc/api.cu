@@ -1,0 +1,327 @@
+// C-ABI entry points: host-side argument validation, workspace layout and
+// kernel launches.  Nothing here computes results; every step of the path
+// runs in the kernels of meta.cu, select.cu, decode.cu and route.cu.
+//
+// Workspace layout (byte offsets from ws, which must be 256-byte aligned):
+//   [0, 256)                 status word (int32) + reserved
+//   [256, 256 + 4*kMaxUnits) last-CTA counters, shared by every call; each
+//                            call uses counters [0, its units) and leaves
+//                            them zero, so calls issued in order on one
+//                            stream can share one workspace
+//   [kScratch, ...)          per-call scratch (scores of select, split
+//                            partials of decode, router tables), not
+//                            preserved between calls
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace sa {
+
+constexpr int kMaxUnits = 65536;
+constexpr size_t kScratch = 256 + 4 * (size_t)kMaxUnits;
+constexpr int kMaxSelectPages = 16384;
+constexpr int kMaxChunkSel = 8192;
+
+size_t select_smem_bytes(int max_pages);
+
+namespace {
+
+size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
+
+bool aligned(const void* p, size_t a) { return ((uintptr_t)p % a) == 0; }
+
+sa_status check_kv(const sa_kv_desc* kv) {
+  if (!kv) return SA_ERR_INVALID;
+  if (kv->batch < 1 || kv->n_kv_heads < 1 || kv->max_pages < 1 || kv->cap_tokens < 1)
+    return SA_ERR_INVALID;
+  if (kv->head_dim != kHeadDim) return SA_ERR_UNSUPPORTED;
+  if (kv->page_size != 0 && (kv->page_size % 16 != 0 || kv->page_size < 16 || kv->page_size > 256))
+    return SA_ERR_UNSUPPORTED;
+  if (kv->cap_tokens > 0x7fffffffLL) return SA_ERR_UNSUPPORTED;
+  if (!kv->k || !kv->v || !aligned(kv->k, 16) || !aligned(kv->v, 16)) return SA_ERR_INVALID;
+  if (!kv->seq_len || !aligned(kv->seq_len, 4)) return SA_ERR_INVALID;
+  if (kv->page_size == 0) {
+    if (!kv->chunk_off || !kv->n_chunks || !aligned(kv->chunk_off, 4) || !aligned(kv->n_chunks, 4))
+      return SA_ERR_INVALID;
+  }
+  return SA_OK;
+}
+
+KvView view(const sa_kv_desc* kv) {
+  KvView v;
+  v.B = kv->batch;
+  v.Hkv = kv->n_kv_heads;
+  v.page_size = kv->page_size;
+  v.cap = kv->cap_tokens;
+  v.k = kv->k;
+  v.v = kv->v;
+  v.seq_len = kv->seq_len;
+  v.chunk_off = kv->chunk_off;
+  v.n_chunks = kv->n_chunks;
+  v.max_pages = kv->max_pages;
+  return v;
+}
+
+sa_status check_group(const sa_kv_desc* kv, int n_q_heads, int* G) {
+  if (n_q_heads < 1 || n_q_heads % kv->n_kv_heads != 0) return SA_ERR_INVALID;
+  *G = n_q_heads / kv->n_kv_heads;
+  if (*G > kMaxGroup) return SA_ERR_UNSUPPORTED;
+  return SA_OK;
+}
+
+sa_status check_ws(void* ws, size_t ws_bytes, size_t need) {
+  if (!ws || !aligned(ws, 256)) return SA_ERR_WORKSPACE;
+  if (ws_bytes < need) return SA_ERR_WORKSPACE;
+  return SA_OK;
+}
+
+sa_status launched(cudaError_t e) {
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return SA_ERR_CUDA;
+  }
+  return SA_OK;
+}
+
+int max_tiles_per_unit(const sa_kv_desc* kv, int max_sel) {
+  const long long t = kv->page_size > 0 ? (long long)max_sel * (kv->page_size / 16)
+                                        : (long long)max_sel * 16;
+  return t > 0x3fffffff ? 0x3fffffff : (int)t;
+}
+
+size_t select_scratch(const sa_kv_desc* kv) {
+  return align256((size_t)kv->batch * kv->n_kv_heads * kv->max_pages * sizeof(float));
+}
+
+size_t decode_scratch(int units, int splits) {
+  if (splits <= 1) return 0;
+  return align256((size_t)units * splits * kMaxGroup * (kHeadDim + 2) * sizeof(float));
+}
+
+}  // namespace
+
+int device_sm_count() {
+  static int cache[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) {
+    cudaGetLastError();
+    return 148;
+  }
+  if (dev >= 0 && dev < 64 && cache[dev] > 0) return cache[dev];
+  int n = 0;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) {
+    cudaGetLastError();
+    return 148;
+  }
+  if (dev >= 0 && dev < 64) cache[dev] = n;
+  return n;
+}
+
+}  // namespace sa
+
+using namespace sa;
+
+extern "C" {
+
+size_t sparse_attn_workspace_size(const sa_kv_desc* kv, int32_t n_q_heads, int32_t n_q_rows,
+                                  int32_t max_sel) {
+  if (check_kv(kv) != SA_OK || max_sel < 1 || n_q_rows < 0) return 0;
+  int G;
+  if (check_group(kv, n_q_heads, &G) != SA_OK) return 0;
+  const int sm = device_sm_count();
+  const int rows = n_q_rows > kv->batch ? n_q_rows : kv->batch;
+  const long long units = (long long)rows * kv->n_kv_heads;
+  if (units > kMaxUnits) return 0;
+  size_t tail = select_scratch(kv);
+  const int splits = decode_splits((int)units, max_tiles_per_unit(kv, max_sel), sm);
+  const size_t dec = decode_scratch((int)units, splits);
+  if (dec > tail) tail = dec;
+  const size_t rt = route_ws_bytes(rows, kv->n_kv_heads, kv->max_pages);
+  if (rt > tail) tail = rt;
+  return kScratch + tail;
+}
+
+sa_status sparse_attn_workspace_init(void* ws, size_t ws_bytes, void* stream) {
+  if (!ws || !aligned(ws, 256) || ws_bytes < kScratch) return SA_ERR_WORKSPACE;
+  return launched(cudaMemsetAsync(ws, 0, ws_bytes, (cudaStream_t)stream));
+}
+
+sa_status sparse_attn_build_meta(const sa_kv_desc* kv, sa_score_rule rule, int32_t first_token,
+                                 void* meta, void* stream) {
+  sa_status s = check_kv(kv);
+  if (s != SA_OK) return s;
+  if (rule != SA_SCORE_ENVELOPE && rule != SA_SCORE_CENTROID) return SA_ERR_INVALID;
+  if (!meta || !aligned(meta, 16)) return SA_ERR_INVALID;
+  return launched(launch_build_meta(view(kv), (int)rule, first_token, meta, nullptr,
+                                    (cudaStream_t)stream));
+}
+
+sa_status sparse_attn_select(const sa_kv_desc* kv, const void* meta, sa_score_rule rule,
+                             const void* q, int32_t n_q_heads, const sa_budget* budget,
+                             int32_t max_sel, int32_t* sel_idx, int32_t* sel_count,
+                             float* scores_out, void* ws, size_t ws_bytes, void* stream) {
+  sa_status s = check_kv(kv);
+  if (s != SA_OK) return s;
+  int G;
+  if ((s = check_group(kv, n_q_heads, &G)) != SA_OK) return s;
+  if (rule != SA_SCORE_ENVELOPE && rule != SA_SCORE_CENTROID) return SA_ERR_INVALID;
+  if (!meta || !aligned(meta, 16) || !q || !aligned(q, 16)) return SA_ERR_INVALID;
+  if (!budget || !sel_idx || !sel_count || max_sel < 1) return SA_ERR_INVALID;
+  if (!aligned(sel_idx, 4) || !aligned(sel_count, 4) || (scores_out && !aligned(scores_out, 4)))
+    return SA_ERR_INVALID;
+  if (kv->max_pages > kMaxSelectPages) return SA_ERR_UNSUPPORTED;
+  const long long units = (long long)kv->batch * kv->n_kv_heads;
+  if (units > kMaxUnits) return SA_ERR_UNSUPPORTED;
+  switch (budget->kind) {
+    case SA_BUDGET_TOPK:
+      if (budget->top_k < 1 || budget->top_k > max_sel) return SA_ERR_INVALID;
+      break;
+    case SA_BUDGET_RATIO: {
+      if (!(budget->topk_ratio > 0.0 && budget->topk_ratio <= 1.0)) return SA_ERR_INVALID;
+      if (budget->topk_val < 0 || budget->bos < 0 || budget->eos < 0) return SA_ERR_INVALID;
+      const long long fl = (long long)std::floor((double)kv->max_pages * budget->topk_ratio);
+      long long K = (long long)budget->topk_val + budget->bos + budget->eos;
+      if (fl > K) K = fl;
+      if (K > kv->max_pages) K = kv->max_pages;
+      if (K > max_sel) return SA_ERR_INVALID;
+      break;
+    }
+    case SA_BUDGET_TOKENS:
+      if (kv->page_size != 0) return SA_ERR_UNSUPPORTED;  // token budgets are for variable chunks
+      if (budget->token_budget < 0) return SA_ERR_INVALID;
+      break;
+    default:
+      return SA_ERR_INVALID;
+  }
+  const size_t need = kScratch + select_scratch(kv);
+  if ((s = check_ws(ws, ws_bytes, need)) != SA_OK) return s;
+
+  SelectArgs a;
+  a.kv = view(kv);
+  a.meta = meta;
+  a.rule = (int)rule;
+  a.q = q;
+  a.Hq = n_q_heads;
+  a.G = G;
+  a.budget_kind = (int)budget->kind;
+  a.top_k = budget->top_k;
+  a.topk_val = budget->topk_val;
+  a.bos = budget->bos;
+  a.eos = budget->eos;
+  a.token_budget = budget->token_budget;
+  a.ratio = budget->topk_ratio;
+  a.max_sel = max_sel;
+  a.sel_idx = sel_idx;
+  a.sel_count = sel_count;
+  a.scores_out = scores_out;
+  a.ws_scores = reinterpret_cast<float*>(reinterpret_cast<char*>(ws) + kScratch);
+  a.ws_count = reinterpret_cast<uint32_t*>(reinterpret_cast<char*>(ws) + 256);
+  a.status = reinterpret_cast<int*>(ws);
+  a.splits = select_splits((int)units, kv->max_pages, device_sm_count());
+  return launched(launch_select(a, (cudaStream_t)stream));
+}
+
+sa_status sparse_attn_decode(const sa_kv_desc* kv, const void* q, int32_t n_q_heads,
+                             int32_t n_q_rows, int32_t q_pos0, int32_t tile_rows, float scale,
+                             const int32_t* idx, const int32_t* count, int32_t max_sel,
+                             float* out, float* lse, void* ws, size_t ws_bytes, void* stream) {
+  sa_status s = check_kv(kv);
+  if (s != SA_OK) return s;
+  int G;
+  if ((s = check_group(kv, n_q_heads, &G)) != SA_OK) return s;
+  if (!q || !aligned(q, 16) || !idx || !count || !aligned(idx, 4) || !aligned(count, 4))
+    return SA_ERR_INVALID;
+  if (!out || !aligned(out, 16) || (lse && !aligned(lse, 4))) return SA_ERR_INVALID;
+  if (max_sel < 1 || tile_rows < 1 || n_q_rows < 1) return SA_ERR_INVALID;
+  if (!std::isfinite(scale)) return SA_ERR_INVALID;
+  if (tile_rows == 1) {
+    if (n_q_rows != kv->batch) return SA_ERR_INVALID;
+  } else {
+    if (kv->batch != 1 || kv->page_size == 0) return SA_ERR_INVALID;
+    return SA_ERR_UNSUPPORTED;  // multi-row tiles: route-tile attention kernel
+  }
+  if (kv->page_size == 0 && max_sel > kMaxChunkSel) return SA_ERR_UNSUPPORTED;
+  const long long units = (long long)n_q_rows * kv->n_kv_heads;
+  if (units > kMaxUnits) return SA_ERR_UNSUPPORTED;
+  const int splits = decode_splits((int)units, max_tiles_per_unit(kv, max_sel), device_sm_count());
+  const size_t need = kScratch + decode_scratch((int)units, splits);
+  if ((s = check_ws(ws, ws_bytes, need)) != SA_OK) return s;
+
+  DecodeArgs a;
+  a.kv = view(kv);
+  a.q = q;
+  a.Hq = n_q_heads;
+  a.G = G;
+  a.n_rows = n_q_rows;
+  a.q_pos0 = q_pos0;
+  a.tile_rows = tile_rows;
+  a.scale_log2 = scale * kLog2e;
+  a.idx = idx;
+  a.count = count;
+  a.max_sel = max_sel;
+  a.out = out;
+  a.lse = lse;
+  a.ws_part = reinterpret_cast<float*>(reinterpret_cast<char*>(ws) + kScratch);
+  a.ws_count = reinterpret_cast<uint32_t*>(reinterpret_cast<char*>(ws) + 256);
+  a.status = reinterpret_cast<int*>(ws);
+  a.splits = splits;
+  return launched(launch_decode(a, (cudaStream_t)stream));
+}
+
+sa_status sparse_attn_route(const sa_kv_desc* kv, const void* meta, sa_score_rule rule,
+                            const void* q, int32_t n_q_heads, int32_t n_q_rows, int32_t q_pos0,
+                            int32_t tile_rows, int32_t k, int32_t rho, float quantile,
+                            const float* tau, int32_t* kv_idx, int32_t* kv_count, float* sigma,
+                            float* sigma_bar, uint8_t* triggered, float* tau_out, void* ws,
+                            size_t ws_bytes, void* stream) {
+  sa_status s = check_kv(kv);
+  if (s != SA_OK) return s;
+  int G;
+  if ((s = check_group(kv, n_q_heads, &G)) != SA_OK) return s;
+  if (rule != SA_SCORE_ENVELOPE && rule != SA_SCORE_CENTROID) return SA_ERR_INVALID;
+  if (!meta || !aligned(meta, 16) || !q || !aligned(q, 16)) return SA_ERR_INVALID;
+  if (!kv_idx || !kv_count || !sigma || !sigma_bar || !triggered) return SA_ERR_INVALID;
+  if (kv->batch != 1 || kv->page_size == 0) return SA_ERR_INVALID;
+  if (n_q_rows < 1 || tile_rows < 1 || k < 1 || rho < 1 || q_pos0 < 0) return SA_ERR_INVALID;
+  if (!(quantile >= 0.f && quantile <= 1.f)) return SA_ERR_INVALID;
+  (void)tau; (void)tau_out; (void)ws; (void)ws_bytes; (void)stream;
+  return SA_ERR_UNSUPPORTED;
+}
+
+sa_status sparse_attn_get_device_status(void* ws, sa_status* host_out, void* stream) {
+  if (!ws || !host_out || !aligned(ws, 256)) return SA_ERR_INVALID;
+  int v = 0;
+  cudaStream_t st = (cudaStream_t)stream;
+  if (cudaMemcpyAsync(&v, ws, sizeof(int), cudaMemcpyDeviceToHost, st) != cudaSuccess) {
+    cudaGetLastError();
+    return SA_ERR_CUDA;
+  }
+  if (cudaStreamSynchronize(st) != cudaSuccess) {
+    cudaGetLastError();
+    return SA_ERR_CUDA;
+  }
+  if (cudaMemsetAsync(ws, 0, sizeof(int), st) != cudaSuccess) {
+    cudaGetLastError();
+    return SA_ERR_CUDA;
+  }
+  *host_out = (sa_status)v;
+  return SA_OK;
+}
+
+const char* sparse_attn_status_string(sa_status s) {
+  switch (s) {
+    case SA_OK: return "ok";
+    case SA_ERR_INVALID: return "invalid argument";
+    case SA_ERR_UNSUPPORTED: return "unsupported shape or option";
+    case SA_ERR_WORKSPACE: return "workspace missing, misaligned or too small";
+    case SA_ERR_CUDA: return "CUDA launch or runtime error";
+    case SA_ERR_TIMEOUT: return "bounded device wait timed out";
+    case SA_ERR_DEVICE_CHECK: return "device-side range check failed";
+  }
+  return "unknown status";
+}
+
+}  // extern "C"

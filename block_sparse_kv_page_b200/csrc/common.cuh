@@ -1,0 +1,163 @@
+// Device helpers shared by the sparse-attention kernels (sm_100a).
+//
+// Fragment conventions (warp-level mma.sync, m16n8k16 bf16 and m16n8k8 tf32):
+// lane = 4*g + c with g = lane / 4 (row group) and c = lane % 4.
+//   A (16 x 16 bf16): reg0 = A[g][2c..2c+1], reg1 = A[g+8][2c..2c+1],
+//                     reg2 = A[g][2c+8..2c+9], reg3 = A[g+8][2c+8..2c+9]
+//   B (16 x 8 bf16):  reg0 = B[2c..2c+1][g], reg1 = B[2c+8..2c+9][g]
+//   C (16 x 8 f32):   c0,c1 = C[g][2c..2c+1], c2,c3 = C[g+8][2c..2c+1]
+// The reduction index k of a dot product may be permuted freely as long as
+// A and B use the same permutation; the kernels pick the permutation that
+// lets every lane fetch whole 16-byte chunks of a row, so global loads are
+// fully coalesced and shared-memory reads are conflict-free.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <stdint.h>
+
+#define SA_DEV __device__ __forceinline__
+
+namespace sa {
+
+constexpr int kHeadDim = 128;
+constexpr int kMetaBytes = 512;      // metadata bytes per (b, kv head, page)
+constexpr int kMaxGroup = 8;         // query heads per KV head handled by one n8 MMA tile
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kLn2 = 0.6931471805599453f;
+
+// ---------------------------------------------------------------- async copy
+SA_DEV uint32_t smem_addr(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+// 16-byte global -> shared copy; when !valid nothing is read and zeros land.
+SA_DEV void cp_async16(void* dst_smem, const void* src_gmem, bool valid) {
+  const int n = valid ? 16 : 0;
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(smem_addr(dst_smem)),
+               "l"(src_gmem), "r"(n)
+               : "memory");
+}
+SA_DEV void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::: "memory"); }
+template <int N>
+SA_DEV void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;\n" ::"n"(N) : "memory");
+}
+
+SA_DEV uint4 lds128(const void* p) {
+  uint4 r;
+  asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];\n"
+               : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+               : "r"(smem_addr(p)));
+  return r;
+}
+
+SA_DEV uint4 ldg_nc128(const void* p) {
+  uint4 r;
+  asm volatile("ld.global.nc.v4.u32 {%0,%1,%2,%3}, [%4];\n"
+               : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+               : "l"(p));
+  return r;
+}
+
+// ---------------------------------------------------------------- tensor-core MMA
+SA_DEV void mma_bf16(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                     uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 "
+      "{%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};\n"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+SA_DEV void mma_tf32(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                     uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 "
+      "{%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};\n"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// FP64 tensor-core MMA m8n8k4: a = A[g][c], b = B[c][g], c0,c1 = C[g][2c..2c+1].
+SA_DEV void mma_f64(double& c0, double& c1, double a, double b) {
+  asm volatile("mma.sync.aligned.m8n8k4.row.col.f64.f64.f64.f64 {%0,%1}, {%2}, {%3}, {%0,%1};\n"
+               : "+d"(c0), "+d"(c1)
+               : "d"(a), "d"(b));
+}
+
+SA_DEV uint32_t to_tf32(float x) {
+  uint32_t r;
+  asm("cvt.rna.tf32.f32 %0, %1;\n" : "=r"(r) : "f"(x));
+  return r;
+}
+
+// Transpose an 8x8 b16 matrix held in the standard fragment layout.
+SA_DEV uint32_t movmatrix_t(uint32_t x) {
+  uint32_t y;
+  asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;\n" : "=r"(y) : "r"(x));
+  return y;
+}
+
+SA_DEV uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
+  uint32_t r;
+  asm("prmt.b32 %0, %1, %2, %3;\n" : "=r"(r) : "r"(a), "r"(b), "r"(sel));
+  return r;
+}
+
+SA_DEV uint32_t pack_bf16(float lo, float hi) {
+  __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&v);
+}
+SA_DEV float bf16_lo(uint32_t x) { return __uint_as_float(x << 16); }
+SA_DEV float bf16_hi(uint32_t x) { return __uint_as_float(x & 0xffff0000u); }
+
+// Elementwise min(x, 0) / max(x, 0) of a packed bf16 pair (exact).
+SA_DEV uint32_t bf16x2_neg_part(uint32_t x) {
+  const uint32_t lo = (x & 0x8000u) ? (x & 0xffffu) : 0u;
+  const uint32_t hi = (x & 0x80000000u) ? (x & 0xffff0000u) : 0u;
+  return lo | hi;
+}
+SA_DEV uint32_t bf16x2_pos_part(uint32_t x) {
+  const uint32_t lo = (x & 0x8000u) ? 0u : (x & 0xffffu);
+  const uint32_t hi = (x & 0x80000000u) ? 0u : (x & 0xffff0000u);
+  return lo | hi;
+}
+
+// ---------------------------------------------------------------- ordering keys
+// Monotone map float -> uint32 (larger float -> larger key); -0.0 maps with +0.0.
+SA_DEV uint32_t order_key(float s) {
+  uint32_t u = __float_as_uint(s + 0.0f);
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+// ---------------------------------------------------------------- status word
+SA_DEV void flag_status(int* status, int code) {
+  if (status) atomicCAS(status, 0, code);
+}
+
+// ---------------------------------------------------------------- block scans
+// Exclusive prefix sum over the block of one uint32 per thread; also returns
+// the block total.  `scratch` holds at least (blockDim.x / 32) words.
+SA_DEV uint32_t block_excl_scan(uint32_t v, uint32_t* scratch, uint32_t& total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  uint32_t x = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    uint32_t y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
+  }
+  if (lane == 31) scratch[warp] = x;
+  __syncthreads();
+  uint32_t base = 0, tot = 0;
+  for (int w = 0; w < nw; ++w) {
+    const uint32_t s = scratch[w];
+    if (w < warp) base += s;
+    tot += s;
+  }
+  __syncthreads();
+  total = tot;
+  return base + x - v;
+}
+
+}  // namespace sa

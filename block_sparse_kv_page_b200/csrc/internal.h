@@ -1,0 +1,105 @@
+// Internal launch interface between the C-ABI entry points (api.cu) and the
+// kernel files.  Host-only declarations; not part of the public ABI.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "sparse_attn.h"
+
+namespace sa {
+
+// Plain copy of the cache view, passed to kernels by value.
+struct KvView {
+  int B, Hkv, page_size;      // page_size 0 = variable chunks
+  long long cap;
+  const void* k;
+  const void* v;
+  const int32_t* seq_len;
+  const int32_t* chunk_off;   // [B][max_pages + 1]
+  const int32_t* n_chunks;
+  int max_pages;
+};
+
+// Workspace regions (byte offsets from ws, each 256-aligned).
+struct WsLayout {
+  size_t status;        // int32 status word
+  size_t sel_count;     // uint32 [units] last-CTA counters of select
+  size_t dec_count;     // uint32 [rows * Hkv] last-CTA counters of decode
+  size_t sel_scores;    // float [units][max_pages] group scores
+  size_t dec_part;      // float partials [slots][G][kHeadDim + 2]
+  size_t route;         // router scratch
+  size_t total;
+  int dec_slots;        // partial slots available (units * splits bound)
+};
+
+int device_sm_count();
+int decode_splits(int units, int max_tiles, int sm_count);
+int select_splits(int units, int max_pages, int sm_count);
+WsLayout workspace_layout(const sa_kv_desc* kv, int n_q_heads, int n_q_rows, int max_sel,
+                          int sm_count);
+
+cudaError_t launch_build_meta(const KvView& kv, int rule, int first_token, void* meta,
+                              int* status, cudaStream_t st);
+
+struct SelectArgs {
+  KvView kv;
+  const void* meta;
+  int rule;
+  const void* q;
+  int Hq, G;
+  int budget_kind, top_k, topk_val, bos, eos, token_budget;
+  double ratio;
+  int max_sel;
+  int32_t* sel_idx;
+  int32_t* sel_count;
+  float* scores_out;
+  float* ws_scores;
+  uint32_t* ws_count;
+  int* status;
+  int splits;
+};
+cudaError_t launch_select(const SelectArgs& a, cudaStream_t st);
+
+struct DecodeArgs {
+  KvView kv;
+  const void* q;
+  int Hq, G;
+  int n_rows, q_pos0, tile_rows;
+  float scale_log2;           // scale * log2(e)
+  const int32_t* idx;
+  const int32_t* count;
+  int max_sel;
+  float* out;
+  float* lse;
+  float* ws_part;
+  uint32_t* ws_count;
+  int* status;
+  int splits;
+};
+cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t st);
+
+struct RouteArgs {
+  KvView kv;
+  const void* meta;
+  int rule;
+  const void* q;
+  int Hq, G;
+  int n_rows, q_pos0, tile_rows, n_tiles;
+  int k, rho;
+  float quantile;
+  const float* tau_in;
+  int32_t* kv_idx;
+  int32_t* kv_count;
+  float* sigma;
+  float* sigma_bar;
+  uint8_t* triggered;
+  float* tau_out;
+  void* ws_route;
+  int* status;
+};
+cudaError_t launch_route(const RouteArgs& a, cudaStream_t st);
+size_t route_ws_bytes(int n_tiles, int Hkv, int max_pages);
+
+}  // namespace sa

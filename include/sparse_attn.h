@@ -1,0 +1,202 @@
+/*
+ * sparse_attn.h -- C ABI of libsparse_attn.so: query-aware block-sparse GQA
+ * decode attention and the uncertainty router, hand-written CUDA for sm_100a.
+ *
+ * Sources (web pages, cited by title and section):
+ *  [OFFLINE]  "Sparse Attention for Web Agents -- Offline Replay Records"
+ *             (dataset card), section "The comparison": every method cuts the
+ *             KV cache into chunks, scores each chunk against the current
+ *             query, keeps the best ones and attends only to those; fixed
+ *             16-token pages (Quest, BlockSparse) or 16-256-token
+ *             structure-aligned chunks (TSA); envelope (per-dimension min/max
+ *             upper bound) or centroid (mean key) scoring; the budget is
+ *             page_size x top_k attended tokens.
+ *  [WEBARENA] "WebArena 0-99 Sparse-Attention Method Comparison" (dataset
+ *             card), section "Method configurations at a glance": kept blocks
+ *             = max(topk_val + bos + eos, int(cached_block_len * topk_ratio))
+ *             with forced first (bos) and last (eos) blocks.
+ *  [ROUTER]   "Technische Samenvatting: Onzekerheidsgestuurde Selectie voor
+ *             Blok-schaarse Aandacht", section "Methodologie", steps 1-5:
+ *             per-tile block scores (max over the tile's rows), the margin
+ *             sigma = (s_(k-1) - s_(k)) / (s_(0) - s_(k)), its mean over
+ *             heads, a per-layer quantile trigger, and expansion to top-rho*k
+ *             with sentinel padding so every tile's list has the same shape.
+ *
+ * Conventions shared by every call
+ *  - All data pointers are DEVICE pointers (global memory of the current
+ *    device) unless stated otherwise; descriptors and budgets are HOST structs
+ *    read during the call only.  The caller owns all memory: the library never
+ *    allocates, frees or synchronises (sparse_attn_get_device_status is the one
+ *    call that waits on its stream).
+ *  - Every compute call validates its arguments on the host first.  A bad
+ *    argument returns SA_ERR_INVALID (or SA_ERR_UNSUPPORTED for a legal but
+ *    unimplemented shape) and nothing is launched.  SA_OK means "enqueued on
+ *    `stream`"; a failed launch returns SA_ERR_CUDA.  `stream` is a
+ *    cudaStream_t (NULL = the legacy default stream).
+ *  - Conditions found on the device (a page index out of range, a selection
+ *    that overflows max_sel) are recorded in a status word inside the
+ *    workspace `ws` and read with sparse_attn_get_device_status.  The offending
+ *    entry is skipped; no kernel traps.
+ *  - Tensors: q, K, V are bf16 with head_dim = 128 (the only supported value).
+ *    K and V of one layer are [batch][n_kv_heads][cap_tokens][128], so a
+ *    16-token page of one KV head is one contiguous 4 KiB block.  Several
+ *    independent layers may be processed in one call by stacking them along
+ *    the batch axis.
+ *  - Metadata (`meta`) holds 512 bytes per (batch, KV head, page):
+ *      SA_SCORE_ENVELOPE: bf16 kmin[128] followed by bf16 kmax[128];
+ *      SA_SCORE_CENTROID: fp32 kmean[128].
+ *    Layout [batch][n_kv_heads][max_pages][512 B].  One buffer serves one rule.
+ *  - Grouped-query attention: query head h belongs to KV head h / G with
+ *    G = n_q_heads / n_kv_heads, 1 <= G <= 8.  One page set is chosen per
+ *    (sequence, KV head) and shared by its G query heads; the group score of a
+ *    page is the maximum of its G per-head scores.
+ *  - Ties: pages are ordered by group score descending, lower page index first
+ *    on equal scores (-0.0 equals +0.0).  NaN or infinite inputs are undefined.
+ */
+#ifndef SPARSE_ATTN_H
+#define SPARSE_ATTN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  SA_OK = 0,
+  SA_ERR_INVALID = 1,       /* bad argument (null/misaligned pointer, out-of-range size) */
+  SA_ERR_UNSUPPORTED = 2,   /* legal but not implemented (head_dim != 128, G > 8, ...) */
+  SA_ERR_WORKSPACE = 3,     /* ws is null, misaligned or smaller than required */
+  SA_ERR_CUDA = 4,          /* a CUDA runtime call or kernel launch failed */
+  SA_ERR_TIMEOUT = 5,       /* reserved: a bounded device-side wait gave up */
+  SA_ERR_DEVICE_CHECK = 6   /* a device-side range check failed (entry skipped) */
+} sa_status;
+
+typedef enum {
+  SA_SCORE_ENVELOPE = 0,    /* sum_d max(q_d*kmin_d, q_d*kmax_d)  [OFFLINE] "The comparison" */
+  SA_SCORE_CENTROID = 1     /* q . mean(K_page)                  [OFFLINE] "The comparison" */
+} sa_score_rule;
+
+typedef enum {
+  SA_BUDGET_TOPK = 0,       /* keep min(top_k, P) pages                       [OFFLINE] */
+  SA_BUDGET_RATIO = 1,      /* keep min(P, max(topk_val+bos+eos, floor(P*ratio))) incl. forced [WEBARENA] */
+  SA_BUDGET_TOKENS = 2      /* longest rank-order prefix of chunks with <= token_budget tokens [OFFLINE] */
+} sa_budget_kind;
+
+/* View of one KV cache (one or more stacked layers). */
+typedef struct {
+  int32_t batch;            /* B >= 1: sequences (x stacked layers) */
+  int32_t n_kv_heads;       /* Hkv >= 1 */
+  int32_t head_dim;         /* must be 128 */
+  int32_t page_size;        /* fixed pages: multiple of 16 in [16, 256]; 0 = variable chunks */
+  int64_t cap_tokens;       /* token capacity per (b, kv head) */
+  const void* k;            /* bf16 [B][Hkv][cap_tokens][128], 16-byte aligned */
+  const void* v;            /* bf16 [B][Hkv][cap_tokens][128], 16-byte aligned */
+  const int32_t* seq_len;   /* [B] tokens N_b in the cache, 1 <= N_b <= cap_tokens (includes the current token) */
+  const int32_t* chunk_off; /* variable chunks only: [B][max_pages + 1] CSR token offsets, chunk c = [off[c], min(off[c+1], N_b)) */
+  const int32_t* n_chunks;  /* variable chunks only: [B] chunk count C_b <= max_pages, off[C_b] = N_b */
+  int32_t max_pages;        /* page/chunk capacity of the metadata axis; P_b = ceil(N_b / page_size) or C_b */
+} sa_kv_desc;
+
+/* Budget of one selection ([OFFLINE] "The comparison"; [WEBARENA]). */
+typedef struct {
+  sa_budget_kind kind;
+  int32_t top_k;            /* TOPK: pages to keep, >= 1 */
+  double topk_ratio;        /* RATIO: 0 < ratio <= 1, read as floor(P * ratio) */
+  int32_t topk_val;         /* RATIO: floor term topk_val + bos + eos (1 on the WebArena card) */
+  int32_t bos;              /* RATIO: first `bos` pages always kept */
+  int32_t eos;              /* RATIO: last `eos` pages always kept (the newest token's page) */
+  int32_t token_budget;     /* TOKENS: attended-token budget, >= 0 */
+} sa_budget;
+
+/* Bytes of workspace that every call below needs for this cache view, query
+ * head count, query-row count (decode: B; router: rows) and selection width.
+ * Returns 0 on invalid arguments.  The workspace must be 256-byte aligned and
+ * zeroed once after allocation by sparse_attn_workspace_init; calls leave its
+ * counters zeroed again, so one workspace serves any number of calls issued
+ * in order on one stream (calls that may overlap need separate workspaces). */
+size_t sparse_attn_workspace_size(const sa_kv_desc* kv, int32_t n_q_heads,
+                                  int32_t n_q_rows, int32_t max_sel);
+
+/* Zero the workspace (counters and status word).  Async on `stream`. */
+sa_status sparse_attn_workspace_init(void* ws, size_t ws_bytes, void* stream);
+
+/* (a) Page metadata ([OFFLINE] "The comparison", scoring column).
+ * For every (b, kv head), recompute the metadata of every page/chunk that
+ * overlaps the token range [t0_b, N_b):
+ *   first_token >= 0: t0_b = first_token            (0 = full build);
+ *   first_token <  0: t0_b = max(0, N_b + first_token)  (-1 = the page of the
+ *                     token just appended: the per-step incremental update).
+ * Envelope: kmin/kmax per dimension, exact bf16.  Centroid: the mean of the
+ * page's keys, accumulated in fp64 and stored as fp32.  Pages outside the
+ * range are not touched.  meta: [B][Hkv][max_pages] x 512 B, 16-byte aligned. */
+sa_status sparse_attn_build_meta(const sa_kv_desc* kv, sa_score_rule rule,
+                                 int32_t first_token, void* meta, void* stream);
+
+/* (b) Score + budgeted top-k ([OFFLINE] "The comparison"; [WEBARENA]).
+ * q: bf16 [B][n_q_heads][128], the current query token of each sequence.
+ * For each (b, kv head): group score of every page (max over the G query
+ * heads), then the pages kept by `budget` under the order (score desc, index
+ * asc).  Output: sel_idx[b][g][0 .. sel_count[b][g]) = the kept page indices
+ * in ASCENDING page order (the set is what the budget defines; ascending
+ * order is what the decode streams); entries past the count are untouched.
+ * scores_out (nullable): [B][Hkv][max_pages] fp32 group score of every page.
+ * max_sel bounds the kept count: TOPK needs top_k <= max_sel; RATIO needs
+ * min(max_pages, max(topk_val+bos+eos, floor(max_pages*ratio))) <= max_sel;
+ * TOKENS keeps at most max_sel chunks (overflow sets SA_ERR_DEVICE_CHECK). */
+sa_status sparse_attn_select(const sa_kv_desc* kv, const void* meta, sa_score_rule rule,
+                             const void* q, int32_t n_q_heads, const sa_budget* budget,
+                             int32_t max_sel, int32_t* sel_idx, int32_t* sel_count,
+                             float* scores_out, void* ws, size_t ws_bytes, void* stream);
+
+/* (c) Sparse paged attention over the kept pages ([OFFLINE] "The comparison":
+ * attend only to the kept chunks; exact softmax over their tokens).
+ *  tile_rows == 1 (decode): q bf16 [B][n_q_heads][128]; n_q_rows == B; query
+ *    head h of sequence b attends to every token of the pages idx[b][h/G][0 ..
+ *    count[b][h/G]) (all tokens of the cache precede the current one).
+ *  tile_rows > 1 (router tiles, [ROUTER] step 5): B == 1; q bf16
+ *    [n_q_rows][n_q_heads][128] at positions q_pos0 + r; idx [T][Hkv][max_sel]
+ *    with T = ceil(n_q_rows / tile_rows), -1 entries skipped; row r attends
+ *    causally (token position <= q_pos0 + r) to the blocks of its tile.
+ * z = scale * q.k, softmax with fp32 accumulation.  out: fp32 [rows][Hq][128];
+ * lse (nullable): fp32 [rows][Hq], natural-log sum of exp(z).  A row with no
+ * visible token gets out = 0 and lse = -inf.  idx entries outside [0, P_b)
+ * are skipped and flag SA_ERR_DEVICE_CHECK. */
+sa_status sparse_attn_decode(const sa_kv_desc* kv, const void* q, int32_t n_q_heads,
+                             int32_t n_q_rows, int32_t q_pos0, int32_t tile_rows, float scale,
+                             const int32_t* idx, const int32_t* count, int32_t max_sel,
+                             float* out, float* lse, void* ws, size_t ws_bytes, void* stream);
+
+/* (d) Uncertainty router over query tiles ([ROUTER] "Methodologie" steps 2-5).
+ * B == 1, fixed blocks (page_size = block size).  q bf16 [n_q_rows][n_q_heads][128]
+ * at positions q_pos0 + r; tiles of tile_rows consecutive rows.  For tile t
+ * and kv head g: the eligible blocks are those whose first token is not after
+ * the tile's last row; the tile score of a block is the max over the tile's
+ * rows and the group's G heads of the per-row score.  sigma[t][g] from the
+ * descending scores (1 if at most k blocks are eligible, 0 if s_(0) = s_(k));
+ * sigma_bar[t] = mean over kv heads; tau = the linear-interpolation quantile
+ * `quantile` of sigma_bar over the tiles (or *tau if tau is non-null);
+ * triggered[t] = sigma_bar[t] < tau.  kv_idx[t][g][0 .. rho*k) lists blocks in
+ * RANK order: the first min(rho*k, E) if triggered else the first min(k, E),
+ * padded with -1; kv_count[t][g] = number of valid entries.
+ * tau_out (nullable): the threshold used. */
+sa_status sparse_attn_route(const sa_kv_desc* kv, const void* meta, sa_score_rule rule,
+                            const void* q, int32_t n_q_heads, int32_t n_q_rows,
+                            int32_t q_pos0, int32_t tile_rows, int32_t k, int32_t rho,
+                            float quantile, const float* tau, int32_t* kv_idx,
+                            int32_t* kv_count, float* sigma, float* sigma_bar,
+                            uint8_t* triggered, float* tau_out, void* ws, size_t ws_bytes,
+                            void* stream);
+
+/* Copy the workspace status word to *host_out (SA_OK if no device check
+ * fired since the last init/clear) and clear it.  Synchronises `stream`. */
+sa_status sparse_attn_get_device_status(void* ws, sa_status* host_out, void* stream);
+
+/* Static description of a status code (never null). */
+const char* sparse_attn_status_string(sa_status s);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* SPARSE_ATTN_H */

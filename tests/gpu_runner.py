@@ -1,0 +1,199 @@
+"""Parity harness: run the CUDA path through the C ABI, run the float64 oracle
+on host copies of the same bf16 tensors, and compare.
+
+Selection parity (the near-tie certificate): the GPU page set must equal the
+oracle's, except when the oracle's last kept score and first dropped score
+differ by less than delta = 1e-5 * max(|s_(K-1)|, |s_(K)|, 1).  In that case
+pages scoring above the band must be kept, pages below it dropped, and the
+count must match.  Attention parity is checked on the set the GPU actually
+chose (the oracle attends over the same pages), max-abs error <= 2e-3 on
+unit-scale inputs (the tolerance the method's specification states; the
+measured errors are far below it).
+"""
+from __future__ import annotations
+
+import math
+
+import numpy as np
+import torch
+
+import block_sparse_kv_page_b200 as sa
+import oracle as O
+
+OUT_TOL = 2e-3
+TIE_REL = 1e-5
+
+
+def to_np(t: torch.Tensor) -> np.ndarray:
+    return t.detach().float().cpu().numpy().astype(np.float64)
+
+
+def budget_struct(bd: dict):
+    if bd["kind"] == "topk":
+        return sa.budget_topk(bd["k"])
+    if bd["kind"] == "ratio":
+        return sa.budget_ratio(bd["ratio"], topk_val=bd.get("topk_val", 1), bos=bd["bos"], eos=bd["eos"])
+    return sa.budget_tokens(bd["budget"])
+
+
+def default_max_sel(bd: dict, max_pages: int) -> int:
+    if bd["kind"] == "topk":
+        return bd["k"]
+    if bd["kind"] == "ratio":
+        return O.ratio_budget_pages(max_pages, bd["ratio"], bd.get("topk_val", 1), bd["bos"], bd["eos"])
+    return max_pages
+
+
+def run_gpu(layer, *, page_size: int, rule: str, budget: dict, scale: float,
+            max_pages: int | None = None, max_sel: int | None = None, ws=None, repeat: int = 1):
+    B, Hkv, cap, D = layer.k.shape
+    Hq = layer.q.shape[1]
+    if max_pages is None:
+        max_pages = -(-cap // page_size) if page_size else layer.chunk_off.shape[1] - 1
+    if max_sel is None:
+        max_sel = default_max_sel(budget, max_pages)
+    kv = sa.KvCache(layer.k, layer.v, layer.seq_len, page_size=page_size, max_pages=max_pages,
+                    chunk_off=layer.chunk_off, n_chunks=layer.n_chunks)
+    dev = layer.k.device
+    meta = kv.meta_buffer()
+    if ws is None:
+        ws = sa.make_workspace(kv, Hq, B, max_sel)
+    sa.sparse_attn_build_meta(kv, rule, 0, meta)
+    results = []
+    for _ in range(repeat):
+        sel_idx = torch.full((B, Hkv, max_sel), -7, dtype=torch.int32, device=dev)
+        sel_count = torch.full((B, Hkv), -7, dtype=torch.int32, device=dev)
+        scores = torch.full((B, Hkv, max_pages), float("nan"), dtype=torch.float32, device=dev)
+        sa.sparse_attn_select(kv, meta, rule, layer.q, budget_struct(budget), max_sel,
+                              sel_idx, sel_count, scores, ws)
+        out = torch.full((B, Hq, 128), float("nan"), dtype=torch.float32, device=dev)
+        lse = torch.full((B, Hq), float("nan"), dtype=torch.float32, device=dev)
+        sa.sparse_attn_decode(kv, layer.q, B, 0, 1, scale, sel_idx, sel_count, max_sel, out, lse, ws)
+        torch.cuda.synchronize()
+        results.append(dict(sel_idx=sel_idx.cpu(), sel_count=sel_count.cpu(), scores=scores.cpu(),
+                            out=out.cpu(), lse=lse.cpu()))
+    status = sa.sparse_attn_get_device_status(ws)
+    r = results[0]
+    r.update(meta=meta, kv=kv, ws=ws, status=status, max_sel=max_sel, max_pages=max_pages,
+             runs=results)
+    return r
+
+
+def _certify_cut(S, order, n_keep, gset, where):
+    """Exact set equality unless the cut is a near-tie; then band rules."""
+    oset = set(int(p) for p in order[:n_keep])
+    if n_keep == 0 or n_keep >= len(order):
+        assert gset == oset, f"{where}: set differs with no cut ({len(gset)} vs {len(oset)})"
+        return False
+    a, b = S[order[n_keep - 1]], S[order[n_keep]]
+    delta = TIE_REL * max(abs(a), abs(b), 1.0)
+    if a - b >= delta:
+        assert gset == oset, f"{where}: set differs at a decisive cut (gap {a - b:.3g})"
+        return False
+    assert len(gset) == len(oset), f"{where}: count {len(gset)} vs {len(oset)}"
+    for p in (int(x) for x in order):
+        if S[p] > a + delta:
+            assert p in gset, f"{where}: page {p} above the tie band dropped"
+        if S[p] < b - delta:
+            assert p not in gset, f"{where}: page {p} below the tie band kept"
+    return True
+
+
+def certify_selection(S, gset: set, budget: dict, lens=None, where=""):
+    """Returns True when a certified near-tie allowed a difference."""
+    S = np.asarray(S, dtype=np.float64)
+    P = len(S)
+    order = O.rank_order(S)
+    kind = budget["kind"]
+    if kind == "topk":
+        return _certify_cut(S, order, min(budget["k"], P), gset, where)
+    if kind == "ratio":
+        K = O.ratio_budget_pages(P, budget["ratio"], budget.get("topk_val", 1), budget["bos"], budget["eos"])
+        forced = set(int(x) for x in O.forced_pages(P, budget["bos"], budget["eos"]))
+        assert forced <= gset, f"{where}: forced pages missing"
+        rest = np.array([p for p in order if int(p) not in forced], dtype=np.int64)
+        Sr = S.copy()
+        return _certify_cut(Sr, rest, K - len(forced), gset - forced, where)
+    # token budget: greedy prefix of the rank order
+    lens = np.asarray(lens, dtype=np.int64)
+    oset = set(int(p) for p in O.select_token_budget(S, lens, budget["budget"]))
+    r = len(oset)
+    near = False
+    for i in (r - 1, r):
+        if 0 <= i and i + 1 < P:
+            a, b = S[order[i]], S[order[i + 1]]
+            if a - b < TIE_REL * max(abs(a), abs(b), 1.0):
+                near = True
+    if not near:
+        assert gset == oset, f"{where}: token-budget set differs"
+        return False
+    assert sum(int(lens[p]) for p in gset) <= budget["budget"], f"{where}: over budget"
+    return True
+
+
+def check_layer(layer, gpu, *, page_size: int, rule: str, budget: dict, scale: float,
+                units=None, score_rel: float = 2e-6, out_tol: float = OUT_TOL):
+    """Compare every (b, g) unit (or the given subset) with the oracle.
+    Returns a dict of statistics (max errors, tie exemptions)."""
+    B, Hkv = layer.k.shape[:2]
+    Hq = layer.q.shape[1]
+    G = Hq // Hkv
+    stats = dict(max_out_err=0.0, max_lse_err=0.0, max_score_err=0.0, ties=0, units=0)
+    if units is None:
+        units = [(b, g) for b in range(B) for g in range(Hkv)]
+    for b, g in units:
+        N = int(layer.seq_len[b])
+        where = f"unit(b={b},g={g})"
+        Qg = to_np(layer.q[b, g * G:(g + 1) * G])
+        K = to_np(layer.k[b, g, :N])
+        V = to_np(layer.v[b, g, :N])
+        if page_size:
+            starts, ends = O.fixed_pages(N, page_size)
+            off = None
+        else:
+            C = int(layer.n_chunks[b])
+            off = layer.chunk_off[b, :C + 1].cpu().numpy().astype(np.int64)
+            starts, ends = O.chunk_pages(off)
+        meta = O.page_metadata(K, starts, ends)
+        P = len(starts)
+        # metadata parity
+        gm = gpu["meta"][b, g, :P]
+        if rule == "envelope":
+            gmin = to_np(gm[:, :256].contiguous().view(torch.bfloat16))
+            gmax = to_np(gm[:, 256:].contiguous().view(torch.bfloat16))
+            assert np.array_equal(gmin, meta[0]) and np.array_equal(gmax, meta[1]), f"{where}: envelope metadata"
+        else:
+            gmean = gm.contiguous().view(torch.float32).cpu().numpy().astype(np.float64)
+            ref32 = meta[2].astype(np.float32).astype(np.float64)
+            ulp = np.spacing(np.abs(ref32).astype(np.float32)).astype(np.float64)
+            assert np.all(np.abs(gmean - ref32) <= ulp), f"{where}: centroid metadata"
+        # scores
+        S = O.group_reduce(O.head_scores(Qg, meta, rule))
+        gs = gpu["scores"][b, g, :P].numpy().astype(np.float64)
+        err = np.abs(gs - S) / np.maximum(np.abs(S), 1.0)
+        stats["max_score_err"] = max(stats["max_score_err"], float(err.max()))
+        assert err.max() <= score_rel, f"{where}: score rel err {err.max():.3g}"
+        # selection
+        cnt = int(gpu["sel_count"][b, g])
+        gl = gpu["sel_idx"][b, g, :cnt].numpy().astype(np.int64)
+        assert np.all(np.diff(gl) > 0), f"{where}: selection not strictly ascending"
+        gset = set(int(x) for x in gl)
+        lens = (ends - starts) if not page_size else None
+        if certify_selection(S, gset, budget, lens, where):
+            stats["ties"] += 1
+        # attention over the pages the GPU kept
+        toks = O.tokens_of(gl, starts, ends)
+        o_ref, l_ref = O.attend(Qg, K, V, toks, scale)
+        o_gpu = gpu["out"][b, g * G:(g + 1) * G].numpy().astype(np.float64)
+        l_gpu = gpu["lse"][b, g * G:(g + 1) * G].numpy().astype(np.float64)
+        if len(toks) == 0:
+            assert np.all(o_gpu == 0) and np.all(np.isneginf(l_gpu)), f"{where}: empty selection"
+        else:
+            e = float(np.abs(o_gpu - o_ref).max())
+            le = float(np.abs(l_gpu - l_ref).max())
+            stats["max_out_err"] = max(stats["max_out_err"], e)
+            stats["max_lse_err"] = max(stats["max_lse_err"], le)
+            assert e <= out_tol, f"{where}: out max-abs err {e:.3g}"
+            assert le <= 1e-3 * max(1.0, float(np.abs(l_ref).max())), f"{where}: lse err {le:.3g}"
+        stats["units"] += 1
+    return stats

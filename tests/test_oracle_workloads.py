@@ -20,16 +20,28 @@ def _np(x):
     return x.float().numpy().astype(np.float64)
 
 
-def test_needles_selected_envelope():
-    lay = DG.workload1_layer("cpu")
-    w = DG.WORKLOADS[1]
-    G = w.Hq // w.Hkv
-    for g in range(w.Hkv):
-        r = O.decode_unit(_np(lay.q[0, g * G:(g + 1) * G]), _np(lay.k[0, g]), _np(lay.v[0, g]),
-                          w.N, rule="envelope", page_size=16,
-                          budget={"kind": "topk", "k": 16}, scale=1 / math.sqrt(128))
-        assert set(lay.extra["needle_pages"][g]) <= set(r.selected.tolist())
-        assert r.n_tokens == 16 * 16
+def test_needles_rank_top_for_their_head():
+    """A needle page (keys N(0,1) + 4 q_h/|q_h|) raises its own head's
+    envelope by about 0.35 |q_h|^2 ~ 45, some 8 standard deviations of the
+    random-page spread, so it ranks in the top 3 of that head's per-head
+    scores.  (Under the group max another head with a larger |q|_1 can
+    outscore it, so selection by the group score is data-dependent and is
+    checked by parity, not here.)"""
+    for seed_offset in range(3):
+        lay = DG.workload1_layer("cpu", seed_offset=seed_offset)
+        w = DG.WORKLOADS[1]
+        G = w.Hq // w.Hkv
+        for g in range(w.Hkv):
+            K = _np(lay.k[0, g])
+            s, e = O.fixed_pages(w.N, 16)
+            meta = O.page_metadata(K, s, e)
+            Qg = _np(lay.q[0, g * G:(g + 1) * G])
+            sh = O.envelope_scores(Qg, meta[0], meta[1])
+            for j, p in enumerate(lay.extra["needle_pages"][g]):
+                assert p in set(np.argsort(-sh[j])[:3].tolist())
+            r = O.decode_unit(Qg, K, _np(lay.v[0, g]), w.N, rule="envelope", page_size=16,
+                              budget={"kind": "topk", "k": 16}, scale=1 / math.sqrt(128), meta=meta)
+            assert r.n_tokens == 16 * 16
 
 
 def test_chunk_generator_ranges():
