@@ -3,7 +3,10 @@
 // runs in the kernels of meta.cu, select.cu, decode.cu and route.cu.
 //
 // Workspace layout (byte offsets from ws, which must be 256-byte aligned):
-//   [0, 256)                 status word (int32) + reserved
+//   [0, 256)                 status word (int32) at 0; item-queue counters of
+//                            the persistent kernels at 64 (select), 72
+//                            (decode), 80 (router); each kernel leaves its
+//                            queue rewound to zero
 //   [256, 256 + 4*kMaxUnits) last-CTA counters, shared by every call; each
 //                            call uses counters [0, its units) and leaves
 //                            them zero, so calls issued in order on one
@@ -21,6 +24,8 @@
 namespace sa {
 
 constexpr int kMaxUnits = 65536;
+constexpr size_t kQueueSelect = 64;
+constexpr size_t kQueueDecode = 72;
 constexpr size_t kScratch = 256 + 4 * (size_t)kMaxUnits;
 constexpr int kMaxSelectPages = 16384;
 constexpr int kMaxChunkSel = 8192;
@@ -102,6 +107,65 @@ size_t decode_scratch(int units, int splits) {
 }
 
 }  // namespace
+
+namespace {
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*,
+                                   CUtensorMapInterleave, CUtensorMapSwizzle, CUtensorMapL2promotion,
+                                   CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static bool tried = false;
+  if (!tried) {
+    tried = true;
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+    else
+      cudaGetLastError();
+  }
+  return fn;
+}
+}  // namespace
+
+bool encode_tmap_2d(CUtensorMap* map, const void* base, unsigned long long rows, int row_bytes,
+                    CUtensorMapDataType dt, int elem_bytes, int box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[2] = {(cuuint64_t)(row_bytes / elem_bytes), (cuuint64_t)rows};
+  const cuuint64_t strides[1] = {(cuuint64_t)row_bytes};
+  const cuuint32_t box[2] = {(cuuint32_t)(128 / elem_bytes), (cuuint32_t)box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  return fn(map, dt, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+            CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+cudaError_t set_smem_attr(const void* func, size_t bytes) {
+  struct Entry {
+    const void* f;
+    int dev;
+    size_t bytes;
+  };
+  static Entry cache[64];
+  static int n = 0;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return cudaGetLastError();
+  for (int i = 0; i < n; ++i)
+    if (cache[i].f == func && cache[i].dev == dev && cache[i].bytes >= bytes) return cudaSuccess;
+  const cudaError_t e = cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+  if (e != cudaSuccess) return e;
+  for (int i = 0; i < n; ++i)
+    if (cache[i].f == func && cache[i].dev == dev) {
+      cache[i].bytes = bytes;
+      return cudaSuccess;
+    }
+  if (n < 64) cache[n++] = Entry{func, dev, bytes};
+  return cudaSuccess;
+}
 
 int device_sm_count() {
   static int cache[64] = {0};
@@ -219,6 +283,7 @@ sa_status sparse_attn_select(const sa_kv_desc* kv, const void* meta, sa_score_ru
   a.scores_out = scores_out;
   a.ws_scores = reinterpret_cast<float*>(reinterpret_cast<char*>(ws) + kScratch);
   a.ws_count = reinterpret_cast<uint32_t*>(reinterpret_cast<char*>(ws) + 256);
+  a.ws_queue = reinterpret_cast<uint32_t*>(reinterpret_cast<char*>(ws) + kQueueSelect);
   a.status = reinterpret_cast<int*>(ws);
   a.splits = select_splits((int)units, kv->max_pages, device_sm_count());
   return launched(launch_select(a, (cudaStream_t)stream));
@@ -246,11 +311,16 @@ sa_status sparse_attn_decode(const sa_kv_desc* kv, const void* q, int32_t n_q_he
   if (kv->page_size == 0 && max_sel > kMaxChunkSel) return SA_ERR_UNSUPPORTED;
   const long long units = (long long)n_q_rows * kv->n_kv_heads;
   if (units > kMaxUnits) return SA_ERR_UNSUPPORTED;
+  const unsigned long long kv_rows = (unsigned long long)kv->batch * kv->n_kv_heads * kv->cap_tokens;
+  if (kv_rows > 0x7fffffffULL) return SA_ERR_UNSUPPORTED;  // TMA row coordinates are int32
   const int splits = decode_splits((int)units, max_tiles_per_unit(kv, max_sel), device_sm_count());
   const size_t need = kScratch + decode_scratch((int)units, splits);
   if ((s = check_ws(ws, ws_bytes, need)) != SA_OK) return s;
 
   DecodeArgs a;
+  if (!encode_tmap_2d(&a.tmap_k, kv->k, kv_rows, kHeadDim * 2, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, 16) ||
+      !encode_tmap_2d(&a.tmap_v, kv->v, kv_rows, kHeadDim * 2, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, 16))
+    return SA_ERR_CUDA;
   a.kv = view(kv);
   a.q = q;
   a.Hq = n_q_heads;
@@ -266,6 +336,7 @@ sa_status sparse_attn_decode(const sa_kv_desc* kv, const void* q, int32_t n_q_he
   a.lse = lse;
   a.ws_part = reinterpret_cast<float*>(reinterpret_cast<char*>(ws) + kScratch);
   a.ws_count = reinterpret_cast<uint32_t*>(reinterpret_cast<char*>(ws) + 256);
+  a.ws_queue = reinterpret_cast<uint32_t*>(reinterpret_cast<char*>(ws) + kQueueDecode);
   a.status = reinterpret_cast<int*>(ws);
   a.splits = splits;
   return launched(launch_decode(a, (cudaStream_t)stream));

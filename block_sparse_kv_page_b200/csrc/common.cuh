@@ -16,6 +16,8 @@
 #include <cuda_bf16.h>
 #include <stdint.h>
 
+#include "sparse_attn.h"
+
 #define SA_DEV __device__ __forceinline__
 
 namespace sa {
@@ -29,6 +31,11 @@ constexpr float kLn2 = 0.6931471805599453f;
 // ---------------------------------------------------------------- async copy
 SA_DEV uint32_t smem_addr(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+// Record the first device-side error code in the workspace status word.
+SA_DEV void flag_status(int* status, int code) {
+  if (status) atomicCAS(status, 0, code);
 }
 
 // 16-byte global -> shared copy; when !valid nothing is read and zeros land.
@@ -58,6 +65,68 @@ SA_DEV uint4 ldg_nc128(const void* p) {
                : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
                : "l"(p));
   return r;
+}
+
+// ---------------------------------------------------------------- TMA + mbarrier
+// 2D tiled bulk copies (no multicast) completing on a CTA-local mbarrier.
+constexpr uint32_t kSpinLimit = 1u << 22;  // bounded waits: give up and flag SA_ERR_TIMEOUT
+
+SA_DEV void mbar_init(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;\n" ::"r"(smem_addr(bar)), "r"(count) : "memory");
+}
+SA_DEV void fence_barrier_init() {
+  asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
+  asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
+}
+SA_DEV void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;\n" ::"r"(smem_addr(bar)), "r"(bytes)
+               : "memory");
+}
+SA_DEV bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}\n"
+      : "=r"(ok)
+      : "r"(smem_addr(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+// Wait for phase `parity` of `bar`; after kSpinLimit polls give up, flag the
+// status word and return false (the caller stops using the stage).
+SA_DEV bool mbar_wait(uint64_t* bar, uint32_t parity, int* status) {
+  for (uint32_t i = 0; i < kSpinLimit; ++i)
+    if (mbar_try_wait(bar, parity)) return true;
+  flag_status(status, SA_ERR_TIMEOUT);
+  return false;
+}
+SA_DEV void tma_load_2d(void* dst, const void* tmap, int x, int y, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes "
+      "[%0], [%1, {%2, %3}], [%4];\n" ::"r"(smem_addr(dst)),
+      "l"(tmap), "r"(x), "r"(y), "r"(smem_addr(bar))
+      : "memory");
+}
+SA_DEV void mbar_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];\n" ::"r"(smem_addr(bar)) : "memory");
+}
+SA_DEV void fence_proxy_async() { asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory"); }
+SA_DEV void prefetch_tmap(const void* tmap) {
+  asm volatile("prefetch.tensormap [%0];\n" ::"l"(tmap) : "memory");
+}
+
+// Byte offset of 16-byte chunk j (0..7) of row r inside a 128B-swizzled box
+// whose rows are 128 bytes (the TMA SWIZZLE_128B pattern: chunk j ^ (r & 7)).
+SA_DEV uint32_t swz128(int r, int j) { return (uint32_t)(r * 128 + ((j ^ (r & 7)) << 4)); }
+
+SA_DEV void ldsm_x4(uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3, const void* p) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];\n"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(smem_addr(p)));
+}
+SA_DEV void ldsm_x4_t(uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3, const void* p) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];\n"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(smem_addr(p)));
 }
 
 // ---------------------------------------------------------------- tensor-core MMA
@@ -129,11 +198,6 @@ SA_DEV uint32_t bf16x2_pos_part(uint32_t x) {
 SA_DEV uint32_t order_key(float s) {
   uint32_t u = __float_as_uint(s + 0.0f);
   return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
-}
-
-// ---------------------------------------------------------------- status word
-SA_DEV void flag_status(int* status, int code) {
-  if (status) atomicCAS(status, 0, code);
 }
 
 // ---------------------------------------------------------------- block scans

@@ -2,6 +2,7 @@
 // kernel files.  Host-only declarations; not part of the public ABI.
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stddef.h>
 #include <stdint.h>
@@ -35,6 +36,13 @@ struct WsLayout {
 };
 
 int device_sm_count();
+// Encode a 2D tiled tensor map: `rows` rows of `row_bytes` bytes at `base`,
+// element type `dt` of `elem_bytes`, box = box_rows x 128 bytes, 128B swizzle.
+bool encode_tmap_2d(CUtensorMap* map, const void* base, unsigned long long rows, int row_bytes,
+                    CUtensorMapDataType dt, int elem_bytes, int box_rows);
+// Opt a kernel into `bytes` of dynamic shared memory on the current device
+// (cached per device and kernel, so repeated launches skip the driver call).
+cudaError_t set_smem_attr(const void* func, size_t bytes);
 int decode_splits(int units, int max_tiles, int sm_count);
 int select_splits(int units, int max_pages, int sm_count);
 WsLayout workspace_layout(const sa_kv_desc* kv, int n_q_heads, int n_q_rows, int max_sel,
@@ -44,6 +52,7 @@ cudaError_t launch_build_meta(const KvView& kv, int rule, int first_token, void*
                               int* status, cudaStream_t st);
 
 struct SelectArgs {
+  CUtensorMap tmap_meta;      // metadata rows [B*Hkv*max_pages][512 B], boxes 16 x 128 B, 128B swizzle
   KvView kv;
   const void* meta;
   int rule;
@@ -57,12 +66,15 @@ struct SelectArgs {
   float* scores_out;
   float* ws_scores;
   uint32_t* ws_count;
+  uint32_t* ws_queue;         // [2] persistent-grid item queue (head, finished CTAs)
   int* status;
   int splits;
 };
 cudaError_t launch_select(const SelectArgs& a, cudaStream_t st);
 
 struct DecodeArgs {
+  CUtensorMap tmap_k;         // K rows [B*Hkv*cap][128 bf16], boxes 16 x 64, 128B swizzle
+  CUtensorMap tmap_v;         // V, same geometry
   KvView kv;
   const void* q;
   int Hq, G;
@@ -75,6 +87,7 @@ struct DecodeArgs {
   float* lse;
   float* ws_part;
   uint32_t* ws_count;
+  uint32_t* ws_queue;
   int* status;
   int splits;
 };

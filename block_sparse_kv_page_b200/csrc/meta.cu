@@ -36,6 +36,7 @@ __device__ int chunk_containing(const int32_t* off, int n, int t) {
   return lo;
 }
 
+template <int RULE>
 __global__ void __launch_bounds__(kMetaWarps * 32) build_meta_kernel(MetaParams p) {
   const int lane = threadIdx.x & 31;
   const long long wid = (long long)blockIdx.x * kMetaWarps + (threadIdx.x >> 5);
@@ -93,36 +94,33 @@ __global__ void __launch_bounds__(kMetaWarps * 32) build_meta_kernel(MetaParams 
     mx[i] = -__int_as_float(0x7f800000);
     sm[i] = 0.0;
   }
-  int t = s;
-  for (; t + 4 <= e; t += 4) {
-    uint2 r[4];
+  // 16 rows per batch, all loads issued before any is used
+  for (int t = s; t < e; t += 16) {
+    const int n = min(16, e - t);
+    uint2 r[16];
 #pragma unroll
-    for (int x = 0; x < 4; ++x)
-      r[x] = __ldg(reinterpret_cast<const uint2*>(K + (size_t)(t + x) * kHeadDim));
+    for (int x = 0; x < 16; ++x)
+      r[x] = x < n ? __ldg(reinterpret_cast<const uint2*>(K + (size_t)(t + x) * kHeadDim))
+                   : make_uint2(0u, 0u);
 #pragma unroll
-    for (int x = 0; x < 4; ++x) {
-      const float f[4] = {bf16_lo(r[x].x), bf16_hi(r[x].x), bf16_lo(r[x].y), bf16_hi(r[x].y)};
+    for (int x = 0; x < 16; ++x) {
+      if (x < n) {
+        const float f[4] = {bf16_lo(r[x].x), bf16_hi(r[x].x), bf16_lo(r[x].y), bf16_hi(r[x].y)};
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        mn[i] = fminf(mn[i], f[i]);
-        mx[i] = fmaxf(mx[i], f[i]);
-        sm[i] += (double)f[i];
+        for (int i = 0; i < 4; ++i) {
+          if (RULE == 0) {
+            mn[i] = fminf(mn[i], f[i]);
+            mx[i] = fmaxf(mx[i], f[i]);
+          } else {
+            sm[i] += (double)f[i];
+          }
+        }
       }
-    }
-  }
-  for (; t < e; ++t) {
-    const uint2 r = __ldg(reinterpret_cast<const uint2*>(K + (size_t)t * kHeadDim));
-    const float f[4] = {bf16_lo(r.x), bf16_hi(r.x), bf16_lo(r.y), bf16_hi(r.y)};
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      mn[i] = fminf(mn[i], f[i]);
-      mx[i] = fmaxf(mx[i], f[i]);
-      sm[i] += (double)f[i];
     }
   }
 
   unsigned char* dst = p.meta + ((size_t)u * p.kv.max_pages + page) * kMetaBytes;
-  if (p.rule == 0) {
+  if (RULE == 0) {
     // bf16 values: min/max of bf16 inputs are bf16 inputs, so the casts are exact.
     uint2 lo, hi;
     lo.x = pack_bf16(mn[0], mn[1]);
@@ -157,7 +155,8 @@ cudaError_t launch_build_meta(const KvView& kv, int rule, int first_token, void*
     ppu = kv.page_size > 0 ? kv.max_pages - first_token / kv.page_size : kv.max_pages;
   } else {
     const long long n = -(long long)first_token;
-    ppu = kv.page_size > 0 ? (int)((n + kv.page_size - 1) / kv.page_size + 1)
+    // pages overlapping the last n tokens: ceil((n - 1) / ps) + 1 at most
+    ppu = kv.page_size > 0 ? (int)((n - 1 + kv.page_size - 1) / kv.page_size + 1)
                            : (int)(n < kv.max_pages ? n : kv.max_pages);
   }
   if (ppu > kv.max_pages) ppu = kv.max_pages;
@@ -166,7 +165,10 @@ cudaError_t launch_build_meta(const KvView& kv, int rule, int first_token, void*
   const long long warps = (long long)kv.B * kv.Hkv * ppu;
   const long long blocks = (warps + kMetaWarps - 1) / kMetaWarps;
   if (blocks > 0x7fffffffLL) return cudaErrorInvalidValue;
-  build_meta_kernel<<<(unsigned)blocks, kMetaWarps * 32, 0, st>>>(p);
+  if (rule == 0)
+    build_meta_kernel<0><<<(unsigned)blocks, kMetaWarps * 32, 0, st>>>(p);
+  else
+    build_meta_kernel<1><<<(unsigned)blocks, kMetaWarps * 32, 0, st>>>(p);
   return cudaGetLastError();
 }
 

@@ -9,14 +9,16 @@
 // max(topk_val + bos + eos, int(blocks * ratio)) with forced bos/eos blocks.
 //
 // Work split.  A unit is one (sequence, KV head).  Its pages are cut into
-// `splits` contiguous ranges of 16-page tiles, one CTA (4 warps) per range.
-// Each warp streams its tiles of 16 metadata rows (512 B each) through a
-// private 3-stage cp.async ring and scores them for all G grouped query heads
-// with one warp-level tensor-core product per tile:
+// `splits` contiguous ranges of 16-page tiles; an item is one (unit, range).
+// A persistent grid pulls items from an atomic queue.  Each of a CTA's 4
+// warps streams its tiles of 16 metadata rows (512 B each) through a private
+// 3-stage cp.async ring (every load instruction covers whole 32-byte sectors)
+// and scores them for all G grouped query heads with tensor-core products:
 //   envelope: S^T[16 pages x 8 heads] = [kmin | kmax] (16 x 256, bf16)
 //             x [q- | q+]^T (256 x 8, bf16), m16n8k16, exact products;
-//   centroid: S^T = kmean (16 x 128, fp32 split into two tf32 terms)
-//             x q^T (128 x 8, exact in tf32), m16n8k8.
+//   centroid: S^T = kmean (16 x 128, fp32) x q^T (128 x 8, bf16), on the
+//             FP64 tensor cores (m8n8k4): exact products and sums, one final
+//             rounding to fp32, so near-ties are resolved as in float64.
 // The group score (max over the G heads) goes to the workspace.  The CTA that
 // finishes a unit last (atomic counter; nobody waits) loads the unit's scores
 // and selects: a weighted MSB-first radix select on order-preserving 32-bit
@@ -32,6 +34,13 @@
 namespace sa {
 namespace {
 
+#ifndef SA_SEL_ITEM_PAGES
+#define SA_SEL_ITEM_PAGES 256
+#endif
+#ifndef SA_SEL_CTAS_PER_SM
+#define SA_SEL_CTAS_PER_SM 2
+#endif
+
 constexpr int kSelWarps = 4;
 constexpr int kSelThreads = kSelWarps * 32;
 constexpr int kSelStages = 3;
@@ -43,7 +52,7 @@ constexpr int kRingBytes = kSelWarps * kSelStages * kStageBytes;
 template <int RULE>
 SA_DEV int chunk_byte(int j, int c) {
   if (RULE == 0) return 16 * (4 * j + c);                 // bf16: elements 32j + 8c .. +8
-  return 16 * (8 * (j >> 1) + 2 * c + (j & 1));          // fp32: floats 32(j/2) + 8c + 4(j&1) .. +4
+  return 16 * (8 * (j >> 1) + 4 * (j & 1) + c);          // fp32: floats 32(j/2) + 16(j&1) + 4c .. +4
 }
 
 struct RadixCut {
@@ -107,18 +116,24 @@ SA_DEV RadixCut radix_cut(const uint32_t* keys, const uint32_t* wts, int P, uint
   return {prefix, rem};
 }
 
+struct SelSmem {
+  unsigned char* smem;   // max(ring, 8 * max_pages) bytes
+  uint32_t* hist;        // 256
+  uint32_t* scan;        // 32
+  uint32_t* bc;          // 4
+  int* last;
+};
+
 template <int RULE>
-__global__ void __launch_bounds__(kSelThreads) select_kernel(SelectArgs a) {
-  extern __shared__ __align__(128) unsigned char smem[];
-  __shared__ uint32_t s_hist[256];
-  __shared__ uint32_t s_scan[32];
-  __shared__ uint32_t s_bc[4];
-  __shared__ int s_last;
+SA_DEV void select_item(const SelectArgs& a, const int u, const int split, const SelSmem& S) {
+  unsigned char* smem = S.smem;
+  uint32_t* s_hist = S.hist;
+  uint32_t* s_scan = S.scan;
+  uint32_t* s_bc = S.bc;
+  int& s_last = *S.last;
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int gq = lane >> 2, c = lane & 3;
-  const int u = blockIdx.x / a.splits;
-  const int split = blockIdx.x % a.splits;
   const int Hkv = a.kv.Hkv;
   const int b = u / Hkv, g = u % Hkv;
 
@@ -161,15 +176,18 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(SelectArgs a) {
       bq[4 * j + 0] = v.x; bq[4 * j + 1] = v.y; bq[4 * j + 2] = v.z; bq[4 * j + 3] = v.w;
     }
   } else {
-    // q[head][32i + 8c + e] as fp64, e = 0..7 (k-step 8i + e of the m8n8k4 chain)
+    // bd[8i + 4h + r] = q[head][32i + 16h + 4c + r] as fp64: the same dimensions
+    // as the metadata chunk (i, h) this lane loads (k-step (2i + h, r))
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-      const uint4 v = head_ok ? ldg_nc128(qrow + 32 * i + 8 * c) : make_uint4(0, 0, 0, 0);
-      const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        bd[8 * i + 2 * e + 0] = (double)bf16_lo(w[e]);
-        bd[8 * i + 2 * e + 1] = (double)bf16_hi(w[e]);
+      for (int hh = 0; hh < 2; ++hh) {
+        uint2 v = make_uint2(0, 0);
+        if (head_ok) v = __ldg(reinterpret_cast<const uint2*>(qrow + 32 * i + 16 * hh + 4 * c));
+        bd[8 * i + 4 * hh + 0] = (double)bf16_lo(v.x);
+        bd[8 * i + 4 * hh + 1] = (double)bf16_hi(v.x);
+        bd[8 * i + 4 * hh + 2] = (double)bf16_lo(v.y);
+        bd[8 * i + 4 * hh + 3] = (double)bf16_hi(v.y);
       }
     }
   }
@@ -219,7 +237,7 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(SelectArgs a) {
       // fp64, so the only rounding left is the final fp64 -> fp32 of the score.
       double c00 = 0.0, c01 = 0.0, c10 = 0.0, c11 = 0.0;  // pages gq / gq + 8
 #pragma unroll
-      for (int j = 0; j < 8; ++j) {  // chunk j = floats 32(j/2) + 8c + 4(j&1) .. +4
+      for (int j = 0; j < 8; ++j) {  // chunk j = floats 32(j/2) + 16(j&1) + 4c .. +4
         const uint4 r0 = lds128(st + j * kSlotBytes);
         const uint4 r1 = lds128(st + (8 + j) * kSlotBytes);
         const uint32_t a0[4] = {r0.x, r0.y, r0.z, r0.w}, a1[4] = {r1.x, r1.y, r1.z, r1.w};
@@ -352,13 +370,44 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(SelectArgs a) {
   }
 }
 
+template <int RULE>
+__global__ void __launch_bounds__(kSelThreads) select_kernel(SelectArgs a) {
+  extern __shared__ __align__(128) unsigned char smem[];
+  __shared__ uint32_t s_hist[256];
+  __shared__ uint32_t s_scan[32];
+  __shared__ uint32_t s_bc[4];
+  __shared__ int s_last, s_item;
+  const SelSmem S{smem, s_hist, s_scan, s_bc, &s_last};
+  const int n_items = a.kv.B * a.kv.Hkv * a.splits;
+  for (;;) {
+    if (threadIdx.x == 0) s_item = (int)atomicAdd(&a.ws_queue[0], 1u);
+    __syncthreads();
+    const int item = s_item;
+    if (item >= n_items) break;
+    select_item<RULE>(a, item / a.splits, item % a.splits, S);
+    __syncthreads();
+  }
+  // the last CTA out rewinds the queue for the next launch
+  if (threadIdx.x == 0) {
+    __threadfence();
+    if (atomicAdd(&a.ws_queue[1], 1u) == gridDim.x - 1) {
+      a.ws_queue[0] = 0;
+      a.ws_queue[1] = 0;
+    }
+  }
+}
+
 }  // namespace
 
+// Splits per unit: items of about SA_SEL_ITEM_PAGES pages, but at least two
+// items per SM when there are few units, and at least one tile per warp.
 int select_splits(int units, int max_pages, int sm_count) {
-  const int target = 2 * sm_count;                   // two resident CTAs per SM
-  int s = (target + units - 1) / units;
-  const int max_s = (max_pages + 63) / 64;           // at least 64 pages (one tile per warp)
-  if (s > max_s) s = max_s;
+  int s = (max_pages + SA_SEL_ITEM_PAGES - 1) / SA_SEL_ITEM_PAGES;
+  const int fill = (2 * sm_count + units - 1) / units;
+  if (fill > s) s = fill;
+  const int cap = (max_pages + 16 * kSelWarps - 1) / (16 * kSelWarps);
+  if (s > cap) s = cap;
+  if (s > 256) s = 256;
   if (s < 1) s = 1;
   return s;
 }
@@ -370,15 +419,18 @@ size_t select_smem_bytes(int max_pages) {
 
 cudaError_t launch_select(const SelectArgs& a, cudaStream_t st) {
   const size_t smem = select_smem_bytes(a.kv.max_pages);
-  const long long grid = (long long)a.kv.B * a.kv.Hkv * a.splits;
-  if (grid > 0x7fffffffLL) return cudaErrorInvalidValue;
+  const long long items = (long long)a.kv.B * a.kv.Hkv * a.splits;
+  if (items > 0x7fffffffLL) return cudaErrorInvalidValue;
+  const int ctas_per_sm = smem <= (size_t)kRingBytes ? SA_SEL_CTAS_PER_SM : 1;
+  long long grid = (long long)device_sm_count() * ctas_per_sm;
+  if (grid > items) grid = items;
   cudaError_t e;
   if (a.rule == 0) {
-    e = cudaFuncSetAttribute(select_kernel<0>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    e = set_smem_attr((const void*)select_kernel<0>, smem);
     if (e != cudaSuccess) return e;
     select_kernel<0><<<(unsigned)grid, kSelThreads, smem, st>>>(a);
   } else {
-    e = cudaFuncSetAttribute(select_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    e = set_smem_attr((const void*)select_kernel<1>, smem);
     if (e != cudaSuccess) return e;
     select_kernel<1><<<(unsigned)grid, kSelThreads, smem, st>>>(a);
   }
