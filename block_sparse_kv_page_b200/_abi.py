@@ -69,6 +69,9 @@ PROTOTYPES = {
                                     C.c_int32, C.c_int32, C.c_int32, C.c_int32, C.c_int32, C.c_float,
                                     C.c_void_p, C.c_void_p, C.c_void_p, C.c_void_p, C.c_void_p, C.c_void_p,
                                     C.c_void_p, C.c_void_p, C.c_size_t, C.c_void_p]),
+    "sparse_attn_decode_static": (C.c_int, [C.POINTER(sa_kv_desc), C.c_void_p, C.c_int32, C.c_int32,
+                                            C.c_int32, C.c_int32, C.c_float, C.c_void_p, C.c_void_p,
+                                            C.c_int32, C.c_void_p, C.c_void_p, C.c_void_p, C.c_void_p]),
     "sparse_attn_get_device_status": (C.c_int, [C.c_void_p, C.POINTER(C.c_int), C.c_void_p]),
     "sparse_attn_status_string": (C.c_char_p, [C.c_int]),
 }

@@ -396,3 +396,104 @@ const char* sparse_attn_status_string(sa_status s) {
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Decode with library-owned scratch, for callers that cannot allocate device
+// memory where they call us (see sparse_attn_decode_static in sparse_attn.h).
+// The scratch is this file's device array; host code only ever uses the
+// address that cudaGetSymbolAddress returns for the current device.
+namespace sa {
+namespace {
+constexpr size_t kStaticScratchBytes = (size_t)8 << 20;
+constexpr int kStaticMaxUnits = 4096;
+constexpr size_t kStaticPartOff = 256 + 4 * (size_t)kStaticMaxUnits;  // after status/queues/counters
+static_assert(kStaticPartOff % 256 == 0, "partials must stay 256-byte aligned");
+}  // namespace
+}  // namespace sa
+
+static __device__ __align__(256) unsigned char g_decode_scratch[sa::kStaticScratchBytes];
+
+namespace sa {
+namespace {
+// Device address of g_decode_scratch on the current device (looked up once per device).
+sa_status static_scratch(unsigned char** out) {
+  static unsigned char* addr[64] = {nullptr};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) {
+    cudaGetLastError();
+    return SA_ERR_CUDA;
+  }
+  if (!addr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_decode_scratch) != cudaSuccess || !p) {
+      cudaGetLastError();
+      return SA_ERR_CUDA;
+    }
+    addr[dev] = static_cast<unsigned char*>(p);
+  }
+  *out = addr[dev];
+  return SA_OK;
+}
+}  // namespace
+}  // namespace sa
+
+extern "C" sa_status sparse_attn_decode_static(const sa_kv_desc* kv, const void* q, int32_t n_q_heads,
+                                               int32_t n_q_rows, int32_t q_pos0, int32_t tile_rows,
+                                               float scale, const int32_t* idx, const int32_t* count,
+                                               int32_t max_sel, float* out, float* lse,
+                                               int32_t* device_status, void* stream) {
+  sa_status s = check_kv(kv);
+  if (s != SA_OK) return s;
+  int G;
+  if ((s = check_group(kv, n_q_heads, &G)) != SA_OK) return s;
+  if (!q || !aligned(q, 16) || !idx || !count || !aligned(idx, 4) || !aligned(count, 4))
+    return SA_ERR_INVALID;
+  if (!out || !aligned(out, 16) || (lse && !aligned(lse, 4))) return SA_ERR_INVALID;
+  if (device_status && !aligned(device_status, 4)) return SA_ERR_INVALID;
+  if (max_sel < 1 || tile_rows < 1 || n_q_rows < 1) return SA_ERR_INVALID;
+  if (!std::isfinite(scale)) return SA_ERR_INVALID;
+  if (tile_rows == 1) {
+    if (n_q_rows != kv->batch) return SA_ERR_INVALID;
+  } else {
+    if (kv->batch != 1 || kv->page_size == 0) return SA_ERR_INVALID;
+    return SA_ERR_UNSUPPORTED;
+  }
+  if (kv->page_size == 0 && max_sel > kMaxChunkSel) return SA_ERR_UNSUPPORTED;
+  const long long units = (long long)n_q_rows * kv->n_kv_heads;
+  if (units > kStaticMaxUnits) return SA_ERR_WORKSPACE;  // beyond the built-in scratch
+  const unsigned long long kv_rows = (unsigned long long)kv->batch * kv->n_kv_heads * kv->cap_tokens;
+  if (kv_rows > 0x7fffffffULL) return SA_ERR_UNSUPPORTED;
+  const int splits = decode_splits((int)units, max_tiles_per_unit(kv, max_sel), device_sm_count());
+  if (kStaticPartOff + decode_scratch((int)units, splits) > kStaticScratchBytes) return SA_ERR_WORKSPACE;
+
+  unsigned char* scratch = nullptr;
+  if ((s = static_scratch(&scratch)) != SA_OK) return s;
+  DecodeArgs a;
+  if (!encode_tmap_2d(&a.tmap_k, kv->k, kv_rows, kHeadDim * 2, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, 16) ||
+      !encode_tmap_2d(&a.tmap_v, kv->v, kv_rows, kHeadDim * 2, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, 16))
+    return SA_ERR_CUDA;
+  // status word, queue and the counters of this call's units start at zero
+  if (cudaMemsetAsync(scratch, 0, 256 + 4 * (size_t)units, (cudaStream_t)stream) != cudaSuccess) {
+    cudaGetLastError();
+    return SA_ERR_CUDA;
+  }
+  a.kv = view(kv);
+  a.q = q;
+  a.Hq = n_q_heads;
+  a.G = G;
+  a.n_rows = n_q_rows;
+  a.q_pos0 = q_pos0;
+  a.tile_rows = tile_rows;
+  a.scale_log2 = scale * kLog2e;
+  a.idx = idx;
+  a.count = count;
+  a.max_sel = max_sel;
+  a.out = out;
+  a.lse = lse;
+  a.ws_part = reinterpret_cast<float*>(scratch + kStaticPartOff);
+  a.ws_count = reinterpret_cast<uint32_t*>(scratch + 256);
+  a.ws_queue = reinterpret_cast<uint32_t*>(scratch + kQueueDecode);
+  a.status = device_status ? reinterpret_cast<int*>(device_status) : reinterpret_cast<int*>(scratch);
+  a.splits = splits;
+  return launched(launch_decode(a, (cudaStream_t)stream));
+}

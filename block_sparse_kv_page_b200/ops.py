@@ -144,6 +144,26 @@ def sparse_attn_decode(kv: KvCache, q: torch.Tensor, n_q_rows: int, q_pos0: int,
            "sparse_attn_decode")
 
 
+def sparse_attn_decode_static(kv: KvCache, q: torch.Tensor, n_q_rows: int, q_pos0: int,
+                              tile_rows: int, scale: float, idx: torch.Tensor, count: torch.Tensor,
+                              max_sel: int, out: torch.Tensor, lse: torch.Tensor | None,
+                              device_status: torch.Tensor | None = None, stream=None) -> None:
+    """sparse_attn_decode without a workspace, for callers that cannot
+    allocate device memory where they run it: the scratch is an 8 MiB array
+    inside the library, shared by every call, so calls must not overlap on
+    the GPU.  device_status: optional zeroed int32 device tensor that receives
+    the first device-side error code."""
+    if q.dtype != torch.bfloat16 or not q.is_contiguous():
+        raise ValueError("q must be contiguous bf16")
+    if out.dtype != torch.float32 or not out.is_contiguous():
+        raise ValueError("out must be contiguous fp32")
+    _check(lib.sparse_attn_decode_static(C.byref(kv.desc), q.data_ptr(), q.shape[-2], int(n_q_rows),
+                                         int(q_pos0), int(tile_rows), float(scale), idx.data_ptr(),
+                                         count.data_ptr(), int(max_sel), out.data_ptr(), _ptr(lse),
+                                         _ptr(device_status), _stream(stream)),
+           "sparse_attn_decode_static")
+
+
 def sparse_attn_route(kv: KvCache, meta: torch.Tensor, rule, q: torch.Tensor, n_q_rows: int,
                       q_pos0: int, tile_rows: int, k: int, rho: int, quantile: float,
                       tau: torch.Tensor | None, kv_idx: torch.Tensor, kv_count: torch.Tensor,

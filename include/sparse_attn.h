@@ -193,6 +193,35 @@ sa_status sparse_attn_route(const sa_kv_desc* kv, const void* meta, sa_score_rul
  * fired since the last init/clear) and clear it.  Synchronises `stream`. */
 sa_status sparse_attn_get_device_status(void* ws, sa_status* host_out, void* stream);
 
+/* (c') Sparse attention without a caller-provided workspace.
+ * The pages have no counterpart for this call; it exists for deployment.
+ * Some callers cannot allocate device memory at the point where they run the
+ * attention: a plugin interface that hands an op only its input and output
+ * pointers at enqueue time, or a latency-bound decode loop that must never
+ * pay the device-wide synchronisation that cudaMalloc can cause.  For them
+ * this call computes exactly what sparse_attn_decode computes (same arguments
+ * minus ws/ws_bytes) using a scratch area built into the library: one
+ * file-scope device array of 8 MiB, which every GPU that loads the library
+ * holds until the process exits.
+ *  - The first call on a device, with that device current, looks up the
+ *    array's device address and caches it; make that first call before any
+ *    stream capture.
+ *  - Every call shares the one array and overwrites it.  Calls that may run at
+ *    the same time on the GPU (different streams, overlapping graph launches,
+ *    several host threads) race and corrupt each other's results: order them
+ *    on one stream.  Each call clears the counters it uses before launching.
+ *  - Limits: at most 4096 (row, KV head) units per call, and the split
+ *    partials of the call must fit the array; beyond either the call returns
+ *    SA_ERR_WORKSPACE and launches nothing.
+ *  - It allocates and frees no memory.
+ *  - device_status (nullable): a device int32, zeroed by the caller, that
+ *    receives the first device-side error code of the call. */
+sa_status sparse_attn_decode_static(const sa_kv_desc* kv, const void* q, int32_t n_q_heads,
+                                    int32_t n_q_rows, int32_t q_pos0, int32_t tile_rows,
+                                    float scale, const int32_t* idx, const int32_t* count,
+                                    int32_t max_sel, float* out, float* lse,
+                                    int32_t* device_status, void* stream);
+
 /* Static description of a status code (never null). */
 const char* sparse_attn_status_string(sa_status s);
 
