@@ -262,8 +262,15 @@ sa_status sparse_attn_select(const sa_kv_desc* kv, const void* meta, sa_score_ru
   }
   const size_t need = kScratch + select_scratch(kv);
   if ((s = check_ws(ws, ws_bytes, need)) != SA_OK) return s;
+  const unsigned long long meta_rows = (unsigned long long)units * kv->max_pages;
+  if (meta_rows > 0x7fffffffULL) return SA_ERR_UNSUPPORTED;  // TMA row coordinates are int32
 
   SelectArgs a;
+  const bool env = rule == SA_SCORE_ENVELOPE;
+  if (!encode_tmap_2d(&a.tmap_meta, meta, meta_rows, kMetaBytes,
+                      env ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32,
+                      env ? 2 : 4, 16))
+    return SA_ERR_CUDA;
   a.kv = view(kv);
   a.meta = meta;
   a.rule = (int)rule;

@@ -35,13 +35,13 @@
 #define SA_DEC_WARPS 4
 #endif
 #ifndef SA_DEC_STAGES
-#define SA_DEC_STAGES 4
+#define SA_DEC_STAGES 2
 #endif
 #ifndef SA_DEC_ITEM_TILES
 #define SA_DEC_ITEM_TILES 64
 #endif
 #ifndef SA_DEC_CTAS_PER_SM
-#define SA_DEC_CTAS_PER_SM 1
+#define SA_DEC_CTAS_PER_SM 3
 #endif
 
 namespace sa {

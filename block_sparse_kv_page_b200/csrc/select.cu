@@ -10,127 +10,76 @@
 //
 // Work split.  A unit is one (sequence, KV head).  Its pages are cut into
 // `splits` contiguous ranges of 16-page tiles; an item is one (unit, range).
-// A persistent grid pulls items from an atomic queue.  Each of a CTA's 4
-// warps streams its tiles of 16 metadata rows (512 B each) through a private
-// 3-stage cp.async ring (every load instruction covers whole 32-byte sectors)
-// and scores them for all G grouped query heads with tensor-core products:
+// A persistent grid pulls items from an atomic queue.
+//
+// Scoring.  The metadata of a tile (16 pages x 512 B) arrives by TMA as four
+// 16 x 128-byte boxes, 128B-swizzled, into a per-warp mbarrier ring; lane 0
+// of each warp keeps several tiles in flight.  All G grouped query heads are
+// scored on tensor cores:
 //   envelope: S^T[16 pages x 8 heads] = [kmin | kmax] (16 x 256, bf16)
-//             x [q- | q+]^T (256 x 8, bf16), m16n8k16, exact products;
-//   centroid: S^T = kmean (16 x 128, fp32) x q^T (128 x 8, bf16), on the
-//             FP64 tensor cores (m8n8k4): exact products and sums, one final
-//             rounding to fp32, so near-ties are resolved as in float64.
-// The group score (max over the G heads) goes to the workspace.  The CTA that
-// finishes a unit last (atomic counter; nobody waits) loads the unit's scores
-// and selects: a weighted MSB-first radix select on order-preserving 32-bit
-// keys finds the cut key T and the capacity left for keys equal to T; equal
-// keys are then taken in ascending page order (the lowest-index tie rule), so
-// the result is exactly "the longest prefix of the (score desc, index asc)
-// order within the budget".  Weight 1 per page gives top-k / ratio; weight =
-// chunk length gives the token budget.  Output is the kept set in ascending
-// page order.
+//             x [q- | q+]^T (256 x 8, bf16), m16n8k16 via ldmatrix, exact
+//             products, fp32 accumulation;
+//   centroid: S^T = kmean (16 x 128, fp32) x q^T (128 x 8, bf16) on the FP64
+//             tensor cores (m8n8k4): exact products and sums, one rounding to
+//             fp32, so near-ties are resolved as in float64.
+// The group score (max over the G heads) goes to the workspace.
+//
+// Selection.  The CTA that finishes a unit's last item (atomic counter;
+// nobody waits) loads the unit's scores and runs a weighted MSB-first radix
+// select on order-preserving 32-bit keys: it finds the cut key T and the
+// capacity left for keys equal to T; equal keys are then taken in ascending
+// page order (the lowest-index tie rule), so the result is exactly "the
+// longest prefix of the (score desc, index asc) order within the budget".
+// Weight 1 per page gives top-k / ratio; weight = chunk length gives the token
+// budget.  Output is the kept set in ascending page order.
 #include "common.cuh"
 #include "internal.h"
+#include "radix.cuh"
+
+#ifndef SA_SEL_ITEM_PAGES
+#define SA_SEL_ITEM_PAGES 512
+#endif
+#ifndef SA_SEL_STAGES
+#define SA_SEL_STAGES 2
+#endif
+#ifndef SA_SEL_CTAS_PER_SM
+#define SA_SEL_CTAS_PER_SM 3
+#endif
 
 namespace sa {
 namespace {
 
-#ifndef SA_SEL_ITEM_PAGES
-#define SA_SEL_ITEM_PAGES 256
-#endif
-#ifndef SA_SEL_CTAS_PER_SM
-#define SA_SEL_CTAS_PER_SM 2
-#endif
-
 constexpr int kSelWarps = 4;
 constexpr int kSelThreads = kSelWarps * 32;
-constexpr int kSelStages = 3;
-constexpr int kSlotBytes = 32 * 16;              // one 16-byte chunk per lane
-constexpr int kStageBytes = 16 * kSlotBytes;     // 16 chunks per lane = 16 rows x 512 B
-constexpr int kRingBytes = kSelWarps * kSelStages * kStageBytes;
-
-// Byte offset, inside a 512-byte metadata row, of the j-th chunk lane c loads.
-template <int RULE>
-SA_DEV int chunk_byte(int j, int c) {
-  if (RULE == 0) return 16 * (4 * j + c);                 // bf16: elements 32j + 8c .. +8
-  return 16 * (8 * (j >> 1) + 4 * (j & 1) + c);          // fp32: floats 32(j/2) + 16(j&1) + 4c .. +4
-}
-
-struct RadixCut {
-  uint32_t T;
-  uint32_t rem;
-};
-
-// Weighted radix select on keys[0..P): the key T such that the total weight of
-// keys > T is <= cap < total weight of keys >= T, and rem = cap - weight(> T).
-// Requires total weight > cap.
-SA_DEV RadixCut radix_cut(const uint32_t* keys, const uint32_t* wts, int P, uint32_t cap,
-                          uint32_t* hist, uint32_t* bc) {
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nt = blockDim.x;
-  uint32_t prefix = 0, mask = 0, rem = cap;
-  for (int pass = 0; pass < 4; ++pass) {
-    const int shift = 24 - 8 * pass;
-    for (int i = tid; i < 256; i += nt) hist[i] = 0;
-    __syncthreads();
-    for (int i = tid; i < P; i += nt) {
-      const uint32_t k = keys[i];
-      if ((k & mask) == prefix) atomicAdd(&hist[(k >> shift) & 255u], wts ? wts[i] : 1u);
-    }
-    __syncthreads();
-    if (warp == 0) {
-      uint32_t h[8], ls = 0;
-#pragma unroll
-      for (int q = 0; q < 8; ++q) {
-        h[q] = hist[255 - 8 * lane - q];
-        ls += h[q];
-      }
-      uint32_t inc = ls;
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const uint32_t y = __shfl_up_sync(0xffffffffu, inc, o);
-        if (lane >= o) inc += y;
-      }
-      const unsigned ball = __ballot_sync(0xffffffffu, inc > rem);
-      const int L = __ffs(ball) - 1;
-      if (lane == L) {
-        uint32_t run = inc - ls;
-        int d = 255 - 8 * lane - 7;
-#pragma unroll
-        for (int q = 0; q < 8; ++q) {
-          if (run + h[q] > rem) {
-            d = 255 - 8 * lane - q;
-            break;
-          }
-          run += h[q];
-        }
-        bc[0] = (uint32_t)d;
-        bc[1] = run;
-      }
-    }
-    __syncthreads();
-    const uint32_t d = bc[0];
-    rem -= bc[1];
-    prefix |= d << shift;
-    mask |= 0xffu << shift;
-    __syncthreads();
-  }
-  return {prefix, rem};
-}
+constexpr int kSelStages = SA_SEL_STAGES;
+constexpr int kTileBytes = 8192;          // 16 pages x 512 B = four 2 KiB boxes
+constexpr int kBoxBytes = 2048;
+constexpr int kRingBytes = kSelWarps * kSelStages * kTileBytes;
+constexpr int kOffBars = kRingBytes;
 
 struct SelSmem {
-  unsigned char* smem;   // max(ring, 8 * max_pages) bytes
+  unsigned char* ring;   // [warp][stage][kTileBytes]; reused for keys/weights in selection
+  uint64_t* bars;        // [warp][stage]
   uint32_t* hist;        // 256
   uint32_t* scan;        // 32
   uint32_t* bc;          // 4
   int* last;
 };
 
+struct WarpState {
+  uint32_t gi;           // stages consumed so far by this warp
+  bool alive;            // false after a barrier wait timed out
+  uint32_t drain_lo, drain_hi;
+};
+
 template <int RULE>
-SA_DEV void select_item(const SelectArgs& a, const int u, const int split, const SelSmem& S) {
-  unsigned char* smem = S.smem;
+SA_DEV void select_item(const SelectArgs& a, const int u, const int split, const SelSmem& S,
+                        WarpState& ws) {
   uint32_t* s_hist = S.hist;
   uint32_t* s_scan = S.scan;
   uint32_t* s_bc = S.bc;
   int& s_last = *S.last;
+  unsigned char* smem = S.ring;
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int gq = lane >> 2, c = lane & 3;
@@ -163,91 +112,96 @@ SA_DEV void select_item(const SelectArgs& a, const int u, const int split, const
   uint32_t bq[RULE == 0 ? 32 : 1];
   double bd[RULE == 0 ? 1 : 32];
   if (RULE == 0) {
+    // k-step ks covers row elements 16ks .. 16ks + 15 of [kmin | kmax];
+    // the paired query vector is [q- | q+] (natural order)
 #pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      uint4 v = head_ok ? ldg_nc128(qrow + 32 * (j & 3) + 8 * c) : make_uint4(0, 0, 0, 0);
-      if (j < 4) {  // paired with kmin: q-
-        v.x = bf16x2_neg_part(v.x); v.y = bf16x2_neg_part(v.y);
-        v.z = bf16x2_neg_part(v.z); v.w = bf16x2_neg_part(v.w);
-      } else {      // paired with kmax: q+
-        v.x = bf16x2_pos_part(v.x); v.y = bf16x2_pos_part(v.y);
-        v.z = bf16x2_pos_part(v.z); v.w = bf16x2_pos_part(v.w);
-      }
-      bq[4 * j + 0] = v.x; bq[4 * j + 1] = v.y; bq[4 * j + 2] = v.z; bq[4 * j + 3] = v.w;
+    for (int ks = 0; ks < 16; ++ks) {
+      const int e = 16 * (ks & 7) + 2 * c;
+      uint32_t lo = head_ok ? __ldg(reinterpret_cast<const uint32_t*>(qrow + e)) : 0u;
+      uint32_t hi = head_ok ? __ldg(reinterpret_cast<const uint32_t*>(qrow + e + 8)) : 0u;
+      if (ks < 8) { lo = bf16x2_neg_part(lo); hi = bf16x2_neg_part(hi); }
+      else        { lo = bf16x2_pos_part(lo); hi = bf16x2_pos_part(hi); }
+      bq[2 * ks] = lo;
+      bq[2 * ks + 1] = hi;
     }
   } else {
-    // bd[8i + 4h + r] = q[head][32i + 16h + 4c + r] as fp64: the same dimensions
-    // as the metadata chunk (i, h) this lane loads (k-step (2i + h, r))
+    // k-step (box bx, chunk j): lane c holds dimension 32 bx + 4 j + c
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
+    for (int bx = 0; bx < 4; ++bx)
 #pragma unroll
-      for (int hh = 0; hh < 2; ++hh) {
-        uint2 v = make_uint2(0, 0);
-        if (head_ok) v = __ldg(reinterpret_cast<const uint2*>(qrow + 32 * i + 16 * hh + 4 * c));
-        bd[8 * i + 4 * hh + 0] = (double)bf16_lo(v.x);
-        bd[8 * i + 4 * hh + 1] = (double)bf16_hi(v.x);
-        bd[8 * i + 4 * hh + 2] = (double)bf16_lo(v.y);
-        bd[8 * i + 4 * hh + 3] = (double)bf16_hi(v.y);
+      for (int j = 0; j < 8; ++j) {
+        const int e = 32 * bx + 4 * j + c;
+        bd[8 * bx + j] = head_ok ? (double)__bfloat162float(qrow[e]) : 0.0;
       }
-    }
   }
 
   // ---- scoring: warp w takes tiles t_begin + w, + 4, ...
-  unsigned char* ring = smem + warp * (kSelStages * kStageBytes);
-  const unsigned char* meta_u =
-      reinterpret_cast<const unsigned char*>(a.meta) + (size_t)u * a.kv.max_pages * kMetaBytes;
   float* sc_u = a.ws_scores + (size_t)u * a.kv.max_pages;
   float* out_u = a.scores_out ? a.scores_out + (size_t)u * a.kv.max_pages : nullptr;
+  unsigned char* ring = S.ring + warp * (kSelStages * kTileBytes);
+  uint64_t* bars = S.bars + warp * kSelStages;
+  const int row_base = u * a.kv.max_pages;
+  const int lrow = (lane & 7) + 8 * ((lane >> 3) & 1);  // ldmatrix: rows 0-7 / 8-15
+  const int lchk = lane >> 4;                            //            chunk +0 / +1
+  const int nt = t_end - t_begin;
+  const int n_it = max(0, (nt - warp + kSelWarps - 1) / kSelWarps);
 
-  auto issue = [&](int it) {
-    const int t = t_begin + warp + it * kSelWarps;
-    if (t < t_end) {
-      unsigned char* st = ring + (it % kSelStages) * kStageBytes;
+  auto issue = [&](int it) {  // lane 0 only
+    const uint32_t g_it = ws.gi + (uint32_t)it;
+    uint64_t* bar = bars + g_it % kSelStages;
+    unsigned char* st = ring + (g_it % kSelStages) * kTileBytes;
+    const int y = row_base + 16 * (t_begin + warp + it * kSelWarps);
+    mbar_arrive_expect_tx(bar, kTileBytes);
+    const int xs = RULE == 0 ? 64 : 32;  // elements per 128-byte box row
 #pragma unroll
-      for (int r = 0; r < 2; ++r) {
-        const int page = t * 16 + gq + 8 * r;
-        const bool ok = page < P;
-        const unsigned char* src = meta_u + (size_t)(ok ? page : 0) * kMetaBytes;
-#pragma unroll
-        for (int j = 0; j < 8; ++j)
-          cp_async16(st + (r * 8 + j) * kSlotBytes + lane * 16, src + chunk_byte<RULE>(j, c), ok);
-      }
-    }
-    cp_async_commit();
+    for (int bx = 0; bx < 4; ++bx) tma_load_2d(st + bx * kBoxBytes, &a.tmap_meta, bx * xs, y, bar);
   };
 
-  const int n_it = (t_end - t_begin - warp + kSelWarps - 1) / kSelWarps;
-#pragma unroll
-  for (int it = 0; it < kSelStages - 1; ++it) issue(it);
-  for (int it = 0; it < n_it; ++it) {
-    cp_async_wait<kSelStages - 2>();
-    issue(it + kSelStages - 1);
-    const unsigned char* st = ring + (it % kSelStages) * kStageBytes + lane * 16;
-    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+  int issued = 0;
+  if (ws.alive) {
+    issued = min(n_it, kSelStages - 1);
+    if (lane == 0)
+      for (int it = 0; it < issued; ++it) issue(it);
+  }
+  for (int it = 0; it < n_it && ws.alive; ++it) {
+    __syncwarp();
+    if (it + kSelStages - 1 < n_it) {
+      if (lane == 0) issue(it + kSelStages - 1);
+      issued = it + kSelStages;
+    }
+    const uint32_t g_it = ws.gi + (uint32_t)it;
+    if (!mbar_wait(bars + g_it % kSelStages, (g_it / kSelStages) & 1u, a.status)) {
+      ws.alive = false;
+      ws.drain_lo = g_it;
+      ws.drain_hi = ws.gi + (uint32_t)issued;
+      break;
+    }
+    const unsigned char* st = ring + (g_it % kSelStages) * kTileBytes;
+    float acc[4];
     if (RULE == 0) {
+      float s0[4] = {0.f, 0.f, 0.f, 0.f}, s1[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        const uint4 lo = lds128(st + j * kSlotBytes);
-        const uint4 hi = lds128(st + (8 + j) * kSlotBytes);
-        mma_bf16(acc, lo.x, hi.x, lo.y, hi.y, bq[4 * j + 0], bq[4 * j + 1]);
-        mma_bf16(acc, lo.z, hi.z, lo.w, hi.w, bq[4 * j + 2], bq[4 * j + 3]);
+      for (int ks = 0; ks < 16; ++ks) {
+        uint32_t a0, a1, a2, a3;
+        ldsm_x4(a0, a1, a2, a3, st + (ks >> 2) * kBoxBytes + swz128(lrow, 2 * (ks & 3) + lchk));
+        if (ks & 1) mma_bf16(s1, a0, a1, a2, a3, bq[2 * ks], bq[2 * ks + 1]);
+        else        mma_bf16(s0, a0, a1, a2, a3, bq[2 * ks], bq[2 * ks + 1]);
       }
+#pragma unroll
+      for (int x = 0; x < 4; ++x) acc[x] = s0[x] + s1[x];
     } else {
-      // Centroid on the FP64 tensor cores: fp32 kmean and bf16 q are exact in
-      // fp64, so the only rounding left is the final fp64 -> fp32 of the score.
+      // FP64 tensor cores: exact products and sums, one final rounding
       double c00 = 0.0, c01 = 0.0, c10 = 0.0, c11 = 0.0;  // pages gq / gq + 8
 #pragma unroll
-      for (int j = 0; j < 8; ++j) {  // chunk j = floats 32(j/2) + 16(j&1) + 4c .. +4
-        const uint4 r0 = lds128(st + j * kSlotBytes);
-        const uint4 r1 = lds128(st + (8 + j) * kSlotBytes);
-        const uint32_t a0[4] = {r0.x, r0.y, r0.z, r0.w}, a1[4] = {r1.x, r1.y, r1.z, r1.w};
+      for (int bx = 0; bx < 4; ++bx)
 #pragma unroll
-        for (int r = 0; r < 4; ++r) {
-          const double b = bd[8 * (j >> 1) + 4 * (j & 1) + r];
-          mma_f64(c00, c01, (double)__uint_as_float(a0[r]), b);
-          mma_f64(c10, c11, (double)__uint_as_float(a1[r]), b);
+        for (int j = 0; j < 8; ++j) {
+          const float x0 = *reinterpret_cast<const float*>(st + bx * kBoxBytes + swz128(gq, j) + 4 * c);
+          const float x1 = *reinterpret_cast<const float*>(st + bx * kBoxBytes + swz128(gq + 8, j) + 4 * c);
+          const double bv = bd[8 * bx + j];
+          mma_f64(c00, c01, (double)x0, bv);
+          mma_f64(c10, c11, (double)x1, bv);
         }
-      }
       acc[0] = (float)c00; acc[1] = (float)c01; acc[2] = (float)c10; acc[3] = (float)c11;
     }
     const float ninf = -__int_as_float(0x7f800000);
@@ -268,7 +222,7 @@ SA_DEV void select_item(const SelectArgs& a, const int u, const int split, const
       }
     }
   }
-  cp_async_wait<0>();
+  ws.gi += (uint32_t)n_it;
 
   // ---- the last CTA of the unit selects
   __syncthreads();
@@ -371,21 +325,40 @@ SA_DEV void select_item(const SelectArgs& a, const int u, const int split, const
 }
 
 template <int RULE>
-__global__ void __launch_bounds__(kSelThreads) select_kernel(SelectArgs a) {
-  extern __shared__ __align__(128) unsigned char smem[];
+__global__ void __launch_bounds__(kSelThreads) select_kernel(const __grid_constant__ SelectArgs a) {
+  extern __shared__ unsigned char smem_raw[];
   __shared__ uint32_t s_hist[256];
   __shared__ uint32_t s_scan[32];
   __shared__ uint32_t s_bc[4];
   __shared__ int s_last, s_item;
-  const SelSmem S{smem, s_hist, s_scan, s_bc, &s_last};
+  unsigned char* base = reinterpret_cast<unsigned char*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  // barriers sit after the ring, or after the keys/weights area when that is larger
+  const int keys_bytes = 8 * a.kv.max_pages;
+  const int bar_off = keys_bytes > kRingBytes ? ((keys_bytes + 1023) & ~1023) : kOffBars;
+  const SelSmem S{base, reinterpret_cast<uint64_t*>(base + bar_off), s_hist, s_scan, s_bc, &s_last};
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  if (lane == 0) {
+    for (int s = 0; s < kSelStages; ++s) mbar_init(S.bars + warp * kSelStages + s, 1);
+    fence_barrier_init();
+  }
+  if (threadIdx.x == 0) prefetch_tmap(&a.tmap_meta);
+  __syncthreads();
+  WarpState ws{0u, true, 0u, 0u};
   const int n_items = a.kv.B * a.kv.Hkv * a.splits;
   for (;;) {
     if (threadIdx.x == 0) s_item = (int)atomicAdd(&a.ws_queue[0], 1u);
     __syncthreads();
     const int item = s_item;
     if (item >= n_items) break;
-    select_item<RULE>(a, item / a.splits, item % a.splits, S);
+    select_item<RULE>(a, item / a.splits, item % a.splits, S, ws);
+    fence_proxy_async();  // generic writes to the ring (keys) before the next TMA writes
     __syncthreads();
+  }
+  if (!ws.alive && lane == 0) {  // a wait timed out: let the copies in flight land (bounded)
+    uint64_t* bars = S.bars + warp * kSelStages;
+    for (uint32_t gg = ws.drain_lo; gg < ws.drain_hi; ++gg)
+      mbar_wait(bars + gg % kSelStages, (gg / kSelStages) & 1u, nullptr);
   }
   // the last CTA out rewinds the queue for the next launch
   if (threadIdx.x == 0) {
@@ -413,16 +386,16 @@ int select_splits(int units, int max_pages, int sm_count) {
 }
 
 size_t select_smem_bytes(int max_pages) {
-  const size_t keys = (size_t)max_pages * 8;
-  return keys > (size_t)kRingBytes ? keys : (size_t)kRingBytes;
+  const size_t keys = ((size_t)max_pages * 8 + 1023) & ~(size_t)1023;
+  const size_t body = keys > (size_t)kRingBytes ? keys : (size_t)kRingBytes;
+  return 1024 + body + kSelWarps * kSelStages * 8;
 }
 
 cudaError_t launch_select(const SelectArgs& a, cudaStream_t st) {
   const size_t smem = select_smem_bytes(a.kv.max_pages);
   const long long items = (long long)a.kv.B * a.kv.Hkv * a.splits;
   if (items > 0x7fffffffLL) return cudaErrorInvalidValue;
-  const int ctas_per_sm = smem <= (size_t)kRingBytes ? SA_SEL_CTAS_PER_SM : 1;
-  long long grid = (long long)device_sm_count() * ctas_per_sm;
+  long long grid = (long long)device_sm_count() * SA_SEL_CTAS_PER_SM;
   if (grid > items) grid = items;
   cudaError_t e;
   if (a.rule == 0) {
