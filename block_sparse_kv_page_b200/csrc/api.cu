@@ -26,6 +26,9 @@ namespace sa {
 constexpr int kMaxUnits = 65536;
 constexpr size_t kQueueSelect = 64;
 constexpr size_t kQueueDecode = 72;
+constexpr size_t kQueueRoute = 80;
+constexpr int kMaxRouteTiles = 1024;
+constexpr int kMaxRouteList = 1023;
 constexpr size_t kScratch = 256 + 4 * (size_t)kMaxUnits;
 constexpr int kMaxSelectPages = 16384;
 constexpr int kMaxChunkSel = 8192;
@@ -203,7 +206,8 @@ size_t sparse_attn_workspace_size(const sa_kv_desc* kv, int32_t n_q_heads, int32
   const int splits = decode_splits((int)units, max_tiles_per_unit(kv, max_sel), sm);
   const size_t dec = decode_scratch((int)units, splits);
   if (dec > tail) tail = dec;
-  const size_t rt = route_ws_bytes(rows, kv->n_kv_heads, kv->max_pages);
+  const int route_tiles = rows < kMaxRouteTiles ? rows : kMaxRouteTiles;  // tiles <= query rows
+  const size_t rt = route_ws_bytes(route_tiles, kv->n_kv_heads, kv->max_pages, max_sel);
   if (rt > tail) tail = rt;
   return kScratch + tail;
 }
@@ -365,8 +369,64 @@ sa_status sparse_attn_route(const sa_kv_desc* kv, const void* meta, sa_score_rul
   if (kv->batch != 1 || kv->page_size == 0) return SA_ERR_INVALID;
   if (n_q_rows < 1 || tile_rows < 1 || k < 1 || rho < 1 || q_pos0 < 0) return SA_ERR_INVALID;
   if (!(quantile >= 0.f && quantile <= 1.f)) return SA_ERR_INVALID;
-  (void)tau; (void)tau_out; (void)ws; (void)ws_bytes; (void)stream;
-  return SA_ERR_UNSUPPORTED;
+  if (!aligned(kv_idx, 4) || !aligned(kv_count, 4) || !aligned(sigma, 4) || !aligned(sigma_bar, 4) ||
+      (tau && !aligned(tau, 4)) || (tau_out && !aligned(tau_out, 4)))
+    return SA_ERR_INVALID;
+  const long long T = ((long long)n_q_rows + tile_rows - 1) / tile_rows;
+  const long long W = (long long)rho * k;
+  if (T > kMaxRouteTiles || W > kMaxRouteList || (long long)k + 1 > kMaxRouteList + 1)
+    return SA_ERR_UNSUPPORTED;
+  if (kv->max_pages > kMaxSelectPages) return SA_ERR_UNSUPPORTED;
+  const long long units = T * kv->n_kv_heads;
+  if (units > kMaxUnits) return SA_ERR_UNSUPPORTED;
+  const unsigned long long meta_rows = (unsigned long long)kv->n_kv_heads * kv->max_pages;
+  if (meta_rows > 0x7fffffffULL) return SA_ERR_UNSUPPORTED;
+  const size_t need = kScratch + route_ws_bytes((int)T, kv->n_kv_heads, kv->max_pages, (int)W);
+  if ((s = check_ws(ws, ws_bytes, need)) != SA_OK) return s;
+
+  RouteArgs a;
+  const bool env = rule == SA_SCORE_ENVELOPE;
+  if (!encode_tmap_2d(&a.tmap_meta, meta, meta_rows, kMetaBytes,
+                      env ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32,
+                      env ? 2 : 4, 16))
+    return SA_ERR_CUDA;
+  a.kv = view(kv);
+  a.rule = (int)rule;
+  a.q = q;
+  a.Hq = n_q_heads;
+  a.G = G;
+  a.n_rows = n_q_rows;
+  a.q_pos0 = q_pos0;
+  a.tile_rows = tile_rows;
+  a.n_tiles = (int)T;
+  a.k = k;
+  a.rho = rho;
+  a.W = (int)W;
+  a.nsplit = route_splits(tile_rows * G);
+  a.quantile = quantile;
+  a.tau_in = tau;
+  a.kv_idx = kv_idx;
+  a.kv_count = kv_count;
+  a.sigma = sigma;
+  a.sigma_bar = sigma_bar;
+  a.triggered = triggered;
+  a.tau_out = tau_out;
+  char* scratch = reinterpret_cast<char*>(ws) + kScratch;
+  const size_t tg = (size_t)units;
+  const size_t keys_bytes = align256(tg * kv->max_pages * 4);
+  a.ws_keys = reinterpret_cast<uint32_t*>(scratch);
+  a.ws_list = reinterpret_cast<int32_t*>(scratch + keys_bytes);
+  a.ws_sigma = reinterpret_cast<double*>(scratch + keys_bytes + align256(tg * W * 4));
+  a.ws_elig = reinterpret_cast<int32_t*>(scratch + keys_bytes + align256(tg * W * 4) + align256(tg * 8));
+  a.ws_count = reinterpret_cast<uint32_t*>(reinterpret_cast<char*>(ws) + 256);
+  a.ws_final = reinterpret_cast<uint32_t*>(reinterpret_cast<char*>(ws) + kQueueRoute);
+  a.status = reinterpret_cast<int*>(ws);
+  // tile-score keys start at 0 (below every score) for the atomicMax merge
+  if (cudaMemsetAsync(a.ws_keys, 0, tg * kv->max_pages * 4, (cudaStream_t)stream) != cudaSuccess) {
+    cudaGetLastError();
+    return SA_ERR_CUDA;
+  }
+  return launched(launch_route(a, (cudaStream_t)stream));
 }
 
 sa_status sparse_attn_get_device_status(void* ws, sa_status* host_out, void* stream) {

@@ -94,13 +94,14 @@ struct DecodeArgs {
 cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t st);
 
 struct RouteArgs {
+  CUtensorMap tmap_meta;      // block metadata rows [Hkv*max_pages][512 B], boxes 16 x 128 B, 128B swizzle
   KvView kv;
-  const void* meta;
   int rule;
-  const void* q;
+  const void* q;              // bf16 [n_rows][Hq][128]
   int Hq, G;
   int n_rows, q_pos0, tile_rows, n_tiles;
-  int k, rho;
+  int k, rho, W;              // W = rho * k: list width
+  int nsplit;                 // query-vector splits per (tile, KV head)
   float quantile;
   const float* tau_in;
   int32_t* kv_idx;
@@ -109,10 +110,17 @@ struct RouteArgs {
   float* sigma_bar;
   uint8_t* triggered;
   float* tau_out;
-  void* ws_route;
+  uint32_t* ws_keys;          // [n_tiles][Hkv][max_pages] tile-score keys (zeroed before launch)
+  int32_t* ws_list;           // [n_tiles][Hkv][W] rank-ordered lists
+  double* ws_sigma;           // [n_tiles][Hkv]
+  int32_t* ws_elig;           // [n_tiles][Hkv] eligible block counts
+  uint32_t* ws_count;         // [n_tiles * Hkv] split counters (left zero)
+  uint32_t* ws_final;         // [1] finalize counter (left zero)
   int* status;
 };
 cudaError_t launch_route(const RouteArgs& a, cudaStream_t st);
-size_t route_ws_bytes(int n_tiles, int Hkv, int max_pages);
+// Router scratch: keys, lists, sigma and eligible counts for n_tiles x Hkv.
+size_t route_ws_bytes(int n_tiles, int Hkv, int max_pages, int W);
+int route_splits(int vectors_per_tile);
 
 }  // namespace sa

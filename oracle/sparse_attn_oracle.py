@@ -114,6 +114,17 @@ def envelope_scores(Q, kmin, kmax) -> np.ndarray:
     return s
 
 
+def envelope_scores_matmul(Q, kmin, kmax) -> np.ndarray:
+    """The same envelope score written with the positive and negative parts of
+    q: max(q_d kmin_d, q_d kmax_d) = q+_d kmax_d + q-_d kmin_d because
+    kmax_d >= kmin_d; summed over d this is two matrix products.  Used for
+    large router workloads; pinned against envelope_scores."""
+    Q = f64(Q)
+    qp = np.maximum(Q, 0.0)
+    qn = np.minimum(Q, 0.0)
+    return qp @ f64(kmax).T + qn @ f64(kmin).T
+
+
 def centroid_scores(Q, kmean) -> np.ndarray:
     """Q: [H, D]; kmean: [P, D].  Returns s[H, P] = q_h . kmean_p."""
     Q = f64(Q)
@@ -125,12 +136,12 @@ def centroid_scores(Q, kmean) -> np.ndarray:
     return s
 
 
-def head_scores(Q, meta, rule: str) -> np.ndarray:
+def head_scores(Q, meta, rule: str, fast: bool = False) -> np.ndarray:
     kmin, kmax, kmean = meta
     if rule == "envelope":
-        return envelope_scores(Q, kmin, kmax)
+        return envelope_scores_matmul(Q, kmin, kmax) if fast else envelope_scores(Q, kmin, kmax)
     if rule == "centroid":
-        return centroid_scores(Q, kmean)
+        return f64(Q) @ f64(kmean).T if fast else centroid_scores(Q, kmean)
     raise ValueError(rule)
 
 
@@ -297,13 +308,16 @@ def decode_unit(Qg, K, V, n_tokens: int, *, rule: str, page_size: int = 16,
 # 6. Uncertainty router over query tiles ([ROUTER] "Methodologie").
 # --------------------------------------------------------------------------
 
-def tile_block_scores(Qtile, meta, rule: str, rows_per_batch: int = 8) -> np.ndarray:
+def tile_block_scores(Qtile, meta, rule: str, rows_per_batch: int = 8, fast: bool = False) -> np.ndarray:
     """Step 2: the tile score of a block is the maximum, over the tile's rows
     (and, under GQA, the query heads that share the KV head), of the per-row
-    block score.  Qtile: [R, G, D] -> scores [P]."""
+    block score.  Qtile: [R, G, D] -> scores [P].  fast=True evaluates the
+    per-row scores as matrix products (envelope_scores_matmul)."""
     Qtile = f64(Qtile)
     R, G, D = Qtile.shape
     flat = Qtile.reshape(R * G, D)
+    if fast:
+        return head_scores(flat, meta, rule, fast=True).max(axis=0)
     best = None
     for i in range(0, flat.shape[0], rows_per_batch):
         s = head_scores(flat[i:i + rows_per_batch], meta, rule)  # [r, P]
@@ -352,7 +366,7 @@ class RouteResult:
 
 def route(Q, metas, rule: str, *, q_pos0: int, tile_rows: int, block_size: int,
           n_blocks: int, k: int, rho: int, quantile: float, tau=None,
-          score_fn=None) -> RouteResult:
+          score_fn=None, fast: bool = False) -> RouteResult:
     """Steps 2-5 over all tiles of one layer.
 
     Q: [rows, Hq, D] query rows at positions q_pos0 .. q_pos0+rows-1.
@@ -381,7 +395,7 @@ def route(Q, metas, rule: str, *, q_pos0: int, tile_rows: int, block_size: int,
             if score_fn is not None:
                 S = score_fn(t, g)
             else:
-                S = tile_block_scores(Qt, metas[g], rule)
+                S = tile_block_scores(Qt, metas[g], rule, fast=fast)
             S = S[:E]
             scores[t, g, :E] = S
             order = rank_order(S)

@@ -440,3 +440,25 @@ def check_tile_attention_sdpa(tile_attention) -> bool:
             if not (np.allclose(out[r, h], o2[0], atol=1e-12, rtol=0) and abs(lse[r, h] - l2[0]) < 1e-12):
                 return False
     return True
+
+
+def check_fast_scores(envelope_fast, tile_block_scores, envelope_scores, centroid_scores,
+                      page_metadata, fixed_pages) -> bool:
+    """The matrix-product envelope (q+ . kmax + q- . kmin) and the fast tile
+    scores agree with the literal per-dimension definitions."""
+    rng = _rng(15)
+    K = _bf16_round(rng.standard_normal((300, 16)) * 2)
+    Q = _bf16_round(rng.standard_normal((9, 16)))
+    s, e = fixed_pages(300, 16)
+    meta = page_metadata(K, s, e)
+    a = envelope_fast(Q, meta[0], meta[1])
+    b = envelope_scores(Q, meta[0], meta[1])
+    if not np.allclose(a, b, rtol=1e-12, atol=1e-12):
+        return False
+    Qt = Q.reshape(3, 3, 16)
+    for rule in ("envelope", "centroid"):
+        f = tile_block_scores(Qt, meta, rule, fast=True)
+        sl = tile_block_scores(Qt, meta, rule, fast=False)
+        if not np.allclose(f, sl, rtol=1e-12, atol=1e-12):
+            return False
+    return True

@@ -92,6 +92,11 @@ def test_tile_attention_sdpa():
     assert P.check_tile_attention_sdpa(O.tile_attention)
 
 
+def test_fast_scores():
+    assert P.check_fast_scores(O.envelope_scores_matmul, O.tile_block_scores, O.envelope_scores,
+                               O.centroid_scores, O.page_metadata, O.fixed_pages)
+
+
 def test_budget_scale_fact():
     """'The comparison': a 4096-token budget at ~29.5k context reads about a
     seventh of it, and the budget is page_size x top_k tokens."""
@@ -223,6 +228,11 @@ def _tile_attn_noncausal(Q, K, V, kv_idx, *, q_pos0, tile_rows, block_size, n_to
                             block_size=block_size, n_tokens=n_tokens, scale=scale)
 
 
+def _env_fast_swapped(Q, kmin, kmax):   # q+ paired with kmin in the matrix form
+    Q = O.f64(Q)
+    return np.maximum(Q, 0) @ O.f64(kmin).T + np.minimum(Q, 0) @ O.f64(kmax).T
+
+
 MISTAKES = [
     ("envelope min instead of max", lambda: P.check_envelope_upper_bound(_env_min, O.page_metadata, O.fixed_pages)
      and P.check_envelope_golden(_env_min, O.centroid_scores, O.page_metadata)),
@@ -251,6 +261,9 @@ MISTAKES = [
     ("tile score mean instead of max", lambda: P.check_tile_max_bruteforce(
         _tile_mean, O.envelope_scores, O.centroid_scores, O.page_metadata, O.fixed_pages)),
     ("trigger on <= instead of <", lambda: P.check_router_invariants(_route_le, O.page_metadata, O.fixed_pages)),
+    ("matrix-form envelope q+/q- swapped", lambda: P.check_fast_scores(
+        _env_fast_swapped, O.tile_block_scores, O.envelope_scores, O.centroid_scores,
+        O.page_metadata, O.fixed_pages)),
     ("tile attention not causal", lambda: P.check_tile_attention_sdpa(_tile_attn_noncausal)),
 ]
 
