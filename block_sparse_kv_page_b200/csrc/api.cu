@@ -187,6 +187,48 @@ int device_sm_count() {
   return n;
 }
 
+namespace {
+// Multi-row tiles (router output): causal attention of each tile over its
+// listed 64-token blocks.  Needs only the status word of the workspace.
+sa_status tile_attention(const sa_kv_desc* kv, const void* q, int n_q_heads, int G, int n_q_rows,
+                         int q_pos0, int tile_rows, float scale, const int32_t* idx,
+                         const int32_t* count, int max_sel, float* out, float* lse, int* status,
+                         void* ws, size_t ws_bytes, void* stream) {
+  if (kv->page_size != 64) return SA_ERR_UNSUPPORTED;
+  if (q_pos0 < 0 || max_sel > kMaxRouteList + 1) return SA_ERR_UNSUPPORTED;
+  const long long T = ((long long)n_q_rows + tile_rows - 1) / tile_rows;
+  if (T * kv->n_kv_heads > kMaxUnits) return SA_ERR_UNSUPPORTED;
+  if (ws) {
+    if (!aligned(ws, 256) || ws_bytes < 256) return SA_ERR_WORKSPACE;
+  } else if (status) {
+    return SA_ERR_WORKSPACE;
+  }
+  const unsigned long long kv_rows = (unsigned long long)kv->n_kv_heads * kv->cap_tokens;
+  if (kv_rows > 0x7fffffffULL) return SA_ERR_UNSUPPORTED;
+  TileAttnArgs a;
+  if (!encode_tmap_2d(&a.tmap_k, kv->k, kv_rows, kHeadDim * 2, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, 64) ||
+      !encode_tmap_2d(&a.tmap_v, kv->v, kv_rows, kHeadDim * 2, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, 64))
+    return SA_ERR_CUDA;
+  a.kv = view(kv);
+  a.q = q;
+  a.Hq = n_q_heads;
+  a.G = G;
+  a.n_rows = n_q_rows;
+  a.q_pos0 = q_pos0;
+  a.tile_rows = tile_rows;
+  a.n_tiles = (int)T;
+  a.n_mchunks = tile_attn_mchunks(tile_rows * G);
+  a.scale_log2 = scale * kLog2e;
+  a.idx = idx;
+  a.count = count;
+  a.max_sel = max_sel;
+  a.out = out;
+  a.lse = lse;
+  a.status = status;
+  return launched(launch_tile_attn(a, (cudaStream_t)stream));
+}
+}  // namespace
+
 }  // namespace sa
 
 using namespace sa;
@@ -317,7 +359,8 @@ sa_status sparse_attn_decode(const sa_kv_desc* kv, const void* q, int32_t n_q_he
     if (n_q_rows != kv->batch) return SA_ERR_INVALID;
   } else {
     if (kv->batch != 1 || kv->page_size == 0) return SA_ERR_INVALID;
-    return SA_ERR_UNSUPPORTED;  // multi-row tiles: route-tile attention kernel
+    return tile_attention(kv, q, n_q_heads, G, n_q_rows, q_pos0, tile_rows, scale, idx, count,
+                          max_sel, out, lse, reinterpret_cast<int*>(ws), ws, ws_bytes, stream);
   }
   if (kv->page_size == 0 && max_sel > kMaxChunkSel) return SA_ERR_UNSUPPORTED;
   const long long units = (long long)n_q_rows * kv->n_kv_heads;

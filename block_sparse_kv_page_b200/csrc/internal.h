@@ -93,6 +93,24 @@ struct DecodeArgs {
 };
 cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t st);
 
+struct TileAttnArgs {
+  CUtensorMap tmap_k;         // K rows [Hkv*cap][128 bf16], boxes 64 x 64, 128B swizzle
+  CUtensorMap tmap_v;
+  KvView kv;                  // batch 1, 64-token blocks
+  const void* q;              // bf16 [n_rows][Hq][128]
+  int Hq, G;
+  int n_rows, q_pos0, tile_rows, n_tiles, n_mchunks;
+  float scale_log2;
+  const int32_t* idx;         // [n_tiles][Hkv][max_sel], -1 = sentinel
+  const int32_t* count;       // [n_tiles][Hkv]
+  int max_sel;
+  float* out;
+  float* lse;
+  int* status;
+};
+cudaError_t launch_tile_attn(const TileAttnArgs& a, cudaStream_t st);
+int tile_attn_mchunks(int vectors_per_tile);
+
 struct RouteArgs {
   CUtensorMap tmap_meta;      // block metadata rows [Hkv*max_pages][512 B], boxes 16 x 128 B, 128B swizzle
   KvView kv;

@@ -159,6 +159,8 @@ sa_status sparse_attn_select(const sa_kv_desc* kv, const void* meta, sa_score_ru
  *    [n_q_rows][n_q_heads][128] at positions q_pos0 + r; idx [T][Hkv][max_sel]
  *    with T = ceil(n_q_rows / tile_rows), -1 entries skipped; row r attends
  *    causally (token position <= q_pos0 + r) to the blocks of its tile.
+ *    Blocks must be 64 tokens (page_size = 64); this path uses only the
+ *    status word of ws (ws may be null: device checks are then not reported).
  * z = scale * q.k, softmax with fp32 accumulation.  out: fp32 [rows][Hq][128];
  * lse (nullable): fp32 [rows][Hq], natural-log sum of exp(z).  A row with no
  * visible token gets out = 0 and lse = -inf.  idx entries outside [0, P_b)
