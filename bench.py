@@ -128,49 +128,69 @@ def cpu_oracle_time(rule: str, k: int, units: int, rounds: int = 1):
 
 
 # --------------------------------------------------------------------------- clocks
+def _clock_poller(index: int, go, stop, out_q):
+    """Child process: once `go` is set, poll NVML (SM clock, clock-event
+    reasons) every ~2 ms until `stop` is set, then send the samples back.
+    Reads only."""
+    samples = []
+    try:
+        import pynvml as nv
+        nv.nvmlInit()
+        h = nv.nvmlDeviceGetHandleByIndex(index)
+        mx = nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM)
+        out_q.put(("ready", mx))
+        while not go.is_set() and not stop.is_set():
+            time.sleep(0.001)
+        while not stop.is_set():
+            samples.append((nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM),
+                            nv.nvmlDeviceGetCurrentClocksEventReasons(h)))
+            time.sleep(0.002)
+    except Exception as e:  # no NVML: report nothing sampled
+        out_q.put(("ready", None))
+        out_q.put(("error", repr(e)))
+    out_q.put(("samples", samples))
+
+
 class ClockSampler:
-    """Polls NVML (SM clock, throttle reasons) in a thread during the timed region."""
+    """Samples the SM clock and clock-event reasons in a separate process
+    during the timed region (a thread would be starved by the launch loop)."""
 
     def __init__(self, index: int):
+        import multiprocessing as mp
+        self.index = index
         self.samples = []
-        self.ok = False
+        self.max_mhz = None
+        self.ctx = mp.get_context("spawn")
+        self.go = self.ctx.Event()
+        self.stop = self.ctx.Event()
+        self.q = self.ctx.Queue()
+        self.p = self.ctx.Process(target=_clock_poller, args=(index, self.go, self.stop, self.q), daemon=True)
+        self.p.start()
         try:
-            import pynvml
-            pynvml.nvmlInit()
-            self.nv = pynvml
-            self.h = pynvml.nvmlDeviceGetHandleByIndex(index)
-            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
-            self.ok = True
+            tag, mx = self.q.get(timeout=60)
+            self.max_mhz = mx
         except Exception:
-            self.max_mhz = None
-        self._stop = threading.Event()
-
-    def _run(self):
-        nv = self.nv
-        while not self._stop.is_set():
-            try:
-                mhz = nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM)
-                rs = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
-                self.samples.append((mhz, rs))
-            except Exception:
-                pass
-            time.sleep(0.002)
+            pass
 
     def __enter__(self):
-        if self.ok:
-            self.t = threading.Thread(target=self._run, daemon=True)
-            self.t.start()
+        self.go.set()
         return self
 
     def __exit__(self, *a):
-        if self.ok:
-            self._stop.set()
-            self.t.join()
+        self.stop.set()
+        try:
+            while True:
+                tag, val = self.q.get(timeout=30)
+                if tag == "samples":
+                    self.samples = val
+                    break
+        except Exception:
+            pass
+        self.p.join(timeout=10)
 
     def summary(self):
-        if not self.ok or not self.samples:
+        if not self.samples:
             return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": ["unsampled"]}
-        nv = self.nv
         names = {
             "gpu_idle": 0x1, "applications_clocks_setting": 0x2, "sw_power_cap": 0x4,
             "hw_slowdown": 0x8, "sync_boost": 0x10, "sw_thermal_slowdown": 0x20,
@@ -186,6 +206,29 @@ class ClockSampler:
                 "reasons": sorted(seen), "samples": len(self.samples)}
 
 
+# --------------------------------------------------------------------------- multi-rank plumbing
+def max_over_ranks(value: float, dist, device) -> float:
+    """A per-rank time reduced to the maximum over ranks (every rank calls this
+    at the same point; no-op on one process)."""
+    if dist is None:
+        return float(value)
+    import torch
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def replica_layer_offset(rank: int) -> int:
+    """Each rank runs its own independent replica of the workload (weak
+    scaling): layer seeds are offset by rank so replicas hold different data."""
+    return rank * 1000
+
+
+def whole_job_value(units_per_rank: float, world: int, ms: float) -> float:
+    """Throughput of the whole job: work of all ranks / max-over-ranks time."""
+    return units_per_rank * world / (ms * 1e-3)
+
+
 # --------------------------------------------------------------------------- GPU arm
 def build_inputs(torch, dev, rank: int, rule: str):
     import block_sparse_kv_page_b200 as sa
@@ -195,7 +238,7 @@ def build_inputs(torch, dev, rank: int, rule: str):
     v_all = torch.empty_like(k_all)
     q_all = torch.empty((L * B, HQ, D), dtype=torch.bfloat16, device=dev)
     for l in range(L):
-        lay = DG.workload2_layer(l + rank * 1000, dev)
+        lay = DG.workload2_layer(l + replica_layer_offset(rank), dev)
         k_all[l * B:(l + 1) * B] = lay.k
         v_all[l * B:(l + 1) * B] = lay.v
         q_all[l * B:(l + 1) * B] = lay.q
@@ -303,11 +346,7 @@ def run_gpu_arm(args, rank, world, dist):
                     fn()
             t1.record(stream)
             torch.cuda.synchronize()
-        ms = t0.elapsed_time(t1)
-        if dist is not None:
-            tt = torch.tensor([ms], device=dev)
-            dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-            ms = float(tt.item())
+        ms = max_over_ranks(t0.elapsed_time(t1), dist, dev)
         kern = None
         if evs:
             kern = {name: sum(e[i].elapsed_time(e[i + 1]) for e in evs) / steps
@@ -324,7 +363,7 @@ def run_gpu_arm(args, rank, world, dist):
     if args.mode == "batched" and kern is None:
         _, kern = timed("batched", args.rule, max(3, min(args.steps, 50)), 2, per_kernel=True)
     tok_heads = args.budget * HQ * L * B
-    value = tok_heads * world / (ms * 1e-3)
+    value = whole_job_value(tok_heads, world, ms)
     meta_bytes = L * B * HKV * (N // PS) * 512
     kv_bytes = L * B * HKV * args.budget * 2 * D * 2
 
@@ -354,11 +393,7 @@ def run_gpu_arm(args, rank, world, dist):
         e2e_step()
     a1.record(stream)
     torch.cuda.synchronize()
-    e2e_ms = a0.elapsed_time(a1) / args.steps
-    if dist is not None:
-        tt = torch.tensor([e2e_ms], device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        e2e_ms = float(tt.item())
+    e2e_ms = max_over_ranks(a0.elapsed_time(a1) / args.steps, dist, dev)
     h2d = q_h.numel() * 2 + knew_h.numel() * 2 + vnew_h.numel() * 2
     d2h = out_h.numel() * 4
 
@@ -376,9 +411,85 @@ def run_gpu_arm(args, rank, world, dist):
     for g in graphs.values():
         del g
     graphs.clear()
+    router = None
+    if not args.no_extra:
+        router = router_leg(torch, dev, max(5, min(args.steps, 50)), max(3, args.warmup))
     return dict(ms=ms, value=value, kern=kern, clocks=clocks.summary(), e2e_ms=e2e_ms, h2d=h2d,
-                d2h=d2h, meta_bytes=meta_bytes, kv_bytes=kv_bytes, extra=extra,
+                d2h=d2h, meta_bytes=meta_bytes, kv_bytes=kv_bytes, extra=extra, router=router,
                 launches_per_step=3 if args.mode == "batched" else 3 * L)
+
+
+def router_leg(torch, dev, steps: int, warmup: int):
+    """The 128K-context router workload (28 query / 4 KV heads, 64-token blocks,
+    2048 chunked-prefill rows in 32 tiles of 64, k = 32, rho = 2, quantile
+    0.25): route + tile attention per backbone, timed with CUDA events.
+    Near-duplicate block pairs are planted in 30% of the (tile, KV head)
+    cells at random positions (their place at the cut needs the oracle; the
+    timing does not depend on it)."""
+    import numpy as np
+
+    import block_sparse_kv_page_b200 as sa
+    import datagen as DG
+    lay = DG.make_router_layer(device=dev)
+    rng = np.random.default_rng(5999)
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(5999)
+    nblk = lay.N // 64
+    for _ in range(int(0.3 * 32 * 4)):
+        g = int(rng.integers(4))
+        a_, b_ = (int(x) for x in rng.choice(nblk, 2, replace=False))
+        DG.duplicate_block(lay.k, g, a_, b_, 64, 1e-3, gen)
+    T, Hkv, Hq, W, k = 32, 4, 28, 64, 32
+    sl = torch.tensor([lay.N], dtype=torch.int32, device=dev)
+    kv = sa.KvCache(lay.k, lay.v, sl, page_size=64, max_pages=nblk)
+    ws = sa.make_workspace(kv, Hq, 2048, W)
+    kv_idx = torch.zeros((T, Hkv, W), dtype=torch.int32, device=dev)
+    kv_count = torch.zeros((T, Hkv), dtype=torch.int32, device=dev)
+    sigma = torch.zeros((T, Hkv), dtype=torch.float32, device=dev)
+    sbar = torch.zeros((T,), dtype=torch.float32, device=dev)
+    trig = torch.zeros((T,), dtype=torch.uint8, device=dev)
+    out = torch.zeros((2048, Hq, 128), dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream()
+    res = {}
+    for rule in ("envelope", "centroid"):
+        meta = kv.meta_buffer()
+        sa.sparse_attn_build_meta(kv, rule, 0, meta)
+
+        def route():
+            sa.sparse_attn_route(kv, meta, rule, lay.q, 2048, lay.q_pos0, 64, k, 2, 0.25, None,
+                                 kv_idx, kv_count, sigma, sbar, trig, None, ws)
+
+        def attend():
+            sa.sparse_attn_decode(kv, lay.q, 2048, lay.q_pos0, 64, 1.0 / math.sqrt(128), kv_idx,
+                                  kv_count, W, out, None, ws)
+
+        for _ in range(warmup):
+            route()
+            attend()
+        ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(steps)]
+        torch.cuda.synchronize()
+        for i in range(steps):
+            ev[i][0].record(stream)
+            route()
+            ev[i][1].record(stream)
+            attend()
+            ev[i][2].record(stream)
+        torch.cuda.synchronize()
+        r_ms = sum(e[0].elapsed_time(e[1]) for e in ev) / steps
+        a_ms = sum(e[1].elapsed_time(e[2]) for e in ev) / steps
+        if sa.sparse_attn_get_device_status(ws) != 0:
+            raise RuntimeError("router leg: device status set")
+        E = np.array([min(nblk, (lay.q_pos0 + 64 * (t + 1) - 1) // 64 + 1) for t in range(T)])
+        kdim = 256 if rule == "envelope" else 128
+        score_flop = float(2 * 448 * E.sum() * kdim * Hkv)
+        kept_tok = float(kv_count.sum().item()) * 64
+        attn_flop = 4.0 * 128 * 448 * kept_tok
+        res[rule] = {"route_ms": round(r_ms, 4), "tile_attention_ms": round(a_ms, 4),
+                     "route_tflops": round(score_flop / (r_ms * 1e-3) / 1e12, 1),
+                     "tile_attention_tflops": round(attn_flop / (a_ms * 1e-3) / 1e12, 1),
+                     "triggered_tiles": int(trig.sum().item()),
+                     "score_gflop": round(score_flop / 1e9, 1), "attention_gflop": round(attn_flop / 1e9, 1)}
+    return res
 
 
 class _Null:
@@ -396,6 +507,23 @@ def peaks():
             d = json.load(f)
         return float(d["hbm_gbs"]), "measured"
     return 6650.0, "fallback"
+
+
+# DRAM bytes read + written per launch (dram__bytes_read.sum + dram__bytes_write.sum),
+# from one ncu capture of the current kernels on this workload (48 stacked
+# layers, 29,504 tokens, envelope, 4096-token budget); other settings: null.
+NCU_TRAFFIC = {
+    ("decode", "envelope", 4096): 403_413_248 + 7_616_512,
+    ("select", "envelope", 4096): 182_304_768 + 4_662_272,
+}
+
+
+def peaks_tflops():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            return float(json.load(f)["bf16_tflops"])
+    return 1590.0
 
 
 def main():
@@ -462,7 +590,8 @@ def main():
     if dom:
         ach = dom_bytes / (dom_ms * 1e-3) / 1e9
         roof = {"kernel": dom, "bound": "hbm", "achieved": round(ach, 1), "peak": peak, "unit": "GB/s",
-                "frac": round(ach / peak, 4), "peak_source": peak_kind, "traffic": None,
+                "frac": round(ach / peak, 4), "peak_source": peak_kind,
+                "traffic": NCU_TRAFFIC.get((dom, args.rule, args.budget)),
                 "algorithmic_bytes_per_launch": dom_bytes,
                 "avg_launch_ms": round(dom_ms, 5)}
     eff = (r["meta_bytes"] + r["kv_bytes"]) / (r["ms"] * 1e-3) / 1e9
@@ -478,11 +607,15 @@ def main():
         "effective_GBps": round(eff, 1), "effective_frac_of_peak": round(eff / peak, 4),
         "per_kernel_ms": {k: round(v, 5) for k, v in kern.items()} if kern else None,
         "roofline": roof, "clocks": r["clocks"],
-        "e2e": {"value": HQ * args.budget * LAYERS * B * world / (r["e2e_ms"] * 1e-3), "unit": UNIT,
+        "e2e": {"value": whole_job_value(HQ * args.budget * LAYERS * B, world, r["e2e_ms"]), "unit": UNIT,
                 "ms_per_step": round(r["e2e_ms"], 5), "h2d_bytes_per_step": r["h2d"],
                 "d2h_bytes_per_step": r["d2h"]},
         "gpu_launches": r["launches_per_step"] * args.steps,
         "cpu_baseline": cpu, "modes": r["extra"],
+        "router": None if r["router"] is None else {
+            "workload": "router-qwen2.5-7b-128k: 28:4 heads, 131072 tokens, 64-token blocks, "
+                        "2048 rows in 32 tiles, k=32, rho=2, q=0.25",
+            "bound": "tensor", "peak_tflops_bf16": peaks_tflops(), **r["router"]},
     }
     print(json.dumps(line))
     return 0
