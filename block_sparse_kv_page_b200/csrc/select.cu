@@ -57,6 +57,9 @@ constexpr int kBoxBytes = 2048;
 constexpr int kRingBytes = kSelWarps * kSelStages * kTileBytes;
 constexpr int kOffBars = kRingBytes;
 
+// Selection-phase shared memory: keys and weights, 4 B each per page.
+__host__ __device__ constexpr int select_keys_bytes(int max_pages) { return 8 * max_pages; }
+
 struct SelSmem {
   unsigned char* ring;   // [warp][stage][kTileBytes]; reused for keys/weights in selection
   uint64_t* bars;        // [warp][stage]
@@ -334,7 +337,7 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(const __grid_consta
   unsigned char* base = reinterpret_cast<unsigned char*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   // barriers sit after the ring, or after the keys/weights area when that is larger
-  const int keys_bytes = 8 * a.kv.max_pages;
+  const int keys_bytes = select_keys_bytes(a.kv.max_pages);
   const int bar_off = keys_bytes > kRingBytes ? ((keys_bytes + 1023) & ~1023) : kOffBars;
   const SelSmem S{base, reinterpret_cast<uint64_t*>(base + bar_off), s_hist, s_scan, s_bc, &s_last};
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -386,7 +389,7 @@ int select_splits(int units, int max_pages, int sm_count) {
 }
 
 size_t select_smem_bytes(int max_pages) {
-  const size_t keys = ((size_t)max_pages * 8 + 1023) & ~(size_t)1023;
+  const size_t keys = ((size_t)select_keys_bytes(max_pages) + 1023) & ~(size_t)1023;
   const size_t body = keys > (size_t)kRingBytes ? keys : (size_t)kRingBytes;
   return 1024 + body + kSelWarps * kSelStages * 8;
 }
