@@ -8,10 +8,15 @@ One step = one pass of the whole path over the 48 layers:
   incremental metadata update of the page holding the newest token
   -> page scoring + top-k selection -> split-K sparse attention + combine.
 Modes:
-  batched    : the 48 independent layers are stacked along the batch axis,
-               so each stage is one launch per step (3 launches);
-  sequential : one call per layer and stage (144 launches per step), replayed
-               as one CUDA graph per step, as a dependent layer sweep would be.
+  step       : (headline) the 48 independent layers are stacked along the
+               batch axis and the whole step is ONE sparse_attn_decode_step
+               launch (scoring, selection and decode items share one
+               persistent grid);
+  step-seq   : one sparse_attn_decode_step per layer (48 launches per step),
+               replayed as one CUDA graph, as a dependent layer sweep would be;
+  batched    : stacked layers, one launch per stage (build_meta, select,
+               decode: 3 launches per step);
+  sequential : one call per layer and stage (144 launches per step) in a graph.
 
 Output: one JSON line on rank 0.  `value` = tokens*heads/s (tokens attended x
 query heads x layers per step / step time, summed over ranks).  Inputs stay
@@ -41,6 +46,8 @@ G = HQ // HKV
 METRIC = "sparse decode attention: tokens·heads/s and effective HBM GB/s vs B200 peak"
 UNIT = "tokens·heads/s"
 WORKLOAD = "qwen3vl30b-a3b-decode-29.5k"
+# launches of our kernels per step in each mode
+MODES = {"step": 1, "step-seq": LAYERS, "batched": 3, "sequential": 3 * LAYERS}
 
 
 def parse():
@@ -49,7 +56,7 @@ def parse():
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--mode", choices=["batched", "sequential"], default="batched")
+    ap.add_argument("--mode", choices=list(MODES), default="step")
     ap.add_argument("--rule", choices=["envelope", "centroid"], default="envelope")
     ap.add_argument("--budget", type=int, default=4096)
     ap.add_argument("--cpu-sample-units", type=int, default=192)
@@ -291,6 +298,19 @@ def run_gpu_arm(args, rank, world, dist):
         sa.sparse_attn_decode(kv, inp["q"], L * B, 0, 1, scale, sel, cnt, k, out, lse, ws)
         if ev: ev[3].record(stream)
 
+    def step_fused(rule, ev=None):
+        if ev: ev[0].record(stream)
+        sa.sparse_attn_decode_step(kv, metas[rule], rule, inp["q"], budget, k, scale, sel, cnt, out,
+                                   lse, ws)
+        if ev: ev[1].record(stream)
+
+    def step_fused_layers(rule):
+        m = metas[rule]
+        for l in range(L):
+            sl = slice(l * B, (l + 1) * B)
+            sa.sparse_attn_decode_step(views[l], m[sl], rule, inp["q"][sl], budget, k, scale, sel[sl],
+                                       cnt[sl], out[sl], lse[sl], lay_ws)
+
     def step_sequential(rule):
         m = metas[rule]
         for l in range(L):
@@ -303,19 +323,20 @@ def run_gpu_arm(args, rank, world, dist):
 
     graphs = {}
 
-    def seq_graph(rule):
-        if rule not in graphs:
+    def seq_graph(mode, rule):
+        if (mode, rule) not in graphs:
+            body = step_fused_layers if mode == "step-seq" else step_sequential
             s = torch.cuda.Stream()
             s.wait_stream(stream)
             with torch.cuda.stream(s):
-                step_sequential(rule)  # warm (attributes, lazy init) outside capture
+                body(rule)  # warm (attributes, lazy init) outside capture
             stream.wait_stream(s)
             torch.cuda.synchronize()
             g = torch.cuda.CUDAGraph()
             with torch.cuda.graph(g):
-                step_sequential(rule)
-            graphs[rule] = g
-        return graphs[rule]
+                body(rule)
+            graphs[(mode, rule)] = g
+        return graphs[(mode, rule)]
 
     def barrier():
         if dist is not None:
@@ -323,16 +344,20 @@ def run_gpu_arm(args, rank, world, dist):
         torch.cuda.synchronize()
 
     def timed(mode, rule, steps, warmup, per_kernel=False, clocks=None):
-        if mode == "sequential":
-            g = seq_graph(rule)
+        if mode in ("sequential", "step-seq"):
+            g = seq_graph(mode, rule)
             fn = g.replay
+        elif mode == "step":
+            fn = lambda: step_fused(rule)  # noqa: E731
         else:
             fn = lambda: step_batched(rule)  # noqa: E731
         for _ in range(warmup):
             fn()
         evs = None
-        if per_kernel and mode == "batched":
-            evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(steps)]
+        names = {"batched": ("build_meta", "select", "decode"), "step": ("step",)}.get(mode)
+        if per_kernel and names:
+            evs = [[torch.cuda.Event(enable_timing=True) for _ in range(len(names) + 1)]
+                   for _ in range(steps)]
         barrier()
         t0 = torch.cuda.Event(enable_timing=True)
         t1 = torch.cuda.Event(enable_timing=True)
@@ -340,7 +365,9 @@ def run_gpu_arm(args, rank, world, dist):
         with ctx:
             t0.record(stream)
             for i in range(steps):
-                if evs:
+                if evs and mode == "step":
+                    step_fused(rule, evs[i])
+                elif evs:
                     step_batched(rule, evs[i])
                 else:
                     fn()
@@ -350,18 +377,18 @@ def run_gpu_arm(args, rank, world, dist):
         kern = None
         if evs:
             kern = {name: sum(e[i].elapsed_time(e[i + 1]) for e in evs) / steps
-                    for i, name in enumerate(("build_meta", "select", "decode"))}
+                    for i, name in enumerate(names)}
         return ms / steps, kern
 
     # ---- headline
     clocks = ClockSampler(dev.index if dev.index is not None else 0)
-    ms, kern = timed(args.mode, args.rule, args.steps, args.warmup, per_kernel=(args.mode == "batched"),
-                     clocks=clocks)
+    ms, kern = timed(args.mode, args.rule, args.steps, args.warmup,
+                     per_kernel=args.mode in ("batched", "step"), clocks=clocks)
     status = sa.sparse_attn_get_device_status(ws)
     if status != 0:
         raise RuntimeError(f"device status {status} after the timed steps")
-    if args.mode == "batched" and kern is None:
-        _, kern = timed("batched", args.rule, max(3, min(args.steps, 50)), 2, per_kernel=True)
+    if kern is None:  # graph modes: per-kernel split of the stacked launches, labelled as such
+        _, kern = timed("step", args.rule, max(3, min(args.steps, 50)), 2, per_kernel=True)
     tok_heads = args.budget * HQ * L * B
     value = whole_job_value(tok_heads, world, ms)
     meta_bytes = L * B * HKV * (N // PS) * 512
@@ -377,8 +404,10 @@ def run_gpu_arm(args, rank, world, dist):
         inp["q"].copy_(q_h, non_blocking=True)
         inp["k"][:, :, N - 1, :].copy_(knew_h, non_blocking=True)
         inp["v"][:, :, N - 1, :].copy_(vnew_h, non_blocking=True)
-        if args.mode == "sequential":
-            seq_graph(args.rule).replay()
+        if args.mode in ("sequential", "step-seq"):
+            seq_graph(args.mode, args.rule).replay()
+        elif args.mode == "step":
+            step_fused(args.rule)
         else:
             step_batched(args.rule)
         out_h.copy_(out, non_blocking=True)
@@ -400,7 +429,7 @@ def run_gpu_arm(args, rank, world, dist):
     # ---- secondary measurements (same timing rules), labelled
     extra = {}
     if not args.no_extra:
-        for mode in ("batched", "sequential"):
+        for mode in MODES:
             for rule in ("envelope", "centroid"):
                 if (mode, rule) == (args.mode, args.rule):
                     continue
@@ -416,7 +445,7 @@ def run_gpu_arm(args, rank, world, dist):
         router = router_leg(torch, dev, max(5, min(args.steps, 50)), max(3, args.warmup))
     return dict(ms=ms, value=value, kern=kern, clocks=clocks.summary(), e2e_ms=e2e_ms, h2d=h2d,
                 d2h=d2h, meta_bytes=meta_bytes, kv_bytes=kv_bytes, extra=extra, router=router,
-                launches_per_step=3 if args.mode == "batched" else 3 * L)
+                launches_per_step=MODES[args.mode])
 
 
 def router_leg(torch, dev, steps: int, warmup: int):
@@ -579,8 +608,10 @@ def main():
     kern = r["kern"] or {}
     dec_ms = kern.get("decode")
     sel_ms = kern.get("select")
-    # dominant kernel: the one with the larger average launch time
-    if dec_ms is not None and (sel_ms is None or dec_ms >= sel_ms):
+    # dominant kernel: the fused step kernel, else the longer of decode / select
+    if kern.get("step") is not None:
+        dom, dom_ms, dom_bytes = "step", kern["step"], r["meta_bytes"] + r["kv_bytes"]
+    elif dec_ms is not None and (sel_ms is None or dec_ms >= sel_ms):
         dom, dom_ms, dom_bytes = "decode", dec_ms, r["kv_bytes"]
     elif sel_ms is not None:
         dom, dom_ms, dom_bytes = "select", sel_ms, r["meta_bytes"]

@@ -1,19 +1,21 @@
 // C-ABI entry points: host-side argument validation, workspace layout and
 // kernel launches.  Nothing here computes results; every step of the path
-// runs in the kernels of meta.cu, select.cu, decode.cu and route.cu.
+// runs in the kernels of meta.cu, select.cu, decode.cu, step.cu, route.cu and
+// tile_attn.cu.
 //
 // Workspace layout (byte offsets from ws, which must be 256-byte aligned):
 //   [0, 256)                 status word (int32) at 0; item-queue counters of
 //                            the persistent kernels at 64 (select), 72
-//                            (decode), 80 (router); each kernel leaves its
-//                            queue rewound to zero
+//                            (decode), 80 (router), 88 (decode step); each
+//                            kernel leaves its queue rewound to zero
 //   [256, 256 + 4*kMaxUnits) last-CTA counters, shared by every call; each
 //                            call uses counters [0, its units) and leaves
 //                            them zero, so calls issued in order on one
 //                            stream can share one workspace
 //   [kScratch, ...)          per-call scratch (scores of select, split
-//                            partials of decode, router tables), not
-//                            preserved between calls
+//                            partials of decode -- after the scores in the
+//                            decode step --, router tables), not preserved
+//                            between calls
 #include <cmath>
 #include <cstdint>
 #include <cstring>
@@ -27,6 +29,7 @@ constexpr int kMaxUnits = 65536;
 constexpr size_t kQueueSelect = 64;
 constexpr size_t kQueueDecode = 72;
 constexpr size_t kQueueRoute = 80;
+constexpr size_t kQueueStep = 88;
 constexpr int kMaxRouteTiles = 1024;
 constexpr int kMaxRouteList = 1023;
 constexpr size_t kScratch = 256 + 4 * (size_t)kMaxUnits;
@@ -227,56 +230,14 @@ sa_status tile_attention(const sa_kv_desc* kv, const void* q, int n_q_heads, int
   a.status = status;
   return launched(launch_tile_attn(a, (cudaStream_t)stream));
 }
-}  // namespace
 
-}  // namespace sa
-
-using namespace sa;
-
-extern "C" {
-
-size_t sparse_attn_workspace_size(const sa_kv_desc* kv, int32_t n_q_heads, int32_t n_q_rows,
-                                  int32_t max_sel) {
-  if (check_kv(kv) != SA_OK || max_sel < 1 || n_q_rows < 0) return 0;
-  int G;
-  if (check_group(kv, n_q_heads, &G) != SA_OK) return 0;
-  const int sm = device_sm_count();
-  const int rows = n_q_rows > kv->batch ? n_q_rows : kv->batch;
-  const long long units = (long long)rows * kv->n_kv_heads;
-  if (units > kMaxUnits) return 0;
-  size_t tail = select_scratch(kv);
-  const int splits = decode_splits((int)units, max_tiles_per_unit(kv, max_sel), sm);
-  const size_t dec = decode_scratch((int)units, splits);
-  if (dec > tail) tail = dec;
-  const int route_tiles = rows < kMaxRouteTiles ? rows : kMaxRouteTiles;  // tiles <= query rows
-  const size_t rt = route_ws_bytes(route_tiles, kv->n_kv_heads, kv->max_pages, max_sel);
-  if (rt > tail) tail = rt;
-  return kScratch + tail;
-}
-
-sa_status sparse_attn_workspace_init(void* ws, size_t ws_bytes, void* stream) {
-  if (!ws || !aligned(ws, 256) || ws_bytes < kScratch) return SA_ERR_WORKSPACE;
-  return launched(cudaMemsetAsync(ws, 0, ws_bytes, (cudaStream_t)stream));
-}
-
-sa_status sparse_attn_build_meta(const sa_kv_desc* kv, sa_score_rule rule, int32_t first_token,
-                                 void* meta, void* stream) {
+// Argument checks of a selection (sparse_attn_select and sparse_attn_decode_step).
+sa_status check_select(const sa_kv_desc* kv, const void* meta, sa_score_rule rule, const void* q,
+                       int n_q_heads, const sa_budget* budget, int max_sel, const int32_t* sel_idx,
+                       const int32_t* sel_count, const float* scores_out, int* G) {
   sa_status s = check_kv(kv);
   if (s != SA_OK) return s;
-  if (rule != SA_SCORE_ENVELOPE && rule != SA_SCORE_CENTROID) return SA_ERR_INVALID;
-  if (!meta || !aligned(meta, 16)) return SA_ERR_INVALID;
-  return launched(launch_build_meta(view(kv), (int)rule, first_token, meta, nullptr,
-                                    (cudaStream_t)stream));
-}
-
-sa_status sparse_attn_select(const sa_kv_desc* kv, const void* meta, sa_score_rule rule,
-                             const void* q, int32_t n_q_heads, const sa_budget* budget,
-                             int32_t max_sel, int32_t* sel_idx, int32_t* sel_count,
-                             float* scores_out, void* ws, size_t ws_bytes, void* stream) {
-  sa_status s = check_kv(kv);
-  if (s != SA_OK) return s;
-  int G;
-  if ((s = check_group(kv, n_q_heads, &G)) != SA_OK) return s;
+  if ((s = check_group(kv, n_q_heads, G)) != SA_OK) return s;
   if (rule != SA_SCORE_ENVELOPE && rule != SA_SCORE_CENTROID) return SA_ERR_INVALID;
   if (!meta || !aligned(meta, 16) || !q || !aligned(q, 16)) return SA_ERR_INVALID;
   if (!budget || !sel_idx || !sel_count || max_sel < 1) return SA_ERR_INVALID;
@@ -306,39 +267,134 @@ sa_status sparse_attn_select(const sa_kv_desc* kv, const void* meta, sa_score_ru
     default:
       return SA_ERR_INVALID;
   }
-  const size_t need = kScratch + select_scratch(kv);
-  if ((s = check_ws(ws, ws_bytes, need)) != SA_OK) return s;
   const unsigned long long meta_rows = (unsigned long long)units * kv->max_pages;
   if (meta_rows > 0x7fffffffULL) return SA_ERR_UNSUPPORTED;  // TMA row coordinates are int32
+  return SA_OK;
+}
 
-  SelectArgs a;
+// Selection arguments (scores in the scratch, unit counters after the
+// header); false if the metadata tensor map cannot be encoded.
+bool fill_select(SelectArgs* a, const sa_kv_desc* kv, const void* meta, sa_score_rule rule,
+                 const void* q, int n_q_heads, int G, const sa_budget* budget, int max_sel,
+                 int32_t* sel_idx, int32_t* sel_count, float* scores_out, void* ws) {
+  const unsigned long long meta_rows = (unsigned long long)kv->batch * kv->n_kv_heads * kv->max_pages;
   const bool env = rule == SA_SCORE_ENVELOPE;
-  if (!encode_tmap_2d(&a.tmap_meta, meta, meta_rows, kMetaBytes,
+  if (!encode_tmap_2d(&a->tmap_meta, meta, meta_rows, kMetaBytes,
                       env ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32,
                       env ? 2 : 4, 16))
+    return false;
+  a->kv = view(kv);
+  a->meta = meta;
+  a->rule = (int)rule;
+  a->q = q;
+  a->Hq = n_q_heads;
+  a->G = G;
+  a->budget_kind = (int)budget->kind;
+  a->top_k = budget->top_k;
+  a->topk_val = budget->topk_val;
+  a->bos = budget->bos;
+  a->eos = budget->eos;
+  a->token_budget = budget->token_budget;
+  a->ratio = budget->topk_ratio;
+  a->max_sel = max_sel;
+  a->sel_idx = sel_idx;
+  a->sel_count = sel_count;
+  a->scores_out = scores_out;
+  a->ws_scores = reinterpret_cast<float*>(reinterpret_cast<char*>(ws) + kScratch);
+  a->ws_count = reinterpret_cast<uint32_t*>(reinterpret_cast<char*>(ws) + 256);
+  a->ws_queue = nullptr;
+  a->status = reinterpret_cast<int*>(ws);
+  a->splits = select_splits(kv->batch * kv->n_kv_heads, kv->max_pages, device_sm_count());
+  a->meta_refresh = nullptr;
+  return true;
+}
+
+// Decode arguments for one query row per sequence (tile_rows = 1); false if
+// the K/V tensor maps cannot be encoded.
+bool fill_decode(DecodeArgs* a, const sa_kv_desc* kv, const void* q, int n_q_heads, int G,
+                 float scale, const int32_t* idx, const int32_t* count, int max_sel, float* out,
+                 float* lse, float* ws_part, uint32_t* ws_count, int* status, int splits) {
+  const unsigned long long kv_rows = (unsigned long long)kv->batch * kv->n_kv_heads * kv->cap_tokens;
+  if (!encode_tmap_2d(&a->tmap_k, kv->k, kv_rows, kHeadDim * 2, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, 16) ||
+      !encode_tmap_2d(&a->tmap_v, kv->v, kv_rows, kHeadDim * 2, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, 16))
+    return false;
+  a->kv = view(kv);
+  a->q = q;
+  a->Hq = n_q_heads;
+  a->G = G;
+  a->n_rows = kv->batch;
+  a->q_pos0 = 0;
+  a->tile_rows = 1;
+  a->scale_log2 = scale * kLog2e;
+  a->idx = idx;
+  a->count = count;
+  a->max_sel = max_sel;
+  a->out = out;
+  a->lse = lse;
+  a->ws_part = ws_part;
+  a->ws_count = ws_count;
+  a->ws_queue = nullptr;
+  a->status = status;
+  a->splits = splits;
+  return true;
+}
+
+}  // namespace
+
+}  // namespace sa
+
+using namespace sa;
+
+extern "C" {
+
+size_t sparse_attn_workspace_size(const sa_kv_desc* kv, int32_t n_q_heads, int32_t n_q_rows,
+                                  int32_t max_sel) {
+  if (check_kv(kv) != SA_OK || max_sel < 1 || n_q_rows < 0) return 0;
+  int G;
+  if (check_group(kv, n_q_heads, &G) != SA_OK) return 0;
+  const int sm = device_sm_count();
+  const int rows = n_q_rows > kv->batch ? n_q_rows : kv->batch;
+  const long long units = (long long)rows * kv->n_kv_heads;
+  if (units > kMaxUnits) return 0;
+  // selection scores + decode partials (both live during sparse_attn_decode_step)
+  const int splits = decode_splits((int)units, max_tiles_per_unit(kv, max_sel), sm);
+  size_t tail = select_scratch(kv) + decode_scratch((int)units, splits);
+  const int route_tiles = rows < kMaxRouteTiles ? rows : kMaxRouteTiles;  // tiles <= query rows
+  const size_t rt = route_ws_bytes(route_tiles, kv->n_kv_heads, kv->max_pages, max_sel);
+  if (rt > tail) tail = rt;
+  return kScratch + tail;
+}
+
+sa_status sparse_attn_workspace_init(void* ws, size_t ws_bytes, void* stream) {
+  if (!ws || !aligned(ws, 256) || ws_bytes < kScratch) return SA_ERR_WORKSPACE;
+  return launched(cudaMemsetAsync(ws, 0, ws_bytes, (cudaStream_t)stream));
+}
+
+sa_status sparse_attn_build_meta(const sa_kv_desc* kv, sa_score_rule rule, int32_t first_token,
+                                 void* meta, void* stream) {
+  sa_status s = check_kv(kv);
+  if (s != SA_OK) return s;
+  if (rule != SA_SCORE_ENVELOPE && rule != SA_SCORE_CENTROID) return SA_ERR_INVALID;
+  if (!meta || !aligned(meta, 16)) return SA_ERR_INVALID;
+  return launched(launch_build_meta(view(kv), (int)rule, first_token, meta, nullptr,
+                                    (cudaStream_t)stream));
+}
+
+sa_status sparse_attn_select(const sa_kv_desc* kv, const void* meta, sa_score_rule rule,
+                             const void* q, int32_t n_q_heads, const sa_budget* budget,
+                             int32_t max_sel, int32_t* sel_idx, int32_t* sel_count,
+                             float* scores_out, void* ws, size_t ws_bytes, void* stream) {
+  int G;
+  sa_status s = check_select(kv, meta, rule, q, n_q_heads, budget, max_sel, sel_idx, sel_count,
+                             scores_out, &G);
+  if (s != SA_OK) return s;
+  const size_t need = kScratch + select_scratch(kv);
+  if ((s = check_ws(ws, ws_bytes, need)) != SA_OK) return s;
+  SelectArgs a;
+  if (!fill_select(&a, kv, meta, rule, q, n_q_heads, G, budget, max_sel, sel_idx, sel_count,
+                   scores_out, ws))
     return SA_ERR_CUDA;
-  a.kv = view(kv);
-  a.meta = meta;
-  a.rule = (int)rule;
-  a.q = q;
-  a.Hq = n_q_heads;
-  a.G = G;
-  a.budget_kind = (int)budget->kind;
-  a.top_k = budget->top_k;
-  a.topk_val = budget->topk_val;
-  a.bos = budget->bos;
-  a.eos = budget->eos;
-  a.token_budget = budget->token_budget;
-  a.ratio = budget->topk_ratio;
-  a.max_sel = max_sel;
-  a.sel_idx = sel_idx;
-  a.sel_count = sel_count;
-  a.scores_out = scores_out;
-  a.ws_scores = reinterpret_cast<float*>(reinterpret_cast<char*>(ws) + kScratch);
-  a.ws_count = reinterpret_cast<uint32_t*>(reinterpret_cast<char*>(ws) + 256);
   a.ws_queue = reinterpret_cast<uint32_t*>(reinterpret_cast<char*>(ws) + kQueueSelect);
-  a.status = reinterpret_cast<int*>(ws);
-  a.splits = select_splits((int)units, kv->max_pages, device_sm_count());
   return launched(launch_select(a, (cudaStream_t)stream));
 }
 
@@ -372,28 +428,54 @@ sa_status sparse_attn_decode(const sa_kv_desc* kv, const void* q, int32_t n_q_he
   if ((s = check_ws(ws, ws_bytes, need)) != SA_OK) return s;
 
   DecodeArgs a;
-  if (!encode_tmap_2d(&a.tmap_k, kv->k, kv_rows, kHeadDim * 2, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, 16) ||
-      !encode_tmap_2d(&a.tmap_v, kv->v, kv_rows, kHeadDim * 2, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, 16))
+  char* w = reinterpret_cast<char*>(ws);
+  if (!fill_decode(&a, kv, q, n_q_heads, G, scale, idx, count, max_sel, out, lse,
+                   reinterpret_cast<float*>(w + kScratch), reinterpret_cast<uint32_t*>(w + 256),
+                   reinterpret_cast<int*>(ws), splits))
     return SA_ERR_CUDA;
-  a.kv = view(kv);
-  a.q = q;
-  a.Hq = n_q_heads;
-  a.G = G;
-  a.n_rows = n_q_rows;
-  a.q_pos0 = q_pos0;
-  a.tile_rows = tile_rows;
-  a.scale_log2 = scale * kLog2e;
-  a.idx = idx;
-  a.count = count;
-  a.max_sel = max_sel;
-  a.out = out;
-  a.lse = lse;
-  a.ws_part = reinterpret_cast<float*>(reinterpret_cast<char*>(ws) + kScratch);
-  a.ws_count = reinterpret_cast<uint32_t*>(reinterpret_cast<char*>(ws) + 256);
-  a.ws_queue = reinterpret_cast<uint32_t*>(reinterpret_cast<char*>(ws) + kQueueDecode);
-  a.status = reinterpret_cast<int*>(ws);
-  a.splits = splits;
+  a.ws_queue = reinterpret_cast<uint32_t*>(w + kQueueDecode);
   return launched(launch_decode(a, (cudaStream_t)stream));
+}
+
+sa_status sparse_attn_decode_step(const sa_kv_desc* kv, void* meta, sa_score_rule rule,
+                                  const void* q, int32_t n_q_heads, const sa_budget* budget,
+                                  int32_t max_sel, float scale, int32_t* sel_idx,
+                                  int32_t* sel_count, float* out, float* lse, void* ws,
+                                  size_t ws_bytes, void* stream) {
+  int G;
+  sa_status s = check_select(kv, meta, rule, q, n_q_heads, budget, max_sel, sel_idx, sel_count,
+                             nullptr, &G);
+  if (s != SA_OK) return s;
+  if (!out || !aligned(out, 16) || (lse && !aligned(lse, 4))) return SA_ERR_INVALID;
+  if (!std::isfinite(scale)) return SA_ERR_INVALID;
+  if (kv->page_size == 0 && max_sel > kMaxChunkSel) return SA_ERR_UNSUPPORTED;
+  const long long units = (long long)kv->batch * kv->n_kv_heads;
+  if (2 * units > kMaxUnits) return SA_ERR_UNSUPPORTED;  // unit flags + split counters
+  const unsigned long long kv_rows = (unsigned long long)kv->batch * kv->n_kv_heads * kv->cap_tokens;
+  if (kv_rows > 0x7fffffffULL) return SA_ERR_UNSUPPORTED;  // TMA row coordinates are int32
+  const int sm = device_sm_count();
+  const int dsplits = decode_splits((int)units, max_tiles_per_unit(kv, max_sel), sm);
+  const size_t sel_bytes = select_scratch(kv);
+  const size_t need = kScratch + sel_bytes + decode_scratch((int)units, dsplits);
+  if ((s = check_ws(ws, ws_bytes, need)) != SA_OK) return s;
+  if (step_smem_bytes(kv->max_pages, max_sel, kv->page_size == 0) > 227 * 1024)
+    return SA_ERR_UNSUPPORTED;
+
+  StepArgs a;
+  char* w = reinterpret_cast<char*>(ws);
+  if (!fill_select(&a.sel, kv, meta, rule, q, n_q_heads, G, budget, max_sel, sel_idx, sel_count,
+                   nullptr, ws) ||
+      !fill_decode(&a.dec, kv, q, n_q_heads, G, scale, sel_idx, sel_count, max_sel, out, lse,
+                   reinterpret_cast<float*>(w + kScratch + sel_bytes),
+                   reinterpret_cast<uint32_t*>(w + 256) + units, reinterpret_cast<int*>(ws), dsplits))
+    return SA_ERR_CUDA;
+  a.sel.meta_refresh = static_cast<unsigned char*>(meta);
+  a.queue = reinterpret_cast<uint32_t*>(w + kQueueStep);
+  const long long n_score = units * a.sel.splits, n_dec = units * dsplits;
+  if (n_score + n_dec > 0x7fffffffLL) return SA_ERR_UNSUPPORTED;
+  a.n_score = (int)n_score;
+  a.n_dec = (int)n_dec;
+  return launched(launch_step(a, (cudaStream_t)stream));
 }
 
 sa_status sparse_attn_route(const sa_kv_desc* kv, const void* meta, sa_score_rule rule,

@@ -114,6 +114,25 @@ SA_DEV void prefetch_tmap(const void* tmap) {
   asm volatile("prefetch.tensormap [%0];\n" ::"l"(tmap) : "memory");
 }
 
+// Position of one warp in its private ring of mbarrier-tracked stages.  The
+// ring outlives work items: stage = gi % stages, phase parity = (gi / stages) & 1.
+struct WarpState {
+  uint32_t gi;           // stages consumed so far by this warp
+  bool alive;            // false after a barrier wait timed out
+  uint32_t drain_lo;     // after a timeout: stages [drain_lo, drain_hi) may still be landing
+  uint32_t drain_hi;
+};
+
+// GPU-scope acquire load / release store of a 32-bit flag in global memory.
+SA_DEV uint32_t ld_acquire_u32(const uint32_t* p) {
+  uint32_t v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];\n" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+SA_DEV void st_release_u32(uint32_t* p, uint32_t v) {
+  asm volatile("st.release.gpu.global.u32 [%0], %1;\n" ::"l"(p), "r"(v) : "memory");
+}
+
 // Byte offset of 16-byte chunk j (0..7) of row r inside a 128B-swizzled box
 // whose rows are 128 bytes (the TMA SWIZZLE_128B pattern: chunk j ^ (r & 7)).
 SA_DEV uint32_t swz128(int r, int j) { return (uint32_t)(r * 128 + ((j ^ (r & 7)) << 4)); }

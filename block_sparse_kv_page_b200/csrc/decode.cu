@@ -1,423 +1,27 @@
-// Sparse paged flash-decode over the selected pages, split-K + combine.
-//
-// "Sparse Attention for Web Agents -- Offline Replay Records", section "The
-// comparison": after choosing the best chunks the methods attend only to
-// them; exact softmax attention over the selected tokens.
-//
-// Work split.  A unit is one (sequence, KV head) with its G <= 8 query heads.
-// Its selected pages are cut into 16-token tiles (a 16-token page is one
-// tile; larger pages and variable chunks give several, the last one ragged)
-// and the tiles into `splits` contiguous ranges; an item is one (unit,
-// range).  A persistent grid (one or two CTAs per SM) pulls items from an
-// atomic queue, so the load balances whatever the unit count.
-//
-// Data movement.  K and V are streamed with TMA: a tile is four 2D boxes of
-// 16 rows x 64 bf16 (K low/high dims, V low/high dims) landing 128B-swizzled
-// in a per-warp ring of mbarrier-tracked stages.  Lane 0 of each warp issues
-// the copies for the warp's tiles several stages ahead; fragments are read
-// with ldmatrix (conflict-free under the swizzle).  Every barrier wait is
-// bounded and reports SA_ERR_TIMEOUT instead of hanging.
-//
-// Math per tile and warp (tensor cores, fp32 accumulation):
-//   QK:  S^T[16 tok x 8 heads] = K (16 x 128) . Q^T, m16n8k16 bf16;
-//   P:   exp2 of the scaled scores, rounded to a bf16 hi + lo pair, moved
-//        from the C layout to the B layout with movmatrix (8x8 transpose);
-//   PV:  O^T[128 dims x 8 heads] += V^T (128 x 16 tok) . P^T (ldmatrix.trans).
-// Each warp keeps its own online-softmax state; the warps merge in shared
-// memory; with several splits the CTA writes its (max, sum, acc) partial to
-// the workspace and the CTA that finishes the unit's last item (atomic
-// counter, no waiting) merges the partials in split order, so results do not
-// depend on scheduling.
+// Standalone sparse paged flash-decode kernel: a persistent grid pulls
+// (unit, tile range) items from an atomic queue and runs dec::decode_item on
+// each (decode_item.cuh: TMA-streamed K/V tiles of the selected pages,
+// tensor-core QK and PV, online softmax, last-CTA split combine).
 #include "common.cuh"
 #include "internal.h"
-
-#ifndef SA_DEC_WARPS
-#define SA_DEC_WARPS 4
-#endif
-#ifndef SA_DEC_STAGES
-#define SA_DEC_STAGES 2
-#endif
-#ifndef SA_DEC_ITEM_TILES
-#define SA_DEC_ITEM_TILES 64
-#endif
-#ifndef SA_DEC_CTAS_PER_SM
-#define SA_DEC_CTAS_PER_SM 3
-#endif
+#include "decode_item.cuh"
 
 namespace sa {
 namespace {
 
-constexpr int kDecWarps = SA_DEC_WARPS;
-constexpr int kDecThreads = kDecWarps * 32;
-constexpr int kDecStages = SA_DEC_STAGES;
-constexpr int kTileBytes = 8192;                 // K box lo | K box hi | V box lo | V box hi
-constexpr int kBoxBytes = 2048;                  // 16 rows x 128 B
-constexpr int kRingBytes = kDecWarps * kDecStages * kTileBytes;
-constexpr int kMaxItemTiles = SA_DEC_ITEM_TILES; // tile refs resolved per round
-constexpr int kPartStride = kMaxGroup * (kHeadDim + 2);  // floats per partial slot
-constexpr int kThreadsPerHead = kDecThreads / kMaxGroup;  // merge: threads per head
-constexpr int kDimsPerThread = kHeadDim / kThreadsPerHead;
-static_assert(kDimsPerThread % 4 == 0, "merge writes float4");
+using namespace dec;
 
-// Dynamic shared memory (offsets from a 1024-aligned base).
-constexpr int kOffBars = kRingBytes;
-constexpr int kOffTiles = kOffBars + kDecWarps * kDecStages * 8;
-constexpr int kOffPre = kOffTiles + kMaxItemTiles * 8;
-
-struct TileRef {
-  int row;     // first tile row in the [B*Hkv*cap] row space (u * cap + token)
-  int n;       // valid tokens (0 = empty tile)
-};
-
-struct Smem {
-  unsigned char* ring;   // [warp][stage][kTileBytes]
-  uint64_t* bars;        // [warp][stage]
-  TileRef* tiles;        // [kMaxItemTiles]
-  int* pre;              // chunk mode: tile prefix [max_sel + 1]
-  uint32_t* scan;        // kDecWarps words
-  int* last;
-  int* ntiles;
-};
-
-struct WarpState {
-  uint32_t gi;           // stages consumed so far by this warp (ring position + parity)
-  bool alive;            // false after a barrier wait timed out
-  uint32_t drain_lo;     // after a timeout: stages [drain_lo, drain_hi) may still be landing
-  uint32_t drain_hi;
-};
-
-SA_DEV void decode_item(const DecodeArgs& a, const int u, const int split, const Smem& sm,
-                        WarpState& ws) {
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int gq = lane >> 2, c = lane & 3;
-  const int Hkv = a.kv.Hkv;
-  const int b = u / Hkv, g = u % Hkv;
-  const int G = a.G;
-  const float ninf = -__int_as_float(0x7f800000);
-
-  // ---- geometry of the unit
-  const int N = a.kv.seq_len[b];
-  bool bad = (N < 1 || N > a.kv.cap);
-  int n_ent = a.count[u];
-  if (n_ent < 0 || n_ent > a.max_sel) bad = true;
-  if (bad) n_ent = 0;
-  const int32_t* idx_u = a.idx + (size_t)u * a.max_sel;
-  const int ps = a.kv.page_size;
-  const int sub = ps > 0 ? ps / 16 : 0;
-  int P = 0;
-  const int32_t* off = nullptr;
-  int* pre = sm.pre;
-  if (ps > 0) {
-    P = (N + ps - 1) / ps;
-    if (tid == 0) *sm.ntiles = n_ent * sub;
-  } else {
-    off = a.kv.chunk_off + (size_t)b * (a.kv.max_pages + 1);
-    P = a.kv.n_chunks[b];
-    if (P < 1 || P > a.kv.max_pages) { bad = true; n_ent = 0; P = 0; }
-    const int per = (n_ent + kDecThreads - 1) / kDecThreads;
-    const int e0 = min(n_ent, tid * per), e1 = min(n_ent, e0 + per);
-    uint32_t loc = 0;
-    for (int e = e0; e < e1; ++e) {
-      const int ch = idx_u[e];
-      int nt = 0;
-      if (ch >= 0 && ch < P && off[ch] >= 0) nt = (max(0, min(off[ch + 1], N) - off[ch]) + 15) >> 4;
-      pre[e] = nt;
-      loc += (uint32_t)nt;
-    }
-    uint32_t tot;
-    uint32_t run = block_excl_scan(loc, sm.scan, tot);
-    for (int e = e0; e < e1; ++e) {
-      const int nt = pre[e];
-      pre[e] = (int)run;
-      run += (uint32_t)nt;
-    }
-    if (tid == 0) { pre[n_ent] = (int)tot; *sm.ntiles = (int)tot; }
-  }
-  if (bad && tid == 0 && split == 0) flag_status(a.status, SA_ERR_DEVICE_CHECK);
-  __syncthreads();
-  const int T = *sm.ntiles;
-  const int t_begin = (int)(((long long)T * split) / a.splits);
-  const int t_end = (int)(((long long)T * (split + 1)) / a.splits);
-  const long long row0 = (long long)u * a.kv.cap;
-
-  // Token range of tile t of the unit (n = 0 for a skipped, invalid entry).
-  auto tile_ref = [&](int t) -> TileRef {
-    TileRef r{0, 0};
-    int start;
-    if (ps > 0) {
-      const int e = t / sub, part = t - e * sub;
-      const int p = idx_u[e];
-      if (p < 0 || p >= P) {
-        flag_status(a.status, SA_ERR_DEVICE_CHECK);
-        return r;
-      }
-      start = p * ps + part * 16;
-      r.n = max(0, min(16, N - start));
-    } else {
-      int lo = 0, hi = n_ent - 1;  // last e with pre[e] <= t
-      while (lo < hi) {
-        const int mid = (lo + hi + 1) >> 1;
-        if (pre[mid] <= t) lo = mid; else hi = mid - 1;
-      }
-      const int ch = idx_u[lo];
-      if (ch < 0 || ch >= P || off[ch] < 0) {
-        flag_status(a.status, SA_ERR_DEVICE_CHECK);
-        return r;
-      }
-      start = off[ch] + (t - pre[lo]) * 16;
-      r.n = max(0, min(16, min(off[ch + 1], N) - start));
-    }
-    r.row = (int)(row0 + start);
-    return r;
-  };
-
-  // ---- Q fragments (B operand, natural k order): q[head][16s + 2c (+8)]
-  const bool head_ok = gq < G;
-  const __nv_bfloat16* qrow = reinterpret_cast<const __nv_bfloat16*>(a.q) +
-                              ((size_t)b * a.Hq + (size_t)g * G + (head_ok ? gq : 0)) * kHeadDim;
-  uint32_t bq[16];
-#pragma unroll
-  for (int s = 0; s < 8; ++s) {
-    bq[2 * s + 0] = head_ok ? __ldg(reinterpret_cast<const uint32_t*>(qrow + 16 * s + 2 * c)) : 0u;
-    bq[2 * s + 1] = head_ok ? __ldg(reinterpret_cast<const uint32_t*>(qrow + 16 * s + 8 + 2 * c)) : 0u;
-  }
-
-  float m0 = ninf, m1 = ninf, l0 = 0.f, l1 = 0.f;
-  float acc[8][4];
-#pragma unroll
-  for (int mt = 0; mt < 8; ++mt) acc[mt][0] = acc[mt][1] = acc[mt][2] = acc[mt][3] = 0.f;
-
-  unsigned char* ring = sm.ring + warp * (kDecStages * kTileBytes);
-  uint64_t* bars = sm.bars + warp * kDecStages;
-  // ldmatrix lane addressing: matrix = lane / 8, row-in-matrix = lane % 8
-  const int lrow_a = (lane & 7) + 8 * ((lane >> 3) & 1);  // K: rows 0-7 / 8-15
-  const int lchk_a = lane >> 4;                            //    chunk +0 / +1
-  const int lrow_v = (lane & 7) + 8 * (lane >> 4);         // V: tokens 0-7 / 8-15
-  const int lchk_v = (lane >> 3) & 1;                      //    chunk +0 / +1
-
-  for (int r0 = t_begin; r0 < t_end; r0 += kMaxItemTiles) {
-    const int nt = min(kMaxItemTiles, t_end - r0);
-    for (int i = tid; i < nt; i += kDecThreads) sm.tiles[i] = tile_ref(r0 + i);
-    __syncthreads();
-
-    const int n_it = max(0, (nt - warp + kDecWarps - 1) / kDecWarps);
-    auto issue = [&](int it) {  // lane 0 only
-      const int t = warp + it * kDecWarps;
-      if (t >= nt) return;
-      const uint32_t g_it = ws.gi + (uint32_t)it;
-      uint64_t* bar = bars + g_it % kDecStages;
-      unsigned char* st = ring + (g_it % kDecStages) * kTileBytes;
-      const TileRef r = sm.tiles[t];
-      if (r.n == 0) {
-        mbar_arrive(bar);  // nothing to load: complete the phase
-        return;
-      }
-      mbar_arrive_expect_tx(bar, kTileBytes);
-      tma_load_2d(st + 0 * kBoxBytes, &a.tmap_k, 0, r.row, bar);
-      tma_load_2d(st + 1 * kBoxBytes, &a.tmap_k, 64, r.row, bar);
-      tma_load_2d(st + 2 * kBoxBytes, &a.tmap_v, 0, r.row, bar);
-      tma_load_2d(st + 3 * kBoxBytes, &a.tmap_v, 64, r.row, bar);
-    };
-    int issued = 0;  // tiles of this round issued so far (identical on every lane)
-    if (ws.alive) {
-      issued = min(n_it, kDecStages - 1);
-      if (lane == 0)
-        for (int it = 0; it < issued; ++it) issue(it);
-    }
-
-    for (int it = 0; it < n_it && ws.alive; ++it) {
-      __syncwarp();  // every lane is done reading the stage about to be refilled
-      if (it + kDecStages - 1 < n_it) {
-        if (lane == 0) issue(it + kDecStages - 1);
-        issued = it + kDecStages;
-      }
-      const uint32_t g_it = ws.gi + (uint32_t)it;
-      if (!mbar_wait(bars + g_it % kDecStages, (g_it / kDecStages) & 1u, a.status)) {
-        ws.alive = false;
-        ws.drain_lo = g_it;
-        ws.drain_hi = ws.gi + (uint32_t)issued;
-        break;
-      }
-      unsigned char* st = ring + (g_it % kDecStages) * kTileBytes;
-      const TileRef r = sm.tiles[warp + it * kDecWarps];
-      if (r.n < 16) {  // zero V rows past the valid tokens (they may hold other data)
-        for (int x = lane; x < (16 - r.n) * 16; x += 32) {
-          const int row = r.n + (x >> 4), ch = x & 15;
-          *reinterpret_cast<uint4*>(st + 2 * kBoxBytes + (ch >> 3) * kBoxBytes + swz128(row, ch & 7)) =
-              make_uint4(0u, 0u, 0u, 0u);
-        }
-        fence_proxy_async();
-        __syncwarp();
-      }
-
-      // S^T = K . Q^T, two independent accumulation chains
-      float s[4] = {0.f, 0.f, 0.f, 0.f}, s2[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-      for (int ks = 0; ks < 8; ++ks) {
-        uint32_t a0, a1, a2, a3;
-        ldsm_x4(a0, a1, a2, a3, st + (ks >> 2) * kBoxBytes + swz128(lrow_a, 2 * (ks & 3) + lchk_a));
-        if (ks & 1) mma_bf16(s2, a0, a1, a2, a3, bq[2 * ks], bq[2 * ks + 1]);
-        else        mma_bf16(s, a0, a1, a2, a3, bq[2 * ks], bq[2 * ks + 1]);
-      }
-      const bool v0 = gq < r.n, v1 = gq + 8 < r.n;
-      const float z0 = v0 ? (s[0] + s2[0]) * a.scale_log2 : ninf;
-      const float z1 = v0 ? (s[1] + s2[1]) * a.scale_log2 : ninf;
-      const float z2 = v1 ? (s[2] + s2[2]) * a.scale_log2 : ninf;
-      const float z3 = v1 ? (s[3] + s2[3]) * a.scale_log2 : ninf;
-      float mx0 = fmaxf(z0, z2), mx1 = fmaxf(z1, z3);
-#pragma unroll
-      for (int o = 4; o < 32; o <<= 1) {
-        mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, o));
-        mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, o));
-      }
-      const float mn0 = fmaxf(m0, mx0), mn1 = fmaxf(m1, mx1);
-      const float al0 = mn0 == ninf ? 1.f : exp2f(m0 - mn0);
-      const float al1 = mn1 == ninf ? 1.f : exp2f(m1 - mn1);
-      const float p0 = mn0 == ninf ? 0.f : exp2f(z0 - mn0);
-      const float p2 = mn0 == ninf ? 0.f : exp2f(z2 - mn0);
-      const float p1 = mn1 == ninf ? 0.f : exp2f(z1 - mn1);
-      const float p3 = mn1 == ninf ? 0.f : exp2f(z3 - mn1);
-      m0 = mn0; m1 = mn1;
-      l0 = l0 * al0 + (p0 + p2);
-      l1 = l1 * al1 + (p1 + p3);
-#pragma unroll
-      for (int mt = 0; mt < 8; ++mt) {
-        acc[mt][0] *= al0; acc[mt][1] *= al1; acc[mt][2] *= al0; acc[mt][3] *= al1;
-      }
-      // P (C layout: [token][head]) -> bf16 hi/lo -> B layout ([head][token])
-      const uint32_t hlo = pack_bf16(p0, p1), hhi = pack_bf16(p2, p3);
-      const uint32_t llo = pack_bf16(p0 - bf16_lo(hlo), p1 - bf16_hi(hlo));
-      const uint32_t lhi = pack_bf16(p2 - bf16_lo(hhi), p3 - bf16_hi(hhi));
-      const uint32_t bh0 = movmatrix_t(hlo), bh1 = movmatrix_t(hhi);
-      const uint32_t bl0 = movmatrix_t(llo), bl1 = movmatrix_t(lhi);
-
-      // O^T += V^T . P^T: m-tile mt = dims 16mt .. 16mt + 15
-#pragma unroll
-      for (int mt = 0; mt < 8; ++mt) {
-        uint32_t a0, a1, a2, a3;
-        ldsm_x4_t(a0, a1, a2, a3,
-                  st + (2 + (mt >> 2)) * kBoxBytes + swz128(lrow_v, 2 * (mt & 3) + lchk_v));
-        mma_bf16(acc[mt], a0, a1, a2, a3, bh0, bh1);
-        mma_bf16(acc[mt], a0, a1, a2, a3, bl0, bl1);
-      }
-    }
-    ws.gi += (uint32_t)n_it;
-    __syncthreads();  // tile refs of this round no longer read
-  }
-
-  // ---- merge the warps in shared memory
-#pragma unroll
-  for (int o = 4; o < 32; o <<= 1) {
-    l0 += __shfl_xor_sync(0xffffffffu, l0, o);
-    l1 += __shfl_xor_sync(0xffffffffu, l1, o);
-  }
-  __syncthreads();  // ring no longer read
-  float* w_acc = reinterpret_cast<float*>(sm.ring);                     // [warp][8][128]
-  float* w_ml = w_acc + kDecWarps * kMaxGroup * kHeadDim;               // [warp][8][2]
-  if (gq == 0) {
-    w_ml[(warp * kMaxGroup + 2 * c) * 2 + 0] = m0;
-    w_ml[(warp * kMaxGroup + 2 * c) * 2 + 1] = l0;
-    w_ml[(warp * kMaxGroup + 2 * c + 1) * 2 + 0] = m1;
-    w_ml[(warp * kMaxGroup + 2 * c + 1) * 2 + 1] = l1;
-  }
-#pragma unroll
-  for (int mt = 0; mt < 8; ++mt) {
-    float* h0 = w_acc + (warp * kMaxGroup + 2 * c) * kHeadDim + 16 * mt + gq;
-    float* h1 = w_acc + (warp * kMaxGroup + 2 * c + 1) * kHeadDim + 16 * mt + gq;
-    h0[0] = acc[mt][0];
-    h1[0] = acc[mt][1];
-    h0[8] = acc[mt][2];
-    h1[8] = acc[mt][3];
-  }
-  __syncthreads();
-
-  const int h = tid / kThreadsPerHead;               // head handled by this thread
-  const int d0 = (tid % kThreadsPerHead) * kDimsPerThread;
-  float M = ninf, L = 0.f, A[kDimsPerThread];
-#pragma unroll
-  for (int x = 0; x < kDimsPerThread; ++x) A[x] = 0.f;
-  if (h < G) {
-#pragma unroll
-    for (int w = 0; w < kDecWarps; ++w) M = fmaxf(M, w_ml[(w * kMaxGroup + h) * 2]);
-    if (M != ninf) {
-#pragma unroll
-      for (int w = 0; w < kDecWarps; ++w) {
-        const float f = exp2f(w_ml[(w * kMaxGroup + h) * 2] - M);
-        L += w_ml[(w * kMaxGroup + h) * 2 + 1] * f;
-        const float* src = w_acc + (w * kMaxGroup + h) * kHeadDim + d0;
-#pragma unroll
-        for (int x = 0; x < kDimsPerThread; ++x) A[x] += src[x] * f;
-      }
-    }
-  }
-  const size_t out_row = (size_t)b * a.Hq + (size_t)g * G + h;
-
-  if (a.splits == 1) {
-    if (h < G) {
-      const float inv = L > 0.f ? 1.f / L : 0.f;
-      float* o = a.out + out_row * kHeadDim + d0;
-#pragma unroll
-      for (int x = 0; x < kDimsPerThread; x += 4)
-        *reinterpret_cast<float4*>(o + x) = make_float4(A[x] * inv, A[x + 1] * inv, A[x + 2] * inv, A[x + 3] * inv);
-      if (a.lse && d0 == 0) a.lse[out_row] = L > 0.f ? M * kLn2 + logf(L) : ninf;
-    }
-    return;
-  }
-
-  // ---- several splits: publish the partial; the last CTA of the unit merges
-  float* part = a.ws_part + ((size_t)u * a.splits + split) * kPartStride;
-  if (h < G) {
-    float* dst = part + h * (kHeadDim + 2);
-#pragma unroll
-    for (int x = 0; x < kDimsPerThread; ++x) dst[d0 + x] = A[x];
-    if (d0 == 0) { dst[kHeadDim] = M; dst[kHeadDim + 1] = L; }
-  }
-  __threadfence();
-  __syncthreads();
-  if (tid == 0) {
-    const uint32_t prev = atomicAdd(&a.ws_count[u], 1u);
-    *sm.last = (prev == (uint32_t)(a.splits - 1));
-  }
-  __syncthreads();
-  if (!*sm.last) return;
-  __threadfence();
-  if (tid == 0) a.ws_count[u] = 0;
-  if (h >= G) return;
-
-  const float* base = a.ws_part + (size_t)u * a.splits * kPartStride + h * (kHeadDim + 2);
-  float MM = ninf;
-  for (int sp = 0; sp < a.splits; ++sp) MM = fmaxf(MM, __ldcg(base + (size_t)sp * kPartStride + kHeadDim));
-  float LL = 0.f, AA[kDimsPerThread];
-#pragma unroll
-  for (int x = 0; x < kDimsPerThread; ++x) AA[x] = 0.f;
-  if (MM != ninf) {
-    for (int sp = 0; sp < a.splits; ++sp) {
-      const float* src = base + (size_t)sp * kPartStride;
-      const float f = exp2f(__ldcg(src + kHeadDim) - MM);
-      LL += __ldcg(src + kHeadDim + 1) * f;
-#pragma unroll
-      for (int x = 0; x < kDimsPerThread; ++x) AA[x] += __ldcg(src + d0 + x) * f;
-    }
-  }
-  const float inv = LL > 0.f ? 1.f / LL : 0.f;
-  float* o = a.out + out_row * kHeadDim + d0;
-#pragma unroll
-  for (int x = 0; x < kDimsPerThread; x += 4)
-    *reinterpret_cast<float4*>(o + x) = make_float4(AA[x] * inv, AA[x + 1] * inv, AA[x + 2] * inv, AA[x + 3] * inv);
-  if (a.lse && d0 == 0) a.lse[out_row] = LL > 0.f ? MM * kLn2 + logf(LL) : ninf;
-}
-
-__global__ void __launch_bounds__(kDecThreads) decode_kernel(const __grid_constant__ DecodeArgs a) {
+__global__ void __launch_bounds__(kThreads) decode_kernel(const __grid_constant__ DecodeArgs a) {
   extern __shared__ unsigned char smem_raw[];
   __shared__ int s_item, s_last, s_ntiles;
-  __shared__ uint32_t s_scan[kDecWarps];
+  __shared__ uint32_t s_scan[kWarps];
   unsigned char* base = reinterpret_cast<unsigned char*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   const Smem sm{base, reinterpret_cast<uint64_t*>(base + kOffBars), reinterpret_cast<TileRef*>(base + kOffTiles),
                 reinterpret_cast<int*>(base + kOffPre), s_scan, &s_last, &s_ntiles};
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   if (lane == 0) {
-    for (int s = 0; s < kDecStages; ++s) mbar_init(sm.bars + warp * kDecStages + s, 1);
+    for (int s = 0; s < kStages; ++s) mbar_init(sm.bars + warp * kStages + s, 1);
     fence_barrier_init();
   }
   if (threadIdx.x == 0) {
@@ -437,9 +41,9 @@ __global__ void __launch_bounds__(kDecThreads) decode_kernel(const __grid_consta
     __syncthreads();
   }
   if (!ws.alive && lane == 0) {  // a wait timed out: let the copies in flight land (bounded)
-    uint64_t* bars = sm.bars + warp * kDecStages;
+    uint64_t* bars = sm.bars + warp * kStages;
     for (uint32_t g = ws.drain_lo; g < ws.drain_hi; ++g)
-      mbar_wait(bars + g % kDecStages, (g / kDecStages) & 1u, nullptr);
+      mbar_wait(bars + g % kStages, (g / kStages) & 1u, nullptr);
   }
   // the last CTA out rewinds the queue for the next launch
   if (threadIdx.x == 0) {
@@ -480,7 +84,7 @@ cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t st) {
   if (grid > items) grid = items;
   const cudaError_t e = set_smem_attr((const void*)decode_kernel, smem);
   if (e != cudaSuccess) return e;
-  decode_kernel<<<(unsigned)grid, kDecThreads, smem, st>>>(a);
+  decode_kernel<<<(unsigned)grid, kThreads, smem, st>>>(a);
   return cudaGetLastError();
 }
 

@@ -69,6 +69,7 @@ struct SelectArgs {
   uint32_t* ws_queue;         // [2] persistent-grid item queue (head, finished CTAs)
   int* status;
   int splits;
+  unsigned char* meta_refresh;  // decode step: writable metadata (same array as meta)
 };
 cudaError_t launch_select(const SelectArgs& a, cudaStream_t st);
 
@@ -92,6 +93,18 @@ struct DecodeArgs {
   int splits;
 };
 cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t st);
+
+// One decode step in one launch: newest-page metadata refresh, scoring,
+// selection and decode.  Scoring items come first in the queue; decode item j
+// of unit u waits (bounded) for u's selection flag.
+struct StepArgs {
+  SelectArgs sel;             // meta_refresh set, ws_count = unit flags [units]
+  DecodeArgs dec;             // idx/count = sel outputs, ws_count = split counters [units]
+  uint32_t* queue;            // [2] item queue (head, finished CTAs)
+  int n_score, n_dec;         // items of each kind
+};
+cudaError_t launch_step(const StepArgs& a, cudaStream_t st);
+size_t step_smem_bytes(int max_pages, int max_sel, bool chunks);
 
 struct TileAttnArgs {
   CUtensorMap tmap_k;         // K rows [Hkv*cap][128 bf16], boxes 64 x 64, 128B swizzle

@@ -4,13 +4,13 @@
 // comparison" (scoring column: per-dimension min/max upper bound, mean of
 // chunk keys).
 //
-// One warp per page; lane l owns dimensions 4l..4l+3 and walks the page's
-// tokens with 8-byte loads (a warp reads each 256-byte key row coalesced).
-// min/max are exact in bf16; the mean is accumulated in fp64 and rounded once
-// to fp32.  Only pages overlapping [t0_b, N_b) are rewritten, so appending a
-// token costs one page per (sequence, KV head).
+// One warp per page (page_meta.cuh: lane l owns dimensions 4l..4l+3; min/max
+// exact in bf16, mean summed in fp64 and rounded once to fp32).  Only pages
+// overlapping [t0_b, N_b) are rewritten, so appending a token costs one page
+// per (sequence, KV head).
 #include "common.cuh"
 #include "internal.h"
+#include "page_meta.cuh"
 
 namespace sa {
 namespace {
@@ -25,16 +25,6 @@ struct MetaParams {
   unsigned char* meta;
   int* status;
 };
-
-__device__ int chunk_containing(const int32_t* off, int n, int t) {
-  // largest c in [0, n) with off[c] <= t
-  int lo = 0, hi = n - 1;
-  while (lo < hi) {
-    const int mid = (lo + hi + 1) >> 1;
-    if (off[mid] <= t) lo = mid; else hi = mid - 1;
-  }
-  return lo;
-}
 
 template <int RULE>
 __global__ void __launch_bounds__(kMetaWarps * 32) build_meta_kernel(MetaParams p) {
@@ -86,58 +76,8 @@ __global__ void __launch_bounds__(kMetaWarps * 32) build_meta_kernel(MetaParams 
 
   const __nv_bfloat16* K = reinterpret_cast<const __nv_bfloat16*>(p.kv.k) +
                            ((size_t)u * p.kv.cap) * kHeadDim + lane * 4;
-  float mn[4], mx[4];
-  double sm[4];
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    mn[i] = __int_as_float(0x7f800000);
-    mx[i] = -__int_as_float(0x7f800000);
-    sm[i] = 0.0;
-  }
-  // 16 rows per batch, all loads issued before any is used
-  for (int t = s; t < e; t += 16) {
-    const int n = min(16, e - t);
-    uint2 r[16];
-#pragma unroll
-    for (int x = 0; x < 16; ++x)
-      r[x] = x < n ? __ldg(reinterpret_cast<const uint2*>(K + (size_t)(t + x) * kHeadDim))
-                   : make_uint2(0u, 0u);
-#pragma unroll
-    for (int x = 0; x < 16; ++x) {
-      if (x < n) {
-        const float f[4] = {bf16_lo(r[x].x), bf16_hi(r[x].x), bf16_lo(r[x].y), bf16_hi(r[x].y)};
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          if (RULE == 0) {
-            mn[i] = fminf(mn[i], f[i]);
-            mx[i] = fmaxf(mx[i], f[i]);
-          } else {
-            sm[i] += (double)f[i];
-          }
-        }
-      }
-    }
-  }
-
-  unsigned char* dst = p.meta + ((size_t)u * p.kv.max_pages + page) * kMetaBytes;
-  if (RULE == 0) {
-    // bf16 values: min/max of bf16 inputs are bf16 inputs, so the casts are exact.
-    uint2 lo, hi;
-    lo.x = pack_bf16(mn[0], mn[1]);
-    lo.y = pack_bf16(mn[2], mn[3]);
-    hi.x = pack_bf16(mx[0], mx[1]);
-    hi.y = pack_bf16(mx[2], mx[3]);
-    reinterpret_cast<uint2*>(dst)[lane] = lo;
-    reinterpret_cast<uint2*>(dst + 256)[lane] = hi;
-  } else {
-    const double inv = 1.0 / (double)(e - s);
-    float4 m;
-    m.x = (float)(sm[0] * inv);
-    m.y = (float)(sm[1] * inv);
-    m.z = (float)(sm[2] * inv);
-    m.w = (float)(sm[3] * inv);
-    reinterpret_cast<float4*>(dst)[lane] = m;
-  }
+  const PageMetaLane m = page_meta_lane<RULE>(K, s, e);
+  store_page_meta<RULE>(p.meta + ((size_t)u * p.kv.max_pages + page) * kMetaBytes, m, lane);
 }
 
 }  // namespace

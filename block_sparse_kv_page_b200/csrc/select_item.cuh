@@ -1,0 +1,383 @@
+// One work item of page scoring + budgeted top-k selection: the scoring of a
+// range of 16-page tiles of one unit (sequence, KV head), and, for the CTA
+// that finishes the unit's last range, the selection.  Called by the
+// standalone selection kernel and by the fused decode step.
+//
+// "Sparse Attention for Web Agents -- Offline Replay Records", section "The
+// comparison": each chunk is scored against the current query (envelope =
+// per-dimension min/max upper bound; centroid = mean key) and the best ones
+// are kept, the budget being page_size x top_k attended tokens; TSA fills a
+// token budget over variable chunks.  "WebArena 0-99 Sparse-Attention Method
+// Comparison", section "Method configurations at a glance": ratio budget
+// max(topk_val + bos + eos, int(blocks * ratio)) with forced bos/eos blocks.
+//
+// Scoring.  The metadata of a tile (16 pages x 512 B) arrives by TMA as four
+// 16 x 128-byte boxes, 128B-swizzled, into a per-warp mbarrier ring; lane 0
+// of each warp keeps several tiles in flight.  All G grouped query heads are
+// scored on tensor cores:
+//   envelope: S^T[16 pages x 8 heads] = [kmin | kmax] (16 x 256, bf16)
+//             x [q- | q+]^T (256 x 8, bf16), m16n8k16 via ldmatrix, exact
+//             products, fp32 accumulation;
+//   centroid: S^T = kmean (16 x 128, fp32) x q^T (128 x 8, bf16) on the FP64
+//             tensor cores (m8n8k4): exact products and sums, one rounding to
+//             fp32, so near-ties are resolved as in float64.
+// The group score (max over the G heads) goes to the workspace.  In the fused
+// step (FUSED), the warp that owns the tile holding the page of the
+// newest token (N - 1) first rebuilds that page's metadata from K, stores it
+// to the metadata array and patches the staged tile, so the step scores the
+// cache as it stands after the append.
+//
+// Selection.  The CTA that finishes a unit's last item (atomic counter;
+// nobody waits) loads the unit's scores and runs a weighted MSB-first radix
+// select on order-preserving 32-bit keys: it finds the cut key T and the
+// capacity left for keys equal to T; equal keys are then taken in ascending
+// page order (the lowest-index tie rule), so the result is exactly "the
+// longest prefix of the (score desc, index asc) order within the budget".
+// Weight 1 per page gives top-k / ratio; weight = chunk length gives the token
+// budget.  Output is the kept set in ascending page order.  In the fused step
+// the unit's counter is left at kUnitSelected (release) once the output
+// is written, for consumers in the same launch.
+#pragma once
+
+#include "common.cuh"
+#include "internal.h"
+#include "page_meta.cuh"
+#include "radix.cuh"
+
+#ifndef SA_SEL_ITEM_PAGES
+#define SA_SEL_ITEM_PAGES 512
+#endif
+#ifndef SA_SEL_STAGES
+#define SA_SEL_STAGES 2
+#endif
+#ifndef SA_SEL_CTAS_PER_SM
+#define SA_SEL_CTAS_PER_SM 3
+#endif
+
+namespace sa {
+namespace sel {
+
+constexpr int kWarps = 4;
+constexpr int kThreads = kWarps * 32;
+constexpr int kStages = SA_SEL_STAGES;
+constexpr int kTileBytes = 8192;          // 16 pages x 512 B = four 2 KiB boxes
+constexpr int kBoxBytes = 2048;
+constexpr int kRingBytes = kWarps * kStages * kTileBytes;
+constexpr uint32_t kUnitSelected = 0x80000000u;
+
+// Selection-phase shared memory: keys and weights, 4 B each per page.
+__host__ __device__ constexpr int keys_bytes(int max_pages) { return 8 * max_pages; }
+
+struct SelSmem {
+  unsigned char* ring;   // [warp][stage][kTileBytes]; reused for keys/weights in selection
+  uint64_t* bars;        // [warp][stage]
+  uint32_t* hist;        // 256
+  uint32_t* scan;        // 32
+  uint32_t* bc;          // 4
+  int* last;
+};
+
+// Selection of unit u from its scores in the workspace: writes sel_idx (ascending
+// page order) and sel_count.  All threads of the CTA call it.
+SA_DEV void select_unit(const SelectArgs& a, const int u, const int b, const int N, const int P,
+                        const SelSmem& S) {
+  const int tid = threadIdx.x;
+  uint32_t* keys = reinterpret_cast<uint32_t*>(S.ring);
+  uint32_t* wts = keys + a.kv.max_pages;
+  const float* sc_u = a.ws_scores + (size_t)u * a.kv.max_pages;
+  const bool weighted = a.budget_kind == SA_BUDGET_TOKENS;
+  const int32_t* off = weighted ? a.kv.chunk_off + (size_t)b * (a.kv.max_pages + 1) : nullptr;
+  int forced_lo = 0, forced_hi = P;  // pages < forced_lo or >= forced_hi are forced (ratio)
+  uint32_t cap;
+  if (a.budget_kind == SA_BUDGET_TOPK) {
+    cap = (uint32_t)min(a.top_k, P);
+  } else if (a.budget_kind == SA_BUDGET_RATIO) {
+    const long long fl = (long long)floor((double)P * a.ratio);
+    long long K = (long long)a.topk_val + a.bos + a.eos;
+    if (fl > K) K = fl;
+    if (K > P) K = P;
+    cap = (uint32_t)K;
+    forced_lo = min(a.bos, P);
+    forced_hi = max(0, P - a.eos);
+  } else {
+    cap = (uint32_t)max(a.token_budget, 0);
+  }
+  uint32_t wall_local = 0;
+  for (int p = tid; p < P; p += blockDim.x) {
+    const float s = __ldcg(sc_u + p);
+    uint32_t key = order_key(s);
+    if (p < forced_lo || p >= forced_hi) key = 0xffffffffu;
+    keys[p] = key;
+    if (weighted) {
+      const int L = min(off[p + 1], N) - off[p];
+      wts[p] = (uint32_t)max(L, 0);
+      wall_local += (uint32_t)max(L, 0);
+    } else {
+      wall_local += 1u;
+    }
+  }
+  uint32_t wall;
+  block_excl_scan(wall_local, S.scan, wall);  // includes a __syncthreads
+
+  int32_t* sel_u = a.sel_idx + (size_t)u * a.max_sel;
+  if (wall <= cap) {  // everything fits
+    for (int p = tid; p < P; p += blockDim.x)
+      if (p < a.max_sel) sel_u[p] = p;
+    if (tid == 0) {
+      if (P > a.max_sel) flag_status(a.status, SA_ERR_DEVICE_CHECK);
+      a.sel_count[u] = min(P, a.max_sel);
+    }
+    return;
+  }
+  const RadixCut cut = radix_cut(keys, weighted ? wts : nullptr, P, cap, S.hist, S.bc);
+
+  const int per = (P + blockDim.x - 1) / blockDim.x;
+  const int i0 = min(P, tid * per), i1 = min(P, i0 + per);
+  uint32_t eqw = 0;
+  for (int i = i0; i < i1; ++i)
+    if (keys[i] == cut.T) eqw += weighted ? wts[i] : 1u;
+  uint32_t dummy;
+  const uint32_t eq0 = block_excl_scan(eqw, S.scan, dummy);
+  uint32_t cnt = 0, eq = eq0;
+  for (int i = i0; i < i1; ++i) {
+    const uint32_t k = keys[i];
+    bool sel = k > cut.T;
+    if (k == cut.T) {
+      eq += weighted ? wts[i] : 1u;
+      sel = eq <= cut.rem;
+    }
+    cnt += sel ? 1u : 0u;
+  }
+  uint32_t total;
+  uint32_t pos = block_excl_scan(cnt, S.scan, total);
+  eq = eq0;
+  for (int i = i0; i < i1; ++i) {
+    const uint32_t k = keys[i];
+    bool sel = k > cut.T;
+    if (k == cut.T) {
+      eq += weighted ? wts[i] : 1u;
+      sel = eq <= cut.rem;
+    }
+    if (sel) {
+      if (pos < (uint32_t)a.max_sel) sel_u[pos] = i;
+      ++pos;
+    }
+  }
+  if (tid == 0) {
+    if (total > (uint32_t)a.max_sel) flag_status(a.status, SA_ERR_DEVICE_CHECK);
+    a.sel_count[u] = (int32_t)min(total, (uint32_t)a.max_sel);
+  }
+}
+
+// FUSED (the decode step): refresh the newest page while scoring and publish
+// the unit's flag after selecting.
+template <int RULE, bool FUSED>
+SA_DEV void select_item(const SelectArgs& a, const int u, const int split, const SelSmem& S,
+                        WarpState& ws) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int gq = lane >> 2, c = lane & 3;
+  const int Hkv = a.kv.Hkv;
+  const int b = u / Hkv, g = u % Hkv;
+
+  // ---- unit geometry (every CTA of the unit computes the same values)
+  const int N = a.kv.seq_len[b];
+  int P;
+  bool bad = (N < 1 || N > a.kv.cap);
+  if (a.kv.page_size > 0) {
+    P = bad ? 0 : (N + a.kv.page_size - 1) / a.kv.page_size;
+  } else {
+    P = a.kv.n_chunks[b];
+    bad = bad || P < 1;
+  }
+  if (P > a.kv.max_pages) bad = true;
+  if (bad) {
+    P = 0;
+    if (tid == 0 && split == 0) flag_status(a.status, SA_ERR_DEVICE_CHECK);
+  }
+  const int TP = (P + 15) >> 4;
+  const int t_begin = (int)(((long long)TP * split) / a.splits);
+  const int t_end = (int)(((long long)TP * (split + 1)) / a.splits);
+
+  // ---- B fragments: the G query heads of this KV group (columns >= G are zero)
+  const bool head_ok = gq < a.G;
+  const __nv_bfloat16* qrow = reinterpret_cast<const __nv_bfloat16*>(a.q) +
+                              ((size_t)b * a.Hq + (size_t)g * a.G + (head_ok ? gq : 0)) * kHeadDim;
+  uint32_t bq[RULE == 0 ? 32 : 1];
+  double bd[RULE == 0 ? 1 : 32];
+  if (RULE == 0) {
+    // k-step ks covers row elements 16ks .. 16ks + 15 of [kmin | kmax];
+    // the paired query vector is [q- | q+] (natural order)
+#pragma unroll
+    for (int ks = 0; ks < 16; ++ks) {
+      const int e = 16 * (ks & 7) + 2 * c;
+      uint32_t lo = head_ok ? __ldg(reinterpret_cast<const uint32_t*>(qrow + e)) : 0u;
+      uint32_t hi = head_ok ? __ldg(reinterpret_cast<const uint32_t*>(qrow + e + 8)) : 0u;
+      if (ks < 8) { lo = bf16x2_neg_part(lo); hi = bf16x2_neg_part(hi); }
+      else        { lo = bf16x2_pos_part(lo); hi = bf16x2_pos_part(hi); }
+      bq[2 * ks] = lo;
+      bq[2 * ks + 1] = hi;
+    }
+  } else {
+    // k-step (box bx, chunk j): lane c holds dimension 32 bx + 4 j + c
+#pragma unroll
+    for (int bx = 0; bx < 4; ++bx)
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const int e = 32 * bx + 4 * j + c;
+        bd[8 * bx + j] = head_ok ? (double)__bfloat162float(qrow[e]) : 0.0;
+      }
+  }
+
+  // ---- scoring: warp w takes tiles t_begin + w, + 4, ...
+  float* sc_u = a.ws_scores + (size_t)u * a.kv.max_pages;
+  float* out_u = a.scores_out ? a.scores_out + (size_t)u * a.kv.max_pages : nullptr;
+  unsigned char* ring = S.ring + warp * (kStages * kTileBytes);
+  uint64_t* bars = S.bars + warp * kStages;
+  const int row_base = u * a.kv.max_pages;
+  const int lrow = (lane & 7) + 8 * ((lane >> 3) & 1);  // ldmatrix: rows 0-7 / 8-15
+  const int lchk = lane >> 4;                            //            chunk +0 / +1
+  const int nt = t_end - t_begin;
+  const int n_it = max(0, (nt - warp + kWarps - 1) / kWarps);
+
+  auto issue = [&](int it) {  // lane 0 only
+    const uint32_t g_it = ws.gi + (uint32_t)it;
+    uint64_t* bar = bars + g_it % kStages;
+    unsigned char* st = ring + (g_it % kStages) * kTileBytes;
+    const int y = row_base + 16 * (t_begin + warp + it * kWarps);
+    mbar_arrive_expect_tx(bar, kTileBytes);
+    const int xs = RULE == 0 ? 64 : 32;  // elements per 128-byte box row
+#pragma unroll
+    for (int bx = 0; bx < 4; ++bx) tma_load_2d(st + bx * kBoxBytes, &a.tmap_meta, bx * xs, y, bar);
+  };
+
+  int issued = 0;
+  if (ws.alive) {
+    issued = min(n_it, kStages - 1);
+    if (lane == 0)
+      for (int it = 0; it < issued; ++it) issue(it);
+  }
+
+  // ---- page of the newest token, when this call refreshes it: rows [r_s, r_e)
+  int p_new = -1, r_s = 0, r_e = 0;
+  if (FUSED && P > 0) {
+    if (a.kv.page_size > 0) {
+      p_new = P - 1;
+      r_s = p_new * a.kv.page_size;
+      r_e = min(r_s + a.kv.page_size, N);
+    } else {
+      const int32_t* off = a.kv.chunk_off + (size_t)b * (a.kv.max_pages + 1);
+      p_new = off[P - 1] <= N - 1 ? P - 1 : chunk_containing(off, P, N - 1);
+      r_s = off[p_new];
+      const int e_raw = off[p_new + 1];
+      if (r_s < 0 || e_raw < r_s) {
+        if (tid == 0 && split == 0) flag_status(a.status, SA_ERR_DEVICE_CHECK);
+        p_new = -1;
+      } else {
+        r_e = min(e_raw, N);  // a chunk table may run ahead of the cache: clip to N
+        if (r_s >= r_e) p_new = -1;
+      }
+    }
+  }
+  const int t_new = p_new >= 0 ? (p_new >> 4) : -1;
+
+  for (int it = 0; it < n_it && ws.alive; ++it) {
+    __syncwarp();
+    if (it + kStages - 1 < n_it) {
+      if (lane == 0) issue(it + kStages - 1);
+      issued = it + kStages;
+    }
+    const uint32_t g_it = ws.gi + (uint32_t)it;
+    if (!mbar_wait(bars + g_it % kStages, (g_it / kStages) & 1u, a.status)) {
+      ws.alive = false;
+      ws.drain_lo = g_it;
+      ws.drain_hi = ws.gi + (uint32_t)issued;
+      break;
+    }
+    unsigned char* st = ring + (g_it % kStages) * kTileBytes;
+    const int t = t_begin + warp + it * kWarps;
+    if (t == t_new) {
+      // rebuild the newest page's metadata, store it, patch the staged row
+      const __nv_bfloat16* k_lane = reinterpret_cast<const __nv_bfloat16*>(a.kv.k) +
+                                    ((size_t)u * a.kv.cap) * kHeadDim + lane * 4;
+      const PageMetaLane m = page_meta_lane<RULE>(k_lane, r_s, r_e);
+      store_page_meta<RULE>(a.meta_refresh + ((size_t)u * a.kv.max_pages + p_new) * kMetaBytes, m, lane);
+      const int r = p_new & 15;
+      if (RULE == 0) {
+        const uint32_t o = swz128(r, (lane & 15) >> 1) + 8 * (lane & 1);
+        *reinterpret_cast<uint2*>(st + (lane >> 4) * kBoxBytes + o) = m.lo;
+        *reinterpret_cast<uint2*>(st + (2 + (lane >> 4)) * kBoxBytes + o) = m.hi;
+      } else {
+        *reinterpret_cast<float4*>(st + (lane >> 3) * kBoxBytes + swz128(r, lane & 7)) = m.mean;
+      }
+      fence_proxy_async();  // generic writes to the stage before its next TMA refill
+      __syncwarp();
+    }
+    float acc[4];
+    if (RULE == 0) {
+      float s0[4] = {0.f, 0.f, 0.f, 0.f}, s1[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int ks = 0; ks < 16; ++ks) {
+        uint32_t a0, a1, a2, a3;
+        ldsm_x4(a0, a1, a2, a3, st + (ks >> 2) * kBoxBytes + swz128(lrow, 2 * (ks & 3) + lchk));
+        if (ks & 1) mma_bf16(s1, a0, a1, a2, a3, bq[2 * ks], bq[2 * ks + 1]);
+        else        mma_bf16(s0, a0, a1, a2, a3, bq[2 * ks], bq[2 * ks + 1]);
+      }
+#pragma unroll
+      for (int x = 0; x < 4; ++x) acc[x] = s0[x] + s1[x];
+    } else {
+      // FP64 tensor cores: exact products and sums, one final rounding
+      double c00 = 0.0, c01 = 0.0, c10 = 0.0, c11 = 0.0;  // pages gq / gq + 8
+#pragma unroll
+      for (int bx = 0; bx < 4; ++bx)
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const float x0 = *reinterpret_cast<const float*>(st + bx * kBoxBytes + swz128(gq, j) + 4 * c);
+          const float x1 = *reinterpret_cast<const float*>(st + bx * kBoxBytes + swz128(gq + 8, j) + 4 * c);
+          const double bv = bd[8 * bx + j];
+          mma_f64(c00, c01, (double)x0, bv);
+          mma_f64(c10, c11, (double)x1, bv);
+        }
+      acc[0] = (float)c00; acc[1] = (float)c01; acc[2] = (float)c10; acc[3] = (float)c11;
+    }
+    const float ninf = -__int_as_float(0x7f800000);
+    const bool c0 = 2 * c < a.G, c1 = 2 * c + 1 < a.G;
+    float mlo = fmaxf(c0 ? acc[0] : ninf, c1 ? acc[1] : ninf);
+    float mhi = fmaxf(c0 ? acc[2] : ninf, c1 ? acc[3] : ninf);
+    mlo = fmaxf(mlo, __shfl_xor_sync(0xffffffffu, mlo, 1));
+    mlo = fmaxf(mlo, __shfl_xor_sync(0xffffffffu, mlo, 2));
+    mhi = fmaxf(mhi, __shfl_xor_sync(0xffffffffu, mhi, 1));
+    mhi = fmaxf(mhi, __shfl_xor_sync(0xffffffffu, mhi, 2));
+    if (c < 2) {
+      const int page = t * 16 + gq + 8 * c;
+      const float s = c == 0 ? mlo : mhi;
+      if (page < P) {
+        sc_u[page] = s;
+        if (out_u) out_u[page] = s;
+      }
+    }
+  }
+  ws.gi += (uint32_t)n_it;
+
+  // ---- the last CTA of the unit selects
+  __syncthreads();
+  if (a.splits > 1) {
+    __threadfence();
+    if (tid == 0) {
+      const uint32_t prev = atomicAdd(&a.ws_count[u], 1u);
+      *S.last = (prev == (uint32_t)(a.splits - 1));
+    }
+    __syncthreads();
+    if (!*S.last) return;
+    __threadfence();
+  }
+  if (tid == 0 && a.splits > 1 && !FUSED) a.ws_count[u] = 0;  // ready for the next call
+  select_unit(a, u, b, N, P, S);
+  if (FUSED) {
+    __threadfence();
+    __syncthreads();
+    if (tid == 0) st_release_u32(&a.ws_count[u], kUnitSelected);
+  }
+}
+
+}  // namespace sel
+}  // namespace sa

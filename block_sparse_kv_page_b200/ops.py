@@ -144,6 +144,22 @@ def sparse_attn_decode(kv: KvCache, q: torch.Tensor, n_q_rows: int, q_pos0: int,
            "sparse_attn_decode")
 
 
+def sparse_attn_decode_step(kv: KvCache, meta: torch.Tensor, rule, q: torch.Tensor, budget: sa_budget,
+                            max_sel: int, scale: float, sel_idx: torch.Tensor, sel_count: torch.Tensor,
+                            out: torch.Tensor, lse: torch.Tensor | None, ws: torch.Tensor,
+                            stream=None) -> None:
+    if q.dtype != torch.bfloat16 or not q.is_contiguous():
+        raise ValueError("q must be contiguous bf16 [B, Hq, 128]")
+    if out.dtype != torch.float32 or not out.is_contiguous():
+        raise ValueError("out must be contiguous fp32")
+    _check(lib.sparse_attn_decode_step(C.byref(kv.desc), meta.data_ptr(), _rule(rule), q.data_ptr(),
+                                       q.shape[-2], C.byref(budget), int(max_sel), float(scale),
+                                       sel_idx.data_ptr(), sel_count.data_ptr(), out.data_ptr(),
+                                       _ptr(lse), ws.data_ptr(), ws.numel() * ws.element_size(),
+                                       _stream(stream)),
+           "sparse_attn_decode_step")
+
+
 def sparse_attn_decode_static(kv: KvCache, q: torch.Tensor, n_q_rows: int, q_pos0: int,
                               tile_rows: int, scale: float, idx: torch.Tensor, count: torch.Tensor,
                               max_sel: int, out: torch.Tensor, lse: torch.Tensor | None,

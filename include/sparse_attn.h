@@ -69,7 +69,7 @@ typedef enum {
   SA_ERR_UNSUPPORTED = 2,   /* legal but not implemented (head_dim != 128, G > 8, ...) */
   SA_ERR_WORKSPACE = 3,     /* ws is null, misaligned or smaller than required */
   SA_ERR_CUDA = 4,          /* a CUDA runtime call or kernel launch failed */
-  SA_ERR_TIMEOUT = 5,       /* reserved: a bounded device-side wait gave up */
+  SA_ERR_TIMEOUT = 5,       /* a bounded device-side wait gave up (re-init the workspace) */
   SA_ERR_DEVICE_CHECK = 6   /* a device-side range check failed (entry skipped) */
 } sa_status;
 
@@ -169,6 +169,29 @@ sa_status sparse_attn_decode(const sa_kv_desc* kv, const void* q, int32_t n_q_he
                              int32_t n_q_rows, int32_t q_pos0, int32_t tile_rows, float scale,
                              const int32_t* idx, const int32_t* count, int32_t max_sel,
                              float* out, float* lse, void* ws, size_t ws_bytes, void* stream);
+
+/* (e) One whole decode step in one launch ([OFFLINE] "The comparison": after
+ * the new token's key is in the cache, score the chunks against the current
+ * query, keep the best ones under the budget and attend only to them).
+ * Computes exactly what this sequence computes, with the same arguments:
+ *   sparse_attn_build_meta(kv, rule, -1, meta);          refresh the newest page
+ *   sparse_attn_select(kv, meta, rule, q, n_q_heads, budget, max_sel,
+ *                      sel_idx, sel_count, NULL, ...);
+ *   sparse_attn_decode(kv, q, n_q_heads, B, 0, 1, scale, sel_idx, sel_count,
+ *                      max_sel, out, lse, ...);
+ * meta is read and written (the metadata of the page or chunk holding token
+ * N_b - 1 is rebuilt from K; every other page must be current).  sel_idx and
+ * sel_count are written as by sparse_attn_select.  Work items of the three
+ * stages share one persistent grid: the decode of a (sequence, KV head) starts
+ * as soon as its selection is written, while other units are still being
+ * scored; a decode item waits for its selection with a bounded wait (about a
+ * second; SA_ERR_TIMEOUT when it runs out).  Needs B * n_kv_heads <= 32768 and
+ * the workspace sized by sparse_attn_workspace_size. */
+sa_status sparse_attn_decode_step(const sa_kv_desc* kv, void* meta, sa_score_rule rule,
+                                  const void* q, int32_t n_q_heads, const sa_budget* budget,
+                                  int32_t max_sel, float scale, int32_t* sel_idx,
+                                  int32_t* sel_count, float* out, float* lse, void* ws,
+                                  size_t ws_bytes, void* stream);
 
 /* (d) Uncertainty router over query tiles ([ROUTER] "Methodologie" steps 2-5).
  * B == 1, fixed blocks (page_size = block size).  q bf16 [n_q_rows][n_q_heads][128]

@@ -110,6 +110,28 @@ def test_decode_validation(lib, abi):
     assert call(desc=_desc(abi, head_dim=256)) == abi.SA_ERR_UNSUPPORTED
 
 
+def test_decode_step_validation(lib, abi):
+    ok = _desc(abi)
+    topk = abi.sa_budget(abi.SA_BUDGET_TOPK, 8, 0.0, 0, 0, 0, 0)
+
+    def call(desc=ok, hq=32, budget=topk, max_sel=16, scale=0.088, meta=0x40000, out=0x80000,
+             ws=0x100000, ws_bytes=1 << 30):
+        return lib.sparse_attn_decode_step(C.byref(desc), meta, 0, 0x50000, hq, C.byref(budget),
+                                           max_sel, scale, 0x60000, 0x70000, out, None, ws,
+                                           ws_bytes, None)
+    assert call(meta=0) == abi.SA_ERR_INVALID
+    assert call(meta=0x40008) == abi.SA_ERR_INVALID       # metadata not 16-byte aligned
+    assert call(max_sel=4) == abi.SA_ERR_INVALID          # top_k > max_sel
+    assert call(out=0x80004) == abi.SA_ERR_INVALID
+    assert call(scale=float("inf")) == abi.SA_ERR_INVALID
+    assert call(hq=64) == abi.SA_ERR_UNSUPPORTED          # G = 16
+    assert call(ws_bytes=4096) == abi.SA_ERR_WORKSPACE
+    assert call(ws=0x100010) == abi.SA_ERR_WORKSPACE
+    assert call(desc=_desc(abi, batch=8193)) == abi.SA_ERR_UNSUPPORTED  # 2 x units > 65536
+    tokens = abi.sa_budget(abi.SA_BUDGET_TOKENS, 0, 0.0, 0, 0, 0, 512)
+    assert call(budget=tokens) == abi.SA_ERR_UNSUPPORTED  # token budgets need chunks
+
+
 def test_build_meta_validation(lib, abi):
     ok = _desc(abi)
     assert lib.sparse_attn_build_meta(C.byref(ok), 7, 0, 0x40000, None) == abi.SA_ERR_INVALID

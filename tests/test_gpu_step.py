@@ -1,0 +1,157 @@
+"""GPU parity of the one-launch decode step (sparse_attn_decode_step): newest
+page metadata refresh + scoring + budgeted top-k + split-K attention in one
+persistent launch.
+
+Each case checks the step two ways:
+* against the float64 oracle on every unit (metadata of every page, the
+  selected set under the near-tie certificate, attention over the kept
+  tokens), after building the metadata for the cache as it stood BEFORE its
+  newest token, so only the step's own refresh makes it current;
+* against the separate calls (build_meta, select, decode) on the same
+  inputs: the page sets, outputs and log-sum-exps must be bit-identical,
+  since the step runs the same item code with the same splits.
+
+Cases span fixed pages of 16 and 64 tokens, G = 7 and 8, ratio budgets with
+forced pages, TSA chunks with a token budget, newest tokens that open a new
+page, one-token caches, and hundreds of units.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import datagen as DG
+
+pytestmark = pytest.mark.gpu
+
+SCALE = 1.0 / math.sqrt(128)
+
+
+@pytest.fixture(scope="module")
+def R():
+    import gpu_runner
+    return gpu_runner
+
+
+def _case(dev, name):
+    """(layer, page_size, budget) of a named case."""
+    if name == "ps16_topk":
+        lay = DG.make_decode_layer(B=2, Hq=32, Hkv=4, seq_lens=[1000, 777], seed=301, device=dev,
+                                   cap=1024, key_scale="channel")
+        return lay, 16, {"kind": "topk", "k": 24}
+    if name == "ps16_new_page":
+        # the newest token opens page 64, page 1 and page 0 respectively
+        lay = DG.make_decode_layer(B=3, Hq=32, Hkv=4, seq_lens=[1025, 17, 1], seed=302, device=dev,
+                                   cap=1040)
+        return lay, 16, {"kind": "topk", "k": 8}
+    if name == "ps64_g7":
+        lay = DG.make_decode_layer(B=2, Hq=28, Hkv=4, seq_lens=[3000, 2100], seed=303, device=dev,
+                                   cap=3008)
+        return lay, 64, {"kind": "topk", "k": 6}
+    if name == "ratio_bos_eos":
+        lay = DG.make_decode_layer(B=3, Hq=64, Hkv=8, seq_lens=[2048, 1999, 40], seed=304, device=dev)
+        return lay, 16, {"kind": "ratio", "ratio": 0.0625, "bos": 1, "eos": 1}
+    if name == "chunks_tokens":
+        lens = DG.workload3_chunks(2, 3000, seed_offset=3)
+        lens[1] = DG.chunk_lengths(np.random.default_rng(6), 1234)
+        lay = DG.make_decode_layer(B=2, Hq=32, Hkv=4, seq_lens=[3000, 1234], seed=305, device=dev,
+                                   cap=3000, chunk_lens=lens, chunk_offset_std=0.5)
+        return lay, 0, {"kind": "tokens", "budget": 1024}
+    if name == "many_units":
+        rng = np.random.default_rng(7)
+        lens = [int(x) for x in rng.integers(1, 2048, size=64)]
+        lay = DG.make_decode_layer(B=64, Hq=16, Hkv=8, seq_lens=lens, seed=306, device=dev, cap=2048)
+        return lay, 16, {"kind": "topk", "k": 16}
+    raise KeyError(name)
+
+
+CASES = ["ps16_topk", "ps16_new_page", "ps64_g7", "ratio_bos_eos", "chunks_tokens", "many_units"]
+
+
+def _pages(lay, b, ps):
+    N = int(lay.seq_len[b])
+    return -(-N // ps) if ps else int(lay.n_chunks[b])
+
+
+def _assert_same(s, c, lay, ps, where):
+    for key in ("sel_idx", "sel_count", "out", "lse"):
+        a, b = s[key], c[key]
+        assert torch.equal(torch.nan_to_num(a, nan=7.0), torch.nan_to_num(b, nan=7.0)), f"{where}: {key}"
+    for b in range(lay.k.shape[0]):
+        P = _pages(lay, b, ps)
+        assert torch.equal(s["meta"][b, :, :P], c["meta"][b, :, :P]), f"{where}: meta of sequence {b}"
+
+
+@pytest.mark.parametrize("rule", ["envelope", "centroid"])
+@pytest.mark.parametrize("name", CASES)
+def test_step_parity(cuda_dev, R, rule, name):
+    if name == "chunks_tokens" and rule == "centroid":
+        pytest.skip("token budgets are run with envelope scoring (TSA)")
+    lay, ps, bd = _case(cuda_dev, name)
+    s = R.run_step(lay, page_size=ps, rule=rule, budget=bd, scale=SCALE, stale=True)
+    assert s["status"] == 0
+    st = R.check_layer(lay, s, page_size=ps, rule=rule, budget=bd, scale=SCALE)
+    assert st["units"] == lay.k.shape[0] * lay.k.shape[1]
+    assert st["max_out_err"] < 1e-4
+    c = R.run_gpu(lay, page_size=ps, rule=rule, budget=bd, scale=SCALE)
+    assert c["status"] == 0
+    _assert_same(s, c, lay, ps, f"{name}/{rule}")
+
+
+def test_step_repeat_and_interleave(cuda_dev, R):
+    """Calls in a row on one workspace: the step leaves its flags, counters
+    and queue cleared, also around the other calls."""
+    import block_sparse_kv_page_b200 as sa
+    lay, ps, bd = _case(cuda_dev, "ps16_topk")
+    s = R.run_step(lay, page_size=ps, rule="envelope", budget=bd, scale=SCALE, repeat=3)
+    assert s["status"] == 0
+    for r in s["runs"][1:]:
+        for key in ("sel_idx", "sel_count", "out", "lse"):
+            assert torch.equal(r[key], s["runs"][0][key]), key
+    # the same workspace through select + decode, then the step again
+    c = R.run_gpu(lay, page_size=ps, rule="envelope", budget=bd, scale=SCALE, ws=s["ws"])
+    assert c["status"] == 0
+    again = R.run_step(lay, page_size=ps, rule="envelope", budget=bd, scale=SCALE, ws=s["ws"])
+    assert again["status"] == 0
+    _assert_same(again, c, lay, ps, "after interleave")
+    assert sa.sparse_attn_get_device_status(s["ws"]) == 0
+
+
+def test_step_refresh_matches_build(cuda_dev, R):
+    """The metadata the step leaves behind equals a full build of the grown
+    cache (every page, both rules, pages and chunks)."""
+    import block_sparse_kv_page_b200 as sa
+    for name in ("ps16_new_page", "ps64_g7", "chunks_tokens"):
+        lay, ps, bd = _case(cuda_dev, name)
+        for rule in ("envelope", "centroid"):
+            s = R.run_step(lay, page_size=ps, rule=rule, budget=bd, scale=SCALE)
+            full = s["kv"].meta_buffer().fill_(0x5A)
+            sa.sparse_attn_build_meta(s["kv"], rule, 0, full)
+            torch.cuda.synchronize()
+            for b in range(lay.k.shape[0]):
+                P = _pages(lay, b, ps)
+                assert torch.equal(s["meta"][b, :, :P], full[b, :, :P]), f"{name}/{rule}/b{b}"
+
+
+def test_step_rejects_bad_arguments(cuda_dev, R):
+    import block_sparse_kv_page_b200 as sa
+    lay, ps, bd = _case(cuda_dev, "ps16_topk")
+    kv = sa.KvCache(lay.k, lay.v, lay.seq_len, page_size=16, max_pages=64)
+    meta = kv.meta_buffer()
+    ws = sa.make_workspace(kv, 32, 2, 24)
+    sel = torch.empty((2, 4, 24), dtype=torch.int32, device=cuda_dev)
+    cnt = torch.empty((2, 4), dtype=torch.int32, device=cuda_dev)
+    out = torch.empty((2, 32, 128), dtype=torch.float32, device=cuda_dev)
+    with pytest.raises(sa.SparseAttnError) as e:  # budget above max_sel
+        sa.sparse_attn_decode_step(kv, meta, "envelope", lay.q, sa.budget_topk(25), 24, SCALE,
+                                   sel, cnt, out, None, ws)
+    assert e.value.status == sa.SA_ERR_INVALID
+    with pytest.raises(sa.SparseAttnError) as e:  # workspace too small
+        sa.sparse_attn_decode_step(kv, meta, "envelope", lay.q, sa.budget_topk(24), 24, SCALE,
+                                   sel, cnt, out, None, ws[:1024])
+    assert e.value.status == sa.SA_ERR_WORKSPACE
+    with pytest.raises(sa.SparseAttnError) as e:  # non-finite scale
+        sa.sparse_attn_decode_step(kv, meta, "envelope", lay.q, sa.budget_topk(24), 24, float("nan"),
+                                   sel, cnt, out, None, ws)
+    assert e.value.status == sa.SA_ERR_INVALID
