@@ -103,13 +103,17 @@ int max_tiles_per_unit(const sa_kv_desc* kv, int max_sel) {
   return t > 0x3fffffff ? 0x3fffffff : (int)t;
 }
 
+// Group scores, one row of max_pages rounded up to 4 floats per unit, so the
+// selecting CTA can read a row with 16-byte loads.
+int score_stride(const sa_kv_desc* kv) { return (kv->max_pages + 3) & ~3; }
+
 size_t select_scratch(const sa_kv_desc* kv) {
-  return align256((size_t)kv->batch * kv->n_kv_heads * kv->max_pages * sizeof(float));
+  return align256((size_t)kv->batch * kv->n_kv_heads * score_stride(kv) * sizeof(float));
 }
 
 size_t decode_scratch(int units, int splits) {
   if (splits <= 1) return 0;
-  return align256((size_t)units * splits * kMaxGroup * (kHeadDim + 2) * sizeof(float));
+  return align256((size_t)units * splits * kMaxGroup * (kHeadDim + 4) * sizeof(float));
 }
 
 }  // namespace
@@ -301,6 +305,7 @@ bool fill_select(SelectArgs* a, const sa_kv_desc* kv, const void* meta, sa_score
   a->sel_count = sel_count;
   a->scores_out = scores_out;
   a->ws_scores = reinterpret_cast<float*>(reinterpret_cast<char*>(ws) + kScratch);
+  a->ws_stride = score_stride(kv);
   a->ws_count = reinterpret_cast<uint32_t*>(reinterpret_cast<char*>(ws) + 256);
   a->ws_queue = nullptr;
   a->status = reinterpret_cast<int*>(ws);

@@ -11,7 +11,7 @@ namespace {
 
 using namespace dec;
 
-__global__ void __launch_bounds__(kThreads) decode_kernel(const __grid_constant__ DecodeArgs a) {
+__global__ void __launch_bounds__(kThreads, SA_DEC_CTAS_PER_SM) decode_kernel(const __grid_constant__ DecodeArgs a) {
   extern __shared__ unsigned char smem_raw[];
   __shared__ int s_item, s_last, s_ntiles;
   __shared__ uint32_t s_scan[kWarps];

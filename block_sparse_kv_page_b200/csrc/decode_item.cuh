@@ -58,7 +58,9 @@ constexpr int kTileBytes = 8192;                 // K box lo | K box hi | V box 
 constexpr int kBoxBytes = 2048;                  // 16 rows x 128 B
 constexpr int kRingBytes = kWarps * kStages * kTileBytes;
 constexpr int kMaxItemTiles = SA_DEC_ITEM_TILES; // tile refs resolved per round
-constexpr int kPartStride = kMaxGroup * (kHeadDim + 2);  // floats per partial slot
+constexpr int kPartHead = kHeadDim + 4;            // acc[128], m, l, 2 pad: 16-byte rows
+constexpr int kPartStride = kMaxGroup * kPartHead;  // floats per partial slot
+constexpr int kMergeBatch = 4;                     // split partials loaded per round trip
 constexpr int kThreadsPerHead = kThreads / kMaxGroup;  // merge: threads per head
 constexpr int kDimsPerThread = kHeadDim / kThreadsPerHead;
 static_assert(kDimsPerThread % 4 == 0, "merge writes float4");
@@ -364,10 +366,11 @@ SA_DEV void decode_item(const DecodeArgs& a, const int u, const int split, const
   // ---- several splits: publish the partial; the last CTA of the unit merges
   float* part = a.ws_part + ((size_t)u * a.splits + split) * kPartStride;
   if (h < G) {
-    float* dst = part + h * (kHeadDim + 2);
+    float* dst = part + h * kPartHead;
 #pragma unroll
-    for (int x = 0; x < kDimsPerThread; ++x) dst[d0 + x] = A[x];
-    if (d0 == 0) { dst[kHeadDim] = M; dst[kHeadDim + 1] = L; }
+    for (int x = 0; x < kDimsPerThread; x += 4)
+      *reinterpret_cast<float4*>(dst + d0 + x) = make_float4(A[x], A[x + 1], A[x + 2], A[x + 3]);
+    if (d0 == 0) *reinterpret_cast<float2*>(dst + kHeadDim) = make_float2(M, L);
   }
   __threadfence();
   __syncthreads();
@@ -381,20 +384,46 @@ SA_DEV void decode_item(const DecodeArgs& a, const int u, const int split, const
   if (tid == 0) a.ws_count[u] = 0;
   if (h >= G) return;
 
-  const float* base = a.ws_part + (size_t)u * a.splits * kPartStride + h * (kHeadDim + 2);
-  float MM = ninf;
-  for (int sp = 0; sp < a.splits; ++sp) MM = fmaxf(MM, __ldcg(base + (size_t)sp * kPartStride + kHeadDim));
-  float LL = 0.f, AA[kDimsPerThread];
+  // Merge in split order, kMergeBatch partials per batch with every load of a
+  // batch issued before any is used (each dependent round trip to L2 costs
+  // about a microsecond under full HBM load).
+  const float* base = a.ws_part + (size_t)u * a.splits * kPartStride + h * kPartHead;
+  float MM = ninf, LL = 0.f, AA[kDimsPerThread];
 #pragma unroll
   for (int x = 0; x < kDimsPerThread; ++x) AA[x] = 0.f;
-  if (MM != ninf) {
-    for (int sp = 0; sp < a.splits; ++sp) {
-      const float* src = base + (size_t)sp * kPartStride;
-      const float f = exp2f(__ldcg(src + kHeadDim) - MM);
-      LL += __ldcg(src + kHeadDim + 1) * f;
+  for (int sp0 = 0; sp0 < a.splits; sp0 += kMergeBatch) {
+    float2 ml[kMergeBatch];
+    float4 v[kMergeBatch][kDimsPerThread / 4];
 #pragma unroll
-      for (int x = 0; x < kDimsPerThread; ++x) AA[x] += __ldcg(src + d0 + x) * f;
+    for (int j = 0; j < kMergeBatch; ++j) {
+      const bool ok = sp0 + j < a.splits;
+      const float* src = base + (size_t)(ok ? sp0 + j : 0) * kPartStride;
+      ml[j] = ok ? __ldcg(reinterpret_cast<const float2*>(src + kHeadDim)) : make_float2(ninf, 0.f);
+#pragma unroll
+      for (int q4 = 0; q4 < kDimsPerThread / 4; ++q4)
+        v[j][q4] = ok ? __ldcg(reinterpret_cast<const float4*>(src + d0) + q4) : make_float4(0.f, 0.f, 0.f, 0.f);
     }
+    float nm = MM;
+#pragma unroll
+    for (int j = 0; j < kMergeBatch; ++j) nm = fmaxf(nm, ml[j].x);
+    if (nm == ninf) continue;
+    const float fo = exp2f(MM - nm);  // 0 while nothing has been merged
+    LL *= fo;
+#pragma unroll
+    for (int x = 0; x < kDimsPerThread; ++x) AA[x] *= fo;
+#pragma unroll
+    for (int j = 0; j < kMergeBatch; ++j) {
+      const float f = exp2f(ml[j].x - nm);
+      LL += ml[j].y * f;
+#pragma unroll
+      for (int q4 = 0; q4 < kDimsPerThread / 4; ++q4) {
+        AA[4 * q4 + 0] += v[j][q4].x * f;
+        AA[4 * q4 + 1] += v[j][q4].y * f;
+        AA[4 * q4 + 2] += v[j][q4].z * f;
+        AA[4 * q4 + 3] += v[j][q4].w * f;
+      }
+    }
+    MM = nm;
   }
   const float inv = LL > 0.f ? 1.f / LL : 0.f;
   float* o = a.out + out_row * kHeadDim + d0;

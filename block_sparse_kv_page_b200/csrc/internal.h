@@ -64,7 +64,8 @@ struct SelectArgs {
   int32_t* sel_idx;
   int32_t* sel_count;
   float* scores_out;
-  float* ws_scores;
+  float* ws_scores;           // [units][ws_stride] group scores
+  int ws_stride;              // max_pages rounded up to a multiple of 4 (16-byte rows)
   uint32_t* ws_count;
   uint32_t* ws_queue;         // [2] persistent-grid item queue (head, finished CTAs)
   int* status;

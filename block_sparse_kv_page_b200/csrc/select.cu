@@ -12,11 +12,11 @@ namespace {
 using namespace sel;
 
 template <int RULE>
-__global__ void __launch_bounds__(kThreads) select_kernel(const __grid_constant__ SelectArgs a) {
+__global__ void __launch_bounds__(kThreads, SA_SEL_CTAS_PER_SM) select_kernel(const __grid_constant__ SelectArgs a) {
   extern __shared__ unsigned char smem_raw[];
-  __shared__ uint32_t s_hist[256];
+  __shared__ uint32_t s_hist[512];
   __shared__ uint32_t s_scan[32];
-  __shared__ uint32_t s_bc[4];
+  __shared__ uint32_t s_bc[8];
   __shared__ int s_last, s_item;
   unsigned char* base = reinterpret_cast<unsigned char*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));

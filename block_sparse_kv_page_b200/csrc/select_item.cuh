@@ -53,17 +53,21 @@
 #ifndef SA_SEL_CTAS_PER_SM
 #define SA_SEL_CTAS_PER_SM 3
 #endif
+#ifndef SA_SEL_WARPS
+#define SA_SEL_WARPS 4
+#endif
 
 namespace sa {
 namespace sel {
 
-constexpr int kWarps = 4;
+constexpr int kWarps = SA_SEL_WARPS;
 constexpr int kThreads = kWarps * 32;
 constexpr int kStages = SA_SEL_STAGES;
 constexpr int kTileBytes = 8192;          // 16 pages x 512 B = four 2 KiB boxes
 constexpr int kBoxBytes = 2048;
 constexpr int kRingBytes = kWarps * kStages * kTileBytes;
 constexpr uint32_t kUnitSelected = 0x80000000u;
+constexpr int kSelBatch = 4;              // 16-byte score loads in flight per thread
 
 // Selection-phase shared memory: keys and weights, 4 B each per page.
 __host__ __device__ constexpr int keys_bytes(int max_pages) { return 8 * max_pages; }
@@ -71,49 +75,58 @@ __host__ __device__ constexpr int keys_bytes(int max_pages) { return 8 * max_pag
 struct SelSmem {
   unsigned char* ring;   // [warp][stage][kTileBytes]; reused for keys/weights in selection
   uint64_t* bars;        // [warp][stage]
-  uint32_t* hist;        // 256
+  uint32_t* hist;        // 512 (two 256-bin buffers)
   uint32_t* scan;        // 32
-  uint32_t* bc;          // 4
+  uint32_t* bc;          // 8
   int* last;
 };
 
-// Selection of unit u from its scores in the workspace: writes sel_idx (ascending
-// page order) and sel_count.  All threads of the CTA call it.
-SA_DEV void select_unit(const SelectArgs& a, const int u, const int b, const int N, const int P,
-                        const SelSmem& S) {
+// Selection from keys staged in shared memory (any P up to max_pages).
+SA_DEV void select_unit_smem(const SelectArgs& a, const int u, const int N, const int P,
+                             const uint32_t cap, const int forced_lo, const int forced_hi,
+                             const int32_t* off, const SelSmem& S) {
   const int tid = threadIdx.x;
   uint32_t* keys = reinterpret_cast<uint32_t*>(S.ring);
   uint32_t* wts = keys + a.kv.max_pages;
-  const float* sc_u = a.ws_scores + (size_t)u * a.kv.max_pages;
-  const bool weighted = a.budget_kind == SA_BUDGET_TOKENS;
-  const int32_t* off = weighted ? a.kv.chunk_off + (size_t)b * (a.kv.max_pages + 1) : nullptr;
-  int forced_lo = 0, forced_hi = P;  // pages < forced_lo or >= forced_hi are forced (ratio)
-  uint32_t cap;
-  if (a.budget_kind == SA_BUDGET_TOPK) {
-    cap = (uint32_t)min(a.top_k, P);
-  } else if (a.budget_kind == SA_BUDGET_RATIO) {
-    const long long fl = (long long)floor((double)P * a.ratio);
-    long long K = (long long)a.topk_val + a.bos + a.eos;
-    if (fl > K) K = fl;
-    if (K > P) K = P;
-    cap = (uint32_t)K;
-    forced_lo = min(a.bos, P);
-    forced_hi = max(0, P - a.eos);
-  } else {
-    cap = (uint32_t)max(a.token_budget, 0);
-  }
+  const float* sc_u = a.ws_scores + (size_t)u * a.ws_stride;
+  const bool weighted = off != nullptr;
+  // Keys (and chunk weights) into shared memory.  Every thread issues all its
+  // loads of a batch before using any: under full HBM load each dependent
+  // round trip to L2 costs about a microsecond.
   uint32_t wall_local = 0;
-  for (int p = tid; p < P; p += blockDim.x) {
-    const float s = __ldcg(sc_u + p);
-    uint32_t key = order_key(s);
-    if (p < forced_lo || p >= forced_hi) key = 0xffffffffu;
-    keys[p] = key;
-    if (weighted) {
-      const int L = min(off[p + 1], N) - off[p];
-      wts[p] = (uint32_t)max(L, 0);
-      wall_local += (uint32_t)max(L, 0);
-    } else {
-      wall_local += 1u;
+  const int P4 = (P + 3) >> 2;  // 16-byte groups of 4 pages (rows are padded to 4)
+  for (int base4 = 0; base4 < P4; base4 += kSelBatch * (int)blockDim.x) {
+    float4 v[kSelBatch];
+    int o[kSelBatch][5];
+#pragma unroll
+    for (int j = 0; j < kSelBatch; ++j) {
+      const int i4 = base4 + j * (int)blockDim.x + tid;
+      v[j] = i4 < P4 ? __ldcg(reinterpret_cast<const float4*>(sc_u) + i4) : make_float4(0.f, 0.f, 0.f, 0.f);
+      if (weighted) {
+#pragma unroll
+        for (int e = 0; e < 5; ++e) o[j][e] = (i4 < P4 && 4 * i4 + e <= P) ? off[4 * i4 + e] : 0;
+      }
+    }
+#pragma unroll
+    for (int j = 0; j < kSelBatch; ++j) {
+      const int i4 = base4 + j * (int)blockDim.x + tid;
+      const float sv[4] = {v[j].x, v[j].y, v[j].z, v[j].w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int p = 4 * i4 + e;
+        if (i4 < P4 && p < P) {
+          uint32_t key = order_key(sv[e]);
+          if (p < forced_lo || p >= forced_hi) key = 0xffffffffu;
+          keys[p] = key;
+          if (weighted) {
+            const int L = max(min(o[j][e + 1], N) - o[j][e], 0);
+            wts[p] = (uint32_t)L;
+            wall_local += (uint32_t)L;
+          } else {
+            wall_local += 1u;
+          }
+        }
+      }
     }
   }
   uint32_t wall;
@@ -167,6 +180,198 @@ SA_DEV void select_unit(const SelectArgs& a, const int u, const int b, const int
     if (total > (uint32_t)a.max_sel) flag_status(a.status, SA_ERR_DEVICE_CHECK);
     a.sel_count[u] = (int32_t)min(total, (uint32_t)a.max_sel);
   }
+}
+
+// Selection with the keys in registers, for P <= KPT * blockDim.x: thread t
+// holds pages [KPT t, KPT t + KPT), so thread order is page order.  The radix
+// digits are histogrammed with shared-memory reductions only (the keys are
+// never re-read from memory) into two alternating 256-bin buffers, so a pass
+// costs two barriers; two block scans then place the kept pages in ascending
+// order (keys equal to the cut taken in page order up to the remaining budget).
+template <int KPT>
+SA_DEV void select_unit_regs(const SelectArgs& a, const int u, const int N, const int P,
+                             const uint32_t cap, const int forced_lo, const int forced_hi,
+                             const int32_t* off, const SelSmem& S) {
+  static_assert(KPT % 4 == 0 && KPT <= 32, "pages per thread");
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nt = blockDim.x;
+  const bool weighted = off != nullptr;
+  const float* sc_u = a.ws_scores + (size_t)u * a.ws_stride;
+  const int p0 = tid * KPT;
+  uint32_t key[KPT], wt[KPT], valid = 0u;
+  {
+    // every load issued before any is used (one round trip to L2)
+    float4 v[KPT / 4];
+#pragma unroll
+    for (int q = 0; q < KPT / 4; ++q)
+      v[q] = p0 + 4 * q < P ? __ldcg(reinterpret_cast<const float4*>(sc_u + p0) + q)
+                            : make_float4(0.f, 0.f, 0.f, 0.f);
+    int o[KPT + 1];
+    if (weighted) {
+#pragma unroll
+      for (int i = 0; i <= KPT; ++i) o[i] = p0 + i <= P ? off[p0 + i] : 0;
+    }
+#pragma unroll
+    for (int q = 0; q < KPT / 4; ++q) {
+      const float sv[4] = {v[q].x, v[q].y, v[q].z, v[q].w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int i = 4 * q + e, p = p0 + i;
+        uint32_t k = order_key(sv[e]);
+        if (p < forced_lo || p >= forced_hi) k = 0xffffffffu;
+        key[i] = k;
+        wt[i] = weighted ? (uint32_t)max(min(o[i + 1], N) - o[i], 0) : 1u;
+        if (p < P) valid |= 1u << i;
+      }
+    }
+  }
+  // common prefix of the valid keys and their total weight
+  uint32_t kmn = 0xffffffffu, kmx = 0u, wsum = 0u;
+#pragma unroll
+  for (int i = 0; i < KPT; ++i)
+    if (valid >> i & 1u) {
+      kmn = min(kmn, key[i]);
+      kmx = max(kmx, key[i]);
+      wsum += wt[i];
+    }
+  kmn = __reduce_min_sync(0xffffffffu, kmn);
+  kmx = __reduce_max_sync(0xffffffffu, kmx);
+  wsum = __reduce_add_sync(0xffffffffu, wsum);
+  uint32_t* bc = S.bc;
+  if (tid < 8) bc[tid] = tid == 0 ? 0xffffffffu : 0u;
+  for (int i = tid; i < 512; i += nt) S.hist[i] = 0u;
+  __syncthreads();
+  if (lane == 0) {
+    atomicMin(&bc[0], kmn);
+    atomicMax(&bc[1], kmx);
+    atomicAdd(&bc[2], wsum);
+  }
+  __syncthreads();
+  const uint32_t gmin = bc[0], gmax = bc[1], wall = bc[2];
+  int32_t* sel_u = a.sel_idx + (size_t)u * a.max_sel;
+  if (wall <= cap) {  // everything fits
+#pragma unroll
+    for (int i = 0; i < KPT; ++i)
+      if ((valid >> i & 1u) && p0 + i < a.max_sel) sel_u[p0 + i] = p0 + i;
+    if (tid == 0) {
+      if (P > a.max_sel) flag_status(a.status, SA_ERR_DEVICE_CHECK);
+      a.sel_count[u] = min(P, a.max_sel);
+    }
+    return;
+  }
+  // MSB-first radix cut: T with weight(keys > T) <= cap < weight(keys >= T)
+  uint32_t T = gmin, rem = cap;
+  const int first = gmin == gmax ? 4 : (__clz(gmin ^ gmax) >> 3);
+  if (first < 4) {
+    uint32_t mask = first == 0 ? 0u : (0xffffffffu << (32 - 8 * first));
+    uint32_t prefix = gmin & mask;
+    for (int pass = first; pass < 4; ++pass) {
+      const int shift = 24 - 8 * pass;
+      uint32_t* H = S.hist + 256 * (pass & 1);
+      uint32_t* Hn = S.hist + 256 * ((pass & 1) ^ 1);
+#pragma unroll
+      for (int i = 0; i < KPT; ++i)
+        if ((valid >> i & 1u) && wt[i] != 0u && (key[i] & mask) == prefix)
+          atomicAdd(&H[(key[i] >> shift) & 255u], wt[i]);
+      __syncthreads();
+      uint32_t* res = bc + 4 + 2 * (pass & 1);
+      if (warp == 0) {
+        // lane l owns buckets 255-8l .. 248-8l (descending); find the bucket
+        // where the running weight from the top first exceeds rem
+        uint32_t h[8], ls = 0;
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+          h[q] = H[255 - 8 * lane - q];
+          ls += h[q];
+        }
+        uint32_t inc = ls;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const uint32_t y = __shfl_up_sync(0xffffffffu, inc, o);
+          if (lane >= o) inc += y;
+        }
+        const unsigned ball = __ballot_sync(0xffffffffu, inc > rem);
+        const int L = __ffs(ball) - 1;
+        if (lane == L) {
+          uint32_t run = inc - ls;
+          int d = 255 - 8 * lane - 7;
+#pragma unroll
+          for (int q = 0; q < 8; ++q) {
+            if (run + h[q] > rem) {
+              d = 255 - 8 * lane - q;
+              break;
+            }
+            run += h[q];
+          }
+          res[0] = (uint32_t)d;
+          res[1] = run;
+        }
+      } else {
+        for (int i = tid - 32; i < 256; i += nt - 32) Hn[i] = 0u;  // the next pass's buffer
+      }
+      __syncthreads();
+      rem -= res[1];
+      prefix |= res[0] << shift;
+      mask |= 0xffu << shift;
+    }
+    T = prefix;
+  }
+  // keys above T are kept; keys equal to T in page order while the weight fits
+  uint32_t eqw = 0u;
+#pragma unroll
+  for (int i = 0; i < KPT; ++i)
+    if ((valid >> i & 1u) && key[i] == T) eqw += wt[i];
+  uint32_t dummy;
+  uint32_t eq = block_excl_scan(eqw, S.scan, dummy);
+  uint32_t keep = 0u;
+#pragma unroll
+  for (int i = 0; i < KPT; ++i) {
+    if (!(valid >> i & 1u)) continue;
+    bool k = key[i] > T;
+    if (key[i] == T) {
+      eq += wt[i];
+      k = eq <= rem;
+    }
+    if (k) keep |= 1u << i;
+  }
+  uint32_t total;
+  uint32_t pos = block_excl_scan((uint32_t)__popc(keep), S.scan, total);
+#pragma unroll
+  for (int i = 0; i < KPT; ++i)
+    if (keep >> i & 1u) {
+      if (pos < (uint32_t)a.max_sel) sel_u[pos] = p0 + i;
+      ++pos;
+    }
+  if (tid == 0) {
+    if (total > (uint32_t)a.max_sel) flag_status(a.status, SA_ERR_DEVICE_CHECK);
+    a.sel_count[u] = (int32_t)min(total, (uint32_t)a.max_sel);
+  }
+}
+
+// Selection of unit u from its scores in the workspace: writes sel_idx
+// (ascending page order) and sel_count.  All threads of the CTA call it.
+SA_DEV void select_unit(const SelectArgs& a, const int u, const int b, const int N, const int P,
+                        const SelSmem& S) {
+  const bool weighted = a.budget_kind == SA_BUDGET_TOKENS;
+  const int32_t* off = weighted ? a.kv.chunk_off + (size_t)b * (a.kv.max_pages + 1) : nullptr;
+  int forced_lo = 0, forced_hi = P;  // pages < forced_lo or >= forced_hi are forced (ratio)
+  uint32_t cap;
+  if (a.budget_kind == SA_BUDGET_TOPK) {
+    cap = (uint32_t)min(a.top_k, P);
+  } else if (a.budget_kind == SA_BUDGET_RATIO) {
+    const long long fl = (long long)floor((double)P * a.ratio);
+    long long K = (long long)a.topk_val + a.bos + a.eos;
+    if (fl > K) K = fl;
+    if (K > P) K = P;
+    cap = (uint32_t)K;
+    forced_lo = min(a.bos, P);
+    forced_hi = max(0, P - a.eos);
+  } else {
+    cap = (uint32_t)max(a.token_budget, 0);
+  }
+  if (P <= 16 * (int)blockDim.x)
+    select_unit_regs<16>(a, u, N, P, cap, forced_lo, forced_hi, off, S);
+  else
+    select_unit_smem(a, u, N, P, cap, forced_lo, forced_hi, off, S);
 }
 
 // FUSED (the decode step): refresh the newest page while scoring and publish
@@ -229,7 +434,7 @@ SA_DEV void select_item(const SelectArgs& a, const int u, const int split, const
   }
 
   // ---- scoring: warp w takes tiles t_begin + w, + 4, ...
-  float* sc_u = a.ws_scores + (size_t)u * a.kv.max_pages;
+  float* sc_u = a.ws_scores + (size_t)u * a.ws_stride;
   float* out_u = a.scores_out ? a.scores_out + (size_t)u * a.kv.max_pages : nullptr;
   unsigned char* ring = S.ring + warp * (kStages * kTileBytes);
   uint64_t* bars = S.bars + warp * kStages;
