@@ -111,9 +111,10 @@ size_t select_scratch(const sa_kv_desc* kv) {
   return align256((size_t)kv->batch * kv->n_kv_heads * score_stride(kv) * sizeof(float));
 }
 
-size_t decode_scratch(int units, int splits) {
-  if (splits <= 1) return 0;
-  return align256((size_t)units * splits * kMaxGroup * (kHeadDim + 4) * sizeof(float));
+// Split partials: one slot per work item (none when no unit is split).
+size_t decode_scratch(const DecodePlan& p) {
+  if (p.splits <= 1 && p.splits_fine <= 1) return 0;
+  return align256((size_t)p.items * kMaxGroup * (kHeadDim + 4) * sizeof(float));
 }
 
 }  // namespace
@@ -318,7 +319,8 @@ bool fill_select(SelectArgs* a, const sa_kv_desc* kv, const void* meta, sa_score
 // the K/V tensor maps cannot be encoded.
 bool fill_decode(DecodeArgs* a, const sa_kv_desc* kv, const void* q, int n_q_heads, int G,
                  float scale, const int32_t* idx, const int32_t* count, int max_sel, float* out,
-                 float* lse, float* ws_part, uint32_t* ws_count, int* status, int splits) {
+                 float* lse, float* ws_part, uint32_t* ws_count, int* status,
+                 const DecodePlan& plan) {
   const unsigned long long kv_rows = (unsigned long long)kv->batch * kv->n_kv_heads * kv->cap_tokens;
   if (!encode_tmap_2d(&a->tmap_k, kv->k, kv_rows, kHeadDim * 2, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, 16) ||
       !encode_tmap_2d(&a->tmap_v, kv->v, kv_rows, kHeadDim * 2, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, 16))
@@ -340,7 +342,10 @@ bool fill_decode(DecodeArgs* a, const sa_kv_desc* kv, const void* q, int n_q_hea
   a->ws_count = ws_count;
   a->ws_queue = nullptr;
   a->status = status;
-  a->splits = splits;
+  a->splits = plan.splits;
+  a->fine_unit0 = plan.fine_unit0;
+  a->splits_fine = plan.splits_fine;
+  a->n_items = (int)plan.items;
   return true;
 }
 
@@ -362,8 +367,8 @@ size_t sparse_attn_workspace_size(const sa_kv_desc* kv, int32_t n_q_heads, int32
   const long long units = (long long)rows * kv->n_kv_heads;
   if (units > kMaxUnits) return 0;
   // selection scores + decode partials (both live during sparse_attn_decode_step)
-  const int splits = decode_splits((int)units, max_tiles_per_unit(kv, max_sel), sm);
-  size_t tail = select_scratch(kv) + decode_scratch((int)units, splits);
+  const DecodePlan plan = decode_plan((int)units, max_tiles_per_unit(kv, max_sel), sm);
+  size_t tail = select_scratch(kv) + decode_scratch(plan);
   const int route_tiles = rows < kMaxRouteTiles ? rows : kMaxRouteTiles;  // tiles <= query rows
   const size_t rt = route_ws_bytes(route_tiles, kv->n_kv_heads, kv->max_pages, max_sel);
   if (rt > tail) tail = rt;
@@ -428,15 +433,16 @@ sa_status sparse_attn_decode(const sa_kv_desc* kv, const void* q, int32_t n_q_he
   if (units > kMaxUnits) return SA_ERR_UNSUPPORTED;
   const unsigned long long kv_rows = (unsigned long long)kv->batch * kv->n_kv_heads * kv->cap_tokens;
   if (kv_rows > 0x7fffffffULL) return SA_ERR_UNSUPPORTED;  // TMA row coordinates are int32
-  const int splits = decode_splits((int)units, max_tiles_per_unit(kv, max_sel), device_sm_count());
-  const size_t need = kScratch + decode_scratch((int)units, splits);
+  const DecodePlan plan = decode_plan((int)units, max_tiles_per_unit(kv, max_sel), device_sm_count());
+  if (plan.items > 0x7fffffffLL) return SA_ERR_UNSUPPORTED;
+  const size_t need = kScratch + decode_scratch(plan);
   if ((s = check_ws(ws, ws_bytes, need)) != SA_OK) return s;
 
   DecodeArgs a;
   char* w = reinterpret_cast<char*>(ws);
   if (!fill_decode(&a, kv, q, n_q_heads, G, scale, idx, count, max_sel, out, lse,
                    reinterpret_cast<float*>(w + kScratch), reinterpret_cast<uint32_t*>(w + 256),
-                   reinterpret_cast<int*>(ws), splits))
+                   reinterpret_cast<int*>(ws), plan))
     return SA_ERR_CUDA;
   a.ws_queue = reinterpret_cast<uint32_t*>(w + kQueueDecode);
   return launched(launch_decode(a, (cudaStream_t)stream));
@@ -459,9 +465,9 @@ sa_status sparse_attn_decode_step(const sa_kv_desc* kv, void* meta, sa_score_rul
   const unsigned long long kv_rows = (unsigned long long)kv->batch * kv->n_kv_heads * kv->cap_tokens;
   if (kv_rows > 0x7fffffffULL) return SA_ERR_UNSUPPORTED;  // TMA row coordinates are int32
   const int sm = device_sm_count();
-  const int dsplits = decode_splits((int)units, max_tiles_per_unit(kv, max_sel), sm);
+  const DecodePlan plan = decode_plan((int)units, max_tiles_per_unit(kv, max_sel), sm);
   const size_t sel_bytes = select_scratch(kv);
-  const size_t need = kScratch + sel_bytes + decode_scratch((int)units, dsplits);
+  const size_t need = kScratch + sel_bytes + decode_scratch(plan);
   if ((s = check_ws(ws, ws_bytes, need)) != SA_OK) return s;
   if (step_smem_bytes(kv->max_pages, max_sel, kv->page_size == 0) > 227 * 1024)
     return SA_ERR_UNSUPPORTED;
@@ -472,11 +478,11 @@ sa_status sparse_attn_decode_step(const sa_kv_desc* kv, void* meta, sa_score_rul
                    nullptr, ws) ||
       !fill_decode(&a.dec, kv, q, n_q_heads, G, scale, sel_idx, sel_count, max_sel, out, lse,
                    reinterpret_cast<float*>(w + kScratch + sel_bytes),
-                   reinterpret_cast<uint32_t*>(w + 256) + units, reinterpret_cast<int*>(ws), dsplits))
+                   reinterpret_cast<uint32_t*>(w + 256) + units, reinterpret_cast<int*>(ws), plan))
     return SA_ERR_CUDA;
   a.sel.meta_refresh = static_cast<unsigned char*>(meta);
   a.queue = reinterpret_cast<uint32_t*>(w + kQueueStep);
-  const long long n_score = units * a.sel.splits, n_dec = units * dsplits;
+  const long long n_score = units * a.sel.splits, n_dec = plan.items;
   if (n_score + n_dec > 0x7fffffffLL) return SA_ERR_UNSUPPORTED;
   a.n_score = (int)n_score;
   a.n_dec = (int)n_dec;
@@ -660,8 +666,8 @@ extern "C" sa_status sparse_attn_decode_static(const sa_kv_desc* kv, const void*
   if (units > kStaticMaxUnits) return SA_ERR_WORKSPACE;  // beyond the built-in scratch
   const unsigned long long kv_rows = (unsigned long long)kv->batch * kv->n_kv_heads * kv->cap_tokens;
   if (kv_rows > 0x7fffffffULL) return SA_ERR_UNSUPPORTED;
-  const int splits = decode_splits((int)units, max_tiles_per_unit(kv, max_sel), device_sm_count());
-  if (kStaticPartOff + decode_scratch((int)units, splits) > kStaticScratchBytes) return SA_ERR_WORKSPACE;
+  const DecodePlan plan = decode_plan((int)units, max_tiles_per_unit(kv, max_sel), device_sm_count());
+  if (kStaticPartOff + decode_scratch(plan) > kStaticScratchBytes) return SA_ERR_WORKSPACE;
 
   unsigned char* scratch = nullptr;
   if ((s = static_scratch(&scratch)) != SA_OK) return s;
@@ -691,6 +697,9 @@ extern "C" sa_status sparse_attn_decode_static(const sa_kv_desc* kv, const void*
   a.ws_count = reinterpret_cast<uint32_t*>(scratch + 256);
   a.ws_queue = reinterpret_cast<uint32_t*>(scratch + kQueueDecode);
   a.status = device_status ? reinterpret_cast<int*>(device_status) : reinterpret_cast<int*>(scratch);
-  a.splits = splits;
+  a.splits = plan.splits;
+  a.fine_unit0 = plan.fine_unit0;
+  a.splits_fine = plan.splits_fine;
+  a.n_items = (int)plan.items;
   return launched(launch_decode(a, (cudaStream_t)stream));
 }

@@ -30,13 +30,14 @@ __global__ void __launch_bounds__(kThreads, SA_DEC_CTAS_PER_SM) decode_kernel(co
   }
   __syncthreads();
   WarpState ws{0u, true, 0u, 0u};
-  const int n_items = a.n_rows * a.kv.Hkv * a.splits;
   for (;;) {
     if (threadIdx.x == 0) s_item = (int)atomicAdd(&a.ws_queue[0], 1u);
     __syncthreads();
     const int item = s_item;
-    if (item >= n_items) break;
-    decode_item(a, item / a.splits, item % a.splits, sm, ws);
+    if (item >= a.n_items) break;
+    int u, split;
+    item_unit(a, item, u, split);
+    decode_item(a, u, split, sm, ws);
     fence_proxy_async();  // generic writes to the ring (merge) before the next TMA writes
     __syncthreads();
   }
@@ -58,8 +59,13 @@ __global__ void __launch_bounds__(kThreads, SA_DEC_CTAS_PER_SM) decode_kernel(co
 }  // namespace
 
 // Splits per unit: items of about SA_DEC_ITEM_TILES tiles, but at least two
-// items per SM when there are few units, and at least 4 tiles per item.
-int decode_splits(int units, int max_tiles, int sm_count) {
+// items per SM when there are few units, and at least 4 tiles per item.  The
+// units of the last wave of items (one item per resident CTA) may get
+// SA_DEC_TAIL_FINE times finer splits, so the launch does not end on a few
+// long items.  Off by default: on the 48-layer decode step a factor of 2 or 4
+// costs more in per-item overhead (about 9 us of claim, setup, pipeline fill
+// and combine per item) than it saves in the tail.
+DecodePlan decode_plan(int units, int max_tiles, int sm_count) {
   int s = (max_tiles + SA_DEC_ITEM_TILES - 1) / SA_DEC_ITEM_TILES;
   const int fill = (2 * sm_count + units - 1) / units;
   if (fill > s) s = fill;
@@ -67,7 +73,18 @@ int decode_splits(int units, int max_tiles, int sm_count) {
   if (s > cap) s = cap;
   if (s > 256) s = 256;
   if (s < 1) s = 1;
-  return s;
+  int fine = SA_DEC_TAIL_FINE * s;
+  if (fine > cap) fine = cap;
+  if (fine > 256) fine = 256;
+  DecodePlan p{s, units, s, 0};
+  if (fine > s) {
+    const int wave = sm_count * SA_DEC_CTAS_PER_SM;
+    const int fine_units = (wave + fine - 1) / fine;
+    p.fine_unit0 = units > fine_units ? units - fine_units : 0;
+    p.splits_fine = fine;
+  }
+  p.items = (long long)p.fine_unit0 * p.splits + (long long)(units - p.fine_unit0) * p.splits_fine;
+  return p;
 }
 
 size_t decode_smem_bytes(int max_sel, bool chunks) {
@@ -78,8 +95,7 @@ size_t decode_smem_bytes(int max_sel, bool chunks) {
 
 cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t st) {
   const size_t smem = decode_smem_bytes(a.max_sel, a.kv.page_size == 0);
-  const long long items = (long long)a.n_rows * a.kv.Hkv * a.splits;
-  if (items > 0x7fffffffLL) return cudaErrorInvalidValue;
+  const long long items = a.n_items;
   long long grid = (long long)device_sm_count() * SA_DEC_CTAS_PER_SM;
   if (grid > items) grid = items;
   const cudaError_t e = set_smem_attr((const void*)decode_kernel, smem);

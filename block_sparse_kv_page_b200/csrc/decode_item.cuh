@@ -47,6 +47,9 @@
 #ifndef SA_DEC_CTAS_PER_SM
 #define SA_DEC_CTAS_PER_SM 3
 #endif
+#ifndef SA_DEC_TAIL_FINE
+#define SA_DEC_TAIL_FINE 1
+#endif
 
 namespace sa {
 namespace dec {
@@ -84,6 +87,19 @@ struct Smem {
   int* last;
   int* ntiles;
 };
+
+// Unit and split of decode item j (queue order: units ascending).
+SA_DEV void item_unit(const DecodeArgs& a, const int j, int& u, int& split) {
+  const int n0 = a.fine_unit0 * a.splits;
+  if (j < n0) {
+    u = j / a.splits;
+    split = j - u * a.splits;
+  } else {
+    const int r = (j - n0) / a.splits_fine;
+    u = a.fine_unit0 + r;
+    split = j - n0 - r * a.splits_fine;
+  }
+}
 
 SA_DEV void decode_item(const DecodeArgs& a, const int u, const int split, const Smem& sm,
                         WarpState& ws) {
@@ -135,8 +151,13 @@ SA_DEV void decode_item(const DecodeArgs& a, const int u, const int split, const
   if (bad && tid == 0 && split == 0) flag_status(a.status, SA_ERR_DEVICE_CHECK);
   __syncthreads();
   const int T = *sm.ntiles;
-  const int t_begin = (int)(((long long)T * split) / a.splits);
-  const int t_end = (int)(((long long)T * (split + 1)) / a.splits);
+  // this unit's split count and first partial slot
+  const bool coarse = u < a.fine_unit0;
+  const int splits = coarse ? a.splits : a.splits_fine;
+  const size_t slot0 = coarse ? (size_t)u * a.splits
+                              : (size_t)a.fine_unit0 * a.splits + (size_t)(u - a.fine_unit0) * a.splits_fine;
+  const int t_begin = (int)(((long long)T * split) / splits);
+  const int t_end = (int)(((long long)T * (split + 1)) / splits);
   const long long row0 = (long long)u * a.kv.cap;
 
   // Token range of tile t of the unit (n = 0 for a skipped, invalid entry).
@@ -351,7 +372,7 @@ SA_DEV void decode_item(const DecodeArgs& a, const int u, const int split, const
   }
   const size_t out_row = (size_t)b * a.Hq + (size_t)g * G + h;
 
-  if (a.splits == 1) {
+  if (splits == 1) {
     if (h < G) {
       const float inv = L > 0.f ? 1.f / L : 0.f;
       float* o = a.out + out_row * kHeadDim + d0;
@@ -364,7 +385,7 @@ SA_DEV void decode_item(const DecodeArgs& a, const int u, const int split, const
   }
 
   // ---- several splits: publish the partial; the last CTA of the unit merges
-  float* part = a.ws_part + ((size_t)u * a.splits + split) * kPartStride;
+  float* part = a.ws_part + (slot0 + split) * kPartStride;
   if (h < G) {
     float* dst = part + h * kPartHead;
 #pragma unroll
@@ -376,7 +397,7 @@ SA_DEV void decode_item(const DecodeArgs& a, const int u, const int split, const
   __syncthreads();
   if (tid == 0) {
     const uint32_t prev = atomicAdd(&a.ws_count[u], 1u);
-    *sm.last = (prev == (uint32_t)(a.splits - 1));
+    *sm.last = (prev == (uint32_t)(splits - 1));
   }
   __syncthreads();
   if (!*sm.last) return;
@@ -387,16 +408,16 @@ SA_DEV void decode_item(const DecodeArgs& a, const int u, const int split, const
   // Merge in split order, kMergeBatch partials per batch with every load of a
   // batch issued before any is used (each dependent round trip to L2 costs
   // about a microsecond under full HBM load).
-  const float* base = a.ws_part + (size_t)u * a.splits * kPartStride + h * kPartHead;
+  const float* base = a.ws_part + slot0 * kPartStride + h * kPartHead;
   float MM = ninf, LL = 0.f, AA[kDimsPerThread];
 #pragma unroll
   for (int x = 0; x < kDimsPerThread; ++x) AA[x] = 0.f;
-  for (int sp0 = 0; sp0 < a.splits; sp0 += kMergeBatch) {
+  for (int sp0 = 0; sp0 < splits; sp0 += kMergeBatch) {
     float2 ml[kMergeBatch];
     float4 v[kMergeBatch][kDimsPerThread / 4];
 #pragma unroll
     for (int j = 0; j < kMergeBatch; ++j) {
-      const bool ok = sp0 + j < a.splits;
+      const bool ok = sp0 + j < splits;
       const float* src = base + (size_t)(ok ? sp0 + j : 0) * kPartStride;
       ml[j] = ok ? __ldcg(reinterpret_cast<const float2*>(src + kHeadDim)) : make_float2(ninf, 0.f);
 #pragma unroll

@@ -43,7 +43,6 @@ bool encode_tmap_2d(CUtensorMap* map, const void* base, unsigned long long rows,
 // Opt a kernel into `bytes` of dynamic shared memory on the current device
 // (cached per device and kernel, so repeated launches skip the driver call).
 cudaError_t set_smem_attr(const void* func, size_t bytes);
-int decode_splits(int units, int max_tiles, int sm_count);
 int select_splits(int units, int max_pages, int sm_count);
 WsLayout workspace_layout(const sa_kv_desc* kv, int n_q_heads, int n_q_rows, int max_sel,
                           int sm_count);
@@ -91,9 +90,21 @@ struct DecodeArgs {
   uint32_t* ws_count;
   uint32_t* ws_queue;
   int* status;
-  int splits;
+  int splits;                 // splits of units [0, fine_unit0)
+  int fine_unit0;             // units from here on (the end of the queue) use splits_fine
+  int splits_fine;
+  int n_items;                // fine_unit0 * splits + (units - fine_unit0) * splits_fine
 };
 cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t st);
+
+// Split plan of a decode launch: `splits` ranges per unit, except that the
+// units at the end of the item queue get `splits_fine` (finer) ranges so the
+// last wave of items is short and the launch drains quickly.
+struct DecodePlan {
+  int splits, fine_unit0, splits_fine;
+  long long items;            // work items = partial slots
+};
+DecodePlan decode_plan(int units, int max_tiles, int sm_count);
 
 // One decode step in one launch: newest-page metadata refresh, scoring,
 // selection and decode.  Scoring items come first in the queue; decode item j

@@ -97,7 +97,8 @@ __global__ void __launch_bounds__(kThreads, SA_STEP_CTAS_PER_SM)
     if (threadIdx.x == 0) {
       int item = (int)atomicAdd(&a.queue[0], 1u);
       if (item >= a.n_score && item < n_items) {
-        const int u = (item - a.n_score) / a.dec.splits;
+        int u, split;
+        dec::item_unit(a.dec, item - a.n_score, u, split);
         if (wait_selected(a.sel.ws_count + u, a.sel.status))
           __threadfence();
         else
@@ -111,8 +112,9 @@ __global__ void __launch_bounds__(kThreads, SA_STEP_CTAS_PER_SM)
     if (item < a.n_score) {
       sel::select_item<RULE, true>(a.sel, item / a.sel.splits, item % a.sel.splits, S, ws);
     } else {
-      const int j = item - a.n_score;
-      dec::decode_item(a.dec, j / a.dec.splits, j % a.dec.splits, D, ws);
+      int u, split;
+      dec::item_unit(a.dec, item - a.n_score, u, split);
+      dec::decode_item(a.dec, u, split, D, ws);
     }
     fence_proxy_async();  // generic writes to the ring (keys, merge) before the next TMA writes
     __syncthreads();
