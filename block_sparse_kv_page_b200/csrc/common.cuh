@@ -123,6 +123,17 @@ struct WarpState {
   uint32_t drain_hi;
 };
 
+// CTA-to-CTA handoff.  After a __syncthreads, one thread's release (or
+// acq_rel) operation at GPU scope publishes the writes of the whole CTA (the
+// PTX memory model makes release cumulative over what the barrier ordered
+// before it); the consumer's acquire makes them visible to its thread, and a
+// __syncthreads passes that on to the rest of its CTA.
+SA_DEV uint32_t atom_add_acq_rel_u32(uint32_t* p, uint32_t v) {
+  uint32_t old;
+  asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], %2;\n" : "=r"(old) : "l"(p), "r"(v) : "memory");
+  return old;
+}
+
 // GPU-scope acquire load / release store of a 32-bit flag in global memory.
 SA_DEV uint32_t ld_acquire_u32(const uint32_t* p) {
   uint32_t v;

@@ -393,15 +393,15 @@ SA_DEV void decode_item(const DecodeArgs& a, const int u, const int split, const
       *reinterpret_cast<float4*>(dst + d0 + x) = make_float4(A[x], A[x + 1], A[x + 2], A[x + 3]);
     if (d0 == 0) *reinterpret_cast<float2*>(dst + kHeadDim) = make_float2(M, L);
   }
-  __threadfence();
+  // the counter increment is acq_rel: it publishes this CTA's partial and,
+  // for the last CTA, acquires the other splits' partials
   __syncthreads();
   if (tid == 0) {
-    const uint32_t prev = atomicAdd(&a.ws_count[u], 1u);
+    const uint32_t prev = atom_add_acq_rel_u32(&a.ws_count[u], 1u);
     *sm.last = (prev == (uint32_t)(splits - 1));
   }
   __syncthreads();
   if (!*sm.last) return;
-  __threadfence();
   if (tid == 0) a.ws_count[u] = 0;
   if (h >= G) return;
 

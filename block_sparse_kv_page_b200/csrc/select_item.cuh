@@ -563,22 +563,20 @@ SA_DEV void select_item(const SelectArgs& a, const int u, const int split, const
   }
   ws.gi += (uint32_t)n_it;
 
-  // ---- the last CTA of the unit selects
+  // ---- the last CTA of the unit selects (its counter increment is acq_rel:
+  // it publishes this CTA's scores and acquires those of the other splits)
   __syncthreads();
   if (a.splits > 1) {
-    __threadfence();
     if (tid == 0) {
-      const uint32_t prev = atomicAdd(&a.ws_count[u], 1u);
+      const uint32_t prev = atom_add_acq_rel_u32(&a.ws_count[u], 1u);
       *S.last = (prev == (uint32_t)(a.splits - 1));
     }
     __syncthreads();
     if (!*S.last) return;
-    __threadfence();
   }
   if (tid == 0 && a.splits > 1 && !FUSED) a.ws_count[u] = 0;  // ready for the next call
   select_unit(a, u, b, N, P, S);
   if (FUSED) {
-    __threadfence();
     __syncthreads();
     if (tid == 0) st_release_u32(&a.ws_count[u], kUnitSelected);
   }

@@ -99,9 +99,7 @@ __global__ void __launch_bounds__(kThreads, SA_STEP_CTAS_PER_SM)
       if (item >= a.n_score && item < n_items) {
         int u, split;
         dec::item_unit(a.dec, item - a.n_score, u, split);
-        if (wait_selected(a.sel.ws_count + u, a.sel.status))
-          __threadfence();
-        else
+        if (!wait_selected(a.sel.ws_count + u, a.sel.status))  // acquire
           item = n_items;  // gave up: this CTA stops taking work
       }
       s_item = item;
