@@ -539,11 +539,10 @@ def peaks():
 
 
 # DRAM bytes read + written per launch (dram__bytes_read.sum + dram__bytes_write.sum),
-# from one ncu capture of the current kernels on this workload (48 stacked
+# from one ncu capture of the current kernel on this workload (48 stacked
 # layers, 29,504 tokens, envelope, 4096-token budget); other settings: null.
 NCU_TRAFFIC = {
-    ("decode", "envelope", 4096): 403_413_248 + 7_616_512,
-    ("select", "envelope", 4096): 182_304_768 + 4_662_272,
+    ("step", "envelope", 4096): 586_376_192 + 7_856_128,
 }
 
 
