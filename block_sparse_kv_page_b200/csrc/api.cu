@@ -526,6 +526,10 @@ sa_status sparse_attn_route(const sa_kv_desc* kv, const void* meta, sa_score_rul
                       env ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32,
                       env ? 2 : 4, 16))
     return SA_ERR_CUDA;
+  if (!encode_tmap_2d(&a.tmap_meta_tc, meta, meta_rows, kMetaBytes,
+                      env ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32,
+                      env ? 2 : 4, 128))
+    return SA_ERR_CUDA;
   a.kv = view(kv);
   a.rule = (int)rule;
   a.q = q;

@@ -138,6 +138,7 @@ int tile_attn_mchunks(int vectors_per_tile);
 
 struct RouteArgs {
   CUtensorMap tmap_meta;      // block metadata rows [Hkv*max_pages][512 B], boxes 16 x 128 B, 128B swizzle
+  CUtensorMap tmap_meta_tc;   // the same rows, boxes 128 x 128 B (tensor-core M tiles)
   KvView kv;
   int rule;
   const void* q;              // bf16 [n_rows][Hq][128]

@@ -33,6 +33,7 @@
 #include "common.cuh"
 #include "internal.h"
 #include "radix.cuh"
+#include "tcgen05.cuh"
 
 namespace sa {
 namespace {
@@ -89,7 +90,19 @@ SA_DEV void route_select_tile(const RouteArgs& a, int t, int g, int E, unsigned 
   uint32_t* keys = reinterpret_cast<uint32_t*>(smem);                         // [E]
   unsigned long long* cand = reinterpret_cast<unsigned long long*>(smem + ((E * 4 + 15) & ~15));
   uint32_t* kp = a.ws_keys + (size_t)tg * a.kv.max_pages;
-  for (int i = tid; i < E; i += blockDim.x) keys[i] = __ldcg(kp + i);
+  for (int b = 0; b < E; b += 8 * (int)blockDim.x) {  // 8 loads in flight per thread
+    uint32_t v[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const int i = b + j * (int)blockDim.x + tid;
+      v[j] = i < E ? __ldcg(kp + i) : 0u;
+    }
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const int i = b + j * (int)blockDim.x + tid;
+      if (i < E) keys[i] = v[j];
+    }
+  }
   __syncthreads();
   const int want = max(a.W, a.k + 1);
   const int cap = min(want, E);
@@ -204,12 +217,52 @@ SA_DEV void route_finalize(const RouteArgs& a, unsigned char* smem) {
     const bool trig = sbar[t] < tau;
     if (tg % Hkv == 0) a.triggered[t] = trig ? 1 : 0;
     const int E = __ldcg(a.ws_elig + tg);
-    const int n = min(trig ? a.W : a.k, E);
-    const int32_t* lst = a.ws_list + (size_t)tg * a.W;
-    int32_t* dst = a.kv_idx + (size_t)tg * a.W;
-    for (int i = 0; i < a.W; ++i) dst[i] = i < n ? __ldcg(lst + i) : -1;
-    a.kv_count[tg] = n;
+    a.kv_count[tg] = min(trig ? a.W : a.k, E);
   }
+  // the lists, every (tile, head, entry) by its own thread: independent loads
+  const int total = T * Hkv * a.W;
+  for (int b = 0; b < total; b += 8 * (int)blockDim.x) {  // 8 loads in flight per thread
+    int32_t v[8], ne[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const int x = b + j * (int)blockDim.x + tid;
+      v[j] = x < total ? __ldcg(a.ws_list + x) : -1;
+      ne[j] = x < total ? __ldcg(a.ws_elig + x / a.W) : 0;
+    }
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const int x = b + j * (int)blockDim.x + tid;
+      if (x >= total) continue;
+      const int tg = x / a.W, i = x - tg * a.W;
+      const int n = min(sbar[tg / Hkv] < tau ? a.W : a.k, ne[j]);
+      a.kv_idx[x] = i < n ? v[j] : -1;
+    }
+  }
+}
+
+// ---------------------------------------------------------------- after scoring
+// The last split CTA of (t, g) selects; the last (t, g) CTA finalizes.  The
+// counter increments are acq_rel after a barrier: they publish this CTA's
+// tile-score keys (or list) and acquire everyone else's.
+SA_DEV void route_tail(const RouteArgs& a, int t, int g, int E, unsigned char* base, uint32_t* hist,
+                       uint32_t* bc, uint32_t* scan, int* flag) {
+  const int tid = threadIdx.x;
+  const int tg = t * a.kv.Hkv + g;
+  __syncthreads();
+  if (tid == 0) {
+    *flag = 1;
+    if (a.nsplit > 1) *flag = atom_add_acq_rel_u32(a.ws_count + tg, 1u) == (uint32_t)(a.nsplit - 1);
+  }
+  __syncthreads();
+  if (!*flag) return;
+  if (tid == 0 && a.nsplit > 1) a.ws_count[tg] = 0;
+  route_select_tile(a, t, g, E, base, hist, bc, scan);
+  __syncthreads();
+  if (tid == 0) *flag = atom_add_acq_rel_u32(a.ws_final, 1u) == (uint32_t)(a.n_tiles * a.kv.Hkv - 1);
+  __syncthreads();
+  if (!*flag) return;
+  if (tid == 0) *a.ws_final = 0;
+  route_finalize(a, base);
 }
 
 // ---------------------------------------------------------------- the kernel
@@ -374,26 +427,221 @@ __global__ void __launch_bounds__(kRtThreads) route_kernel(const __grid_constant
     for (int tb = tb_fail; tb < hi; ++tb) mbar_wait(bars + tb % kRtStages, (tb / kRtStages) & 1u, nullptr);
   }
 
-  // ---- the last split of (t, g) selects; the last (t, g) finalizes
-  __threadfence();
-  __syncthreads();
+  route_tail(a, t, g, geo.E, base, s_hist, s_bc, s_scan, &s_flag);
+}
+
+// ---------------------------------------------------------------- tensor-core (tcgen05) envelope scoring
+// CTA = (tile t, KV head g, split of <= 224 query vectors), one per SM.  The
+// scores of 128 blocks against the split's vectors are one tcgen05 GEMM
+//   D[128 blocks x 224 vectors] = [kmin|kmax] (128 x 256 bf16, K-major)
+//                                 . [q-|q+]^T (224 x 256 bf16, K-major)
+// accumulated in tensor memory (fp32).  Warp-specialised:
+//   warp 4 (one thread)  copies metadata by TMA in 16 KiB K-chunks (128 blocks
+//                        x 128 B) into a kTcStages ring;
+//   warp 5 (one thread)  issues the MMAs (4 per chunk, 32 B of K each) and
+//                        commits: a chunk's stage is freed when its MMAs are
+//                        done, an accumulator is marked full after 4 chunks;
+//   warps 0-3            epilogue: thread i owns block i of the M tile (TMEM
+//                        lane i), takes the max over the vectors in registers
+//                        and folds it into the tile-score keys (atomicMax).
+// The two accumulators alternate, so the epilogue of one M tile overlaps the
+// MMAs of the next; every wait is bounded.
+constexpr int kTcEpiWarps = 4;
+constexpr int kTcThreads = 32 * (kTcEpiWarps + 2);
+constexpr int kTcProducerWarp = kTcEpiWarps;
+constexpr int kTcMmaWarp = kTcEpiWarps + 1;
+constexpr int kTcStages = 6;
+constexpr int kTcChunkBytes = 128 * 128;
+constexpr int kTcAccCols = 256;                               // one accumulator (224 used)
+constexpr int kTcOffRing = kQsBytes;
+constexpr int kTcOffBars = kTcOffRing + kTcStages * kTcChunkBytes;
+constexpr int kTcNumBars = 2 * kTcStages + 4 + 1;             // full, empty, acc full x2, acc empty x2, drain
+constexpr int kTcSmemBytes = kTcOffBars + kTcNumBars * 8 + 16;
+static_assert(kRtVecs % 16 == 0 && kRtVecs <= kTcAccCols, "MMA N");
+static_assert(1024 + kTcSmemBytes > 114 * 1024, "one CTA per SM: it allocates all 512 TMEM columns");
+
+__global__ void __launch_bounds__(kTcThreads, 1) route_tc_kernel(const __grid_constant__ RouteArgs a) {
+  extern __shared__ unsigned char smem_raw[];
+  __shared__ uint32_t s_hist[256];
+  __shared__ uint32_t s_scan[32];
+  __shared__ uint32_t s_bc[4];
+  __shared__ int s_flag;
+  __shared__ uint32_t s_tmem;
+  unsigned char* base = reinterpret_cast<unsigned char*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  unsigned char* qs = base;
+  unsigned char* ring = base + kTcOffRing;
+  uint64_t* full = reinterpret_cast<uint64_t*>(base + kTcOffBars);
+  uint64_t* empty = full + kTcStages;
+  uint64_t* acc_full = empty + kTcStages;
+  uint64_t* acc_empty = acc_full + 2;
+  uint64_t* drain = acc_empty + 2;
+
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int Hkv = a.kv.Hkv;
+  const int sp = blockIdx.x % a.nsplit;
+  const int tg = blockIdx.x / a.nsplit;
+  const int t = tg / Hkv, g = tg % Hkv;
+  const int N = a.kv.seq_len[0];
+  const RouteGeom geo = route_geom(a, t, N);
+  const int v0 = sp * kRtVecs;
+
   if (tid == 0) {
-    s_flag = 1;
-    if (a.nsplit > 1) s_flag = atomicAdd(a.ws_count + tg, 1u) == (uint32_t)(a.nsplit - 1);
+    for (int s = 0; s < kTcStages; ++s) {
+      mbar_init(full + s, 1);
+      mbar_init(empty + s, 1);
+    }
+    mbar_init(acc_full, 1);
+    mbar_init(acc_full + 1, 1);
+    mbar_init(acc_empty, kTcEpiWarps);
+    mbar_init(acc_empty + 1, kTcEpiWarps);
+    mbar_init(drain, 1);
+    fence_barrier_init();
+    prefetch_tmap(&a.tmap_meta_tc);
   }
+  if (warp == 0) {
+    tc::tmem_alloc(&s_tmem, 2 * kTcAccCols);
+    tc::tmem_relinquish();
+  }
+  __syncthreads();  // barriers initialised
+  const int n_mt = (geo.E + 127) >> 7;  // M tiles of 128 blocks
+  const int n_ch = 4 * n_mt;            // K-chunks
+  const int row_base = g * a.kv.max_pages;
+  // the first ring of metadata copies needs no wait: start it before the queries load
+  const int n_pre = min(kTcStages, n_ch);
+  if (warp == kTcProducerWarp && lane == 0)
+    for (int j = 0; j < n_pre; ++j) {
+      mbar_arrive_expect_tx(full + j, kTcChunkBytes);
+      tma_load_2d(ring + j * kTcChunkBytes, &a.tmap_meta_tc, (j & 3) * 64, row_base + 128 * (j >> 2), full + j);
+    }
+
+  // ---- [q- | q+] of this split's vectors: K-major, 128B-swizzled chunks (the
+  // MMA's B operand); kQBatch 16-byte loads per thread in flight at once
+  constexpr int kQPieces = kRtVecs * 16;  // 16-byte pieces of the 224 x 128 bf16 queries
+  constexpr int kQBatch = 8;
+  const __nv_bfloat16* Q = reinterpret_cast<const __nv_bfloat16*>(a.q);
+#pragma unroll 1
+  for (int b0 = 0; b0 < kQPieces; b0 += kQBatch * kTcThreads) {
+    uint4 rw[kQBatch];
+#pragma unroll
+    for (int i = 0; i < kQBatch; ++i) {
+      const int x = b0 + i * kTcThreads + tid;
+      const int vi = x >> 4, d8 = x & 15;
+      const int v = v0 + vi;
+      rw[i] = make_uint4(0u, 0u, 0u, 0u);
+      if (x < kQPieces && v < geo.V) {
+        const int r = v / a.G, j = v - r * a.G;
+        rw[i] = ldg_nc128(Q + ((size_t)(geo.row0 + r) * a.Hq + (size_t)g * a.G + j) * kHeadDim + 8 * d8);
+      }
+    }
+#pragma unroll
+    for (int i = 0; i < kQBatch; ++i) {
+      const int x = b0 + i * kTcThreads + tid;
+      if (x >= kQPieces) continue;
+      const int vi = x >> 4, d8 = x & 15;
+      const uint4 raw = rw[i];
+      uint4 neg, pos;
+      neg.x = bf16x2_neg_part(raw.x); neg.y = bf16x2_neg_part(raw.y);
+      neg.z = bf16x2_neg_part(raw.z); neg.w = bf16x2_neg_part(raw.w);
+      pos.x = bf16x2_pos_part(raw.x); pos.y = bf16x2_pos_part(raw.y);
+      pos.z = bf16x2_pos_part(raw.z); pos.w = bf16x2_pos_part(raw.w);
+      *reinterpret_cast<uint4*>(qs + (d8 >> 3) * kQsChunk + swz128(vi, d8 & 7)) = neg;
+      *reinterpret_cast<uint4*>(qs + (2 + (d8 >> 3)) * kQsChunk + swz128(vi, d8 & 7)) = pos;
+    }
+  }
+  fence_proxy_async();  // generic writes of qs before the tensor cores read it
+  tc::fence_before_sync();
   __syncthreads();
-  if (!s_flag) return;
-  __threadfence();
-  if (tid == 0 && a.nsplit > 1) a.ws_count[tg] = 0;
-  route_select_tile(a, t, g, geo.E, base, s_hist, s_bc, s_scan);
-  __threadfence();
+  tc::fence_after_sync();
+  const uint32_t tmem = s_tmem;
+
+  int fail = 0;                         // this thread saw a wait run out
+
+  if (warp == kTcProducerWarp) {
+    // ---- TMA producer: chunk j -> stage j % kTcStages
+    if (lane == 0) {
+      int issued = n_pre;
+      for (int j = n_pre; j < n_ch; ++j) {
+        const int s = j % kTcStages;
+        if (j >= kTcStages && !mbar_wait(empty + s, ((j / kTcStages) - 1) & 1u, a.status)) {
+          fail = 1;
+          break;
+        }
+        mbar_arrive_expect_tx(full + s, kTcChunkBytes);
+        tma_load_2d(ring + s * kTcChunkBytes, &a.tmap_meta_tc, (j & 3) * 64, row_base + 128 * (j >> 2), full + s);
+        issued = j + 1;
+      }
+      // every copy issued has landed before the CTA moves on (bounded)
+      for (int j = max(0, issued - kTcStages); j < issued; ++j)
+        mbar_wait(full + (j % kTcStages), (j / kTcStages) & 1u, nullptr);
+    }
+  } else if (warp == kTcMmaWarp) {
+    // ---- MMA issuer
+    if (lane == 0) {
+      const uint32_t idesc = tc::idesc_f32acc(tc::kFmtBF16, 128, kRtVecs);
+      for (int m = 0; m < n_mt && !fail; ++m) {
+        if (m >= 2 && !mbar_wait(acc_empty + (m & 1), ((m >> 1) - 1) & 1u, a.status)) {
+          fail = 1;
+          break;
+        }
+        tc::fence_after_sync();
+        const uint32_t d = tmem + (uint32_t)((m & 1) * kTcAccCols);
+        for (int c = 0; c < 4; ++c) {
+          const int j = 4 * m + c, s = j % kTcStages;
+          if (!mbar_wait(full + s, (j / kTcStages) & 1u, a.status)) {
+            fail = 1;
+            break;
+          }
+#pragma unroll
+          for (int k = 0; k < 4; ++k)
+            tc::mma_bf16_ss(d, tc::smem_desc_sw128(ring + s * kTcChunkBytes + 32 * k),
+                            tc::smem_desc_sw128(qs + c * kQsChunk + 32 * k), idesc, (c | k) != 0);
+          tc::commit(empty + s);
+        }
+        if (!fail) tc::commit(acc_full + (m & 1));
+      }
+      // every MMA issued has completed before TMEM is freed (bounded)
+      tc::commit(drain);
+      mbar_wait(drain, 0, nullptr);
+    }
+  } else {
+    // ---- epilogue: thread tid owns block 128 e + tid of M tile e (TMEM lane tid)
+    uint32_t* keys_tg = a.ws_keys + (size_t)tg * a.kv.max_pages;
+    const float ninf = -__int_as_float(0x7f800000);
+    const int nv = min(kRtVecs, geo.V - v0);
+    for (int e = 0; e < n_mt; ++e) {
+      const bool ok = mbar_wait(acc_full + (e & 1), (e >> 1) & 1u, a.status);
+      if (!__all_sync(0xffffffffu, ok)) {
+        fail = 1;
+        break;
+      }
+      tc::fence_after_sync();
+      const uint32_t ta = tmem + (uint32_t)((e & 1) * kTcAccCols) + ((uint32_t)(32 * warp) << 16);
+      float mx = ninf;
+#pragma unroll
+      for (int cc = 0; cc < kRtVecs / 16; cc += 2) {
+        uint32_t r0[16], r1[16];
+        tc::ld_32x32b_x16(ta + 16 * cc, r0);
+        tc::ld_32x32b_x16(ta + 16 * cc + 16, r1);
+        tc::wait_ld();
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          if (16 * cc + i < nv) mx = fmaxf(mx, __uint_as_float(r0[i]));
+          if (16 * cc + 16 + i < nv) mx = fmaxf(mx, __uint_as_float(r1[i]));
+        }
+      }
+      tc::fence_before_sync();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(acc_empty + (e & 1));
+      const int blk = 128 * e + tid;
+      if (blk < geo.E && mx != ninf) atomicMax(keys_tg + blk, order_key(mx));
+    }
+  }
+  tc::fence_before_sync();
   __syncthreads();
-  if (tid == 0) s_flag = atomicAdd(a.ws_final, 1u) == (uint32_t)(a.n_tiles * Hkv - 1);
-  __syncthreads();
-  if (!s_flag) return;
-  __threadfence();
-  if (tid == 0) *a.ws_final = 0;
-  route_finalize(a, base);
+  tc::fence_after_sync();
+  if (warp == 0) tc::tmem_dealloc(tmem, 2 * kTcAccCols);
+  route_tail(a, t, g, geo.E, base, s_hist, s_bc, s_scan, &s_flag);
 }
 
 }  // namespace
@@ -412,9 +660,10 @@ cudaError_t launch_route(const RouteArgs& a, cudaStream_t st) {
   if (grid > 0x7fffffffLL) return cudaErrorInvalidValue;
   cudaError_t e;
   if (a.rule == 0) {
-    e = set_smem_attr((const void*)route_kernel<0>, smem);
+    const size_t smem_tc = 1024 + kTcSmemBytes;
+    e = set_smem_attr((const void*)route_tc_kernel, smem_tc);
     if (e != cudaSuccess) return e;
-    route_kernel<0><<<(unsigned)grid, kRtThreads, smem, st>>>(a);
+    route_tc_kernel<<<(unsigned)grid, kTcThreads, smem_tc, st>>>(a);
   } else {
     e = set_smem_attr((const void*)route_kernel<1>, smem);
     if (e != cudaSuccess) return e;
