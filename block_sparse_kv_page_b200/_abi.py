@@ -85,7 +85,7 @@ def load(path: str = LIB_PATH) -> C.CDLL:
     if not os.path.exists(path):
         raise ImportError(
             f"libsparse_attn.so not found at {path}; build it with "
-            "`python -m block_sparse_kv_page_b200.build` (there is no CPU fallback)")
+            "`python block_sparse_kv_page_b200/build.py` (there is no CPU fallback)")
     lib = C.CDLL(path)
     for name, (res, args) in PROTOTYPES.items():
         fn = getattr(lib, name)

@@ -1,6 +1,8 @@
 """Build libsparse_attn.so in-tree with nvcc for sm_100a.
 
-    python -m block_sparse_kv_page_b200.build [--verbose]
+    python block_sparse_kv_page_b200/build.py [--verbose]
+
+(run as a script: importing the package loads the library this builds)
 
 Compiles every csrc/*.cu to an object under _build/ (skipped when the object
 is newer than its sources and headers) and links them with the static CUDA

@@ -1,7 +1,7 @@
 // C-ABI entry points: host-side argument validation, workspace layout and
 // kernel launches.  Nothing here computes results; every step of the path
 // runs in the kernels of meta.cu, select.cu, decode.cu, step.cu, route.cu and
-// tile_attn.cu.
+// tile_attn_tc.cu.
 //
 // Workspace layout (byte offsets from ws, which must be 256-byte aligned):
 //   [0, 256)                 status word (int32) at 0; item-queue counters of
@@ -225,7 +225,7 @@ sa_status tile_attention(const sa_kv_desc* kv, const void* q, int n_q_heads, int
   a.q_pos0 = q_pos0;
   a.tile_rows = tile_rows;
   a.n_tiles = (int)T;
-  a.n_mchunks = tile_attn_mchunks(tile_rows * G);
+  a.n_mchunks = tile_attn_tc_mchunks(tile_rows * G);
   a.scale_log2 = scale * kLog2e;
   a.idx = idx;
   a.count = count;
@@ -233,7 +233,7 @@ sa_status tile_attention(const sa_kv_desc* kv, const void* q, int n_q_heads, int
   a.out = out;
   a.lse = lse;
   a.status = status;
-  return launched(launch_tile_attn(a, (cudaStream_t)stream));
+  return launched(launch_tile_attn_tc(a, (cudaStream_t)stream));
 }
 
 // Argument checks of a selection (sparse_attn_select and sparse_attn_decode_step).

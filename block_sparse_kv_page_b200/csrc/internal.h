@@ -120,7 +120,7 @@ size_t step_smem_bytes(int max_pages, int max_sel, bool chunks);
 
 struct TileAttnArgs {
   CUtensorMap tmap_k;         // K rows [Hkv*cap][128 bf16], boxes 64 x 64, 128B swizzle
-  CUtensorMap tmap_v;
+  CUtensorMap tmap_v;         // V, same geometry (read MN-major by the PV MMA)
   KvView kv;                  // batch 1, 64-token blocks
   const void* q;              // bf16 [n_rows][Hq][128]
   int Hq, G;
@@ -133,8 +133,9 @@ struct TileAttnArgs {
   float* lse;
   int* status;
 };
-cudaError_t launch_tile_attn(const TileAttnArgs& a, cudaStream_t st);
-int tile_attn_mchunks(int vectors_per_tile);
+// Tile attention on tcgen05 (CTA = 128 query vectors of a (tile, KV head)).
+cudaError_t launch_tile_attn_tc(const TileAttnArgs& a, cudaStream_t st);
+int tile_attn_tc_mchunks(int vectors_per_tile);
 
 struct RouteArgs {
   CUtensorMap tmap_meta;      // block metadata rows [Hkv*max_pages][512 B], boxes 16 x 128 B, 128B swizzle
