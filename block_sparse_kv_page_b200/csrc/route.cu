@@ -17,14 +17,13 @@
 // One launch, no CTA waits on another:
 //   * CTA (tile t, KV head g, split sp) scores every eligible block of head g
 //     against its share (<= 224) of the tile's query vectors (row x head) on
-//     tensor cores -- block metadata streamed by TMA (16 blocks x 512 B per
-//     stage, 128B swizzle), query vectors resident in shared memory:
-//       envelope: [kmin|kmax] (16 x 256 bf16) x [q-|q+]^T, m16n8k16, exact products;
-//       centroid: kmean (16 x 128 fp32) x q^T on m16n8k8 tf32 with kmean split
-//                 into a tf32 head and its exact remainder (products exact to
-//                 about 2^-21);
-//     and folds its per-block maxima into the tile-score keys with atomicMax
-//     on order-preserving uint32 keys.
+//     the 5th-generation tensor cores (tcgen05, accumulators in tensor memory):
+//       envelope: [kmin|kmax] (128 blocks x 256 bf16) . [q-|q+]^T, exact
+//                 products, fp32 accumulation;
+//       centroid: kmean (fp32) split into three bf16 parts hi + mid + lo,
+//                 three bf16 GEMMs against the exact bf16 queries;
+//     each block's max over the vectors is folded into the tile-score keys
+//     with atomicMax on order-preserving uint32 keys.
 //   * The last split CTA of (t, g) (atomic counter) selects the top
 //     max(rho*k, k+1) eligible blocks by radix select, sorts them to rank
 //     order (score desc, index asc) and computes sigma in double.
@@ -38,24 +37,9 @@
 namespace sa {
 namespace {
 
-constexpr int kRtWarps = 4;
-constexpr int kRtThreads = 32 * kRtWarps;
-constexpr int kRtNTilesPerWarp = 7;                         // n8 tiles of query vectors per warp
-constexpr int kRtVecs = 8 * kRtNTilesPerWarp * kRtWarps;     // 224 query vectors per CTA
-constexpr int kRtStages = 3;
-constexpr int kTileBytes = 8192;                             // 16 blocks x 512 B
-constexpr int kBoxBytes = 2048;
+constexpr int kRtVecs = 224;                                // query vectors per CTA (MMA N)
 constexpr int kQsChunk = kRtVecs * 128;                      // one 128-byte K chunk of all vectors
-constexpr int kQsBytes = 4 * kQsChunk;                       // 112 KiB
-constexpr int kOffRing = kQsBytes;
-constexpr int kOffBars = kOffRing + kRtStages * kTileBytes;
-constexpr int kSmemBytes = kOffBars + kRtStages * 8;
-
-SA_DEV void ldsm_x2(uint32_t& r0, uint32_t& r1, const void* p) {
-  asm volatile("ldmatrix.sync.aligned.m8n8.x2.shared.b16 {%0,%1}, [%2];\n"
-               : "=r"(r0), "=r"(r1)
-               : "r"(smem_addr(p)));
-}
+constexpr int kQsBytes = 4 * kQsChunk;                       // 112 KiB ([q- | q+], 256 bf16)
 
 // Inverse of order_key.
 SA_DEV float key_to_float(uint32_t k) {
@@ -263,171 +247,6 @@ SA_DEV void route_tail(const RouteArgs& a, int t, int g, int E, unsigned char* b
   if (!*flag) return;
   if (tid == 0) *a.ws_final = 0;
   route_finalize(a, base);
-}
-
-// ---------------------------------------------------------------- the kernel
-template <int RULE>
-__global__ void __launch_bounds__(kRtThreads) route_kernel(const __grid_constant__ RouteArgs a) {
-  extern __shared__ unsigned char smem_raw[];
-  __shared__ float s_wmax[2][kRtWarps][16];
-  __shared__ uint32_t s_hist[256];
-  __shared__ uint32_t s_scan[32];
-  __shared__ uint32_t s_bc[4];
-  __shared__ int s_flag;
-  unsigned char* base = reinterpret_cast<unsigned char*>(
-      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-  unsigned char* qs = base;
-  unsigned char* ring = base + kOffRing;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(base + kOffBars);
-
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int gq = lane >> 2, c = lane & 3;
-  const int Hkv = a.kv.Hkv;
-  const int sp = blockIdx.x % a.nsplit;
-  const int tg = blockIdx.x / a.nsplit;
-  const int t = tg / Hkv, g = tg % Hkv;
-  const int N = a.kv.seq_len[0];
-  const RouteGeom geo = route_geom(a, t, N);
-  const int v0 = sp * kRtVecs;
-
-  if (tid == 0) {
-    for (int s = 0; s < kRtStages; ++s) mbar_init(bars + s, 1);
-    fence_barrier_init();
-    prefetch_tmap(&a.tmap_meta);
-  }
-
-  // ---- query vectors of this split into shared memory (K-major, 128B-swizzled chunks)
-  const __nv_bfloat16* Q = reinterpret_cast<const __nv_bfloat16*>(a.q);
-  for (int x = tid; x < kRtVecs * 16; x += kRtThreads) {
-    const int vi = x >> 4, d8 = x & 15;  // vector, 8-element chunk of the 128-dim query
-    const int v = v0 + vi;
-    uint4 raw = make_uint4(0u, 0u, 0u, 0u);
-    if (v < geo.V) {
-      const int r = v / a.G, j = v - (v / a.G) * a.G;
-      raw = ldg_nc128(Q + ((size_t)(geo.row0 + r) * a.Hq + (size_t)g * a.G + j) * kHeadDim + 8 * d8);
-    }
-    if (RULE == 0) {  // [q- | q+]: element e of 256 -> chunk e/64, 16-byte piece (e%64)/8
-      uint4 neg, pos;
-      neg.x = bf16x2_neg_part(raw.x); neg.y = bf16x2_neg_part(raw.y);
-      neg.z = bf16x2_neg_part(raw.z); neg.w = bf16x2_neg_part(raw.w);
-      pos.x = bf16x2_pos_part(raw.x); pos.y = bf16x2_pos_part(raw.y);
-      pos.z = bf16x2_pos_part(raw.z); pos.w = bf16x2_pos_part(raw.w);
-      *reinterpret_cast<uint4*>(qs + (d8 >> 3) * kQsChunk + swz128(vi, d8 & 7)) = neg;
-      *reinterpret_cast<uint4*>(qs + (2 + (d8 >> 3)) * kQsChunk + swz128(vi, d8 & 7)) = pos;
-    } else {  // fp32 [128]: element d -> chunk d/32, piece (d%32)/4
-      const float4 lo = make_float4(bf16_lo(raw.x), bf16_hi(raw.x), bf16_lo(raw.y), bf16_hi(raw.y));
-      const float4 hi = make_float4(bf16_lo(raw.z), bf16_hi(raw.z), bf16_lo(raw.w), bf16_hi(raw.w));
-      const int ch = d8 >> 2, pc = 2 * (d8 & 3);
-      *reinterpret_cast<float4*>(qs + ch * kQsChunk + swz128(vi, pc)) = lo;
-      *reinterpret_cast<float4*>(qs + ch * kQsChunk + swz128(vi, pc + 1)) = hi;
-    }
-  }
-  __syncthreads();
-
-  // ---- stream the eligible blocks of head g, 16 per stage
-  const int TB = (geo.E + 15) >> 4;
-  const int row_base = g * a.kv.max_pages;
-  auto issue = [&](int tb) {
-    uint64_t* bar = bars + tb % kRtStages;
-    unsigned char* st = ring + (tb % kRtStages) * kTileBytes;
-    mbar_arrive_expect_tx(bar, kTileBytes);
-    const int xs = RULE == 0 ? 64 : 32;
-#pragma unroll
-    for (int bx = 0; bx < 4; ++bx) tma_load_2d(st + bx * kBoxBytes, &a.tmap_meta, bx * xs, row_base + 16 * tb, bar);
-  };
-  if (tid == 0)
-    for (int tb = 0; tb < min(TB, kRtStages); ++tb) issue(tb);
-
-  const float ninf = -__int_as_float(0x7f800000);
-  const int lrow = (lane & 7) + 8 * ((lane >> 3) & 1);
-  const int lchk = lane >> 4;
-  const int brow = lane & 7, bchk = (lane >> 3) & 1;  // ldmatrix.x2 for B (lanes 0-15)
-  uint32_t* keys_tg = a.ws_keys + (size_t)tg * a.kv.max_pages;
-  int tb_fail = -1;  // first stage whose wait timed out (CTA-uniform)
-
-  for (int tb = 0; tb < TB; ++tb) {
-    const bool ok = mbar_wait(bars + tb % kRtStages, (tb / kRtStages) & 1u, a.status);
-    if (!__syncthreads_and(ok)) {
-      tb_fail = tb;
-      break;
-    }
-    const bool alive = true;
-    const unsigned char* st = ring + (tb % kRtStages) * kTileBytes;
-    float acc[kRtNTilesPerWarp][4];
-#pragma unroll
-    for (int i = 0; i < kRtNTilesPerWarp; ++i) acc[i][0] = acc[i][1] = acc[i][2] = acc[i][3] = 0.f;
-    if (alive) {
-      if (RULE == 0) {
-#pragma unroll 4
-        for (int ks = 0; ks < 16; ++ks) {
-          uint32_t a0, a1, a2, a3;
-          ldsm_x4(a0, a1, a2, a3, st + (ks >> 2) * kBoxBytes + swz128(lrow, 2 * (ks & 3) + lchk));
-#pragma unroll
-          for (int i = 0; i < kRtNTilesPerWarp; ++i) {
-            const int nt = warp * kRtNTilesPerWarp + i;
-            uint32_t b0, b1;
-            ldsm_x2(b0, b1, qs + (ks >> 2) * kQsChunk + swz128(8 * nt + brow, 2 * (ks & 3) + bchk));
-            mma_bf16(acc[i], a0, a1, a2, a3, b0, b1);
-          }
-        }
-      } else {
-#pragma unroll 2
-        for (int ks = 0; ks < 16; ++ks) {  // dims 8ks .. 8ks + 7
-          const int bx = ks >> 2, ch = 2 * (ks & 3);
-          const float x0 = *reinterpret_cast<const float*>(st + bx * kBoxBytes + swz128(gq, ch) + 4 * c);
-          const float x1 = *reinterpret_cast<const float*>(st + bx * kBoxBytes + swz128(gq + 8, ch) + 4 * c);
-          const float x2 = *reinterpret_cast<const float*>(st + bx * kBoxBytes + swz128(gq, ch + 1) + 4 * c);
-          const float x3 = *reinterpret_cast<const float*>(st + bx * kBoxBytes + swz128(gq + 8, ch + 1) + 4 * c);
-          const uint32_t h0 = __float_as_uint(x0) & 0xffffe000u, h1 = __float_as_uint(x1) & 0xffffe000u;
-          const uint32_t h2 = __float_as_uint(x2) & 0xffffe000u, h3 = __float_as_uint(x3) & 0xffffe000u;
-          const uint32_t l0 = __float_as_uint(x0 - __uint_as_float(h0));
-          const uint32_t l1 = __float_as_uint(x1 - __uint_as_float(h1));
-          const uint32_t l2 = __float_as_uint(x2 - __uint_as_float(h2));
-          const uint32_t l3 = __float_as_uint(x3 - __uint_as_float(h3));
-#pragma unroll
-          for (int i = 0; i < kRtNTilesPerWarp; ++i) {
-            const int v = 8 * (warp * kRtNTilesPerWarp + i) + gq;
-            const uint32_t b0 = *reinterpret_cast<const uint32_t*>(qs + bx * kQsChunk + swz128(v, ch) + 4 * c);
-            const uint32_t b1 = *reinterpret_cast<const uint32_t*>(qs + bx * kQsChunk + swz128(v, ch + 1) + 4 * c);
-            mma_tf32(acc[i], h0, h1, h2, h3, b0, b1);
-            mma_tf32(acc[i], l0, l1, l2, l3, b0, b1);
-          }
-        }
-      }
-    }
-    // max over this warp's query vectors (C[block][vector]: c0,c1 block gq, c2,c3 block gq+8)
-    float mlo = ninf, mhi = ninf;
-#pragma unroll
-    for (int i = 0; i < kRtNTilesPerWarp; ++i) {
-      const int vcol = v0 + 8 * (warp * kRtNTilesPerWarp + i) + 2 * c;
-      const bool ok0 = vcol < geo.V, ok1 = vcol + 1 < geo.V;
-      mlo = fmaxf(mlo, fmaxf(ok0 ? acc[i][0] : ninf, ok1 ? acc[i][1] : ninf));
-      mhi = fmaxf(mhi, fmaxf(ok0 ? acc[i][2] : ninf, ok1 ? acc[i][3] : ninf));
-    }
-    mlo = fmaxf(mlo, __shfl_xor_sync(0xffffffffu, mlo, 1));
-    mlo = fmaxf(mlo, __shfl_xor_sync(0xffffffffu, mlo, 2));
-    mhi = fmaxf(mhi, __shfl_xor_sync(0xffffffffu, mhi, 1));
-    mhi = fmaxf(mhi, __shfl_xor_sync(0xffffffffu, mhi, 2));
-    if (c == 0) {
-      s_wmax[tb & 1][warp][gq] = mlo;
-      s_wmax[tb & 1][warp][gq + 8] = mhi;
-    }
-    __syncthreads();  // stage tb consumed by every warp; wmax[tb & 1] complete
-    if (tid == 0 && tb + kRtStages < TB) issue(tb + kRtStages);
-    if (tid < 16) {
-      const int blk = 16 * tb + tid;
-      float m = s_wmax[tb & 1][0][tid];
-#pragma unroll
-      for (int w = 1; w < kRtWarps; ++w) m = fmaxf(m, s_wmax[tb & 1][w][tid]);
-      if (blk < geo.E && m != ninf) atomicMax(keys_tg + blk, order_key(m));
-    }
-  }
-  if (tb_fail >= 0 && tid == 0) {  // let the copies still in flight land (bounded) before leaving
-    const int hi = min(TB, tb_fail + kRtStages);
-    for (int tb = tb_fail; tb < hi; ++tb) mbar_wait(bars + tb % kRtStages, (tb / kRtStages) & 1u, nullptr);
-  }
-
-  route_tail(a, t, g, geo.E, base, s_hist, s_bc, s_scan, &s_flag);
 }
 
 // ---------------------------------------------------------------- tensor-core (tcgen05) envelope scoring
@@ -644,6 +463,257 @@ __global__ void __launch_bounds__(kTcThreads, 1) route_tc_kernel(const __grid_co
   route_tail(a, t, g, geo.E, base, s_hist, s_bc, s_scan, &s_flag);
 }
 
+// ---------------------------------------------------------------- tensor-core (tcgen05) centroid scoring
+// The block means are fp32; the MMA takes bf16.  Each mean is split into
+// three bf16 parts hi + mid + lo (each the round-to-nearest of what the
+// previous parts left, so together they carry the fp32 mantissa), and the
+// scores are three bf16 GEMMs against the exact bf16 queries accumulated in
+// one fp32 accumulator: products exact, only the fp32 sums round.
+//   warp 4 (one thread)  copies the fp32 means by TMA in half-chunks (128
+//                        blocks x 64 dims = two 16 KiB boxes) into kCrRaw stages;
+//   warps 0-3            split each half-chunk into the three bf16 parts
+//                        (128B-swizzled K-major tiles, kCrConv stages), then
+//                        run the max epilogue of the previous M tile;
+//   warp 5 (one thread)  issues 3 parts x 4 MMAs per half-chunk.
+constexpr int kCrRaw = 2;                                    // fp32 half-chunk stages (32 KiB)
+constexpr int kCrConv = 2;                                   // bf16 stages (3 parts x 16 KiB)
+constexpr int kCrQChunk = kRtVecs * 128;                     // 224 vectors x 64 bf16 dims
+constexpr int kCrOffRaw = 2 * kCrQChunk;
+constexpr int kCrOffConv = kCrOffRaw + kCrRaw * 2 * kTcChunkBytes;
+constexpr int kCrOffBars = kCrOffConv + kCrConv * 3 * kTcChunkBytes;
+constexpr int kCrNumBars = 4 * kCrRaw + 4 + 1;               // raw full/empty, conv full/empty, acc x4, drain
+constexpr int kCrSmemBytes = kCrOffBars + kCrNumBars * 8 + 16;
+static_assert(kCrQChunk % 1024 == 0 && kCrOffRaw % 1024 == 0 && kCrOffConv % 1024 == 0, "1 KiB atoms");
+static_assert(1024 + kCrSmemBytes > 114 * 1024 && 1024 + kCrSmemBytes <= 227 * 1024, "one CTA per SM");
+
+__global__ void __launch_bounds__(kTcThreads, 1) route_tc_centroid_kernel(const __grid_constant__ RouteArgs a) {
+  extern __shared__ unsigned char smem_raw[];
+  __shared__ uint32_t s_hist[256];
+  __shared__ uint32_t s_scan[32];
+  __shared__ uint32_t s_bc[4];
+  __shared__ int s_flag;
+  __shared__ uint32_t s_tmem;
+  unsigned char* base = reinterpret_cast<unsigned char*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  unsigned char* qs = base;
+  unsigned char* raw = base + kCrOffRaw;
+  unsigned char* conv = base + kCrOffConv;
+  uint64_t* raw_full = reinterpret_cast<uint64_t*>(base + kCrOffBars);
+  uint64_t* raw_empty = raw_full + kCrRaw;
+  uint64_t* conv_full = raw_empty + kCrRaw;
+  uint64_t* conv_empty = conv_full + kCrConv;
+  uint64_t* acc_full = conv_empty + kCrConv;
+  uint64_t* acc_empty = acc_full + 2;
+  uint64_t* drain = acc_empty + 2;
+
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int Hkv = a.kv.Hkv;
+  const int sp = blockIdx.x % a.nsplit;
+  const int tg = blockIdx.x / a.nsplit;
+  const int t = tg / Hkv, g = tg % Hkv;
+  const int N = a.kv.seq_len[0];
+  const RouteGeom geo = route_geom(a, t, N);
+  const int v0 = sp * kRtVecs;
+
+  if (tid == 0) {
+    for (int s = 0; s < kCrRaw; ++s) {
+      mbar_init(raw_full + s, 1);
+      mbar_init(raw_empty + s, kTcEpiWarps);
+    }
+    for (int s = 0; s < kCrConv; ++s) {
+      mbar_init(conv_full + s, kTcEpiWarps);
+      mbar_init(conv_empty + s, 1);
+    }
+    mbar_init(acc_full, 1);
+    mbar_init(acc_full + 1, 1);
+    mbar_init(acc_empty, kTcEpiWarps);
+    mbar_init(acc_empty + 1, kTcEpiWarps);
+    mbar_init(drain, 1);
+    fence_barrier_init();
+    prefetch_tmap(&a.tmap_meta_tc);
+  }
+  if (warp == 0) {
+    tc::tmem_alloc(&s_tmem, 2 * kTcAccCols);
+    tc::tmem_relinquish();
+  }
+  __syncthreads();  // barriers initialised
+  const int n_mt = (geo.E + 127) >> 7;  // M tiles of 128 blocks
+  const int n_hc = 2 * n_mt;            // half-chunks (64 dims each)
+  const int row_base = g * a.kv.max_pages;
+  auto load = [&](int j) {  // producer thread: fp32 dims [64 (j&1), +64) of M tile j >> 1
+    const int s = j % kCrRaw;
+    unsigned char* dst = raw + s * (2 * kTcChunkBytes);
+    mbar_arrive_expect_tx(raw_full + s, 2 * kTcChunkBytes);
+    tma_load_2d(dst, &a.tmap_meta_tc, 64 * (j & 1), row_base + 128 * (j >> 1), raw_full + s);
+    tma_load_2d(dst + kTcChunkBytes, &a.tmap_meta_tc, 64 * (j & 1) + 32, row_base + 128 * (j >> 1), raw_full + s);
+  };
+  const int n_pre = min(kCrRaw, n_hc);
+  if (warp == kTcProducerWarp && lane == 0)
+    for (int j = 0; j < n_pre; ++j) load(j);
+
+  // ---- the split's queries as bf16, K-major 128B-swizzled (the MMA's B operand)
+  constexpr int kQPieces = kRtVecs * 16;
+  const __nv_bfloat16* Q = reinterpret_cast<const __nv_bfloat16*>(a.q);
+#pragma unroll 1
+  for (int b0 = 0; b0 < kQPieces; b0 += 8 * kTcThreads) {
+    uint4 rw[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int x = b0 + i * kTcThreads + tid;
+      const int vi = x >> 4, d8 = x & 15, v = v0 + vi;
+      rw[i] = make_uint4(0u, 0u, 0u, 0u);
+      if (x < kQPieces && v < geo.V) {
+        const int r = v / a.G, j = v - r * a.G;
+        rw[i] = ldg_nc128(Q + ((size_t)(geo.row0 + r) * a.Hq + (size_t)g * a.G + j) * kHeadDim + 8 * d8);
+      }
+    }
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int x = b0 + i * kTcThreads + tid;
+      if (x >= kQPieces) continue;
+      const int vi = x >> 4, d8 = x & 15;
+      *reinterpret_cast<uint4*>(qs + (d8 >> 3) * kCrQChunk + swz128(vi, d8 & 7)) = rw[i];
+    }
+  }
+  fence_proxy_async();
+  tc::fence_before_sync();
+  __syncthreads();
+  tc::fence_after_sync();
+  const uint32_t tmem = s_tmem;
+  int fail = 0;
+
+  if (warp == kTcProducerWarp) {
+    if (lane == 0) {
+      int issued = n_pre;
+      for (int j = n_pre; j < n_hc; ++j) {
+        const int s = j % kCrRaw;
+        if (!mbar_wait(raw_empty + s, ((j / kCrRaw) - 1) & 1u, a.status)) {
+          fail = 1;
+          break;
+        }
+        load(j);
+        issued = j + 1;
+      }
+      for (int j = max(0, issued - kCrRaw); j < issued; ++j)  // every copy has landed (bounded)
+        mbar_wait(raw_full + (j % kCrRaw), (j / kCrRaw) & 1u, nullptr);
+    }
+  } else if (warp == kTcMmaWarp) {
+    if (lane == 0) {
+      const uint32_t idesc = tc::idesc_f32acc(tc::kFmtBF16, 128, kRtVecs);
+      for (int m = 0; m < n_mt && !fail; ++m) {
+        if (m >= 2 && !mbar_wait(acc_empty + (m & 1), ((m >> 1) - 1) & 1u, a.status)) {
+          fail = 1;
+          break;
+        }
+        tc::fence_after_sync();
+        const uint32_t d = tmem + (uint32_t)((m & 1) * kTcAccCols);
+        for (int c = 0; c < 2; ++c) {
+          const int j = 2 * m + c, s = j % kCrConv;
+          if (!mbar_wait(conv_full + s, (j / kCrConv) & 1u, a.status)) {
+            fail = 1;
+            break;
+          }
+          const unsigned char* cs = conv + s * (3 * kTcChunkBytes);
+#pragma unroll
+          for (int part = 0; part < 3; ++part)
+#pragma unroll
+            for (int k = 0; k < 4; ++k)
+              tc::mma_bf16_ss(d, tc::smem_desc_sw128(cs + part * kTcChunkBytes + 32 * k),
+                              tc::smem_desc_sw128(qs + c * kCrQChunk + 32 * k), idesc, (c | part | k) != 0);
+          tc::commit(conv_empty + s);
+        }
+        if (!fail) tc::commit(acc_full + (m & 1));
+      }
+      tc::commit(drain);
+      mbar_wait(drain, 0, nullptr);
+    }
+  } else {
+    // ---- warps 0-3: thread tid is block (row) tid of every M tile
+    // split half-chunk j (fp32, two swizzled boxes) into three bf16 parts
+    auto convert = [&](int j) -> bool {
+      const int sr = j % kCrRaw, sc = j % kCrConv;
+      bool ok = mbar_wait(raw_full + sr, (j / kCrRaw) & 1u, a.status);
+      if (ok && j >= kCrConv) ok = mbar_wait(conv_empty + sc, ((j / kCrConv) - 1) & 1u, a.status);
+      if (!__all_sync(0xffffffffu, ok)) return false;
+      tc::fence_after_sync();
+      const unsigned char* src = raw + sr * (2 * kTcChunkBytes);
+      unsigned char* dst = conv + sc * (3 * kTcChunkBytes);
+#pragma unroll 2
+      for (int p8 = 0; p8 < 8; ++p8) {  // output piece p8: dims 8 p8 .. 8 p8 + 7 of the half-chunk
+        const unsigned char* box = src + (p8 >> 2) * kTcChunkBytes;
+        const uint4 xa = lds128(box + swz128(tid, 2 * (p8 & 3)));
+        const uint4 xb = lds128(box + swz128(tid, 2 * (p8 & 3) + 1));
+        const float x[8] = {__uint_as_float(xa.x), __uint_as_float(xa.y), __uint_as_float(xa.z),
+                            __uint_as_float(xa.w), __uint_as_float(xb.x), __uint_as_float(xb.y),
+                            __uint_as_float(xb.z), __uint_as_float(xb.w)};
+        uint32_t hi[4], mid[4], lo[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          hi[e] = pack_bf16(x[2 * e], x[2 * e + 1]);
+          const float r0 = x[2 * e] - bf16_lo(hi[e]), r1 = x[2 * e + 1] - bf16_hi(hi[e]);
+          mid[e] = pack_bf16(r0, r1);
+          lo[e] = pack_bf16(r0 - bf16_lo(mid[e]), r1 - bf16_hi(mid[e]));
+        }
+        const uint32_t o = swz128(tid, p8);
+        *reinterpret_cast<uint4*>(dst + o) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+        *reinterpret_cast<uint4*>(dst + kTcChunkBytes + o) = make_uint4(mid[0], mid[1], mid[2], mid[3]);
+        *reinterpret_cast<uint4*>(dst + 2 * kTcChunkBytes + o) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+      }
+      fence_proxy_async();  // generic accesses of both stages before the async proxy's next ones
+      tc::fence_before_sync();
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(conv_full + sc);
+        mbar_arrive(raw_empty + sr);
+      }
+      return true;
+    };
+    uint32_t* keys_tg = a.ws_keys + (size_t)tg * a.kv.max_pages;
+    const float ninf = -__int_as_float(0x7f800000);
+    const int nv = min(kRtVecs, geo.V - v0);
+    for (int j = 0; j < min(2, n_hc) && !fail; ++j)
+      if (!convert(j)) fail = 1;
+    for (int e = 0; e < n_mt && !fail; ++e) {
+      for (int j = 2 * (e + 1); j < min(2 * (e + 2), n_hc); ++j)  // the next M tile's parts first
+        if (!convert(j)) {
+          fail = 1;
+          break;
+        }
+      if (fail) break;
+      const bool ok = mbar_wait(acc_full + (e & 1), (e >> 1) & 1u, a.status);
+      if (!__all_sync(0xffffffffu, ok)) {
+        fail = 1;
+        break;
+      }
+      tc::fence_after_sync();
+      const uint32_t ta = tmem + (uint32_t)((e & 1) * kTcAccCols) + ((uint32_t)(32 * warp) << 16);
+      float mx = ninf;
+#pragma unroll
+      for (int cc = 0; cc < kRtVecs / 16; cc += 2) {
+        uint32_t r0[16], r1[16];
+        tc::ld_32x32b_x16(ta + 16 * cc, r0);
+        tc::ld_32x32b_x16(ta + 16 * cc + 16, r1);
+        tc::wait_ld();
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          if (16 * cc + i < nv) mx = fmaxf(mx, __uint_as_float(r0[i]));
+          if (16 * cc + 16 + i < nv) mx = fmaxf(mx, __uint_as_float(r1[i]));
+        }
+      }
+      tc::fence_before_sync();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(acc_empty + (e & 1));
+      const int blk = 128 * e + tid;
+      if (blk < geo.E && mx != ninf) atomicMax(keys_tg + blk, order_key(mx));
+    }
+  }
+  tc::fence_before_sync();
+  __syncthreads();
+  tc::fence_after_sync();
+  if (warp == 0) tc::tmem_dealloc(tmem, 2 * kTcAccCols);
+  route_tail(a, t, g, geo.E, base, s_hist, s_bc, s_scan, &s_flag);
+}
+
 }  // namespace
 
 int route_splits(int vectors_per_tile) { return (vectors_per_tile + kRtVecs - 1) / kRtVecs; }
@@ -655,7 +725,6 @@ size_t route_ws_bytes(int n_tiles, int Hkv, int max_pages, int W) {
 }
 
 cudaError_t launch_route(const RouteArgs& a, cudaStream_t st) {
-  const size_t smem = 1024 + kSmemBytes;
   const long long grid = (long long)a.n_tiles * a.kv.Hkv * a.nsplit;
   if (grid > 0x7fffffffLL) return cudaErrorInvalidValue;
   cudaError_t e;
@@ -665,9 +734,10 @@ cudaError_t launch_route(const RouteArgs& a, cudaStream_t st) {
     if (e != cudaSuccess) return e;
     route_tc_kernel<<<(unsigned)grid, kTcThreads, smem_tc, st>>>(a);
   } else {
-    e = set_smem_attr((const void*)route_kernel<1>, smem);
+    const size_t smem_tc = 1024 + kCrSmemBytes;
+    e = set_smem_attr((const void*)route_tc_centroid_kernel, smem_tc);
     if (e != cudaSuccess) return e;
-    route_kernel<1><<<(unsigned)grid, kRtThreads, smem, st>>>(a);
+    route_tc_centroid_kernel<<<(unsigned)grid, kTcThreads, smem_tc, st>>>(a);
   }
   return cudaGetLastError();
 }
