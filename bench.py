@@ -62,6 +62,8 @@ def parse():
     ap.add_argument("--cpu-sample-units", type=int, default=192)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-extra", action="store_true", help="skip the secondary modes/rules")
+    ap.add_argument("--router-only", action="store_true",
+                    help="time only the router workload (route + tile attention) and print its JSON")
     return ap.parse_args()
 
 
@@ -584,6 +586,12 @@ def main():
         return 0
 
     import torch
+    if args.router_only:
+        dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", 0)))
+        torch.cuda.set_device(dev)
+        if rank == 0:
+            print(json.dumps({"router": router_leg(torch, dev, args.steps, max(3, args.warmup))}))
+        return 0
     if world > 1:
         import datetime
 
