@@ -59,7 +59,8 @@ __global__ void __launch_bounds__(kThreads, SA_DEC_CTAS_PER_SM) decode_kernel(co
 }  // namespace
 
 // Splits per unit: items of about SA_DEC_ITEM_TILES tiles, but at least two
-// items per SM when there are few units, and at least 4 tiles per item.  The
+// items per SM when there are few units, and at least SA_DEC_MIN_ITEM_TILES
+// tiles per item (each item pays a fixed setup and combine cost).  The
 // units of the last wave of items (one item per resident CTA) may get
 // SA_DEC_TAIL_FINE times finer splits, so the launch does not end on a few
 // long items.  Off by default: on the 48-layer decode step a factor of 2 or 4
@@ -69,7 +70,7 @@ DecodePlan decode_plan(int units, int max_tiles, int sm_count) {
   int s = (max_tiles + SA_DEC_ITEM_TILES - 1) / SA_DEC_ITEM_TILES;
   const int fill = (2 * sm_count + units - 1) / units;
   if (fill > s) s = fill;
-  const int cap = (max_tiles + 3) / 4;
+  const int cap = (max_tiles + SA_DEC_MIN_ITEM_TILES - 1) / SA_DEC_MIN_ITEM_TILES;
   if (s > cap) s = cap;
   if (s > 256) s = 256;
   if (s < 1) s = 1;

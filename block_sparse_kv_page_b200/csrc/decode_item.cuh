@@ -50,6 +50,9 @@
 #ifndef SA_DEC_TAIL_FINE
 #define SA_DEC_TAIL_FINE 1
 #endif
+#ifndef SA_DEC_MIN_ITEM_TILES
+#define SA_DEC_MIN_ITEM_TILES 16
+#endif
 
 namespace sa {
 namespace dec {

@@ -60,12 +60,14 @@ __global__ void __launch_bounds__(kThreads, SA_SEL_CTAS_PER_SM) select_kernel(co
 }  // namespace
 
 // Splits per unit: items of about SA_SEL_ITEM_PAGES pages, but at least two
-// items per SM when there are few units, and at least one tile per warp.
+// items per SM when there are few units, and at least
+// SA_SEL_MIN_ITEM_TILES_PER_WARP tiles per warp.
 int select_splits(int units, int max_pages, int sm_count) {
   int s = (max_pages + SA_SEL_ITEM_PAGES - 1) / SA_SEL_ITEM_PAGES;
   const int fill = (2 * sm_count + units - 1) / units;
   if (fill > s) s = fill;
-  const int cap = (max_pages + 16 * kWarps - 1) / (16 * kWarps);
+  const int min_pages = 16 * kWarps * SA_SEL_MIN_ITEM_TILES_PER_WARP;
+  const int cap = (max_pages + min_pages - 1) / min_pages;
   if (s > cap) s = cap;
   if (s > 256) s = 256;
   if (s < 1) s = 1;

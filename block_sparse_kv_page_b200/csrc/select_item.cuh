@@ -56,6 +56,9 @@
 #ifndef SA_SEL_WARPS
 #define SA_SEL_WARPS 4
 #endif
+#ifndef SA_SEL_MIN_ITEM_TILES_PER_WARP
+#define SA_SEL_MIN_ITEM_TILES_PER_WARP 2
+#endif
 
 namespace sa {
 namespace sel {
