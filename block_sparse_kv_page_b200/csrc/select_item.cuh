@@ -185,22 +185,46 @@ SA_DEV void select_unit_smem(const SelectArgs& a, const int u, const int N, cons
   }
 }
 
-// Selection with the keys in registers, for P <= KPT * blockDim.x: thread t
-// holds pages [KPT t, KPT t + KPT), so thread order is page order.  The radix
-// digits are histogrammed with shared-memory reductions only (the keys are
-// never re-read from memory) into two alternating 256-bin buffers, so a pass
-// costs two barriers; two block scans then place the kept pages in ascending
-// order (keys equal to the cut taken in page order up to the remaining budget).
-template <int KPT>
+// Selection with the keys in registers, for P <= KPT * 128 (four warps):
+// thread t holds pages [KPT t, KPT t + KPT), so thread order is page order.
+// WEIGHTED: chunk lengths (token budget), else every page weighs 1.
+//
+// The cut T (weight(keys > T) <= cap < weight(keys >= T)) comes from an
+// MSB-first radix search over 12-bit windows of the keys, histogrammed with
+// shared-memory reductions only (the keys are never re-read from memory):
+//  - all-ones keys (forced pages) are settled first: if they overflow the
+//    budget they are the cut, else their weight is spent up front;
+//  - the first window starts at the highest bit where the other keys differ
+//    (the scores of one unit often share sign and exponent), so it spreads
+//    them over up to 4096 bins; the second usually isolates the cut; with unit
+//    weights the search stops as soon as the budget is met exactly at a bin
+//    edge (nothing of the cut bin is taken);
+//  - a pass costs two barriers: thread t sums bin row 127 - t (32 bins, rows
+//    in descending order) and publishes the sum; then every warp, on its own,
+//    scans the 128 row sums, picks the row holding the cut and scans its 32
+//    bins, so the cut needs no broadcast.  Bin rows are 16-byte-chunk XOR
+//    swizzled so that the row sums are conflict-free vector loads.
+// Keys above T are kept, keys equal to T in page order while the weight fits;
+// block scans give each thread its first output slot (one packed scan with
+// unit weights).  The bins live in the ring area, idle during selection.
+SA_DEV uint32_t bin_slot(uint32_t b) {  // physical word of bin b in a 4096-bin buffer
+  const uint32_t r = b >> 5, w = b & 31u;
+  return (r << 5) | ((((w >> 2) ^ (r & 7u)) << 2) | (w & 3u));
+}
+
+template <int KPT, bool WEIGHTED>
 SA_DEV void select_unit_regs(const SelectArgs& a, const int u, const int N, const int P,
                              const uint32_t cap, const int forced_lo, const int forced_hi,
                              const int32_t* off, const SelSmem& S) {
   static_assert(KPT % 4 == 0 && KPT <= 32, "pages per thread");
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nt = blockDim.x;
-  const bool weighted = off != nullptr;
+  static_assert(kThreads == 128, "the register path maps 4096 bins onto 128 threads");
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const float* sc_u = a.ws_scores + (size_t)u * a.ws_stride;
   const int p0 = tid * KPT;
-  uint32_t key[KPT], wt[KPT], valid = 0u;
+  uint32_t* H0 = reinterpret_cast<uint32_t*>(S.ring);  // [2][4096] bins
+  uint32_t* tsum = H0 + 2 * 4096;                       // [128] row sums
+  uint32_t* wred = tsum + 128;                          // [4 warps][4]
+  uint32_t key[KPT], wt[WEIGHTED ? KPT : 1], valid = 0u;
   {
     // every load issued before any is used (one round trip to L2)
     float4 v[KPT / 4];
@@ -208,8 +232,8 @@ SA_DEV void select_unit_regs(const SelectArgs& a, const int u, const int N, cons
     for (int q = 0; q < KPT / 4; ++q)
       v[q] = p0 + 4 * q < P ? __ldcg(reinterpret_cast<const float4*>(sc_u + p0) + q)
                             : make_float4(0.f, 0.f, 0.f, 0.f);
-    int o[KPT + 1];
-    if (weighted) {
+    int o[WEIGHTED ? KPT + 1 : 1];
+    if (WEIGHTED) {
 #pragma unroll
       for (int i = 0; i <= KPT; ++i) o[i] = p0 + i <= P ? off[p0 + i] : 0;
     }
@@ -222,34 +246,43 @@ SA_DEV void select_unit_regs(const SelectArgs& a, const int u, const int N, cons
         uint32_t k = order_key(sv[e]);
         if (p < forced_lo || p >= forced_hi) k = 0xffffffffu;
         key[i] = k;
-        wt[i] = weighted ? (uint32_t)max(min(o[i + 1], N) - o[i], 0) : 1u;
+        if (WEIGHTED) wt[i] = (uint32_t)max(min(o[i + 1], N) - o[i], 0);
         if (p < P) valid |= 1u << i;
       }
     }
   }
-  // common prefix of the valid keys and their total weight
-  uint32_t kmn = 0xffffffffu, kmx = 0u, wsum = 0u;
+  auto W = [&](int i) -> uint32_t { return WEIGHTED ? wt[i] : 1u; };
+  // range of the keys below all-ones, weight of the all-ones keys, total weight
+  uint32_t kmn = 0xffffffffu, kmx = 0u, wsum = 0u, wtop = 0u;
 #pragma unroll
   for (int i = 0; i < KPT; ++i)
     if (valid >> i & 1u) {
-      kmn = min(kmn, key[i]);
-      kmx = max(kmx, key[i]);
-      wsum += wt[i];
+      wsum += W(i);
+      if (key[i] == 0xffffffffu) {
+        wtop += W(i);
+      } else {
+        kmn = min(kmn, key[i]);
+        kmx = max(kmx, key[i]);
+      }
     }
   kmn = __reduce_min_sync(0xffffffffu, kmn);
   kmx = __reduce_max_sync(0xffffffffu, kmx);
   wsum = __reduce_add_sync(0xffffffffu, wsum);
-  uint32_t* bc = S.bc;
-  if (tid < 8) bc[tid] = tid == 0 ? 0xffffffffu : 0u;
-  for (int i = tid; i < 512; i += nt) S.hist[i] = 0u;
+  wtop = __reduce_add_sync(0xffffffffu, wtop);
+  if (lane == 0) *reinterpret_cast<uint4*>(wred + 4 * warp) = make_uint4(kmn, kmx, wsum, wtop);
+#pragma unroll
+  for (int x = 0; x < 8; ++x)  // first pass's bins
+    reinterpret_cast<uint4*>(H0)[tid + 128 * x] = make_uint4(0u, 0u, 0u, 0u);
   __syncthreads();
-  if (lane == 0) {
-    atomicMin(&bc[0], kmn);
-    atomicMax(&bc[1], kmx);
-    atomicAdd(&bc[2], wsum);
+  uint32_t gmin = 0xffffffffu, gmax = 0u, wall = 0u, wtop_all = 0u;
+#pragma unroll
+  for (int x = 0; x < kWarps; ++x) {
+    const uint4 r = *reinterpret_cast<const uint4*>(wred + 4 * x);
+    gmin = min(gmin, r.x);
+    gmax = max(gmax, r.y);
+    wall += r.z;
+    wtop_all += r.w;
   }
-  __syncthreads();
-  const uint32_t gmin = bc[0], gmax = bc[1], wall = bc[2];
   int32_t* sel_u = a.sel_idx + (size_t)u * a.max_sel;
   if (wall <= cap) {  // everything fits
 #pragma unroll
@@ -261,83 +294,131 @@ SA_DEV void select_unit_regs(const SelectArgs& a, const int u, const int N, cons
     }
     return;
   }
-  // MSB-first radix cut: T with weight(keys > T) <= cap < weight(keys >= T)
-  uint32_t T = gmin, rem = cap;
-  const int first = gmin == gmax ? 4 : (__clz(gmin ^ gmax) >> 3);
-  if (first < 4) {
-    uint32_t mask = first == 0 ? 0u : (0xffffffffu << (32 - 8 * first));
-    uint32_t prefix = gmin & mask;
-    for (int pass = first; pass < 4; ++pass) {
-      const int shift = 24 - 8 * pass;
-      uint32_t* H = S.hist + 256 * (pass & 1);
-      uint32_t* Hn = S.hist + 256 * ((pass & 1) ^ 1);
+  // ---- the cut
+  uint32_t T, rem;
+  if (wtop_all > cap) {
+    T = 0xffffffffu;
+    rem = cap;
+  } else if (gmin == gmax || (!WEIGHTED && cap == wtop_all)) {
+    T = gmax;  // with nothing left to spend, no key <= gmax is taken
+    rem = cap - wtop_all;
+  } else {
+    rem = cap - wtop_all;
+    int hi = 32 - __clz(gmin ^ gmax);  // bits [hi, 32) are common to [gmin, gmax]
+    uint32_t prefix = hi == 32 ? 0u : (gmin >> hi) << hi;
+    for (int pass = 0; hi > 0; ++pass) {
+      // window = key bits [hi - 12, hi), or [0, hi) left-aligned in 12 bits
+      const int sr = hi >= 12 ? hi - 12 : 0, sl = hi >= 12 ? 0 : 12 - hi;
+      uint32_t* H = H0 + 4096 * (pass & 1);
+      uint32_t* Hn = H0 + 4096 * ((pass & 1) ^ 1);
 #pragma unroll
-      for (int i = 0; i < KPT; ++i)
-        if ((valid >> i & 1u) && wt[i] != 0u && (key[i] & mask) == prefix)
-          atomicAdd(&H[(key[i] >> shift) & 255u], wt[i]);
-      __syncthreads();
-      uint32_t* res = bc + 4 + 2 * (pass & 1);
-      if (warp == 0) {
-        // lane l owns buckets 255-8l .. 248-8l (descending); find the bucket
-        // where the running weight from the top first exceeds rem
-        uint32_t h[8], ls = 0;
-#pragma unroll
-        for (int q = 0; q < 8; ++q) {
-          h[q] = H[255 - 8 * lane - q];
-          ls += h[q];
-        }
-        uint32_t inc = ls;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-          const uint32_t y = __shfl_up_sync(0xffffffffu, inc, o);
-          if (lane >= o) inc += y;
-        }
-        const unsigned ball = __ballot_sync(0xffffffffu, inc > rem);
-        const int L = __ffs(ball) - 1;
-        if (lane == L) {
-          uint32_t run = inc - ls;
-          int d = 255 - 8 * lane - 7;
-#pragma unroll
-          for (int q = 0; q < 8; ++q) {
-            if (run + h[q] > rem) {
-              d = 255 - 8 * lane - q;
-              break;
-            }
-            run += h[q];
-          }
-          res[0] = (uint32_t)d;
-          res[1] = run;
-        }
-      } else {
-        for (int i = tid - 32; i < 256; i += nt - 32) Hn[i] = 0u;  // the next pass's buffer
+      for (int x = 0; x < KPT; ++x) {
+        const bool in = (valid >> x & 1u) && (!WEIGHTED || W(x) != 0u) && key[x] != 0xffffffffu &&
+                        (hi == 32 || ((key[x] ^ prefix) >> hi) == 0u);
+        if (in) atomicAdd(&H[bin_slot(((key[x] >> sr) << sl) & 4095u)], W(x));
       }
       __syncthreads();
-      rem -= res[1];
-      prefix |= res[0] << shift;
-      mask |= 0xffu << shift;
+      {
+        // row 127 - tid: its 8 chunks in an order that spreads a quarter-warp over the banks
+        const uint4* row = reinterpret_cast<const uint4*>(H + 32 * (127 - tid));
+        uint32_t sum = 0u;
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+          const uint4 v = row[c ^ (tid & 7)];
+          sum += v.x + v.y + v.z + v.w;
+        }
+        tsum[tid] = sum;
+#pragma unroll
+        for (int x = 0; x < 8; ++x)  // next pass's bins (last read a pass ago)
+          reinterpret_cast<uint4*>(Hn)[tid + 128 * x] = make_uint4(0u, 0u, 0u, 0u);
+      }
+      __syncthreads();
+      // every warp: the thread (row) holding the cut, then the bin inside it
+      const uint4 t4 = *reinterpret_cast<const uint4*>(tsum + 4 * lane);  // threads 4l .. 4l+3
+      const uint32_t s4 = t4.x + t4.y + t4.z + t4.w;
+      uint32_t inc = s4;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t y = __shfl_up_sync(0xffffffffu, inc, o);
+        if (lane >= o) inc += y;
+      }
+      const int L = __ffs(__ballot_sync(0xffffffffu, inc > rem)) - 1;
+      uint32_t above = __shfl_sync(0xffffffffu, inc - s4, L);
+      const uint32_t tv[4] = {__shfl_sync(0xffffffffu, t4.x, L), __shfl_sync(0xffffffffu, t4.y, L),
+                              __shfl_sync(0xffffffffu, t4.z, L), __shfl_sync(0xffffffffu, t4.w, L)};
+      int tt = 4 * L + 3;
+#pragma unroll
+      for (int x = 0; x < 3; ++x) {
+        if (above + tv[x] > rem) { tt = 4 * L + x; break; }
+        above += tv[x];
+      }
+      const uint32_t bin = 32u * (uint32_t)(127 - tt) + (uint32_t)(31 - lane);  // descending
+      const uint32_t hv = H[bin_slot(bin)];
+      uint32_t binc = hv;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t y = __shfl_up_sync(0xffffffffu, binc, o);
+        if (lane >= o) binc += y;
+      }
+      const int J = __ffs(__ballot_sync(0xffffffffu, above + binc > rem)) - 1;
+      const uint32_t run = above + __shfl_sync(0xffffffffu, binc - hv, J);
+      const uint32_t cb = 32u * (uint32_t)(127 - tt) + (uint32_t)(31 - J);
+      rem -= run;
+      if (hi >= 12) {
+        prefix |= cb << sr;
+        hi = sr;
+      } else {
+        prefix |= cb >> sl;
+        hi = 0;
+      }
+      if (!WEIGHTED && rem == 0u && hi > 0 && (prefix | ((1u << hi) - 1u)) != 0xffffffffu) {
+        prefix |= (1u << hi) - 1u;  // every key of the cut bin is below this T
+        break;
+      }
     }
     T = prefix;
   }
-  // keys above T are kept; keys equal to T in page order while the weight fits
-  uint32_t eqw = 0u;
+  // ---- kept pages: keys above T, keys equal to T in page order while the weight fits
+  uint32_t keep = 0u, total, pos;
+  if (!WEIGHTED) {
+    uint32_t gt = 0u, eqc = 0u;
 #pragma unroll
-  for (int i = 0; i < KPT; ++i)
-    if ((valid >> i & 1u) && key[i] == T) eqw += wt[i];
-  uint32_t dummy;
-  uint32_t eq = block_excl_scan(eqw, S.scan, dummy);
-  uint32_t keep = 0u;
+    for (int i = 0; i < KPT; ++i)
+      if (valid >> i & 1u) {
+        gt += key[i] > T ? 1u : 0u;
+        eqc += key[i] == T ? 1u : 0u;
+      }
+    uint32_t tot2;
+    const uint32_t ex = block_excl_scan((gt << 16) | eqc, S.scan, tot2);  // both < 2^16
+    uint32_t eq = ex & 0xffffu;
 #pragma unroll
-  for (int i = 0; i < KPT; ++i) {
-    if (!(valid >> i & 1u)) continue;
-    bool k = key[i] > T;
-    if (key[i] == T) {
-      eq += wt[i];
-      k = eq <= rem;
+    for (int i = 0; i < KPT; ++i) {
+      if (!(valid >> i & 1u)) continue;
+      bool k = key[i] > T;
+      if (key[i] == T) k = ++eq <= rem;
+      if (k) keep |= 1u << i;
     }
-    if (k) keep |= 1u << i;
+    pos = (ex >> 16) + min(ex & 0xffffu, rem);
+    total = (tot2 >> 16) + min(tot2 & 0xffffu, rem);
+  } else {
+    uint32_t eqw = 0u;
+#pragma unroll
+    for (int i = 0; i < KPT; ++i)
+      if ((valid >> i & 1u) && key[i] == T) eqw += W(i);
+    uint32_t dummy;
+    uint32_t eq = block_excl_scan(eqw, S.scan, dummy);
+#pragma unroll
+    for (int i = 0; i < KPT; ++i) {
+      if (!(valid >> i & 1u)) continue;
+      bool k = key[i] > T;
+      if (key[i] == T) {
+        eq += W(i);
+        k = eq <= rem;
+      }
+      if (k) keep |= 1u << i;
+    }
+    pos = block_excl_scan((uint32_t)__popc(keep), S.scan, total);
   }
-  uint32_t total;
-  uint32_t pos = block_excl_scan((uint32_t)__popc(keep), S.scan, total);
 #pragma unroll
   for (int i = 0; i < KPT; ++i)
     if (keep >> i & 1u) {
@@ -371,9 +452,12 @@ SA_DEV void select_unit(const SelectArgs& a, const int u, const int b, const int
   } else {
     cap = (uint32_t)max(a.token_budget, 0);
   }
-  if (P <= 16 * (int)blockDim.x)
-    select_unit_regs<16>(a, u, N, P, cap, forced_lo, forced_hi, off, S);
-  else
+  if (P <= 16 * kThreads) {
+    if (weighted)
+      select_unit_regs<16, true>(a, u, N, P, cap, forced_lo, forced_hi, off, S);
+    else
+      select_unit_regs<16, false>(a, u, N, P, cap, forced_lo, forced_hi, off, S);
+  } else
     select_unit_smem(a, u, N, P, cap, forced_lo, forced_hi, off, S);
 }
 
