@@ -64,6 +64,8 @@ def parse():
     ap.add_argument("--no-extra", action="store_true", help="skip the secondary modes/rules")
     ap.add_argument("--router-only", action="store_true",
                     help="time only the router workload (route + tile attention) and print its JSON")
+    ap.add_argument("--tsa-only", action="store_true",
+                    help="print only the TSA workload's timings (token and chunk-count budgets)")
     return ap.parse_args()
 
 
@@ -396,22 +398,35 @@ def run_gpu_arm(args, rank, world, dist):
     meta_bytes = L * B * HKV * (N // PS) * 512
     kv_bytes = L * B * HKV * args.budget * 2 * D * 2
 
-    # ---- end to end through the public API with host buffers
-    q_h = inp["q"].cpu().pin_memory()
-    knew_h = inp["k"][:, :, N - 1, :].contiguous().cpu().pin_memory()
-    vnew_h = inp["v"][:, :, N - 1, :].contiguous().cpu().pin_memory()
+    # ---- end to end through the public API with host buffers.  A step's
+    # inputs (q, and the newest token's K and V per (layer, KV head)) sit in
+    # one pinned host buffer and go over in one copy; the one-launch step
+    # stores the newest K/V into the cache itself (the append variant).  The
+    # other modes scatter them into the cache with a device copy first.
+    nq, nk = inp["q"].numel(), L * B * HKV * D
+    host_in = torch.empty(nq + 2 * nk, dtype=torch.bfloat16).pin_memory()
+    host_in[:nq] = inp["q"].flatten().cpu()
+    host_in[nq:nq + nk] = inp["k"][:, :, N - 1, :].flatten().cpu()
+    host_in[nq + nk:] = inp["v"][:, :, N - 1, :].flatten().cpu()
+    dev_in = torch.empty(host_in.shape, dtype=torch.bfloat16, device=dev)
+    q_d = dev_in[:nq].view(inp["q"].shape)
+    knew_d = dev_in[nq:nq + nk].view(L * B, HKV, D)
+    vnew_d = dev_in[nq + nk:].view(L * B, HKV, D)
     out_h = torch.empty(out.shape, dtype=out.dtype).pin_memory()
 
     def e2e_step():
-        inp["q"].copy_(q_h, non_blocking=True)
-        inp["k"][:, :, N - 1, :].copy_(knew_h, non_blocking=True)
-        inp["v"][:, :, N - 1, :].copy_(vnew_h, non_blocking=True)
-        if args.mode in ("sequential", "step-seq"):
-            seq_graph(args.mode, args.rule).replay()
-        elif args.mode == "step":
-            step_fused(args.rule)
+        dev_in.copy_(host_in, non_blocking=True)
+        if args.mode == "step":
+            sa.sparse_attn_decode_step_append(kv, metas[args.rule], args.rule, q_d, knew_d, vnew_d, budget,
+                                              k, scale, sel, cnt, out, lse, ws)
         else:
-            step_batched(args.rule)
+            inp["q"].copy_(q_d)
+            inp["k"][:, :, N - 1, :].copy_(knew_d)
+            inp["v"][:, :, N - 1, :].copy_(vnew_d)
+            if args.mode in ("sequential", "step-seq"):
+                seq_graph(args.mode, args.rule).replay()
+            else:
+                step_batched(args.rule)
         out_h.copy_(out, non_blocking=True)
 
     for _ in range(args.warmup):
@@ -425,8 +440,10 @@ def run_gpu_arm(args, rank, world, dist):
     a1.record(stream)
     torch.cuda.synchronize()
     e2e_ms = max_over_ranks(a0.elapsed_time(a1) / args.steps, dist, dev)
-    h2d = q_h.numel() * 2 + knew_h.numel() * 2 + vnew_h.numel() * 2
+    h2d = host_in.numel() * host_in.element_size()
     d2h = out_h.numel() * 4
+    if sa.sparse_attn_get_device_status(ws) != 0:
+        raise RuntimeError("device status set after the end-to-end steps")
 
     # ---- secondary measurements (same timing rules), labelled
     extra = {}
@@ -442,11 +459,12 @@ def run_gpu_arm(args, rank, world, dist):
     for g in graphs.values():
         del g
     graphs.clear()
-    router = None
+    router = tsa = None
     if not args.no_extra:
         router = router_leg(torch, dev, max(5, min(args.steps, 50)), max(3, args.warmup))
+        tsa = tsa_leg(torch, dev, max(10, min(args.steps, 50)), max(3, args.warmup))
     return dict(ms=ms, value=value, kern=kern, clocks=clocks.summary(), e2e_ms=e2e_ms, h2d=h2d,
-                d2h=d2h, meta_bytes=meta_bytes, kv_bytes=kv_bytes, extra=extra, router=router,
+                d2h=d2h, meta_bytes=meta_bytes, kv_bytes=kv_bytes, extra=extra, router=router, tsa=tsa,
                 launches_per_step=MODES[args.mode])
 
 
@@ -523,6 +541,89 @@ def router_leg(torch, dev, steps: int, warmup: int):
     return res
 
 
+def tsa_leg(torch, dev, steps: int, warmup: int):
+    """The TSA workload (48 layers x 4 sequences stacked along the batch axis,
+    32 query / 4 KV heads, 29,504 tokens in structure-aligned chunks of 16-256
+    tokens, per-chunk key offsets): the one-launch decode step under token
+    budgets (min/max scoring) and chunk-count budgets (top 64 / top 32 chunks,
+    min/max and centroid scoring), timed with CUDA events.  Effective bytes =
+    metadata of every chunk + K/V of the tokens the kept chunks hold."""
+    import numpy as np
+
+    import block_sparse_kv_page_b200 as sa
+    import datagen as DG
+    w = DG.WORKLOADS[3]
+    L, Bw, Nw = w.layers, w.B, w.N
+    lens = DG.workload3_chunks(Bw, Nw)
+    k_all = torch.empty((L * Bw, w.Hkv, Nw, D), dtype=torch.bfloat16, device=dev)
+    v_all = torch.empty_like(k_all)
+    q_all = torch.empty((L * Bw, w.Hq, D), dtype=torch.bfloat16, device=dev)
+    for l in range(L):
+        lay = DG.workload3_layer(l, dev, chunk_lens=lens)
+        k_all[l * Bw:(l + 1) * Bw] = lay.k
+        v_all[l * Bw:(l + 1) * Bw] = lay.v
+        q_all[l * Bw:(l + 1) * Bw] = lay.q
+        off1, nch1 = lay.chunk_off, lay.n_chunks
+        del lay
+    off = off1.repeat(L, 1).contiguous()
+    nch = nch1.repeat(L).contiguous()
+    seq = torch.full((L * Bw,), Nw, dtype=torch.int32, device=dev)
+    maxc = off.shape[1] - 1
+    kv = sa.KvCache(k_all, v_all, seq, page_size=0, max_pages=maxc, chunk_off=off, n_chunks=nch)
+    units = L * Bw * w.Hkv
+    meta_bytes = float(nch.sum().item()) * w.Hkv * 512
+    off_h = off.cpu().numpy().astype(np.int64)
+    stream = torch.cuda.current_stream()
+    res = {}
+    for rule, kind, val in (("envelope", "tokens", 4096), ("envelope", "tokens", 8192),
+                            ("envelope", "chunks", 64), ("centroid", "chunks", 64),
+                            ("centroid", "chunks", 32)):
+        meta = kv.meta_buffer()
+        sa.sparse_attn_build_meta(kv, rule, 0, meta)
+        max_sel = val if kind == "chunks" else maxc
+        bud = sa.budget_topk(val) if kind == "chunks" else sa.budget_tokens(val)
+        ws = sa.make_workspace(kv, w.Hq, L * Bw, max_sel)
+        sel = torch.zeros((L * Bw, w.Hkv, max_sel), dtype=torch.int32, device=dev)
+        cnt = torch.zeros((L * Bw, w.Hkv), dtype=torch.int32, device=dev)
+        out = torch.zeros((L * Bw, w.Hq, D), dtype=torch.float32, device=dev)
+
+        def step():
+            sa.sparse_attn_decode_step(kv, meta, rule, q_all, bud, max_sel, 1.0 / math.sqrt(D), sel, cnt,
+                                       out, None, ws)
+
+        for _ in range(warmup):
+            step()
+        torch.cuda.synchronize()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(steps):
+            step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        ms = e0.elapsed_time(e1) / steps
+        if sa.sparse_attn_get_device_status(ws) != 0:
+            raise RuntimeError("TSA leg: device status set")
+        # tokens held by the kept chunks (host-side accounting of the outputs)
+        sel_h = sel.cpu().numpy()
+        cnt_h = cnt.cpu().numpy()
+        tok = 0
+        for r in range(L * Bw):
+            o = off_h[r]
+            for g in range(w.Hkv):
+                c = sel_h[r, g, :cnt_h[r, g]]
+                tok += int((np.minimum(o[c + 1], Nw) - o[c]).sum())
+        eff = (meta_bytes + tok * 512.0) / (ms * 1e-3)
+        name = f"{rule}/{'top' + str(val) + '_chunks' if kind == 'chunks' else 'tokens' + str(val)}"
+        res[name] = {"ms_per_step": round(ms, 4),
+                     "value": tok * (w.Hq // w.Hkv) / (ms * 1e-3),
+                     "tokens_attended_per_unit": round(tok / units, 1),
+                     "effective_bytes": int(meta_bytes + tok * 512.0),
+                     "eff_GBps": round(eff / 1e9, 1)}
+        del ws, sel, cnt, out, meta
+    return res
+
+
 class _Null:
     def __enter__(self):
         return self
@@ -586,6 +687,12 @@ def main():
         return 0
 
     import torch
+    if args.tsa_only:
+        dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", 0)))
+        torch.cuda.set_device(dev)
+        if rank == 0:
+            print(json.dumps({"tsa": tsa_leg(torch, dev, args.steps, max(3, args.warmup))}))
+        return 0
     if args.router_only:
         dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", 0)))
         torch.cuda.set_device(dev)
@@ -654,6 +761,10 @@ def main():
             "workload": "router-qwen2.5-7b-128k: 28:4 heads, 131072 tokens, 64-token blocks, "
                         "2048 rows in 32 tiles, k=32, rho=2, q=0.25",
             "bound": "tensor", "peak_tflops_bf16": peaks_tflops(), **r["router"]},
+        "tsa": None if r["tsa"] is None else {
+            "workload": "tsa-chunks-29.5k-b4: 48 layers x 4 sequences, 32:4 heads, 29504 tokens, "
+                        "chunks U{16..256} with per-chunk key offsets, one-launch decode step",
+            "bound": "hbm", **r["tsa"]},
     }
     print(json.dumps(line))
     return 0

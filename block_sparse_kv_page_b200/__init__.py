@@ -7,6 +7,7 @@ package fails if the library has not been built (no CPU fallback).
 from .ops import (KvCache, SparseAttnError, budget_ratio, budget_tokens, budget_topk,  # noqa: F401
                   lib, make_workspace, sparse_attn_build_meta, sparse_attn_decode,
                   sparse_attn_decode_static, sparse_attn_decode_step,
+                  sparse_attn_decode_step_append,
                   sparse_attn_get_device_status, sparse_attn_route, sparse_attn_select,
                   sparse_attn_status_string, sparse_attn_workspace_init,
                   sparse_attn_workspace_size)

@@ -97,6 +97,15 @@ sa_status launched(cudaError_t e) {
   return SA_OK;
 }
 
+// Tiles a unit is expected to hold under a token budget: the budget in 16-token
+// tiles plus an eighth for the ragged last tiles of the kept chunks.  It only
+// sizes the work split of the decode step (any actual count is handled).
+int token_budget_tiles(int token_budget) {
+  const long long t = ((long long)token_budget + 15) / 16;
+  const long long e = t + (t + 7) / 8;
+  return e < 1 ? 1 : (e > 0x3fffffff ? 0x3fffffff : (int)e);
+}
+
 int max_tiles_per_unit(const sa_kv_desc* kv, int max_sel) {
   const long long t = kv->page_size > 0 ? (long long)max_sel * (kv->page_size / 16)
                                         : (long long)max_sel * 16;
@@ -312,6 +321,8 @@ bool fill_select(SelectArgs* a, const sa_kv_desc* kv, const void* meta, sa_score
   a->status = reinterpret_cast<int*>(ws);
   a->splits = select_splits(kv->batch * kv->n_kv_heads, kv->max_pages, device_sm_count());
   a->meta_refresh = nullptr;
+  a->k_new = a->v_new = nullptr;
+  a->k_dst = a->v_dst = nullptr;
   return true;
 }
 
@@ -448,11 +459,12 @@ sa_status sparse_attn_decode(const sa_kv_desc* kv, const void* q, int32_t n_q_he
   return launched(launch_decode(a, (cudaStream_t)stream));
 }
 
-sa_status sparse_attn_decode_step(const sa_kv_desc* kv, void* meta, sa_score_rule rule,
-                                  const void* q, int32_t n_q_heads, const sa_budget* budget,
-                                  int32_t max_sel, float scale, int32_t* sel_idx,
-                                  int32_t* sel_count, float* out, float* lse, void* ws,
-                                  size_t ws_bytes, void* stream) {
+// The decode step with or without the append of the newest token's K/V.
+static sa_status decode_step(const sa_kv_desc* kv, void* meta, sa_score_rule rule,
+                             const void* q, int32_t n_q_heads, const void* k_new,
+                             const void* v_new, const sa_budget* budget, int32_t max_sel,
+                             float scale, int32_t* sel_idx, int32_t* sel_count, float* out,
+                             float* lse, void* ws, size_t ws_bytes, void* stream) {
   int G;
   sa_status s = check_select(kv, meta, rule, q, n_q_heads, budget, max_sel, sel_idx, sel_count,
                              nullptr, &G);
@@ -465,7 +477,12 @@ sa_status sparse_attn_decode_step(const sa_kv_desc* kv, void* meta, sa_score_rul
   const unsigned long long kv_rows = (unsigned long long)kv->batch * kv->n_kv_heads * kv->cap_tokens;
   if (kv_rows > 0x7fffffffULL) return SA_ERR_UNSUPPORTED;  // TMA row coordinates are int32
   const int sm = device_sm_count();
-  const DecodePlan plan = decode_plan((int)units, max_tiles_per_unit(kv, max_sel), sm);
+  int plan_tiles = max_tiles_per_unit(kv, max_sel);
+  if (budget->kind == SA_BUDGET_TOKENS) {  // the budget, not max_sel, bounds what is attended
+    const int t = token_budget_tiles(budget->token_budget);
+    if (t < plan_tiles) plan_tiles = t;
+  }
+  const DecodePlan plan = decode_plan((int)units, plan_tiles, sm);
   const size_t sel_bytes = select_scratch(kv);
   const size_t need = kScratch + sel_bytes + decode_scratch(plan);
   if ((s = check_ws(ws, ws_bytes, need)) != SA_OK) return s;
@@ -481,12 +498,38 @@ sa_status sparse_attn_decode_step(const sa_kv_desc* kv, void* meta, sa_score_rul
                    reinterpret_cast<uint32_t*>(w + 256) + units, reinterpret_cast<int*>(ws), plan))
     return SA_ERR_CUDA;
   a.sel.meta_refresh = static_cast<unsigned char*>(meta);
+  if (k_new) {
+    a.sel.k_new = k_new;
+    a.sel.v_new = v_new;
+    a.sel.k_dst = const_cast<void*>(kv->k);
+    a.sel.v_dst = const_cast<void*>(kv->v);
+  }
   a.queue = reinterpret_cast<uint32_t*>(w + kQueueStep);
   const long long n_score = units * a.sel.splits, n_dec = plan.items;
   if (n_score + n_dec > 0x7fffffffLL) return SA_ERR_UNSUPPORTED;
   a.n_score = (int)n_score;
   a.n_dec = (int)n_dec;
   return launched(launch_step(a, (cudaStream_t)stream));
+}
+
+sa_status sparse_attn_decode_step(const sa_kv_desc* kv, void* meta, sa_score_rule rule,
+                                  const void* q, int32_t n_q_heads, const sa_budget* budget,
+                                  int32_t max_sel, float scale, int32_t* sel_idx,
+                                  int32_t* sel_count, float* out, float* lse, void* ws,
+                                  size_t ws_bytes, void* stream) {
+  return decode_step(kv, meta, rule, q, n_q_heads, nullptr, nullptr, budget, max_sel, scale, sel_idx,
+                     sel_count, out, lse, ws, ws_bytes, stream);
+}
+
+sa_status sparse_attn_decode_step_append(const sa_kv_desc* kv, void* meta, sa_score_rule rule,
+                                         const void* q, int32_t n_q_heads, const void* k_new,
+                                         const void* v_new, const sa_budget* budget,
+                                         int32_t max_sel, float scale, int32_t* sel_idx,
+                                         int32_t* sel_count, float* out, float* lse, void* ws,
+                                         size_t ws_bytes, void* stream) {
+  if (!k_new || !v_new || !aligned(k_new, 8) || !aligned(v_new, 8)) return SA_ERR_INVALID;
+  return decode_step(kv, meta, rule, q, n_q_heads, k_new, v_new, budget, max_sel, scale, sel_idx,
+                     sel_count, out, lse, ws, ws_bytes, stream);
 }
 
 sa_status sparse_attn_route(const sa_kv_desc* kv, const void* meta, sa_score_rule rule,

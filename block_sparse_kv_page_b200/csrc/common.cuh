@@ -110,6 +110,10 @@ SA_DEV void mbar_arrive(uint64_t* bar) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];\n" ::"r"(smem_addr(bar)) : "memory");
 }
 SA_DEV void fence_proxy_async() { asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory"); }
+// Orders this thread's generic-proxy global accesses with its async-proxy
+// (TMA) ones: global data written with plain stores in the same launch and
+// read by a later TMA copy takes one on each side of the handoff.
+SA_DEV void fence_proxy_async_global() { asm volatile("fence.proxy.async.global;\n" ::: "memory"); }
 SA_DEV void prefetch_tmap(const void* tmap) {
   asm volatile("prefetch.tensormap [%0];\n" ::"l"(tmap) : "memory");
 }

@@ -70,6 +70,13 @@ struct SelectArgs {
   int* status;
   int splits;
   unsigned char* meta_refresh;  // decode step: writable metadata (same array as meta)
+  // decode step with append (all null otherwise): the newest token's key and
+  // value, bf16 [B][Hkv][128], stored into the cache (k_dst / v_dst = the
+  // cache arrays) at row seq_len[b] - 1
+  const void* k_new;
+  const void* v_new;
+  void* k_dst;
+  void* v_dst;
 };
 cudaError_t launch_select(const SelectArgs& a, cudaStream_t st);
 

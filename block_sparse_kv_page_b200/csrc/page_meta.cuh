@@ -22,9 +22,12 @@ struct PageMetaLane {
 };
 
 // k_lane = first key row of the (sequence, KV head) + 4 * lane elements;
-// the page covers rows [s, e), e > s.
+// the page covers rows [s, e), e > s.  With use_last, row e - 1 is taken from
+// `last` (this lane's 4 elements) instead of memory: the fused step appends
+// the newest key and folds it in without reading it back.
 template <int RULE>
-SA_DEV PageMetaLane page_meta_lane(const __nv_bfloat16* k_lane, int s, int e) {
+SA_DEV PageMetaLane page_meta_lane(const __nv_bfloat16* k_lane, int s, int e, bool use_last = false,
+                                   uint2 last = make_uint2(0u, 0u)) {
   float mn[4], mx[4];
   double sm[4];
 #pragma unroll
@@ -39,8 +42,9 @@ SA_DEV PageMetaLane page_meta_lane(const __nv_bfloat16* k_lane, int s, int e) {
     uint2 r[16];
 #pragma unroll
     for (int x = 0; x < 16; ++x)
-      r[x] = x < n ? __ldg(reinterpret_cast<const uint2*>(k_lane + (size_t)(t + x) * kHeadDim))
-                   : make_uint2(0u, 0u);
+      r[x] = x >= n                    ? make_uint2(0u, 0u)
+             : use_last && t + x == e - 1 ? last
+                                          : __ldg(reinterpret_cast<const uint2*>(k_lane + (size_t)(t + x) * kHeadDim));
 #pragma unroll
     for (int x = 0; x < 16; ++x) {
       if (x < n) {

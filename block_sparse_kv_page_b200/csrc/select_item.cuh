@@ -588,10 +588,23 @@ SA_DEV void select_item(const SelectArgs& a, const int u, const int split, const
     unsigned char* st = ring + (g_it % kStages) * kTileBytes;
     const int t = t_begin + warp + it * kWarps;
     if (t == t_new) {
+      // with append: store the newest key and value at row N - 1 (lane l
+      // owns elements 4l .. 4l + 3), and use the key without reading it back
+      const bool app = a.k_new != nullptr;
+      uint2 knew = make_uint2(0u, 0u);
+      if (app) {
+        const size_t src = (size_t)u * kHeadDim + lane * 4;
+        const size_t dst = ((size_t)u * a.kv.cap + (size_t)(N - 1)) * kHeadDim + lane * 4;
+        knew = __ldg(reinterpret_cast<const uint2*>(static_cast<const __nv_bfloat16*>(a.k_new) + src));
+        const uint2 vnew = __ldg(reinterpret_cast<const uint2*>(static_cast<const __nv_bfloat16*>(a.v_new) + src));
+        *reinterpret_cast<uint2*>(static_cast<__nv_bfloat16*>(a.k_dst) + dst) = knew;
+        *reinterpret_cast<uint2*>(static_cast<__nv_bfloat16*>(a.v_dst) + dst) = vnew;
+        fence_proxy_async_global();  // the decode items read the row with TMA
+      }
       // rebuild the newest page's metadata, store it, patch the staged row
       const __nv_bfloat16* k_lane = reinterpret_cast<const __nv_bfloat16*>(a.kv.k) +
                                     ((size_t)u * a.kv.cap) * kHeadDim + lane * 4;
-      const PageMetaLane m = page_meta_lane<RULE>(k_lane, r_s, r_e);
+      const PageMetaLane m = page_meta_lane<RULE>(k_lane, r_s, r_e, app, knew);
       store_page_meta<RULE>(a.meta_refresh + ((size_t)u * a.kv.max_pages + p_new) * kMetaBytes, m, lane);
       const int r = p_new & 15;
       if (RULE == 0) {

@@ -112,6 +112,7 @@ __global__ void __launch_bounds__(kThreads, SA_STEP_CTAS_PER_SM)
     } else {
       int u, split;
       dec::item_unit(a.dec, item - a.n_score, u, split);
+      if (a.sel.k_new != nullptr && lane == 0) fence_proxy_async_global();  // appended rows, then TMA
       dec::decode_item(a.dec, u, split, D, ws);
     }
     fence_proxy_async();  // generic writes to the ring (keys, merge) before the next TMA writes

@@ -160,6 +160,29 @@ def sparse_attn_decode_step(kv: KvCache, meta: torch.Tensor, rule, q: torch.Tens
            "sparse_attn_decode_step")
 
 
+def sparse_attn_decode_step_append(kv: KvCache, meta: torch.Tensor, rule, q: torch.Tensor,
+                                   k_new: torch.Tensor, v_new: torch.Tensor, budget: sa_budget,
+                                   max_sel: int, scale: float, sel_idx: torch.Tensor,
+                                   sel_count: torch.Tensor, out: torch.Tensor, lse: torch.Tensor | None,
+                                   ws: torch.Tensor, stream=None) -> None:
+    """The decode step with the newest token's key and value (bf16 [B, Hkv, 128])
+    stored into the cache at row seq_len - 1 inside the same launch."""
+    if q.dtype != torch.bfloat16 or not q.is_contiguous():
+        raise ValueError("q must be contiguous bf16 [B, Hq, 128]")
+    for name, t in (("k_new", k_new), ("v_new", v_new)):
+        if t.dtype != torch.bfloat16 or not t.is_contiguous() or tuple(t.shape) != (kv.batch, kv.k.shape[1], 128):
+            raise ValueError(f"{name} must be contiguous bf16 [B, Hkv, 128]")
+    if out.dtype != torch.float32 or not out.is_contiguous():
+        raise ValueError("out must be contiguous fp32")
+    _check(lib.sparse_attn_decode_step_append(C.byref(kv.desc), meta.data_ptr(), _rule(rule), q.data_ptr(),
+                                              q.shape[-2], k_new.data_ptr(), v_new.data_ptr(),
+                                              C.byref(budget), int(max_sel), float(scale),
+                                              sel_idx.data_ptr(), sel_count.data_ptr(), out.data_ptr(),
+                                              _ptr(lse), ws.data_ptr(), ws.numel() * ws.element_size(),
+                                              _stream(stream)),
+           "sparse_attn_decode_step_append")
+
+
 def sparse_attn_decode_static(kv: KvCache, q: torch.Tensor, n_q_rows: int, q_pos0: int,
                               tile_rows: int, scale: float, idx: torch.Tensor, count: torch.Tensor,
                               max_sel: int, out: torch.Tensor, lse: torch.Tensor | None,

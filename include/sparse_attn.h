@@ -179,6 +179,11 @@ sa_status sparse_attn_decode(const sa_kv_desc* kv, const void* q, int32_t n_q_he
  *                      sel_idx, sel_count, NULL, ...);
  *   sparse_attn_decode(kv, q, n_q_heads, B, 0, 1, scale, sel_idx, sel_count,
  *                      max_sel, out, lse, ...);
+ * Results are bit-identical to that sequence, except under a token budget,
+ * where the step divides the attention work by the budget (the separate decode
+ * call does not know it and divides by max_sel): out and lse then agree to
+ * rounding (the split partials merge in a different grouping), meta, sel_idx
+ * and sel_count exactly.
  * meta is read and written (the metadata of the page or chunk holding token
  * N_b - 1 is rebuilt from K; every other page must be current).  sel_idx and
  * sel_count are written as by sparse_attn_select.  Work items of the three
@@ -192,6 +197,26 @@ sa_status sparse_attn_decode_step(const sa_kv_desc* kv, void* meta, sa_score_rul
                                   int32_t max_sel, float scale, int32_t* sel_idx,
                                   int32_t* sel_count, float* out, float* lse, void* ws,
                                   size_t ws_bytes, void* stream);
+
+/* (e') The decode step with the append of the newest token fused in
+ * ([OFFLINE] "The comparison": the cache grows by one token per decode step,
+ * and that token is scored and attended in the same step).  Same as
+ * sparse_attn_decode_step, except that row N_b - 1 of the cache does not have
+ * to hold the newest token yet: k_new and v_new (device, bf16
+ * [B][n_kv_heads][128], 8-byte aligned, read only) are stored into the cache
+ * at row N_b - 1 of every (sequence, KV head), so kv->k and kv->v must be
+ * writable.  The newest page's metadata is rebuilt with k_new, and the
+ * attention reads the appended row.  Results (meta, sel_idx, sel_count, out,
+ * lse) and the cache contents afterwards are identical to storing the row
+ * first and calling sparse_attn_decode_step.  A (sequence, KV head) whose
+ * length is out of range is not appended (SA_ERR_DEVICE_CHECK).  Null or
+ * misaligned k_new / v_new: SA_ERR_INVALID. */
+sa_status sparse_attn_decode_step_append(const sa_kv_desc* kv, void* meta, sa_score_rule rule,
+                                         const void* q, int32_t n_q_heads, const void* k_new,
+                                         const void* v_new, const sa_budget* budget,
+                                         int32_t max_sel, float scale, int32_t* sel_idx,
+                                         int32_t* sel_count, float* out, float* lse, void* ws,
+                                         size_t ws_bytes, void* stream);
 
 /* (d) Uncertainty router over query tiles ([ROUTER] "Methodologie" steps 2-5).
  * B == 1, fixed blocks (page_size = block size).  q bf16 [n_q_rows][n_q_heads][128]

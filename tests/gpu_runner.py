@@ -81,11 +81,12 @@ def run_gpu(layer, *, page_size: int, rule: str, budget: dict, scale: float,
 
 def run_step(layer, *, page_size: int, rule: str, budget: dict, scale: float,
              max_pages: int | None = None, max_sel: int | None = None, ws=None, repeat: int = 1,
-             stale: bool = True):
+             stale: bool = True, append=None):
     """One-launch decode step through the C ABI.  With `stale`, the metadata is
     first built for the cache as it stood before its newest token (seq_len - 1;
     pages never built hold a fill pattern), so the step's own refresh of the
-    newest page is what makes the metadata current."""
+    newest page is what makes the metadata current.  append = (k_new, v_new):
+    run the step that stores the newest token's key and value itself."""
     B, Hkv, cap, D = layer.k.shape
     Hq = layer.q.shape[1]
     if max_pages is None:
@@ -115,8 +116,13 @@ def run_step(layer, *, page_size: int, rule: str, budget: dict, scale: float,
         sel_count = torch.full((B, Hkv), -7, dtype=torch.int32, device=dev)
         out = torch.full((B, Hq, 128), float("nan"), dtype=torch.float32, device=dev)
         lse = torch.full((B, Hq), float("nan"), dtype=torch.float32, device=dev)
-        sa.sparse_attn_decode_step(kv, meta, rule, layer.q, budget_struct(budget), max_sel, scale,
-                                   sel_idx, sel_count, out, lse, ws)
+        if append is None:
+            sa.sparse_attn_decode_step(kv, meta, rule, layer.q, budget_struct(budget), max_sel, scale,
+                                       sel_idx, sel_count, out, lse, ws)
+        else:
+            sa.sparse_attn_decode_step_append(kv, meta, rule, layer.q, append[0], append[1],
+                                              budget_struct(budget), max_sel, scale, sel_idx, sel_count,
+                                              out, lse, ws)
         torch.cuda.synchronize()
         results.append(dict(sel_idx=sel_idx.cpu(), sel_count=sel_count.cpu(), out=out.cpu(),
                             lse=lse.cpu()))

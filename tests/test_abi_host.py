@@ -132,6 +132,21 @@ def test_decode_step_validation(lib, abi):
     assert call(budget=tokens) == abi.SA_ERR_UNSUPPORTED  # token budgets need chunks
 
 
+def test_decode_step_append_validation(lib, abi):
+    ok = _desc(abi)
+    topk = abi.sa_budget(abi.SA_BUDGET_TOPK, 8, 0.0, 0, 0, 0, 0)
+
+    def call(k_new=0x90000, v_new=0xa0000, max_sel=16, ws_bytes=1 << 30):
+        return lib.sparse_attn_decode_step_append(C.byref(ok), 0x40000, 0, 0x50000, 32, k_new, v_new,
+                                                  C.byref(topk), max_sel, 0.088, 0x60000, 0x70000,
+                                                  0x80000, None, 0x100000, ws_bytes, None)
+    assert call(k_new=0) == abi.SA_ERR_INVALID
+    assert call(v_new=0) == abi.SA_ERR_INVALID
+    assert call(k_new=0x90004) == abi.SA_ERR_INVALID      # not 8-byte aligned
+    assert call(max_sel=4) == abi.SA_ERR_INVALID          # the step's own checks still apply
+    assert call(ws_bytes=4096) == abi.SA_ERR_WORKSPACE
+
+
 def test_build_meta_validation(lib, abi):
     ok = _desc(abi)
     assert lib.sparse_attn_build_meta(C.byref(ok), 7, 0, 0x40000, None) == abi.SA_ERR_INVALID

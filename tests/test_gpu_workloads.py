@@ -83,6 +83,32 @@ def test_tsa_chunks_full(cuda_dev, R, budget):
     print(f"\ntokens@{budget}: {st}")
 
 
+@pytest.mark.parametrize("rule,k", [("envelope", 64), ("centroid", 64), ("centroid", 32)])
+def test_tsa_chunk_count_full(cuda_dev, R, rule, k):
+    """TSA with a chunk-count budget (top 64 / top 32 chunks), min/max and
+    centroid scoring, on the full 29,504-token batch-4 workload."""
+    layers = [DG.workload3_layer(l, cuda_dev) for l in (0, 47)]
+    lay = _stack(layers)
+    bd = {"kind": "topk", "k": k}
+    g = R.run_gpu(lay, page_size=0, rule=rule, budget=bd, scale=SCALE)
+    assert g["status"] == 0
+    assert (g["sel_count"] == k).all()
+    st = R.check_layer(lay, g, page_size=0, rule=rule, budget=bd, scale=SCALE)
+    assert st["units"] == 8 * 4
+    assert st["max_out_err"] < 1e-4
+    print(f"\n{rule} top-{k} chunks: {st}")
+
+
+def test_tsa_centroid_tokens_full(cuda_dev, R):
+    layers = [DG.workload3_layer(l, cuda_dev) for l in (3,)]
+    lay = _stack(layers)
+    bd = {"kind": "tokens", "budget": 4096}
+    g = R.run_gpu(lay, page_size=0, rule="centroid", budget=bd, scale=SCALE)
+    assert g["status"] == 0
+    st = R.check_layer(lay, g, page_size=0, rule="centroid", budget=bd, scale=SCALE)
+    assert st["units"] == 4 * 4
+
+
 def test_tsa_full_budget_equals_dense(cuda_dev, R):
     lay = DG.workload3_layer(5, cuda_dev, N=16384)
     bd = {"kind": "tokens", "budget": 16384}
