@@ -444,6 +444,29 @@ def run_gpu_arm(args, rank, world, dist):
     d2h = out_h.numel() * 4
     if sa.sparse_attn_get_device_status(ws) != 0:
         raise RuntimeError("device status set after the end-to-end steps")
+    # the same, reading the output back as bf16 (the fp32 result rounded)
+    e2e_bf16 = None
+    if args.mode == "step":
+        out_bf = torch.empty(out.shape, dtype=torch.bfloat16, device=dev)
+        outbf_h = torch.empty(out.shape, dtype=torch.bfloat16).pin_memory()
+
+        def e2e_bf16_step():
+            dev_in.copy_(host_in, non_blocking=True)
+            sa.sparse_attn_decode_step_append(kv, metas[args.rule], args.rule, q_d, knew_d, vnew_d, budget,
+                                              k, scale, sel, cnt, out_bf, lse, ws)
+            outbf_h.copy_(out_bf, non_blocking=True)
+
+        for _ in range(args.warmup):
+            e2e_bf16_step()
+        barrier()
+        a0.record(stream)
+        for _ in range(args.steps):
+            e2e_bf16_step()
+        a1.record(stream)
+        torch.cuda.synchronize()
+        ms_bf = max_over_ranks(a0.elapsed_time(a1) / args.steps, dist, dev)
+        e2e_bf16 = {"ms_per_step": round(ms_bf, 5), "h2d_bytes_per_step": h2d,
+                    "d2h_bytes_per_step": out_h.numel() * 2}
 
     # ---- secondary measurements (same timing rules), labelled
     extra = {}
@@ -463,7 +486,7 @@ def run_gpu_arm(args, rank, world, dist):
     if not args.no_extra:
         router = router_leg(torch, dev, max(5, min(args.steps, 50)), max(3, args.warmup))
         tsa = tsa_leg(torch, dev, max(10, min(args.steps, 50)), max(3, args.warmup))
-    return dict(ms=ms, value=value, kern=kern, clocks=clocks.summary(), e2e_ms=e2e_ms, h2d=h2d,
+    return dict(ms=ms, value=value, kern=kern, clocks=clocks.summary(), e2e_ms=e2e_ms, e2e_bf16=e2e_bf16, h2d=h2d,
                 d2h=d2h, meta_bytes=meta_bytes, kv_bytes=kv_bytes, extra=extra, router=router, tsa=tsa,
                 launches_per_step=MODES[args.mode])
 
@@ -755,6 +778,9 @@ def main():
         "e2e": {"value": whole_job_value(HQ * args.budget * LAYERS * B, world, r["e2e_ms"]), "unit": UNIT,
                 "ms_per_step": round(r["e2e_ms"], 5), "h2d_bytes_per_step": r["h2d"],
                 "d2h_bytes_per_step": r["d2h"]},
+        "e2e_bf16_out": None if r["e2e_bf16"] is None else {
+            "value": whole_job_value(HQ * args.budget * LAYERS * B, world, r["e2e_bf16"]["ms_per_step"]),
+            "unit": UNIT, **r["e2e_bf16"]},
         "gpu_launches": r["launches_per_step"] * args.steps,
         "cpu_baseline": cpu, "modes": r["extra"],
         "router": None if r["router"] is None else {

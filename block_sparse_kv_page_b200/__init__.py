@@ -13,4 +13,5 @@ from .ops import (KvCache, SparseAttnError, budget_ratio, budget_tokens, budget_
                   sparse_attn_workspace_size)
 from ._abi import (SA_BUDGET_RATIO, SA_BUDGET_TOKENS, SA_BUDGET_TOPK, SA_ERR_CUDA,  # noqa: F401
                    SA_ERR_DEVICE_CHECK, SA_ERR_INVALID, SA_ERR_TIMEOUT, SA_ERR_UNSUPPORTED,
-                   SA_ERR_WORKSPACE, SA_OK, SA_SCORE_CENTROID, SA_SCORE_ENVELOPE)
+                   SA_ERR_WORKSPACE, SA_OK, SA_OUT_BF16, SA_OUT_F32, SA_SCORE_CENTROID,
+                   SA_SCORE_ENVELOPE)

@@ -21,6 +21,9 @@ SA_ERR_DEVICE_CHECK = 6
 SA_SCORE_ENVELOPE = 0
 SA_SCORE_CENTROID = 1
 
+SA_OUT_F32 = 0
+SA_OUT_BF16 = 1
+
 SA_BUDGET_TOPK = 0
 SA_BUDGET_RATIO = 1
 SA_BUDGET_TOKENS = 2
@@ -72,7 +75,7 @@ PROTOTYPES = {
     "sparse_attn_decode_step_append": (C.c_int, [C.POINTER(sa_kv_desc), C.c_void_p, C.c_int, C.c_void_p,
                                                  C.c_int32, C.c_void_p, C.c_void_p, C.POINTER(sa_budget),
                                                  C.c_int32, C.c_float, C.c_void_p, C.c_void_p, C.c_void_p,
-                                                 C.c_void_p, C.c_void_p, C.c_size_t, C.c_void_p]),
+                                                 C.c_int, C.c_void_p, C.c_void_p, C.c_size_t, C.c_void_p]),
     "sparse_attn_route": (C.c_int, [C.POINTER(sa_kv_desc), C.c_void_p, C.c_int, C.c_void_p, C.c_int32,
                                     C.c_int32, C.c_int32, C.c_int32, C.c_int32, C.c_int32, C.c_float,
                                     C.c_void_p, C.c_void_p, C.c_void_p, C.c_void_p, C.c_void_p, C.c_void_p,

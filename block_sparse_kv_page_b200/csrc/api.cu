@@ -348,6 +348,7 @@ bool fill_decode(DecodeArgs* a, const sa_kv_desc* kv, const void* q, int n_q_hea
   a->count = count;
   a->max_sel = max_sel;
   a->out = out;
+  a->out_bf16 = nullptr;
   a->lse = lse;
   a->ws_part = ws_part;
   a->ws_count = ws_count;
@@ -463,8 +464,8 @@ sa_status sparse_attn_decode(const sa_kv_desc* kv, const void* q, int32_t n_q_he
 static sa_status decode_step(const sa_kv_desc* kv, void* meta, sa_score_rule rule,
                              const void* q, int32_t n_q_heads, const void* k_new,
                              const void* v_new, const sa_budget* budget, int32_t max_sel,
-                             float scale, int32_t* sel_idx, int32_t* sel_count, float* out,
-                             float* lse, void* ws, size_t ws_bytes, void* stream) {
+                             float scale, int32_t* sel_idx, int32_t* sel_count, void* out,
+                             bool out_bf16, float* lse, void* ws, size_t ws_bytes, void* stream) {
   int G;
   sa_status s = check_select(kv, meta, rule, q, n_q_heads, budget, max_sel, sel_idx, sel_count,
                              nullptr, &G);
@@ -493,10 +494,12 @@ static sa_status decode_step(const sa_kv_desc* kv, void* meta, sa_score_rule rul
   char* w = reinterpret_cast<char*>(ws);
   if (!fill_select(&a.sel, kv, meta, rule, q, n_q_heads, G, budget, max_sel, sel_idx, sel_count,
                    nullptr, ws) ||
-      !fill_decode(&a.dec, kv, q, n_q_heads, G, scale, sel_idx, sel_count, max_sel, out, lse,
+      !fill_decode(&a.dec, kv, q, n_q_heads, G, scale, sel_idx, sel_count, max_sel,
+                   out_bf16 ? nullptr : static_cast<float*>(out), lse,
                    reinterpret_cast<float*>(w + kScratch + sel_bytes),
                    reinterpret_cast<uint32_t*>(w + 256) + units, reinterpret_cast<int*>(ws), plan))
     return SA_ERR_CUDA;
+  if (out_bf16) a.dec.out_bf16 = static_cast<__nv_bfloat16*>(out);
   a.sel.meta_refresh = static_cast<unsigned char*>(meta);
   if (k_new) {
     a.sel.k_new = k_new;
@@ -518,18 +521,19 @@ sa_status sparse_attn_decode_step(const sa_kv_desc* kv, void* meta, sa_score_rul
                                   int32_t* sel_count, float* out, float* lse, void* ws,
                                   size_t ws_bytes, void* stream) {
   return decode_step(kv, meta, rule, q, n_q_heads, nullptr, nullptr, budget, max_sel, scale, sel_idx,
-                     sel_count, out, lse, ws, ws_bytes, stream);
+                     sel_count, out, false, lse, ws, ws_bytes, stream);
 }
 
 sa_status sparse_attn_decode_step_append(const sa_kv_desc* kv, void* meta, sa_score_rule rule,
                                          const void* q, int32_t n_q_heads, const void* k_new,
                                          const void* v_new, const sa_budget* budget,
                                          int32_t max_sel, float scale, int32_t* sel_idx,
-                                         int32_t* sel_count, float* out, float* lse, void* ws,
-                                         size_t ws_bytes, void* stream) {
+                                         int32_t* sel_count, void* out, sa_out_dtype out_dtype,
+                                         float* lse, void* ws, size_t ws_bytes, void* stream) {
   if (!k_new || !v_new || !aligned(k_new, 8) || !aligned(v_new, 8)) return SA_ERR_INVALID;
+  if (out_dtype != SA_OUT_F32 && out_dtype != SA_OUT_BF16) return SA_ERR_INVALID;
   return decode_step(kv, meta, rule, q, n_q_heads, k_new, v_new, budget, max_sel, scale, sel_idx,
-                     sel_count, out, lse, ws, ws_bytes, stream);
+                     sel_count, out, out_dtype == SA_OUT_BF16, lse, ws, ws_bytes, stream);
 }
 
 sa_status sparse_attn_route(const sa_kv_desc* kv, const void* meta, sa_score_rule rule,
@@ -739,6 +743,7 @@ extern "C" sa_status sparse_attn_decode_static(const sa_kv_desc* kv, const void*
   a.count = count;
   a.max_sel = max_sel;
   a.out = out;
+  a.out_bf16 = nullptr;
   a.lse = lse;
   a.ws_part = reinterpret_cast<float*>(scratch + kStaticPartOff);
   a.ws_count = reinterpret_cast<uint32_t*>(scratch + 256);

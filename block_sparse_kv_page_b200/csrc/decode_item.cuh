@@ -104,6 +104,24 @@ SA_DEV void item_unit(const DecodeArgs& a, const int j, int& u, int& split) {
   }
 }
 
+// Output row `row`, dims d0 .. d0 + kDimsPerThread - 1 = A * inv, as fp32 or
+// rounded to bf16 (round to nearest even).
+SA_DEV void store_out(const DecodeArgs& a, size_t row, int d0, const float (&A)[kDimsPerThread],
+                      float inv) {
+  if (a.out_bf16) {
+    __nv_bfloat16* o = a.out_bf16 + row * kHeadDim + d0;
+#pragma unroll
+    for (int x = 0; x < kDimsPerThread; x += 4)
+      *reinterpret_cast<uint2*>(o + x) = make_uint2(pack_bf16(A[x] * inv, A[x + 1] * inv),
+                                                    pack_bf16(A[x + 2] * inv, A[x + 3] * inv));
+  } else {
+    float* o = a.out + row * kHeadDim + d0;
+#pragma unroll
+    for (int x = 0; x < kDimsPerThread; x += 4)
+      *reinterpret_cast<float4*>(o + x) = make_float4(A[x] * inv, A[x + 1] * inv, A[x + 2] * inv, A[x + 3] * inv);
+  }
+}
+
 SA_DEV void decode_item(const DecodeArgs& a, const int u, const int split, const Smem& sm,
                         WarpState& ws) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -378,10 +396,7 @@ SA_DEV void decode_item(const DecodeArgs& a, const int u, const int split, const
   if (splits == 1) {
     if (h < G) {
       const float inv = L > 0.f ? 1.f / L : 0.f;
-      float* o = a.out + out_row * kHeadDim + d0;
-#pragma unroll
-      for (int x = 0; x < kDimsPerThread; x += 4)
-        *reinterpret_cast<float4*>(o + x) = make_float4(A[x] * inv, A[x + 1] * inv, A[x + 2] * inv, A[x + 3] * inv);
+      store_out(a, out_row, d0, A, inv);
       if (a.lse && d0 == 0) a.lse[out_row] = L > 0.f ? M * kLn2 + logf(L) : ninf;
     }
     return;
@@ -450,10 +465,7 @@ SA_DEV void decode_item(const DecodeArgs& a, const int u, const int split, const
     MM = nm;
   }
   const float inv = LL > 0.f ? 1.f / LL : 0.f;
-  float* o = a.out + out_row * kHeadDim + d0;
-#pragma unroll
-  for (int x = 0; x < kDimsPerThread; x += 4)
-    *reinterpret_cast<float4*>(o + x) = make_float4(AA[x] * inv, AA[x + 1] * inv, AA[x + 2] * inv, AA[x + 3] * inv);
+  store_out(a, out_row, d0, AA, inv);
   if (a.lse && d0 == 0) a.lse[out_row] = LL > 0.f ? MM * kLn2 + logf(LL) : ninf;
 }
 

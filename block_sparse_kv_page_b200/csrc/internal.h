@@ -92,6 +92,7 @@ struct DecodeArgs {
   const int32_t* count;
   int max_sel;
   float* out;
+  __nv_bfloat16* out_bf16;    // non-null: the output goes here, rounded to bf16, instead of `out`
   float* lse;
   float* ws_part;
   uint32_t* ws_count;

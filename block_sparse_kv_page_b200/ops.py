@@ -166,20 +166,22 @@ def sparse_attn_decode_step_append(kv: KvCache, meta: torch.Tensor, rule, q: tor
                                    sel_count: torch.Tensor, out: torch.Tensor, lse: torch.Tensor | None,
                                    ws: torch.Tensor, stream=None) -> None:
     """The decode step with the newest token's key and value (bf16 [B, Hkv, 128])
-    stored into the cache at row seq_len - 1 inside the same launch."""
+    stored into the cache at row seq_len - 1 inside the same launch.  out is
+    fp32 or bf16 [B, Hq, 128] (bf16: the fp32 result rounded to nearest even)."""
     if q.dtype != torch.bfloat16 or not q.is_contiguous():
         raise ValueError("q must be contiguous bf16 [B, Hq, 128]")
     for name, t in (("k_new", k_new), ("v_new", v_new)):
         if t.dtype != torch.bfloat16 or not t.is_contiguous() or tuple(t.shape) != (kv.batch, kv.k.shape[1], 128):
             raise ValueError(f"{name} must be contiguous bf16 [B, Hkv, 128]")
-    if out.dtype != torch.float32 or not out.is_contiguous():
-        raise ValueError("out must be contiguous fp32")
+    if out.dtype not in (torch.float32, torch.bfloat16) or not out.is_contiguous():
+        raise ValueError("out must be contiguous fp32 or bf16")
+    out_dtype = _abi.SA_OUT_BF16 if out.dtype == torch.bfloat16 else _abi.SA_OUT_F32
     _check(lib.sparse_attn_decode_step_append(C.byref(kv.desc), meta.data_ptr(), _rule(rule), q.data_ptr(),
                                               q.shape[-2], k_new.data_ptr(), v_new.data_ptr(),
                                               C.byref(budget), int(max_sel), float(scale),
                                               sel_idx.data_ptr(), sel_count.data_ptr(), out.data_ptr(),
-                                              _ptr(lse), ws.data_ptr(), ws.numel() * ws.element_size(),
-                                              _stream(stream)),
+                                              out_dtype, _ptr(lse), ws.data_ptr(),
+                                              ws.numel() * ws.element_size(), _stream(stream)),
            "sparse_attn_decode_step_append")
 
 

@@ -198,6 +198,12 @@ sa_status sparse_attn_decode_step(const sa_kv_desc* kv, void* meta, sa_score_rul
                                   int32_t* sel_count, float* out, float* lse, void* ws,
                                   size_t ws_bytes, void* stream);
 
+/* Element type of the attention output of sparse_attn_decode_step_append. */
+typedef enum {
+  SA_OUT_F32 = 0,   /* fp32 [B][Hq][128] */
+  SA_OUT_BF16 = 1   /* bf16 [B][Hq][128]: the fp32 result rounded to nearest even */
+} sa_out_dtype;
+
 /* (e') The decode step with the append of the newest token fused in
  * ([OFFLINE] "The comparison": the cache grows by one token per decode step,
  * and that token is scored and attended in the same step).  Same as
@@ -208,15 +214,18 @@ sa_status sparse_attn_decode_step(const sa_kv_desc* kv, void* meta, sa_score_rul
  * writable.  The newest page's metadata is rebuilt with k_new, and the
  * attention reads the appended row.  Results (meta, sel_idx, sel_count, out,
  * lse) and the cache contents afterwards are identical to storing the row
- * first and calling sparse_attn_decode_step.  A (sequence, KV head) whose
- * length is out of range is not appended (SA_ERR_DEVICE_CHECK).  Null or
- * misaligned k_new / v_new: SA_ERR_INVALID. */
+ * first and calling sparse_attn_decode_step.  out (16-byte aligned) holds
+ * out_dtype elements: SA_OUT_F32 as in sparse_attn_decode_step, or SA_OUT_BF16,
+ * the same fp32 values rounded to bf16 (half the bytes to read back; lse stays
+ * fp32).  A (sequence, KV head) whose length is out of range is not appended
+ * (SA_ERR_DEVICE_CHECK).  Null or misaligned k_new / v_new, or an unknown
+ * out_dtype: SA_ERR_INVALID. */
 sa_status sparse_attn_decode_step_append(const sa_kv_desc* kv, void* meta, sa_score_rule rule,
                                          const void* q, int32_t n_q_heads, const void* k_new,
                                          const void* v_new, const sa_budget* budget,
                                          int32_t max_sel, float scale, int32_t* sel_idx,
-                                         int32_t* sel_count, float* out, float* lse, void* ws,
-                                         size_t ws_bytes, void* stream);
+                                         int32_t* sel_count, void* out, sa_out_dtype out_dtype,
+                                         float* lse, void* ws, size_t ws_bytes, void* stream);
 
 /* (d) Uncertainty router over query tiles ([ROUTER] "Methodologie" steps 2-5).
  * B == 1, fixed blocks (page_size = block size).  q bf16 [n_q_rows][n_q_heads][128]

@@ -81,7 +81,7 @@ def run_gpu(layer, *, page_size: int, rule: str, budget: dict, scale: float,
 
 def run_step(layer, *, page_size: int, rule: str, budget: dict, scale: float,
              max_pages: int | None = None, max_sel: int | None = None, ws=None, repeat: int = 1,
-             stale: bool = True, append=None):
+             stale: bool = True, append=None, out_dtype=torch.float32):
     """One-launch decode step through the C ABI.  With `stale`, the metadata is
     first built for the cache as it stood before its newest token (seq_len - 1;
     pages never built hold a fill pattern), so the step's own refresh of the
@@ -114,7 +114,7 @@ def run_step(layer, *, page_size: int, rule: str, budget: dict, scale: float,
     for _ in range(repeat):
         sel_idx = torch.full((B, Hkv, max_sel), -7, dtype=torch.int32, device=dev)
         sel_count = torch.full((B, Hkv), -7, dtype=torch.int32, device=dev)
-        out = torch.full((B, Hq, 128), float("nan"), dtype=torch.float32, device=dev)
+        out = torch.full((B, Hq, 128), float("nan"), dtype=out_dtype, device=dev)
         lse = torch.full((B, Hq), float("nan"), dtype=torch.float32, device=dev)
         if append is None:
             sa.sparse_attn_decode_step(kv, meta, rule, layer.q, budget_struct(budget), max_sel, scale,

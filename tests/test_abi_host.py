@@ -136,10 +136,11 @@ def test_decode_step_append_validation(lib, abi):
     ok = _desc(abi)
     topk = abi.sa_budget(abi.SA_BUDGET_TOPK, 8, 0.0, 0, 0, 0, 0)
 
-    def call(k_new=0x90000, v_new=0xa0000, max_sel=16, ws_bytes=1 << 30):
+    def call(k_new=0x90000, v_new=0xa0000, max_sel=16, ws_bytes=1 << 30, out_dtype=abi.SA_OUT_F32):
         return lib.sparse_attn_decode_step_append(C.byref(ok), 0x40000, 0, 0x50000, 32, k_new, v_new,
                                                   C.byref(topk), max_sel, 0.088, 0x60000, 0x70000,
-                                                  0x80000, None, 0x100000, ws_bytes, None)
+                                                  0x80000, out_dtype, None, 0x100000, ws_bytes, None)
+    assert call(out_dtype=2) == abi.SA_ERR_INVALID
     assert call(k_new=0) == abi.SA_ERR_INVALID
     assert call(v_new=0) == abi.SA_ERR_INVALID
     assert call(k_new=0x90004) == abi.SA_ERR_INVALID      # not 8-byte aligned

@@ -143,6 +143,12 @@ def test_step_append(cuda_dev, R, rule, name):
         for key in ("sel_idx", "sel_count", "out", "lse"):
             assert torch.equal(r[key], app["runs"][0][key]), key
     assert torch.equal(lay2.k, lay.k) and torch.equal(lay2.v, lay.v)
+    # bf16 output: the same fp32 results rounded to nearest even
+    bf = R.run_step(lay2, page_size=ps, rule=rule, budget=bd, scale=SCALE, stale=True,
+                    append=(k_new, v_new), out_dtype=torch.bfloat16)
+    assert bf["status"] == 0 and bf["out"].dtype == torch.bfloat16
+    assert torch.equal(bf["out"], ref["out"].to(torch.bfloat16)), f"bf16 output {name}/{rule}"
+    assert torch.equal(bf["lse"], ref["lse"]) and torch.equal(bf["sel_idx"], ref["sel_idx"])
 
 
 def test_step_repeat_and_interleave(cuda_dev, R):
