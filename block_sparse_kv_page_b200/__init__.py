@@ -5,7 +5,9 @@ The Python side only marshals arguments to libsparse_attn.so; importing the
 package fails if the library has not been built (no CPU fallback).
 """
 from .ops import (KvCache, SparseAttnError, budget_ratio, budget_tokens, budget_topk,  # noqa: F401
-                  lib, make_workspace, sparse_attn_build_meta, sparse_attn_decode,
+                  lib, make_workspace, make_workspace_per_head, sparse_attn_build_meta,
+                  sparse_attn_decode, sparse_attn_decode_per_head, sparse_attn_select_per_head,
+                  sparse_attn_workspace_size_per_head,
                   sparse_attn_decode_static, sparse_attn_decode_step,
                   sparse_attn_decode_step_append,
                   sparse_attn_get_device_status, sparse_attn_route, sparse_attn_select,

@@ -76,6 +76,13 @@ PROTOTYPES = {
                                                  C.c_int32, C.c_void_p, C.c_void_p, C.POINTER(sa_budget),
                                                  C.c_int32, C.c_float, C.c_void_p, C.c_void_p, C.c_void_p,
                                                  C.c_int, C.c_void_p, C.c_void_p, C.c_size_t, C.c_void_p]),
+    "sparse_attn_workspace_size_per_head": (C.c_size_t, [C.POINTER(sa_kv_desc), C.c_int32, C.c_int32]),
+    "sparse_attn_select_per_head": (C.c_int, [C.POINTER(sa_kv_desc), C.c_void_p, C.c_int, C.c_void_p, C.c_int32,
+                                              C.POINTER(sa_budget), C.c_int32, C.c_void_p, C.c_void_p,
+                                              C.c_void_p, C.c_void_p, C.c_size_t, C.c_void_p]),
+    "sparse_attn_decode_per_head": (C.c_int, [C.POINTER(sa_kv_desc), C.c_void_p, C.c_int32, C.c_float,
+                                              C.c_void_p, C.c_void_p, C.c_int32, C.c_void_p, C.c_void_p,
+                                              C.c_void_p, C.c_size_t, C.c_void_p]),
     "sparse_attn_route": (C.c_int, [C.POINTER(sa_kv_desc), C.c_void_p, C.c_int, C.c_void_p, C.c_int32,
                                     C.c_int32, C.c_int32, C.c_int32, C.c_int32, C.c_int32, C.c_float,
                                     C.c_void_p, C.c_void_p, C.c_void_p, C.c_void_p, C.c_void_p, C.c_void_p,

@@ -116,8 +116,9 @@ int max_tiles_per_unit(const sa_kv_desc* kv, int max_sel) {
 // selecting CTA can read a row with 16-byte loads.
 int score_stride(const sa_kv_desc* kv) { return (kv->max_pages + 3) & ~3; }
 
-size_t select_scratch(const sa_kv_desc* kv) {
-  return align256((size_t)kv->batch * kv->n_kv_heads * score_stride(kv) * sizeof(float));
+size_t select_scratch(const sa_kv_desc* kv, bool per_head = false, int n_q_heads = 0) {
+  const size_t units = (size_t)kv->batch * (per_head ? n_q_heads : kv->n_kv_heads);
+  return align256(units * score_stride(kv) * sizeof(float));
 }
 
 // Split partials: one slot per work item (none when no unit is split).
@@ -321,6 +322,7 @@ bool fill_select(SelectArgs* a, const sa_kv_desc* kv, const void* meta, sa_score
   a->status = reinterpret_cast<int*>(ws);
   a->splits = select_splits(kv->batch * kv->n_kv_heads, kv->max_pages, device_sm_count());
   a->meta_refresh = nullptr;
+  a->per_head = 0;
   a->k_new = a->v_new = nullptr;
   a->k_dst = a->v_dst = nullptr;
   return true;
@@ -349,6 +351,7 @@ bool fill_decode(DecodeArgs* a, const sa_kv_desc* kv, const void* q, int n_q_hea
   a->max_sel = max_sel;
   a->out = out;
   a->out_bf16 = nullptr;
+  a->per_head = 0;
   a->lse = lse;
   a->ws_part = ws_part;
   a->ws_count = ws_count;
@@ -387,6 +390,18 @@ size_t sparse_attn_workspace_size(const sa_kv_desc* kv, int32_t n_q_heads, int32
   return kScratch + tail;
 }
 
+size_t sparse_attn_workspace_size_per_head(const sa_kv_desc* kv, int32_t n_q_heads, int32_t max_sel) {
+  if (check_kv(kv) != SA_OK || max_sel < 1) return 0;
+  int G;
+  if (check_group(kv, n_q_heads, &G) != SA_OK) return 0;
+  const long long units = (long long)kv->batch * n_q_heads;
+  if (units > kMaxUnits) return 0;
+  const DecodePlan plan = decode_plan((int)units, max_tiles_per_unit(kv, max_sel), device_sm_count());
+  const size_t sel = select_scratch(kv, true, n_q_heads);
+  const size_t dec = decode_scratch(plan);
+  return kScratch + (sel > dec ? sel : dec);
+}
+
 sa_status sparse_attn_workspace_init(void* ws, size_t ws_bytes, void* stream) {
   if (!ws || !aligned(ws, 256) || ws_bytes < kScratch) return SA_ERR_WORKSPACE;
   return launched(cudaMemsetAsync(ws, 0, ws_bytes, (cudaStream_t)stream));
@@ -402,22 +417,73 @@ sa_status sparse_attn_build_meta(const sa_kv_desc* kv, sa_score_rule rule, int32
                                     (cudaStream_t)stream));
 }
 
-sa_status sparse_attn_select(const sa_kv_desc* kv, const void* meta, sa_score_rule rule,
+// Selection per (sequence, KV head), or per (sequence, query head).
+static sa_status select_impl(const sa_kv_desc* kv, const void* meta, sa_score_rule rule,
                              const void* q, int32_t n_q_heads, const sa_budget* budget,
                              int32_t max_sel, int32_t* sel_idx, int32_t* sel_count,
-                             float* scores_out, void* ws, size_t ws_bytes, void* stream) {
+                             float* scores_out, bool per_head, void* ws, size_t ws_bytes,
+                             void* stream) {
   int G;
   sa_status s = check_select(kv, meta, rule, q, n_q_heads, budget, max_sel, sel_idx, sel_count,
                              scores_out, &G);
   if (s != SA_OK) return s;
-  const size_t need = kScratch + select_scratch(kv);
+  if (per_head && (long long)kv->batch * n_q_heads > kMaxUnits) return SA_ERR_UNSUPPORTED;
+  const size_t need = kScratch + select_scratch(kv, per_head, n_q_heads);
   if ((s = check_ws(ws, ws_bytes, need)) != SA_OK) return s;
   SelectArgs a;
   if (!fill_select(&a, kv, meta, rule, q, n_q_heads, G, budget, max_sel, sel_idx, sel_count,
                    scores_out, ws))
     return SA_ERR_CUDA;
+  if (per_head) {
+    a.per_head = 1;
+    a.splits = select_splits(kv->batch * n_q_heads, kv->max_pages, device_sm_count());
+  }
   a.ws_queue = reinterpret_cast<uint32_t*>(reinterpret_cast<char*>(ws) + kQueueSelect);
   return launched(launch_select(a, (cudaStream_t)stream));
+}
+
+sa_status sparse_attn_select(const sa_kv_desc* kv, const void* meta, sa_score_rule rule,
+                             const void* q, int32_t n_q_heads, const sa_budget* budget,
+                             int32_t max_sel, int32_t* sel_idx, int32_t* sel_count,
+                             float* scores_out, void* ws, size_t ws_bytes, void* stream) {
+  return select_impl(kv, meta, rule, q, n_q_heads, budget, max_sel, sel_idx, sel_count, scores_out,
+                     false, ws, ws_bytes, stream);
+}
+
+sa_status sparse_attn_select_per_head(const sa_kv_desc* kv, const void* meta, sa_score_rule rule,
+                                      const void* q, int32_t n_q_heads, const sa_budget* budget,
+                                      int32_t max_sel, int32_t* sel_idx, int32_t* sel_count,
+                                      float* scores_out, void* ws, size_t ws_bytes, void* stream) {
+  return select_impl(kv, meta, rule, q, n_q_heads, budget, max_sel, sel_idx, sel_count, scores_out,
+                     true, ws, ws_bytes, stream);
+}
+
+// Decode of one query row per sequence (validated arguments), per KV head or
+// per query head.
+static sa_status decode_rows(const sa_kv_desc* kv, const void* q, int32_t n_q_heads, int G,
+                             float scale, const int32_t* idx, const int32_t* count, int32_t max_sel,
+                             float* out, float* lse, bool per_head, void* ws, size_t ws_bytes,
+                             void* stream) {
+  if (kv->page_size == 0 && max_sel > kMaxChunkSel) return SA_ERR_UNSUPPORTED;
+  const long long units = (long long)kv->batch * (per_head ? n_q_heads : kv->n_kv_heads);
+  if (units > kMaxUnits) return SA_ERR_UNSUPPORTED;
+  const unsigned long long kv_rows = (unsigned long long)kv->batch * kv->n_kv_heads * kv->cap_tokens;
+  if (kv_rows > 0x7fffffffULL) return SA_ERR_UNSUPPORTED;  // TMA row coordinates are int32
+  const DecodePlan plan = decode_plan((int)units, max_tiles_per_unit(kv, max_sel), device_sm_count());
+  if (plan.items > 0x7fffffffLL) return SA_ERR_UNSUPPORTED;
+  const size_t need = kScratch + decode_scratch(plan);
+  sa_status s;
+  if ((s = check_ws(ws, ws_bytes, need)) != SA_OK) return s;
+
+  DecodeArgs a;
+  char* w = reinterpret_cast<char*>(ws);
+  if (!fill_decode(&a, kv, q, n_q_heads, G, scale, idx, count, max_sel, out, lse,
+                   reinterpret_cast<float*>(w + kScratch), reinterpret_cast<uint32_t*>(w + 256),
+                   reinterpret_cast<int*>(ws), plan))
+    return SA_ERR_CUDA;
+  a.per_head = per_head ? 1 : 0;
+  a.ws_queue = reinterpret_cast<uint32_t*>(w + kQueueDecode);
+  return launched(launch_decode(a, (cudaStream_t)stream));
 }
 
 sa_status sparse_attn_decode(const sa_kv_desc* kv, const void* q, int32_t n_q_heads,
@@ -440,24 +506,25 @@ sa_status sparse_attn_decode(const sa_kv_desc* kv, const void* q, int32_t n_q_he
     return tile_attention(kv, q, n_q_heads, G, n_q_rows, q_pos0, tile_rows, scale, idx, count,
                           max_sel, out, lse, reinterpret_cast<int*>(ws), ws, ws_bytes, stream);
   }
-  if (kv->page_size == 0 && max_sel > kMaxChunkSel) return SA_ERR_UNSUPPORTED;
-  const long long units = (long long)n_q_rows * kv->n_kv_heads;
-  if (units > kMaxUnits) return SA_ERR_UNSUPPORTED;
-  const unsigned long long kv_rows = (unsigned long long)kv->batch * kv->n_kv_heads * kv->cap_tokens;
-  if (kv_rows > 0x7fffffffULL) return SA_ERR_UNSUPPORTED;  // TMA row coordinates are int32
-  const DecodePlan plan = decode_plan((int)units, max_tiles_per_unit(kv, max_sel), device_sm_count());
-  if (plan.items > 0x7fffffffLL) return SA_ERR_UNSUPPORTED;
-  const size_t need = kScratch + decode_scratch(plan);
-  if ((s = check_ws(ws, ws_bytes, need)) != SA_OK) return s;
+  return decode_rows(kv, q, n_q_heads, G, scale, idx, count, max_sel, out, lse, false, ws, ws_bytes,
+                     stream);
+}
 
-  DecodeArgs a;
-  char* w = reinterpret_cast<char*>(ws);
-  if (!fill_decode(&a, kv, q, n_q_heads, G, scale, idx, count, max_sel, out, lse,
-                   reinterpret_cast<float*>(w + kScratch), reinterpret_cast<uint32_t*>(w + 256),
-                   reinterpret_cast<int*>(ws), plan))
-    return SA_ERR_CUDA;
-  a.ws_queue = reinterpret_cast<uint32_t*>(w + kQueueDecode);
-  return launched(launch_decode(a, (cudaStream_t)stream));
+sa_status sparse_attn_decode_per_head(const sa_kv_desc* kv, const void* q, int32_t n_q_heads,
+                                      float scale, const int32_t* idx, const int32_t* count,
+                                      int32_t max_sel, float* out, float* lse, void* ws,
+                                      size_t ws_bytes, void* stream) {
+  sa_status s = check_kv(kv);
+  if (s != SA_OK) return s;
+  int G;
+  if ((s = check_group(kv, n_q_heads, &G)) != SA_OK) return s;
+  if (!q || !aligned(q, 16) || !idx || !count || !aligned(idx, 4) || !aligned(count, 4))
+    return SA_ERR_INVALID;
+  if (!out || !aligned(out, 16) || (lse && !aligned(lse, 4))) return SA_ERR_INVALID;
+  if (max_sel < 1) return SA_ERR_INVALID;
+  if (!std::isfinite(scale)) return SA_ERR_INVALID;
+  return decode_rows(kv, q, n_q_heads, G, scale, idx, count, max_sel, out, lse, true, ws, ws_bytes,
+                     stream);
 }
 
 // The decode step with or without the append of the newest token's K/V.
@@ -744,6 +811,7 @@ extern "C" sa_status sparse_attn_decode_static(const sa_kv_desc* kv, const void*
   a.max_sel = max_sel;
   a.out = out;
   a.out_bf16 = nullptr;
+  a.per_head = 0;
   a.lse = lse;
   a.ws_part = reinterpret_cast<float*>(scratch + kStaticPartOff);
   a.ws_count = reinterpret_cast<uint32_t*>(scratch + 256);

@@ -126,9 +126,9 @@ SA_DEV void decode_item(const DecodeArgs& a, const int u, const int split, const
                         WarpState& ws) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int gq = lane >> 2, c = lane & 3;
-  const int Hkv = a.kv.Hkv;
-  const int b = u / Hkv, g = u % Hkv;
-  const int G = a.G;
+  const UnitMap um = unit_map(u, a.per_head, a.kv.Hkv, a.Hq, a.G);
+  const int b = um.b;
+  const int G = um.n_heads;  // query heads attending this unit's pages
   const float ninf = -__int_as_float(0x7f800000);
 
   // ---- geometry of the unit
@@ -179,7 +179,7 @@ SA_DEV void decode_item(const DecodeArgs& a, const int u, const int split, const
                               : (size_t)a.fine_unit0 * a.splits + (size_t)(u - a.fine_unit0) * a.splits_fine;
   const int t_begin = (int)(((long long)T * split) / splits);
   const int t_end = (int)(((long long)T * (split + 1)) / splits);
-  const long long row0 = (long long)u * a.kv.cap;
+  const long long row0 = (long long)um.kvu * a.kv.cap;
 
   // Token range of tile t of the unit (n = 0 for a skipped, invalid entry).
   auto tile_ref = [&](int t) -> TileRef {
@@ -215,7 +215,7 @@ SA_DEV void decode_item(const DecodeArgs& a, const int u, const int split, const
   // ---- Q fragments (B operand, natural k order): q[head][16s + 2c (+8)]
   const bool head_ok = gq < G;
   const __nv_bfloat16* qrow = reinterpret_cast<const __nv_bfloat16*>(a.q) +
-                              ((size_t)b * a.Hq + (size_t)g * G + (head_ok ? gq : 0)) * kHeadDim;
+                              ((size_t)b * a.Hq + (size_t)um.h0 + (head_ok ? gq : 0)) * kHeadDim;
   uint32_t bq[16];
 #pragma unroll
   for (int s = 0; s < 8; ++s) {
@@ -391,7 +391,7 @@ SA_DEV void decode_item(const DecodeArgs& a, const int u, const int split, const
       }
     }
   }
-  const size_t out_row = (size_t)b * a.Hq + (size_t)g * G + h;
+  const size_t out_row = (size_t)b * a.Hq + (size_t)um.h0 + h;
 
   if (splits == 1) {
     if (h < G) {

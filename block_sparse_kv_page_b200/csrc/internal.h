@@ -50,6 +50,30 @@ WsLayout workspace_layout(const sa_kv_desc* kv, int n_q_heads, int n_q_rows, int
 cudaError_t launch_build_meta(const KvView& kv, int rule, int first_token, void* meta,
                               int* status, cudaStream_t st);
 
+// Work unit u of a selection or decode: sequence b, KV head g (its K/V and
+// metadata rows belong to kv unit b * Hkv + g), and the query heads
+// [h0, h0 + n_heads) that share the unit's page set: the G heads of KV head g,
+// or a single query head when every query head selects its own pages.
+struct UnitMap {
+  int b, g, kvu, h0, n_heads;
+};
+__host__ __device__ inline UnitMap unit_map(int u, int per_head, int Hkv, int Hq, int G) {
+  UnitMap m;
+  if (per_head) {
+    m.b = u / Hq;
+    m.h0 = u - m.b * Hq;
+    m.g = m.h0 / G;
+    m.n_heads = 1;
+  } else {
+    m.b = u / Hkv;
+    m.g = u - m.b * Hkv;
+    m.h0 = m.g * G;
+    m.n_heads = G;
+  }
+  m.kvu = m.b * Hkv + m.g;
+  return m;
+}
+
 struct SelectArgs {
   CUtensorMap tmap_meta;      // metadata rows [B*Hkv*max_pages][512 B], boxes 16 x 128 B, 128B swizzle
   KvView kv;
@@ -59,6 +83,7 @@ struct SelectArgs {
   int Hq, G;
   int budget_kind, top_k, topk_val, bos, eos, token_budget;
   double ratio;
+  int per_head;               // 1: one unit per (sequence, query head), else per (sequence, KV head)
   int max_sel;
   int32_t* sel_idx;
   int32_t* sel_count;
@@ -86,6 +111,7 @@ struct DecodeArgs {
   KvView kv;
   const void* q;
   int Hq, G;
+  int per_head;               // 1: one unit per (row, query head), else per (row, KV head)
   int n_rows, q_pos0, tile_rows;
   float scale_log2;           // scale * log2(e)
   const int32_t* idx;

@@ -32,7 +32,7 @@ __global__ void __launch_bounds__(kThreads, SA_SEL_CTAS_PER_SM) select_kernel(co
   if (threadIdx.x == 0) prefetch_tmap(&a.tmap_meta);
   __syncthreads();
   WarpState ws{0u, true, 0u, 0u};
-  const int n_items = a.kv.B * a.kv.Hkv * a.splits;
+  const int n_items = a.kv.B * (a.per_head ? a.Hq : a.kv.Hkv) * a.splits;
   for (;;) {
     if (threadIdx.x == 0) s_item = (int)atomicAdd(&a.ws_queue[0], 1u);
     __syncthreads();
@@ -82,7 +82,7 @@ size_t select_smem_bytes(int max_pages) {
 
 cudaError_t launch_select(const SelectArgs& a, cudaStream_t st) {
   const size_t smem = select_smem_bytes(a.kv.max_pages);
-  const long long items = (long long)a.kv.B * a.kv.Hkv * a.splits;
+  const long long items = (long long)a.kv.B * (a.per_head ? a.Hq : a.kv.Hkv) * a.splits;
   if (items > 0x7fffffffLL) return cudaErrorInvalidValue;
   long long grid = (long long)device_sm_count() * SA_SEL_CTAS_PER_SM;
   if (grid > items) grid = items;

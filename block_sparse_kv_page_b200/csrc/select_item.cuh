@@ -469,7 +469,12 @@ SA_DEV void select_item(const SelectArgs& a, const int u, const int split, const
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int gq = lane >> 2, c = lane & 3;
   const int Hkv = a.kv.Hkv;
-  const int b = u / Hkv, g = u % Hkv;
+  const UnitMap um = unit_map(u, a.per_head, Hkv, a.Hq, a.G);
+  const int b = um.b, kvu = um.kvu;
+  // per-query-head units share their KV head's metadata, cache rows and the
+  // newest-page refresh: one of them (the first head of the group) stores
+  // what is shared, every one patches its own staged copy
+  const bool kv_owner = !a.per_head || um.h0 % a.G == 0;
 
   // ---- unit geometry (every CTA of the unit computes the same values)
   const int N = a.kv.seq_len[b];
@@ -490,10 +495,10 @@ SA_DEV void select_item(const SelectArgs& a, const int u, const int split, const
   const int t_begin = (int)(((long long)TP * split) / a.splits);
   const int t_end = (int)(((long long)TP * (split + 1)) / a.splits);
 
-  // ---- B fragments: the G query heads of this KV group (columns >= G are zero)
-  const bool head_ok = gq < a.G;
+  // ---- B fragments: the unit's query heads (columns >= n_heads are zero)
+  const bool head_ok = gq < um.n_heads;
   const __nv_bfloat16* qrow = reinterpret_cast<const __nv_bfloat16*>(a.q) +
-                              ((size_t)b * a.Hq + (size_t)g * a.G + (head_ok ? gq : 0)) * kHeadDim;
+                              ((size_t)b * a.Hq + (size_t)um.h0 + (head_ok ? gq : 0)) * kHeadDim;
   uint32_t bq[RULE == 0 ? 32 : 1];
   double bd[RULE == 0 ? 1 : 32];
   if (RULE == 0) {
@@ -525,7 +530,7 @@ SA_DEV void select_item(const SelectArgs& a, const int u, const int split, const
   float* out_u = a.scores_out ? a.scores_out + (size_t)u * a.kv.max_pages : nullptr;
   unsigned char* ring = S.ring + warp * (kStages * kTileBytes);
   uint64_t* bars = S.bars + warp * kStages;
-  const int row_base = u * a.kv.max_pages;
+  const int row_base = kvu * a.kv.max_pages;
   const int lrow = (lane & 7) + 8 * ((lane >> 3) & 1);  // ldmatrix: rows 0-7 / 8-15
   const int lchk = lane >> 4;                            //            chunk +0 / +1
   const int nt = t_end - t_begin;
@@ -593,19 +598,22 @@ SA_DEV void select_item(const SelectArgs& a, const int u, const int split, const
       const bool app = a.k_new != nullptr;
       uint2 knew = make_uint2(0u, 0u);
       if (app) {
-        const size_t src = (size_t)u * kHeadDim + lane * 4;
-        const size_t dst = ((size_t)u * a.kv.cap + (size_t)(N - 1)) * kHeadDim + lane * 4;
+        const size_t src = (size_t)kvu * kHeadDim + lane * 4;
         knew = __ldg(reinterpret_cast<const uint2*>(static_cast<const __nv_bfloat16*>(a.k_new) + src));
-        const uint2 vnew = __ldg(reinterpret_cast<const uint2*>(static_cast<const __nv_bfloat16*>(a.v_new) + src));
-        *reinterpret_cast<uint2*>(static_cast<__nv_bfloat16*>(a.k_dst) + dst) = knew;
-        *reinterpret_cast<uint2*>(static_cast<__nv_bfloat16*>(a.v_dst) + dst) = vnew;
-        fence_proxy_async_global();  // the decode items read the row with TMA
+        if (kv_owner) {
+          const size_t dst = ((size_t)kvu * a.kv.cap + (size_t)(N - 1)) * kHeadDim + lane * 4;
+          const uint2 vnew = __ldg(reinterpret_cast<const uint2*>(static_cast<const __nv_bfloat16*>(a.v_new) + src));
+          *reinterpret_cast<uint2*>(static_cast<__nv_bfloat16*>(a.k_dst) + dst) = knew;
+          *reinterpret_cast<uint2*>(static_cast<__nv_bfloat16*>(a.v_dst) + dst) = vnew;
+          fence_proxy_async_global();  // the decode items read the row with TMA
+        }
       }
       // rebuild the newest page's metadata, store it, patch the staged row
       const __nv_bfloat16* k_lane = reinterpret_cast<const __nv_bfloat16*>(a.kv.k) +
-                                    ((size_t)u * a.kv.cap) * kHeadDim + lane * 4;
+                                    ((size_t)kvu * a.kv.cap) * kHeadDim + lane * 4;
       const PageMetaLane m = page_meta_lane<RULE>(k_lane, r_s, r_e, app, knew);
-      store_page_meta<RULE>(a.meta_refresh + ((size_t)u * a.kv.max_pages + p_new) * kMetaBytes, m, lane);
+      if (kv_owner)
+        store_page_meta<RULE>(a.meta_refresh + ((size_t)kvu * a.kv.max_pages + p_new) * kMetaBytes, m, lane);
       const int r = p_new & 15;
       if (RULE == 0) {
         const uint32_t o = swz128(r, (lane & 15) >> 1) + 8 * (lane & 1);
@@ -645,7 +653,7 @@ SA_DEV void select_item(const SelectArgs& a, const int u, const int split, const
       acc[0] = (float)c00; acc[1] = (float)c01; acc[2] = (float)c10; acc[3] = (float)c11;
     }
     const float ninf = -__int_as_float(0x7f800000);
-    const bool c0 = 2 * c < a.G, c1 = 2 * c + 1 < a.G;
+    const bool c0 = 2 * c < um.n_heads, c1 = 2 * c + 1 < um.n_heads;
     float mlo = fmaxf(c0 ? acc[0] : ninf, c1 ? acc[1] : ninf);
     float mhi = fmaxf(c0 ? acc[2] : ninf, c1 ? acc[3] : ninf);
     mlo = fmaxf(mlo, __shfl_xor_sync(0xffffffffu, mlo, 1));

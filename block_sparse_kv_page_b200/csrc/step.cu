@@ -131,7 +131,7 @@ __global__ void __launch_bounds__(kThreads, SA_STEP_CTAS_PER_SM)
   __syncthreads();
   if (s_last) {
     __threadfence();
-    const int units = a.sel.kv.B * a.sel.kv.Hkv;
+    const int units = a.sel.kv.B * (a.sel.per_head ? a.sel.Hq : a.sel.kv.Hkv);
     for (int i = threadIdx.x; i < units; i += blockDim.x) {
       a.sel.ws_count[i] = 0;
       a.dec.ws_count[i] = 0;

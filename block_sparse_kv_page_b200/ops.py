@@ -112,6 +112,20 @@ def make_workspace(kv: KvCache, n_q_heads: int, n_q_rows: int, max_sel: int, str
     return ws
 
 
+def sparse_attn_workspace_size_per_head(kv: KvCache, n_q_heads: int, max_sel: int) -> int:
+    return int(lib.sparse_attn_workspace_size_per_head(C.byref(kv.desc), int(n_q_heads), int(max_sel)))
+
+
+def make_workspace_per_head(kv: KvCache, n_q_heads: int, max_sel: int, stream=None) -> torch.Tensor:
+    """Workspace for sparse_attn_select_per_head / sparse_attn_decode_per_head."""
+    n = sparse_attn_workspace_size_per_head(kv, n_q_heads, max_sel)
+    if n == 0:
+        raise SparseAttnError(_abi.SA_ERR_INVALID, "sparse_attn_workspace_size_per_head")
+    ws = torch.empty(n, dtype=torch.uint8, device=kv.k.device)
+    sparse_attn_workspace_init(ws, stream)
+    return ws
+
+
 def sparse_attn_build_meta(kv: KvCache, rule, first_token: int, meta: torch.Tensor, stream=None) -> None:
     _check(lib.sparse_attn_build_meta(C.byref(kv.desc), _rule(rule), int(first_token),
                                       meta.data_ptr(), _stream(stream)), "sparse_attn_build_meta")
@@ -127,6 +141,34 @@ def sparse_attn_select(kv: KvCache, meta: torch.Tensor, rule, q: torch.Tensor, b
                                   sel_count.data_ptr(), _ptr(scores_out), ws.data_ptr(),
                                   ws.numel() * ws.element_size(), _stream(stream)),
            "sparse_attn_select")
+
+
+def sparse_attn_select_per_head(kv: KvCache, meta: torch.Tensor, rule, q: torch.Tensor, budget: sa_budget,
+                                max_sel: int, sel_idx: torch.Tensor, sel_count: torch.Tensor,
+                                scores_out: torch.Tensor | None, ws: torch.Tensor, stream=None) -> None:
+    """One page set per query head: sel_idx [B, Hq, max_sel], sel_count [B, Hq]."""
+    if q.dtype != torch.bfloat16 or not q.is_contiguous():
+        raise ValueError("q must be contiguous bf16 [B, Hq, 128]")
+    _check(lib.sparse_attn_select_per_head(C.byref(kv.desc), meta.data_ptr(), _rule(rule), q.data_ptr(),
+                                           q.shape[-2], C.byref(budget), int(max_sel), sel_idx.data_ptr(),
+                                           sel_count.data_ptr(), _ptr(scores_out), ws.data_ptr(),
+                                           ws.numel() * ws.element_size(), _stream(stream)),
+           "sparse_attn_select_per_head")
+
+
+def sparse_attn_decode_per_head(kv: KvCache, q: torch.Tensor, scale: float, idx: torch.Tensor,
+                                count: torch.Tensor, max_sel: int, out: torch.Tensor,
+                                lse: torch.Tensor | None, ws: torch.Tensor, stream=None) -> None:
+    """Decode where query head h attends its own page list idx[b, h]."""
+    if q.dtype != torch.bfloat16 or not q.is_contiguous():
+        raise ValueError("q must be contiguous bf16 [B, Hq, 128]")
+    if out.dtype != torch.float32 or not out.is_contiguous():
+        raise ValueError("out must be contiguous fp32")
+    _check(lib.sparse_attn_decode_per_head(C.byref(kv.desc), q.data_ptr(), q.shape[-2], float(scale),
+                                           idx.data_ptr(), count.data_ptr(), int(max_sel), out.data_ptr(),
+                                           _ptr(lse), ws.data_ptr(), ws.numel() * ws.element_size(),
+                                           _stream(stream)),
+           "sparse_attn_decode_per_head")
 
 
 def sparse_attn_decode(kv: KvCache, q: torch.Tensor, n_q_rows: int, q_pos0: int, tile_rows: int,

@@ -227,6 +227,32 @@ sa_status sparse_attn_decode_step_append(const sa_kv_desc* kv, void* meta, sa_sc
                                          int32_t* sel_count, void* out, sa_out_dtype out_dtype,
                                          float* lse, void* ws, size_t ws_bytes, void* stream);
 
+/* (f) Per-query-head selection: every query head keeps its own page set,
+ * the other reading of how GQA shares a selection ([OFFLINE] "The comparison"
+ * scores chunks against the current query; here "the query" is one head
+ * rather than the group of G heads that share a KV head).
+ *   sparse_attn_select_per_head: as sparse_attn_select, except that the unit
+ *     is (sequence, query head h): the score of a page is head h's own score
+ *     (no group maximum) against the metadata of KV head h / G, and
+ *     sel_idx is [B][n_q_heads][max_sel], sel_count [B][n_q_heads],
+ *     scores_out [B][n_q_heads][max_pages].
+ *   sparse_attn_decode_per_head: decode (one row per sequence) where query
+ *     head h attends the pages listed for it in idx [B][n_q_heads][max_sel]
+ *     (count [B][n_q_heads]), reading K/V of KV head h / G.  out and lse as
+ *     in sparse_attn_decode.
+ * Both take the workspace sized by sparse_attn_workspace_size_per_head (B *
+ * n_q_heads <= 65536 units); other checks and errors as in the shared calls.
+ * K/V bytes read grow with the number of distinct pages the G heads keep. */
+size_t sparse_attn_workspace_size_per_head(const sa_kv_desc* kv, int32_t n_q_heads, int32_t max_sel);
+sa_status sparse_attn_select_per_head(const sa_kv_desc* kv, const void* meta, sa_score_rule rule,
+                                      const void* q, int32_t n_q_heads, const sa_budget* budget,
+                                      int32_t max_sel, int32_t* sel_idx, int32_t* sel_count,
+                                      float* scores_out, void* ws, size_t ws_bytes, void* stream);
+sa_status sparse_attn_decode_per_head(const sa_kv_desc* kv, const void* q, int32_t n_q_heads,
+                                      float scale, const int32_t* idx, const int32_t* count,
+                                      int32_t max_sel, float* out, float* lse, void* ws,
+                                      size_t ws_bytes, void* stream);
+
 /* (d) Uncertainty router over query tiles ([ROUTER] "Methodologie" steps 2-5).
  * B == 1, fixed blocks (page_size = block size).  q bf16 [n_q_rows][n_q_heads][128]
  * at positions q_pos0 + r; tiles of tile_rows consecutive rows.  For tile t

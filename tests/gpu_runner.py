@@ -45,7 +45,10 @@ def default_max_sel(bd: dict, max_pages: int) -> int:
 
 
 def run_gpu(layer, *, page_size: int, rule: str, budget: dict, scale: float,
-            max_pages: int | None = None, max_sel: int | None = None, ws=None, repeat: int = 1):
+            max_pages: int | None = None, max_sel: int | None = None, ws=None, repeat: int = 1,
+            per_head: bool = False):
+    """build_meta + select + decode through the C ABI.  per_head: one page set
+    per query head (the *_per_head calls); selection rows are then [B, Hq]."""
     B, Hkv, cap, D = layer.k.shape
     Hq = layer.q.shape[1]
     if max_pages is None:
@@ -57,18 +60,25 @@ def run_gpu(layer, *, page_size: int, rule: str, budget: dict, scale: float,
     dev = layer.k.device
     meta = kv.meta_buffer()
     if ws is None:
-        ws = sa.make_workspace(kv, Hq, B, max_sel)
+        ws = (sa.make_workspace_per_head(kv, Hq, max_sel) if per_head
+              else sa.make_workspace(kv, Hq, B, max_sel))
     sa.sparse_attn_build_meta(kv, rule, 0, meta)
+    U = Hq if per_head else Hkv
     results = []
     for _ in range(repeat):
-        sel_idx = torch.full((B, Hkv, max_sel), -7, dtype=torch.int32, device=dev)
-        sel_count = torch.full((B, Hkv), -7, dtype=torch.int32, device=dev)
-        scores = torch.full((B, Hkv, max_pages), float("nan"), dtype=torch.float32, device=dev)
-        sa.sparse_attn_select(kv, meta, rule, layer.q, budget_struct(budget), max_sel,
-                              sel_idx, sel_count, scores, ws)
+        sel_idx = torch.full((B, U, max_sel), -7, dtype=torch.int32, device=dev)
+        sel_count = torch.full((B, U), -7, dtype=torch.int32, device=dev)
+        scores = torch.full((B, U, max_pages), float("nan"), dtype=torch.float32, device=dev)
         out = torch.full((B, Hq, 128), float("nan"), dtype=torch.float32, device=dev)
         lse = torch.full((B, Hq), float("nan"), dtype=torch.float32, device=dev)
-        sa.sparse_attn_decode(kv, layer.q, B, 0, 1, scale, sel_idx, sel_count, max_sel, out, lse, ws)
+        if per_head:
+            sa.sparse_attn_select_per_head(kv, meta, rule, layer.q, budget_struct(budget), max_sel,
+                                           sel_idx, sel_count, scores, ws)
+            sa.sparse_attn_decode_per_head(kv, layer.q, scale, sel_idx, sel_count, max_sel, out, lse, ws)
+        else:
+            sa.sparse_attn_select(kv, meta, rule, layer.q, budget_struct(budget), max_sel,
+                                  sel_idx, sel_count, scores, ws)
+            sa.sparse_attn_decode(kv, layer.q, B, 0, 1, scale, sel_idx, sel_count, max_sel, out, lse, ws)
         torch.cuda.synchronize()
         results.append(dict(sel_idx=sel_idx.cpu(), sel_count=sel_count.cpu(), scores=scores.cpu(),
                             out=out.cpu(), lse=lse.cpu()))
@@ -186,19 +196,23 @@ def certify_selection(S, gset: set, budget: dict, lens=None, where=""):
 
 
 def check_layer(layer, gpu, *, page_size: int, rule: str, budget: dict, scale: float,
-                units=None, score_rel: float = 2e-6, out_tol: float = OUT_TOL):
+                units=None, score_rel: float = 2e-6, out_tol: float = OUT_TOL, per_head: bool = False):
     """Compare every (b, g) unit (or the given subset) with the oracle.
+    per_head: units are (b, query head h), each with its own page set; the
+    oracle is the same one applied to the single head h (its group is {h}).
     Returns a dict of statistics (max errors, tie exemptions)."""
     B, Hkv = layer.k.shape[:2]
     Hq = layer.q.shape[1]
     G = Hq // Hkv
     stats = dict(max_out_err=0.0, max_lse_err=0.0, max_score_err=0.0, ties=0, units=0)
     if units is None:
-        units = [(b, g) for b in range(B) for g in range(Hkv)]
-    for b, g in units:
+        units = [(b, x) for b in range(B) for x in range(Hq if per_head else Hkv)]
+    for b, x in units:
+        # x: the unit's row in the selection outputs; g: its KV head; heads [h0, h1)
+        g, h0, h1 = (x // G, x, x + 1) if per_head else (x, x * G, (x + 1) * G)
         N = int(layer.seq_len[b])
-        where = f"unit(b={b},g={g})"
-        Qg = to_np(layer.q[b, g * G:(g + 1) * G])
+        where = f"unit(b={b},{'h' if per_head else 'g'}={x})"
+        Qg = to_np(layer.q[b, h0:h1])
         K = to_np(layer.k[b, g, :N])
         V = to_np(layer.v[b, g, :N])
         if page_size:
@@ -224,13 +238,13 @@ def check_layer(layer, gpu, *, page_size: int, rule: str, budget: dict, scale: f
         # scores (when the call under test reports them)
         S = O.group_reduce(O.head_scores(Qg, meta, rule))
         if gpu.get("scores") is not None:
-            gs = gpu["scores"][b, g, :P].numpy().astype(np.float64)
+            gs = gpu["scores"][b, x, :P].numpy().astype(np.float64)
             err = np.abs(gs - S) / np.maximum(np.abs(S), 1.0)
             stats["max_score_err"] = max(stats["max_score_err"], float(err.max()))
             assert err.max() <= score_rel, f"{where}: score rel err {err.max():.3g}"
         # selection
-        cnt = int(gpu["sel_count"][b, g])
-        gl = gpu["sel_idx"][b, g, :cnt].numpy().astype(np.int64)
+        cnt = int(gpu["sel_count"][b, x])
+        gl = gpu["sel_idx"][b, x, :cnt].numpy().astype(np.int64)
         assert np.all(np.diff(gl) > 0), f"{where}: selection not strictly ascending"
         gset = set(int(x) for x in gl)
         lens = (ends - starts) if not page_size else None
@@ -239,8 +253,8 @@ def check_layer(layer, gpu, *, page_size: int, rule: str, budget: dict, scale: f
         # attention over the pages the GPU kept
         toks = O.tokens_of(gl, starts, ends)
         o_ref, l_ref = O.attend(Qg, K, V, toks, scale)
-        o_gpu = gpu["out"][b, g * G:(g + 1) * G].numpy().astype(np.float64)
-        l_gpu = gpu["lse"][b, g * G:(g + 1) * G].numpy().astype(np.float64)
+        o_gpu = gpu["out"][b, h0:h1].numpy().astype(np.float64)
+        l_gpu = gpu["lse"][b, h0:h1].numpy().astype(np.float64)
         if len(toks) == 0:
             assert np.all(o_gpu == 0) and np.all(np.isneginf(l_gpu)), f"{where}: empty selection"
         else:

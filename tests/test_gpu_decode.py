@@ -75,6 +75,32 @@ def test_tiny_caches(cuda_dev, R, rule, N):
         assert int(g["sel_count"].min()) == min(k, P)
 
 
+@pytest.mark.parametrize("rule", ["envelope", "centroid"])
+@pytest.mark.parametrize("case", ["topk", "ratio", "tokens"])
+def test_per_query_head_selection(cuda_dev, R, rule, case):
+    """One page set per query head: each (sequence, query head) is checked
+    against the oracle run on that head alone (its group is the head itself)."""
+    if case == "tokens":
+        lens = DG.workload3_chunks(2, 2000, seed_offset=9)
+        lay = _layer(cuda_dev, 2, 32, 4, [2000, 2000], seed=91, cap=2000, chunk_lens=lens,
+                     chunk_offset_std=0.5)
+        ps, bd = 0, {"kind": "tokens", "budget": 700}
+    elif case == "ratio":
+        lay = _layer(cuda_dev, 2, 28, 4, [1500, 999], seed=92, cap=1504)
+        ps, bd = 16, {"kind": "ratio", "ratio": 0.0625, "bos": 1, "eos": 1}
+    else:
+        lay = _layer(cuda_dev, 3, 32, 4, [1000, 777, 17], seed=93, cap=1024, key_scale="channel")
+        ps, bd = 16, {"kind": "topk", "k": 20}
+    g = R.run_gpu(lay, page_size=ps, rule=rule, budget=bd, scale=SCALE, per_head=True)
+    assert g["status"] == 0
+    st = R.check_layer(lay, g, page_size=ps, rule=rule, budget=bd, scale=SCALE, per_head=True)
+    assert st["units"] == lay.k.shape[0] * lay.q.shape[1]
+    assert st["max_out_err"] < 1e-4
+    # heads of one group pick different pages (else the variant would be moot)
+    sel = g["sel_idx"]
+    assert not torch.equal(sel[0, 0, :8], sel[0, 1, :8]) or not torch.equal(sel[0, 0, :8], sel[0, 2, :8])
+
+
 def test_exact_duplicate_pages_lowest_index(cuda_dev, R):
     """Identical pages have identical scores; the lower index must win."""
     lay = _layer(cuda_dev, 1, 32, 4, [512], seed=51, cap=512)
