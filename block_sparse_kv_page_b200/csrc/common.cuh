@@ -91,6 +91,17 @@ SA_DEV bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
       : "memory");
   return ok != 0;
 }
+// Non-blocking test of phase `parity` of `bar` (for a thread that polls
+// several barriers in turn).
+SA_DEV bool mbar_test(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}\n"
+      : "=r"(ok)
+      : "r"(smem_addr(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
 // Wait for phase `parity` of `bar`; after kSpinLimit polls give up, flag the
 // status word and return false (the caller stops using the stage).
 SA_DEV bool mbar_wait(uint64_t* bar, uint32_t parity, int* status) {

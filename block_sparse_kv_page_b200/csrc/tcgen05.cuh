@@ -73,6 +73,16 @@ SA_DEV void mma_tf32_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint3
       "l"(a_desc), "l"(b_desc), "r"(idesc), "r"((uint32_t)acc)
       : "memory");
 }
+// D[tmem] (+)= A[tmem] . B[smem]^T: A (M = 128 rows) in tensor memory, row m in
+// lane m, two bf16 of the K axis per 32-bit column (lower K index in the low
+// half), so a K = 16 step starts 8 columns after the previous one.
+SA_DEV void mma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc, bool acc) {
+  asm volatile(
+      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+      " tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n}\n" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"((uint32_t)acc)
+      : "memory");
+}
 // Arrive on `bar` once every tcgen05 operation this thread issued so far is done.
 SA_DEV void commit(uint64_t* bar) {
   asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n" ::"r"(
@@ -91,6 +101,25 @@ SA_DEV void ld_32x32b_x16(uint32_t taddr, uint32_t (&r)[16]) {
       : "r"(taddr));
 }
 SA_DEV void wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;\n" ::: "memory"); }
+// Ties 16 registers filled by ld_32x32b_x16 to this point of the program:
+// placed after wait_ld(), it keeps the compiler from moving their uses above
+// the wait (the asm reads and "writes" them; it emits no instruction).
+SA_DEV void reg_fence(uint32_t (&r)[16]) {
+  asm volatile(""
+               : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]), "+r"(r[7]),
+                 "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]), "+r"(r[14]),
+                 "+r"(r[15])::"memory");
+}
+// Store 16 consecutive fp32 columns of this thread's TMEM lane (same lane
+// mapping as ld_32x32b_x16).  Complete after wait_st().
+SA_DEV void st_32x32b_x16(uint32_t taddr, const uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};\n"
+      ::"r"(taddr), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+      "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
+      : "memory");
+}
+SA_DEV void wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;\n" ::: "memory"); }
 
 }  // namespace tc
 }  // namespace sa

@@ -9,20 +9,23 @@
 // CTA = (tile, KV head, 128 query vectors), one CTA per SM; a query vector is
 // one (row, query head) pair of the tile and owns one lane of tensor memory.
 // Warp-specialised, all waits bounded:
-//   warp 4 (one thread)  streams each kept block (64 keys) of K and V by TMA
+//   warp 8 (one thread)  streams each kept block (64 keys) of K and V by TMA
 //                        into a kStages ring (four 64-row x 128 B boxes);
-//   warp 5 (one thread)  issues, per block i, S_i = Q K_i^T (M = 128 vectors,
+//   warp 9 (one thread)  issues, per block i, S_i = Q K_i^T (M = 128 vectors,
 //                        N = 64 keys, K = 128 dims; K-major operands) into one
-//                        of two S accumulators, and O_i = [P_hi | P_lo] .
-//                        [V_i ; V_i] (N = 128 dims, K = 2 x 64 keys; V read
-//                        MN-major) into one of two O accumulators; QK of the
-//                        next block is issued before PV of this one, so the
+//                        of two S accumulators, and O += [P_hi | P_lo] .
+//                        [V_i ; V_i] (A from tensor memory; N = 128 dims,
+//                        K = 2 x 64 keys; V read MN-major) into the O
+//                        accumulator; QK of the next
+//                        block is issued before PV of this one, so the
 //                        softmax overlaps the tensor cores;
-//   warps 0-3            per vector (thread): mask (causal, cache end), online
-//                        softmax in the log2 domain, P split into a bf16
-//                        hi + lo pair (error ~2^-17) written to shared memory
-//                        as the next MMA's A operand, and the block's O_i
-//                        folded into fp32 registers with the running rescale.
+//   warps 0-7            two per TMEM lane quarter (query vector): mask
+//                        (causal, cache end), online softmax in the log2
+//                        domain against a reference max, P split into a bf16
+//                        hi + lo pair (error ~2^-17) stored to tensor memory
+//                        as the next MMA's A operand; O stays in tensor
+//                        memory and is rescaled in place only when a row's
+//                        max grows by more than 2^8.
 // Accumulation order per vector is the block order of the list, so results
 // do not depend on scheduling.
 #include "common.cuh"
@@ -37,21 +40,23 @@ constexpr int kSmWarps = 8;                    // softmax warps: two per TMEM la
 constexpr int kThreadsTc = 32 * (kSmWarps + 2);
 constexpr int kProducerWarp = kSmWarps;
 constexpr int kMmaWarp = kSmWarps + 1;
-constexpr int kStages = 3;
+#ifndef SA_TA_STAGES
+#define SA_TA_STAGES 3
+#endif
+constexpr int kStages = SA_TA_STAGES;
 constexpr int kBox = kBlk * 128;               // 64 rows x 128 B
 constexpr int kStage = 4 * kBox;               // K lo | K hi | V lo | V hi = 32 KiB
 constexpr int kQBytes = 2 * 128 * 128;         // 128 vectors x 128 dims bf16, two K chunks
-constexpr int kPBytes = 2 * 128 * 128;         // 128 rows x (64 hi | 64 lo) bf16
 constexpr int kOffQ = 0;
 constexpr int kOffRing = kOffQ + kQBytes;
-constexpr int kOffP = kOffRing + kStages * kStage;
-constexpr int kOffBars = kOffP + 2 * kPBytes;
-// kv full/empty, s full/empty, p full, o full/empty, drain
-constexpr int kNumBars = 2 * kStages + 2 * 2 + 2 + 2 * 2 + 1;
+constexpr int kOffBars = kOffRing + kStages * kStage;
+// kv full/empty, s full/empty, p full, o full (PV of even / odd blocks), drain
+constexpr int kNumBars = 2 * kStages + 2 * 2 + 2 + 2 + 1;
 constexpr int kOffRed = kOffBars + kNumBars * 8 + 8;        // softmax row sums, 2 halves x 128 rows
 constexpr int kOffList = kOffRed + 2 * 128 * 4;
 constexpr uint32_t kColS = 0;                  // S accumulators: columns [0, 128)
-constexpr uint32_t kColO = 128;                // O accumulators: columns [128, 384)
+constexpr uint32_t kColO = 128;                // O accumulator: columns [128, 256)
+constexpr uint32_t kColP = 256;                // P_hi | P_lo (bf16 pairs), two buffers: [256, 384)
 static_assert(1024 + kOffList > 114 * 1024, "one CTA per SM: it allocates all 512 TMEM columns");
 
 // MN-major view of V (keys x dims, dims contiguous): 8-key atoms 1 KiB apart,
@@ -76,15 +81,13 @@ __global__ void __launch_bounds__(kThreadsTc, 1) tile_attn_tc_kernel(const __gri
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   unsigned char* qs = base + kOffQ;
   unsigned char* ring = base + kOffRing;
-  unsigned char* pbuf = base + kOffP;
   uint64_t* kv_full = reinterpret_cast<uint64_t*>(base + kOffBars);
   uint64_t* kv_empty = kv_full + kStages;
   uint64_t* s_full = kv_empty + kStages;
   uint64_t* s_empty = s_full + 2;
   uint64_t* p_full = s_empty + 2;
   uint64_t* o_full = p_full + 2;
-  uint64_t* o_empty = o_full + 2;
-  uint64_t* drain = o_empty + 2;
+  uint64_t* drain = o_full + 2;
   int* blist = reinterpret_cast<int*>(base + kOffList);
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -110,7 +113,6 @@ __global__ void __launch_bounds__(kThreadsTc, 1) tile_attn_tc_kernel(const __gri
       mbar_init(s_empty + b, kSmWarps);
       mbar_init(p_full + b, kSmWarps);
       mbar_init(o_full + b, 1);
-      mbar_init(o_empty + b, kSmWarps);
     }
     mbar_init(drain, 1);
     fence_barrier_init();
@@ -183,7 +185,7 @@ __global__ void __launch_bounds__(kThreadsTc, 1) tile_attn_tc_kernel(const __gri
   const bool vok = v < V;
   const int qpos = vok ? a.q_pos0 + row0 + v / G : -1;
   float* red = reinterpret_cast<float*>(base + kOffRed);  // [2 halves][128 rows] row sums
-  float m = ninf, lh = 0.f;
+  float mref = ninf, lh = 0.f;  // reference max (log2 units) and row sum against it
   float o[64];
 #pragma unroll
   for (int d = 0; d < 64; ++d) o[d] = 0.f;
@@ -217,11 +219,12 @@ __global__ void __launch_bounds__(kThreadsTc, 1) tile_attn_tc_kernel(const __gri
     if (lane == 0) {
       const uint32_t idesc_s = tc::idesc_f32acc(tc::kFmtBF16, 128, kBlk);
       const uint32_t idesc_o = tc::idesc_f32acc(tc::kFmtBF16, 128, kHeadDim) | (1u << 16);  // V MN-major
-      auto qk = [&](int i) -> bool {
+      // Both queues are polled without blocking: QK of block i + 1 needs its
+      // K/V stage and a free S buffer, PV of block i needs P_i; whichever is
+      // ready goes first, so a late K/V stage never holds back a PV whose P is
+      // written (and the stage it frees).  QK runs at most one block ahead.
+      auto qk = [&](int i) {
         const int s = i % kStages, b = i & 1;
-        if (!mbar_wait(kv_full + s, (i / kStages) & 1u, a.status)) return false;
-        if (i >= 2 && !mbar_wait(s_empty + b, ((i >> 1) - 1) & 1u, a.status)) return false;
-        tc::fence_after_sync();
         const unsigned char* kb = ring + s * kStage;
 #pragma unroll
         for (int c = 0; c < 2; ++c)
@@ -230,32 +233,39 @@ __global__ void __launch_bounds__(kThreadsTc, 1) tile_attn_tc_kernel(const __gri
             tc::mma_bf16_ss(tmem + kColS + 64u * b, tc::smem_desc_sw128(qs + c * (128 * 128) + 32 * k),
                             tc::smem_desc_sw128(kb + c * kBox + 32 * k), idesc_s, (c | k) != 0);
         tc::commit(s_full + b);
-        return true;
       };
-      auto pv = [&](int i) -> bool {
+      auto pv = [&](int i) {
         const int s = i % kStages, b = i & 1;
-        if (!mbar_wait(p_full + b, (i >> 1) & 1u, a.status)) return false;
-        if (i >= 2 && !mbar_wait(o_empty + b, ((i >> 1) - 1) & 1u, a.status)) return false;
-        tc::fence_after_sync();
         const unsigned char* vb = ring + s * kStage + 2 * kBox;
-        const unsigned char* pb = pbuf + b * kPBytes;
 #pragma unroll
-        for (int h = 0; h < 2; ++h)  // P hi, then P lo, against the same V rows
-#pragma unroll
-          for (int k = 0; k < 4; ++k)
-            tc::mma_bf16_ss(tmem + kColO + 128u * b, tc::smem_desc_sw128(pb + h * (128 * 128) + 32 * k),
-                            v_desc(vb + 16 * 128 * k), idesc_o, (h | k) != 0);
+        for (int j = 0; j < 8; ++j)  // K = [P_hi keys 0-63 | P_lo keys 0-63], 16 per step
+          tc::mma_bf16_ts(tmem + kColO, tmem + kColP + 64u * b + 8u * j, v_desc(vb + 16 * 128 * (j & 3)),
+                          idesc_o, i > 0 || j != 0);
         tc::commit(o_full + b);
         tc::commit(kv_empty + s);
-        return true;
       };
-      if (nb > 0 && !qk(0)) fail = 1;
-      for (int i = 0; i < nb && !fail; ++i) {
-        if (i + 1 < nb && !qk(i + 1)) {
+      int nq = 0, npv = 0;
+      uint32_t idle = 0;
+      while (npv < nb) {
+        bool progress = false;
+        if (nq < nb && nq <= npv + 1 && mbar_test(kv_full + nq % kStages, (nq / kStages) & 1u) &&
+            (nq < 2 || mbar_test(s_empty + (nq & 1), ((nq >> 1) - 1) & 1u))) {
+          tc::fence_after_sync();
+          qk(nq++);
+          progress = true;
+        }
+        if (npv < nq && mbar_test(p_full + (npv & 1), (npv >> 1) & 1u)) {
+          tc::fence_after_sync();
+          pv(npv++);
+          progress = true;
+        }
+        if (progress) {
+          idle = 0;
+        } else if (++idle >= kSpinLimit) {
+          flag_status(a.status, SA_ERR_TIMEOUT);
           fail = 1;
           break;
         }
-        if (!pv(i)) fail = 1;
       }
       // every MMA issued has completed before TMEM is freed (bounded)
       tc::commit(drain);
@@ -263,126 +273,167 @@ __global__ void __launch_bounds__(kThreadsTc, 1) tile_attn_tc_kernel(const __gri
     }
   } else {
     // ---- softmax: TMEM lane r = 32 (warp % 4) + lane is query vector v0 + r;
-    // half h = warp / 4 exponentiates keys [32 h, 32 h + 32) of S and folds
-    // dims [64 h, 64 h + 64) of O.  Both halves read the whole S row, so they
-    // hold the same running max without exchanging anything; their row sums
-    // are added after the CTA's final barrier.
+    // half h = warp / 4 exponentiates keys [32 h, 32 h + 32) of S and owns dims
+    // [64 h, 64 h + 64) of O.  Both halves read the whole S row, so they hold the
+    // same maxima without exchanging anything; their row sums are added after
+    // the CTA's final barrier.  O accumulates in tensor memory over the blocks,
+    // against a reference max mref that may lag the row's running max: P =
+    // 2^(s - mref) stays below 2^8, and O and the row sum are rescaled in place
+    // only when a row's max passes mref by more than 8 (log2 units), which with
+    // bounded scores happens in the first blocks only.
     const uint32_t lane_off = (uint32_t)(32 * quarter) << 16;
-    float alpha_prev = 1.f;
-    for (int i = 0; i <= nb; ++i) {
-      float alpha_cur = 1.f;
-      if (i < nb) {
-        const int b = i & 1;
-        const bool ok = mbar_wait(s_full + b, (i >> 1) & 1u, a.status);
-        if (!__all_sync(0xffffffffu, ok)) {
-          fail = 1;
-          break;
-        }
-        tc::fence_after_sync();
-        const int kb0 = blist[i] * kBlk;
-        const uint32_t ts = tmem + lane_off + kColS + 64u * b;
-        uint32_t r0[16], r1[16], r2[16], r3[16];  // own half: r0, r1; other half: r2, r3
-        tc::ld_32x32b_x16(ts + 32u * h, r0);
-        tc::ld_32x32b_x16(ts + 32u * h + 16, r1);
-        tc::ld_32x32b_x16(ts + 32u * (h ^ 1), r2);
-        tc::ld_32x32b_x16(ts + 32u * (h ^ 1) + 16, r3);
-        tc::wait_ld();
-        tc::fence_before_sync();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(s_empty + b);  // S_i read: the buffer may take S_{i+2}
-        // scores in registers: this half's 32 keys in sv, the row max over all 64.
-        // Blocks fully visible to every row of the warp (all but the diagonal and
-        // the cache end) skip the masks, and with a positive scale the max is
-        // taken on raw scores (scaling commutes with max).
-        const float sl2 = a.scale_log2;
-        const bool fast = sl2 > 0.f && __all_sync(0xffffffffu, kb0 + kBlk - 1 <= qpos && kb0 + kBlk <= N);
-        float sv[32], mx = ninf, mul;
-        if (fast) {
+    const uint32_t to = tmem + lane_off + kColO + 64u * h;
+    int o_seen = 0;  // PV results waited for: blocks [0, o_seen)
+    auto wait_pv = [&](int j) -> bool {  // PV of block j complete (phases in order)
+      const bool ok = mbar_wait(o_full + (j & 1), (j >> 1) & 1u, a.status);
+      return __all_sync(0xffffffffu, ok);
+    };
+    // S of block i in r0..r3 (own half: r0, r1; other half: r2, r3); the loads of
+    // block i + 1 are issued before waiting for PV of block i - 1, so their
+    // latency overlaps that wait
+    uint32_t r0[16], r1[16], r2[16], r3[16];
+    auto load_s = [&](int i) -> bool {
+      const int b = i & 1;
+      const bool ok = mbar_wait(s_full + b, (i >> 1) & 1u, a.status);
+      if (!__all_sync(0xffffffffu, ok)) return false;
+      tc::fence_after_sync();
+      const uint32_t ts = tmem + lane_off + kColS + 64u * b;
+      tc::ld_32x32b_x16(ts + 32u * h, r0);
+      tc::ld_32x32b_x16(ts + 32u * h + 16, r1);
+      tc::ld_32x32b_x16(ts + 32u * (h ^ 1), r2);
+      tc::ld_32x32b_x16(ts + 32u * (h ^ 1) + 16, r3);
+      return true;
+    };
+    if (nb > 0 && !load_s(0)) fail = 1;
+    for (int i = 0; i < nb && !fail; ++i) {
+      const int b = i & 1;
+      tc::wait_ld();
+      tc::reg_fence(r0);
+      tc::reg_fence(r1);
+      tc::reg_fence(r2);
+      tc::reg_fence(r3);
+      tc::fence_before_sync();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(s_empty + b);  // S_i read: the buffer may take S_{i+2}
+      const int kb0 = blist[i] * kBlk;
+      // scores in registers: this half's 32 keys in sv, the row max over all 64.
+      // Blocks fully visible to every row of the warp (all but the diagonal and
+      // the cache end) skip the masks, and with a positive scale the max is
+      // taken on raw scores (scaling commutes with max).
+      const float sl2 = a.scale_log2;
+      const bool fast = sl2 > 0.f && __all_sync(0xffffffffu, kb0 + kBlk - 1 <= qpos && kb0 + kBlk <= N);
+      // (four independent max chains: the reduction is latency-bound)
+      float sv[32], mq[4] = {ninf, ninf, ninf, ninf}, mul;
+      if (fast) {
 #pragma unroll
-          for (int x = 0; x < 16; ++x) {
-            sv[x] = __uint_as_float(r0[x]);
-            sv[16 + x] = __uint_as_float(r1[x]);
-            mx = fmaxf(fmaxf(mx, fmaxf(sv[x], sv[16 + x])),
-                       fmaxf(__uint_as_float(r2[x]), __uint_as_float(r3[x])));
-          }
-          mx *= sl2;
-          mul = sl2;
-        } else {
-          const int kv0 = kb0 + 32 * h, kw0 = kb0 + 32 * (h ^ 1);
-#pragma unroll
-          for (int x = 0; x < 16; ++x) {
-            const int k0 = kv0 + x, k1 = k0 + 16, w0 = kw0 + x, w1 = w0 + 16;
-            sv[x] = (k0 <= qpos && k0 < N) ? __uint_as_float(r0[x]) * sl2 : ninf;
-            sv[16 + x] = (k1 <= qpos && k1 < N) ? __uint_as_float(r1[x]) * sl2 : ninf;
-            const float u0 = (w0 <= qpos && w0 < N) ? __uint_as_float(r2[x]) * sl2 : ninf;
-            const float u1 = (w1 <= qpos && w1 < N) ? __uint_as_float(r3[x]) * sl2 : ninf;
-            mx = fmaxf(mx, fmaxf(fmaxf(sv[x], sv[16 + x]), fmaxf(u0, u1)));
-          }
-          mul = 1.f;
+        for (int x = 0; x < 16; ++x) {
+          sv[x] = __uint_as_float(r0[x]);
+          sv[16 + x] = __uint_as_float(r1[x]);
+          mq[x & 3] = fmaxf(mq[x & 3], fmaxf(fmaxf(sv[x], sv[16 + x]),
+                                             fmaxf(__uint_as_float(r2[x]), __uint_as_float(r3[x]))));
         }
-        const float mn = fmaxf(m, mx);
-        alpha_cur = mn == ninf ? 1.f : fast_exp2(m - mn);
-        const float nmn = mn == ninf ? 0.f : -mn;  // all masked so far: every p is exp2(-inf) = 0
-        // P = exp2(s - m) as a bf16 hi + lo pair, pieces 4 h .. 4 h + 3 of the row
-        unsigned char* prow = pbuf + b * kPBytes;
-        float rs = 0.f;
+        mul = sl2;
+      } else {
+        const int kv0 = kb0 + 32 * h, kw0 = kb0 + 32 * (h ^ 1);
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          uint4 hi, lo;
-          uint32_t* hp = &hi.x;
-          uint32_t* lp = &lo.x;
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const float p0 = fast_exp2(fmaf(sv[8 * q + 2 * e], mul, nmn));
-            const float p1 = fast_exp2(fmaf(sv[8 * q + 2 * e + 1], mul, nmn));
-            rs += p0 + p1;
-            hp[e] = pack_bf16(p0, p1);
-            lp[e] = pack_bf16(p0 - bf16_lo(hp[e]), p1 - bf16_hi(hp[e]));
-          }
-          *reinterpret_cast<uint4*>(prow + swz128(r, 4 * h + q)) = hi;
-          *reinterpret_cast<uint4*>(prow + 128 * 128 + swz128(r, 4 * h + q)) = lo;
+        for (int x = 0; x < 16; ++x) {
+          const int k0 = kv0 + x, k1 = k0 + 16, w0 = kw0 + x, w1 = w0 + 16;
+          sv[x] = (k0 <= qpos && k0 < N) ? __uint_as_float(r0[x]) * sl2 : ninf;
+          sv[16 + x] = (k1 <= qpos && k1 < N) ? __uint_as_float(r1[x]) * sl2 : ninf;
+          const float u0 = (w0 <= qpos && w0 < N) ? __uint_as_float(r2[x]) * sl2 : ninf;
+          const float u1 = (w1 <= qpos && w1 < N) ? __uint_as_float(r3[x]) * sl2 : ninf;
+          mq[x & 3] = fmaxf(mq[x & 3], fmaxf(fmaxf(sv[x], sv[16 + x]), fmaxf(u0, u1)));
         }
-        lh = lh * alpha_cur + rs;
-        m = mn;
-        // V rows past the cache end hold other data: zero them before PV reads them
-        if (kb0 + kBlk > N) {
-          unsigned char* st = ring + (i % kStages) * kStage;
-          for (int x = 32 * warp + lane; x < (kb0 + kBlk - N) * 16; x += 32 * kSmWarps) {
-            const int row = (N - kb0) + (x >> 4), ch = x & 15;
-            *reinterpret_cast<uint4*>(st + (2 + (ch >> 3)) * kBox + swz128(row, ch & 7)) = make_uint4(0u, 0u, 0u, 0u);
-          }
-        }
-        fence_proxy_async();  // P (and zeroed V rows) before the tensor cores read them
-        __syncwarp();
-        if (lane == 0) mbar_arrive(p_full + b);
+        mul = 1.f;
       }
-      if (i >= 1) {
-        // fold O_{i-1} = P_{i-1} V_{i-1} (this half's 64 dims) into the registers
-        const int j = i - 1, b = j & 1;
-        const bool ok = mbar_wait(o_full + b, (j >> 1) & 1u, a.status);
-        if (!__all_sync(0xffffffffu, ok)) {
-          fail = 1;
-          break;
+      float mx = fmaxf(fmaxf(mq[0], mq[1]), fmaxf(mq[2], mq[3]));
+      if (fast) mx *= sl2;
+      // raise the reference max when the row's max passes it by more than 8
+      const float mn = fmaxf(mref, mx);
+      const bool upd = mn != ninf && (mref == ninf || mn > mref + 8.f);
+      const float alpha = !upd ? 1.f : (mref == ninf ? 0.f : fast_exp2(mref - mn));
+      if (upd) mref = mn;
+      lh *= alpha;
+      if (i > 0 && __any_sync(0xffffffffu, upd)) {
+        // O holds blocks [0, i): once the last of them is in, scale this half in place
+        if (o_seen < i) {
+          if (!wait_pv(i - 1)) {
+            fail = 1;
+            break;
+          }
+          o_seen = i;
         }
         tc::fence_after_sync();
-        const uint32_t to = tmem + lane_off + kColO + 128u * b + 64u * h;
 #pragma unroll
-        for (int c8 = 0; c8 < 4; c8 += 2) {
-          uint32_t q0[16], q1[16];
-          tc::ld_32x32b_x16(to + 16 * c8, q0);
-          tc::ld_32x32b_x16(to + 16 * c8 + 16, q1);
+        for (int c = 0; c < 4; ++c) {
+          uint32_t q[16];
+          tc::ld_32x32b_x16(to + 16 * c, q);
           tc::wait_ld();
 #pragma unroll
-          for (int x = 0; x < 16; ++x) {
-            o[16 * c8 + x] = o[16 * c8 + x] * alpha_prev + __uint_as_float(q0[x]);
-            o[16 * c8 + 16 + x] = o[16 * c8 + 16 + x] * alpha_prev + __uint_as_float(q1[x]);
-          }
+          for (int x = 0; x < 16; ++x) q[x] = __float_as_uint(__uint_as_float(q[x]) * alpha);
+          tc::st_32x32b_x16(to + 16 * c, q);
         }
-        tc::fence_before_sync();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(o_empty + b);
+        tc::wait_st();
       }
-      alpha_prev = alpha_cur;
+      const float nmn = mref == ninf ? 0.f : -mref;  // all masked so far: every p is exp2(-inf) = 0
+      // P = exp2(s - mref) as a bf16 hi + lo pair into tensor memory, this
+      // half's keys: hi pairs in columns 16 h .. 16 h + 15, lo pairs 32 further
+      uint32_t phi[16], plo[16];
+      float rq[4] = {0.f, 0.f, 0.f, 0.f};  // four independent partial row sums
+#pragma unroll
+      for (int j = 0; j < 16; ++j) {
+        const float p0 = fast_exp2(fmaf(sv[2 * j], mul, nmn));
+        const float p1 = fast_exp2(fmaf(sv[2 * j + 1], mul, nmn));
+        rq[j & 3] += p0 + p1;
+        // hi = p truncated to bf16 (the upper halves, one byte permute); lo = the
+        // exact remainder p - hi (< 2^-7 p) rounded to bf16: |p - hi - lo| < 2^-16 p
+        phi[j] = pack_bf16(p0, p1);
+        plo[j] = pack_bf16(p0 - bf16_lo(phi[j]), p1 - bf16_hi(phi[j]));
+      }
+      const uint32_t tp = tmem + lane_off + kColP + 64u * b + 16u * h;
+      tc::st_32x32b_x16(tp, phi);
+      tc::st_32x32b_x16(tp + 32, plo);
+      lh += (rq[0] + rq[1]) + (rq[2] + rq[3]);
+      // V rows past the cache end hold other data: zero them before PV reads them
+      if (kb0 + kBlk > N) {
+        unsigned char* st = ring + (i % kStages) * kStage;
+        for (int x = 32 * warp + lane; x < (kb0 + kBlk - N) * 16; x += 32 * kSmWarps) {
+          const int row = (N - kb0) + (x >> 4), ch = x & 15;
+          *reinterpret_cast<uint4*>(st + (2 + (ch >> 3)) * kBox + swz128(row, ch & 7)) = make_uint4(0u, 0u, 0u, 0u);
+        }
+        fence_proxy_async();  // the zeroed V rows before the tensor cores read them
+      }
+      tc::wait_st();
+      tc::fence_before_sync();  // P and the rescaled O before PV_i reads them
+      __syncwarp();
+      if (lane == 0) mbar_arrive(p_full + b);
+      if (i + 1 < nb && !load_s(i + 1)) {
+        fail = 1;
+        break;
+      }
+      // PV_{i-1} done before P_{i+1} overwrites its buffer
+      if (i >= 1 && o_seen < i) {
+        if (!wait_pv(i - 1)) {
+          fail = 1;
+          break;
+        }
+        o_seen = i;
+      }
+    }
+    tc::wait_ld();  // no TMEM load of S left in flight (a failed wait may leave one)
+    // the result: PV of the last block, then this half of O into registers
+    for (int j = o_seen; j < nb && !fail; ++j)
+      if (!wait_pv(j)) fail = 1;
+    if (!fail && nb > 0) {
+      tc::fence_after_sync();
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        uint32_t q[16];
+        tc::ld_32x32b_x16(to + 16 * c, q);
+        tc::wait_ld();
+#pragma unroll
+        for (int x = 0; x < 16; ++x) o[16 * c + x] = __uint_as_float(q[x]);
+      }
     }
     red[h * 128 + r] = lh;  // added to the other half's after the final barrier
   }
@@ -399,7 +450,7 @@ __global__ void __launch_bounds__(kThreadsTc, 1) tile_attn_tc_kernel(const __gri
 #pragma unroll
     for (int d = 0; d < 64; d += 4)
       *reinterpret_cast<float4*>(dst + d) = make_float4(o[d] * inv, o[d + 1] * inv, o[d + 2] * inv, o[d + 3] * inv);
-    if (a.lse && h == 0) a.lse[orow] = l > 0.f ? m * kLn2 + logf(l) : ninf;
+    if (a.lse && h == 0) a.lse[orow] = l > 0.f ? mref * kLn2 + logf(l) : ninf;
   }
 }
 
