@@ -11,6 +11,7 @@ namespace {
 
 using namespace dec;
 
+template <bool PER_HEAD>
 __global__ void __launch_bounds__(kThreads, SA_DEC_CTAS_PER_SM) decode_kernel(const __grid_constant__ DecodeArgs a) {
   extern __shared__ unsigned char smem_raw[];
   __shared__ int s_item, s_last, s_ntiles;
@@ -37,7 +38,7 @@ __global__ void __launch_bounds__(kThreads, SA_DEC_CTAS_PER_SM) decode_kernel(co
     if (item >= a.n_items) break;
     int u, split;
     item_unit(a, item, u, split);
-    decode_item(a, u, split, sm, ws);
+    decode_item<PER_HEAD>(a, u, split, sm, ws);
     fence_proxy_async();  // generic writes to the ring (merge) before the next TMA writes
     __syncthreads();
   }
@@ -99,9 +100,11 @@ cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t st) {
   const long long items = a.n_items;
   long long grid = (long long)device_sm_count() * SA_DEC_CTAS_PER_SM;
   if (grid > items) grid = items;
-  const cudaError_t e = set_smem_attr((const void*)decode_kernel, smem);
+  const void* fn = a.per_head ? (const void*)decode_kernel<true> : (const void*)decode_kernel<false>;
+  const cudaError_t e = set_smem_attr(fn, smem);
   if (e != cudaSuccess) return e;
-  decode_kernel<<<(unsigned)grid, kThreads, smem, st>>>(a);
+  if (a.per_head) decode_kernel<true><<<(unsigned)grid, kThreads, smem, st>>>(a);
+  else decode_kernel<false><<<(unsigned)grid, kThreads, smem, st>>>(a);
   return cudaGetLastError();
 }
 

@@ -122,11 +122,12 @@ SA_DEV void store_out(const DecodeArgs& a, size_t row, int d0, const float (&A)[
   }
 }
 
+template <bool PER_HEAD = false>
 SA_DEV void decode_item(const DecodeArgs& a, const int u, const int split, const Smem& sm,
                         WarpState& ws) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int gq = lane >> 2, c = lane & 3;
-  const UnitMap um = unit_map(u, a.per_head, a.kv.Hkv, a.Hq, a.G);
+  const UnitMap um = unit_map<PER_HEAD>(u, a.kv.Hkv, a.Hq, a.G);
   const int b = um.b;
   const int G = um.n_heads;  // query heads attending this unit's pages
   const float ninf = -__int_as_float(0x7f800000);

@@ -57,9 +57,12 @@ cudaError_t launch_build_meta(const KvView& kv, int rule, int first_token, void*
 struct UnitMap {
   int b, g, kvu, h0, n_heads;
 };
-__host__ __device__ inline UnitMap unit_map(int u, int per_head, int Hkv, int Hq, int G) {
+// PER_HEAD is a compile-time choice: the shared-selection kernels keep their
+// plain (sequence, KV head) indexing.
+template <bool PER_HEAD>
+__host__ __device__ inline UnitMap unit_map(int u, int Hkv, int Hq, int G) {
   UnitMap m;
-  if (per_head) {
+  if (PER_HEAD) {
     m.b = u / Hq;
     m.h0 = u - m.b * Hq;
     m.g = m.h0 / G;

@@ -11,7 +11,7 @@ namespace {
 
 using namespace sel;
 
-template <int RULE>
+template <int RULE, bool PER_HEAD>
 __global__ void __launch_bounds__(kThreads, SA_SEL_CTAS_PER_SM) select_kernel(const __grid_constant__ SelectArgs a) {
   extern __shared__ unsigned char smem_raw[];
   __shared__ uint32_t s_hist[512];
@@ -32,13 +32,13 @@ __global__ void __launch_bounds__(kThreads, SA_SEL_CTAS_PER_SM) select_kernel(co
   if (threadIdx.x == 0) prefetch_tmap(&a.tmap_meta);
   __syncthreads();
   WarpState ws{0u, true, 0u, 0u};
-  const int n_items = a.kv.B * (a.per_head ? a.Hq : a.kv.Hkv) * a.splits;
+  const int n_items = a.kv.B * (PER_HEAD ? a.Hq : a.kv.Hkv) * a.splits;
   for (;;) {
     if (threadIdx.x == 0) s_item = (int)atomicAdd(&a.ws_queue[0], 1u);
     __syncthreads();
     const int item = s_item;
     if (item >= n_items) break;
-    select_item<RULE, false>(a, item / a.splits, item % a.splits, S, ws);
+    select_item<RULE, false, PER_HEAD>(a, item / a.splits, item % a.splits, S, ws);
     fence_proxy_async();  // generic writes to the ring (keys) before the next TMA writes
     __syncthreads();
   }
@@ -86,15 +86,16 @@ cudaError_t launch_select(const SelectArgs& a, cudaStream_t st) {
   if (items > 0x7fffffffLL) return cudaErrorInvalidValue;
   long long grid = (long long)device_sm_count() * SA_SEL_CTAS_PER_SM;
   if (grid > items) grid = items;
-  cudaError_t e;
+  const void* fn = a.rule == 0 ? (a.per_head ? (const void*)select_kernel<0, true> : (const void*)select_kernel<0, false>)
+                                : (a.per_head ? (const void*)select_kernel<1, true> : (const void*)select_kernel<1, false>);
+  const cudaError_t e = set_smem_attr(fn, smem);
+  if (e != cudaSuccess) return e;
   if (a.rule == 0) {
-    e = set_smem_attr((const void*)select_kernel<0>, smem);
-    if (e != cudaSuccess) return e;
-    select_kernel<0><<<(unsigned)grid, kThreads, smem, st>>>(a);
+    if (a.per_head) select_kernel<0, true><<<(unsigned)grid, kThreads, smem, st>>>(a);
+    else select_kernel<0, false><<<(unsigned)grid, kThreads, smem, st>>>(a);
   } else {
-    e = set_smem_attr((const void*)select_kernel<1>, smem);
-    if (e != cudaSuccess) return e;
-    select_kernel<1><<<(unsigned)grid, kThreads, smem, st>>>(a);
+    if (a.per_head) select_kernel<1, true><<<(unsigned)grid, kThreads, smem, st>>>(a);
+    else select_kernel<1, false><<<(unsigned)grid, kThreads, smem, st>>>(a);
   }
   return cudaGetLastError();
 }

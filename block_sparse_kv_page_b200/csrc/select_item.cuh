@@ -463,18 +463,18 @@ SA_DEV void select_unit(const SelectArgs& a, const int u, const int b, const int
 
 // FUSED (the decode step): refresh the newest page while scoring and publish
 // the unit's flag after selecting.
-template <int RULE, bool FUSED>
+template <int RULE, bool FUSED, bool PER_HEAD = false>
 SA_DEV void select_item(const SelectArgs& a, const int u, const int split, const SelSmem& S,
                         WarpState& ws) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int gq = lane >> 2, c = lane & 3;
   const int Hkv = a.kv.Hkv;
-  const UnitMap um = unit_map(u, a.per_head, Hkv, a.Hq, a.G);
+  const UnitMap um = unit_map<PER_HEAD>(u, Hkv, a.Hq, a.G);
   const int b = um.b, kvu = um.kvu;
   // per-query-head units share their KV head's metadata, cache rows and the
   // newest-page refresh: one of them (the first head of the group) stores
   // what is shared, every one patches its own staged copy
-  const bool kv_owner = !a.per_head || um.h0 % a.G == 0;
+  const bool kv_owner = !PER_HEAD || um.h0 % a.G == 0;
 
   // ---- unit geometry (every CTA of the unit computes the same values)
   const int N = a.kv.seq_len[b];
