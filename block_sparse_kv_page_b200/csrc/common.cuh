@@ -125,6 +125,14 @@ SA_DEV void fence_proxy_async() { asm volatile("fence.proxy.async.shared::cta;\n
 // (TMA) ones: global data written with plain stores in the same launch and
 // read by a later TMA copy takes one on each side of the handoff.
 SA_DEV void fence_proxy_async_global() { asm volatile("fence.proxy.async.global;\n" ::: "memory"); }
+// Programmatic dependent launch: a kernel launched with programmatic stream
+// serialisation may start while the previous kernel of the stream is still
+// running; grid_dep_wait() returns once that kernel has completed and its
+// memory operations are visible (at once when there is none), so it goes
+// before the first global access.  grid_dep_trigger() lets the next such
+// kernel begin launching (once every CTA of this grid has triggered or exited).
+SA_DEV void grid_dep_wait() { asm volatile("griddepcontrol.wait;\n" ::: "memory"); }
+SA_DEV void grid_dep_trigger() { asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory"); }
 SA_DEV void prefetch_tmap(const void* tmap) {
   asm volatile("prefetch.tensormap [%0];\n" ::"l"(tmap) : "memory");
 }

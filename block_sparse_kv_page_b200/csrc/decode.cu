@@ -30,12 +30,16 @@ __global__ void __launch_bounds__(kThreads, SA_DEC_CTAS_PER_SM) decode_kernel(co
     prefetch_tmap(&a.tmap_v);
   }
   __syncthreads();
+  grid_dep_wait();  // the previous kernel of the stream has completed (no global access before)
   WarpState ws{0u, true, 0u, 0u};
   for (;;) {
     if (threadIdx.x == 0) s_item = (int)atomicAdd(&a.ws_queue[0], 1u);
     __syncthreads();
     const int item = s_item;
-    if (item >= a.n_items) break;
+    if (item >= a.n_items) {
+      grid_dep_trigger();  // no work left here: the next kernel may start launching
+      break;
+    }
     int u, split;
     item_unit(a, item, u, split);
     decode_item<PER_HEAD>(a, u, split, sm, ws);
@@ -103,9 +107,8 @@ cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t st) {
   const void* fn = a.per_head ? (const void*)decode_kernel<true> : (const void*)decode_kernel<false>;
   const cudaError_t e = set_smem_attr(fn, smem);
   if (e != cudaSuccess) return e;
-  if (a.per_head) decode_kernel<true><<<(unsigned)grid, kThreads, smem, st>>>(a);
-  else decode_kernel<false><<<(unsigned)grid, kThreads, smem, st>>>(a);
-  return cudaGetLastError();
+  return a.per_head ? launch_pdl(decode_kernel<true>, (unsigned)grid, kThreads, smem, st, a)
+                    : launch_pdl(decode_kernel<false>, (unsigned)grid, kThreads, smem, st, a);
 }
 
 }  // namespace sa

@@ -43,6 +43,26 @@ bool encode_tmap_2d(CUtensorMap* map, const void* base, unsigned long long rows,
 // Opt a kernel into `bytes` of dynamic shared memory on the current device
 // (cached per device and kernel, so repeated launches skip the driver call).
 cudaError_t set_smem_attr(const void* func, size_t bytes);
+
+// Launch with programmatic stream serialisation (programmatic dependent
+// launch): the grid may be scheduled while the previous kernel of the stream
+// drains.  Every kernel launched this way calls grid_dep_wait() before its
+// first global access and grid_dep_trigger() once it has no work left.
+template <typename... Params, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(Params...), unsigned grid, unsigned block, size_t smem,
+                       cudaStream_t st, const Args&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(block);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, args...);
+}
 int select_splits(int units, int max_pages, int sm_count);
 WsLayout workspace_layout(const sa_kv_desc* kv, int n_q_heads, int n_q_rows, int max_sel,
                           int sm_count);

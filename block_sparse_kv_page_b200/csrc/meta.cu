@@ -28,6 +28,8 @@ struct MetaParams {
 
 template <int RULE>
 __global__ void __launch_bounds__(kMetaWarps * 32) build_meta_kernel(MetaParams p) {
+  grid_dep_wait();     // the previous kernel of the stream has completed
+  grid_dep_trigger();  // one short pass: the next kernel may start launching
   const int lane = threadIdx.x & 31;
   const long long wid = (long long)blockIdx.x * kMetaWarps + (threadIdx.x >> 5);
   const long long units = (long long)p.kv.B * p.kv.Hkv;
@@ -105,11 +107,8 @@ cudaError_t launch_build_meta(const KvView& kv, int rule, int first_token, void*
   const long long warps = (long long)kv.B * kv.Hkv * ppu;
   const long long blocks = (warps + kMetaWarps - 1) / kMetaWarps;
   if (blocks > 0x7fffffffLL) return cudaErrorInvalidValue;
-  if (rule == 0)
-    build_meta_kernel<0><<<(unsigned)blocks, kMetaWarps * 32, 0, st>>>(p);
-  else
-    build_meta_kernel<1><<<(unsigned)blocks, kMetaWarps * 32, 0, st>>>(p);
-  return cudaGetLastError();
+  if (rule == 0) return launch_pdl(build_meta_kernel<0>, (unsigned)blocks, kMetaWarps * 32, 0, st, p);
+  return launch_pdl(build_meta_kernel<1>, (unsigned)blocks, kMetaWarps * 32, 0, st, p);
 }
 
 }  // namespace sa

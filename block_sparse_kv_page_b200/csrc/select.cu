@@ -31,13 +31,17 @@ __global__ void __launch_bounds__(kThreads, SA_SEL_CTAS_PER_SM) select_kernel(co
   }
   if (threadIdx.x == 0) prefetch_tmap(&a.tmap_meta);
   __syncthreads();
+  grid_dep_wait();  // the previous kernel of the stream has completed (no global access before)
   WarpState ws{0u, true, 0u, 0u};
   const int n_items = a.kv.B * (PER_HEAD ? a.Hq : a.kv.Hkv) * a.splits;
   for (;;) {
     if (threadIdx.x == 0) s_item = (int)atomicAdd(&a.ws_queue[0], 1u);
     __syncthreads();
     const int item = s_item;
-    if (item >= n_items) break;
+    if (item >= n_items) {
+      grid_dep_trigger();  // no work left here: the next kernel may start launching
+      break;
+    }
     select_item<RULE, false, PER_HEAD>(a, item / a.splits, item % a.splits, S, ws);
     fence_proxy_async();  // generic writes to the ring (keys) before the next TMA writes
     __syncthreads();
@@ -90,14 +94,12 @@ cudaError_t launch_select(const SelectArgs& a, cudaStream_t st) {
                                 : (a.per_head ? (const void*)select_kernel<1, true> : (const void*)select_kernel<1, false>);
   const cudaError_t e = set_smem_attr(fn, smem);
   if (e != cudaSuccess) return e;
-  if (a.rule == 0) {
-    if (a.per_head) select_kernel<0, true><<<(unsigned)grid, kThreads, smem, st>>>(a);
-    else select_kernel<0, false><<<(unsigned)grid, kThreads, smem, st>>>(a);
-  } else {
-    if (a.per_head) select_kernel<1, true><<<(unsigned)grid, kThreads, smem, st>>>(a);
-    else select_kernel<1, false><<<(unsigned)grid, kThreads, smem, st>>>(a);
-  }
-  return cudaGetLastError();
+  const unsigned g = (unsigned)grid;
+  if (a.rule == 0)
+    return a.per_head ? launch_pdl(select_kernel<0, true>, g, kThreads, smem, st, a)
+                      : launch_pdl(select_kernel<0, false>, g, kThreads, smem, st, a);
+  return a.per_head ? launch_pdl(select_kernel<1, true>, g, kThreads, smem, st, a)
+                    : launch_pdl(select_kernel<1, false>, g, kThreads, smem, st, a);
 }
 
 }  // namespace sa

@@ -91,6 +91,7 @@ __global__ void __launch_bounds__(kThreads, SA_STEP_CTAS_PER_SM)
     prefetch_tmap(&a.dec.tmap_v);
   }
   __syncthreads();
+  grid_dep_wait();  // the previous kernel of the stream has completed (no global access before)
   WarpState ws{0u, true, 0u, 0u};
   const int n_items = a.n_score + a.n_dec;
   for (;;) {
@@ -106,7 +107,10 @@ __global__ void __launch_bounds__(kThreads, SA_STEP_CTAS_PER_SM)
     }
     __syncthreads();
     const int item = s_item;
-    if (item >= n_items) break;
+    if (item >= n_items) {
+      grid_dep_trigger();  // no work left here: the next kernel may start launching
+      break;
+    }
     if (item < a.n_score) {
       sel::select_item<RULE, true>(a.sel, item / a.sel.splits, item % a.sel.splits, S, ws);
     } else {
@@ -189,11 +193,8 @@ cudaError_t launch_step(const StepArgs& a, cudaStream_t st) {
   if (occ > SA_STEP_CTAS_PER_SM) occ = SA_STEP_CTAS_PER_SM;
   long long grid = (long long)device_sm_count() * occ;
   if (grid > items) grid = items;
-  if (a.sel.rule == 0)
-    step_kernel<0><<<(unsigned)grid, kThreads, smem, st>>>(a);
-  else
-    step_kernel<1><<<(unsigned)grid, kThreads, smem, st>>>(a);
-  return cudaGetLastError();
+  if (a.sel.rule == 0) return launch_pdl(step_kernel<0>, (unsigned)grid, kThreads, smem, st, a);
+  return launch_pdl(step_kernel<1>, (unsigned)grid, kThreads, smem, st, a);
 }
 
 }  // namespace sa
