@@ -514,6 +514,44 @@ def run_gpu_arm(args, rank, world, dist):
         if sa.sparse_attn_get_device_status(ws_h) != 0:
             raise RuntimeError("per-head leg: device status set")
         del ws_h, sel_h, cnt_h
+        # the router applied to decode: each (layer) row is a one-row tile; top k pages,
+        # top 2k for the sequences whose sigma_bar falls below the 0.25 quantile
+        rho, W = 2, 2 * k
+        ws_r = sa.make_workspace(kv, HQ, L * B, W)
+        idx_r = torch.zeros((L * B, HKV, W), dtype=torch.int32, device=dev)
+        cnt_r = torch.zeros((L * B, HKV), dtype=torch.int32, device=dev)
+        sig_r = torch.zeros((L * B, HKV), dtype=torch.float32, device=dev)
+        sbar_r = torch.zeros((L * B,), dtype=torch.float32, device=dev)
+        trig_r = torch.zeros((L * B,), dtype=torch.uint8, device=dev)
+        for rule in ("envelope", "centroid"):
+            def routed_step():
+                sa.sparse_attn_build_meta(kv, rule, -1, metas[rule])
+                sa.sparse_attn_route_decode(kv, metas[rule], rule, inp["q"], k, rho, 0.25, None, idx_r, cnt_r,
+                                            sig_r, sbar_r, trig_r, None, ws_r)
+                sa.sparse_attn_decode(kv, inp["q"], L * B, 0, 1, scale, idx_r, cnt_r, W, out, lse, ws_r)
+            for _ in range(max(3, args.warmup)):
+                routed_step()
+            barrier()
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            n_rep = max(10, args.steps // 2)
+            e0.record(stream)
+            for _ in range(n_rep):
+                routed_step()
+            e1.record(stream)
+            torch.cuda.synchronize()
+            m2 = max_over_ranks(e0.elapsed_time(e1) / n_rep, dist, dev)
+            kept = int(cnt_r.sum().item())
+            kv_r = kept * PS * 2 * D * 2
+            extra[f"router-decode/{rule}"] = {
+                "ms_per_step": round(m2, 4), "value": kept * PS * (HQ // HKV) * world / (m2 * 1e-3),
+                "eff_GBps": (meta_bytes + kv_r) / (m2 * 1e-3) / 1e9,
+                "triggered_rows": int(trig_r.sum().item()), "pages_kept_per_unit": round(kept / (L * B * HKV), 1),
+                "note": "three launches per step (metadata refresh; score-only pass + router selection; decode "
+                        "over the routed lists); k = 256 pages, rho = 2, quantile 0.25 over the 48 rows"}
+        if sa.sparse_attn_get_device_status(ws_r) != 0:
+            raise RuntimeError("router-decode leg: device status set")
+        del ws_r, idx_r, cnt_r, sig_r, sbar_r, trig_r
     for g in graphs.values():
         del g
     graphs.clear()

@@ -10,7 +10,8 @@ from .ops import (KvCache, SparseAttnError, budget_ratio, budget_tokens, budget_
                   sparse_attn_workspace_size_per_head,
                   sparse_attn_decode_static, sparse_attn_decode_step,
                   sparse_attn_decode_step_append,
-                  sparse_attn_get_device_status, sparse_attn_route, sparse_attn_select,
+                  sparse_attn_get_device_status, sparse_attn_route, sparse_attn_route_decode,
+                  sparse_attn_select,
                   sparse_attn_status_string, sparse_attn_workspace_init,
                   sparse_attn_workspace_size)
 from ._abi import (SA_BUDGET_RATIO, SA_BUDGET_TOKENS, SA_BUDGET_TOPK, SA_ERR_CUDA,  # noqa: F401

@@ -116,6 +116,12 @@ int max_tiles_per_unit(const sa_kv_desc* kv, int max_sel) {
 // selecting CTA can read a row with 16-byte loads.
 int score_stride(const sa_kv_desc* kv) { return (kv->max_pages + 3) & ~3; }
 
+// Decode router scratch after the scores: lists [units][W], sigma (double)
+// and eligible counts per unit.
+size_t route_decode_ws_bytes(long long units, int W) {
+  return align256((size_t)units * W * 4) + align256((size_t)units * 8) + align256((size_t)units * 4);
+}
+
 size_t select_scratch(const sa_kv_desc* kv, bool per_head = false, int n_q_heads = 0) {
   const size_t units = (size_t)kv->batch * (per_head ? n_q_heads : kv->n_kv_heads);
   return align256(units * score_stride(kv) * sizeof(float));
@@ -323,6 +329,7 @@ bool fill_select(SelectArgs* a, const sa_kv_desc* kv, const void* meta, sa_score
   a->splits = select_splits(kv->batch * kv->n_kv_heads, kv->max_pages, device_sm_count());
   a->meta_refresh = nullptr;
   a->per_head = 0;
+  a->score_only = 0;
   a->k_new = a->v_new = nullptr;
   a->k_dst = a->v_dst = nullptr;
   return true;
@@ -387,6 +394,10 @@ size_t sparse_attn_workspace_size(const sa_kv_desc* kv, int32_t n_q_heads, int32
   const int route_tiles = rows < kMaxRouteTiles ? rows : kMaxRouteTiles;  // tiles <= query rows
   const size_t rt = route_ws_bytes(route_tiles, kv->n_kv_heads, kv->max_pages, max_sel);
   if (rt > tail) tail = rt;
+  if (kv->batch <= kMaxRouteTiles && kv->page_size > 0) {  // decode router: scores + router scratch
+    const size_t rd = select_scratch(kv) + route_decode_ws_bytes(kv->batch * kv->n_kv_heads, max_sel);
+    if (rd > tail) tail = rd;
+  }
   return kScratch + tail;
 }
 
@@ -681,6 +692,76 @@ sa_status sparse_attn_route(const sa_kv_desc* kv, const void* meta, sa_score_rul
     return SA_ERR_CUDA;
   }
   return launched(launch_route(a, (cudaStream_t)stream));
+}
+
+sa_status sparse_attn_route_decode(const sa_kv_desc* kv, const void* meta, sa_score_rule rule,
+                                   const void* q, int32_t n_q_heads, int32_t k, int32_t rho,
+                                   float quantile, const float* tau, int32_t* kv_idx,
+                                   int32_t* kv_count, float* sigma, float* sigma_bar,
+                                   uint8_t* triggered, float* tau_out, void* ws, size_t ws_bytes,
+                                   void* stream) {
+  if (!kv || kv->page_size <= 0) return kv ? SA_ERR_UNSUPPORTED : SA_ERR_INVALID;
+  if (k < 1 || rho < 1) return SA_ERR_INVALID;
+  if (!(quantile >= 0.f && quantile <= 1.f)) return SA_ERR_INVALID;
+  if (!kv_idx || !kv_count || !sigma || !sigma_bar || !triggered) return SA_ERR_INVALID;
+  if (!aligned(sigma, 4) || !aligned(sigma_bar, 4) || (tau && !aligned(tau, 4)) ||
+      (tau_out && !aligned(tau_out, 4)))
+    return SA_ERR_INVALID;
+  const long long W = (long long)rho * k;
+  if (W > kMaxRouteList || (long long)k + 1 > kMaxRouteList + 1) return SA_ERR_UNSUPPORTED;
+  if (kv->batch > kMaxRouteTiles) return SA_ERR_UNSUPPORTED;
+  // the scores: the decode scoring items in score-only mode
+  int G;
+  const sa_budget dummy{SA_BUDGET_TOPK, 1, 0.f, 0, 0, 0, 0};
+  sa_status s = check_select(kv, meta, rule, q, n_q_heads, &dummy, (int)W, kv_idx, kv_count, nullptr, &G);
+  if (s != SA_OK) return s;
+  const long long units = (long long)kv->batch * kv->n_kv_heads;
+  const size_t sel_bytes = select_scratch(kv);
+  const size_t need = kScratch + sel_bytes + route_decode_ws_bytes(units, (int)W);
+  if ((s = check_ws(ws, ws_bytes, need)) != SA_OK) return s;
+  if (route_decode_smem_bytes(kv->max_pages, (int)W, k, kv->batch) > 227 * 1024) return SA_ERR_UNSUPPORTED;
+  SelectArgs sa_;
+  if (!fill_select(&sa_, kv, meta, rule, q, n_q_heads, G, &dummy, (int)W, kv_idx, kv_count, nullptr, ws))
+    return SA_ERR_CUDA;
+  sa_.score_only = 1;
+  sa_.ws_queue = reinterpret_cast<uint32_t*>(reinterpret_cast<char*>(ws) + kQueueSelect);
+  if ((s = launched(launch_select(sa_, (cudaStream_t)stream))) != SA_OK) return s;
+
+  // the router's selection, sigma, quantile, triggers and lists over those scores
+  RouteArgs a;
+  memset(&a, 0, sizeof(a));
+  a.kv = view(kv);
+  a.rule = (int)rule;
+  a.q = q;
+  a.Hq = n_q_heads;
+  a.G = G;
+  a.n_rows = kv->batch;
+  a.q_pos0 = 0;
+  a.tile_rows = 1;
+  a.n_tiles = kv->batch;
+  a.k = k;
+  a.rho = rho;
+  a.W = (int)W;
+  a.nsplit = 1;
+  a.quantile = quantile;
+  a.tau_in = tau;
+  a.kv_idx = kv_idx;
+  a.kv_count = kv_count;
+  a.sigma = sigma;
+  a.sigma_bar = sigma_bar;
+  a.triggered = triggered;
+  a.tau_out = tau_out;
+  a.ws_keys = nullptr;
+  a.dec_scores = sa_.ws_scores;
+  a.dec_stride = score_stride(kv);
+  char* rbase = reinterpret_cast<char*>(ws) + kScratch + sel_bytes;
+  a.ws_list = reinterpret_cast<int32_t*>(rbase);
+  a.ws_sigma = reinterpret_cast<double*>(rbase + align256((size_t)units * W * 4));
+  a.ws_elig = reinterpret_cast<int32_t*>(rbase + align256((size_t)units * W * 4) + align256((size_t)units * 8));
+  a.ws_count = reinterpret_cast<uint32_t*>(reinterpret_cast<char*>(ws) + 256);
+  a.ws_final = reinterpret_cast<uint32_t*>(reinterpret_cast<char*>(ws) + kQueueRoute);
+  a.status = reinterpret_cast<int*>(ws);
+  return launched(launch_route_decode(a, (cudaStream_t)stream));
 }
 
 sa_status sparse_attn_get_device_status(void* ws, sa_status* host_out, void* stream) {

@@ -107,6 +107,7 @@ struct SelectArgs {
   int budget_kind, top_k, topk_val, bos, eos, token_budget;
   double ratio;
   int per_head;               // 1: one unit per (sequence, query head), else per (sequence, KV head)
+  int score_only;             // 1: group scores to ws_scores only (no selection, sel_* unused)
   int max_sel;
   int32_t* sel_idx;
   int32_t* sel_count;
@@ -213,6 +214,8 @@ struct RouteArgs {
   uint8_t* triggered;
   float* tau_out;
   uint32_t* ws_keys;          // [n_tiles][Hkv][max_pages] tile-score keys (zeroed before launch)
+  const float* dec_scores;    // decode router: group scores [B*Hkv][dec_stride] (the tiles are
+  int dec_stride;             // the sequences, one query row each); null for query tiles
   int32_t* ws_list;           // [n_tiles][Hkv][W] rank-ordered lists
   double* ws_sigma;           // [n_tiles][Hkv]
   int32_t* ws_elig;           // [n_tiles][Hkv] eligible block counts
@@ -221,6 +224,9 @@ struct RouteArgs {
   int* status;
 };
 cudaError_t launch_route(const RouteArgs& a, cudaStream_t st);
+// Decode router tail: one CTA per (sequence, KV head) over dec_scores.
+cudaError_t launch_route_decode(const RouteArgs& a, cudaStream_t st);
+size_t route_decode_smem_bytes(int max_pages, int W, int k, int n_tiles);
 // Router scratch: keys, lists, sigma and eligible counts for n_tiles x Hkv.
 size_t route_ws_bytes(int n_tiles, int Hkv, int max_pages, int W);
 int route_splits(int vectors_per_tile);

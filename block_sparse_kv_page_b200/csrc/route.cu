@@ -74,12 +74,14 @@ SA_DEV void route_select_tile(const RouteArgs& a, int t, int g, int E, unsigned 
   uint32_t* keys = reinterpret_cast<uint32_t*>(smem);                         // [E]
   unsigned long long* cand = reinterpret_cast<unsigned long long*>(smem + ((E * 4 + 15) & ~15));
   uint32_t* kp = a.ws_keys + (size_t)tg * a.kv.max_pages;
+  const float* sp = a.dec_scores ? a.dec_scores + (size_t)tg * a.dec_stride : nullptr;
   for (int b = 0; b < E; b += 8 * (int)blockDim.x) {  // 8 loads in flight per thread
     uint32_t v[8];
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
       const int i = b + j * (int)blockDim.x + tid;
-      v[j] = i < E ? __ldcg(kp + i) : 0u;
+      // tile-score keys, or (decode router) group scores turned into keys
+      v[j] = i >= E ? 0u : (sp ? order_key(__ldcg(sp + i)) : __ldcg(kp + i));
     }
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
@@ -246,6 +248,46 @@ SA_DEV void route_tail(const RouteArgs& a, int t, int g, int E, unsigned char* b
   __syncthreads();
   if (!*flag) return;
   if (tid == 0) *a.ws_final = 0;
+  route_finalize(a, base);
+}
+
+// ---------------------------------------------------------------- decode router
+// The router applied to decode: every sequence of the batch is a tile of one
+// query row (position N_b - 1), so all of its pages are eligible and its
+// block scores are the group scores the decode scoring wrote (max over the G
+// heads).  CTA = (sequence, KV head): rank-order selection and sigma; the last
+// CTA computes sigma_bar, the quantile threshold over the batch's sequences,
+// the triggers and the sentinel-padded lists.
+constexpr int kRdThreads = 256;
+
+__global__ void __launch_bounds__(kRdThreads) route_decode_kernel(const __grid_constant__ RouteArgs a) {
+  extern __shared__ unsigned char smem_raw[];
+  __shared__ uint32_t s_hist[512];
+  __shared__ uint32_t s_scan[32];
+  __shared__ uint32_t s_bc[8];
+  __shared__ int s_flag;
+  unsigned char* base = reinterpret_cast<unsigned char*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 15) & ~static_cast<uintptr_t>(15));
+  grid_dep_wait();  // the scores come from the previous kernel of the stream
+  const int tg = blockIdx.x;
+  const int b = tg / a.kv.Hkv, g = tg - b * a.kv.Hkv;
+  const int N = a.kv.seq_len[b];
+  int E = 0;
+  if (N < 1 || N > a.kv.cap) {
+    if (threadIdx.x == 0 && g == 0) flag_status(a.status, SA_ERR_DEVICE_CHECK);
+  } else {
+    E = (N + a.kv.page_size - 1) / a.kv.page_size;
+    if (E > a.kv.max_pages) {
+      if (threadIdx.x == 0 && g == 0) flag_status(a.status, SA_ERR_DEVICE_CHECK);
+      E = 0;
+    }
+  }
+  route_select_tile(a, b, g, E, base, s_hist, s_bc, s_scan);
+  __syncthreads();
+  if (threadIdx.x == 0) s_flag = atom_add_acq_rel_u32(a.ws_final, 1u) == (uint32_t)(gridDim.x - 1);
+  __syncthreads();
+  if (!s_flag) return;
+  if (threadIdx.x == 0) *a.ws_final = 0;
   route_finalize(a, base);
 }
 
@@ -722,6 +764,23 @@ size_t route_ws_bytes(int n_tiles, int Hkv, int max_pages, int W) {
   auto al = [](size_t x) { return (x + 255) & ~(size_t)255; };
   const size_t tg = (size_t)n_tiles * Hkv;
   return al(tg * max_pages * 4) + al(tg * W * 4) + al(tg * 8) + al(tg * 4);
+}
+
+size_t route_decode_smem_bytes(int max_pages, int W, int k, int n_tiles) {
+  int cap = W > k + 1 ? W : k + 1;
+  if (cap > max_pages) cap = max_pages;
+  int n2 = 1;
+  while (n2 < cap) n2 <<= 1;
+  const size_t sel = (((size_t)max_pages * 4 + 15) & ~(size_t)15) + (size_t)n2 * 8;
+  const size_t fin = (size_t)n_tiles * 16;
+  return 16 + (sel > fin ? sel : fin);
+}
+
+cudaError_t launch_route_decode(const RouteArgs& a, cudaStream_t st) {
+  const size_t smem = route_decode_smem_bytes(a.kv.max_pages, a.W, a.k, a.n_tiles);
+  const cudaError_t e = set_smem_attr((const void*)route_decode_kernel, smem);
+  if (e != cudaSuccess) return e;
+  return launch_pdl(route_decode_kernel, (unsigned)(a.n_tiles * a.kv.Hkv), kRdThreads, smem, st, a);
 }
 
 cudaError_t launch_route(const RouteArgs& a, cudaStream_t st) {

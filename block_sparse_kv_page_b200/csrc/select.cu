@@ -11,8 +11,11 @@ namespace {
 
 using namespace sel;
 
-template <int RULE, bool PER_HEAD>
+// MODE 0: one page set per (sequence, KV head); 1: per (sequence, query head);
+// 2: group scores only.
+template <int RULE, int MODE>
 __global__ void __launch_bounds__(kThreads, SA_SEL_CTAS_PER_SM) select_kernel(const __grid_constant__ SelectArgs a) {
+  constexpr bool PER_HEAD = MODE == 1;
   extern __shared__ unsigned char smem_raw[];
   __shared__ uint32_t s_hist[512];
   __shared__ uint32_t s_scan[32];
@@ -42,7 +45,7 @@ __global__ void __launch_bounds__(kThreads, SA_SEL_CTAS_PER_SM) select_kernel(co
       grid_dep_trigger();  // no work left here: the next kernel may start launching
       break;
     }
-    select_item<RULE, false, PER_HEAD>(a, item / a.splits, item % a.splits, S, ws);
+    select_item<RULE, false, PER_HEAD, MODE == 2>(a, item / a.splits, item % a.splits, S, ws);
     fence_proxy_async();  // generic writes to the ring (keys) before the next TMA writes
     __syncthreads();
   }
@@ -90,16 +93,13 @@ cudaError_t launch_select(const SelectArgs& a, cudaStream_t st) {
   if (items > 0x7fffffffLL) return cudaErrorInvalidValue;
   long long grid = (long long)device_sm_count() * SA_SEL_CTAS_PER_SM;
   if (grid > items) grid = items;
-  const void* fn = a.rule == 0 ? (a.per_head ? (const void*)select_kernel<0, true> : (const void*)select_kernel<0, false>)
-                                : (a.per_head ? (const void*)select_kernel<1, true> : (const void*)select_kernel<1, false>);
-  const cudaError_t e = set_smem_attr(fn, smem);
+  const int mode = a.score_only ? 2 : (a.per_head ? 1 : 0);
+  void (*const fns[2][3])(SelectArgs) = {{select_kernel<0, 0>, select_kernel<0, 1>, select_kernel<0, 2>},
+                                         {select_kernel<1, 0>, select_kernel<1, 1>, select_kernel<1, 2>}};
+  auto fn = fns[a.rule == 0 ? 0 : 1][mode];
+  const cudaError_t e = set_smem_attr((const void*)fn, smem);
   if (e != cudaSuccess) return e;
-  const unsigned g = (unsigned)grid;
-  if (a.rule == 0)
-    return a.per_head ? launch_pdl(select_kernel<0, true>, g, kThreads, smem, st, a)
-                      : launch_pdl(select_kernel<0, false>, g, kThreads, smem, st, a);
-  return a.per_head ? launch_pdl(select_kernel<1, true>, g, kThreads, smem, st, a)
-                    : launch_pdl(select_kernel<1, false>, g, kThreads, smem, st, a);
+  return launch_pdl(fn, (unsigned)grid, kThreads, smem, st, a);
 }
 
 }  // namespace sa

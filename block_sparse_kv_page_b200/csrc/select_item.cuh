@@ -463,7 +463,9 @@ SA_DEV void select_unit(const SelectArgs& a, const int u, const int b, const int
 
 // FUSED (the decode step): refresh the newest page while scoring and publish
 // the unit's flag after selecting.
-template <int RULE, bool FUSED, bool PER_HEAD = false>
+// SCORE_ONLY: write the group scores and stop (no selection; the unit
+// counters are not touched).
+template <int RULE, bool FUSED, bool PER_HEAD = false, bool SCORE_ONLY = false>
 SA_DEV void select_item(const SelectArgs& a, const int u, const int split, const SelSmem& S,
                         WarpState& ws) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -670,6 +672,7 @@ SA_DEV void select_item(const SelectArgs& a, const int u, const int split, const
     }
   }
   ws.gi += (uint32_t)n_it;
+  if (SCORE_ONLY) return;
 
   // ---- the last CTA of the unit selects (its counter increment is acq_rel:
   // it publishes this CTA's scores and acquires those of the other splits)

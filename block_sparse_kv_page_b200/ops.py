@@ -247,6 +247,24 @@ def sparse_attn_decode_static(kv: KvCache, q: torch.Tensor, n_q_rows: int, q_pos
            "sparse_attn_decode_static")
 
 
+def sparse_attn_route_decode(kv: KvCache, meta: torch.Tensor, rule, q: torch.Tensor, k: int, rho: int,
+                             quantile: float, tau: torch.Tensor | None, kv_idx: torch.Tensor,
+                             kv_count: torch.Tensor, sigma: torch.Tensor, sigma_bar: torch.Tensor,
+                             triggered: torch.Tensor, tau_out: torch.Tensor | None, ws: torch.Tensor,
+                             stream=None) -> None:
+    """The router with one-row tiles: every sequence's decode query is a tile.
+    kv_idx [B, Hkv, rho*k] rank-ordered, -1 padded; kv_count [B, Hkv];
+    sigma [B, Hkv]; sigma_bar [B]; triggered [B] uint8."""
+    if q.dtype != torch.bfloat16 or not q.is_contiguous():
+        raise ValueError("q must be contiguous bf16 [B, Hq, 128]")
+    _check(lib.sparse_attn_route_decode(C.byref(kv.desc), meta.data_ptr(), _rule(rule), q.data_ptr(),
+                                        q.shape[-2], int(k), int(rho), float(quantile), _ptr(tau),
+                                        kv_idx.data_ptr(), kv_count.data_ptr(), sigma.data_ptr(),
+                                        sigma_bar.data_ptr(), triggered.data_ptr(), _ptr(tau_out),
+                                        ws.data_ptr(), ws.numel() * ws.element_size(), _stream(stream)),
+           "sparse_attn_route_decode")
+
+
 def sparse_attn_route(kv: KvCache, meta: torch.Tensor, rule, q: torch.Tensor, n_q_rows: int,
                       q_pos0: int, tile_rows: int, k: int, rho: int, quantile: float,
                       tau: torch.Tensor | None, kv_idx: torch.Tensor, kv_count: torch.Tensor,

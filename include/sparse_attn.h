@@ -274,6 +274,29 @@ sa_status sparse_attn_route(const sa_kv_desc* kv, const void* meta, sa_score_rul
                             uint8_t* triggered, float* tau_out, void* ws, size_t ws_bytes,
                             void* stream);
 
+/* (d') The router applied to decode ([ROUTER] "Methodologie" steps 2-5 with
+ * tiles of one query row): every sequence b of the batch is a tile whose one
+ * row sits at position N_b - 1, so all P_b = ceil(N_b / page_size) pages are
+ * eligible, and its block score for KV head g is the decode group score
+ * (max over the G heads of the envelope or centroid score, as in
+ * sparse_attn_select).  sigma[b][g] from the descending scores (1 if P_b <= k,
+ * 0 if s_(0) = s_(k)); sigma_bar[b] = mean over kv heads; tau = the
+ * linear-interpolation quantile `quantile` of sigma_bar over the batch's
+ * sequences (or *tau if tau is non-null); triggered[b] = sigma_bar[b] < tau.
+ * kv_idx[b][g][0 .. rho*k) lists pages in RANK order (score descending, lower
+ * index first): the first min(rho*k, P_b) if triggered else the first
+ * min(k, P_b), padded with -1; kv_count[b][g] = number of valid entries, so
+ * sparse_attn_decode(..., idx = kv_idx, count = kv_count, max_sel = rho*k)
+ * attends exactly the listed pages.  Fixed pages only (page_size > 0), B <=
+ * 1024, rho*k <= 1023; the workspace sized by sparse_attn_workspace_size with
+ * max_sel >= rho*k.  tau_out (nullable): the threshold used.  Two launches. */
+sa_status sparse_attn_route_decode(const sa_kv_desc* kv, const void* meta, sa_score_rule rule,
+                                   const void* q, int32_t n_q_heads, int32_t k, int32_t rho,
+                                   float quantile, const float* tau, int32_t* kv_idx,
+                                   int32_t* kv_count, float* sigma, float* sigma_bar,
+                                   uint8_t* triggered, float* tau_out, void* ws, size_t ws_bytes,
+                                   void* stream);
+
 /* Copy the workspace status word to *host_out (SA_OK if no device check
  * fired since the last init/clear) and clear it.  Synchronises `stream`. */
 sa_status sparse_attn_get_device_status(void* ws, sa_status* host_out, void* stream);

@@ -414,6 +414,44 @@ def route(Q, metas, rule: str, *, q_pos0: int, tile_rows: int, block_size: int,
     return RouteResult(kv_idx, kv_count, sigma, sigma_bar, float(tau), triggered, scores)
 
 
+def route_decode(unit_scores, *, k: int, rho: int, quantile: float, tau=None) -> RouteResult:
+    """Steps 3-5 with tiles of one query row: in a decode batch, sequence b is
+    a tile whose only row is its newest token, so every page of the sequence
+    is eligible, and its block scores for KV head g are the decode group
+    scores S(p) (group_reduce of head_scores).  unit_scores[b][g]: those
+    scores, [P_b].  sigma per (b, g) on the descending scores, sigma_bar the
+    mean over KV heads, tau the linear quantile of sigma_bar over the batch's
+    sequences (or the given tau), trigger iff sigma_bar < tau; lists in rank
+    order, the first rho*k (triggered) or k pages, padded with -1."""
+    B = len(unit_scores)
+    Hkv = len(unit_scores[0])
+    W = rho * k
+    Pmax = max(len(unit_scores[b][g]) for b in range(B) for g in range(Hkv))
+    kv_idx = np.full((B, Hkv, W), -1, dtype=np.int64)
+    kv_count = np.zeros((B, Hkv), dtype=np.int64)
+    sigma = np.zeros((B, Hkv))
+    scores = np.full((B, Hkv, Pmax), NEG_INF)
+    orders = {}
+    for b in range(B):
+        for g in range(Hkv):
+            S = f64(unit_scores[b][g])
+            scores[b, g, :len(S)] = S
+            order = rank_order(S)
+            orders[(b, g)] = order
+            sigma[b, g] = sigma_margin(S[order], k)
+    sigma_bar = sigma.mean(axis=1)
+    if tau is None:
+        tau = quantile_linear(sigma_bar, quantile)
+    triggered = sigma_bar < tau
+    for b in range(B):
+        for g in range(Hkv):
+            order = orders[(b, g)]
+            n = min(W if triggered[b] else k, len(order))
+            kv_idx[b, g, :n] = order[:n]
+            kv_count[b, g] = n
+    return RouteResult(kv_idx, kv_count, sigma, sigma_bar, float(tau), triggered, scores)
+
+
 def tile_attention(Q, K, V, kv_idx, *, q_pos0: int, tile_rows: int,
                    block_size: int, n_tokens: int, scale: float):
     """Causal softmax attention of every query row over the tokens of its

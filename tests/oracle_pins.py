@@ -407,6 +407,52 @@ def check_router_invariants(route, page_metadata, fixed_pages) -> bool:
     return True
 
 
+def check_route_decode(route_decode, route, page_metadata, fixed_pages, head_scores, group_reduce) -> bool:
+    """The decode router equals route() when the batch has one sequence (its
+    query row is a one-row tile at the newest position, every block
+    eligible), and over a batch it keeps the router's invariants: rho = 1
+    gives the plain top-k prefix, top-k is a prefix of top-rho*k, sentinels
+    pad untriggered lists, quantile 0 triggers nothing."""
+    rng = _rng(41)
+    bs, Hkv, G, D = 4, 2, 3, 8
+    lens = [37, 29, 41, 16]
+    metas, Qs = [], []
+    for N in lens:
+        K = _bf16_round(rng.normal(size=(Hkv, N, D)))
+        s_, e_ = fixed_pages(N, bs)
+        metas.append([page_metadata(K[g], s_, e_) for g in range(Hkv)])
+        Qs.append(_bf16_round(rng.normal(size=(Hkv * G, D))))
+    for rule in ("envelope", "centroid"):
+        unit = [[group_reduce(head_scores(Qs[b][g * G:(g + 1) * G], metas[b][g], rule)) for g in range(Hkv)]
+                for b in range(len(lens))]
+        # one sequence: the same as route() with one one-row tile at position N - 1
+        N0 = lens[0]
+        one = route_decode(unit[:1], k=3, rho=2, quantile=0.5)
+        ref = route(Qs[0][None], metas[0], rule, q_pos0=N0 - 1, tile_rows=1, block_size=bs,
+                    n_blocks=len(fixed_pages(N0, bs)[0]), k=3, rho=2, quantile=0.5)
+        if not (np.array_equal(one.kv_idx, ref.kv_idx) and np.array_equal(one.kv_count, ref.kv_count)
+                and np.allclose(one.sigma, ref.sigma, rtol=0, atol=1e-12)):
+            return False
+        base = route_decode(unit, k=3, rho=1, quantile=0.5)
+        exp = route_decode(unit, k=3, rho=2, quantile=0.5)
+        for b in range(len(lens)):
+            for g in range(Hkv):
+                S = unit[b][g]
+                order = sorted(range(len(S)), key=lambda i: (-S[i], i))
+                if list(base.kv_idx[b, g]) != order[:3]:
+                    return False
+                row = list(exp.kv_idx[b, g])
+                if row[:3] != order[:3]:
+                    return False
+                if not exp.triggered[b] and row[3:] != [-1, -1, -1]:
+                    return False
+        if not np.allclose(exp.sigma_bar, exp.sigma.mean(axis=1), rtol=0, atol=0):
+            return False
+        if route_decode(unit, k=3, rho=2, quantile=0.0).triggered.any():
+            return False
+    return True
+
+
 def check_tile_attention_sdpa(tile_attention) -> bool:
     """Causal attention over the tile's selected blocks, against torch SDPA
     with an explicit boolean mask built row by row."""

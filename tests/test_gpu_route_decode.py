@@ -1,0 +1,136 @@
+"""GPU parity of the router applied to decode (sparse_attn_route_decode):
+every sequence of a decode batch is a one-row tile at its newest position
+("Onzekerheidsgestuurde Selectie voor Blok-schaarse Aandacht", "Methodologie"
+steps 2-5 with tiles of one row), checked against the float64 oracle with the
+router harness's rules (sets exact except certified near-ties, rank order,
+sigma / sigma_bar / tau within 1e-4, triggers exact away from tau), and the
+decode over the routed lists against oracle attention over the listed pages.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import datagen as DG
+import oracle as O
+
+pytestmark = pytest.mark.gpu
+
+SCALE = 1.0 / math.sqrt(128)
+
+
+@pytest.fixture(scope="module")
+def H():
+    import router_harness
+    return router_harness
+
+
+def _run_gpu(sa, lay, *, rule, ps, k, rho, quantile, tau):
+    B, Hkv, cap, D = lay.k.shape
+    Hq = lay.q.shape[1]
+    dev = lay.k.device
+    kv = sa.KvCache(lay.k, lay.v, lay.seq_len, page_size=ps, max_pages=-(-cap // ps))
+    meta = kv.meta_buffer()
+    sa.sparse_attn_build_meta(kv, rule, 0, meta)
+    W = rho * k
+    ws = sa.make_workspace(kv, Hq, B, W)
+    kv_idx = torch.full((B, Hkv, W), -7, dtype=torch.int32, device=dev)
+    kv_count = torch.full((B, Hkv), -7, dtype=torch.int32, device=dev)
+    sigma = torch.full((B, Hkv), float("nan"), dtype=torch.float32, device=dev)
+    sbar = torch.full((B,), float("nan"), dtype=torch.float32, device=dev)
+    trig = torch.full((B,), 7, dtype=torch.uint8, device=dev)
+    tau_out = torch.full((1,), float("nan"), dtype=torch.float32, device=dev)
+    tau_t = None if tau is None else torch.tensor([tau], dtype=torch.float32, device=dev)
+    sa.sparse_attn_route_decode(kv, meta, rule, lay.q, k, rho, quantile, tau_t, kv_idx, kv_count, sigma,
+                                sbar, trig, tau_out, ws)
+    out = torch.full((B, Hq, 128), float("nan"), dtype=torch.float32, device=dev)
+    lse = torch.full((B, Hq), float("nan"), dtype=torch.float32, device=dev)
+    sa.sparse_attn_decode(kv, lay.q, B, 0, 1, SCALE, kv_idx, kv_count, W, out, lse, ws)
+    torch.cuda.synchronize()
+    status = sa.sparse_attn_get_device_status(ws)
+    return dict(kv_idx=kv_idx.cpu().numpy(), kv_count=kv_count.cpu().numpy(),
+                sigma=sigma.cpu().numpy().astype(np.float64), sigma_bar=sbar.cpu().numpy().astype(np.float64),
+                triggered=trig.cpu().numpy().astype(bool), tau=float(tau_out.item()), status=status,
+                out=out.cpu(), lse=lse.cpu())
+
+
+def _oracle(H, lay, *, rule, ps, k, rho, quantile, tau):
+    B, Hkv = lay.k.shape[:2]
+    G = lay.q.shape[1] // Hkv
+    unit = []
+    for b in range(B):
+        N = int(lay.seq_len[b])
+        s, e = O.fixed_pages(N, ps)
+        row = []
+        for g in range(Hkv):
+            meta = O.page_metadata(H.to_np(lay.k[b, g, :N]), s, e)
+            row.append(O.group_reduce(O.head_scores(H.to_np(lay.q[b, g * G:(g + 1) * G]), meta, rule, fast=True)))
+        unit.append(row)
+    return O.route_decode(unit, k=k, rho=rho, quantile=quantile, tau=tau)
+
+
+def _check_attention(H, lay, g_res, ps):
+    B, Hkv = lay.k.shape[:2]
+    G = lay.q.shape[1] // Hkv
+    worst = 0.0
+    for b in range(B):
+        N = int(lay.seq_len[b])
+        s, e = O.fixed_pages(N, ps)
+        for g in range(Hkv):
+            n = int(g_res["kv_count"][b, g])
+            pages = np.sort(g_res["kv_idx"][b, g, :n].astype(np.int64))
+            toks = O.tokens_of(pages, s, e)
+            o, l = O.attend(H.to_np(lay.q[b, g * G:(g + 1) * G]), H.to_np(lay.k[b, g, :N]),
+                            H.to_np(lay.v[b, g, :N]), toks, SCALE)
+            err = float(np.abs(g_res["out"][b, g * G:(g + 1) * G].numpy() - o).max())
+            worst = max(worst, err)
+            assert err < 2e-3, f"({b},{g}) out err {err}"
+    return worst
+
+
+@pytest.mark.parametrize("rule", ["envelope", "centroid"])
+@pytest.mark.parametrize("ps,k,rho,quantile,tau", [
+    (16, 16, 2, 0.25, None),
+    (16, 16, 2, 0.5, 0.3),
+    (16, 12, 1, 0.25, None),
+    (64, 4, 3, 0.75, None),
+])
+def test_route_decode_parity(cuda_dev, H, rule, ps, k, rho, quantile, tau):
+    import block_sparse_kv_page_b200 as sa
+    rng = np.random.default_rng(ps * 31 + k)
+    B = 24
+    lens = [int(x) for x in rng.integers(200, 4000, size=B)]
+    lens[3] = 50  # fewer pages than k at 16-token pages: sigma = 1, every page listed
+    lay = DG.make_decode_layer(B=B, Hq=32, Hkv=4, seq_lens=lens, seed=801 + k, device=cuda_dev,
+                               cap=4000, key_scale="channel")
+    g_res = _run_gpu(sa, lay, rule=rule, ps=ps, k=k, rho=rho, quantile=quantile, tau=tau)
+    ref = _oracle(H, lay, rule=rule, ps=ps, k=k, rho=rho, quantile=quantile, tau=tau)
+    stats = H.compare(g_res, ref, k=k, rho=rho)
+    assert g_res["triggered"].any() or quantile < 0.3 or tau is not None
+    _check_attention(H, lay, g_res, ps)
+    print(f"\n{rule} ps={ps} k={k} rho={rho}: {stats}, triggered {int(g_res['triggered'].sum())}/{B}")
+
+
+def test_route_decode_rejects_bad_arguments(cuda_dev):
+    import block_sparse_kv_page_b200 as sa
+    lay = DG.make_decode_layer(B=2, Hq=32, Hkv=4, seq_lens=[300, 200], seed=811, device=cuda_dev)
+    kv = sa.KvCache(lay.k, lay.v, lay.seq_len, page_size=16, max_pages=19)
+    meta = kv.meta_buffer()
+    ws = sa.make_workspace(kv, 32, 2, 32)
+    dev = lay.k.device
+    idx = torch.empty((2, 4, 32), dtype=torch.int32, device=dev)
+    cnt = torch.empty((2, 4), dtype=torch.int32, device=dev)
+    sig = torch.empty((2, 4), dtype=torch.float32, device=dev)
+    sb = torch.empty((2,), dtype=torch.float32, device=dev)
+    tr = torch.empty((2,), dtype=torch.uint8, device=dev)
+    with pytest.raises(sa.SparseAttnError) as e:   # quantile outside [0, 1]
+        sa.sparse_attn_route_decode(kv, meta, "envelope", lay.q, 16, 2, 1.5, None, idx, cnt, sig, sb, tr, None, ws)
+    assert e.value.status == sa.SA_ERR_INVALID
+    chunks = sa.KvCache(lay.k, lay.v, lay.seq_len, page_size=0, max_pages=19,
+                        chunk_off=torch.zeros((2, 20), dtype=torch.int32, device=dev),
+                        n_chunks=torch.ones((2,), dtype=torch.int32, device=dev))
+    with pytest.raises(sa.SparseAttnError) as e:   # variable chunks are not routed
+        sa.sparse_attn_route_decode(chunks, meta, "envelope", lay.q, 16, 2, 0.5, None, idx, cnt, sig, sb, tr,
+                                    None, ws)
+    assert e.value.status == sa.SA_ERR_UNSUPPORTED

@@ -88,6 +88,11 @@ def test_router_invariants():
     assert P.check_router_invariants(O.route, O.page_metadata, O.fixed_pages)
 
 
+def test_route_decode():
+    assert P.check_route_decode(O.route_decode, O.route, O.page_metadata, O.fixed_pages, O.head_scores,
+                                O.group_reduce)
+
+
 def test_tile_attention_sdpa():
     assert P.check_tile_attention_sdpa(O.tile_attention)
 
@@ -223,6 +228,21 @@ def _route_le(Q, metas, rule, **kw):
     return r
 
 
+def _route_decode_page_order(unit_scores, **kw):   # lists in page order instead of rank order
+    r = O.route_decode(unit_scores, **kw)
+    for b in range(r.kv_idx.shape[0]):
+        for g in range(r.kv_idx.shape[1]):
+            n = int(r.kv_count[b, g])
+            r.kv_idx[b, g, :n] = np.sort(r.kv_idx[b, g, :n])
+    return r
+
+
+def _route_decode_sigma_max(unit_scores, **kw):   # sigma_bar as the max over KV heads
+    r = O.route_decode(unit_scores, **kw)
+    r.sigma_bar = r.sigma.max(axis=1)
+    return r
+
+
 def _tile_attn_noncausal(Q, K, V, kv_idx, *, q_pos0, tile_rows, block_size, n_tokens, scale):
     return O.tile_attention(Q, K, V, kv_idx, q_pos0=q_pos0 + 10 ** 9, tile_rows=tile_rows,
                             block_size=block_size, n_tokens=n_tokens, scale=scale)
@@ -265,6 +285,10 @@ MISTAKES = [
         _env_fast_swapped, O.tile_block_scores, O.envelope_scores, O.centroid_scores,
         O.page_metadata, O.fixed_pages)),
     ("tile attention not causal", lambda: P.check_tile_attention_sdpa(_tile_attn_noncausal)),
+    ("decode router lists in page order", lambda: P.check_route_decode(
+        _route_decode_page_order, O.route, O.page_metadata, O.fixed_pages, O.head_scores, O.group_reduce)),
+    ("decode router sigma_bar as max", lambda: P.check_route_decode(
+        _route_decode_sigma_max, O.route, O.page_metadata, O.fixed_pages, O.head_scores, O.group_reduce)),
 ]
 
 
