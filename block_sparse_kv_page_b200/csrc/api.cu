@@ -229,7 +229,7 @@ sa_status tile_attention(const sa_kv_desc* kv, const void* q, int n_q_heads, int
   }
   const unsigned long long kv_rows = (unsigned long long)kv->n_kv_heads * kv->cap_tokens;
   if (kv_rows > 0x7fffffffULL) return SA_ERR_UNSUPPORTED;
-  TileAttnArgs a;
+  TileAttnArgs a{};  // every field zero unless set below
   if (!encode_tmap_2d(&a.tmap_k, kv->k, kv_rows, kHeadDim * 2, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, 64) ||
       !encode_tmap_2d(&a.tmap_v, kv->v, kv_rows, kHeadDim * 2, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, 64))
     return SA_ERR_CUDA;
@@ -441,7 +441,7 @@ static sa_status select_impl(const sa_kv_desc* kv, const void* meta, sa_score_ru
   if (per_head && (long long)kv->batch * n_q_heads > kMaxUnits) return SA_ERR_UNSUPPORTED;
   const size_t need = kScratch + select_scratch(kv, per_head, n_q_heads);
   if ((s = check_ws(ws, ws_bytes, need)) != SA_OK) return s;
-  SelectArgs a;
+  SelectArgs a{};  // every field zero unless set below
   if (!fill_select(&a, kv, meta, rule, q, n_q_heads, G, budget, max_sel, sel_idx, sel_count,
                    scores_out, ws))
     return SA_ERR_CUDA;
@@ -486,7 +486,7 @@ static sa_status decode_rows(const sa_kv_desc* kv, const void* q, int32_t n_q_he
   sa_status s;
   if ((s = check_ws(ws, ws_bytes, need)) != SA_OK) return s;
 
-  DecodeArgs a;
+  DecodeArgs a{};  // every field zero unless set below
   char* w = reinterpret_cast<char*>(ws);
   if (!fill_decode(&a, kv, q, n_q_heads, G, scale, idx, count, max_sel, out, lse,
                    reinterpret_cast<float*>(w + kScratch), reinterpret_cast<uint32_t*>(w + 256),
@@ -568,7 +568,7 @@ static sa_status decode_step(const sa_kv_desc* kv, void* meta, sa_score_rule rul
   if (step_smem_bytes(kv->max_pages, max_sel, kv->page_size == 0) > 227 * 1024)
     return SA_ERR_UNSUPPORTED;
 
-  StepArgs a;
+  StepArgs a{};  // every field zero unless set below
   char* w = reinterpret_cast<char*>(ws);
   if (!fill_select(&a.sel, kv, meta, rule, q, n_q_heads, G, budget, max_sel, sel_idx, sel_count,
                    nullptr, ws) ||
@@ -645,7 +645,7 @@ sa_status sparse_attn_route(const sa_kv_desc* kv, const void* meta, sa_score_rul
   const size_t need = kScratch + route_ws_bytes((int)T, kv->n_kv_heads, kv->max_pages, (int)W);
   if ((s = check_ws(ws, ws_bytes, need)) != SA_OK) return s;
 
-  RouteArgs a;
+  RouteArgs a{};  // every field zero unless set below
   const bool env = rule == SA_SCORE_ENVELOPE;
   if (!encode_tmap_2d(&a.tmap_meta, meta, meta_rows, kMetaBytes,
                       env ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32,
@@ -680,6 +680,8 @@ sa_status sparse_attn_route(const sa_kv_desc* kv, const void* meta, sa_score_rul
   const size_t tg = (size_t)units;
   const size_t keys_bytes = align256(tg * kv->max_pages * 4);
   a.ws_keys = reinterpret_cast<uint32_t*>(scratch);
+  a.dec_scores = nullptr;  // query tiles: the keys above, not decode group scores
+  a.dec_stride = 0;
   a.ws_list = reinterpret_cast<int32_t*>(scratch + keys_bytes);
   a.ws_sigma = reinterpret_cast<double*>(scratch + keys_bytes + align256(tg * W * 4));
   a.ws_elig = reinterpret_cast<int32_t*>(scratch + keys_bytes + align256(tg * W * 4) + align256(tg * 8));
@@ -720,7 +722,7 @@ sa_status sparse_attn_route_decode(const sa_kv_desc* kv, const void* meta, sa_sc
   const size_t need = kScratch + sel_bytes + route_decode_ws_bytes(units, (int)W);
   if ((s = check_ws(ws, ws_bytes, need)) != SA_OK) return s;
   if (route_decode_smem_bytes(kv->max_pages, (int)W, k, kv->batch) > 227 * 1024) return SA_ERR_UNSUPPORTED;
-  SelectArgs sa_;
+  SelectArgs sa_{};  // every field zero unless set below
   if (!fill_select(&sa_, kv, meta, rule, q, n_q_heads, G, &dummy, (int)W, kv_idx, kv_count, nullptr, ws))
     return SA_ERR_CUDA;
   sa_.score_only = 1;
@@ -728,8 +730,7 @@ sa_status sparse_attn_route_decode(const sa_kv_desc* kv, const void* meta, sa_sc
   if ((s = launched(launch_select(sa_, (cudaStream_t)stream))) != SA_OK) return s;
 
   // the router's selection, sigma, quantile, triggers and lists over those scores
-  RouteArgs a;
-  memset(&a, 0, sizeof(a));
+  RouteArgs a{};  // every field zero unless set below
   a.kv = view(kv);
   a.rule = (int)rule;
   a.q = q;
@@ -870,7 +871,7 @@ extern "C" sa_status sparse_attn_decode_static(const sa_kv_desc* kv, const void*
 
   unsigned char* scratch = nullptr;
   if ((s = static_scratch(&scratch)) != SA_OK) return s;
-  DecodeArgs a;
+  DecodeArgs a{};  // every field zero unless set below
   if (!encode_tmap_2d(&a.tmap_k, kv->k, kv_rows, kHeadDim * 2, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, 16) ||
       !encode_tmap_2d(&a.tmap_v, kv->v, kv_rows, kHeadDim * 2, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, 16))
     return SA_ERR_CUDA;

@@ -86,7 +86,7 @@ __global__ void __launch_bounds__(kMetaWarps * 32) build_meta_kernel(MetaParams 
 
 cudaError_t launch_build_meta(const KvView& kv, int rule, int first_token, void* meta,
                               int* status, cudaStream_t st) {
-  MetaParams p;
+  MetaParams p{};
   p.kv = kv;
   p.rule = rule;
   p.first_token = first_token;
