@@ -6,28 +6,32 @@
 // entries are skipped.  Chunked-prefill rows attend causally: row r at
 // position q_pos0 + r sees only keys at positions <= its own.
 //
-// CTA = (tile, KV head, 128 query vectors), one CTA per SM; a query vector is
-// one (row, query head) pair of the tile and owns one lane of tensor memory.
+// CTA = (tile, KV head, 256 query vectors) = two Q tiles of 128 vectors that
+// share every K/V block, one CTA per SM; a query vector is one (row, query
+// head) pair of the tile and owns one TMEM lane in its Q tile's columns.
 // Warp-specialised, all waits bounded:
 //   warp 8 (one thread)  streams each kept block (64 keys) of K and V by TMA
 //                        into a kStages ring (four 64-row x 128 B boxes);
-//   warp 9 (one thread)  issues, per block i, S_i = Q K_i^T (M = 128 vectors,
-//                        N = 64 keys, K = 128 dims; K-major operands) into one
-//                        of two S accumulators, and O += [P_hi | P_lo] .
-//                        [V_i ; V_i] (A from tensor memory; N = 128 dims,
-//                        K = 2 x 64 keys; V read MN-major) into the O
-//                        accumulator; QK of the next
-//                        block is issued before PV of this one, so the
-//                        softmax overlaps the tensor cores;
-//   warps 0-7            two per TMEM lane quarter (query vector): mask
-//                        (causal, cache end), online softmax in the log2
-//                        domain against a reference max, P split into a bf16
-//                        hi + lo pair (error ~2^-17) stored to tensor memory
-//                        as the next MMA's A operand; O stays in tensor
-//                        memory and is rescaled in place only when a row's
-//                        max grows by more than 2^8.
-// Accumulation order per vector is the block order of the list, so results
-// do not depend on scheduling.
+//   warp 9 (one thread)  issues, for each Q tile t and block i,
+//                        S = Q_t K_i^T (M = 128 vectors, N = 64 keys, K = 128
+//                        dims; K-major operands) into one of the tile's two
+//                        S/P buffers, and O_t += [P_hi | P_lo] . [V_i ; V_i]
+//                        (A = P read from tensor memory, N = 128 dims,
+//                        K = 2 x 64 keys; V read MN-major); it polls both
+//                        tiles' queues, so one tile's softmax and handoffs
+//                        overlap the other tile's MMAs;
+//   warps 0-3 / 4-7      the softmax of tile 0 / 1: thread = query vector
+//                        (TMEM lane 32 (warp % 4) + lane), its whole row of
+//                        64 keys: masks (causal, cache end) only on the
+//                        diagonal and cache-end blocks, online softmax in the
+//                        log2 domain against a reference max, P split into a
+//                        bf16 hi + lo pair (error ~2^-17) stored over S in
+//                        tensor memory as the PV MMA's A operand.
+// O stays in tensor memory; it is rescaled in place only when a row's max
+// grows past the reference by more than 2^8.  The MMAs of one issuing thread
+// run in issue order, so the S/P buffer of block i + 2 is written only after
+// the PV of block i has read it.  Accumulation order per vector is the block
+// order of the list, so results do not depend on scheduling.
 #include "common.cuh"
 #include "internal.h"
 #include "tcgen05.cuh"
@@ -36,7 +40,8 @@ namespace sa {
 namespace {
 
 constexpr int kBlk = 64;                       // keys per block
-constexpr int kSmWarps = 8;                    // softmax warps: two per TMEM lane quarter
+constexpr int kTiles = 2;                      // Q tiles of 128 vectors per CTA
+constexpr int kSmWarps = 4 * kTiles;           // softmax: one warp per TMEM lane quarter and tile
 constexpr int kThreadsTc = 32 * (kSmWarps + 2);
 constexpr int kProducerWarp = kSmWarps;
 constexpr int kMmaWarp = kSmWarps + 1;
@@ -46,21 +51,20 @@ constexpr int kMmaWarp = kSmWarps + 1;
 constexpr int kStages = SA_TA_STAGES;
 constexpr int kBox = kBlk * 128;               // 64 rows x 128 B
 constexpr int kStage = 4 * kBox;               // K lo | K hi | V lo | V hi = 32 KiB
-constexpr int kQBytes = 2 * 128 * 128;         // 128 vectors x 128 dims bf16, two K chunks
+constexpr int kQTile = 2 * 128 * 128;          // 128 vectors x 128 dims bf16, two K chunks
 constexpr int kOffQ = 0;
-constexpr int kOffRing = kOffQ + kQBytes;
+constexpr int kOffRing = kOffQ + kTiles * kQTile;
 constexpr int kOffBars = kOffRing + kStages * kStage;
-// kv full/empty, s full/empty, p full, o full (PV of even / odd blocks), drain
-constexpr int kNumBars = 2 * kStages + 2 * 2 + 2 + 2 + 1;
-constexpr int kOffRed = kOffBars + kNumBars * 8 + 8;        // softmax row sums, 2 halves x 128 rows
-constexpr int kOffList = kOffRed + 2 * 128 * 4;
-constexpr uint32_t kColS = 0;                  // S accumulators: columns [0, 128)
-constexpr uint32_t kColO = 128;                // O accumulator: columns [128, 256)
-constexpr uint32_t kColP = 256;                // P_hi | P_lo (bf16 pairs), two buffers: [256, 384)
+// kv full/empty per stage; per tile and buffer: S full, P full, PV done; drain
+constexpr int kNumBars = 2 * kStages + 3 * kTiles * 2 + 1;
+constexpr int kOffList = kOffBars + kNumBars * 8 + 8;
+// tensor memory: tile t's two S/P buffers at columns [128 t, 128 t + 128) (64
+// fp32 columns each; P's bf16 hi | lo pairs overwrite them), its O
+// accumulator at [256 + 128 t, 256 + 128 t + 128)
+constexpr uint32_t kColSP = 0;
+constexpr uint32_t kColO = 256;
 static_assert(1024 + kOffList > 114 * 1024, "one CTA per SM: it allocates all 512 TMEM columns");
 
-// MN-major view of V (keys x dims, dims contiguous): 8-key atoms 1 KiB apart,
-// the two 64-dim boxes 8 KiB apart.
 // 2^x by the hardware approximation (relative error about 2^-22; 2^-inf = +0).
 SA_DEV float fast_exp2(float x) {
   float y;
@@ -68,6 +72,8 @@ SA_DEV float fast_exp2(float x) {
   return y;
 }
 
+// MN-major view of V (keys x dims, dims contiguous): 8-key atoms 1 KiB apart,
+// the two 64-dim boxes 8 KiB apart.
 SA_DEV uint64_t v_desc(const unsigned char* v) {
   const uint64_t d = tc::smem_desc_sw128(v);
   return (d & ~(0x3FFFull << 16)) | ((uint64_t)(kBox >> 4) << 16);
@@ -83,18 +89,44 @@ __global__ void __launch_bounds__(kThreadsTc, 1) tile_attn_tc_kernel(const __gri
   unsigned char* ring = base + kOffRing;
   uint64_t* kv_full = reinterpret_cast<uint64_t*>(base + kOffBars);
   uint64_t* kv_empty = kv_full + kStages;
-  uint64_t* s_full = kv_empty + kStages;
-  uint64_t* s_empty = s_full + 2;
-  uint64_t* p_full = s_empty + 2;
-  uint64_t* o_full = p_full + 2;
-  uint64_t* drain = o_full + 2;
+  uint64_t* s_full = kv_empty + kStages;   // [tile][buffer]
+  uint64_t* p_full = s_full + 2 * kTiles;  // [tile][buffer]
+  uint64_t* o_full = p_full + 2 * kTiles;  // [tile][block parity]: PV of the block done
+  uint64_t* drain = o_full + 2 * kTiles;
   int* blist = reinterpret_cast<int*>(base + kOffList);
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int Hkv = a.kv.Hkv, G = a.G;
   const int nmc = a.n_mchunks;
   const int mc = blockIdx.x % nmc;
-  const int tg = blockIdx.x / nmc;
+  // (tile, KV head) of this CTA.  With few enough pairs the CTAs take them
+  // longest list first (the hardware starts CTAs in index order, so the long
+  // lists of triggered tiles start in the first wave instead of ending the
+  // launch): every CTA ranks all pairs by (count desc, index asc) and takes
+  // the pair of rank blockIdx.x / nmc.
+  __shared__ int s_cnt[kThreadsTc];
+  __shared__ int s_pair;
+  const int n_pairs = a.n_tiles * Hkv;
+  int tg = blockIdx.x / nmc;
+  if (n_pairs <= kThreadsTc) {
+    int mine = 0;
+    if (tid < n_pairs) {
+      mine = __ldg(a.count + tid);
+      if (mine < 0 || mine > a.max_sel) mine = 0;
+      s_cnt[tid] = mine;
+    }
+    __syncthreads();
+    if (tid < n_pairs) {
+      int rank = 0;
+      for (int u = 0; u < n_pairs; ++u) {
+        const int c = s_cnt[u];
+        rank += (c > mine || (c == mine && u < tid)) ? 1 : 0;
+      }
+      if (rank == tg) s_pair = tid;
+    }
+    __syncthreads();
+    tg = s_pair;
+  }
   const int t = tg / Hkv, g = tg % Hkv;
   const int N = a.kv.seq_len[0];
   const int P = (N + kBlk - 1) / kBlk;
@@ -108,11 +140,10 @@ __global__ void __launch_bounds__(kThreadsTc, 1) tile_attn_tc_kernel(const __gri
       mbar_init(kv_full + s, 1);
       mbar_init(kv_empty + s, 1);
     }
-    for (int b = 0; b < 2; ++b) {
-      mbar_init(s_full + b, 1);
-      mbar_init(s_empty + b, kSmWarps);
-      mbar_init(p_full + b, kSmWarps);
-      mbar_init(o_full + b, 1);
+    for (int x = 0; x < 2 * kTiles; ++x) {
+      mbar_init(s_full + x, 1);
+      mbar_init(p_full + x, 4);  // the tile's four softmax warps
+      mbar_init(o_full + x, 1);
     }
     mbar_init(drain, 1);
     fence_barrier_init();
@@ -148,11 +179,11 @@ __global__ void __launch_bounds__(kThreadsTc, 1) tile_attn_tc_kernel(const __gri
   }
   const int nb = (int)nb_u;
 
-  // ---- the CTA's 128 query vectors (K-major, 128B-swizzled, rows past V zero);
-  // 8 loads in flight per thread
+  // ---- the CTA's 256 query vectors: tile vi / 128, row vi % 128 of its
+  // K-major, 128B-swizzled Q (rows past V zero); 8 loads in flight per thread
   const __nv_bfloat16* Q = reinterpret_cast<const __nv_bfloat16*>(a.q);
-  const int v0 = mc * 128;
-  constexpr int kQPieces = 128 * 16;
+  const int v0 = mc * 128 * kTiles;
+  constexpr int kQPieces = 128 * kTiles * 16;
 #pragma unroll 1
   for (int b0 = 0; b0 < kQPieces; b0 += 8 * kThreadsTc) {
     uint4 rw[8];
@@ -169,7 +200,8 @@ __global__ void __launch_bounds__(kThreadsTc, 1) tile_attn_tc_kernel(const __gri
       const int x = b0 + i * kThreadsTc + tid;
       if (x >= kQPieces) continue;
       const int vi = x >> 4, d8 = x & 15;
-      *reinterpret_cast<uint4*>(qs + (d8 >> 3) * (128 * 128) + swz128(vi, d8 & 7)) = rw[i];
+      *reinterpret_cast<uint4*>(qs + (vi >> 7) * kQTile + (d8 >> 3) * (128 * 128) + swz128(vi & 127, d8 & 7)) =
+          rw[i];
     }
   }
   fence_proxy_async();  // generic writes (queries, list) before the async proxy reads them
@@ -178,20 +210,9 @@ __global__ void __launch_bounds__(kThreadsTc, 1) tile_attn_tc_kernel(const __gri
   tc::fence_after_sync();
   const uint32_t tmem = s_tmem;
   int fail = 0;
-  // softmax-warp state, used after the final barrier (other warps: unused)
-  const int quarter = warp & 3, h = (warp >> 2) & 1;
-  const int r = 32 * quarter + lane;
-  const int v = v0 + r;
-  const bool vok = v < V;
-  const int qpos = vok ? a.q_pos0 + row0 + v / G : -1;
-  float* red = reinterpret_cast<float*>(base + kOffRed);  // [2 halves][128 rows] row sums
-  float mref = ninf, lh = 0.f;  // reference max (log2 units) and row sum against it
-  float o[64];
-#pragma unroll
-  for (int d = 0; d < 64; ++d) o[d] = 0.f;
 
   if (warp == kProducerWarp) {
-    // ---- TMA producer: block i -> stage i % kStages
+    // ---- TMA producer: block i -> stage i % kStages (freed once both tiles' PV read it)
     if (lane == 0) {
       const long long rowbase = (long long)g * a.kv.cap;  // B == 1: unit = KV head
       int issued = 0;
@@ -215,49 +236,56 @@ __global__ void __launch_bounds__(kThreadsTc, 1) tile_attn_tc_kernel(const __gri
         mbar_wait(kv_full + (i % kStages), (i / kStages) & 1u, nullptr);
     }
   } else if (warp == kMmaWarp) {
-    // ---- MMA issuer: qk(0), then per block i: qk(i + 1), pv(i)
+    // ---- MMA issuer.  Per tile: QK of block i needs its K/V stage and a free
+    // S/P buffer (the PV of block i - 2 issued before it); PV of block i needs
+    // P_i.  Both tiles' queues are polled without blocking and whatever is
+    // ready goes first; the K/V stage is released after the second of the two
+    // PVs that read it.
     if (lane == 0) {
       const uint32_t idesc_s = tc::idesc_f32acc(tc::kFmtBF16, 128, kBlk);
       const uint32_t idesc_o = tc::idesc_f32acc(tc::kFmtBF16, 128, kHeadDim) | (1u << 16);  // V MN-major
-      // Both queues are polled without blocking: QK of block i + 1 needs its
-      // K/V stage and a free S buffer, PV of block i needs P_i; whichever is
-      // ready goes first, so a late K/V stage never holds back a PV whose P is
-      // written (and the stage it frees).  QK runs at most one block ahead.
-      auto qk = [&](int i) {
+      auto qk = [&](int tt, int i) {
         const int s = i % kStages, b = i & 1;
         const unsigned char* kb = ring + s * kStage;
+        const unsigned char* qt = qs + tt * kQTile;
 #pragma unroll
         for (int c = 0; c < 2; ++c)
 #pragma unroll
           for (int k = 0; k < 4; ++k)
-            tc::mma_bf16_ss(tmem + kColS + 64u * b, tc::smem_desc_sw128(qs + c * (128 * 128) + 32 * k),
+            tc::mma_bf16_ss(tmem + kColSP + 128u * tt + 64u * b, tc::smem_desc_sw128(qt + c * (128 * 128) + 32 * k),
                             tc::smem_desc_sw128(kb + c * kBox + 32 * k), idesc_s, (c | k) != 0);
-        tc::commit(s_full + b);
+        tc::commit(s_full + 2 * tt + b);
       };
-      auto pv = [&](int i) {
+      auto pv = [&](int tt, int i) {
         const int s = i % kStages, b = i & 1;
         const unsigned char* vb = ring + s * kStage + 2 * kBox;
 #pragma unroll
         for (int j = 0; j < 8; ++j)  // K = [P_hi keys 0-63 | P_lo keys 0-63], 16 per step
-          tc::mma_bf16_ts(tmem + kColO, tmem + kColP + 64u * b + 8u * j, v_desc(vb + 16 * 128 * (j & 3)),
-                          idesc_o, i > 0 || j != 0);
-        tc::commit(o_full + b);
-        tc::commit(kv_empty + s);
+          tc::mma_bf16_ts(tmem + kColO + 128u * tt, tmem + kColSP + 128u * tt + 64u * b + 8u * j,
+                          v_desc(vb + 16 * 128 * (j & 3)), idesc_o, i > 0 || j != 0);
+        tc::commit(o_full + 2 * tt + b);
       };
-      int nq = 0, npv = 0;
+      int nq[kTiles] = {0, 0}, npv[kTiles] = {0, 0};
       uint32_t idle = 0;
-      while (npv < nb) {
+      while (npv[0] < nb || npv[1] < nb) {
         bool progress = false;
-        if (nq < nb && nq <= npv + 1 && mbar_test(kv_full + nq % kStages, (nq / kStages) & 1u) &&
-            (nq < 2 || mbar_test(s_empty + (nq & 1), ((nq >> 1) - 1) & 1u))) {
-          tc::fence_after_sync();
-          qk(nq++);
-          progress = true;
-        }
-        if (npv < nq && mbar_test(p_full + (npv & 1), (npv >> 1) & 1u)) {
-          tc::fence_after_sync();
-          pv(npv++);
-          progress = true;
+#pragma unroll
+        for (int tt = 0; tt < kTiles; ++tt) {
+          const int q = nq[tt];
+          if (q < nb && q < npv[tt] + 2 && mbar_test(kv_full + q % kStages, (q / kStages) & 1u)) {
+            tc::fence_after_sync();
+            qk(tt, q);
+            nq[tt] = q + 1;
+            progress = true;
+          }
+          const int p = npv[tt];
+          if (p < nq[tt] && mbar_test(p_full + 2 * tt + (p & 1), (p >> 1) & 1u)) {
+            tc::fence_after_sync();
+            pv(tt, p);
+            if (npv[tt ^ 1] > p) tc::commit(kv_empty + p % kStages);  // the other tile's PV of p is issued
+            npv[tt] = p + 1;
+            progress = true;
+          }
         }
         if (progress) {
           idle = 0;
@@ -272,77 +300,70 @@ __global__ void __launch_bounds__(kThreadsTc, 1) tile_attn_tc_kernel(const __gri
       mbar_wait(drain, 0, nullptr);
     }
   } else {
-    // ---- softmax: TMEM lane r = 32 (warp % 4) + lane is query vector v0 + r;
-    // half h = warp / 4 exponentiates keys [32 h, 32 h + 32) of S and owns dims
-    // [64 h, 64 h + 64) of O.  Both halves read the whole S row, so they hold the
-    // same maxima without exchanging anything; their row sums are added after
-    // the CTA's final barrier.  O accumulates in tensor memory over the blocks,
-    // against a reference max mref that may lag the row's running max: P =
-    // 2^(s - mref) stays below 2^8, and O and the row sum are rescaled in place
-    // only when a row's max passes mref by more than 8 (log2 units), which with
-    // bounded scores happens in the first blocks only.
+    // ---- softmax of tile tt: TMEM lane r = 32 (warp % 4) + lane is query
+    // vector v0 + 128 tt + r; the thread owns that vector's whole row.
+    const int tt = warp >> 2, quarter = warp & 3;
+    const int r = 32 * quarter + lane;
+    const int v = v0 + 128 * tt + r;
+    const bool vok = v < V;
+    const int qpos = vok ? a.q_pos0 + row0 + v / G : -1;
     const uint32_t lane_off = (uint32_t)(32 * quarter) << 16;
-    const uint32_t to = tmem + lane_off + kColO + 64u * h;
-    int o_seen = 0;  // PV results waited for: blocks [0, o_seen)
-    auto wait_pv = [&](int j) -> bool {  // PV of block j complete (phases in order)
-      const bool ok = mbar_wait(o_full + (j & 1), (j >> 1) & 1u, a.status);
+    const uint32_t sp_base = tmem + lane_off + kColSP + 128u * tt;
+    const uint32_t to = tmem + lane_off + kColO + 128u * tt;
+    uint64_t* s_full_t = s_full + 2 * tt;
+    uint64_t* p_full_t = p_full + 2 * tt;
+    uint64_t* o_full_t = o_full + 2 * tt;
+    // PV of block j complete.  A tile's PV barrier for one block parity never
+    // runs two phases ahead of a wait here: PV of block j + 2 needs P_{j+2},
+    // which this thread writes later (or, after the loop, does not exist).
+    auto wait_pv = [&](int j) -> bool {
+      const bool ok = mbar_wait(o_full_t + (j & 1), (j >> 1) & 1u, a.status);
       return __all_sync(0xffffffffu, ok);
     };
-    // S of block i in r0..r3 (own half: r0, r1; other half: r2, r3); the loads of
-    // block i + 1 are issued before waiting for PV of block i - 1, so their
-    // latency overlaps that wait
-    uint32_t r0[16], r1[16], r2[16], r3[16];
-    auto load_s = [&](int i) -> bool {
+    float mref = ninf, lh = 0.f;  // reference max (log2 units) and the row sum against it
+    const float sl2 = a.scale_log2;
+    for (int i = 0; i < nb; ++i) {
       const int b = i & 1;
-      const bool ok = mbar_wait(s_full + b, (i >> 1) & 1u, a.status);
-      if (!__all_sync(0xffffffffu, ok)) return false;
+      const bool ok = mbar_wait(s_full_t + b, (i >> 1) & 1u, a.status);
+      if (!__all_sync(0xffffffffu, ok)) {
+        fail = 1;
+        break;
+      }
       tc::fence_after_sync();
-      const uint32_t ts = tmem + lane_off + kColS + 64u * b;
-      tc::ld_32x32b_x16(ts + 32u * h, r0);
-      tc::ld_32x32b_x16(ts + 32u * h + 16, r1);
-      tc::ld_32x32b_x16(ts + 32u * (h ^ 1), r2);
-      tc::ld_32x32b_x16(ts + 32u * (h ^ 1) + 16, r3);
-      return true;
-    };
-    if (nb > 0 && !load_s(0)) fail = 1;
-    for (int i = 0; i < nb && !fail; ++i) {
-      const int b = i & 1;
+      const uint32_t ts = sp_base + 64u * b;
+      uint32_t r0[16], r1[16], r2[16], r3[16];  // keys 0-15, 16-31, 32-47, 48-63
+      tc::ld_32x32b_x16(ts, r0);
+      tc::ld_32x32b_x16(ts + 16, r1);
+      tc::ld_32x32b_x16(ts + 32, r2);
+      tc::ld_32x32b_x16(ts + 48, r3);
       tc::wait_ld();
       tc::reg_fence(r0);
       tc::reg_fence(r1);
       tc::reg_fence(r2);
       tc::reg_fence(r3);
-      tc::fence_before_sync();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(s_empty + b);  // S_i read: the buffer may take S_{i+2}
       const int kb0 = blist[i] * kBlk;
-      // scores in registers: this half's 32 keys in sv, the row max over all 64.
       // Blocks fully visible to every row of the warp (all but the diagonal and
       // the cache end) skip the masks, and with a positive scale the max is
-      // taken on raw scores (scaling commutes with max).
-      const float sl2 = a.scale_log2;
+      // taken on raw scores (scaling commutes with max); four max chains.
       const bool fast = sl2 > 0.f && __all_sync(0xffffffffu, kb0 + kBlk - 1 <= qpos && kb0 + kBlk <= N);
-      // (four independent max chains: the reduction is latency-bound)
-      float sv[32], mq[4] = {ninf, ninf, ninf, ninf}, mul;
+      float sv[64], mq[4] = {ninf, ninf, ninf, ninf}, mul;
+#pragma unroll
+      for (int x = 0; x < 16; ++x) {
+        sv[x] = __uint_as_float(r0[x]);
+        sv[16 + x] = __uint_as_float(r1[x]);
+        sv[32 + x] = __uint_as_float(r2[x]);
+        sv[48 + x] = __uint_as_float(r3[x]);
+      }
       if (fast) {
 #pragma unroll
-        for (int x = 0; x < 16; ++x) {
-          sv[x] = __uint_as_float(r0[x]);
-          sv[16 + x] = __uint_as_float(r1[x]);
-          mq[x & 3] = fmaxf(mq[x & 3], fmaxf(fmaxf(sv[x], sv[16 + x]),
-                                             fmaxf(__uint_as_float(r2[x]), __uint_as_float(r3[x]))));
-        }
+        for (int x = 0; x < 64; ++x) mq[x & 3] = fmaxf(mq[x & 3], sv[x]);
         mul = sl2;
       } else {
-        const int kv0 = kb0 + 32 * h, kw0 = kb0 + 32 * (h ^ 1);
 #pragma unroll
-        for (int x = 0; x < 16; ++x) {
-          const int k0 = kv0 + x, k1 = k0 + 16, w0 = kw0 + x, w1 = w0 + 16;
-          sv[x] = (k0 <= qpos && k0 < N) ? __uint_as_float(r0[x]) * sl2 : ninf;
-          sv[16 + x] = (k1 <= qpos && k1 < N) ? __uint_as_float(r1[x]) * sl2 : ninf;
-          const float u0 = (w0 <= qpos && w0 < N) ? __uint_as_float(r2[x]) * sl2 : ninf;
-          const float u1 = (w1 <= qpos && w1 < N) ? __uint_as_float(r3[x]) * sl2 : ninf;
-          mq[x & 3] = fmaxf(mq[x & 3], fmaxf(fmaxf(sv[x], sv[16 + x]), fmaxf(u0, u1)));
+        for (int x = 0; x < 64; ++x) {
+          const int key = kb0 + x;
+          sv[x] = (key <= qpos && key < N) ? sv[x] * sl2 : ninf;
+          mq[x & 3] = fmaxf(mq[x & 3], sv[x]);
         }
         mul = 1.f;
       }
@@ -355,17 +376,14 @@ __global__ void __launch_bounds__(kThreadsTc, 1) tile_attn_tc_kernel(const __gri
       if (upd) mref = mn;
       lh *= alpha;
       if (i > 0 && __any_sync(0xffffffffu, upd)) {
-        // O holds blocks [0, i): once the last of them is in, scale this half in place
-        if (o_seen < i) {
-          if (!wait_pv(i - 1)) {
-            fail = 1;
-            break;
-          }
-          o_seen = i;
+        // O holds blocks [0, i): once the last of them is in, scale this row in place
+        if (!wait_pv(i - 1)) {
+          fail = 1;
+          break;
         }
         tc::fence_after_sync();
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
+        for (int c = 0; c < 8; ++c) {
           uint32_t q[16];
           tc::ld_32x32b_x16(to + 16 * c, q);
           tc::wait_ld();
@@ -373,31 +391,31 @@ __global__ void __launch_bounds__(kThreadsTc, 1) tile_attn_tc_kernel(const __gri
           for (int x = 0; x < 16; ++x) q[x] = __float_as_uint(__uint_as_float(q[x]) * alpha);
           tc::st_32x32b_x16(to + 16 * c, q);
         }
-        tc::wait_st();
       }
       const float nmn = mref == ninf ? 0.f : -mref;  // all masked so far: every p is exp2(-inf) = 0
-      // P = exp2(s - mref) as a bf16 hi + lo pair into tensor memory, this
-      // half's keys: hi pairs in columns 16 h .. 16 h + 15, lo pairs 32 further
-      uint32_t phi[16], plo[16];
+      // P = exp2(s - mref) as bf16 hi + lo pairs over S: hi pairs in columns
+      // 0-31, lo pairs in 32-63 (S of this block was read above)
       float rq[4] = {0.f, 0.f, 0.f, 0.f};  // four independent partial row sums
 #pragma unroll
-      for (int j = 0; j < 16; ++j) {
-        const float p0 = fast_exp2(fmaf(sv[2 * j], mul, nmn));
-        const float p1 = fast_exp2(fmaf(sv[2 * j + 1], mul, nmn));
-        rq[j & 3] += p0 + p1;
-        // hi = p truncated to bf16 (the upper halves, one byte permute); lo = the
-        // exact remainder p - hi (< 2^-7 p) rounded to bf16: |p - hi - lo| < 2^-16 p
-        phi[j] = pack_bf16(p0, p1);
-        plo[j] = pack_bf16(p0 - bf16_lo(phi[j]), p1 - bf16_hi(phi[j]));
+      for (int h2 = 0; h2 < 2; ++h2) {
+        uint32_t phi[16], plo[16];
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+          const float p0 = fast_exp2(fmaf(sv[32 * h2 + 2 * j], mul, nmn));
+          const float p1 = fast_exp2(fmaf(sv[32 * h2 + 2 * j + 1], mul, nmn));
+          rq[j & 3] += p0 + p1;
+          phi[j] = pack_bf16(p0, p1);
+          plo[j] = pack_bf16(p0 - bf16_lo(phi[j]), p1 - bf16_hi(phi[j]));
+        }
+        tc::st_32x32b_x16(ts + 16 * h2, phi);
+        tc::st_32x32b_x16(ts + 32 + 16 * h2, plo);
       }
-      const uint32_t tp = tmem + lane_off + kColP + 64u * b + 16u * h;
-      tc::st_32x32b_x16(tp, phi);
-      tc::st_32x32b_x16(tp + 32, plo);
       lh += (rq[0] + rq[1]) + (rq[2] + rq[3]);
-      // V rows past the cache end hold other data: zero them before PV reads them
+      // V rows past the cache end hold other data: zero them before PV reads
+      // them (each tile's warps do it, as each tile's PV waits only for its own)
       if (kb0 + kBlk > N) {
         unsigned char* st = ring + (i % kStages) * kStage;
-        for (int x = 32 * warp + lane; x < (kb0 + kBlk - N) * 16; x += 32 * kSmWarps) {
+        for (int x = r; x < (kb0 + kBlk - N) * 16; x += 128) {
           const int row = (N - kb0) + (x >> 4), ch = x & 15;
           *reinterpret_cast<uint4*>(st + (2 + (ch >> 3)) * kBox + swz128(row, ch & 7)) = make_uint4(0u, 0u, 0u, 0u);
         }
@@ -406,52 +424,41 @@ __global__ void __launch_bounds__(kThreadsTc, 1) tile_attn_tc_kernel(const __gri
       tc::wait_st();
       tc::fence_before_sync();  // P and the rescaled O before PV_i reads them
       __syncwarp();
-      if (lane == 0) mbar_arrive(p_full + b);
-      if (i + 1 < nb && !load_s(i + 1)) {
-        fail = 1;
-        break;
-      }
-      // PV_{i-1} done before P_{i+1} overwrites its buffer
-      if (i >= 1 && o_seen < i) {
-        if (!wait_pv(i - 1)) {
-          fail = 1;
-          break;
-        }
-        o_seen = i;
-      }
+      if (lane == 0) mbar_arrive(p_full_t + b);
     }
-    tc::wait_ld();  // no TMEM load of S left in flight (a failed wait may leave one)
-    // the result: PV of the last block, then this half of O into registers
-    for (int j = o_seen; j < nb && !fail; ++j)
-      if (!wait_pv(j)) fail = 1;
-    if (!fail && nb > 0) {
+    // the row's output: PV of the last block (the earlier ones ran before it),
+    // then O / l straight from tensor memory
+    if (!fail && nb > 0 && !wait_pv(nb - 1)) fail = 1;
+    if (!fail) {
       tc::fence_after_sync();
-#pragma unroll
-      for (int c = 0; c < 4; ++c) {
+      const size_t orow = (size_t)(row0 + v / G) * a.Hq + (size_t)g * G + v % G;
+      const float inv = lh > 0.f ? 1.f / lh : 0.f;
+#pragma unroll 1
+      for (int c = 0; c < 8; ++c) {
         uint32_t q[16];
-        tc::ld_32x32b_x16(to + 16 * c, q);
-        tc::wait_ld();
+        if (nb > 0) {
+          tc::ld_32x32b_x16(to + 16 * c, q);
+          tc::wait_ld();
+        } else {
 #pragma unroll
-        for (int x = 0; x < 16; ++x) o[16 * c + x] = __uint_as_float(q[x]);
+          for (int x = 0; x < 16; ++x) q[x] = 0u;
+        }
+        if (vok) {
+          float* dst = a.out + orow * kHeadDim + 16 * c;
+#pragma unroll
+          for (int x = 0; x < 16; x += 4)
+            *reinterpret_cast<float4*>(dst + x) =
+                make_float4(__uint_as_float(q[x]) * inv, __uint_as_float(q[x + 1]) * inv,
+                            __uint_as_float(q[x + 2]) * inv, __uint_as_float(q[x + 3]) * inv);
+        }
       }
+      if (vok && a.lse) a.lse[orow] = lh > 0.f ? mref * kLn2 + logf(lh) : ninf;
     }
-    red[h * 128 + r] = lh;  // added to the other half's after the final barrier
   }
   tc::fence_before_sync();
-  const int all_ok = __syncthreads_and(!fail);
+  __syncthreads_and(!fail);
   tc::fence_after_sync();
   if (warp == 0) tc::tmem_dealloc(tmem, 512);
-  // ---- softmax warps: row sum of both halves, this half's 64 dims of the output
-  if (warp < kSmWarps && all_ok && vok) {
-    const float l = lh + red[(h ^ 1) * 128 + r];
-    const float inv = l > 0.f ? 1.f / l : 0.f;
-    const size_t orow = (size_t)(row0 + v / G) * a.Hq + (size_t)g * G + v % G;
-    float* dst = a.out + orow * kHeadDim + 64 * h;
-#pragma unroll
-    for (int d = 0; d < 64; d += 4)
-      *reinterpret_cast<float4*>(dst + d) = make_float4(o[d] * inv, o[d + 1] * inv, o[d + 2] * inv, o[d + 3] * inv);
-    if (a.lse && h == 0) a.lse[orow] = l > 0.f ? mref * kLn2 + logf(l) : ninf;
-  }
 }
 
 }  // namespace
@@ -468,6 +475,7 @@ cudaError_t launch_tile_attn_tc(const TileAttnArgs& a, cudaStream_t st) {
   return cudaGetLastError();
 }
 
-int tile_attn_tc_mchunks(int vectors_per_tile) { return (vectors_per_tile + 127) / 128; }
+// CTAs per (tile, KV head): 256 query vectors each.
+int tile_attn_tc_mchunks(int vectors_per_tile) { return (vectors_per_tile + 128 * kTiles - 1) / (128 * kTiles); }
 
 }  // namespace sa
