@@ -41,6 +41,37 @@ constexpr int kRtVecs = 224;                                // query vectors per
 constexpr int kQsChunk = kRtVecs * 128;                      // one 128-byte K chunk of all vectors
 constexpr int kQsBytes = 4 * kQsChunk;                       // 112 KiB ([q- | q+], 256 bf16)
 
+// Max over the first nv (<= kRtVecs) fp32 columns of this thread's TMEM lane
+// starting at ta: four loads in flight per wait, four independent max chains,
+// no per-column test when every column is valid.
+SA_DEV float acc_row_max(uint32_t ta, int nv) {
+  const float ninf = -__int_as_float(0x7f800000);
+  float m[4] = {ninf, ninf, ninf, ninf};
+  constexpr int kChunks = kRtVecs / 16;  // 14
+#pragma unroll
+  for (int c0 = 0; c0 < kChunks; c0 += 4) {
+    uint32_t r[4][16];
+#pragma unroll
+    for (int c = 0; c < 4; ++c)
+      if (c0 + c < kChunks) tc::ld_32x32b_x16(ta + 16 * (c0 + c), r[c]);
+    tc::wait_ld();
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      if (c0 + c >= kChunks) continue;
+      tc::reg_fence(r[c]);
+      if (nv >= kRtVecs) {
+#pragma unroll
+        for (int i = 0; i < 16; ++i) m[i & 3] = fmaxf(m[i & 3], __uint_as_float(r[c][i]));
+      } else {
+#pragma unroll
+        for (int i = 0; i < 16; ++i)
+          if (16 * (c0 + c) + i < nv) m[i & 3] = fmaxf(m[i & 3], __uint_as_float(r[c][i]));
+      }
+    }
+  }
+  return fmaxf(fmaxf(m[0], m[1]), fmaxf(m[2], m[3]));
+}
+
 // Inverse of order_key.
 SA_DEV float key_to_float(uint32_t k) {
   const uint32_t u = (k & 0x80000000u) ? (k & 0x7fffffffu) : ~k;
@@ -478,19 +509,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) route_tc_kernel(const __grid_co
       }
       tc::fence_after_sync();
       const uint32_t ta = tmem + (uint32_t)((e & 1) * kTcAccCols) + ((uint32_t)(32 * warp) << 16);
-      float mx = ninf;
-#pragma unroll
-      for (int cc = 0; cc < kRtVecs / 16; cc += 2) {
-        uint32_t r0[16], r1[16];
-        tc::ld_32x32b_x16(ta + 16 * cc, r0);
-        tc::ld_32x32b_x16(ta + 16 * cc + 16, r1);
-        tc::wait_ld();
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          if (16 * cc + i < nv) mx = fmaxf(mx, __uint_as_float(r0[i]));
-          if (16 * cc + 16 + i < nv) mx = fmaxf(mx, __uint_as_float(r1[i]));
-        }
-      }
+      const float mx = acc_row_max(ta, nv);
       tc::fence_before_sync();
       __syncwarp();
       if (lane == 0) mbar_arrive(acc_empty + (e & 1));
@@ -729,19 +748,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) route_tc_centroid_kernel(const 
       }
       tc::fence_after_sync();
       const uint32_t ta = tmem + (uint32_t)((e & 1) * kTcAccCols) + ((uint32_t)(32 * warp) << 16);
-      float mx = ninf;
-#pragma unroll
-      for (int cc = 0; cc < kRtVecs / 16; cc += 2) {
-        uint32_t r0[16], r1[16];
-        tc::ld_32x32b_x16(ta + 16 * cc, r0);
-        tc::ld_32x32b_x16(ta + 16 * cc + 16, r1);
-        tc::wait_ld();
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          if (16 * cc + i < nv) mx = fmaxf(mx, __uint_as_float(r0[i]));
-          if (16 * cc + 16 + i < nv) mx = fmaxf(mx, __uint_as_float(r1[i]));
-        }
-      }
+      const float mx = acc_row_max(ta, nv);
       tc::fence_before_sync();
       __syncwarp();
       if (lane == 0) mbar_arrive(acc_empty + (e & 1));
