@@ -64,6 +64,8 @@ def parse():
     ap.add_argument("--no-extra", action="store_true", help="skip the secondary modes/rules")
     ap.add_argument("--router-only", action="store_true",
                     help="time only the router workload (route + tile attention) and print its JSON")
+    ap.add_argument("--ratio-only", action="store_true",
+                    help="print only the ratio-budget workload's timings")
     ap.add_argument("--tsa-only", action="store_true",
                     help="print only the TSA workload's timings (token and chunk-count budgets)")
     return ap.parse_args()
@@ -555,12 +557,14 @@ def run_gpu_arm(args, rank, world, dist):
     for g in graphs.values():
         del g
     graphs.clear()
-    router = tsa = None
+    router = tsa = ratio = None
     if not args.no_extra:
         router = router_leg(torch, dev, max(5, min(args.steps, 50)), max(3, args.warmup))
         tsa = tsa_leg(torch, dev, max(10, min(args.steps, 50)), max(3, args.warmup))
+        torch.cuda.empty_cache()
+        ratio = ratio_leg(torch, dev, max(5, min(args.steps, 20)), max(3, args.warmup))
     return dict(ms=ms, value=value, kern=kern, clocks=clocks.summary(), e2e_ms=e2e_ms, e2e_bf16=e2e_bf16, h2d=h2d,
-                d2h=d2h, meta_bytes=meta_bytes, kv_bytes=kv_bytes, extra=extra, router=router, tsa=tsa,
+                d2h=d2h, meta_bytes=meta_bytes, kv_bytes=kv_bytes, extra=extra, router=router, tsa=tsa, ratio=ratio,
                 launches_per_step=MODES[args.mode])
 
 
@@ -720,6 +724,74 @@ def tsa_leg(torch, dev, steps: int, warmup: int):
     return res
 
 
+def ratio_leg(torch, dev, steps: int, warmup: int):
+    """The ratio-budget workload (64 layers x 8 sequences stacked along the
+    batch axis, 64 query / 8 KV heads, 32,768 tokens = 2048 16-token pages):
+    the one-launch decode step under the ratio budget K = max(topk_val + bos
+    + eos, floor(P ratio)) with forced first / last pages, for the centroid
+    (bos = eos = 1) and envelope (bos = 0, eos = 1) methods at three ratios.
+    Effective bytes = metadata of every page + K/V of the K kept pages."""
+    import block_sparse_kv_page_b200 as sa
+    import datagen as DG
+    w = DG.WORKLOADS[4]
+    L, Bw, Nw, ps = w.layers, w.B, w.N, w.page_size
+    P = Nw // ps
+    k_all = torch.empty((L * Bw, w.Hkv, Nw, D), dtype=torch.bfloat16, device=dev)
+    v_all = torch.empty_like(k_all)
+    q_all = torch.empty((L * Bw, w.Hq, D), dtype=torch.bfloat16, device=dev)
+    for l in range(L):
+        lay = DG.workload4_layer(l, dev)
+        k_all[l * Bw:(l + 1) * Bw] = lay.k
+        v_all[l * Bw:(l + 1) * Bw] = lay.v
+        q_all[l * Bw:(l + 1) * Bw] = lay.q
+        del lay
+    seq = torch.full((L * Bw,), Nw, dtype=torch.int32, device=dev)
+    kv = sa.KvCache(k_all, v_all, seq, page_size=ps, max_pages=P)
+    units = L * Bw * w.Hkv
+    meta_bytes = float(units) * P * 512
+    stream = torch.cuda.current_stream()
+    res = {}
+    for rule, bos, eos in (("centroid", 1, 1), ("envelope", 0, 1)):
+        meta = kv.meta_buffer()
+        sa.sparse_attn_build_meta(kv, rule, 0, meta)
+        for ratio in (0.5, 0.125, 0.015625):
+            K = max(1 + bos + eos, int(math.floor(P * ratio)))
+            bud = sa.budget_ratio(ratio, topk_val=1, bos=bos, eos=eos)
+            ws = sa.make_workspace(kv, w.Hq, L * Bw, K)
+            sel = torch.zeros((L * Bw, w.Hkv, K), dtype=torch.int32, device=dev)
+            cnt = torch.zeros((L * Bw, w.Hkv), dtype=torch.int32, device=dev)
+            out = torch.zeros((L * Bw, w.Hq, D), dtype=torch.float32, device=dev)
+
+            def step():
+                sa.sparse_attn_decode_step(kv, meta, rule, q_all, bud, K, 1.0 / math.sqrt(D), sel, cnt, out,
+                                           None, ws)
+
+            for _ in range(warmup):
+                step()
+            torch.cuda.synchronize()
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            for _ in range(steps):
+                step()
+            e1.record(stream)
+            torch.cuda.synchronize()
+            ms = e0.elapsed_time(e1) / steps
+            if sa.sparse_attn_get_device_status(ws) != 0:
+                raise RuntimeError("ratio leg: device status set")
+            kv_bytes = float(units) * K * ps * 512
+            res[f"{rule}/ratio{ratio}"] = {
+                "ms_per_step": round(ms, 4), "pages_kept": K,
+                "value": units * K * ps * (w.Hq // w.Hkv) / (ms * 1e-3),
+                "effective_bytes": int(meta_bytes + kv_bytes),
+                "eff_GBps": round((meta_bytes + kv_bytes) / (ms * 1e-3) / 1e9, 1)}
+            del ws, sel, cnt, out
+        del meta
+    del kv, k_all, v_all, q_all, seq
+    torch.cuda.empty_cache()
+    return res
+
+
 class _Null:
     def __enter__(self):
         return self
@@ -783,6 +855,12 @@ def main():
         return 0
 
     import torch
+    if args.ratio_only:
+        dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", 0)))
+        torch.cuda.set_device(dev)
+        if rank == 0:
+            print(json.dumps({"ratio": ratio_leg(torch, dev, args.steps, max(3, args.warmup))}))
+        return 0
     if args.tsa_only:
         dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", 0)))
         torch.cuda.set_device(dev)
@@ -864,6 +942,10 @@ def main():
             "workload": "tsa-chunks-29.5k-b4: 48 layers x 4 sequences, 32:4 heads, 29504 tokens, "
                         "chunks U{16..256} with per-chunk key offsets, one-launch decode step",
             "bound": "hbm", **r["tsa"]},
+        "ratio": None if r["ratio"] is None else {
+            "workload": "qwen3-32b-ratio-32k-b8: 64 layers x 8 sequences, 64:8 heads, 32768 tokens, "
+                        "16-token pages, ratio budget with forced bos/eos pages, one-launch decode step",
+            "bound": "hbm", **r["ratio"]},
     }
     print(json.dumps(line))
     return 0
