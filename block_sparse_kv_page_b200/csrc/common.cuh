@@ -1,6 +1,6 @@
 // Device helpers shared by the sparse-attention kernels (sm_100a).
 //
-// Fragment conventions (warp-level mma.sync, m16n8k16 bf16 and m16n8k8 tf32):
+// Fragment conventions (warp-level mma.sync, m16n8k16 bf16):
 // lane = 4*g + c with g = lane / 4 (row group) and c = lane % 4.
 //   A (16 x 16 bf16): reg0 = A[g][2c..2c+1], reg1 = A[g+8][2c..2c+1],
 //                     reg2 = A[g][2c+8..2c+9], reg3 = A[g+8][2c+8..2c+9]
@@ -36,19 +36,6 @@ SA_DEV uint32_t smem_addr(const void* p) {
 // Record the first device-side error code in the workspace status word.
 SA_DEV void flag_status(int* status, int code) {
   if (status) atomicCAS(status, 0, code);
-}
-
-// 16-byte global -> shared copy; when !valid nothing is read and zeros land.
-SA_DEV void cp_async16(void* dst_smem, const void* src_gmem, bool valid) {
-  const int n = valid ? 16 : 0;
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(smem_addr(dst_smem)),
-               "l"(src_gmem), "r"(n)
-               : "memory");
-}
-SA_DEV void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::: "memory"); }
-template <int N>
-SA_DEV void cp_async_wait() {
-  asm volatile("cp.async.wait_group %0;\n" ::"n"(N) : "memory");
 }
 
 SA_DEV uint4 lds128(const void* p) {
@@ -192,26 +179,11 @@ SA_DEV void mma_bf16(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint3
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
-SA_DEV void mma_tf32(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
-                     uint32_t b0, uint32_t b1) {
-  asm volatile(
-      "mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 "
-      "{%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};\n"
-      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
-}
-
 // FP64 tensor-core MMA m8n8k4: a = A[g][c], b = B[c][g], c0,c1 = C[g][2c..2c+1].
 SA_DEV void mma_f64(double& c0, double& c1, double a, double b) {
   asm volatile("mma.sync.aligned.m8n8k4.row.col.f64.f64.f64.f64 {%0,%1}, {%2}, {%3}, {%0,%1};\n"
                : "+d"(c0), "+d"(c1)
                : "d"(a), "d"(b));
-}
-
-SA_DEV uint32_t to_tf32(float x) {
-  uint32_t r;
-  asm("cvt.rna.tf32.f32 %0, %1;\n" : "=r"(r) : "f"(x));
-  return r;
 }
 
 // Transpose an 8x8 b16 matrix held in the standard fragment layout.

@@ -6,7 +6,7 @@
 // SWIZZLE_128B, i.e. rows of 128 bytes (64 bf16 or 32 fp32 of the K axis), 8-row
 // swizzle atoms of 1024 bytes, each K-chunk of 128 bytes a separate
 // [rows][128 B] region whose base is 1024-byte aligned.  One MMA consumes 32
-// bytes of K per row (16 bf16 or 8 tf32), so step k of chunk c starts at
+// bytes of K per row (16 bf16), so step k of chunk c starts at
 // chunk_base(c) + 32 * (k % 4); the hardware applies the swizzle from the
 // address bits, as TMA did when it wrote the tile.
 #pragma once
@@ -48,14 +48,13 @@ SA_DEV uint64_t smem_desc_sw128(const void* p) {
 }
 
 // Instruction descriptor, dense, fp32 accumulator (bits [4,6) = 1), both
-// operands K-major; `fmt` = 1 for bf16 (kind::f16) or 2 for tf32 (kind::tf32)
-// in the A [7,10) and B [10,13) format fields; N >> 3 in [17,23), M >> 4 in
+// operands K-major; `fmt` = 1 for bf16 (kind::f16) in the A [7,10) and B
+// [10,13) format fields; N >> 3 in [17,23), M >> 4 in
 // [24,29).
 __host__ __device__ constexpr uint32_t idesc_f32acc(uint32_t fmt, uint32_t M, uint32_t N) {
   return (1u << 4) | (fmt << 7) | (fmt << 10) | ((N >> 3) << 17) | ((M >> 4) << 24);
 }
 constexpr uint32_t kFmtBF16 = 1;
-constexpr uint32_t kFmtTF32 = 2;
 
 // ---------------------------------------------------------------- MMA
 // D[tmem] (+)= A[smem] . B[smem]^T, issued by a single thread.
@@ -63,13 +62,6 @@ SA_DEV void mma_bf16_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint3
   asm volatile(
       "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
       " tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}\n" ::"r"(d_tmem),
-      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"((uint32_t)acc)
-      : "memory");
-}
-SA_DEV void mma_tf32_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc, bool acc) {
-  asm volatile(
-      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
-      " tcgen05.mma.cta_group::1.kind::tf32 [%0], %1, %2, %3, p;\n}\n" ::"r"(d_tmem),
       "l"(a_desc), "l"(b_desc), "r"(idesc), "r"((uint32_t)acc)
       : "memory");
 }
