@@ -18,6 +18,12 @@ Modes:
                decode: 3 launches per step);
   sequential : one call per layer and stage (144 launches per step) in a graph.
 
+Secondary legs (single-GPU runs, unless --no-extra), reported under "modes",
+"router", "tsa" and "ratio" in the same line: the other modes and rule, the
+per-query-head selection, the router applied to decode, the 128K-context
+router (route + tile attention), the TSA workload (token and chunk-count
+budgets) and the ratio-budget workload (64 layers x 8 sequences, 32K tokens).
+
 Output: one JSON line on rank 0.  `value` = tokens*heads/s (tokens attended x
 query heads x layers per step / step time, summed over ranks).  Inputs stay
 resident in HBM; each step touches ~0.58 GB (> the 126 MB L2), so no L2 flush
@@ -472,7 +478,7 @@ def run_gpu_arm(args, rank, world, dist):
 
     # ---- secondary measurements (same timing rules), labelled
     extra = {}
-    if not args.no_extra:
+    if not args.no_extra and world == 1:  # secondary legs: single-GPU runs only
         for mode in MODES:
             for rule in ("envelope", "centroid"):
                 if (mode, rule) == (args.mode, args.rule):
@@ -558,7 +564,7 @@ def run_gpu_arm(args, rank, world, dist):
         del g
     graphs.clear()
     router = tsa = ratio = None
-    if not args.no_extra:
+    if not args.no_extra and world == 1:  # secondary legs: single-GPU runs only
         router = router_leg(torch, dev, max(5, min(args.steps, 50)), max(3, args.warmup))
         tsa = tsa_leg(torch, dev, max(10, min(args.steps, 50)), max(3, args.warmup))
         torch.cuda.empty_cache()
