@@ -930,6 +930,7 @@ def main():
                    "parallelism": f"replicas{world}" if world > 1 else "single",
                    "l2": "inputs larger than L2 (~0.58 GB touched per step), no flush"},
         "effective_GBps": round(eff, 1), "effective_frac_of_peak": round(eff / peak, 4),
+        "selected_token_fraction": round(args.budget / N, 4),
         "per_kernel_ms": {k: round(v, 5) for k, v in kern.items()} if kern else None,
         "roofline": roof, "clocks": r["clocks"],
         "e2e": {"value": whole_job_value(HQ * args.budget * LAYERS * B, world, r["e2e_ms"]), "unit": UNIT,
