@@ -6,6 +6,8 @@ layouts, against the float64 oracle through the C ABI.
   register path; 2500 pages; 2300 variable chunks under a token budget).
 * Exactly 2048 pages: the largest unit the register path takes.
 * A single KV head (G = 8) and G = 1 (every query head its own KV head).
+* The largest sizes the calls take: 16,384 pages in one unit, 32,768 units in
+  one decode step.
 Each case runs the separate calls and the one-launch step (which must agree
 with them bit for bit).
 """
@@ -13,6 +15,7 @@ import math
 
 import numpy as np
 import pytest
+import torch
 
 import datagen as DG
 
@@ -70,3 +73,35 @@ def test_many_chunks_token_budget(cuda_dev, R, rule):
 def test_group_of_one(cuda_dev, R, rule):
     lay = DG.make_decode_layer(B=2, Hq=4, Hkv=4, seq_lens=[3000, 1200], seed=721, device=cuda_dev)
     _check_both(R, lay, 16, rule, {"kind": "topk", "k": 33})
+
+
+@pytest.mark.parametrize("rule", ["envelope", "centroid"])
+def test_max_pages_per_unit(cuda_dev, R, rule):
+    """16,384 pages in one (sequence, KV head), the largest page axis the
+    selection takes (its keys fill 128 KiB of shared memory in the step)."""
+    N = 16384 * 16
+    lay = DG.make_decode_layer(B=1, Hq=8, Hkv=1, seq_lens=[N], seed=731, device=cuda_dev)
+    _check_both(R, lay, 16, rule, {"kind": "topk", "k": 1000})
+
+
+def test_max_units_in_one_step(cuda_dev, R):
+    """32,768 (sequence, KV head) units in one decode step (its limit: unit
+    flags and split counters share the workspace header), short ragged
+    caches; a seeded sample of units is checked against the oracle and all of
+    them against the separate calls."""
+    rng = np.random.default_rng(741)
+    B, Hkv = 8192, 4
+    lens = [int(x) for x in rng.integers(1, 200, size=B)]
+    lay = DG.make_decode_layer(B=B, Hq=16, Hkv=Hkv, seq_lens=lens, seed=741, device=cuda_dev, cap=200)
+    bd = {"kind": "topk", "k": 4}
+    s = R.run_step(lay, page_size=16, rule="envelope", budget=bd, scale=SCALE, stale=True)
+    assert s["status"] == 0
+    picks = rng.choice(B * Hkv, size=48, replace=False)
+    units = [(int(u) // Hkv, int(u) % Hkv) for u in picks]
+    st = R.check_layer(lay, s, page_size=16, rule="envelope", budget=bd, scale=SCALE, units=units)
+    assert st["max_out_err"] < 1e-4
+    g = R.run_gpu(lay, page_size=16, rule="envelope", budget=bd, scale=SCALE)
+    assert g["status"] == 0
+    for key in ("sel_idx", "sel_count", "out", "lse"):
+        a_, b_ = torch.nan_to_num(s[key], nan=7.0), torch.nan_to_num(g[key], nan=7.0)
+        assert torch.equal(a_, b_), key
