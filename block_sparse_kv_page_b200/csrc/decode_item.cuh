@@ -122,9 +122,12 @@ SA_DEV void store_out(const DecodeArgs& a, size_t row, int d0, const float (&A)[
   }
 }
 
+// n_known >= 0: the unit's kept count, already read by the caller (the fused
+// step takes it from the unit's selection flag); else it is loaded here.
+// n_tok_known >= 0 likewise stands for the sequence length.
 template <bool PER_HEAD = false>
 SA_DEV void decode_item(const DecodeArgs& a, const int u, const int split, const Smem& sm,
-                        WarpState& ws) {
+                        WarpState& ws, const int n_known = -1, const int n_tok_known = -1) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int gq = lane >> 2, c = lane & 3;
   const UnitMap um = unit_map<PER_HEAD>(u, a.kv.Hkv, a.Hq, a.G);
@@ -133,9 +136,9 @@ SA_DEV void decode_item(const DecodeArgs& a, const int u, const int split, const
   const float ninf = -__int_as_float(0x7f800000);
 
   // ---- geometry of the unit
-  const int N = a.kv.seq_len[b];
+  const int N = n_tok_known >= 0 ? n_tok_known : a.kv.seq_len[b];
   bool bad = (N < 1 || N > a.kv.cap);
-  int n_ent = __ldcg(a.count + u);  // L2: may be written earlier in the launch
+  int n_ent = n_known >= 0 ? n_known : __ldcg(a.count + u);  // L2: may be written earlier in the launch
   if (n_ent < 0 || n_ent > a.max_sel) bad = true;
   if (bad) n_ent = 0;
   const int32_t* idx_u = a.idx + (size_t)u * a.max_sel;

@@ -35,8 +35,8 @@
 // longest prefix of the (score desc, index asc) order within the budget".
 // Weight 1 per page gives top-k / ratio; weight = chunk length gives the token
 // budget.  Output is the kept set in ascending page order.  In the fused step
-// the unit's counter is left at kUnitSelected (release) once the output
-// is written, for consumers in the same launch.
+// the unit's counter is left at kUnitSelected | kept count (release) once the
+// output is written, for consumers in the same launch.
 #pragma once
 
 #include "common.cuh"
@@ -692,7 +692,9 @@ SA_DEV void select_item(const SelectArgs& a, const int u, const int split, const
   select_unit(a, u, b, N, P, S);
   if (FUSED) {
     __syncthreads();
-    if (tid == 0) st_release_u32(&a.ws_count[u], kUnitSelected);
+    // the flag carries the kept count too (thread 0 wrote it), so a decode
+    // item reads both with its one acquire
+    if (tid == 0) st_release_u32(&a.ws_count[u], kUnitSelected | (uint32_t)a.sel_count[u]);
   }
 }
 

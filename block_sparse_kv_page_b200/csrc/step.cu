@@ -51,17 +51,18 @@ __host__ __device__ int body_bytes(int max_pages) {
   return kb > sel::kRingBytes ? kb : sel::kRingBytes;
 }
 
-// Wait until a unit's selection is published; false (and SA_ERR_TIMEOUT) if
-// the bound runs out.
-SA_DEV bool wait_selected(const uint32_t* flag, int* status) {
+// Wait until a unit's selection is published and return its kept count (the
+// flag's low bits); -1 (and SA_ERR_TIMEOUT) if the bound runs out.
+SA_DEV int wait_selected(const uint32_t* flag, int* status) {
   uint32_t ns = 32;
   for (uint32_t i = 0; i < kFlagSpinLimit; ++i) {
-    if (ld_acquire_u32(flag) == sel::kUnitSelected) return true;
+    const uint32_t v = ld_acquire_u32(flag);
+    if (v & sel::kUnitSelected) return (int)(v & ~sel::kUnitSelected);
     __nanosleep(ns);
     if (ns < 256) ns <<= 1;
   }
   flag_status(status, SA_ERR_TIMEOUT);
-  return false;
+  return -1;
 }
 
 template <int RULE>
@@ -71,7 +72,7 @@ __global__ void __launch_bounds__(kThreads, SA_STEP_CTAS_PER_SM)
   __shared__ uint32_t s_hist[512];
   __shared__ uint32_t s_scan[32];
   __shared__ uint32_t s_bc[8];
-  __shared__ int s_last, s_item, s_ntiles;
+  __shared__ int s_last, s_item, s_ntiles, s_count, s_ntok;
   unsigned char* base = reinterpret_cast<unsigned char*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   const int body = body_bytes(a.sel.kv.max_pages);
@@ -100,8 +101,13 @@ __global__ void __launch_bounds__(kThreads, SA_STEP_CTAS_PER_SM)
       if (item >= a.n_score && item < n_items) {
         int u, split;
         dec::item_unit(a.dec, item - a.n_score, u, split);
-        if (!wait_selected(a.sel.ws_count + u, a.sel.status))  // acquire
-          item = n_items;  // gave up: this CTA stops taking work
+        // the sequence length is an input of the launch: its load (kept in a
+        // register until after the wait) overlaps the acquire
+        const int ntok = a.dec.kv.seq_len[unit_map<false>(u, a.dec.kv.Hkv, a.dec.Hq, a.dec.G).b];
+        const int cnt = wait_selected(a.sel.ws_count + u, a.sel.status);  // acquire
+        s_count = cnt;
+        s_ntok = ntok;
+        if (cnt < 0) item = n_items;  // gave up: this CTA stops taking work
       }
       s_item = item;
     }
@@ -117,7 +123,7 @@ __global__ void __launch_bounds__(kThreads, SA_STEP_CTAS_PER_SM)
       int u, split;
       dec::item_unit(a.dec, item - a.n_score, u, split);
       if (a.sel.k_new != nullptr && lane == 0) fence_proxy_async_global();  // appended rows, then TMA
-      dec::decode_item(a.dec, u, split, D, ws);
+      dec::decode_item(a.dec, u, split, D, ws, s_count, s_ntok);  // count from the unit's flag
     }
     fence_proxy_async();  // generic writes to the ring (keys, merge) before the next TMA writes
     __syncthreads();
