@@ -500,33 +500,41 @@ def run_gpu_arm(args, rank, world, dist):
         sel_h = torch.zeros((L * B, HQ, k), dtype=torch.int32, device=dev)
         cnt_h = torch.zeros((L * B, HQ), dtype=torch.int32, device=dev)
         for rule in ("envelope", "centroid"):
-            def per_head_step():
+            def per_head_calls():
                 sa.sparse_attn_build_meta(kv, rule, -1, metas[rule])
                 sa.sparse_attn_select_per_head(kv, metas[rule], rule, inp["q"], budget, k, sel_h, cnt_h, None,
                                                ws_h)
                 sa.sparse_attn_decode_per_head(kv, inp["q"], scale, sel_h, cnt_h, k, out, lse, ws_h)
-            for _ in range(max(3, args.warmup)):
-                per_head_step()
-            barrier()
-            e0 = torch.cuda.Event(enable_timing=True)
-            e1 = torch.cuda.Event(enable_timing=True)
-            n_rep = max(10, args.steps // 2)
-            e0.record(stream)
-            for _ in range(n_rep):
-                per_head_step()
-            e1.record(stream)
-            torch.cuda.synchronize()
-            m2 = max_over_ranks(e0.elapsed_time(e1) / n_rep, dist, dev)
-            # K/V of the distinct pages the G heads of a KV head keep (the union)
-            sh = sel_h.view(L * B, HKV, HQ // HKV, k).cpu()
-            distinct = sum(int(torch.unique(sh[r, g2]).numel()) for r in range(L * B) for g2 in range(HKV))
-            kv_union = distinct * PS * 2 * D * 2
-            extra[f"per-head-batched/{rule}"] = {
-                "ms_per_step": round(m2, 4), "value": tok_heads * world / (m2 * 1e-3),
-                "eff_GBps": (meta_bytes + kv_union) / (m2 * 1e-3) / 1e9,
-                "distinct_pages_per_kv_head": round(distinct / (L * B * HKV), 1),
-                "note": "one page set per query head (separate build_meta, select, decode calls); effective "
-                        "bytes = metadata once + K/V of the union of a KV head's query-head page sets"}
+
+            def per_head_fused():
+                sa.sparse_attn_decode_step_per_head(kv, metas[rule], rule, inp["q"], budget, k, scale, sel_h,
+                                                    cnt_h, out, lse, ws_h)
+            for label, fn, how in (("per-head-batched", per_head_calls, "separate build_meta, select, decode "
+                                    "calls"),
+                                   ("per-head-step", per_head_fused, "one sparse_attn_decode_step_per_head "
+                                    "launch")):
+                for _ in range(max(3, args.warmup)):
+                    fn()
+                barrier()
+                e0 = torch.cuda.Event(enable_timing=True)
+                e1 = torch.cuda.Event(enable_timing=True)
+                n_rep = max(10, args.steps // 2)
+                e0.record(stream)
+                for _ in range(n_rep):
+                    fn()
+                e1.record(stream)
+                torch.cuda.synchronize()
+                m2 = max_over_ranks(e0.elapsed_time(e1) / n_rep, dist, dev)
+                # K/V of the distinct pages the G heads of a KV head keep (the union)
+                sh = sel_h.view(L * B, HKV, HQ // HKV, k).cpu()
+                distinct = sum(int(torch.unique(sh[r, g2]).numel()) for r in range(L * B) for g2 in range(HKV))
+                kv_union = distinct * PS * 2 * D * 2
+                extra[f"{label}/{rule}"] = {
+                    "ms_per_step": round(m2, 4), "value": tok_heads * world / (m2 * 1e-3),
+                    "eff_GBps": (meta_bytes + kv_union) / (m2 * 1e-3) / 1e9,
+                    "distinct_pages_per_kv_head": round(distinct / (L * B * HKV), 1),
+                    "note": f"one page set per query head ({how}); effective bytes = metadata once + K/V of "
+                            "the union of a KV head's query-head page sets"}
         if sa.sparse_attn_get_device_status(ws_h) != 0:
             raise RuntimeError("per-head leg: device status set")
         del ws_h, sel_h, cnt_h

@@ -408,9 +408,8 @@ size_t sparse_attn_workspace_size_per_head(const sa_kv_desc* kv, int32_t n_q_hea
   const long long units = (long long)kv->batch * n_q_heads;
   if (units > kMaxUnits) return 0;
   const DecodePlan plan = decode_plan((int)units, max_tiles_per_unit(kv, max_sel), device_sm_count());
-  const size_t sel = select_scratch(kv, true, n_q_heads);
-  const size_t dec = decode_scratch(plan);
-  return kScratch + (sel > dec ? sel : dec);
+  // the fused per-head step keeps the scores and the split partials at once
+  return kScratch + select_scratch(kv, true, n_q_heads) + decode_scratch(plan);
 }
 
 sa_status sparse_attn_workspace_init(void* ws, size_t ws_bytes, void* stream) {
@@ -543,7 +542,8 @@ static sa_status decode_step(const sa_kv_desc* kv, void* meta, sa_score_rule rul
                              const void* q, int32_t n_q_heads, const void* k_new,
                              const void* v_new, const sa_budget* budget, int32_t max_sel,
                              float scale, int32_t* sel_idx, int32_t* sel_count, void* out,
-                             bool out_bf16, float* lse, void* ws, size_t ws_bytes, void* stream) {
+                             bool out_bf16, float* lse, bool per_head, void* ws, size_t ws_bytes,
+                             void* stream) {
   int G;
   sa_status s = check_select(kv, meta, rule, q, n_q_heads, budget, max_sel, sel_idx, sel_count,
                              nullptr, &G);
@@ -551,7 +551,7 @@ static sa_status decode_step(const sa_kv_desc* kv, void* meta, sa_score_rule rul
   if (!out || !aligned(out, 16) || (lse && !aligned(lse, 4))) return SA_ERR_INVALID;
   if (!std::isfinite(scale)) return SA_ERR_INVALID;
   if (kv->page_size == 0 && max_sel > kMaxChunkSel) return SA_ERR_UNSUPPORTED;
-  const long long units = (long long)kv->batch * kv->n_kv_heads;
+  const long long units = (long long)kv->batch * (per_head ? n_q_heads : kv->n_kv_heads);
   if (2 * units > kMaxUnits) return SA_ERR_UNSUPPORTED;  // unit flags + split counters
   const unsigned long long kv_rows = (unsigned long long)kv->batch * kv->n_kv_heads * kv->cap_tokens;
   if (kv_rows > 0x7fffffffULL) return SA_ERR_UNSUPPORTED;  // TMA row coordinates are int32
@@ -562,7 +562,7 @@ static sa_status decode_step(const sa_kv_desc* kv, void* meta, sa_score_rule rul
     if (t < plan_tiles) plan_tiles = t;
   }
   const DecodePlan plan = decode_plan((int)units, plan_tiles, sm);
-  const size_t sel_bytes = select_scratch(kv);
+  const size_t sel_bytes = select_scratch(kv, per_head, n_q_heads);
   const size_t need = kScratch + sel_bytes + decode_scratch(plan);
   if ((s = check_ws(ws, ws_bytes, need)) != SA_OK) return s;
   if (step_smem_bytes(kv->max_pages, max_sel, kv->page_size == 0) > 227 * 1024)
@@ -578,6 +578,11 @@ static sa_status decode_step(const sa_kv_desc* kv, void* meta, sa_score_rule rul
                    reinterpret_cast<uint32_t*>(w + 256) + units, reinterpret_cast<int*>(ws), plan))
     return SA_ERR_CUDA;
   if (out_bf16) a.dec.out_bf16 = static_cast<__nv_bfloat16*>(out);
+  if (per_head) {
+    a.sel.per_head = 1;
+    a.sel.splits = select_splits((int)units, kv->max_pages, sm);
+    a.dec.per_head = 1;
+  }
   a.sel.meta_refresh = static_cast<unsigned char*>(meta);
   if (k_new) {
     a.sel.k_new = k_new;
@@ -599,7 +604,16 @@ sa_status sparse_attn_decode_step(const sa_kv_desc* kv, void* meta, sa_score_rul
                                   int32_t* sel_count, float* out, float* lse, void* ws,
                                   size_t ws_bytes, void* stream) {
   return decode_step(kv, meta, rule, q, n_q_heads, nullptr, nullptr, budget, max_sel, scale, sel_idx,
-                     sel_count, out, false, lse, ws, ws_bytes, stream);
+                     sel_count, out, false, lse, false, ws, ws_bytes, stream);
+}
+
+sa_status sparse_attn_decode_step_per_head(const sa_kv_desc* kv, void* meta, sa_score_rule rule,
+                                           const void* q, int32_t n_q_heads, const sa_budget* budget,
+                                           int32_t max_sel, float scale, int32_t* sel_idx,
+                                           int32_t* sel_count, float* out, float* lse, void* ws,
+                                           size_t ws_bytes, void* stream) {
+  return decode_step(kv, meta, rule, q, n_q_heads, nullptr, nullptr, budget, max_sel, scale, sel_idx,
+                     sel_count, out, false, lse, true, ws, ws_bytes, stream);
 }
 
 sa_status sparse_attn_decode_step_append(const sa_kv_desc* kv, void* meta, sa_score_rule rule,
@@ -611,7 +625,7 @@ sa_status sparse_attn_decode_step_append(const sa_kv_desc* kv, void* meta, sa_sc
   if (!k_new || !v_new || !aligned(k_new, 8) || !aligned(v_new, 8)) return SA_ERR_INVALID;
   if (out_dtype != SA_OUT_F32 && out_dtype != SA_OUT_BF16) return SA_ERR_INVALID;
   return decode_step(kv, meta, rule, q, n_q_heads, k_new, v_new, budget, max_sel, scale, sel_idx,
-                     sel_count, out, out_dtype == SA_OUT_BF16, lse, ws, ws_bytes, stream);
+                     sel_count, out, out_dtype == SA_OUT_BF16, lse, false, ws, ws_bytes, stream);
 }
 
 sa_status sparse_attn_route(const sa_kv_desc* kv, const void* meta, sa_score_rule rule,

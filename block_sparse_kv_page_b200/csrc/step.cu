@@ -65,7 +65,8 @@ SA_DEV int wait_selected(const uint32_t* flag, int* status) {
   return -1;
 }
 
-template <int RULE>
+// PER_HEAD: units are (sequence, query head), each selecting its own pages.
+template <int RULE, bool PER_HEAD>
 __global__ void __launch_bounds__(kThreads, SA_STEP_CTAS_PER_SM)
     step_kernel(const __grid_constant__ StepArgs a) {
   extern __shared__ unsigned char smem_raw[];
@@ -103,7 +104,7 @@ __global__ void __launch_bounds__(kThreads, SA_STEP_CTAS_PER_SM)
         dec::item_unit(a.dec, item - a.n_score, u, split);
         // the sequence length is an input of the launch: its load (kept in a
         // register until after the wait) overlaps the acquire
-        const int ntok = a.dec.kv.seq_len[unit_map<false>(u, a.dec.kv.Hkv, a.dec.Hq, a.dec.G).b];
+        const int ntok = a.dec.kv.seq_len[unit_map<PER_HEAD>(u, a.dec.kv.Hkv, a.dec.Hq, a.dec.G).b];
         const int cnt = wait_selected(a.sel.ws_count + u, a.sel.status);  // acquire
         s_count = cnt;
         s_ntok = ntok;
@@ -118,12 +119,12 @@ __global__ void __launch_bounds__(kThreads, SA_STEP_CTAS_PER_SM)
       break;
     }
     if (item < a.n_score) {
-      sel::select_item<RULE, true>(a.sel, item / a.sel.splits, item % a.sel.splits, S, ws);
+      sel::select_item<RULE, true, PER_HEAD>(a.sel, item / a.sel.splits, item % a.sel.splits, S, ws);
     } else {
       int u, split;
       dec::item_unit(a.dec, item - a.n_score, u, split);
       if (a.sel.k_new != nullptr && lane == 0) fence_proxy_async_global();  // appended rows, then TMA
-      dec::decode_item(a.dec, u, split, D, ws, s_count, s_ntok);  // count from the unit's flag
+      dec::decode_item<PER_HEAD>(a.dec, u, split, D, ws, s_count, s_ntok);  // count from the unit's flag
     }
     fence_proxy_async();  // generic writes to the ring (keys, merge) before the next TMA writes
     __syncthreads();
@@ -191,7 +192,10 @@ cudaError_t launch_step(const StepArgs& a, cudaStream_t st) {
   const size_t smem = step_smem_bytes(a.sel.kv.max_pages, a.dec.max_sel, a.sel.kv.page_size == 0);
   const long long items = (long long)a.n_score + a.n_dec;
   if (items > 0x7fffffffLL) return cudaErrorInvalidValue;
-  const void* fn = a.sel.rule == 0 ? (const void*)step_kernel<0> : (const void*)step_kernel<1>;
+  using Fn = void (*)(const StepArgs);
+  const Fn fns[2][2] = {{step_kernel<0, false>, step_kernel<0, true>}, {step_kernel<1, false>, step_kernel<1, true>}};
+  const Fn f = fns[a.sel.rule == 0 ? 0 : 1][a.sel.per_head ? 1 : 0];
+  const void* fn = (const void*)f;
   cudaError_t e = set_smem_attr(fn, smem);
   if (e != cudaSuccess) return e;
   int occ = step_occupancy(fn, smem);
@@ -199,8 +203,7 @@ cudaError_t launch_step(const StepArgs& a, cudaStream_t st) {
   if (occ > SA_STEP_CTAS_PER_SM) occ = SA_STEP_CTAS_PER_SM;
   long long grid = (long long)device_sm_count() * occ;
   if (grid > items) grid = items;
-  if (a.sel.rule == 0) return launch_pdl(step_kernel<0>, (unsigned)grid, kThreads, smem, st, a);
-  return launch_pdl(step_kernel<1>, (unsigned)grid, kThreads, smem, st, a);
+  return launch_pdl(f, (unsigned)grid, kThreads, smem, st, a);
 }
 
 }  // namespace sa

@@ -117,7 +117,8 @@ def sparse_attn_workspace_size_per_head(kv: KvCache, n_q_heads: int, max_sel: in
 
 
 def make_workspace_per_head(kv: KvCache, n_q_heads: int, max_sel: int, stream=None) -> torch.Tensor:
-    """Workspace for sparse_attn_select_per_head / sparse_attn_decode_per_head."""
+    """Workspace for sparse_attn_select_per_head / sparse_attn_decode_per_head /
+    sparse_attn_decode_step_per_head."""
     n = sparse_attn_workspace_size_per_head(kv, n_q_heads, max_sel)
     if n == 0:
         raise SparseAttnError(_abi.SA_ERR_INVALID, "sparse_attn_workspace_size_per_head")
@@ -200,6 +201,24 @@ def sparse_attn_decode_step(kv: KvCache, meta: torch.Tensor, rule, q: torch.Tens
                                        _ptr(lse), ws.data_ptr(), ws.numel() * ws.element_size(),
                                        _stream(stream)),
            "sparse_attn_decode_step")
+
+
+def sparse_attn_decode_step_per_head(kv: KvCache, meta: torch.Tensor, rule, q: torch.Tensor,
+                                     budget: sa_budget, max_sel: int, scale: float, sel_idx: torch.Tensor,
+                                     sel_count: torch.Tensor, out: torch.Tensor, lse: torch.Tensor | None,
+                                     ws: torch.Tensor, stream=None) -> None:
+    """The decode step with one page set per query head: sel_idx [B, Hq, max_sel],
+    sel_count [B, Hq]; ws from make_workspace_per_head."""
+    if q.dtype != torch.bfloat16 or not q.is_contiguous():
+        raise ValueError("q must be contiguous bf16 [B, Hq, 128]")
+    if out.dtype != torch.float32 or not out.is_contiguous():
+        raise ValueError("out must be contiguous fp32")
+    _check(lib.sparse_attn_decode_step_per_head(C.byref(kv.desc), meta.data_ptr(), _rule(rule), q.data_ptr(),
+                                                q.shape[-2], C.byref(budget), int(max_sel), float(scale),
+                                                sel_idx.data_ptr(), sel_count.data_ptr(), out.data_ptr(),
+                                                _ptr(lse), ws.data_ptr(), ws.numel() * ws.element_size(),
+                                                _stream(stream)),
+           "sparse_attn_decode_step_per_head")
 
 
 def sparse_attn_decode_step_append(kv: KvCache, meta: torch.Tensor, rule, q: torch.Tensor,

@@ -240,9 +240,17 @@ sa_status sparse_attn_decode_step_append(const sa_kv_desc* kv, void* meta, sa_sc
  *     head h attends the pages listed for it in idx [B][n_q_heads][max_sel]
  *     (count [B][n_q_heads]), reading K/V of KV head h / G.  out and lse as
  *     in sparse_attn_decode.
- * Both take the workspace sized by sparse_attn_workspace_size_per_head (B *
- * n_q_heads <= 65536 units); other checks and errors as in the shared calls.
- * K/V bytes read grow with the number of distinct pages the G heads keep. */
+ *   sparse_attn_decode_step_per_head: sparse_attn_decode_step with per-head
+ *     units: one launch computes what build_meta(first_token = -1) ->
+ *     sparse_attn_select_per_head -> sparse_attn_decode_per_head compute
+ *     (the newest page's metadata is refreshed once per KV head); sel_idx,
+ *     sel_count as in sparse_attn_select_per_head.  As with the shared step,
+ *     token budgets may round differently from the separate calls (the
+ *     attention splits follow the budget, not max_sel).
+ * All take the workspace sized by sparse_attn_workspace_size_per_head (B *
+ * n_q_heads <= 65536 units; the step needs 2 * B * n_q_heads <= 65536); other
+ * checks and errors as in the shared calls.  K/V bytes read grow with the
+ * number of distinct pages the G heads keep. */
 size_t sparse_attn_workspace_size_per_head(const sa_kv_desc* kv, int32_t n_q_heads, int32_t max_sel);
 sa_status sparse_attn_select_per_head(const sa_kv_desc* kv, const void* meta, sa_score_rule rule,
                                       const void* q, int32_t n_q_heads, const sa_budget* budget,
@@ -252,6 +260,11 @@ sa_status sparse_attn_decode_per_head(const sa_kv_desc* kv, const void* q, int32
                                       float scale, const int32_t* idx, const int32_t* count,
                                       int32_t max_sel, float* out, float* lse, void* ws,
                                       size_t ws_bytes, void* stream);
+sa_status sparse_attn_decode_step_per_head(const sa_kv_desc* kv, void* meta, sa_score_rule rule,
+                                           const void* q, int32_t n_q_heads, const sa_budget* budget,
+                                           int32_t max_sel, float scale, int32_t* sel_idx,
+                                           int32_t* sel_count, float* out, float* lse, void* ws,
+                                           size_t ws_bytes, void* stream);
 
 /* (d) Uncertainty router over query tiles ([ROUTER] "Methodologie" steps 2-5).
  * B == 1, fixed blocks (page_size = block size).  q bf16 [n_q_rows][n_q_heads][128]

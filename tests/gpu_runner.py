@@ -91,12 +91,13 @@ def run_gpu(layer, *, page_size: int, rule: str, budget: dict, scale: float,
 
 def run_step(layer, *, page_size: int, rule: str, budget: dict, scale: float,
              max_pages: int | None = None, max_sel: int | None = None, ws=None, repeat: int = 1,
-             stale: bool = True, append=None, out_dtype=torch.float32):
+             stale: bool = True, append=None, out_dtype=torch.float32, per_head: bool = False):
     """One-launch decode step through the C ABI.  With `stale`, the metadata is
     first built for the cache as it stood before its newest token (seq_len - 1;
     pages never built hold a fill pattern), so the step's own refresh of the
     newest page is what makes the metadata current.  append = (k_new, v_new):
-    run the step that stores the newest token's key and value itself."""
+    run the step that stores the newest token's key and value itself.
+    per_head: the step with one page set per query head (rows [B, Hq])."""
     B, Hkv, cap, D = layer.k.shape
     Hq = layer.q.shape[1]
     if max_pages is None:
@@ -119,14 +120,18 @@ def run_step(layer, *, page_size: int, rule: str, budget: dict, scale: float,
     else:
         sa.sparse_attn_build_meta(kv, rule, 0, meta)
     if ws is None:
-        ws = sa.make_workspace(kv, Hq, B, max_sel)
+        ws = sa.make_workspace_per_head(kv, Hq, max_sel) if per_head else sa.make_workspace(kv, Hq, B, max_sel)
+    U = Hq if per_head else Hkv
     results = []
     for _ in range(repeat):
-        sel_idx = torch.full((B, Hkv, max_sel), -7, dtype=torch.int32, device=dev)
-        sel_count = torch.full((B, Hkv), -7, dtype=torch.int32, device=dev)
+        sel_idx = torch.full((B, U, max_sel), -7, dtype=torch.int32, device=dev)
+        sel_count = torch.full((B, U), -7, dtype=torch.int32, device=dev)
         out = torch.full((B, Hq, 128), float("nan"), dtype=out_dtype, device=dev)
         lse = torch.full((B, Hq), float("nan"), dtype=torch.float32, device=dev)
-        if append is None:
+        if per_head:
+            sa.sparse_attn_decode_step_per_head(kv, meta, rule, layer.q, budget_struct(budget), max_sel,
+                                                scale, sel_idx, sel_count, out, lse, ws)
+        elif append is None:
             sa.sparse_attn_decode_step(kv, meta, rule, layer.q, budget_struct(budget), max_sel, scale,
                                        sel_idx, sel_count, out, lse, ws)
         else:

@@ -132,6 +132,24 @@ def test_decode_step_validation(lib, abi):
     assert call(budget=tokens) == abi.SA_ERR_UNSUPPORTED  # token budgets need chunks
 
 
+def test_decode_step_per_head_validation(lib, abi):
+    """The per-query-head step takes the per-head workspace, which holds the
+    per-head scores and the decode partials at once; its units are
+    (sequence, query head), so the unit bound is reached 8x sooner."""
+    ok = _desc(abi)
+    topk = abi.sa_budget(abi.SA_BUDGET_TOPK, 8, 0.0, 0, 0, 0, 0)
+    need = lib.sparse_attn_workspace_size_per_head(C.byref(ok), 32, 16)
+    assert need > lib.sparse_attn_workspace_size(C.byref(ok), 32, 1, 16)
+
+    def call(desc=ok, max_sel=16, ws_bytes=need):
+        return lib.sparse_attn_decode_step_per_head(C.byref(desc), 0x40000, 0, 0x50000, 32, C.byref(topk),
+                                                    max_sel, 0.088, 0x60000, 0x70000, 0x80000, None,
+                                                    0x100000, ws_bytes, None)
+    assert call(ws_bytes=need - 256) == abi.SA_ERR_WORKSPACE
+    assert call(max_sel=4) == abi.SA_ERR_INVALID          # top_k > max_sel
+    assert call(desc=_desc(abi, batch=1025)) == abi.SA_ERR_UNSUPPORTED  # 2 x 1025 x 32 > 65536
+
+
 def test_decode_step_append_validation(lib, abi):
     ok = _desc(abi)
     topk = abi.sa_budget(abi.SA_BUDGET_TOPK, 8, 0.0, 0, 0, 0, 0)

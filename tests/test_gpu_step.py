@@ -117,6 +117,24 @@ def test_step_parity(cuda_dev, R, rule, name):
 
 
 @pytest.mark.parametrize("rule", ["envelope", "centroid"])
+@pytest.mark.parametrize("name", ["ps16_topk", "ps16_new_page", "ps64_g7", "ratio_bos_eos", "chunks_tokens",
+                                  "many_units"])
+def test_step_per_head_parity(cuda_dev, R, rule, name):
+    """The per-query-head step: every (sequence, query head) against the
+    oracle run on that head alone, and against the separate per-head calls
+    (same page sets; outputs bit-identical except under a token budget)."""
+    lay, ps, bd = _case(cuda_dev, name)
+    s = R.run_step(lay, page_size=ps, rule=rule, budget=bd, scale=SCALE, stale=True, per_head=True)
+    assert s["status"] == 0
+    st = R.check_layer(lay, s, page_size=ps, rule=rule, budget=bd, scale=SCALE, per_head=True)
+    assert st["units"] == lay.k.shape[0] * lay.q.shape[1]
+    assert st["max_out_err"] < 1e-4
+    c = R.run_gpu(lay, page_size=ps, rule=rule, budget=bd, scale=SCALE, per_head=True)
+    assert c["status"] == 0
+    _assert_same(s, c, lay, ps, f"{name}/{rule}/per-head", exact=bd["kind"] != "tokens")
+
+
+@pytest.mark.parametrize("rule", ["envelope", "centroid"])
 @pytest.mark.parametrize("name", ["ps16_topk", "ps16_new_page", "ps64_g7", "chunks_topk", "chunks_tokens"])
 def test_step_append(cuda_dev, R, rule, name):
     """The step that stores the newest token's key and value itself equals
