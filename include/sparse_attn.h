@@ -191,7 +191,10 @@ sa_status sparse_attn_decode(const sa_kv_desc* kv, const void* q, int32_t n_q_he
  * as soon as its selection is written, while other units are still being
  * scored; a decode item waits for its selection with a bounded wait (about a
  * second; SA_ERR_TIMEOUT when it runs out).  Needs B * n_kv_heads <= 32768 and
- * the workspace sized by sparse_attn_workspace_size. */
+ * the workspace sized by sparse_attn_workspace_size.  out (and lse) may lie in
+ * device memory or in pinned host memory, which the device addresses directly
+ * under unified addressing: the result then crosses PCIe while the launch
+ * runs, each unit's rows as its attention completes. */
 sa_status sparse_attn_decode_step(const sa_kv_desc* kv, void* meta, sa_score_rule rule,
                                   const void* q, int32_t n_q_heads, const sa_budget* budget,
                                   int32_t max_sel, float scale, int32_t* sel_idx,

@@ -169,6 +169,27 @@ def test_step_append(cuda_dev, R, rule, name):
     assert torch.equal(bf["lse"], ref["lse"]) and torch.equal(bf["sel_idx"], ref["sel_idx"])
 
 
+def test_step_output_to_pinned_host_memory(cuda_dev, R):
+    """The step may write its result straight into pinned host memory (which
+    the device reaches under unified addressing): the same bits as a device
+    output, with the device status clear."""
+    import block_sparse_kv_page_b200 as sa
+    lay, ps, bd = _case(cuda_dev, "ps16_topk")
+    ref = R.run_step(lay, page_size=ps, rule="envelope", budget=bd, scale=SCALE, stale=True)
+    assert ref["status"] == 0
+    B, Hkv = lay.k.shape[:2]
+    Hq = lay.q.shape[1]
+    sel = torch.full((B, Hkv, ref["max_sel"]), -7, dtype=torch.int32, device=cuda_dev)
+    cnt = torch.full((B, Hkv), -7, dtype=torch.int32, device=cuda_dev)
+    out_h = torch.full((B, Hq, 128), float("nan"), dtype=torch.float32).pin_memory()
+    sa.sparse_attn_decode_step(ref["kv"], ref["meta"], "envelope", lay.q, R.budget_struct(bd), ref["max_sel"],
+                               SCALE, sel, cnt, out_h, None, ref["ws"])
+    torch.cuda.synchronize()
+    assert sa.sparse_attn_get_device_status(ref["ws"]) == 0
+    assert torch.equal(out_h, ref["out"])
+    assert torch.equal(sel.cpu(), ref["sel_idx"]) and torch.equal(cnt.cpu(), ref["sel_count"])
+
+
 def test_step_repeat_and_interleave(cuda_dev, R):
     """Calls in a row on one workspace: the step leaves its flags, counters
     and queue cleared, also around the other calls."""
