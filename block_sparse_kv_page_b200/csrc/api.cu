@@ -118,8 +118,8 @@ int score_stride(const sa_kv_desc* kv) { return (kv->max_pages + 3) & ~3; }
 
 // Decode router scratch after the scores: lists [units][W], sigma (double)
 // and eligible counts per unit.
-size_t route_decode_ws_bytes(long long units, int W) {
-  return align256((size_t)units * W * 4) + align256((size_t)units * 8) + align256((size_t)units * 4);
+size_t route_decode_ws_bytes(long long units) {
+  return align256((size_t)units * 8) + align256((size_t)units * 4);
 }
 
 size_t select_scratch(const sa_kv_desc* kv, bool per_head = false, int n_q_heads = 0) {
@@ -395,7 +395,7 @@ size_t sparse_attn_workspace_size(const sa_kv_desc* kv, int32_t n_q_heads, int32
   const size_t rt = route_ws_bytes(route_tiles, kv->n_kv_heads, kv->max_pages, max_sel);
   if (rt > tail) tail = rt;
   if (kv->batch <= kMaxRouteTiles && kv->page_size > 0) {  // decode router: scores + router scratch
-    const size_t rd = select_scratch(kv) + route_decode_ws_bytes(kv->batch * kv->n_kv_heads, max_sel);
+    const size_t rd = select_scratch(kv) + route_decode_ws_bytes(kv->batch * kv->n_kv_heads);
     if (rd > tail) tail = rd;
   }
   return kScratch + tail;
@@ -696,9 +696,8 @@ sa_status sparse_attn_route(const sa_kv_desc* kv, const void* meta, sa_score_rul
   a.ws_keys = reinterpret_cast<uint32_t*>(scratch);
   a.dec_scores = nullptr;  // query tiles: the keys above, not decode group scores
   a.dec_stride = 0;
-  a.ws_list = reinterpret_cast<int32_t*>(scratch + keys_bytes);
-  a.ws_sigma = reinterpret_cast<double*>(scratch + keys_bytes + align256(tg * W * 4));
-  a.ws_elig = reinterpret_cast<int32_t*>(scratch + keys_bytes + align256(tg * W * 4) + align256(tg * 8));
+  a.ws_sigma = reinterpret_cast<double*>(scratch + keys_bytes);
+  a.ws_elig = reinterpret_cast<int32_t*>(scratch + keys_bytes + align256(tg * 8));
   a.ws_count = reinterpret_cast<uint32_t*>(reinterpret_cast<char*>(ws) + 256);
   a.ws_final = reinterpret_cast<uint32_t*>(reinterpret_cast<char*>(ws) + kQueueRoute);
   a.status = reinterpret_cast<int*>(ws);
@@ -733,7 +732,7 @@ sa_status sparse_attn_route_decode(const sa_kv_desc* kv, const void* meta, sa_sc
   if (s != SA_OK) return s;
   const long long units = (long long)kv->batch * kv->n_kv_heads;
   const size_t sel_bytes = select_scratch(kv);
-  const size_t need = kScratch + sel_bytes + route_decode_ws_bytes(units, (int)W);
+  const size_t need = kScratch + sel_bytes + route_decode_ws_bytes(units);
   if ((s = check_ws(ws, ws_bytes, need)) != SA_OK) return s;
   if (route_decode_smem_bytes(kv->max_pages, (int)W, k, kv->batch) > 227 * 1024) return SA_ERR_UNSUPPORTED;
   SelectArgs sa_{};  // every field zero unless set below
@@ -770,9 +769,8 @@ sa_status sparse_attn_route_decode(const sa_kv_desc* kv, const void* meta, sa_sc
   a.dec_scores = sa_.ws_scores;
   a.dec_stride = score_stride(kv);
   char* rbase = reinterpret_cast<char*>(ws) + kScratch + sel_bytes;
-  a.ws_list = reinterpret_cast<int32_t*>(rbase);
-  a.ws_sigma = reinterpret_cast<double*>(rbase + align256((size_t)units * W * 4));
-  a.ws_elig = reinterpret_cast<int32_t*>(rbase + align256((size_t)units * W * 4) + align256((size_t)units * 8));
+  a.ws_sigma = reinterpret_cast<double*>(rbase);
+  a.ws_elig = reinterpret_cast<int32_t*>(rbase + align256((size_t)units * 8));
   a.ws_count = reinterpret_cast<uint32_t*>(reinterpret_cast<char*>(ws) + 256);
   a.ws_final = reinterpret_cast<uint32_t*>(reinterpret_cast<char*>(ws) + kQueueRoute);
   a.status = reinterpret_cast<int*>(ws);

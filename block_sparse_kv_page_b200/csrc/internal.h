@@ -216,7 +216,6 @@ struct RouteArgs {
   uint32_t* ws_keys;          // [n_tiles][Hkv][max_pages] tile-score keys (zeroed before launch)
   const float* dec_scores;    // decode router: group scores [B*Hkv][dec_stride] (the tiles are
   int dec_stride;             // the sequences, one query row each); null for query tiles
-  int32_t* ws_list;           // [n_tiles][Hkv][W] rank-ordered lists
   double* ws_sigma;           // [n_tiles][Hkv]
   int32_t* ws_elig;           // [n_tiles][Hkv] eligible block counts
   uint32_t* ws_count;         // [n_tiles * Hkv] split counters (left zero)

@@ -188,9 +188,12 @@ SA_DEV void route_select_tile(const RouteArgs& a, int t, int g, int E, unsigned 
     a.sigma[tg] = (float)sg;
     a.ws_elig[tg] = E;
   }
-  int32_t* lst = a.ws_list + (size_t)tg * a.W;
+  // the list as if the tile triggers (the top rho k, -1 past the eligible
+  // blocks); the finalize trims the tiles that do not trigger to k
+  int32_t* lst = a.kv_idx + (size_t)tg * a.W;
   for (int i = tid; i < a.W; i += blockDim.x)
     lst[i] = i < n_sel ? (int32_t)(0xffffffffu - (uint32_t)(cand[i] & 0xffffffffu)) : -1;
+  if (tid == 0) a.kv_count[tg] = min(a.W, E);
 }
 
 // ---------------------------------------------------------------- finalize (one CTA)
@@ -229,30 +232,17 @@ SA_DEV void route_finalize(const RouteArgs& a, unsigned char* smem) {
   }
   __syncthreads();
   const double tau = s_tau;
-  for (int tg = tid; tg < T * Hkv; tg += blockDim.x) {
-    const int t = tg / Hkv;
-    const bool trig = sbar[t] < tau;
-    if (tg % Hkv == 0) a.triggered[t] = trig ? 1 : 0;
-    const int E = __ldcg(a.ws_elig + tg);
-    a.kv_count[tg] = min(trig ? a.W : a.k, E);
-  }
-  // the lists, every (tile, head, entry) by its own thread: independent loads
-  const int total = T * Hkv * a.W;
-  for (int b = 0; b < total; b += 8 * (int)blockDim.x) {  // 8 loads in flight per thread
-    int32_t v[8], ne[8];
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      const int x = b + j * (int)blockDim.x + tid;
-      v[j] = x < total ? __ldcg(a.ws_list + x) : -1;
-      ne[j] = x < total ? __ldcg(a.ws_elig + x / a.W) : 0;
-    }
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      const int x = b + j * (int)blockDim.x + tid;
-      if (x >= total) continue;
-      const int tg = x / a.W, i = x - tg * a.W;
-      const int n = min(sbar[tg / Hkv] < tau ? a.W : a.k, ne[j]);
-      a.kv_idx[x] = i < n ? v[j] : -1;
+  for (int t = tid; t < T; t += blockDim.x) a.triggered[t] = sbar[t] < tau ? 1 : 0;
+  // the selecting CTAs wrote every list as if its tile triggered: trim the
+  // others to their top k (entries k .. W - 1 become sentinels), one thread
+  // per (tile, head, entry) past k
+  if (a.W > a.k) {
+    const int tail = a.W - a.k;
+    for (int x = tid; x < T * Hkv * tail; x += blockDim.x) {
+      const int tg = x / tail, i = a.k + (x - tg * tail);
+      if (sbar[tg / Hkv] < tau) continue;
+      a.kv_idx[(size_t)tg * a.W + i] = -1;
+      if (i == a.k) a.kv_count[tg] = min(a.k, __ldcg(a.ws_elig + tg));
     }
   }
 }
@@ -770,7 +760,7 @@ int route_splits(int vectors_per_tile) { return (vectors_per_tile + kRtVecs - 1)
 size_t route_ws_bytes(int n_tiles, int Hkv, int max_pages, int W) {
   auto al = [](size_t x) { return (x + 255) & ~(size_t)255; };
   const size_t tg = (size_t)n_tiles * Hkv;
-  return al(tg * max_pages * 4) + al(tg * W * 4) + al(tg * 8) + al(tg * 4);
+  return al(tg * max_pages * 4) + al(tg * 8) + al(tg * 4);
 }
 
 size_t route_decode_smem_bytes(int max_pages, int W, int k, int n_tiles) {
