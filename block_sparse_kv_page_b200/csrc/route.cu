@@ -234,15 +234,18 @@ SA_DEV void route_finalize(const RouteArgs& a, unsigned char* smem) {
   const double tau = s_tau;
   for (int t = tid; t < T; t += blockDim.x) a.triggered[t] = sbar[t] < tau ? 1 : 0;
   // the selecting CTAs wrote every list as if its tile triggered: trim the
-  // others to their top k (entries k .. W - 1 become sentinels), one thread
-  // per (tile, head, entry) past k
+  // others to their top k (entries k .. W - 1 become sentinels), a warp per
+  // tile, lanes along the entries
   if (a.W > a.k) {
-    const int tail = a.W - a.k;
-    for (int x = tid; x < T * Hkv * tail; x += blockDim.x) {
-      const int tg = x / tail, i = a.k + (x - tg * tail);
-      if (sbar[tg / Hkv] < tau) continue;
-      a.kv_idx[(size_t)tg * a.W + i] = -1;
-      if (i == a.k) a.kv_count[tg] = min(a.k, __ldcg(a.ws_elig + tg));
+    const int lane = tid & 31, nw = blockDim.x >> 5;
+    for (int t = tid >> 5; t < T; t += nw) {  // warp per tile
+      if (sbar[t] < tau) continue;
+      for (int g = 0; g < Hkv; ++g) {
+        const int tg = t * Hkv + g;
+        int32_t* row = a.kv_idx + (size_t)tg * a.W;
+        for (int i = a.k + lane; i < a.W; i += 32) row[i] = -1;
+        if (lane == 0) a.kv_count[tg] = min(a.k, __ldcg(a.ws_elig + tg));
+      }
     }
   }
 }
