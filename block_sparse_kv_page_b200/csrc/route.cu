@@ -158,8 +158,13 @@ SA_DEV void route_select_tile(const RouteArgs& a, int t, int g, int E, unsigned 
   while (n2 < n_sel) n2 <<= 1;
   for (int i = n_sel + tid; i < n2; i += blockDim.x) cand[i] = 0ull;
   __syncthreads();
+  // Strides of 32 and up pair elements of different warps (shared memory, a
+  // barrier each); the strides below 32 of one size run in registers, a warp
+  // per 32 consecutive elements exchanging by shuffles, then one barrier.
+  const int lane = tid & 31, nw = (int)blockDim.x >> 5;
   for (int size = 2; size <= n2; size <<= 1) {
-    for (int stride = size >> 1; stride > 0; stride >>= 1) {
+    int stride = size >> 1;
+    for (; stride >= 32; stride >>= 1) {
       for (int i = tid; i < n2; i += blockDim.x) {
         const int j = i ^ stride;
         if (j > i) {
@@ -173,6 +178,18 @@ SA_DEV void route_select_tile(const RouteArgs& a, int t, int g, int E, unsigned 
       }
       __syncthreads();
     }
+    for (int r = tid >> 5; 32 * r < n2; r += nw) {
+      const int e = 32 * r + lane;
+      unsigned long long v = e < n2 ? cand[e] : 0ull;
+      const bool desc = (e & size) == 0;
+      for (int st = stride; st > 0; st >>= 1) {
+        const unsigned long long w = __shfl_xor_sync(0xffffffffu, v, st);
+        // the lower index of a pair keeps the larger value when descending
+        v = (((e & st) == 0) == desc) ? (v > w ? v : w) : (v < w ? v : w);
+      }
+      if (e < n2) cand[e] = v;
+    }
+    __syncthreads();
   }
   if (tid == 0) {
     double sg;
