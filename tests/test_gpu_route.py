@@ -27,6 +27,7 @@ def _small(dev, N, rows, seed):
     (2048, 96, 32, 4, 3, 0.25),      # 3 tiles, one split
     (1024, 64, 64, 16, 1, 0.25),     # rho = 1: lists are plain top-k
     (640, 128, 64, 12, 2, 1.0),      # few eligible blocks (E near k), quantile 1
+    (4096, 256, 64, 8, 2, 0.0),      # quantile 0: no tile triggers, every list is trimmed to k
 ])
 def test_route_small(cuda_dev, H, rule, N, rows, tile_rows, k, rho, q):
     lay = _small(cuda_dev, N, rows, seed=7000 + N + rows)

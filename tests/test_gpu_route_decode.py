@@ -95,6 +95,7 @@ def _check_attention(H, lay, g_res, ps):
     (16, 16, 2, 0.5, 0.3),
     (16, 12, 1, 0.25, None),
     (64, 4, 3, 0.75, None),
+    (16, 16, 2, 0.0, None),          # no sequence triggers: every list trimmed to k
 ])
 def test_route_decode_parity(cuda_dev, H, rule, ps, k, rho, quantile, tau):
     import block_sparse_kv_page_b200 as sa
