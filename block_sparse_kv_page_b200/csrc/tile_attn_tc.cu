@@ -12,13 +12,14 @@
 // Warp-specialised, all waits bounded:
 //   warp 8 (one thread)  streams each kept block (64 keys) of K and V by TMA
 //                        into a kStages ring (four 64-row x 128 B boxes);
-//   warp 9 (one thread)  issues, for each Q tile t and block i,
+//   warp 9 + t (one thread) issues, for Q tile t and block i in order,
 //                        S = Q_t K_i^T (M = 128 vectors, N = 64 keys, K = 128
 //                        dims; K-major operands) into one of the tile's two
-//                        S/P buffers, and O_t += [P_hi | P_lo] . [V_i ; V_i]
-//                        (A = P read from tensor memory, N = 128 dims,
-//                        K = 2 x 64 keys; V read MN-major); it polls both
-//                        tiles' queues, so one tile's softmax and handoffs
+//                        S/P buffers, then O_t += [P_hi | P_lo] . [V_{i-1} ;
+//                        V_{i-1}] (A = P read from tensor memory, N = 128
+//                        dims, K = 2 x 64 keys; V read MN-major) once
+//                        P_{i-1} is written; the tensor pipe interleaves the
+//                        two tiles' MMAs, so one tile's softmax and handoffs
 //                        overlap the other tile's MMAs;
 //   warps 0-3 / 4-7      the softmax of tile 0 / 1: thread = query vector
 //                        (TMEM lane 32 (warp % 4) + lane), its whole row of
@@ -42,9 +43,9 @@ namespace {
 constexpr int kBlk = 64;                       // keys per block
 constexpr int kTiles = 2;                      // Q tiles of 128 vectors per CTA
 constexpr int kSmWarps = 4 * kTiles;           // softmax: one warp per TMEM lane quarter and tile
-constexpr int kThreadsTc = 32 * (kSmWarps + 2);
+constexpr int kThreadsTc = 32 * (kSmWarps + 1 + kTiles);
 constexpr int kProducerWarp = kSmWarps;
-constexpr int kMmaWarp = kSmWarps + 1;
+constexpr int kMmaWarp0 = kSmWarps + 1;        // warp kMmaWarp0 + t issues tile t's MMAs
 #ifndef SA_TA_STAGES
 #define SA_TA_STAGES 3
 #endif
@@ -138,14 +139,14 @@ __global__ void __launch_bounds__(kThreadsTc, 1) tile_attn_tc_kernel(const __gri
   if (tid == 0) {
     for (int s = 0; s < kStages; ++s) {
       mbar_init(kv_full + s, 1);
-      mbar_init(kv_empty + s, 1);
+      mbar_init(kv_empty + s, kTiles);  // each tile's MMA thread commits after its PV
     }
     for (int x = 0; x < 2 * kTiles; ++x) {
       mbar_init(s_full + x, 1);
       mbar_init(p_full + x, 4);  // the tile's four softmax warps
       mbar_init(o_full + x, 1);
     }
-    mbar_init(drain, 1);
+    mbar_init(drain, kTiles);
     fence_barrier_init();
     prefetch_tmap(&a.tmap_k);
     prefetch_tmap(&a.tmap_v);
@@ -235,19 +236,40 @@ __global__ void __launch_bounds__(kThreadsTc, 1) tile_attn_tc_kernel(const __gri
       for (int i = max(0, issued - kStages); i < issued; ++i)
         mbar_wait(kv_full + (i % kStages), (i / kStages) & 1u, nullptr);
     }
-  } else if (warp == kMmaWarp) {
-    // ---- MMA issuer.  Per tile: QK of block i needs its K/V stage and a free
-    // S/P buffer (the PV of block i - 2 issued before it); PV of block i needs
-    // P_i.  Both tiles' queues are polled without blocking and whatever is
-    // ready goes first; the K/V stage is released after the second of the two
-    // PVs that read it.
+  } else if (warp >= kMmaWarp0) {
+    // ---- MMA issuer of tile tt, in order: QK of block i (its K/V stage
+    // landed; its S/P buffer was last read by the PV of block i - 2, issued
+    // before), then the PV of block i - 1 once P_{i-1} is written.  One thread
+    // per tile: an MMA issue returns about when the tensor pipe has taken the
+    // MMAs, so a single thread serving both tiles held each tile's PV behind
+    // the other tile's QKs; the pipe interleaves the two threads' MMAs.  A K/V
+    // stage is free once both tiles' PVs that read it are done.
+    const int tt = warp - kMmaWarp0;
     if (lane == 0) {
       const uint32_t idesc_s = tc::idesc_f32acc(tc::kFmtBF16, 128, kBlk);
       const uint32_t idesc_o = tc::idesc_f32acc(tc::kFmtBF16, 128, kHeadDim) | (1u << 16);  // V MN-major
-      auto qk = [&](int tt, int i) {
+      const unsigned char* qt = qs + tt * kQTile;
+      auto pv = [&](int i) -> bool {
         const int s = i % kStages, b = i & 1;
+        if (!mbar_wait(p_full + 2 * tt + b, (i >> 1) & 1u, a.status)) return false;
+        tc::fence_after_sync();
+        const unsigned char* vb = ring + s * kStage + 2 * kBox;
+#pragma unroll
+        for (int j = 0; j < 8; ++j)  // K = [P_hi keys 0-63 | P_lo keys 0-63], 16 per step
+          tc::mma_bf16_ts(tmem + kColO + 128u * tt, tmem + kColSP + 128u * tt + 64u * b + 8u * j,
+                          v_desc(vb + 16 * 128 * (j & 3)), idesc_o, i > 0 || j != 0);
+        tc::commit(o_full + 2 * tt + b);
+        tc::commit(kv_empty + s);
+        return true;
+      };
+      for (int i = 0; i < nb && !fail; ++i) {
+        const int s = i % kStages, b = i & 1;
+        if (!mbar_wait(kv_full + s, (i / kStages) & 1u, a.status)) {
+          fail = 1;
+          break;
+        }
+        tc::fence_after_sync();
         const unsigned char* kb = ring + s * kStage;
-        const unsigned char* qt = qs + tt * kQTile;
 #pragma unroll
         for (int c = 0; c < 2; ++c)
 #pragma unroll
@@ -255,46 +277,9 @@ __global__ void __launch_bounds__(kThreadsTc, 1) tile_attn_tc_kernel(const __gri
             tc::mma_bf16_ss(tmem + kColSP + 128u * tt + 64u * b, tc::smem_desc_sw128(qt + c * (128 * 128) + 32 * k),
                             tc::smem_desc_sw128(kb + c * kBox + 32 * k), idesc_s, (c | k) != 0);
         tc::commit(s_full + 2 * tt + b);
-      };
-      auto pv = [&](int tt, int i) {
-        const int s = i % kStages, b = i & 1;
-        const unsigned char* vb = ring + s * kStage + 2 * kBox;
-#pragma unroll
-        for (int j = 0; j < 8; ++j)  // K = [P_hi keys 0-63 | P_lo keys 0-63], 16 per step
-          tc::mma_bf16_ts(tmem + kColO + 128u * tt, tmem + kColSP + 128u * tt + 64u * b + 8u * j,
-                          v_desc(vb + 16 * 128 * (j & 3)), idesc_o, i > 0 || j != 0);
-        tc::commit(o_full + 2 * tt + b);
-      };
-      int nq[kTiles] = {0, 0}, npv[kTiles] = {0, 0};
-      uint32_t idle = 0;
-      while (npv[0] < nb || npv[1] < nb) {
-        bool progress = false;
-#pragma unroll
-        for (int tt = 0; tt < kTiles; ++tt) {
-          const int q = nq[tt];
-          if (q < nb && q < npv[tt] + 2 && mbar_test(kv_full + q % kStages, (q / kStages) & 1u)) {
-            tc::fence_after_sync();
-            qk(tt, q);
-            nq[tt] = q + 1;
-            progress = true;
-          }
-          const int p = npv[tt];
-          if (p < nq[tt] && mbar_test(p_full + 2 * tt + (p & 1), (p >> 1) & 1u)) {
-            tc::fence_after_sync();
-            pv(tt, p);
-            if (npv[tt ^ 1] > p) tc::commit(kv_empty + p % kStages);  // the other tile's PV of p is issued
-            npv[tt] = p + 1;
-            progress = true;
-          }
-        }
-        if (progress) {
-          idle = 0;
-        } else if (++idle >= kSpinLimit) {
-          flag_status(a.status, SA_ERR_TIMEOUT);
-          fail = 1;
-          break;
-        }
+        if (i > 0 && !pv(i - 1)) fail = 1;
       }
+      if (!fail && nb > 0 && !pv(nb - 1)) fail = 1;
       // every MMA issued has completed before TMEM is freed (bounded)
       tc::commit(drain);
       mbar_wait(drain, 0, nullptr);
