@@ -74,6 +74,21 @@ def test_tile_attention_on_routed_lists(cuda_dev, rule):
     assert _check(lay, out, lse, kv_idx, tile_rows=64) < 1e-4
 
 
+@pytest.mark.parametrize("tile_rows", [32, 128])
+def test_tile_attention_other_tile_heights(cuda_dev, tile_rows):
+    """Tiles of 32 rows (224 query vectors: one CTA, its second Q tile partly
+    empty) and 128 rows (896 vectors: four CTAs) on router lists."""
+    import router_harness as H
+    lay = DG.make_router_layer(Hq=28, Hkv=4, N=4096, rows=256, seed=7600 + tile_rows, device=cuda_dev)
+    g = H.run_route_gpu(lay.k, lay.q, rule="envelope", block=64, q_pos0=lay.q_pos0, tile_rows=tile_rows,
+                        k=8, rho=2, quantile=0.25)
+    kv_idx = torch.from_numpy(g["kv_idx"]).to(cuda_dev)
+    kv_count = torch.from_numpy(g["kv_count"]).to(cuda_dev)
+    out, lse, status = _tile_attn_gpu(lay, kv_idx, kv_count, tile_rows=tile_rows)
+    assert status == 0
+    assert _check(lay, out, lse, kv_idx, tile_rows=tile_rows) < 1e-4
+
+
 def test_tile_attention_ragged_and_sentinels(cuda_dev):
     """Partial last block (N = 4000), a ragged last tile (200 rows, tiles of
     64), lists with sentinels in the middle, an empty list, and the diagonal
