@@ -381,8 +381,13 @@ __global__ void __launch_bounds__(kTcThreads, 1) route_tc_kernel(const __grid_co
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int Hkv = a.kv.Hkv;
-  const int sp = blockIdx.x % a.nsplit;
-  const int tg = blockIdx.x / a.nsplit;
+  // CTA -> (split, tile, KV head), split-major: the first wave holds the
+  // first split of every (tile, KV head), so the selection that the last split
+  // of a pair runs falls at the end of its SM's work, not in front of a
+  // second-wave CTA
+  const int n_tg = a.n_tiles * a.kv.Hkv;
+  const int sp = blockIdx.x / n_tg;
+  const int tg = blockIdx.x % n_tg;
   const int t = tg / Hkv, g = tg % Hkv;
   const int N = a.kv.seq_len[0];
   const RouteGeom geo = route_geom(a, t, N);
@@ -579,8 +584,13 @@ __global__ void __launch_bounds__(kTcThreads, 1) route_tc_centroid_kernel(const 
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int Hkv = a.kv.Hkv;
-  const int sp = blockIdx.x % a.nsplit;
-  const int tg = blockIdx.x / a.nsplit;
+  // CTA -> (split, tile, KV head), split-major: the first wave holds the
+  // first split of every (tile, KV head), so the selection that the last split
+  // of a pair runs falls at the end of its SM's work, not in front of a
+  // second-wave CTA
+  const int n_tg = a.n_tiles * a.kv.Hkv;
+  const int sp = blockIdx.x / n_tg;
+  const int tg = blockIdx.x % n_tg;
   const int t = tg / Hkv, g = tg % Hkv;
   const int N = a.kv.seq_len[0];
   const RouteGeom geo = route_geom(a, t, N);
