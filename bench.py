@@ -70,6 +70,8 @@ def parse():
     ap.add_argument("--no-extra", action="store_true", help="skip the secondary modes/rules")
     ap.add_argument("--router-only", action="store_true",
                     help="time only the router workload (route + tile attention) and print its JSON")
+    ap.add_argument("--router-decode-only", action="store_true",
+                    help="print only the decode router leg's timings (headline workload)")
     ap.add_argument("--ratio-only", action="store_true",
                     help="print only the ratio-budget workload's timings")
     ap.add_argument("--tsa-only", action="store_true",
@@ -566,44 +568,8 @@ def run_gpu_arm(args, rank, world, dist):
         if sa.sparse_attn_get_device_status(ws_h) != 0:
             raise RuntimeError("per-head leg: device status set")
         del ws_h, sel_h, cnt_h
-        # the router applied to decode: each (layer) row is a one-row tile; top k pages,
-        # top 2k for the sequences whose sigma_bar falls below the 0.25 quantile
-        rho, W = 2, 2 * k
-        ws_r = sa.make_workspace(kv, HQ, L * B, W)
-        idx_r = torch.zeros((L * B, HKV, W), dtype=torch.int32, device=dev)
-        cnt_r = torch.zeros((L * B, HKV), dtype=torch.int32, device=dev)
-        sig_r = torch.zeros((L * B, HKV), dtype=torch.float32, device=dev)
-        sbar_r = torch.zeros((L * B,), dtype=torch.float32, device=dev)
-        trig_r = torch.zeros((L * B,), dtype=torch.uint8, device=dev)
-        for rule in ("envelope", "centroid"):
-            def routed_step():
-                sa.sparse_attn_build_meta(kv, rule, -1, metas[rule])
-                sa.sparse_attn_route_decode(kv, metas[rule], rule, inp["q"], k, rho, 0.25, None, idx_r, cnt_r,
-                                            sig_r, sbar_r, trig_r, None, ws_r)
-                sa.sparse_attn_decode(kv, inp["q"], L * B, 0, 1, scale, idx_r, cnt_r, W, out, lse, ws_r)
-            for _ in range(max(3, args.warmup)):
-                routed_step()
-            barrier()
-            e0 = torch.cuda.Event(enable_timing=True)
-            e1 = torch.cuda.Event(enable_timing=True)
-            n_rep = max(10, args.steps // 2)
-            e0.record(stream)
-            for _ in range(n_rep):
-                routed_step()
-            e1.record(stream)
-            torch.cuda.synchronize()
-            m2 = max_over_ranks(e0.elapsed_time(e1) / n_rep, dist, dev)
-            kept = int(cnt_r.sum().item())
-            kv_r = kept * PS * 2 * D * 2
-            extra[f"router-decode/{rule}"] = {
-                "ms_per_step": round(m2, 4), "value": kept * PS * (HQ // HKV) * world / (m2 * 1e-3),
-                "eff_GBps": (meta_bytes + kv_r) / (m2 * 1e-3) / 1e9,
-                "triggered_rows": int(trig_r.sum().item()), "pages_kept_per_unit": round(kept / (L * B * HKV), 1),
-                "note": "three launches per step (metadata refresh; score-only pass + router selection; decode "
-                        "over the routed lists); k = 256 pages, rho = 2, quantile 0.25 over the 48 rows"}
-        if sa.sparse_attn_get_device_status(ws_r) != 0:
-            raise RuntimeError("router-decode leg: device status set")
-        del ws_r, idx_r, cnt_r, sig_r, sbar_r, trig_r
+        extra.update(router_decode_leg(torch, dev, sa, kv, inp, metas, out, lse, k, scale,
+                                       max(10, args.steps // 2), max(3, args.warmup), dist, world))
     for g in graphs.values():
         del g
     graphs.clear()
@@ -617,6 +583,62 @@ def run_gpu_arm(args, rank, world, dist):
                 e2e_zc=e2e_zc, h2d=h2d,
                 d2h=d2h, meta_bytes=meta_bytes, kv_bytes=kv_bytes, extra=extra, router=router, tsa=tsa, ratio=ratio,
                 launches_per_step=MODES[args.mode])
+
+
+def router_decode_leg(torch, dev, sa, kv, inp, metas, out, lse, k: int, scale: float, steps: int, warmup: int,
+                      dist, world: int):
+    """The uncertainty router applied to decode on the headline workload: each
+    (layer) row is a one-row tile; metadata refresh, the router call and the
+    decode over the routed lists per step."""
+    stream = torch.cuda.current_stream()
+    L = LAYERS
+    meta_bytes = L * B * HKV * (N // PS) * 512
+
+    def barrier():
+        if dist is not None:
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    res = {}
+    # the router applied to decode: each (layer) row is a one-row tile; top k pages,
+    # top 2k for the sequences whose sigma_bar falls below the 0.25 quantile
+    rho, W = 2, 2 * k
+    ws_r = sa.make_workspace(kv, HQ, L * B, W)
+    idx_r = torch.zeros((L * B, HKV, W), dtype=torch.int32, device=dev)
+    cnt_r = torch.zeros((L * B, HKV), dtype=torch.int32, device=dev)
+    sig_r = torch.zeros((L * B, HKV), dtype=torch.float32, device=dev)
+    sbar_r = torch.zeros((L * B,), dtype=torch.float32, device=dev)
+    trig_r = torch.zeros((L * B,), dtype=torch.uint8, device=dev)
+    for rule in ("envelope", "centroid"):
+        def routed_step():
+            sa.sparse_attn_build_meta(kv, rule, -1, metas[rule])
+            sa.sparse_attn_route_decode(kv, metas[rule], rule, inp["q"], k, rho, 0.25, None, idx_r, cnt_r,
+                                        sig_r, sbar_r, trig_r, None, ws_r)
+            sa.sparse_attn_decode(kv, inp["q"], L * B, 0, 1, scale, idx_r, cnt_r, W, out, lse, ws_r)
+        for _ in range(warmup):
+            routed_step()
+        barrier()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        n_rep = steps
+        e0.record(stream)
+        for _ in range(n_rep):
+            routed_step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        m2 = max_over_ranks(e0.elapsed_time(e1) / n_rep, dist, dev)
+        kept = int(cnt_r.sum().item())
+        kv_r = kept * PS * 2 * D * 2
+        res[f"router-decode/{rule}"] = {
+            "ms_per_step": round(m2, 4), "value": kept * PS * (HQ // HKV) * world / (m2 * 1e-3),
+            "eff_GBps": (meta_bytes + kv_r) / (m2 * 1e-3) / 1e9,
+            "triggered_rows": int(trig_r.sum().item()), "pages_kept_per_unit": round(kept / (L * B * HKV), 1),
+            "note": "three launches per step (metadata refresh; score-only pass + router selection; decode "
+                    "over the routed lists); k = 256 pages, rho = 2, quantile 0.25 over the 48 rows"}
+    if sa.sparse_attn_get_device_status(ws_r) != 0:
+        raise RuntimeError("router-decode leg: device status set")
+    del ws_r, idx_r, cnt_r, sig_r, sbar_r, trig_r
+    return res
 
 
 def router_leg(torch, dev, steps: int, warmup: int):
@@ -917,6 +939,22 @@ def main():
         torch.cuda.set_device(dev)
         if rank == 0:
             print(json.dumps({"tsa": tsa_leg(torch, dev, args.steps, max(3, args.warmup))}))
+        return 0
+    if args.router_decode_only:
+        import block_sparse_kv_page_b200 as sa
+        dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", 0)))
+        torch.cuda.set_device(dev)
+        inp = build_inputs(torch, dev, rank, "envelope")
+        kv = inp["kv"]
+        metas = {r: kv.meta_buffer() for r in ("envelope", "centroid")}
+        for r_, m_ in metas.items():
+            sa.sparse_attn_build_meta(kv, r_, 0, m_)
+        out = torch.zeros((LAYERS * B, HQ, D), dtype=torch.float32, device=dev)
+        lse = torch.zeros((LAYERS * B, HQ), dtype=torch.float32, device=dev)
+        res = router_decode_leg(torch, dev, sa, kv, inp, metas, out, lse, args.budget // PS,
+                                1.0 / math.sqrt(D), args.steps, max(3, args.warmup), None, 1)
+        if rank == 0:
+            print(json.dumps({"router_decode": res}))
         return 0
     if args.router_only:
         dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", 0)))
