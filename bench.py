@@ -149,9 +149,10 @@ def cpu_oracle_time(rule: str, k: int, units: int, rounds: int = 1):
 
 
 # --------------------------------------------------------------------------- clocks
-def _clock_poller(index: int, go, stop, out_q):
-    """Child process: once `go` is set, poll NVML (SM clock, clock-event
-    reasons) every ~2 ms until `stop` is set, then send the samples back.
+def _clock_poller(index: int, tag, stop, out_q):
+    """Child process: while `tag` >= 0 (a timed region is open), poll NVML (SM
+    clock, clock-event reasons) about every 0.5 ms, recording the region's
+    tag with each sample, until `stop` is set; then send the samples back.
     Reads only."""
     samples = []
     try:
@@ -160,44 +161,73 @@ def _clock_poller(index: int, go, stop, out_q):
         h = nv.nvmlDeviceGetHandleByIndex(index)
         mx = nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM)
         out_q.put(("ready", mx))
-        while not go.is_set() and not stop.is_set():
-            time.sleep(0.001)
         while not stop.is_set():
-            samples.append((nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM),
-                            nv.nvmlDeviceGetCurrentClocksEventReasons(h)))
-            time.sleep(0.002)
+            t = tag.value
+            if t >= 0:
+                samples.append((t, nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM),
+                                nv.nvmlDeviceGetCurrentClocksEventReasons(h)))
+            time.sleep(0.0005)
     except Exception as e:  # no NVML: report nothing sampled
         out_q.put(("ready", None))
         out_q.put(("error", repr(e)))
     out_q.put(("samples", samples))
 
 
+_REASON_BITS = {
+    "gpu_idle": 0x1, "applications_clocks_setting": 0x2, "sw_power_cap": 0x4,
+    "hw_slowdown": 0x8, "sync_boost": 0x10, "sw_thermal_slowdown": 0x20,
+    "hw_thermal_slowdown": 0x40, "hw_power_brake_slowdown": 0x80,
+    "display_clock_setting": 0x100,
+}
+
+
 class ClockSampler:
-    """Samples the SM clock and clock-event reasons in a separate process
-    during the timed region (a thread would be starved by the launch loop)."""
+    """Samples the SM clock and clock-event reasons in a separate process (a
+    thread would be starved by the launch loop) during every timed region of
+    the run: `with sampler.region("name"):` around each timed loop.  The
+    summary covers all regions, with the headline region's own figures and
+    the sample count of every region."""
 
     def __init__(self, index: int):
         import multiprocessing as mp
         self.index = index
         self.samples = []
         self.max_mhz = None
+        self.tags = []
         self.ctx = mp.get_context("spawn")
-        self.go = self.ctx.Event()
+        self.tag = self.ctx.Value("i", -1, lock=False)
         self.stop = self.ctx.Event()
         self.q = self.ctx.Queue()
-        self.p = self.ctx.Process(target=_clock_poller, args=(index, self.go, self.stop, self.q), daemon=True)
+        self.p = self.ctx.Process(target=_clock_poller, args=(index, self.tag, self.stop, self.q), daemon=True)
         self.p.start()
+        self.closed = False
         try:
             tag, mx = self.q.get(timeout=60)
             self.max_mhz = mx
         except Exception:
             pass
 
-    def __enter__(self):
-        self.go.set()
-        return self
+    class _Region:
+        def __init__(self, outer, i):
+            self.outer, self.i = outer, i
 
-    def __exit__(self, *a):
+        def __enter__(self):
+            self.outer.tag.value = self.i
+            return self
+
+        def __exit__(self, *a):
+            self.outer.tag.value = -1
+
+    def region(self, name: str):
+        if name not in self.tags:
+            self.tags.append(name)
+        return ClockSampler._Region(self, self.tags.index(name))
+
+    def close(self):
+        if self.closed:
+            return
+        self.closed = True
+        self.tag.value = -1
         self.stop.set()
         try:
             while True:
@@ -209,22 +239,28 @@ class ClockSampler:
             pass
         self.p.join(timeout=10)
 
-    def summary(self):
-        if not self.samples:
-            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": ["unsampled"]}
-        names = {
-            "gpu_idle": 0x1, "applications_clocks_setting": 0x2, "sw_power_cap": 0x4,
-            "hw_slowdown": 0x8, "sync_boost": 0x10, "sw_thermal_slowdown": 0x20,
-            "hw_thermal_slowdown": 0x40, "hw_power_brake_slowdown": 0x80,
-            "display_clock_setting": 0x100,
-        }
+    @staticmethod
+    def _reasons(samples):
         seen = set()
-        for _, rs in self.samples:
-            for n, bit in names.items():
+        for _, _, rs in samples:
+            for n, bit in _REASON_BITS.items():
                 if rs & bit:
                     seen.add(n)
-        return {"sm_mhz": statistics.median(m for m, _ in self.samples), "sm_max_mhz": self.max_mhz,
-                "reasons": sorted(seen), "samples": len(self.samples)}
+        return sorted(seen)
+
+    def summary(self, headline: str = "headline"):
+        self.close()
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": ["unsampled"], "samples": 0}
+        hi = self.tags.index(headline) if headline in self.tags else -2
+        head = [x for x in self.samples if x[0] == hi]
+        per = {name: sum(1 for x in self.samples if x[0] == i) for i, name in enumerate(self.tags)}
+        return {"sm_mhz": statistics.median(m for _, m, _ in self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": self._reasons(self.samples), "samples": len(self.samples),
+                "scope": "every timed region of the run (headline, end-to-end and secondary legs)",
+                "headline": {"sm_mhz": statistics.median(m for _, m, _ in head) if head else None,
+                             "reasons": self._reasons(head), "samples": len(head)},
+                "samples_per_region": per}
 
 
 # --------------------------------------------------------------------------- multi-rank plumbing
@@ -285,6 +321,7 @@ def run_gpu_arm(args, rank, world, dist):
     import block_sparse_kv_page_b200 as sa
     dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", 0)))
     torch.cuda.set_device(dev)
+    clocks = ClockSampler(dev.index if dev.index is not None else 0)
     inp = build_inputs(torch, dev, rank, args.rule)
     kv = inp["kv"]
     k = args.budget // PS
@@ -357,7 +394,7 @@ def run_gpu_arm(args, rank, world, dist):
             dist.barrier()
         torch.cuda.synchronize()
 
-    def timed(mode, rule, steps, warmup, per_kernel=False, clocks=None):
+    def timed(mode, rule, steps, warmup, per_kernel=False, region=None):
         if mode in ("sequential", "step-seq"):
             g = seq_graph(mode, rule)
             fn = g.replay
@@ -375,8 +412,7 @@ def run_gpu_arm(args, rank, world, dist):
         barrier()
         t0 = torch.cuda.Event(enable_timing=True)
         t1 = torch.cuda.Event(enable_timing=True)
-        ctx = clocks if clocks is not None else _Null()
-        with ctx:
+        with clocks.region(region or f"{mode}/{rule}"):
             t0.record(stream)
             for i in range(steps):
                 if evs and mode == "step":
@@ -400,9 +436,8 @@ def run_gpu_arm(args, rank, world, dist):
     # step is that kernel's duration plus any gap, so it serves as the
     # kernel's time too.  The three-launch mode records events around each
     # kernel to split the step.
-    clocks = ClockSampler(dev.index if dev.index is not None else 0)
     ms, kern = timed(args.mode, args.rule, args.steps, args.warmup,
-                     per_kernel=args.mode == "batched", clocks=clocks)
+                     per_kernel=args.mode == "batched", region="headline")
     status = sa.sparse_attn_get_device_status(ws)
     if status != 0:
         raise RuntimeError(f"device status {status} after the timed steps")
@@ -452,11 +487,12 @@ def run_gpu_arm(args, rank, world, dist):
     barrier()
     a0 = torch.cuda.Event(enable_timing=True)
     a1 = torch.cuda.Event(enable_timing=True)
-    a0.record(stream)
-    for _ in range(args.steps):
-        e2e_step()
-    a1.record(stream)
-    torch.cuda.synchronize()
+    with clocks.region("e2e"):
+        a0.record(stream)
+        for _ in range(args.steps):
+            e2e_step()
+        a1.record(stream)
+        torch.cuda.synchronize()
     e2e_ms = max_over_ranks(a0.elapsed_time(a1) / args.steps, dist, dev)
     h2d = host_in.numel() * host_in.element_size()
     d2h = out_h.numel() * 4
@@ -477,11 +513,12 @@ def run_gpu_arm(args, rank, world, dist):
         for _ in range(args.warmup):
             e2e_bf16_step()
         barrier()
-        a0.record(stream)
-        for _ in range(args.steps):
-            e2e_bf16_step()
-        a1.record(stream)
-        torch.cuda.synchronize()
+        with clocks.region("e2e-bf16"):
+            a0.record(stream)
+            for _ in range(args.steps):
+                e2e_bf16_step()
+            a1.record(stream)
+            torch.cuda.synchronize()
         ms_bf = max_over_ranks(a0.elapsed_time(a1) / args.steps, dist, dev)
         e2e_bf16 = {"ms_per_step": round(ms_bf, 5), "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": out_h.numel() * 2}
@@ -501,11 +538,12 @@ def run_gpu_arm(args, rank, world, dist):
         for _ in range(args.warmup):
             e2e_zc_step()
         barrier()
-        a0.record(stream)
-        for _ in range(args.steps):
-            e2e_zc_step()
-        a1.record(stream)
-        torch.cuda.synchronize()
+        with clocks.region("e2e-host-out"):
+            a0.record(stream)
+            for _ in range(args.steps):
+                e2e_zc_step()
+            a1.record(stream)
+            torch.cuda.synchronize()
         ms_zc = max_over_ranks(a0.elapsed_time(a1) / args.steps, dist, dev)
         e2e_step()  # the copy-based path once more on the same inputs: both results must agree exactly
         torch.cuda.synchronize()
@@ -549,11 +587,12 @@ def run_gpu_arm(args, rank, world, dist):
                 e0 = torch.cuda.Event(enable_timing=True)
                 e1 = torch.cuda.Event(enable_timing=True)
                 n_rep = max(10, args.steps // 2)
-                e0.record(stream)
-                for _ in range(n_rep):
-                    fn()
-                e1.record(stream)
-                torch.cuda.synchronize()
+                with clocks.region(f"{label}/{rule}"):
+                    e0.record(stream)
+                    for _ in range(n_rep):
+                        fn()
+                    e1.record(stream)
+                    torch.cuda.synchronize()
                 m2 = max_over_ranks(e0.elapsed_time(e1) / n_rep, dist, dev)
                 # K/V of the distinct pages the G heads of a KV head keep (the union)
                 sh = sel_h.view(L * B, HKV, HQ // HKV, k).cpu()
@@ -569,16 +608,16 @@ def run_gpu_arm(args, rank, world, dist):
             raise RuntimeError("per-head leg: device status set")
         del ws_h, sel_h, cnt_h
         extra.update(router_decode_leg(torch, dev, sa, kv, inp, metas, out, lse, k, scale,
-                                       max(10, args.steps // 2), max(3, args.warmup), dist, world))
+                                       max(10, args.steps // 2), max(3, args.warmup), dist, world, clocks))
     for g in graphs.values():
         del g
     graphs.clear()
     router = tsa = ratio = None
     if not args.no_extra and world == 1:  # secondary legs: single-GPU runs only
-        router = router_leg(torch, dev, max(5, min(args.steps, 50)), max(3, args.warmup))
-        tsa = tsa_leg(torch, dev, max(10, min(args.steps, 50)), max(3, args.warmup))
+        router = router_leg(torch, dev, max(5, min(args.steps, 50)), max(3, args.warmup), clocks)
+        tsa = tsa_leg(torch, dev, max(10, min(args.steps, 50)), max(3, args.warmup), clocks)
         torch.cuda.empty_cache()
-        ratio = ratio_leg(torch, dev, max(5, min(args.steps, 20)), max(3, args.warmup))
+        ratio = ratio_leg(torch, dev, max(5, min(args.steps, 20)), max(3, args.warmup), clocks)
     return dict(ms=ms, value=value, kern=kern, clocks=clocks.summary(), e2e_ms=e2e_ms, e2e_bf16=e2e_bf16,
                 e2e_zc=e2e_zc, h2d=h2d,
                 d2h=d2h, meta_bytes=meta_bytes, kv_bytes=kv_bytes, extra=extra, router=router, tsa=tsa, ratio=ratio,
@@ -586,7 +625,7 @@ def run_gpu_arm(args, rank, world, dist):
 
 
 def router_decode_leg(torch, dev, sa, kv, inp, metas, out, lse, k: int, scale: float, steps: int, warmup: int,
-                      dist, world: int):
+                      dist, world: int, clocks=None):
     """The uncertainty router applied to decode on the headline workload: each
     (layer) row is a one-row tile; metadata refresh, the router call and the
     decode over the routed lists per step."""
@@ -621,11 +660,12 @@ def router_decode_leg(torch, dev, sa, kv, inp, metas, out, lse, k: int, scale: f
         e0 = torch.cuda.Event(enable_timing=True)
         e1 = torch.cuda.Event(enable_timing=True)
         n_rep = steps
-        e0.record(stream)
-        for _ in range(n_rep):
-            routed_step()
-        e1.record(stream)
-        torch.cuda.synchronize()
+        with _region(clocks, f"router-decode/{rule}"):
+            e0.record(stream)
+            for _ in range(n_rep):
+                routed_step()
+            e1.record(stream)
+            torch.cuda.synchronize()
         m2 = max_over_ranks(e0.elapsed_time(e1) / n_rep, dist, dev)
         kept = int(cnt_r.sum().item())
         kv_r = kept * PS * 2 * D * 2
@@ -641,7 +681,7 @@ def router_decode_leg(torch, dev, sa, kv, inp, metas, out, lse, k: int, scale: f
     return res
 
 
-def router_leg(torch, dev, steps: int, warmup: int):
+def router_leg(torch, dev, steps: int, warmup: int, clocks=None):
     """The 128K-context router workload (28 query / 4 KV heads, 64-token blocks,
     2048 chunked-prefill rows in 32 tiles of 64, k = 32, rho = 2, quantile
     0.25): route + tile attention per backbone, timed with CUDA events.
@@ -690,13 +730,14 @@ def router_leg(torch, dev, steps: int, warmup: int):
             attend()
         ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(steps)]
         torch.cuda.synchronize()
-        for i in range(steps):
-            ev[i][0].record(stream)
-            route()
-            ev[i][1].record(stream)
-            attend()
-            ev[i][2].record(stream)
-        torch.cuda.synchronize()
+        with _region(clocks, f"router/{rule}"):
+            for i in range(steps):
+                ev[i][0].record(stream)
+                route()
+                ev[i][1].record(stream)
+                attend()
+                ev[i][2].record(stream)
+            torch.cuda.synchronize()
         r_ms = sum(e[0].elapsed_time(e[1]) for e in ev) / steps
         a_ms = sum(e[1].elapsed_time(e[2]) for e in ev) / steps
         if sa.sparse_attn_get_device_status(ws) != 0:
@@ -714,7 +755,7 @@ def router_leg(torch, dev, steps: int, warmup: int):
     return res
 
 
-def tsa_leg(torch, dev, steps: int, warmup: int):
+def tsa_leg(torch, dev, steps: int, warmup: int, clocks=None):
     """The TSA workload (48 layers x 4 sequences stacked along the batch axis,
     32 query / 4 KV heads, 29,504 tokens in structure-aligned chunks of 16-256
     tokens, per-chunk key offsets): the one-launch decode step under token
@@ -769,11 +810,12 @@ def tsa_leg(torch, dev, steps: int, warmup: int):
         torch.cuda.synchronize()
         e0 = torch.cuda.Event(enable_timing=True)
         e1 = torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        for _ in range(steps):
-            step()
-        e1.record(stream)
-        torch.cuda.synchronize()
+        with _region(clocks, f"tsa/{rule}/{kind}{val}"):
+            e0.record(stream)
+            for _ in range(steps):
+                step()
+            e1.record(stream)
+            torch.cuda.synchronize()
         ms = e0.elapsed_time(e1) / steps
         if sa.sparse_attn_get_device_status(ws) != 0:
             raise RuntimeError("TSA leg: device status set")
@@ -797,7 +839,7 @@ def tsa_leg(torch, dev, steps: int, warmup: int):
     return res
 
 
-def ratio_leg(torch, dev, steps: int, warmup: int):
+def ratio_leg(torch, dev, steps: int, warmup: int, clocks=None):
     """The ratio-budget workload (64 layers x 8 sequences stacked along the
     batch axis, 64 query / 8 KV heads, 32,768 tokens = 2048 16-token pages):
     the one-launch decode step under the ratio budget K = max(topk_val + bos
@@ -844,11 +886,12 @@ def ratio_leg(torch, dev, steps: int, warmup: int):
             torch.cuda.synchronize()
             e0 = torch.cuda.Event(enable_timing=True)
             e1 = torch.cuda.Event(enable_timing=True)
-            e0.record(stream)
-            for _ in range(steps):
-                step()
-            e1.record(stream)
-            torch.cuda.synchronize()
+            with _region(clocks, f"ratio/{rule}/{ratio}"):
+                e0.record(stream)
+                for _ in range(steps):
+                    step()
+                e1.record(stream)
+                torch.cuda.synchronize()
             ms = e0.elapsed_time(e1) / steps
             if sa.sparse_attn_get_device_status(ws) != 0:
                 raise RuntimeError("ratio leg: device status set")
@@ -863,6 +906,10 @@ def ratio_leg(torch, dev, steps: int, warmup: int):
     del kv, k_all, v_all, q_all, seq
     torch.cuda.empty_cache()
     return res
+
+
+def _region(clocks, name):
+    return clocks.region(name) if clocks is not None else _Null()
 
 
 class _Null:

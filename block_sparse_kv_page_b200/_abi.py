@@ -72,6 +72,11 @@ PROTOTYPES = {
                                           C.POINTER(sa_budget), C.c_int32, C.c_float, C.c_void_p,
                                           C.c_void_p, C.c_void_p, C.c_void_p, C.c_void_p, C.c_size_t,
                                           C.c_void_p]),
+    "sparse_attn_decode_step_wait_test": (C.c_int, [C.POINTER(sa_kv_desc), C.c_void_p, C.c_int, C.c_void_p,
+                                                    C.c_int32, C.POINTER(sa_budget), C.c_int32, C.c_float,
+                                                    C.c_void_p, C.c_void_p, C.c_void_p, C.c_void_p,
+                                                    C.c_int32, C.c_uint32, C.c_void_p, C.c_size_t,
+                                                    C.c_void_p]),
     "sparse_attn_decode_step_per_head": (C.c_int, [C.POINTER(sa_kv_desc), C.c_void_p, C.c_int, C.c_void_p,
                                                    C.c_int32, C.POINTER(sa_budget), C.c_int32, C.c_float,
                                                    C.c_void_p, C.c_void_p, C.c_void_p, C.c_void_p,

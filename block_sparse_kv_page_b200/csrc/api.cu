@@ -16,6 +16,7 @@
 //                            partials of decode -- after the scores in the
 //                            decode step --, router tables), not preserved
 //                            between calls
+#include <atomic>
 #include <cmath>
 #include <cstdint>
 #include <cstring>
@@ -543,7 +544,7 @@ static sa_status decode_step(const sa_kv_desc* kv, void* meta, sa_score_rule rul
                              const void* v_new, const sa_budget* budget, int32_t max_sel,
                              float scale, int32_t* sel_idx, int32_t* sel_count, void* out,
                              bool out_bf16, float* lse, bool per_head, void* ws, size_t ws_bytes,
-                             void* stream) {
+                             void* stream, int hold_flag_of = 0, uint32_t flag_spin_limit = 0) {
   int G;
   sa_status s = check_select(kv, meta, rule, q, n_q_heads, budget, max_sel, sel_idx, sel_count,
                              nullptr, &G);
@@ -591,6 +592,8 @@ static sa_status decode_step(const sa_kv_desc* kv, void* meta, sa_score_rule rul
     a.sel.v_dst = const_cast<void*>(kv->v);
   }
   a.queue = reinterpret_cast<uint32_t*>(w + kQueueStep);
+  a.sel.hold_flag_of = hold_flag_of;
+  a.flag_spin_limit = flag_spin_limit;
   const long long n_score = units * a.sel.splits, n_dec = plan.items;
   if (n_score + n_dec > 0x7fffffffLL) return SA_ERR_UNSUPPORTED;
   a.n_score = (int)n_score;
@@ -626,6 +629,19 @@ sa_status sparse_attn_decode_step_append(const sa_kv_desc* kv, void* meta, sa_sc
   if (out_dtype != SA_OUT_F32 && out_dtype != SA_OUT_BF16) return SA_ERR_INVALID;
   return decode_step(kv, meta, rule, q, n_q_heads, k_new, v_new, budget, max_sel, scale, sel_idx,
                      sel_count, out, out_dtype == SA_OUT_BF16, lse, false, ws, ws_bytes, stream);
+}
+
+sa_status sparse_attn_decode_step_wait_test(const sa_kv_desc* kv, void* meta, sa_score_rule rule,
+                                            const void* q, int32_t n_q_heads, const sa_budget* budget,
+                                            int32_t max_sel, float scale, int32_t* sel_idx,
+                                            int32_t* sel_count, float* out, float* lse,
+                                            int32_t held_unit, uint32_t flag_spin_limit, void* ws,
+                                            size_t ws_bytes, void* stream) {
+  const long long units = kv ? (long long)kv->batch * kv->n_kv_heads : 0;
+  if (held_unit < 0 || held_unit >= units || flag_spin_limit < 1) return SA_ERR_INVALID;
+  return decode_step(kv, meta, rule, q, n_q_heads, nullptr, nullptr, budget, max_sel, scale, sel_idx,
+                     sel_count, out, false, lse, false, ws, ws_bytes, stream, held_unit + 1,
+                     flag_spin_limit);
 }
 
 sa_status sparse_attn_route(const sa_kv_desc* kv, const void* meta, sa_score_rule rule,
@@ -830,23 +846,27 @@ static __device__ __align__(256) unsigned char g_decode_scratch[sa::kStaticScrat
 
 namespace sa {
 namespace {
-// Device address of g_decode_scratch on the current device (looked up once per device).
+// Device address of g_decode_scratch on the current device, looked up once
+// per device.  Host threads may race on a device's first call: each slot is
+// atomic, and every racer stores the same address.
 sa_status static_scratch(unsigned char** out) {
-  static unsigned char* addr[64] = {nullptr};
+  static std::atomic<unsigned char*> addr[64];
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) {
     cudaGetLastError();
     return SA_ERR_CUDA;
   }
-  if (!addr[dev]) {
+  unsigned char* a = addr[dev].load(std::memory_order_acquire);
+  if (!a) {
     void* p = nullptr;
     if (cudaGetSymbolAddress(&p, g_decode_scratch) != cudaSuccess || !p) {
       cudaGetLastError();
       return SA_ERR_CUDA;
     }
-    addr[dev] = static_cast<unsigned char*>(p);
+    a = static_cast<unsigned char*>(p);
+    addr[dev].store(a, std::memory_order_release);
   }
-  *out = addr[dev];
+  *out = a;
   return SA_OK;
 }
 }  // namespace

@@ -126,6 +126,10 @@ struct SelectArgs {
   const void* v_new;
   void* k_dst;
   void* v_dst;
+  // decode step, test of the bounded wait only: 1 + the unit whose selection
+  // flag is never published (its decode items run their wait out and report
+  // SA_ERR_TIMEOUT); 0 = none
+  int hold_flag_of;
 };
 cudaError_t launch_select(const SelectArgs& a, cudaStream_t st);
 
@@ -172,6 +176,7 @@ struct StepArgs {
   DecodeArgs dec;             // idx/count = sel outputs, ws_count = split counters [units]
   uint32_t* queue;            // [2] item queue (head, finished CTAs)
   int n_score, n_dec;         // items of each kind
+  uint32_t flag_spin_limit;   // polls of a unit-flag wait before SA_ERR_TIMEOUT; 0 = default (~1 s)
 };
 cudaError_t launch_step(const StepArgs& a, cudaStream_t st);
 size_t step_smem_bytes(int max_pages, int max_sel, bool chunks);

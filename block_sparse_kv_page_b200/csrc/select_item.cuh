@@ -694,7 +694,8 @@ SA_DEV void select_item(const SelectArgs& a, const int u, const int split, const
     __syncthreads();
     // the flag carries the kept count too (thread 0 wrote it), so a decode
     // item reads both with its one acquire
-    if (tid == 0) st_release_u32(&a.ws_count[u], kUnitSelected | (uint32_t)a.sel_count[u]);
+    if (tid == 0 && a.hold_flag_of != u + 1)
+      st_release_u32(&a.ws_count[u], kUnitSelected | (uint32_t)a.sel_count[u]);
   }
 }
 

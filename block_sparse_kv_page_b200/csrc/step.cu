@@ -52,10 +52,10 @@ __host__ __device__ int body_bytes(int max_pages) {
 }
 
 // Wait until a unit's selection is published and return its kept count (the
-// flag's low bits); -1 (and SA_ERR_TIMEOUT) if the bound runs out.
-SA_DEV int wait_selected(const uint32_t* flag, int* status) {
+// flag's low bits); -1 (and SA_ERR_TIMEOUT) after `limit` polls.
+SA_DEV int wait_selected(const uint32_t* flag, int* status, uint32_t limit) {
   uint32_t ns = 32;
-  for (uint32_t i = 0; i < kFlagSpinLimit; ++i) {
+  for (uint32_t i = 0; i < limit; ++i) {
     const uint32_t v = ld_acquire_u32(flag);
     if (v & sel::kUnitSelected) return (int)(v & ~sel::kUnitSelected);
     __nanosleep(ns);
@@ -105,7 +105,8 @@ __global__ void __launch_bounds__(kThreads, SA_STEP_CTAS_PER_SM)
         // the sequence length is an input of the launch: its load (kept in a
         // register until after the wait) overlaps the acquire
         const int ntok = a.dec.kv.seq_len[unit_map<PER_HEAD>(u, a.dec.kv.Hkv, a.dec.Hq, a.dec.G).b];
-        const int cnt = wait_selected(a.sel.ws_count + u, a.sel.status);  // acquire
+        const int cnt = wait_selected(a.sel.ws_count + u, a.sel.status,
+                                      a.flag_spin_limit ? a.flag_spin_limit : kFlagSpinLimit);  // acquire
         s_count = cnt;
         s_ntok = ntok;
         if (cnt < 0) item = n_items;  // gave up: this CTA stops taking work

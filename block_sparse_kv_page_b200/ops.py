@@ -203,6 +203,27 @@ def sparse_attn_decode_step(kv: KvCache, meta: torch.Tensor, rule, q: torch.Tens
            "sparse_attn_decode_step")
 
 
+def sparse_attn_decode_step_wait_test(kv: KvCache, meta: torch.Tensor, rule, q: torch.Tensor,
+                                      budget: sa_budget, max_sel: int, scale: float, sel_idx: torch.Tensor,
+                                      sel_count: torch.Tensor, out: torch.Tensor, lse: torch.Tensor | None,
+                                      held_unit: int, flag_spin_limit: int, ws: torch.Tensor,
+                                      stream=None) -> None:
+    """The decode step with unit `held_unit`'s selection never published, so
+    that its decode items run their bounded wait out (SA_ERR_TIMEOUT in the
+    workspace status word).  A test of the error path; outputs unspecified."""
+    if q.dtype != torch.bfloat16 or not q.is_contiguous():
+        raise ValueError("q must be contiguous bf16 [B, Hq, 128]")
+    if out.dtype != torch.float32 or not out.is_contiguous():
+        raise ValueError("out must be contiguous fp32")
+    _check(lib.sparse_attn_decode_step_wait_test(C.byref(kv.desc), meta.data_ptr(), _rule(rule), q.data_ptr(),
+                                                 q.shape[-2], C.byref(budget), int(max_sel), float(scale),
+                                                 sel_idx.data_ptr(), sel_count.data_ptr(), out.data_ptr(),
+                                                 _ptr(lse), int(held_unit), int(flag_spin_limit),
+                                                 ws.data_ptr(), ws.numel() * ws.element_size(),
+                                                 _stream(stream)),
+           "sparse_attn_decode_step_wait_test")
+
+
 def sparse_attn_decode_step_per_head(kv: KvCache, meta: torch.Tensor, rule, q: torch.Tensor,
                                      budget: sa_budget, max_sel: int, scale: float, sel_idx: torch.Tensor,
                                      sel_count: torch.Tensor, out: torch.Tensor, lse: torch.Tensor | None,
@@ -253,8 +274,9 @@ def sparse_attn_decode_static(kv: KvCache, q: torch.Tensor, n_q_rows: int, q_pos
     """sparse_attn_decode without a workspace, for callers that cannot
     allocate device memory where they run it: the scratch is an 8 MiB array
     inside the library, shared by every call, so calls must not overlap on
-    the GPU.  device_status: optional zeroed int32 device tensor that receives
-    the first device-side error code."""
+    the GPU.  One-row decode only (tile_rows == 1).  device_status: optional
+    zeroed int32 device tensor that receives the first device-side error
+    code; without it, device-side errors of the call are not reported."""
     if q.dtype != torch.bfloat16 or not q.is_contiguous():
         raise ValueError("q must be contiguous bf16")
     if out.dtype != torch.float32 or not out.is_contiguous():

@@ -313,6 +313,26 @@ sa_status sparse_attn_route_decode(const sa_kv_desc* kv, const void* meta, sa_sc
                                    uint8_t* triggered, float* tau_out, void* ws, size_t ws_bytes,
                                    void* stream);
 
+/* Test of the step's bounded wait (failure detection without a GPU fault).
+ * Runs sparse_attn_decode_step, except that the selection of unit
+ * `held_unit` (= b * n_kv_heads + g) is never published: the decode items of
+ * that unit poll its flag `flag_spin_limit` times (each poll a load and a
+ * sleep of at most 256 ns), then record SA_ERR_TIMEOUT in the workspace
+ * status word, and the CTA that waited stops taking work.  The launch still
+ * ends, every other CTA finishes its items, and the last CTA out leaves the
+ * workspace's counters and queue clean, so the next call on the same
+ * workspace runs normally (read and clear the status first with
+ * sparse_attn_get_device_status).  Outputs of this call are unspecified.
+ * SA_ERR_INVALID: held_unit out of range or flag_spin_limit == 0; otherwise
+ * the errors of sparse_attn_decode_step.  The pages have no counterpart: it
+ * exists to test the error path. */
+sa_status sparse_attn_decode_step_wait_test(const sa_kv_desc* kv, void* meta, sa_score_rule rule,
+                                            const void* q, int32_t n_q_heads, const sa_budget* budget,
+                                            int32_t max_sel, float scale, int32_t* sel_idx,
+                                            int32_t* sel_count, float* out, float* lse,
+                                            int32_t held_unit, uint32_t flag_spin_limit, void* ws,
+                                            size_t ws_bytes, void* stream);
+
 /* Copy the workspace status word to *host_out (SA_OK if no device check
  * fired since the last init/clear) and clear it.  Synchronises `stream`. */
 sa_status sparse_attn_get_device_status(void* ws, sa_status* host_out, void* stream);
@@ -334,12 +354,16 @@ sa_status sparse_attn_get_device_status(void* ws, sa_status* host_out, void* str
  *    the same time on the GPU (different streams, overlapping graph launches,
  *    several host threads) race and corrupt each other's results: order them
  *    on one stream.  Each call clears the counters it uses before launching.
- *  - Limits: at most 4096 (row, KV head) units per call, and the split
- *    partials of the call must fit the array; beyond either the call returns
- *    SA_ERR_WORKSPACE and launches nothing.
+ *  - Limits: one-row decode only (tile_rows == 1; multi-row tile attention,
+ *    tile_rows > 1, returns SA_ERR_UNSUPPORTED); at most 4096 (row, KV head)
+ *    units per call, and the split partials of the call must fit the array;
+ *    beyond either the call returns SA_ERR_WORKSPACE and launches nothing.
  *  - It allocates and frees no memory.
  *  - device_status (nullable): a device int32, zeroed by the caller, that
- *    receives the first device-side error code of the call. */
+ *    receives the first device-side error code of the call (a range check or
+ *    a bounded-wait timeout).  With device_status null such errors are NOT
+ *    reported: they land in the array's own status word, which the next call
+ *    clears before anyone could read it.  Pass one to see them. */
 sa_status sparse_attn_decode_static(const sa_kv_desc* kv, const void* q, int32_t n_q_heads,
                                     int32_t n_q_rows, int32_t q_pos0, int32_t tile_rows,
                                     float scale, const int32_t* idx, const int32_t* count,

@@ -19,9 +19,9 @@ import torch
 
 import block_sparse_kv_page_b200 as sa
 import oracle as O
+from certify import TIE_REL, certify_selection  # noqa: F401
 
 OUT_TOL = 2e-3
-TIE_REL = 1e-5
 
 
 def to_np(t: torch.Tensor) -> np.ndarray:
@@ -148,63 +148,15 @@ def run_step(layer, *, page_size: int, rule: str, budget: dict, scale: float,
     return r
 
 
-def _certify_cut(S, order, n_keep, gset, where):
-    """Exact set equality unless the cut is a near-tie; then band rules."""
-    oset = set(int(p) for p in order[:n_keep])
-    if n_keep == 0 or n_keep >= len(order):
-        assert gset == oset, f"{where}: set differs with no cut ({len(gset)} vs {len(oset)})"
-        return False
-    a, b = S[order[n_keep - 1]], S[order[n_keep]]
-    delta = TIE_REL * max(abs(a), abs(b), 1.0)
-    if a - b >= delta:
-        assert gset == oset, f"{where}: set differs at a decisive cut (gap {a - b:.3g})"
-        return False
-    assert len(gset) == len(oset), f"{where}: count {len(gset)} vs {len(oset)}"
-    for p in (int(x) for x in order):
-        if S[p] > a + delta:
-            assert p in gset, f"{where}: page {p} above the tie band dropped"
-        if S[p] < b - delta:
-            assert p not in gset, f"{where}: page {p} below the tie band kept"
-    return True
-
-
-def certify_selection(S, gset: set, budget: dict, lens=None, where=""):
-    """Returns True when a certified near-tie allowed a difference."""
-    S = np.asarray(S, dtype=np.float64)
-    P = len(S)
-    order = O.rank_order(S)
-    kind = budget["kind"]
-    if kind == "topk":
-        return _certify_cut(S, order, min(budget["k"], P), gset, where)
-    if kind == "ratio":
-        K = O.ratio_budget_pages(P, budget["ratio"], budget.get("topk_val", 1), budget["bos"], budget["eos"])
-        forced = set(int(x) for x in O.forced_pages(P, budget["bos"], budget["eos"]))
-        assert forced <= gset, f"{where}: forced pages missing"
-        rest = np.array([p for p in order if int(p) not in forced], dtype=np.int64)
-        Sr = S.copy()
-        return _certify_cut(Sr, rest, K - len(forced), gset - forced, where)
-    # token budget: greedy prefix of the rank order
-    lens = np.asarray(lens, dtype=np.int64)
-    oset = set(int(p) for p in O.select_token_budget(S, lens, budget["budget"]))
-    r = len(oset)
-    near = False
-    for i in (r - 1, r):
-        if 0 <= i and i + 1 < P:
-            a, b = S[order[i]], S[order[i + 1]]
-            if a - b < TIE_REL * max(abs(a), abs(b), 1.0):
-                near = True
-    if not near:
-        assert gset == oset, f"{where}: token-budget set differs"
-        return False
-    assert sum(int(lens[p]) for p in gset) <= budget["budget"], f"{where}: over budget"
-    return True
-
-
 def check_layer(layer, gpu, *, page_size: int, rule: str, budget: dict, scale: float,
-                units=None, score_rel: float = 2e-6, out_tol: float = OUT_TOL, per_head: bool = False):
+                units=None, score_rel: float = 2e-6, out_tol: float = OUT_TOL, per_head: bool = False,
+                host_cache: dict | None = None):
     """Compare every (b, g) unit (or the given subset) with the oracle.
     per_head: units are (b, query head h), each with its own page set; the
     oracle is the same one applied to the single head h (its group is {h}).
+    host_cache: a dict that keeps the last unit's host copies of K, V and its
+    oracle metadata, so that several runs over the same cache checked unit by
+    unit compute them once.
     Returns a dict of statistics (max errors, tie exemptions)."""
     B, Hkv = layer.k.shape[:2]
     Hq = layer.q.shape[1]
@@ -218,16 +170,22 @@ def check_layer(layer, gpu, *, page_size: int, rule: str, budget: dict, scale: f
         N = int(layer.seq_len[b])
         where = f"unit(b={b},{'h' if per_head else 'g'}={x})"
         Qg = to_np(layer.q[b, h0:h1])
-        K = to_np(layer.k[b, g, :N])
-        V = to_np(layer.v[b, g, :N])
-        if page_size:
-            starts, ends = O.fixed_pages(N, page_size)
-            off = None
+        key = (id(layer), b, g, N)
+        if host_cache is not None and host_cache.get("key") == key:
+            K, V, starts, ends, meta = host_cache["val"]
         else:
-            C = int(layer.n_chunks[b])
-            off = layer.chunk_off[b, :C + 1].cpu().numpy().astype(np.int64)
-            starts, ends = O.chunk_pages(off)
-        meta = O.page_metadata(K, starts, ends)
+            K = to_np(layer.k[b, g, :N])
+            V = to_np(layer.v[b, g, :N])
+            if page_size:
+                starts, ends = O.fixed_pages(N, page_size)
+            else:
+                C = int(layer.n_chunks[b])
+                off = layer.chunk_off[b, :C + 1].cpu().numpy().astype(np.int64)
+                starts, ends = O.chunk_pages(off)
+            meta = O.page_metadata(K, starts, ends)
+            if host_cache is not None:
+                host_cache["key"] = key
+                host_cache["val"] = (K, V, starts, ends, meta)
         P = len(starts)
         # metadata parity
         gm = gpu["meta"][b, g, :P]
@@ -271,3 +229,92 @@ def check_layer(layer, gpu, *, page_size: int, rule: str, budget: dict, scale: f
             assert le <= 1e-3 * max(1.0, float(np.abs(l_ref).max())), f"{where}: lse err {le:.3g}"
         stats["units"] += 1
     return stats
+
+
+# ---------------------------------------------------------------------------
+# Unit checks in spawned worker processes (full-size workloads).
+_POOL = None
+
+
+def oracle_pool():
+    """A process pool for the oracle side of the checks.  Spawned (never
+    forked: this process holds a CUDA context), one BLAS thread per worker."""
+    global _POOL
+    if _POOL is None:
+        import atexit
+        import multiprocessing as mp
+        import os
+        n = max(1, min(32, len(os.sched_getaffinity(0))))
+        keep = {k: os.environ.get(k) for k in ("OMP_NUM_THREADS", "OPENBLAS_NUM_THREADS", "MKL_NUM_THREADS")}
+        for k in keep:
+            os.environ[k] = "1"
+        try:
+            _POOL = mp.get_context("spawn").Pool(n)
+        finally:
+            for k, v in keep.items():
+                if v is None:
+                    os.environ.pop(k, None)
+                else:
+                    os.environ[k] = v
+        atexit.register(_POOL.terminate)
+    return _POOL
+
+
+def _host_f32(t: torch.Tensor) -> np.ndarray:
+    return t.detach().float().cpu().numpy()
+
+
+def check_units_parallel(layer, runs, *, page_size: int, scale: float, units=None,
+                         score_rel: float = 2e-6, out_tol: float = OUT_TOL, per_head: bool = False,
+                         batch_units: int | None = None):
+    """Check the given units (default: all) of every run against the oracle,
+    several units at a time in the oracle pool.  runs: list of (gpu, rule,
+    budget) over the same cache, gpu as returned by run_gpu / run_step.
+    Returns aggregate statistics per run (max errors, certified ties)."""
+    import unit_check
+    B, Hkv = layer.k.shape[:2]
+    Hq = layer.q.shape[1]
+    G = Hq // Hkv
+    if units is None:
+        units = [(b, x) for b in range(B) for x in range(Hq if per_head else Hkv)]
+    pool = oracle_pool()
+    if batch_units is None:
+        batch_units = 2 * pool._processes
+    agg = [dict(max_out_err=0.0, max_lse_err=0.0, max_score_err=0.0, ties=0, units=0) for _ in runs]
+    kw = dict(scale=scale, score_rel=score_rel, out_tol=out_tol)
+
+    def task(b, x):
+        g, h0, h1 = (x // G, x, x + 1) if per_head else (x, x * G, (x + 1) * G)
+        N = int(layer.seq_len[b])
+        if page_size:
+            starts, ends = O.fixed_pages(N, page_size)
+        else:
+            C = int(layer.n_chunks[b])
+            off = layer.chunk_off[b, :C + 1].cpu().numpy().astype(np.int64)
+            starts, ends = O.chunk_pages(off)
+        P = len(starts)
+        host = dict(Q=_host_f32(layer.q[b, h0:h1]), K=_host_f32(layer.k[b, g, :N]),
+                    V=_host_f32(layer.v[b, g, :N]), starts=starts, ends=ends, chunks=not page_size)
+        rr = []
+        for gpu, rule, budget in runs:
+            cnt = int(gpu["sel_count"][b, x])
+            sc = gpu.get("scores")
+            rr.append(dict(rule=rule, budget=budget,
+                           meta=gpu["meta"][b, g, :P].cpu().numpy(),
+                           scores=None if sc is None else sc[b, x, :P].numpy(),
+                           sel=gpu["sel_idx"][b, x, :cnt].numpy().astype(np.int64),
+                           out=gpu["out"][b, h0:h1].float().numpy(),
+                           lse=gpu["lse"][b, h0:h1].numpy()))
+        return host, rr, dict(kw, where=f"unit(b={b},{'h' if per_head else 'g'}={x})")
+
+    for i in range(0, len(units), batch_units):
+        tasks = [task(b, x) for b, x in units[i:i + batch_units]]
+        for ok, val in pool.map(unit_check.check_unit_task, tasks, chunksize=1):
+            assert ok, val
+            for a, s in zip(agg, val):
+                a["max_out_err"] = max(a["max_out_err"], s["max_out_err"])
+                a["max_lse_err"] = max(a["max_lse_err"], s["max_lse_err"])
+                a["max_score_err"] = max(a["max_score_err"], s["max_score_err"])
+                a["ties"] += int(s["tie"])
+                a["units"] += 1
+    return agg

@@ -193,3 +193,16 @@ def test_workspace_size(lib, abi):
     assert lib.sparse_attn_workspace_size(C.byref(ok), 30, 1, 16) == 0
     assert lib.sparse_attn_workspace_size(C.byref(_desc(abi, head_dim=64)), 32, 1, 16) == 0
     assert lib.sparse_attn_workspace_init(None, 1 << 20, None) == abi.SA_ERR_WORKSPACE
+
+
+def test_decode_static_rejects_tile_attention(lib, abi):
+    """The workspace-free decode serves one-row decode only: multi-row tiles
+    (tile_rows > 1) are refused on the host, before any CUDA call."""
+    d = _desc(abi, batch=1)
+    r = lib.sparse_attn_decode_static(C.byref(d), 0x50000, 32, 64, 0, 64, 0.088, 0x60000, 0x70000, 16,
+                                      0x80000, None, None, None)
+    assert r == abi.SA_ERR_UNSUPPORTED
+    # and a one-row call with a bad row count is invalid, also before any launch
+    r = lib.sparse_attn_decode_static(C.byref(d), 0x50000, 32, 3, 0, 1, 0.088, 0x60000, 0x70000, 16,
+                                      0x80000, None, None, None)
+    assert r == abi.SA_ERR_INVALID

@@ -3,9 +3,10 @@
 sparse_attn_decode_static serves callers that cannot allocate device memory
 where they run the attention (a plugin handed only its input/output pointers
 at enqueue time, or a decode loop that must not pay cudaMalloc's device-wide
-synchronisation).  Its scratch is an array built into the library, so two
-calls in a row must both give the same result as sparse_attn_decode with a
-caller-provided workspace, within the output tolerance the parity tests use.
+synchronisation).  Its scratch is an array built into the library.  It runs
+the same kernel with the same work split as sparse_attn_decode, so two calls
+in a row must both reproduce sparse_attn_decode's output bit for bit, and
+the calls must leave the device's free memory unchanged.
 
 This file is collected last on purpose; it passes alone in a fresh process
 (the first call looks up the array's address) and after the other tests.
@@ -20,40 +21,50 @@ import datagen as DG
 
 pytestmark = pytest.mark.gpu
 
-OUT_TOL = 2e-3
 
-
-def _problem(dev):
+def _problem(dev, B, seq_lens, k, seed):
     import block_sparse_kv_page_b200 as sa
-    lay = DG.make_decode_layer(B=2, Hq=32, Hkv=4, seq_lens=[3000, 2222], cap=3008, seed=4242,
-                               device=dev, key_scale="channel")
-    kv = sa.KvCache(lay.k, lay.v, lay.seq_len, page_size=16, max_pages=188)
-    k = 64
+    cap = max(seq_lens)
+    lay = DG.make_decode_layer(B=B, Hq=32, Hkv=4, seq_lens=seq_lens, cap=cap, seed=seed, device=dev,
+                               key_scale="channel")
+    P = -(-cap // 16)
+    kv = sa.KvCache(lay.k, lay.v, lay.seq_len, page_size=16, max_pages=P)
     meta = kv.meta_buffer()
-    ws = sa.make_workspace(kv, 32, 2, k)
-    sel = torch.empty((2, 4, k), dtype=torch.int32, device=dev)
-    cnt = torch.empty((2, 4), dtype=torch.int32, device=dev)
+    ws = sa.make_workspace(kv, 32, B, k)
+    sel = torch.empty((B, 4, k), dtype=torch.int32, device=dev)
+    cnt = torch.empty((B, 4), dtype=torch.int32, device=dev)
     sa.sparse_attn_build_meta(kv, "envelope", 0, meta)
     sa.sparse_attn_select(kv, meta, "envelope", lay.q, sa.budget_topk(k), k, sel, cnt, None, ws)
-    return sa, lay, kv, ws, sel, cnt, k
+    return sa, lay, kv, ws, sel, cnt
 
 
-def test_static_scratch_matches_workspace_decode(cuda_dev):
-    sa, lay, kv, ws, sel, cnt, k = _problem(cuda_dev)
+@pytest.mark.parametrize("B,seq_lens,k", [(2, [3000, 2222], 64), (4, [8192, 5000, 7777, 16], 256)])
+def test_static_scratch_matches_workspace_decode(cuda_dev, B, seq_lens, k):
+    sa, lay, kv, ws, sel, cnt = _problem(cuda_dev, B, seq_lens, k, seed=4242 + B)
+    # the work is split, so the split partials in the built-in array are used:
+    # at most 2 x SMs units' worth of items makes every unit take >= 2 splits
+    # when its page budget allows (>= 32 pages, i.e. two 16-tile items)
+    sms = torch.cuda.get_device_properties(cuda_dev).multi_processor_count
+    units = B * 4
+    assert (2 * sms + units - 1) // units >= 2 and (k + 15) // 16 >= 2
     scale = 1.0 / math.sqrt(128)
-    ref = torch.empty((2, 32, 128), dtype=torch.float32, device=cuda_dev)
-    ref_lse = torch.empty((2, 32), dtype=torch.float32, device=cuda_dev)
-    sa.sparse_attn_decode(kv, lay.q, 2, 0, 1, scale, sel, cnt, k, ref, ref_lse, ws)
+    ref = torch.empty((B, 32, 128), dtype=torch.float32, device=cuda_dev)
+    ref_lse = torch.empty((B, 32), dtype=torch.float32, device=cuda_dev)
+    sa.sparse_attn_decode(kv, lay.q, B, 0, 1, scale, sel, cnt, k, ref, ref_lse, ws)
     status = torch.zeros(1, dtype=torch.int32, device=cuda_dev)
-    for call in range(2):
-        out = torch.full_like(ref, float("nan"))
-        lse = torch.full_like(ref_lse, float("nan"))
-        sa.sparse_attn_decode_static(kv, lay.q, 2, 0, 1, scale, sel, cnt, k, out, lse, status)
-        torch.cuda.synchronize()
-        assert torch.isfinite(out).all(), f"call {call}: non-finite output"
-        err = (out - ref).abs().max().item()
-        assert err <= OUT_TOL, f"call {call}: max-abs difference {err}"
-        assert (lse - ref_lse).abs().max().item() <= 1e-3, f"call {call}: lse differs"
+    outs = [torch.full_like(ref, float("nan")) for _ in range(3)]
+    lses = [torch.full_like(ref_lse, float("nan")) for _ in range(3)]
+    # first call: on a fresh process it looks up the array's address
+    sa.sparse_attn_decode_static(kv, lay.q, B, 0, 1, scale, sel, cnt, k, outs[0], lses[0], status)
+    torch.cuda.synchronize()
+    free0 = torch.cuda.mem_get_info(cuda_dev)[0]
+    for call in (1, 2):  # two calls in a row
+        sa.sparse_attn_decode_static(kv, lay.q, B, 0, 1, scale, sel, cnt, k, outs[call], lses[call], status)
+    torch.cuda.synchronize()
+    assert torch.cuda.mem_get_info(cuda_dev)[0] == free0, "the calls changed the device's free memory"
+    for call in range(3):
+        assert torch.equal(outs[call], ref), f"call {call}: output differs from sparse_attn_decode"
+        assert torch.equal(lses[call], ref_lse), f"call {call}: lse differs from sparse_attn_decode"
     assert int(status.item()) == 0
 
 
