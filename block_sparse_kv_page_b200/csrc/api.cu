@@ -594,6 +594,17 @@ static sa_status decode_step(const sa_kv_desc* kv, void* meta, sa_score_rule rul
   a.queue = reinterpret_cast<uint32_t*>(w + kQueueStep);
   a.sel.hold_flag_of = hold_flag_of;
   a.flag_spin_limit = flag_spin_limit;
+  // few units (one layer at batch 1, say): one thread-block cluster per unit;
+  // the flag-wait test needs the persistent kernel (it exercises its flags)
+  const int C = (per_head || hold_flag_of) ? 0 : step_cluster_size((int)units, plan.splits, sm);
+  if (C > 0 && plan.fine_unit0 == units) {
+    StepArgs c = a;
+    c.sel.splits = C;
+    c.n_score = (int)(units * C);
+    c.n_dec = (int)plan.items;
+    if (launch_step_cluster(c, C, (cudaStream_t)stream) == cudaSuccess) return SA_OK;
+    cudaGetLastError();  // the cluster shape could not be launched here: use the persistent kernel
+  }
   const long long n_score = units * a.sel.splits, n_dec = plan.items;
   if (n_score + n_dec > 0x7fffffffLL) return SA_ERR_UNSUPPORTED;
   a.n_score = (int)n_score;

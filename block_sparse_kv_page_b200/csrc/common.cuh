@@ -120,6 +120,28 @@ SA_DEV void fence_proxy_async_global() { asm volatile("fence.proxy.async.global;
 // kernel begin launching (once every CTA of this grid has triggered or exited).
 SA_DEV void grid_dep_wait() { asm volatile("griddepcontrol.wait;\n" ::: "memory"); }
 SA_DEV void grid_dep_trigger() { asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory"); }
+// Thread-block clusters: this CTA's rank in its cluster, the cluster's CTA
+// count and its index in the grid (x).  cluster_sync(): every thread of every
+// CTA of the cluster arrives (release at cluster scope) and waits (acquire),
+// so each CTA's earlier writes, global or shared, are visible to the others.
+SA_DEV uint32_t cluster_ctarank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;\n" : "=r"(r));
+  return r;
+}
+SA_DEV uint32_t cluster_nctarank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_nctarank;\n" : "=r"(r));
+  return r;
+}
+SA_DEV uint32_t cluster_id_x() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%clusterid.x;\n" : "=r"(r));
+  return r;
+}
+SA_DEV void cluster_sync() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\nbarrier.cluster.wait.acquire.aligned;\n" ::: "memory");
+}
 SA_DEV void prefetch_tmap(const void* tmap) {
   asm volatile("prefetch.tensormap [%0];\n" ::"l"(tmap) : "memory");
 }

@@ -179,6 +179,9 @@ struct StepArgs {
   uint32_t flag_spin_limit;   // polls of a unit-flag wait before SA_ERR_TIMEOUT; 0 = default (~1 s)
 };
 cudaError_t launch_step(const StepArgs& a, cudaStream_t st);
+// Few units: one cluster of C CTAs per unit (sel.splits must be C).
+int step_cluster_size(int units, int dec_splits, int sm_count);
+cudaError_t launch_step_cluster(const StepArgs& a, int C, cudaStream_t st);
 size_t step_smem_bytes(int max_pages, int max_sel, bool chunks);
 
 struct TileAttnArgs {

@@ -464,6 +464,31 @@ SA_DEV void select_unit(const SelectArgs& a, const int u, const int b, const int
     select_unit_smem(a, u, N, P, cap, forced_lo, forced_hi, off, S);
 }
 
+// Tokens N and pages (or chunks) P of sequence b; false (and P = 0) when
+// they are out of range.
+SA_DEV bool unit_geometry(const SelectArgs& a, const int b, int& N, int& P) {
+  N = a.kv.seq_len[b];
+  bool bad = (N < 1 || N > a.kv.cap);
+  if (a.kv.page_size > 0) {
+    P = bad ? 0 : (N + a.kv.page_size - 1) / a.kv.page_size;
+  } else {
+    P = a.kv.n_chunks[b];
+    bad = bad || P < 1;
+  }
+  if (P > a.kv.max_pages) bad = true;
+  if (bad) P = 0;
+  return !bad;
+}
+
+// Selection of unit u (sequence, KV head) from the group scores its scoring
+// items wrote; the caller has made them visible to this CTA.
+SA_DEV void select_unit_of(const SelectArgs& a, const int u, const SelSmem& S) {
+  const int b = u / a.kv.Hkv;
+  int N, P;
+  unit_geometry(a, b, N, P);  // a bad geometry was flagged by the scoring
+  select_unit(a, u, b, N, P, S);
+}
+
 // FUSED (the decode step): refresh the newest page while scoring and publish
 // the unit's flag after selecting.
 // SCORE_ONLY: write the group scores and stop (no selection; the unit
@@ -482,20 +507,8 @@ SA_DEV void select_item(const SelectArgs& a, const int u, const int split, const
   const bool kv_owner = !PER_HEAD || um.h0 % a.G == 0;
 
   // ---- unit geometry (every CTA of the unit computes the same values)
-  const int N = a.kv.seq_len[b];
-  int P;
-  bool bad = (N < 1 || N > a.kv.cap);
-  if (a.kv.page_size > 0) {
-    P = bad ? 0 : (N + a.kv.page_size - 1) / a.kv.page_size;
-  } else {
-    P = a.kv.n_chunks[b];
-    bad = bad || P < 1;
-  }
-  if (P > a.kv.max_pages) bad = true;
-  if (bad) {
-    P = 0;
-    if (tid == 0 && split == 0) flag_status(a.status, SA_ERR_DEVICE_CHECK);
-  }
+  int N, P;
+  if (!unit_geometry(a, b, N, P) && tid == 0 && split == 0) flag_status(a.status, SA_ERR_DEVICE_CHECK);
   const int TP = (P + 15) >> 4;
   const int t_begin = (int)(((long long)TP * split) / a.splits);
   const int t_end = (int)(((long long)TP * (split + 1)) / a.splits);

@@ -30,6 +30,11 @@
 #ifndef SA_STEP_CTAS_PER_SM
 #define SA_STEP_CTAS_PER_SM 3
 #endif
+// CTAs per cluster of the small-unit decode step (16 needs the non-portable
+// cluster size; 8 is portable)
+#ifndef SA_STEP_CLUSTER
+#define SA_STEP_CLUSTER 16
+#endif
 
 namespace sa {
 namespace {
@@ -44,6 +49,7 @@ constexpr int kStages = sel::kStages;
 constexpr int kBarBytes = kWarps * kStages * 8;
 constexpr int kTileRefBytes = dec::kMaxItemTiles * (int)sizeof(dec::TileRef);
 constexpr uint32_t kFlagSpinLimit = 1u << 22;  // x (load + <= 256 ns sleep): about a second
+constexpr size_t kClusterMinSmem = 116 * 1024;  // more than half an SM's shared memory
 
 // Ring, or the selection keys/weights when those are larger.
 __host__ __device__ int body_bytes(int max_pages) {
@@ -155,6 +161,70 @@ __global__ void __launch_bounds__(kThreads, SA_STEP_CTAS_PER_SM)
   }
 }
 
+// The decode step for few units (a single layer at batch 1, say): one
+// thread-block cluster of C CTAs per unit (sequence, KV head), so the
+// handoffs between stages are hardware cluster barriers instead of global
+// item claims and flag polls.  CTA r of the cluster scores tile range r of C
+// (the one holding the newest page also refreshes it); after a cluster
+// barrier the leader (rank 0) selects the unit's pages; after another, CTA r
+// runs decode splits r, r + C, ... of the unit, merged by the last of them
+// as in the persistent kernel.  The same item code with the same splits as
+// the separate calls, so results are identical to them.
+template <int RULE>
+__global__ void __launch_bounds__(kThreads, 1) step_cluster_kernel(const __grid_constant__ StepArgs a) {
+  extern __shared__ unsigned char smem_raw[];
+  __shared__ uint32_t s_hist[512];
+  __shared__ uint32_t s_scan[32];
+  __shared__ uint32_t s_bc[8];
+  __shared__ int s_last, s_ntiles;
+  unsigned char* base = reinterpret_cast<unsigned char*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  const int body = body_bytes(a.sel.kv.max_pages);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(base + body);
+  const sel::SelSmem S{base, bars, s_hist, s_scan, s_bc, &s_last};
+  const dec::Smem D{base, bars, reinterpret_cast<dec::TileRef*>(base + body + kBarBytes),
+                    reinterpret_cast<int*>(base + body + kBarBytes + kTileRefBytes), s_scan, &s_last,
+                    &s_ntiles};
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  if (lane == 0) {
+    for (int s = 0; s < kStages; ++s) mbar_init(bars + warp * kStages + s, 1);
+    fence_barrier_init();
+  }
+  if (threadIdx.x == 0) {
+    prefetch_tmap(&a.sel.tmap_meta);
+    prefetch_tmap(&a.dec.tmap_k);
+    prefetch_tmap(&a.dec.tmap_v);
+  }
+  __syncthreads();
+  grid_dep_wait();     // the previous kernel of the stream has completed (no global access before)
+  grid_dep_trigger();  // the next kernel may be scheduled now; it waits for this one to complete
+  const int r = (int)cluster_ctarank(), C = (int)cluster_nctarank();
+  const int u = (int)cluster_id_x();
+  WarpState ws{0u, true, 0u, 0u};
+  // 1. scoring of tile range r of C (a.sel.splits == C)
+  sel::select_item<RULE, true, false, true>(a.sel, u, r, S, ws);
+  fence_proxy_async();  // generic writes to the ring (the refresh patch) before its next TMA writes
+  __syncthreads();
+  cluster_sync();       // every range's scores are visible to the leader
+  // 2. the leader selects
+  if (r == 0) sel::select_unit_of(a.sel, u, S);
+  fence_proxy_async();  // the ring held the keys
+  __syncthreads();
+  cluster_sync();       // the selection is visible to every CTA of the cluster
+  // 3. decode splits r, r + C, ... (each reads the kept count and pages)
+  if (a.sel.k_new != nullptr && lane == 0) fence_proxy_async_global();  // appended rows, then TMA
+  for (int split = r; split < a.dec.splits; split += C) {
+    dec::decode_item<false>(a.dec, u, split, D, ws);
+    fence_proxy_async();
+    __syncthreads();
+  }
+  if (!ws.alive && lane == 0) {  // a wait timed out: let the copies in flight land (bounded)
+    uint64_t* wb = bars + warp * kStages;
+    for (uint32_t g = ws.drain_lo; g < ws.drain_hi; ++g)
+      mbar_wait(wb + g % kStages, (g / kStages) & 1u, nullptr);
+  }
+}
+
 // Resident CTAs per SM of a step kernel for a shared-memory size (cached).
 int step_occupancy(const void* fn, size_t smem) {
   struct Entry {
@@ -187,6 +257,44 @@ size_t step_smem_bytes(int max_pages, int max_sel, bool chunks) {
   size_t s = 1024 + (size_t)body_bytes(max_pages) + kBarBytes + kTileRefBytes;
   if (chunks) s += (size_t)(max_sel + 1) * 4;  // decode: tile prefix of the kept chunks
   return s;
+}
+
+// Cluster size of the small-unit decode step: C CTAs per unit, one CTA per
+// SM, when all units' clusters fit the GPU at once and the unit's decode
+// splits fill them; 0 = use the persistent kernel.
+int step_cluster_size(int units, int dec_splits, int sm_count) {
+  if (units < 1 || dec_splits < SA_STEP_CLUSTER) return 0;
+  if ((long long)units * SA_STEP_CLUSTER > sm_count) return 0;
+  return SA_STEP_CLUSTER;
+}
+
+cudaError_t launch_step_cluster(const StepArgs& a, int C, cudaStream_t st) {
+  size_t smem = step_smem_bytes(a.sel.kv.max_pages, a.dec.max_sel, a.sel.kv.page_size == 0);
+  if (smem < kClusterMinSmem) smem = kClusterMinSmem;  // one CTA per SM
+  const int units = a.sel.kv.B * a.sel.kv.Hkv;
+  const void* fn = a.sel.rule == 0 ? (const void*)step_cluster_kernel<0> : (const void*)step_cluster_kernel<1>;
+  cudaError_t e = set_smem_attr(fn, smem);
+  if (e != cudaSuccess) return e;
+  if (C > 8) {
+    e = cudaFuncSetAttribute(fn, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+    if (e != cudaSuccess) return e;
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)(units * C));
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  attr[1].id = cudaLaunchAttributeClusterDimension;
+  attr[1].val.clusterDim.x = (unsigned)C;
+  attr[1].val.clusterDim.y = 1;
+  attr[1].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 2;
+  if (a.sel.rule == 0) return cudaLaunchKernelEx(&cfg, step_cluster_kernel<0>, a);
+  return cudaLaunchKernelEx(&cfg, step_cluster_kernel<1>, a);
 }
 
 cudaError_t launch_step(const StepArgs& a, cudaStream_t st) {

@@ -16,7 +16,9 @@ Each case checks the step two ways:
 Cases span fixed pages of 16 and 64 tokens, G = 7 and 8, ratio budgets with
 forced pages, TSA chunks with a token budget and with a chunk-count budget
 (both scoring rules), newest tokens that open a new page, one-token caches,
-and hundreds of units.
+and hundreds of units; the cluster_* cases have few units with at least 16
+decode splits each, which the step runs as one thread-block cluster per unit
+(one and two decode splits per CTA).
 """
 import math
 
@@ -68,6 +70,26 @@ def _case(dev, name):
         lay = DG.make_decode_layer(B=3, Hq=32, Hkv=4, seq_lens=[4000, 3900, 2500], seed=307, device=dev,
                                    cap=4000, chunk_lens=lens, chunk_offset_std=0.5)
         return lay, 0, {"kind": "topk", "k": 32}
+    # few units with at least 16 decode splits each: the one-cluster-per-unit launch
+    if name == "cluster_ps16":
+        lay = DG.make_decode_layer(B=1, Hq=32, Hkv=4, seq_lens=[8000], seed=311, device=dev,
+                                   key_scale="channel")
+        return lay, 16, {"kind": "topk", "k": 256}
+    if name == "cluster_two_rounds":
+        # 32 decode splits per unit: each CTA of a cluster runs two
+        lay = DG.make_decode_layer(B=2, Hq=32, Hkv=4, seq_lens=[8192, 6001], seed=312, device=dev, cap=8192)
+        return lay, 16, {"kind": "topk", "k": 512}
+    if name == "cluster_chunks_tokens":
+        lens = DG.workload3_chunks(1, 12000, seed_offset=5)
+        lay = DG.make_decode_layer(B=1, Hq=32, Hkv=4, seq_lens=[12000], seed=313, device=dev,
+                                   chunk_lens=lens, chunk_offset_std=0.5)
+        return lay, 0, {"kind": "tokens", "budget": 4096}
+    if name == "cluster_ratio":
+        lay = DG.make_decode_layer(B=1, Hq=64, Hkv=8, seq_lens=[32768], seed=314, device=dev)
+        return lay, 16, {"kind": "ratio", "ratio": 0.25, "bos": 1, "eos": 1}
+    if name == "cluster_ps64_g7":
+        lay = DG.make_decode_layer(B=1, Hq=28, Hkv=4, seq_lens=[20001], seed=315, device=dev, cap=20032)
+        return lay, 64, {"kind": "topk", "k": 64}
     if name == "many_units":
         rng = np.random.default_rng(7)
         lens = [int(x) for x in rng.integers(1, 2048, size=64)]
@@ -77,7 +99,8 @@ def _case(dev, name):
 
 
 CASES = ["ps16_topk", "ps16_new_page", "ps64_g7", "ratio_bos_eos", "chunks_tokens", "chunks_topk",
-         "many_units"]
+         "many_units", "cluster_ps16", "cluster_two_rounds", "cluster_chunks_tokens", "cluster_ratio",
+         "cluster_ps64_g7"]
 
 
 def _pages(lay, b, ps):
@@ -135,7 +158,8 @@ def test_step_per_head_parity(cuda_dev, R, rule, name):
 
 
 @pytest.mark.parametrize("rule", ["envelope", "centroid"])
-@pytest.mark.parametrize("name", ["ps16_topk", "ps16_new_page", "ps64_g7", "chunks_topk", "chunks_tokens"])
+@pytest.mark.parametrize("name", ["ps16_topk", "ps16_new_page", "ps64_g7", "chunks_topk", "chunks_tokens",
+                                  "cluster_ps16", "cluster_chunks_tokens"])
 def test_step_append(cuda_dev, R, rule, name):
     """The step that stores the newest token's key and value itself equals
     storing them first and running the step, bit for bit, and leaves the same

@@ -97,6 +97,28 @@ def test_step_48_layers_every_unit(cuda_dev, R, qwen3vl_48, rule):
         print(f"\n{rule}@{bd['k'] * 16}: {st}")
 
 
+# --------------------------------------------------------------------------- one layer per launch
+@pytest.mark.parametrize("rule", ["envelope", "centroid"])
+@pytest.mark.parametrize("budget", [4096, 8192])
+def test_step_one_layer_every_unit(cuda_dev, R, rule, budget):
+    """The dependent per-layer sweep's launch: one layer (batch 1, 4 KV heads,
+    29,504 tokens) per sparse_attn_decode_step, run as one thread-block
+    cluster per (sequence, KV head); every unit against the oracle and bit for
+    bit against the separate calls."""
+    bd = {"kind": "topk", "k": budget // 16}
+    for layer in (0, 47):
+        lay = DG.workload2_layer(layer, cuda_dev)
+        g = R.run_step(lay, page_size=16, rule=rule, budget=bd, scale=SCALE, stale=True, repeat=2)
+        assert g["status"] == 0
+        sep = R.run_gpu(lay, page_size=16, rule=rule, budget=bd, scale=SCALE)
+        _same(g, sep, f"layer {layer} {rule}@{budget}")
+        for r in g["runs"][1:]:
+            for key in ("sel_idx", "sel_count", "out", "lse"):
+                assert torch.equal(r[key], g["runs"][0][key]), key
+        st = R.check_layer(lay, g, page_size=16, rule=rule, budget=bd, scale=SCALE)
+        assert st["units"] == 4 and st["max_out_err"] < 1e-4
+
+
 # --------------------------------------------------------------------------- TSA
 @pytest.mark.slow
 def test_tsa_48_layers_every_unit(cuda_dev, R):
