@@ -68,6 +68,9 @@ def parse():
     ap.add_argument("--cpu-sample-units", type=int, default=192)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-extra", action="store_true", help="skip the secondary modes/rules")
+    ap.add_argument("--shard", choices=["heads", "replicas"], default="heads",
+                    help="N > 1 GPUs: split the KV heads (and, past the head count, the layers) of one "
+                         "workload over the ranks (strong scaling), or run N independent replicas (weak)")
     ap.add_argument("--router-only", action="store_true",
                     help="time only the router workload (route + tile attention) and print its JSON")
     ap.add_argument("--router-decode-only", action="store_true",
@@ -286,29 +289,79 @@ def whole_job_value(units_per_rank: float, world: int, ms: float) -> float:
     return units_per_rank * world / (ms * 1e-3)
 
 
+def shard_plan(rank: int, world: int, layers: int = LAYERS, hkv: int = HKV) -> dict:
+    """KV-head sharding of one workload over `world` ranks: the KV heads of
+    every layer are split into gcd(world, hkv) equal groups, and when there
+    are more ranks than head groups the layers are split too (world =
+    head groups x layer groups).  Rank r owns KV heads [g0, g1) -- with their
+    query heads [g0 G, g1 G) -- of layers [l0, l1).  Units are independent,
+    so no collective runs in the data path; a following tensor-parallel
+    output projection would consume the head slices as they are."""
+    if world < 1 or not 0 <= rank < world:
+        raise ValueError("bad rank / world")
+    hs = math.gcd(world, hkv)
+    ls = world // hs
+    if ls > layers:
+        raise ValueError(f"{world} ranks cannot share {layers} layers x {hkv} KV heads")
+    hg, lg = rank % hs, rank // hs
+    per = hkv // hs
+    return dict(g0=hg * per, g1=(hg + 1) * per, l0=lg * layers // ls, l1=(lg + 1) * layers // ls,
+                head_groups=hs, layer_groups=ls)
+
+
+def shard_layer(q, k, v, plan: dict, group: int):
+    """The rank's slice of one layer: KV heads [g0, g1) of K and V
+    ([B, Hkv, N, D]) and their query heads of q ([B, Hq, D])."""
+    g0, g1 = plan["g0"], plan["g1"]
+    return q[:, g0 * group:g1 * group], k[:, g0:g1], v[:, g0:g1]
+
+
+def reassemble_heads(parts, plans, group: int, layers: int = LAYERS):
+    """Per-rank outputs [L_r * B, (g1 - g0) * G, D] back to the whole
+    workload's [layers * B, Hkv * G, D] (the inverse of the shard plan; used
+    by the tests, never on the timed path)."""
+    import torch
+    b = parts[0].shape[0] // (plans[0]["l1"] - plans[0]["l0"])
+    hkv = max(p["g1"] for p in plans)
+    full = torch.empty((layers * b, hkv * group) + tuple(parts[0].shape[2:]), dtype=parts[0].dtype)
+    for part, p in zip(parts, plans):
+        full[p["l0"] * b:p["l1"] * b, p["g0"] * group:p["g1"] * group] = part
+    return full
+
+
 # --------------------------------------------------------------------------- GPU arm
-def build_inputs(torch, dev, rank: int, rule: str):
+def build_inputs(torch, dev, rank: int, rule: str, plan: dict | None = None):
+    """The rank's layers stacked along the batch axis.  plan None: the whole
+    workload, seeded per rank (an independent replica); else the rank's
+    shard (shard_plan) of the one workload every rank shares."""
     import block_sparse_kv_page_b200 as sa
     import datagen as DG
-    L = LAYERS
-    k_all = torch.empty((L * B, HKV, N, D), dtype=torch.bfloat16, device=dev)
+    if plan is None:
+        plan = dict(g0=0, g1=HKV, l0=0, l1=LAYERS)
+        seed_off = replica_layer_offset(rank)
+    else:
+        seed_off = 0
+    L = plan["l1"] - plan["l0"]
+    hkv = plan["g1"] - plan["g0"]
+    k_all = torch.empty((L * B, hkv, N, D), dtype=torch.bfloat16, device=dev)
     v_all = torch.empty_like(k_all)
-    q_all = torch.empty((L * B, HQ, D), dtype=torch.bfloat16, device=dev)
-    for l in range(L):
-        lay = DG.workload2_layer(l + replica_layer_offset(rank), dev)
-        k_all[l * B:(l + 1) * B] = lay.k
-        v_all[l * B:(l + 1) * B] = lay.v
-        q_all[l * B:(l + 1) * B] = lay.q
+    q_all = torch.empty((L * B, hkv * G, D), dtype=torch.bfloat16, device=dev)
+    for i, l in enumerate(range(plan["l0"], plan["l1"])):
+        lay = DG.workload2_layer(l + seed_off, dev)
+        q_s, k_s, v_s = shard_layer(lay.q, lay.k, lay.v, plan, G)
+        k_all[i * B:(i + 1) * B] = k_s
+        v_all[i * B:(i + 1) * B] = v_s
+        q_all[i * B:(i + 1) * B] = q_s
         del lay
     seq = torch.full((L * B,), N, dtype=torch.int32, device=dev)
     P = N // PS
     kv_all = sa.KvCache(k_all, v_all, seq, page_size=PS, max_pages=P)
-    return dict(k=k_all, v=v_all, q=q_all, seq=seq, kv=kv_all, P=P)
+    return dict(k=k_all, v=v_all, q=q_all, seq=seq, kv=kv_all, P=P, L=L, hkv=hkv, hq=hkv * G)
 
 
 def per_layer_views(sa, inp):
     kvs = []
-    for l in range(LAYERS):
+    for l in range(inp["L"]):
         sl = slice(l * B, (l + 1) * B)
         kvs.append(sa.KvCache(inp["k"][sl], inp["v"][sl], inp["seq"][sl], page_size=PS,
                               max_pages=inp["P"]))
@@ -322,19 +375,20 @@ def run_gpu_arm(args, rank, world, dist):
     dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", 0)))
     torch.cuda.set_device(dev)
     clocks = ClockSampler(dev.index if dev.index is not None else 0)
-    inp = build_inputs(torch, dev, rank, args.rule)
+    plan = shard_plan(rank, world) if (world > 1 and args.shard == "heads") else None
+    inp = build_inputs(torch, dev, rank, args.rule, plan)
     kv = inp["kv"]
     k = args.budget // PS
     scale = 1.0 / math.sqrt(D)
-    L = LAYERS
+    L, hkv, hq = inp["L"], inp["hkv"], inp["hq"]
     metas = {r: kv.meta_buffer() for r in ("envelope", "centroid")}
     for r, m in metas.items():
         sa.sparse_attn_build_meta(kv, r, 0, m)
-    ws = sa.make_workspace(kv, HQ, L * B, k)
-    sel = torch.zeros((L * B, HKV, k), dtype=torch.int32, device=dev)
-    cnt = torch.zeros((L * B, HKV), dtype=torch.int32, device=dev)
-    out = torch.zeros((L * B, HQ, D), dtype=torch.float32, device=dev)
-    lse = torch.zeros((L * B, HQ), dtype=torch.float32, device=dev)
+    ws = sa.make_workspace(kv, hq, L * B, k)
+    sel = torch.zeros((L * B, hkv, k), dtype=torch.int32, device=dev)
+    cnt = torch.zeros((L * B, hkv), dtype=torch.int32, device=dev)
+    out = torch.zeros((L * B, hq, D), dtype=torch.float32, device=dev)
+    lse = torch.zeros((L * B, hq), dtype=torch.float32, device=dev)
     budget = sa.budget_topk(k)
     stream = torch.cuda.current_stream()
     views = per_layer_views(sa, inp)
@@ -446,25 +500,27 @@ def run_gpu_arm(args, rank, world, dist):
     if kern is None:  # graph modes: the one-launch step's kernel time, labelled as such
         ms_step, _ = timed("step", args.rule, max(3, min(args.steps, 50)), 2)
         kern = {"step": ms_step}
-    tok_heads = args.budget * HQ * L * B
-    value = whole_job_value(tok_heads, world, ms)
-    meta_bytes = L * B * HKV * (N // PS) * 512
-    kv_bytes = L * B * HKV * args.budget * 2 * D * 2
+    tok_heads = args.budget * hq * L * B
+    # work of the whole job per step: the shards of one workload, or N replicas
+    job_tok_heads = args.budget * HQ * LAYERS * B if plan is not None else tok_heads * world
+    value = job_tok_heads / (ms * 1e-3)
+    meta_bytes = L * B * hkv * (N // PS) * 512
+    kv_bytes = L * B * hkv * args.budget * 2 * D * 2
 
     # ---- end to end through the public API with host buffers.  A step's
     # inputs (q, and the newest token's K and V per (layer, KV head)) sit in
     # one pinned host buffer and go over in one copy; the one-launch step
     # stores the newest K/V into the cache itself (the append variant).  The
     # other modes scatter them into the cache with a device copy first.
-    nq, nk = inp["q"].numel(), L * B * HKV * D
+    nq, nk = inp["q"].numel(), L * B * hkv * D
     host_in = torch.empty(nq + 2 * nk, dtype=torch.bfloat16).pin_memory()
     host_in[:nq] = inp["q"].flatten().cpu()
     host_in[nq:nq + nk] = inp["k"][:, :, N - 1, :].flatten().cpu()
     host_in[nq + nk:] = inp["v"][:, :, N - 1, :].flatten().cpu()
     dev_in = torch.empty(host_in.shape, dtype=torch.bfloat16, device=dev)
     q_d = dev_in[:nq].view(inp["q"].shape)
-    knew_d = dev_in[nq:nq + nk].view(L * B, HKV, D)
-    vnew_d = dev_in[nq + nk:].view(L * B, HKV, D)
+    knew_d = dev_in[nq:nq + nk].view(L * B, hkv, D)
+    vnew_d = dev_in[nq + nk:].view(L * B, hkv, D)
     out_h = torch.empty(out.shape, dtype=out.dtype).pin_memory()
 
     def e2e_step():
@@ -564,9 +620,9 @@ def run_gpu_arm(args, rank, world, dist):
                                            "value": tok_heads * world / (m2 * 1e-3),
                                            "eff_GBps": (meta_bytes + kv_bytes) / (m2 * 1e-3) / 1e9}
         # per-query-head selection (one page set per query head), separate calls
-        ws_h = sa.make_workspace_per_head(kv, HQ, k)
-        sel_h = torch.zeros((L * B, HQ, k), dtype=torch.int32, device=dev)
-        cnt_h = torch.zeros((L * B, HQ), dtype=torch.int32, device=dev)
+        ws_h = sa.make_workspace_per_head(kv, hq, k)
+        sel_h = torch.zeros((L * B, hq, k), dtype=torch.int32, device=dev)
+        cnt_h = torch.zeros((L * B, hq), dtype=torch.int32, device=dev)
         for rule in ("envelope", "centroid"):
             def per_head_calls():
                 sa.sparse_attn_build_meta(kv, rule, -1, metas[rule])
@@ -595,13 +651,13 @@ def run_gpu_arm(args, rank, world, dist):
                     torch.cuda.synchronize()
                 m2 = max_over_ranks(e0.elapsed_time(e1) / n_rep, dist, dev)
                 # K/V of the distinct pages the G heads of a KV head keep (the union)
-                sh = sel_h.view(L * B, HKV, HQ // HKV, k).cpu()
-                distinct = sum(int(torch.unique(sh[r, g2]).numel()) for r in range(L * B) for g2 in range(HKV))
+                sh = sel_h.view(L * B, hkv, hq // hkv, k).cpu()
+                distinct = sum(int(torch.unique(sh[r, g2]).numel()) for r in range(L * B) for g2 in range(hkv))
                 kv_union = distinct * PS * 2 * D * 2
                 extra[f"{label}/{rule}"] = {
                     "ms_per_step": round(m2, 4), "value": tok_heads * world / (m2 * 1e-3),
                     "eff_GBps": (meta_bytes + kv_union) / (m2 * 1e-3) / 1e9,
-                    "distinct_pages_per_kv_head": round(distinct / (L * B * HKV), 1),
+                    "distinct_pages_per_kv_head": round(distinct / (L * B * hkv), 1),
                     "note": f"one page set per query head ({how}); effective bytes = metadata once + K/V of "
                             "the union of a KV head's query-head page sets"}
         if sa.sparse_attn_get_device_status(ws_h) != 0:
@@ -618,7 +674,8 @@ def run_gpu_arm(args, rank, world, dist):
         tsa = tsa_leg(torch, dev, max(10, min(args.steps, 50)), max(3, args.warmup), clocks)
         torch.cuda.empty_cache()
         ratio = ratio_leg(torch, dev, max(5, min(args.steps, 20)), max(3, args.warmup), clocks)
-    return dict(ms=ms, value=value, kern=kern, clocks=clocks.summary(), e2e_ms=e2e_ms, e2e_bf16=e2e_bf16,
+    return dict(ms=ms, value=value, job_tok_heads=job_tok_heads, plan=plan, kern=kern, clocks=clocks.summary(),
+                e2e_ms=e2e_ms, e2e_bf16=e2e_bf16,
                 e2e_zc=e2e_zc, h2d=h2d,
                 d2h=d2h, meta_bytes=meta_bytes, kv_bytes=kv_bytes, extra=extra, router=router, tsa=tsa, ratio=ratio,
                 launches_per_step=MODES[args.mode])
@@ -1053,24 +1110,27 @@ def main():
     line = {
         "metric": METRIC, "value": r["value"], "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(r["ms"], 5), "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "scaling": "strong" if r["plan"] is not None else "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic",
         "config": {"workload": WORKLOAD, "layers": LAYERS, "batch": B, "q_heads": HQ, "kv_heads": HKV,
                    "head_dim": D, "context": N, "page_size": PS, "budget_tokens": args.budget,
                    "top_k": args.budget // PS, "rule": args.rule, "mode": args.mode,
-                   "parallelism": f"replicas{world}" if world > 1 else "single",
+                   "parallelism": ("single" if world == 1 else
+                                   f"kvheads{r['plan']['head_groups']}x{r['plan']['layer_groups']}layers"
+                                   if r["plan"] is not None else f"replicas{world}"),
                    "l2": "inputs larger than L2 (~0.58 GB touched per step), no flush"},
         "effective_GBps": round(eff, 1), "effective_frac_of_peak": round(eff / peak, 4),
         "selected_token_fraction": round(args.budget / N, 4),
         "per_kernel_ms": {k: round(v, 5) for k, v in kern.items()} if kern else None,
         "roofline": roof, "clocks": r["clocks"],
-        "e2e": {"value": whole_job_value(HQ * args.budget * LAYERS * B, world, r["e2e_ms"]), "unit": UNIT,
+        "e2e": {"value": r["job_tok_heads"] / (r["e2e_ms"] * 1e-3), "unit": UNIT,
                 "ms_per_step": round(r["e2e_ms"], 5), "h2d_bytes_per_step": r["h2d"],
                 "d2h_bytes_per_step": r["d2h"]},
         "e2e_bf16_out": None if r["e2e_bf16"] is None else {
-            "value": whole_job_value(HQ * args.budget * LAYERS * B, world, r["e2e_bf16"]["ms_per_step"]),
+            "value": r["job_tok_heads"] / (r["e2e_bf16"]["ms_per_step"] * 1e-3),
             "unit": UNIT, **r["e2e_bf16"]},
         "e2e_host_written_out": None if r["e2e_zc"] is None else {
-            "value": whole_job_value(HQ * args.budget * LAYERS * B, world, r["e2e_zc"]["ms_per_step"]),
+            "value": r["job_tok_heads"] / (r["e2e_zc"]["ms_per_step"] * 1e-3),
             "unit": UNIT, **r["e2e_zc"]},
         "gpu_launches": r["launches_per_step"] * args.steps,
         "cpu_baseline": cpu, "modes": r["extra"],

@@ -15,22 +15,19 @@
 //   warp 9 + t (one thread) issues, for Q tile t and block i in order,
 //                        S = Q_t K_i^T (M = 128 vectors, N = 64 keys, K = 128
 //                        dims; K-major operands) into one of the tile's two
-//                        S/P buffers, then O_t += P . V_{i-1} (A = P read
-//                        from tensor memory, N = 128 dims, K = 64 keys; V
-//                        read MN-major) once P_{i-1} is written; the tensor
-//                        pipe interleaves the
+//                        S/P buffers, then O_t += [P_hi | P_lo] . [V_{i-1} ;
+//                        V_{i-1}] (A = P read from tensor memory, N = 128
+//                        dims, K = 2 x 64 keys; V read MN-major) once
+//                        P_{i-1} is written; the tensor pipe interleaves the
 //                        two tiles' MMAs, so one tile's softmax and handoffs
 //                        overlap the other tile's MMAs;
 //   warps 0-3 / 4-7      the softmax of tile 0 / 1: thread = query vector
 //                        (TMEM lane 32 (warp % 4) + lane), its whole row of
 //                        64 keys: masks (causal, cache end) only on the
 //                        diagonal and cache-end blocks, online softmax in the
-//                        log2 domain against a reference max, P rounded to
-//                        bf16 and stored over S in tensor memory as the PV
-//                        MMA's A operand; the row sum adds the rounded
-//                        weights, so the output is an exact convex
-//                        combination of V rows with weights within 2^-9
-//                        (relative) of the softmax's.
+//                        log2 domain against a reference max, P split into a
+//                        bf16 hi + lo pair (error ~2^-17) stored over S in
+//                        tensor memory as the PV MMA's A operand.
 // O stays in tensor memory; it is rescaled in place only when a row's max
 // grows past the reference by more than 2^8.  The MMAs of one issuing thread
 // run in issue order, so the S/P buffer of block i + 2 is written only after
@@ -258,9 +255,9 @@ __global__ void __launch_bounds__(kThreadsTc, 1) tile_attn_tc_kernel(const __gri
         tc::fence_after_sync();
         const unsigned char* vb = ring + s * kStage + 2 * kBox;
 #pragma unroll
-        for (int j = 0; j < 4; ++j)  // K = 64 keys of P, 16 per step (8 columns of bf16 pairs)
+        for (int j = 0; j < 8; ++j)  // K = [P_hi keys 0-63 | P_lo keys 0-63], 16 per step
           tc::mma_bf16_ts(tmem + kColO + 128u * tt, tmem + kColSP + 128u * tt + 64u * b + 8u * j,
-                          v_desc(vb + 16 * 128 * j), idesc_o, i > 0 || j != 0);
+                          v_desc(vb + 16 * 128 * (j & 3)), idesc_o, i > 0 || j != 0);
         tc::commit(o_full + 2 * tt + b);
         tc::commit(kv_empty + s);
         return true;
@@ -381,20 +378,22 @@ __global__ void __launch_bounds__(kThreadsTc, 1) tile_attn_tc_kernel(const __gri
         }
       }
       const float nmn = mref == ninf ? 0.f : -mref;  // all masked so far: every p is exp2(-inf) = 0
-      // P = exp2(s - mref) rounded to bf16, as pairs in columns 0-31 over S
-      // (S of this block was read above); the row sum adds the rounded values
+      // P = exp2(s - mref) as bf16 hi + lo pairs over S: hi pairs in columns
+      // 0-31, lo pairs in 32-63 (S of this block was read above)
       float rq[4] = {0.f, 0.f, 0.f, 0.f};  // four independent partial row sums
 #pragma unroll
       for (int h2 = 0; h2 < 2; ++h2) {
-        uint32_t ph[16];
+        uint32_t phi[16], plo[16];
 #pragma unroll
         for (int j = 0; j < 16; ++j) {
           const float p0 = fast_exp2(fmaf(sv[32 * h2 + 2 * j], mul, nmn));
           const float p1 = fast_exp2(fmaf(sv[32 * h2 + 2 * j + 1], mul, nmn));
-          ph[j] = pack_bf16(p0, p1);
-          rq[j & 3] += bf16_lo(ph[j]) + bf16_hi(ph[j]);
+          rq[j & 3] += p0 + p1;
+          phi[j] = pack_bf16(p0, p1);
+          plo[j] = pack_bf16(p0 - bf16_lo(phi[j]), p1 - bf16_hi(phi[j]));
         }
-        tc::st_32x32b_x16(ts + 16 * h2, ph);
+        tc::st_32x32b_x16(ts + 16 * h2, phi);
+        tc::st_32x32b_x16(ts + 32 + 16 * h2, plo);
       }
       lh += (rq[0] + rq[1]) + (rq[2] + rq[3]);
       // V rows past the cache end hold other data: zero them before PV reads
