@@ -122,12 +122,72 @@ SA_DEV void store_out(const DecodeArgs& a, size_t row, int d0, const float (&A)[
   }
 }
 
+// Merge of a unit's split partials for head h, dims d0 .. d0 + 7, in split
+// order, kMergeBatch partials per batch with every load of a batch issued
+// before any is used (each dependent round trip to L2 costs about a
+// microsecond under full HBM load).  base = slot 0 of the unit, head h;
+// LOCAL: the partials are in (this CTA's) shared memory, else in global
+// memory written earlier in the launch.  The same arithmetic either way.
+template <bool LOCAL>
+SA_DEV void merge_splits(const DecodeArgs& a, const float* base, const int splits, const size_t out_row,
+                         const int d0) {
+  const float ninf = -__int_as_float(0x7f800000);
+  float MM = ninf, LL = 0.f, AA[kDimsPerThread];
+#pragma unroll
+  for (int x = 0; x < kDimsPerThread; ++x) AA[x] = 0.f;
+  for (int sp0 = 0; sp0 < splits; sp0 += kMergeBatch) {
+    float2 ml[kMergeBatch];
+    float4 v[kMergeBatch][kDimsPerThread / 4];
+#pragma unroll
+    for (int j = 0; j < kMergeBatch; ++j) {
+      const bool ok = sp0 + j < splits;
+      const float* src = base + (size_t)(ok ? sp0 + j : 0) * kPartStride;
+      const float2* pml = reinterpret_cast<const float2*>(src + kHeadDim);
+      ml[j] = ok ? (LOCAL ? *pml : __ldcg(pml)) : make_float2(ninf, 0.f);
+#pragma unroll
+      for (int q4 = 0; q4 < kDimsPerThread / 4; ++q4) {
+        const float4* pv = reinterpret_cast<const float4*>(src + d0) + q4;
+        v[j][q4] = ok ? (LOCAL ? *pv : __ldcg(pv)) : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+    }
+    float nm = MM;
+#pragma unroll
+    for (int j = 0; j < kMergeBatch; ++j) nm = fmaxf(nm, ml[j].x);
+    if (nm == ninf) continue;
+    const float fo = exp2f(MM - nm);  // 0 while nothing has been merged
+    LL *= fo;
+#pragma unroll
+    for (int x = 0; x < kDimsPerThread; ++x) AA[x] *= fo;
+#pragma unroll
+    for (int j = 0; j < kMergeBatch; ++j) {
+      const float f = exp2f(ml[j].x - nm);
+      LL += ml[j].y * f;
+#pragma unroll
+      for (int q4 = 0; q4 < kDimsPerThread / 4; ++q4) {
+        AA[4 * q4 + 0] += v[j][q4].x * f;
+        AA[4 * q4 + 1] += v[j][q4].y * f;
+        AA[4 * q4 + 2] += v[j][q4].z * f;
+        AA[4 * q4 + 3] += v[j][q4].w * f;
+      }
+    }
+    MM = nm;
+  }
+  const float inv = LL > 0.f ? 1.f / LL : 0.f;
+  store_out(a, out_row, d0, AA, inv);
+  if (a.lse && d0 == 0) a.lse[out_row] = LL > 0.f ? MM * kLn2 + logf(LL) : ninf;
+}
+
 // n_known >= 0: the unit's kept count, already read by the caller (the fused
 // step takes it from the unit's selection flag); else it is loaded here.
 // n_tok_known >= 0 likewise stands for the sequence length.
-template <bool PER_HEAD = false>
+// STAGES: depth of the per-warp TMA ring (its barriers: sm.bars[warp][STAGES]).
+// part_dst (several splits only): write the split's partial to part_dst +
+// split * kPartStride (another CTA's shared memory, say) and return; the
+// caller merges (merge_splits) once every split's partial is there.
+template <bool PER_HEAD = false, int STAGES = kStages>
 SA_DEV void decode_item(const DecodeArgs& a, const int u, const int split, const Smem& sm,
-                        WarpState& ws, const int n_known = -1, const int n_tok_known = -1) {
+                        WarpState& ws, const int n_known = -1, const int n_tok_known = -1,
+                        float* part_dst = nullptr) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int gq = lane >> 2, c = lane & 3;
   const UnitMap um = unit_map<PER_HEAD>(u, a.kv.Hkv, a.Hq, a.G);
@@ -232,8 +292,8 @@ SA_DEV void decode_item(const DecodeArgs& a, const int u, const int split, const
 #pragma unroll
   for (int mt = 0; mt < 8; ++mt) acc[mt][0] = acc[mt][1] = acc[mt][2] = acc[mt][3] = 0.f;
 
-  unsigned char* ring = sm.ring + warp * (kStages * kTileBytes);
-  uint64_t* bars = sm.bars + warp * kStages;
+  unsigned char* ring = sm.ring + warp * (STAGES * kTileBytes);
+  uint64_t* bars = sm.bars + warp * STAGES;
   // ldmatrix lane addressing: matrix = lane / 8, row-in-matrix = lane % 8
   const int lrow_a = (lane & 7) + 8 * ((lane >> 3) & 1);  // K: rows 0-7 / 8-15
   const int lchk_a = lane >> 4;                            //    chunk +0 / +1
@@ -250,8 +310,8 @@ SA_DEV void decode_item(const DecodeArgs& a, const int u, const int split, const
       const int t = warp + it * kWarps;
       if (t >= nt) return;
       const uint32_t g_it = ws.gi + (uint32_t)it;
-      uint64_t* bar = bars + g_it % kStages;
-      unsigned char* st = ring + (g_it % kStages) * kTileBytes;
+      uint64_t* bar = bars + g_it % STAGES;
+      unsigned char* st = ring + (g_it % STAGES) * kTileBytes;
       const TileRef r = sm.tiles[t];
       if (r.n == 0) {
         mbar_arrive(bar);  // nothing to load: complete the phase
@@ -265,25 +325,25 @@ SA_DEV void decode_item(const DecodeArgs& a, const int u, const int split, const
     };
     int issued = 0;  // tiles of this round issued so far (identical on every lane)
     if (ws.alive) {
-      issued = min(n_it, kStages - 1);
+      issued = min(n_it, STAGES - 1);
       if (lane == 0)
         for (int it = 0; it < issued; ++it) issue(it);
     }
 
     for (int it = 0; it < n_it && ws.alive; ++it) {
       __syncwarp();  // every lane is done reading the stage about to be refilled
-      if (it + kStages - 1 < n_it) {
-        if (lane == 0) issue(it + kStages - 1);
-        issued = it + kStages;
+      if (it + STAGES - 1 < n_it) {
+        if (lane == 0) issue(it + STAGES - 1);
+        issued = it + STAGES;
       }
       const uint32_t g_it = ws.gi + (uint32_t)it;
-      if (!mbar_wait(bars + g_it % kStages, (g_it / kStages) & 1u, a.status)) {
+      if (!mbar_wait(bars + g_it % STAGES, (g_it / STAGES) & 1u, a.status)) {
         ws.alive = false;
         ws.drain_lo = g_it;
         ws.drain_hi = ws.gi + (uint32_t)issued;
         break;
       }
-      unsigned char* st = ring + (g_it % kStages) * kTileBytes;
+      unsigned char* st = ring + (g_it % STAGES) * kTileBytes;
       const TileRef r = sm.tiles[warp + it * kWarps];
       if (r.n < 16) {  // zero V rows past the valid tokens (they may hold other data)
         for (int x = lane; x < (16 - r.n) * 16; x += 32) {
@@ -406,7 +466,17 @@ SA_DEV void decode_item(const DecodeArgs& a, const int u, const int split, const
     return;
   }
 
-  // ---- several splits: publish the partial; the last CTA of the unit merges
+  // ---- several splits: publish the partial; the merge runs once all are in
+  if (part_dst != nullptr) {
+    if (h < G) {
+      float* dst = part_dst + (size_t)split * kPartStride + h * kPartHead;
+#pragma unroll
+      for (int x = 0; x < kDimsPerThread; x += 4)
+        *reinterpret_cast<float4*>(dst + d0 + x) = make_float4(A[x], A[x + 1], A[x + 2], A[x + 3]);
+      if (d0 == 0) *reinterpret_cast<float2*>(dst + kHeadDim) = make_float2(M, L);
+    }
+    return;
+  }
   float* part = a.ws_part + (slot0 + split) * kPartStride;
   if (h < G) {
     float* dst = part + h * kPartHead;
@@ -426,51 +496,7 @@ SA_DEV void decode_item(const DecodeArgs& a, const int u, const int split, const
   if (!*sm.last) return;
   if (tid == 0) a.ws_count[u] = 0;
   if (h >= G) return;
-
-  // Merge in split order, kMergeBatch partials per batch with every load of a
-  // batch issued before any is used (each dependent round trip to L2 costs
-  // about a microsecond under full HBM load).
-  const float* base = a.ws_part + slot0 * kPartStride + h * kPartHead;
-  float MM = ninf, LL = 0.f, AA[kDimsPerThread];
-#pragma unroll
-  for (int x = 0; x < kDimsPerThread; ++x) AA[x] = 0.f;
-  for (int sp0 = 0; sp0 < splits; sp0 += kMergeBatch) {
-    float2 ml[kMergeBatch];
-    float4 v[kMergeBatch][kDimsPerThread / 4];
-#pragma unroll
-    for (int j = 0; j < kMergeBatch; ++j) {
-      const bool ok = sp0 + j < splits;
-      const float* src = base + (size_t)(ok ? sp0 + j : 0) * kPartStride;
-      ml[j] = ok ? __ldcg(reinterpret_cast<const float2*>(src + kHeadDim)) : make_float2(ninf, 0.f);
-#pragma unroll
-      for (int q4 = 0; q4 < kDimsPerThread / 4; ++q4)
-        v[j][q4] = ok ? __ldcg(reinterpret_cast<const float4*>(src + d0) + q4) : make_float4(0.f, 0.f, 0.f, 0.f);
-    }
-    float nm = MM;
-#pragma unroll
-    for (int j = 0; j < kMergeBatch; ++j) nm = fmaxf(nm, ml[j].x);
-    if (nm == ninf) continue;
-    const float fo = exp2f(MM - nm);  // 0 while nothing has been merged
-    LL *= fo;
-#pragma unroll
-    for (int x = 0; x < kDimsPerThread; ++x) AA[x] *= fo;
-#pragma unroll
-    for (int j = 0; j < kMergeBatch; ++j) {
-      const float f = exp2f(ml[j].x - nm);
-      LL += ml[j].y * f;
-#pragma unroll
-      for (int q4 = 0; q4 < kDimsPerThread / 4; ++q4) {
-        AA[4 * q4 + 0] += v[j][q4].x * f;
-        AA[4 * q4 + 1] += v[j][q4].y * f;
-        AA[4 * q4 + 2] += v[j][q4].z * f;
-        AA[4 * q4 + 3] += v[j][q4].w * f;
-      }
-    }
-    MM = nm;
-  }
-  const float inv = LL > 0.f ? 1.f / LL : 0.f;
-  store_out(a, out_row, d0, AA, inv);
-  if (a.lse && d0 == 0) a.lse[out_row] = LL > 0.f ? MM * kLn2 + logf(LL) : ninf;
+  merge_splits<false>(a, a.ws_part + slot0 * kPartStride + h * kPartHead, splits, out_row, d0);
 }
 
 }  // namespace dec

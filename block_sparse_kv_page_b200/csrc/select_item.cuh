@@ -90,11 +90,11 @@ struct SelSmem {
 // Selection from keys staged in shared memory (any P up to max_pages).
 SA_DEV void select_unit_smem(const SelectArgs& a, const int u, const int N, const int P,
                              const uint32_t cap, const int forced_lo, const int forced_hi,
-                             const int32_t* off, const SelSmem& S) {
+                             const int32_t* off, const SelSmem& S, const float* sc_local) {
   const int tid = threadIdx.x;
   uint32_t* keys = reinterpret_cast<uint32_t*>(S.ring);
   uint32_t* wts = keys + a.kv.max_pages;
-  const float* sc_u = a.ws_scores + (size_t)u * a.ws_stride;
+  const float* sc_u = sc_local ? sc_local : a.ws_scores + (size_t)u * a.ws_stride;
   const bool weighted = off != nullptr;
   // Keys (and chunk weights) into shared memory.  Every thread issues all its
   // loads of a batch before using any: under full HBM load each dependent
@@ -107,7 +107,8 @@ SA_DEV void select_unit_smem(const SelectArgs& a, const int u, const int N, cons
 #pragma unroll
     for (int j = 0; j < kSelBatch; ++j) {
       const int i4 = base4 + j * (int)blockDim.x + tid;
-      v[j] = i4 < P4 ? __ldcg(reinterpret_cast<const float4*>(sc_u) + i4) : make_float4(0.f, 0.f, 0.f, 0.f);
+      const float4* src = reinterpret_cast<const float4*>(sc_u) + i4;
+      v[j] = i4 < P4 ? (sc_local ? *src : __ldcg(src)) : make_float4(0.f, 0.f, 0.f, 0.f);
       if (weighted) {
 #pragma unroll
         for (int e = 0; e < 5; ++e) o[j][e] = (i4 < P4 && 4 * i4 + e <= P) ? off[4 * i4 + e] : 0;
@@ -218,11 +219,11 @@ SA_DEV uint32_t bin_slot(uint32_t b) {  // physical word of bin b in a 4096-bin 
 template <int KPT, bool WEIGHTED>
 SA_DEV void select_unit_regs(const SelectArgs& a, const int u, const int N, const int P,
                              const uint32_t cap, const int forced_lo, const int forced_hi,
-                             const int32_t* off, const SelSmem& S) {
+                             const int32_t* off, const SelSmem& S, const float* sc_local) {
   static_assert(KPT % 4 == 0 && KPT <= 32, "pages per thread");
   static_assert(kThreads == 128, "the register path maps 4096 bins onto 128 threads");
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const float* sc_u = a.ws_scores + (size_t)u * a.ws_stride;
+  const float* sc_u = sc_local ? sc_local : a.ws_scores + (size_t)u * a.ws_stride;
   const int p0 = tid * KPT;
   uint32_t* H0 = reinterpret_cast<uint32_t*>(S.ring);  // [2][4096] bins
   uint32_t* tsum = H0 + 2 * 4096;                       // [128] row sums
@@ -232,9 +233,10 @@ SA_DEV void select_unit_regs(const SelectArgs& a, const int u, const int N, cons
     // every load issued before any is used (one round trip to L2)
     float4 v[KPT / 4];
 #pragma unroll
-    for (int q = 0; q < KPT / 4; ++q)
-      v[q] = p0 + 4 * q < P ? __ldcg(reinterpret_cast<const float4*>(sc_u + p0) + q)
-                            : make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int q = 0; q < KPT / 4; ++q) {
+      const float4* src = reinterpret_cast<const float4*>(sc_u + p0) + q;
+      v[q] = p0 + 4 * q < P ? (sc_local ? *src : __ldcg(src)) : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
     int o[WEIGHTED ? KPT + 1 : 1];
     if (WEIGHTED) {
 #pragma unroll
@@ -434,10 +436,11 @@ SA_DEV void select_unit_regs(const SelectArgs& a, const int u, const int N, cons
   }
 }
 
-// Selection of unit u from its scores in the workspace: writes sel_idx
-// (ascending page order) and sel_count.  All threads of the CTA call it.
+// Selection of unit u from its scores -- in the workspace, or at sc_local in
+// this CTA's shared memory (16-byte aligned, rows padded to 4): writes
+// sel_idx (ascending page order) and sel_count.  All threads of the CTA call it.
 SA_DEV void select_unit(const SelectArgs& a, const int u, const int b, const int N, const int P,
-                        const SelSmem& S) {
+                        const SelSmem& S, const float* sc_local = nullptr) {
   const bool weighted = a.budget_kind == SA_BUDGET_TOKENS;
   const int32_t* off = weighted ? a.kv.chunk_off + (size_t)b * (a.kv.max_pages + 1) : nullptr;
   int forced_lo = 0, forced_hi = P;  // pages < forced_lo or >= forced_hi are forced (ratio)
@@ -457,11 +460,11 @@ SA_DEV void select_unit(const SelectArgs& a, const int u, const int b, const int
   }
   if (P <= 16 * kThreads) {
     if (weighted)
-      select_unit_regs<16, true>(a, u, N, P, cap, forced_lo, forced_hi, off, S);
+      select_unit_regs<16, true>(a, u, N, P, cap, forced_lo, forced_hi, off, S, sc_local);
     else
-      select_unit_regs<16, false>(a, u, N, P, cap, forced_lo, forced_hi, off, S);
+      select_unit_regs<16, false>(a, u, N, P, cap, forced_lo, forced_hi, off, S, sc_local);
   } else
-    select_unit_smem(a, u, N, P, cap, forced_lo, forced_hi, off, S);
+    select_unit_smem(a, u, N, P, cap, forced_lo, forced_hi, off, S, sc_local);
 }
 
 // Tokens N and pages (or chunks) P of sequence b; false (and P = 0) when
@@ -481,21 +484,24 @@ SA_DEV bool unit_geometry(const SelectArgs& a, const int b, int& N, int& P) {
 }
 
 // Selection of unit u (sequence, KV head) from the group scores its scoring
-// items wrote; the caller has made them visible to this CTA.
-SA_DEV void select_unit_of(const SelectArgs& a, const int u, const SelSmem& S) {
+// items wrote (at sc_local in shared memory, or in the workspace); the caller
+// has made them visible to this CTA.
+SA_DEV void select_unit_of(const SelectArgs& a, const int u, const SelSmem& S, const float* sc_local) {
   const int b = u / a.kv.Hkv;
   int N, P;
   unit_geometry(a, b, N, P);  // a bad geometry was flagged by the scoring
-  select_unit(a, u, b, N, P, S);
+  select_unit(a, u, b, N, P, S, sc_local);
 }
 
 // FUSED (the decode step): refresh the newest page while scoring and publish
 // the unit's flag after selecting.
 // SCORE_ONLY: write the group scores and stop (no selection; the unit
 // counters are not touched).
+// score_dst (non-null): where the unit's group scores go, indexed by page
+// (another CTA's shared memory, say), instead of the workspace.
 template <int RULE, bool FUSED, bool PER_HEAD = false, bool SCORE_ONLY = false>
 SA_DEV void select_item(const SelectArgs& a, const int u, const int split, const SelSmem& S,
-                        WarpState& ws) {
+                        WarpState& ws, float* score_dst = nullptr) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int gq = lane >> 2, c = lane & 3;
   const int Hkv = a.kv.Hkv;
@@ -544,7 +550,7 @@ SA_DEV void select_item(const SelectArgs& a, const int u, const int split, const
   }
 
   // ---- scoring: warp w takes tiles t_begin + w, + 4, ...
-  float* sc_u = a.ws_scores + (size_t)u * a.ws_stride;
+  float* sc_u = score_dst ? score_dst : a.ws_scores + (size_t)u * a.ws_stride;
   float* out_u = a.scores_out ? a.scores_out + (size_t)u * a.kv.max_pages : nullptr;
   unsigned char* ring = S.ring + warp * (kStages * kTileBytes);
   uint64_t* bars = S.bars + warp * kStages;

@@ -22,10 +22,14 @@
 // All item kinds share one per-warp TMA ring (same stage count and tile size),
 // so one WarpState carries the ring position from item to item.  The last CTA
 // out clears the unit flags and split counters and rewinds the queue.
+#include <cooperative_groups.h>
+
 #include "common.cuh"
 #include "internal.h"
 #include "decode_item.cuh"
 #include "select_item.cuh"
+
+namespace cg = cooperative_groups;
 
 #ifndef SA_STEP_CTAS_PER_SM
 #define SA_STEP_CTAS_PER_SM 3
@@ -162,14 +166,43 @@ __global__ void __launch_bounds__(kThreads, SA_STEP_CTAS_PER_SM)
 }
 
 // The decode step for few units (a single layer at batch 1, say): one
-// thread-block cluster of C CTAs per unit (sequence, KV head), so the
-// handoffs between stages are hardware cluster barriers instead of global
-// item claims and flag polls.  CTA r of the cluster scores tile range r of C
-// (the one holding the newest page also refreshes it); after a cluster
-// barrier the leader (rank 0) selects the unit's pages; after another, CTA r
-// runs decode splits r, r + C, ... of the unit, merged by the last of them
-// as in the persistent kernel.  The same item code with the same splits as
-// the separate calls, so results are identical to them.
+// thread-block cluster of C CTAs per unit (sequence, KV head), one CTA per
+// SM, so the handoffs between stages are cluster barriers and distributed
+// shared memory instead of global item claims, flag polls and L2 round trips:
+//  1. CTA r scores tile range r of C (the one holding the newest page also
+//     refreshes it) and writes the group scores straight into the leader's
+//     (rank 0) shared memory;
+//  2. cluster barrier; the leader selects the unit's pages from its shared
+//     memory and writes them out;
+//  3. cluster barrier; CTA r runs decode splits r, r + C, ... with a deeper
+//     TMA ring (kClStages per warp: a split's tiles are all in flight at
+//     once).  With exactly C splits each CTA writes its partial into the
+//     leader's shared memory and, after a last barrier, the leader merges
+//     them; with more, the splits merge through the workspace as in the
+//     persistent kernel.
+// The same item code and splits as the separate calls and the same merge
+// arithmetic, so results are identical to them.
+constexpr int kClStages = 4;  // decode ring depth per warp in the cluster kernel
+
+struct ClusterLayout {
+  int ring, bars_sel, bars_dec, tiles, pre, scores, parts, total;
+};
+__host__ __device__ inline ClusterLayout cluster_layout(int max_pages, int max_sel, bool chunks, int C,
+                                                        bool local_merge) {
+  ClusterLayout L;
+  const int dec_ring = dec::kWarps * kClStages * dec::kTileBytes;
+  const int sel_body = body_bytes(max_pages);
+  L.ring = 0;
+  L.bars_sel = sel_body > dec_ring ? sel_body : dec_ring;
+  L.bars_dec = L.bars_sel + kBarBytes;
+  L.tiles = L.bars_dec + dec::kWarps * kClStages * 8;
+  L.pre = L.tiles + kTileRefBytes;
+  L.scores = (L.pre + (chunks ? (max_sel + 1) * 4 : 0) + 15) & ~15;
+  L.parts = (L.scores + ((max_pages + 3) & ~3) * 4 + 15) & ~15;
+  L.total = L.parts + (local_merge ? C * dec::kPartStride * 4 : 0);
+  return L;
+}
+
 template <int RULE>
 __global__ void __launch_bounds__(kThreads, 1) step_cluster_kernel(const __grid_constant__ StepArgs a) {
   extern __shared__ unsigned char smem_raw[];
@@ -179,15 +212,25 @@ __global__ void __launch_bounds__(kThreads, 1) step_cluster_kernel(const __grid_
   __shared__ int s_last, s_ntiles;
   unsigned char* base = reinterpret_cast<unsigned char*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-  const int body = body_bytes(a.sel.kv.max_pages);
-  uint64_t* bars = reinterpret_cast<uint64_t*>(base + body);
-  const sel::SelSmem S{base, bars, s_hist, s_scan, s_bc, &s_last};
-  const dec::Smem D{base, bars, reinterpret_cast<dec::TileRef*>(base + body + kBarBytes),
-                    reinterpret_cast<int*>(base + body + kBarBytes + kTileRefBytes), s_scan, &s_last,
-                    &s_ntiles};
+  const int r = (int)cluster_ctarank(), C = (int)cluster_nctarank();
+  const int u = (int)cluster_id_x();
+  const bool local_merge = a.dec.splits == C;
+  const ClusterLayout Lo = cluster_layout(a.sel.kv.max_pages, a.dec.max_sel, a.sel.kv.page_size == 0, C,
+                                          local_merge);
+  uint64_t* bars_sel = reinterpret_cast<uint64_t*>(base + Lo.bars_sel);
+  uint64_t* bars_dec = reinterpret_cast<uint64_t*>(base + Lo.bars_dec);
+  float* my_scores = reinterpret_cast<float*>(base + Lo.scores);
+  float* my_parts = reinterpret_cast<float*>(base + Lo.parts);
+  const sel::SelSmem S{base, bars_sel, s_hist, s_scan, s_bc, &s_last};
+  const dec::Smem D{base, bars_dec, reinterpret_cast<dec::TileRef*>(base + Lo.tiles),
+                    reinterpret_cast<int*>(base + Lo.pre), s_scan, &s_last, &s_ntiles};
+  cg::cluster_group cl = cg::this_cluster();
+  float* lead_scores = cl.map_shared_rank(my_scores, 0);
+  float* lead_parts = cl.map_shared_rank(my_parts, 0);
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   if (lane == 0) {
-    for (int s = 0; s < kStages; ++s) mbar_init(bars + warp * kStages + s, 1);
+    for (int s = 0; s < kStages; ++s) mbar_init(bars_sel + warp * kStages + s, 1);
+    for (int s = 0; s < kClStages; ++s) mbar_init(bars_dec + warp * kClStages + s, 1);
     fence_barrier_init();
   }
   if (threadIdx.x == 0) {
@@ -198,30 +241,42 @@ __global__ void __launch_bounds__(kThreads, 1) step_cluster_kernel(const __grid_
   __syncthreads();
   grid_dep_wait();     // the previous kernel of the stream has completed (no global access before)
   grid_dep_trigger();  // the next kernel may be scheduled now; it waits for this one to complete
-  const int r = (int)cluster_ctarank(), C = (int)cluster_nctarank();
-  const int u = (int)cluster_id_x();
   WarpState ws{0u, true, 0u, 0u};
-  // 1. scoring of tile range r of C (a.sel.splits == C)
-  sel::select_item<RULE, true, false, true>(a.sel, u, r, S, ws);
-  fence_proxy_async();  // generic writes to the ring (the refresh patch) before its next TMA writes
+  // 1. scoring of tile range r of C (a.sel.splits == C), scores to the leader
+  sel::select_item<RULE, true, false, true>(a.sel, u, r, S, ws, lead_scores);
+  if (!ws.alive && lane == 0) {  // a wait timed out: let the copies in flight land (bounded)
+    for (uint32_t g = ws.drain_lo; g < ws.drain_hi; ++g)
+      mbar_wait(bars_sel + warp * kStages + g % kStages, (g / kStages) & 1u, nullptr);
+  }
+  fence_proxy_async();  // generic writes to the ring (the refresh patch) before it is reused
   __syncthreads();
-  cluster_sync();       // every range's scores are visible to the leader
+  cluster_sync();       // every range's scores are in the leader's shared memory
   // 2. the leader selects
-  if (r == 0) sel::select_unit_of(a.sel, u, S);
-  fence_proxy_async();  // the ring held the keys
+  if (r == 0) sel::select_unit_of(a.sel, u, S, my_scores);
+  fence_proxy_async();  // the ring held the keys: generic writes before the decode TMA writes
   __syncthreads();
   cluster_sync();       // the selection is visible to every CTA of the cluster
   // 3. decode splits r, r + C, ... (each reads the kept count and pages)
   if (a.sel.k_new != nullptr && lane == 0) fence_proxy_async_global();  // appended rows, then TMA
+  WarpState wd{0u, ws.alive, 0u, 0u};
   for (int split = r; split < a.dec.splits; split += C) {
-    dec::decode_item<false>(a.dec, u, split, D, ws);
+    dec::decode_item<false, kClStages>(a.dec, u, split, D, wd, -1, -1, local_merge ? lead_parts : nullptr);
     fence_proxy_async();
     __syncthreads();
   }
-  if (!ws.alive && lane == 0) {  // a wait timed out: let the copies in flight land (bounded)
-    uint64_t* wb = bars + warp * kStages;
-    for (uint32_t g = ws.drain_lo; g < ws.drain_hi; ++g)
-      mbar_wait(wb + g % kStages, (g / kStages) & 1u, nullptr);
+  if (!wd.alive && ws.alive && lane == 0) {  // a wait timed out: let the copies in flight land (bounded)
+    for (uint32_t g = wd.drain_lo; g < wd.drain_hi; ++g)
+      mbar_wait(bars_dec + warp * kClStages + g % kClStages, (g / kClStages) & 1u, nullptr);
+  }
+  if (local_merge) {
+    cluster_sync();  // every split's partial is in the leader's shared memory
+    const int h = threadIdx.x / dec::kThreadsPerHead;
+    const int d0 = (threadIdx.x % dec::kThreadsPerHead) * dec::kDimsPerThread;
+    if (r == 0 && h < a.dec.G) {
+      const int b = u / a.dec.kv.Hkv, g = u - b * a.dec.kv.Hkv;
+      dec::merge_splits<true>(a.dec, my_parts + h * dec::kPartHead, C,
+                              (size_t)b * a.dec.Hq + (size_t)g * a.dec.G + h, d0);
+    }
   }
 }
 
@@ -269,7 +324,10 @@ int step_cluster_size(int units, int dec_splits, int sm_count) {
 }
 
 cudaError_t launch_step_cluster(const StepArgs& a, int C, cudaStream_t st) {
-  size_t smem = step_smem_bytes(a.sel.kv.max_pages, a.dec.max_sel, a.sel.kv.page_size == 0);
+  const ClusterLayout Lo = cluster_layout(a.sel.kv.max_pages, a.dec.max_sel, a.sel.kv.page_size == 0, C,
+                                          a.dec.splits == C);
+  size_t smem = 1024 + (size_t)Lo.total;
+  if (smem > 227 * 1024) return cudaErrorInvalidValue;
   if (smem < kClusterMinSmem) smem = kClusterMinSmem;  // one CTA per SM
   const int units = a.sel.kv.B * a.sel.kv.Hkv;
   const void* fn = a.sel.rule == 0 ? (const void*)step_cluster_kernel<0> : (const void*)step_cluster_kernel<1>;
