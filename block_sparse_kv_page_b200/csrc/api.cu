@@ -553,7 +553,9 @@ static sa_status decode_step(const sa_kv_desc* kv, void* meta, sa_score_rule rul
   if (!std::isfinite(scale)) return SA_ERR_INVALID;
   if (kv->page_size == 0 && max_sel > kMaxChunkSel) return SA_ERR_UNSUPPORTED;
   const long long units = (long long)kv->batch * (per_head ? n_q_heads : kv->n_kv_heads);
-  if (2 * units > kMaxUnits) return SA_ERR_UNSUPPORTED;  // unit flags + split counters
+  const long long kv_units = (long long)kv->batch * kv->n_kv_heads;
+  // unit flags + split counters (+ per-head step: scoring counts per KV head)
+  if (2 * units + (per_head ? kv_units : 0) > kMaxUnits) return SA_ERR_UNSUPPORTED;
   const unsigned long long kv_rows = (unsigned long long)kv->batch * kv->n_kv_heads * kv->cap_tokens;
   if (kv_rows > 0x7fffffffULL) return SA_ERR_UNSUPPORTED;  // TMA row coordinates are int32
   const int sm = device_sm_count();
@@ -580,9 +582,12 @@ static sa_status decode_step(const sa_kv_desc* kv, void* meta, sa_score_rule rul
     return SA_ERR_CUDA;
   if (out_bf16) a.dec.out_bf16 = static_cast<__nv_bfloat16*>(out);
   if (per_head) {
+    // scoring items per (sequence, KV head) write the G heads' rows; then one
+    // selection item per (sequence, query head)
     a.sel.per_head = 1;
-    a.sel.splits = select_splits((int)units, kv->max_pages, sm);
+    a.sel.kv_scored = reinterpret_cast<uint32_t*>(w + 256) + 2 * units;
     a.dec.per_head = 1;
+    a.n_sel = (int)units;
   }
   a.sel.meta_refresh = static_cast<unsigned char*>(meta);
   if (k_new) {
@@ -605,8 +610,8 @@ static sa_status decode_step(const sa_kv_desc* kv, void* meta, sa_score_rule rul
     if (launch_step_cluster(c, C, (cudaStream_t)stream) == cudaSuccess) return SA_OK;
     cudaGetLastError();  // the cluster shape could not be launched here: use the persistent kernel
   }
-  const long long n_score = units * a.sel.splits, n_dec = plan.items;
-  if (n_score + n_dec > 0x7fffffffLL) return SA_ERR_UNSUPPORTED;
+  const long long n_score = (per_head ? kv_units : units) * a.sel.splits, n_dec = plan.items;
+  if (n_score + a.n_sel + n_dec > 0x7fffffffLL) return SA_ERR_UNSUPPORTED;
   a.n_score = (int)n_score;
   a.n_dec = (int)n_dec;
   return launched(launch_step(a, (cudaStream_t)stream));

@@ -130,6 +130,10 @@ struct SelectArgs {
   // flag is never published (its decode items run their wait out and report
   // SA_ERR_TIMEOUT); 0 = none
   int hold_flag_of;
+  // per-query-head decode step: scoring items per (sequence, KV head) count
+  // their completions here [B * Hkv]; the per-head selection items wait for
+  // the count to reach `splits`
+  uint32_t* kv_scored;
 };
 cudaError_t launch_select(const SelectArgs& a, cudaStream_t st);
 
@@ -176,6 +180,7 @@ struct StepArgs {
   DecodeArgs dec;             // idx/count = sel outputs, ws_count = split counters [units]
   uint32_t* queue;            // [2] item queue (head, finished CTAs)
   int n_score, n_dec;         // items of each kind
+  int n_sel;                  // per-query-head step: selection items (one per (sequence, query head))
   uint32_t flag_spin_limit;   // polls of a unit-flag wait before SA_ERR_TIMEOUT; 0 = default (~1 s)
 };
 cudaError_t launch_step(const StepArgs& a, cudaStream_t st);

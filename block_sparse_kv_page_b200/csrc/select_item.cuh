@@ -486,8 +486,10 @@ SA_DEV bool unit_geometry(const SelectArgs& a, const int b, int& N, int& P) {
 // Selection of unit u (sequence, KV head) from the group scores its scoring
 // items wrote (at sc_local in shared memory, or in the workspace); the caller
 // has made them visible to this CTA.
-SA_DEV void select_unit_of(const SelectArgs& a, const int u, const SelSmem& S, const float* sc_local) {
-  const int b = u / a.kv.Hkv;
+// units_per_seq: units of one sequence (Hkv, or Hq for per-query-head units).
+SA_DEV void select_unit_of(const SelectArgs& a, const int u, const SelSmem& S, const float* sc_local,
+                           const int units_per_seq) {
+  const int b = u / units_per_seq;
   int N, P;
   unit_geometry(a, b, N, P);  // a bad geometry was flagged by the scoring
   select_unit(a, u, b, N, P, S, sc_local);
@@ -499,9 +501,13 @@ SA_DEV void select_unit_of(const SelectArgs& a, const int u, const SelSmem& S, c
 // counters are not touched).
 // score_dst (non-null): where the unit's group scores go, indexed by page
 // (another CTA's shared memory, say), instead of the workspace.
-template <int RULE, bool FUSED, bool PER_HEAD = false, bool SCORE_ONLY = false>
+// HEAD_ROWS (with SCORE_ONLY, per (sequence, KV head) units): the G query
+// heads' own scores go to their rows b * Hq + h of the workspace (no group
+// max), and the item then counts itself done in a.kv_scored[u] (release).
+template <int RULE, bool FUSED, bool PER_HEAD = false, bool SCORE_ONLY = false, bool HEAD_ROWS = false>
 SA_DEV void select_item(const SelectArgs& a, const int u, const int split, const SelSmem& S,
                         WarpState& ws, float* score_dst = nullptr) {
+  static_assert(!HEAD_ROWS || (SCORE_ONLY && !PER_HEAD), "head rows: score-only items of KV units");
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int gq = lane >> 2, c = lane & 3;
   const int Hkv = a.kv.Hkv;
@@ -600,6 +606,13 @@ SA_DEV void select_item(const SelectArgs& a, const int u, const int split, const
     }
   }
   const int t_new = p_new >= 0 ? (p_new >> 4) : -1;
+  if (t_new >= t_begin && t_new < t_end && (t_new - t_begin) % kWarps == warp && ws.alive) {
+    // the warp that will refresh the newest page starts pulling its key rows
+    // into L2 while the metadata tiles land (with few units the refresh is on
+    // the critical path of the launch)
+    const char* k0 = static_cast<const char*>(a.kv.k) + ((size_t)kvu * a.kv.cap + (size_t)r_s) * (2 * kHeadDim);
+    for (int i = lane; i < 2 * (r_e - r_s); i += 32) prefetch_l2(k0 + (size_t)i * 128);
+  }
 
   for (int it = 0; it < n_it && ws.alive; ++it) {
     __syncwarp();
@@ -678,6 +691,20 @@ SA_DEV void select_item(const SelectArgs& a, const int u, const int split, const
     }
     const float ninf = -__int_as_float(0x7f800000);
     const bool c0 = 2 * c < um.n_heads, c1 = 2 * c + 1 < um.n_heads;
+    if (HEAD_ROWS) {
+      // lane (gq, c) holds heads 2c, 2c + 1 of pages gq and gq + 8
+      const int pg0 = t * 16 + gq, pg1 = pg0 + 8;
+      float* row = a.ws_scores + ((size_t)b * a.Hq + (size_t)um.h0 + 2 * c) * a.ws_stride;
+      if (c0) {
+        if (pg0 < P) row[pg0] = acc[0];
+        if (pg1 < P) row[pg1] = acc[2];
+      }
+      if (c1) {
+        if (pg0 < P) row[a.ws_stride + pg0] = acc[1];
+        if (pg1 < P) row[a.ws_stride + pg1] = acc[3];
+      }
+      continue;
+    }
     float mlo = fmaxf(c0 ? acc[0] : ninf, c1 ? acc[1] : ninf);
     float mhi = fmaxf(c0 ? acc[2] : ninf, c1 ? acc[3] : ninf);
     mlo = fmaxf(mlo, __shfl_xor_sync(0xffffffffu, mlo, 1));
@@ -694,6 +721,10 @@ SA_DEV void select_item(const SelectArgs& a, const int u, const int split, const
     }
   }
   ws.gi += (uint32_t)n_it;
+  if (HEAD_ROWS) {
+    __syncthreads();  // then one acq_rel increment publishes the CTA's score rows
+    if (tid == 0) atom_add_acq_rel_u32(&a.kv_scored[u], 1u);
+  }
   if (SCORE_ONLY) return;
 
   // ---- the last CTA of the unit selects (its counter increment is acq_rel:

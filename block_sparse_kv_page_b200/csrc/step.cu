@@ -75,7 +75,26 @@ SA_DEV int wait_selected(const uint32_t* flag, int* status, uint32_t limit) {
   return -1;
 }
 
+// Wait until *count reaches `target` (acquire); false (and SA_ERR_TIMEOUT)
+// after `limit` polls.
+SA_DEV bool wait_count(const uint32_t* count, uint32_t target, int* status, uint32_t limit) {
+  uint32_t ns = 32;
+  for (uint32_t i = 0; i < limit; ++i) {
+    if (ld_acquire_u32(count) >= target) return true;
+    __nanosleep(ns);
+    if (ns < 256) ns <<= 1;
+  }
+  flag_status(status, SA_ERR_TIMEOUT);
+  return false;
+}
+
 // PER_HEAD: units are (sequence, query head), each selecting its own pages.
+// Their scores still come from one scoring pass per (sequence, KV head)
+// (items [0, n_score) write the G heads' own score rows); items
+// [n_score, n_score + n_sel) are the per-head selections, each waiting
+// (bounded) until its KV head's scoring items are all done; the decode items
+// follow.  Every wait is on items handed out earlier that never wait on
+// later ones, so none can deadlock.
 template <int RULE, bool PER_HEAD>
 __global__ void __launch_bounds__(kThreads, SA_STEP_CTAS_PER_SM)
     step_kernel(const __grid_constant__ StepArgs a) {
@@ -105,18 +124,24 @@ __global__ void __launch_bounds__(kThreads, SA_STEP_CTAS_PER_SM)
   __syncthreads();
   grid_dep_wait();  // the previous kernel of the stream has completed (no global access before)
   WarpState ws{0u, true, 0u, 0u};
-  const int n_items = a.n_score + a.n_dec;
+  const int n_pre = a.n_score + a.n_sel;  // items before the decode items
+  const int n_items = n_pre + a.n_dec;
+  const uint32_t limit = a.flag_spin_limit ? a.flag_spin_limit : kFlagSpinLimit;
   for (;;) {
     if (threadIdx.x == 0) {
       int item = (int)atomicAdd(&a.queue[0], 1u);
-      if (item >= a.n_score && item < n_items) {
+      if (PER_HEAD && item >= a.n_score && item < n_pre) {
+        const int u = item - a.n_score, b = u / a.sel.Hq;
+        const int kvu = b * a.sel.kv.Hkv + (u - b * a.sel.Hq) / a.sel.G;
+        if (!wait_count(a.sel.kv_scored + kvu, (uint32_t)a.sel.splits, a.sel.status, limit))
+          item = n_items;  // gave up: this CTA stops taking work
+      } else if (item >= n_pre && item < n_items) {
         int u, split;
-        dec::item_unit(a.dec, item - a.n_score, u, split);
+        dec::item_unit(a.dec, item - n_pre, u, split);
         // the sequence length is an input of the launch: its load (kept in a
         // register until after the wait) overlaps the acquire
         const int ntok = a.dec.kv.seq_len[unit_map<PER_HEAD>(u, a.dec.kv.Hkv, a.dec.Hq, a.dec.G).b];
-        const int cnt = wait_selected(a.sel.ws_count + u, a.sel.status,
-                                      a.flag_spin_limit ? a.flag_spin_limit : kFlagSpinLimit);  // acquire
+        const int cnt = wait_selected(a.sel.ws_count + u, a.sel.status, limit);  // acquire
         s_count = cnt;
         s_ntok = ntok;
         if (cnt < 0) item = n_items;  // gave up: this CTA stops taking work
@@ -130,10 +155,20 @@ __global__ void __launch_bounds__(kThreads, SA_STEP_CTAS_PER_SM)
       break;
     }
     if (item < a.n_score) {
-      sel::select_item<RULE, true, PER_HEAD>(a.sel, item / a.sel.splits, item % a.sel.splits, S, ws);
+      if (PER_HEAD)  // the G heads' score rows of one (sequence, KV head)
+        sel::select_item<RULE, true, false, true, true>(a.sel, item / a.sel.splits, item % a.sel.splits, S, ws);
+      else
+        sel::select_item<RULE, true, false>(a.sel, item / a.sel.splits, item % a.sel.splits, S, ws);
+    } else if (PER_HEAD && item < n_pre) {
+      // one query head's selection from its score row; then its flag
+      const int u = item - a.n_score;
+      sel::select_unit_of(a.sel, u, S, nullptr, a.sel.Hq);
+      __syncthreads();
+      if (threadIdx.x == 0 && a.sel.hold_flag_of != u + 1)
+        st_release_u32(&a.sel.ws_count[u], sel::kUnitSelected | (uint32_t)a.sel.sel_count[u]);
     } else {
       int u, split;
-      dec::item_unit(a.dec, item - a.n_score, u, split);
+      dec::item_unit(a.dec, item - n_pre, u, split);
       if (a.sel.k_new != nullptr && lane == 0) fence_proxy_async_global();  // appended rows, then TMA
       dec::decode_item<PER_HEAD>(a.dec, u, split, D, ws, s_count, s_ntok);  // count from the unit's flag
     }
@@ -158,6 +193,8 @@ __global__ void __launch_bounds__(kThreads, SA_STEP_CTAS_PER_SM)
       a.sel.ws_count[i] = 0;
       a.dec.ws_count[i] = 0;
     }
+    if (PER_HEAD)
+      for (int i = threadIdx.x; i < a.sel.kv.B * a.sel.kv.Hkv; i += blockDim.x) a.sel.kv_scored[i] = 0;
     if (threadIdx.x == 0) {
       a.queue[0] = 0;
       a.queue[1] = 0;
@@ -252,7 +289,7 @@ __global__ void __launch_bounds__(kThreads, 1) step_cluster_kernel(const __grid_
   __syncthreads();
   cluster_sync();       // every range's scores are in the leader's shared memory
   // 2. the leader selects
-  if (r == 0) sel::select_unit_of(a.sel, u, S, my_scores);
+  if (r == 0) sel::select_unit_of(a.sel, u, S, my_scores, a.sel.kv.Hkv);
   fence_proxy_async();  // the ring held the keys: generic writes before the decode TMA writes
   __syncthreads();
   cluster_sync();       // the selection is visible to every CTA of the cluster
@@ -357,7 +394,7 @@ cudaError_t launch_step_cluster(const StepArgs& a, int C, cudaStream_t st) {
 
 cudaError_t launch_step(const StepArgs& a, cudaStream_t st) {
   const size_t smem = step_smem_bytes(a.sel.kv.max_pages, a.dec.max_sel, a.sel.kv.page_size == 0);
-  const long long items = (long long)a.n_score + a.n_dec;
+  const long long items = (long long)a.n_score + a.n_sel + a.n_dec;
   if (items > 0x7fffffffLL) return cudaErrorInvalidValue;
   using Fn = void (*)(const StepArgs);
   const Fn fns[2][2] = {{step_kernel<0, false>, step_kernel<0, true>}, {step_kernel<1, false>, step_kernel<1, true>}};
