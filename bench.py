@@ -706,32 +706,43 @@ def router_decode_leg(torch, dev, sa, kv, inp, metas, out, lse, k: int, scale: f
     sbar_r = torch.zeros((L * B,), dtype=torch.float32, device=dev)
     trig_r = torch.zeros((L * B,), dtype=torch.uint8, device=dev)
     for rule in ("envelope", "centroid"):
-        def routed_step():
+        def routed_calls():
             sa.sparse_attn_build_meta(kv, rule, -1, metas[rule])
             sa.sparse_attn_route_decode(kv, metas[rule], rule, inp["q"], k, rho, 0.25, None, idx_r, cnt_r,
                                         sig_r, sbar_r, trig_r, None, ws_r)
             sa.sparse_attn_decode(kv, inp["q"], L * B, 0, 1, scale, idx_r, cnt_r, W, out, lse, ws_r)
-        for _ in range(warmup):
-            routed_step()
-        barrier()
-        e0 = torch.cuda.Event(enable_timing=True)
-        e1 = torch.cuda.Event(enable_timing=True)
-        n_rep = steps
-        with _region(clocks, f"router-decode/{rule}"):
-            e0.record(stream)
-            for _ in range(n_rep):
-                routed_step()
-            e1.record(stream)
-            torch.cuda.synchronize()
-        m2 = max_over_ranks(e0.elapsed_time(e1) / n_rep, dist, dev)
-        kept = int(cnt_r.sum().item())
-        kv_r = kept * PS * 2 * D * 2
-        res[f"router-decode/{rule}"] = {
-            "ms_per_step": round(m2, 4), "value": kept * PS * (HQ // HKV) * world / (m2 * 1e-3),
-            "eff_GBps": (meta_bytes + kv_r) / (m2 * 1e-3) / 1e9,
-            "triggered_rows": int(trig_r.sum().item()), "pages_kept_per_unit": round(kept / (L * B * HKV), 1),
-            "note": "three launches per step (metadata refresh; score-only pass + router selection; decode "
-                    "over the routed lists); k = 256 pages, rho = 2, quantile 0.25 over the 48 rows"}
+
+        def routed_step():
+            sa.sparse_attn_route_decode_step(kv, metas[rule], rule, inp["q"], k, rho, 0.25, None, scale, idx_r,
+                                             cnt_r, sig_r, sbar_r, trig_r, None, out, lse, ws_r)
+        for label, fn, note in (
+                ("router-decode", routed_step,
+                 "one sparse_attn_route_decode_step launch per step (metadata refresh, scoring, the router's "
+                 "selection and triggers, decode of every top k as soon as its unit is selected and of the "
+                 "triggered expansions)"),
+                ("router-decode-calls", routed_calls,
+                 "three calls per step (metadata refresh; score-only pass + router selection; decode over the "
+                 "routed lists)")):
+            for _ in range(warmup):
+                fn()
+            barrier()
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            n_rep = steps
+            with _region(clocks, f"{label}/{rule}"):
+                e0.record(stream)
+                for _ in range(n_rep):
+                    fn()
+                e1.record(stream)
+                torch.cuda.synchronize()
+            m2 = max_over_ranks(e0.elapsed_time(e1) / n_rep, dist, dev)
+            kept = int(cnt_r.sum().item())
+            kv_r = kept * PS * 2 * D * 2
+            res[f"{label}/{rule}"] = {
+                "ms_per_step": round(m2, 4), "value": kept * PS * (HQ // HKV) * world / (m2 * 1e-3),
+                "eff_GBps": (meta_bytes + kv_r) / (m2 * 1e-3) / 1e9,
+                "triggered_rows": int(trig_r.sum().item()), "pages_kept_per_unit": round(kept / (L * B * HKV), 1),
+                "note": note + "; k = 256 pages, rho = 2, quantile 0.25 over the 48 rows"}
     if sa.sparse_attn_get_device_status(ws_r) != 0:
         raise RuntimeError("router-decode leg: device status set")
     del ws_r, idx_r, cnt_r, sig_r, sbar_r, trig_r

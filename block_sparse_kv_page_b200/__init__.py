@@ -12,6 +12,7 @@ from .ops import (KvCache, SparseAttnError, budget_ratio, budget_tokens, budget_
                   sparse_attn_decode_step_append, sparse_attn_decode_step_per_head,
                   sparse_attn_decode_step_wait_test,
                   sparse_attn_get_device_status, sparse_attn_route, sparse_attn_route_decode,
+                  sparse_attn_route_decode_step,
                   sparse_attn_select,
                   sparse_attn_status_string, sparse_attn_workspace_init,
                   sparse_attn_workspace_size)

@@ -6,8 +6,9 @@
 // Workspace layout (byte offsets from ws, which must be 256-byte aligned):
 //   [0, 256)                 status word (int32) at 0; item-queue counters of
 //                            the persistent kernels at 64 (select), 72
-//                            (decode), 80 (router), 88 (decode step); each
-//                            kernel leaves its queue rewound to zero
+//                            (decode), 80 (router), 88 (decode step), 96
+//                            (routed decode step's counters); each kernel
+//                            leaves its queue rewound to zero
 //   [256, 256 + 4*kMaxUnits) last-CTA counters, shared by every call; each
 //                            call uses counters [0, its units) and leaves
 //                            them zero, so calls issued in order on one
@@ -31,6 +32,7 @@ constexpr size_t kQueueSelect = 64;
 constexpr size_t kQueueDecode = 72;
 constexpr size_t kQueueRoute = 80;
 constexpr size_t kQueueStep = 88;
+constexpr size_t kQueueRouteStep = 96;  // routed decode step: units selected, triggers-published flag
 constexpr int kMaxRouteTiles = 1024;
 constexpr int kMaxRouteList = 1023;
 constexpr size_t kScratch = 256 + 4 * (size_t)kMaxUnits;
@@ -396,7 +398,12 @@ size_t sparse_attn_workspace_size(const sa_kv_desc* kv, int32_t n_q_heads, int32
   const size_t rt = route_ws_bytes(route_tiles, kv->n_kv_heads, kv->max_pages, max_sel);
   if (rt > tail) tail = rt;
   if (kv->batch <= kMaxRouteTiles && kv->page_size > 0) {  // decode router: scores + router scratch
-    const size_t rd = select_scratch(kv) + route_decode_ws_bytes(kv->batch * kv->n_kv_heads);
+    const long long ru = (long long)kv->batch * kv->n_kv_heads;
+    size_t rd = select_scratch(kv) + route_decode_ws_bytes(ru);
+    // the routed decode step adds split partials of its top-k and expansion
+    // windows, each at most the splits of a plain decode over max_sel
+    const DecodePlan rp = decode_plan((int)ru, max_tiles_per_unit(kv, max_sel), sm);
+    rd += decode_scratch(DecodePlan{2 * rp.splits, (int)ru, 2 * rp.splits, ru * 2 * rp.splits});
     if (rd > tail) tail = rd;
   }
   return kScratch + tail;
@@ -807,6 +814,98 @@ sa_status sparse_attn_route_decode(const sa_kv_desc* kv, const void* meta, sa_sc
   a.ws_final = reinterpret_cast<uint32_t*>(reinterpret_cast<char*>(ws) + kQueueRoute);
   a.status = reinterpret_cast<int*>(ws);
   return launched(launch_route_decode(a, (cudaStream_t)stream));
+}
+
+sa_status sparse_attn_route_decode_step(const sa_kv_desc* kv, void* meta, sa_score_rule rule,
+                                        const void* q, int32_t n_q_heads, int32_t k, int32_t rho,
+                                        float quantile, const float* tau, float scale, int32_t* kv_idx,
+                                        int32_t* kv_count, float* sigma, float* sigma_bar,
+                                        uint8_t* triggered, float* tau_out, float* out, float* lse,
+                                        void* ws, size_t ws_bytes, void* stream) {
+  if (!kv || kv->page_size <= 0) return kv ? SA_ERR_UNSUPPORTED : SA_ERR_INVALID;
+  if (k < 1 || rho < 1) return SA_ERR_INVALID;
+  if (!(quantile >= 0.f && quantile <= 1.f)) return SA_ERR_INVALID;
+  if (!kv_idx || !kv_count || !sigma || !sigma_bar || !triggered) return SA_ERR_INVALID;
+  if (!aligned(sigma, 4) || !aligned(sigma_bar, 4) || (tau && !aligned(tau, 4)) ||
+      (tau_out && !aligned(tau_out, 4)))
+    return SA_ERR_INVALID;
+  if (!out || !aligned(out, 16) || (lse && !aligned(lse, 4))) return SA_ERR_INVALID;
+  if (!std::isfinite(scale)) return SA_ERR_INVALID;
+  const long long W = (long long)rho * k;
+  if (W > kMaxRouteList || (long long)k + 1 > kMaxRouteList + 1) return SA_ERR_UNSUPPORTED;
+  if (kv->batch > kMaxRouteTiles) return SA_ERR_UNSUPPORTED;
+  int G;
+  const sa_budget dummy{SA_BUDGET_TOPK, 1, 0.f, 0, 0, 0, 0};
+  sa_status s = check_select(kv, meta, rule, q, n_q_heads, &dummy, (int)W, kv_idx, kv_count, nullptr, &G);
+  if (s != SA_OK) return s;
+  const long long units = (long long)kv->batch * kv->n_kv_heads;
+  if (2 * units > kMaxUnits) return SA_ERR_UNSUPPORTED;  // unit flags + split counters
+  const unsigned long long kv_rows = (unsigned long long)kv->batch * kv->n_kv_heads * kv->cap_tokens;
+  if (kv_rows > 0x7fffffffULL) return SA_ERR_UNSUPPORTED;
+  if (route_decode_smem_bytes(kv->max_pages, (int)W, k, kv->batch) >
+      (size_t)(kv->max_pages * 8 > 65536 ? kv->max_pages * 8 : 65536))
+    return SA_ERR_UNSUPPORTED;  // the selection's keys and candidates live in the step's ring
+  if (step_smem_bytes(kv->max_pages, (int)W, false) > 227 * 1024) return SA_ERR_UNSUPPORTED;
+  // the top-k windows and the expansion windows get their own splits
+  const int sm = device_sm_count();
+  const int sub = kv->page_size / 16;
+  const int sb = decode_plan((int)units, k * sub, sm).splits;
+  const int se = W > k ? decode_plan((int)units, (int)(W - k) * sub, sm).splits : 0;
+  DecodePlan plan{sb + se, (int)units, sb + se, units * (sb + se)};
+  const size_t sel_bytes = select_scratch(kv);
+  const size_t rt_bytes = route_decode_ws_bytes(units);
+  const size_t need = kScratch + sel_bytes + rt_bytes + decode_scratch(plan);
+  if ((s = check_ws(ws, ws_bytes, need)) != SA_OK) return s;
+
+  RouteStepArgs ra{};  // every field zero unless set below
+  StepArgs& a = ra.st;
+  char* w = reinterpret_cast<char*>(ws);
+  if (!fill_select(&a.sel, kv, meta, rule, q, n_q_heads, G, &dummy, (int)W, kv_idx, kv_count, nullptr, ws) ||
+      !fill_decode(&a.dec, kv, q, n_q_heads, G, scale, kv_idx, kv_count, (int)W, out, lse,
+                   reinterpret_cast<float*>(w + kScratch + sel_bytes + rt_bytes),
+                   reinterpret_cast<uint32_t*>(w + 256) + units, reinterpret_cast<int*>(ws), plan))
+    return SA_ERR_CUDA;
+  a.sel.meta_refresh = static_cast<unsigned char*>(meta);
+  a.dec.route_k = k;
+  a.dec.route_w = (int)W;
+  a.dec.route_base_splits = sb;
+  a.queue = reinterpret_cast<uint32_t*>(w + kQueueStep);
+  RouteArgs& r = ra.route;
+  r.kv = view(kv);
+  r.rule = (int)rule;
+  r.q = q;
+  r.Hq = n_q_heads;
+  r.G = G;
+  r.n_rows = kv->batch;
+  r.q_pos0 = 0;
+  r.tile_rows = 1;
+  r.n_tiles = kv->batch;
+  r.k = k;
+  r.rho = rho;
+  r.W = (int)W;
+  r.nsplit = 1;
+  r.quantile = quantile;
+  r.tau_in = tau;
+  r.kv_idx = kv_idx;
+  r.kv_count = kv_count;
+  r.sigma = sigma;
+  r.sigma_bar = sigma_bar;
+  r.triggered = triggered;
+  r.tau_out = tau_out;
+  r.ws_keys = nullptr;
+  r.dec_scores = a.sel.ws_scores;
+  r.dec_stride = score_stride(kv);
+  char* rbase = w + kScratch + sel_bytes;
+  r.ws_sigma = reinterpret_cast<double*>(rbase);
+  r.ws_elig = reinterpret_cast<int32_t*>(rbase + align256((size_t)units * 8));
+  r.status = reinterpret_cast<int*>(ws);
+  ra.routed = reinterpret_cast<uint32_t*>(w + kQueueRouteStep);
+  const long long n_score = units * a.sel.splits;
+  if (n_score + plan.items > 0x7fffffffLL) return SA_ERR_UNSUPPORTED;
+  a.n_score = (int)n_score;
+  a.n_dec = (int)plan.items;
+  ra.n_base = (int)(units * sb);
+  return launched(launch_route_step(ra, (cudaStream_t)stream));
 }
 
 sa_status sparse_attn_get_device_status(void* ws, sa_status* host_out, void* stream) {

@@ -241,8 +241,21 @@ SA_DEV void decode_item(const DecodeArgs& a, const int u, const int split, const
   const int splits = coarse ? a.splits : a.splits_fine;
   const size_t slot0 = coarse ? (size_t)u * a.splits
                               : (size_t)a.fine_unit0 * a.splits + (size_t)(u - a.fine_unit0) * a.splits_fine;
-  const int t_begin = (int)(((long long)T * split) / splits);
-  const int t_end = (int)(((long long)T * (split + 1)) / splits);
+  int t_begin = (int)(((long long)T * split) / splits);
+  int t_end = (int)(((long long)T * (split + 1)) / splits);
+  if (a.route_k > 0) {  // routed lists: the top-k window, then the expansion window
+    const int sb = a.route_base_splits, se = splits - sb;
+    const long long kt = (long long)a.route_k * sub, wt = (long long)a.route_w * sub;
+    if (split < sb) {
+      t_begin = (int)(kt * split / sb);
+      t_end = (int)(kt * (split + 1) / sb);
+    } else {
+      t_begin = (int)(kt + (wt - kt) * (split - sb) / se);
+      t_end = (int)(kt + (wt - kt) * (split - sb + 1) / se);
+    }
+    t_begin = min(t_begin, T);
+    t_end = min(t_end, T);
+  }
   const long long row0 = (long long)um.kvu * a.kv.cap;
 
   // Token range of tile t of the unit (n = 0 for a skipped, invalid entry).

@@ -160,6 +160,12 @@ struct DecodeArgs {
   int fine_unit0;             // units from here on (the end of the queue) use splits_fine
   int splits_fine;
   int n_items;                // fine_unit0 * splits + (units - fine_unit0) * splits_fine
+  // routed decode step (0 = off): the units' lists are in rank order; splits
+  // [0, route_base_splits) cover list entries [0, route_k) (the top k, decoded
+  // as soon as the unit is selected), the others entries [route_k, route_w)
+  // (the expansion, decoded once the trigger is known); each clipped to the
+  // unit's count
+  int route_k, route_w, route_base_splits;
 };
 cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t st);
 
@@ -171,42 +177,6 @@ struct DecodePlan {
   long long items;            // work items = partial slots
 };
 DecodePlan decode_plan(int units, int max_tiles, int sm_count);
-
-// One decode step in one launch: newest-page metadata refresh, scoring,
-// selection and decode.  Scoring items come first in the queue; decode item j
-// of unit u waits (bounded) for u's selection flag.
-struct StepArgs {
-  SelectArgs sel;             // meta_refresh set, ws_count = unit flags [units]
-  DecodeArgs dec;             // idx/count = sel outputs, ws_count = split counters [units]
-  uint32_t* queue;            // [2] item queue (head, finished CTAs)
-  int n_score, n_dec;         // items of each kind
-  int n_sel;                  // per-query-head step: selection items (one per (sequence, query head))
-  uint32_t flag_spin_limit;   // polls of a unit-flag wait before SA_ERR_TIMEOUT; 0 = default (~1 s)
-};
-cudaError_t launch_step(const StepArgs& a, cudaStream_t st);
-// Few units: one cluster of C CTAs per unit (sel.splits must be C).
-int step_cluster_size(int units, int dec_splits, int sm_count);
-cudaError_t launch_step_cluster(const StepArgs& a, int C, cudaStream_t st);
-size_t step_smem_bytes(int max_pages, int max_sel, bool chunks);
-
-struct TileAttnArgs {
-  CUtensorMap tmap_k;         // K rows [Hkv*cap][128 bf16], boxes 64 x 64, 128B swizzle
-  CUtensorMap tmap_v;         // V, same geometry (read MN-major by the PV MMA)
-  KvView kv;                  // batch 1, 64-token blocks
-  const void* q;              // bf16 [n_rows][Hq][128]
-  int Hq, G;
-  int n_rows, q_pos0, tile_rows, n_tiles, n_mchunks;
-  float scale_log2;
-  const int32_t* idx;         // [n_tiles][Hkv][max_sel], -1 = sentinel
-  const int32_t* count;       // [n_tiles][Hkv]
-  int max_sel;
-  float* out;
-  float* lse;
-  int* status;
-};
-// Tile attention on tcgen05 (CTA = 128 query vectors of a (tile, KV head)).
-cudaError_t launch_tile_attn_tc(const TileAttnArgs& a, cudaStream_t st);
-int tile_attn_tc_mchunks(int vectors_per_tile);
 
 struct RouteArgs {
   CUtensorMap tmap_meta;      // block metadata rows [Hkv*max_pages][512 B], boxes 16 x 128 B, 128B swizzle
@@ -235,6 +205,55 @@ struct RouteArgs {
   uint32_t* ws_final;         // [1] finalize counter (left zero)
   int* status;
 };
+// One decode step in one launch: newest-page metadata refresh, scoring,
+// selection and decode.  Scoring items come first in the queue; decode item j
+// of unit u waits (bounded) for u's selection flag.
+struct StepArgs {
+  SelectArgs sel;             // meta_refresh set, ws_count = unit flags [units]
+  DecodeArgs dec;             // idx/count = sel outputs, ws_count = split counters [units]
+  uint32_t* queue;            // [2] item queue (head, finished CTAs)
+  int n_score, n_dec;         // items of each kind
+  int n_sel;                  // per-query-head step: selection items (one per (sequence, query head))
+  uint32_t flag_spin_limit;   // polls of a unit-flag wait before SA_ERR_TIMEOUT; 0 = default (~1 s)
+};
+cudaError_t launch_step(const StepArgs& a, cudaStream_t st);
+
+// The router applied to decode, in one launch: scoring items, each unit's
+// rank-order selection and sigma (the last scoring CTA of the unit), the
+// batch's quantile and triggers (the last unit), and the decode of every
+// unit's top k (as soon as the unit is selected) and of the expansion of the
+// triggered units (once the triggers are known).
+struct RouteStepArgs {
+  StepArgs st;                // sel: score-only scoring; dec: route_k/w set, idx/count = the lists
+  RouteArgs route;            // dec_scores = the group scores; tiles = the sequences
+  uint32_t* routed;           // [2]: units selected so far, triggers published (flag)
+  int n_base;                 // decode items of the top-k windows (unit order), then the expansions
+};
+cudaError_t launch_route_step(const RouteStepArgs& a, cudaStream_t st);
+// Few units: one cluster of C CTAs per unit (sel.splits must be C).
+int step_cluster_size(int units, int dec_splits, int sm_count);
+cudaError_t launch_step_cluster(const StepArgs& a, int C, cudaStream_t st);
+size_t step_smem_bytes(int max_pages, int max_sel, bool chunks);
+
+struct TileAttnArgs {
+  CUtensorMap tmap_k;         // K rows [Hkv*cap][128 bf16], boxes 64 x 64, 128B swizzle
+  CUtensorMap tmap_v;         // V, same geometry (read MN-major by the PV MMA)
+  KvView kv;                  // batch 1, 64-token blocks
+  const void* q;              // bf16 [n_rows][Hq][128]
+  int Hq, G;
+  int n_rows, q_pos0, tile_rows, n_tiles, n_mchunks;
+  float scale_log2;
+  const int32_t* idx;         // [n_tiles][Hkv][max_sel], -1 = sentinel
+  const int32_t* count;       // [n_tiles][Hkv]
+  int max_sel;
+  float* out;
+  float* lse;
+  int* status;
+};
+// Tile attention on tcgen05 (CTA = 128 query vectors of a (tile, KV head)).
+cudaError_t launch_tile_attn_tc(const TileAttnArgs& a, cudaStream_t st);
+int tile_attn_tc_mchunks(int vectors_per_tile);
+
 cudaError_t launch_route(const RouteArgs& a, cudaStream_t st);
 // Decode router tail: one CTA per (sequence, KV head) over dec_scores.
 cudaError_t launch_route_decode(const RouteArgs& a, cudaStream_t st);

@@ -27,6 +27,7 @@
 #include "common.cuh"
 #include "internal.h"
 #include "decode_item.cuh"
+#include "route_select.cuh"
 #include "select_item.cuh"
 
 namespace cg = cooperative_groups;
@@ -317,6 +318,139 @@ __global__ void __launch_bounds__(kThreads, 1) step_cluster_kernel(const __grid_
   }
 }
 
+// The router applied to decode in one launch (see RouteStepArgs).  Queue:
+// [0, n_score) scoring items (newest-page refresh, group scores to the
+// workspace); the CTA finishing a unit's last one selects the unit's top
+// max(rho k, k + 1) pages in rank order with sigma (the router's selection)
+// and publishes the unit's flag (with its list count); the CTA finishing the
+// last unit computes sigma_bar, the quantile threshold and the triggers,
+// trims the untriggered lists to k, and publishes the `routed` flag.  Then
+// [n_score, n_score + n_base) the top-k windows of the units' lists (each
+// waits for its unit's flag), then the expansion windows (each waits for the
+// routed flag; an untriggered unit's are empty).  The last CTA of a unit
+// merges every window's partials in split order.  Waits only ever point to
+// items handed out earlier that never wait, so none can deadlock.
+template <int RULE>
+__global__ void __launch_bounds__(kThreads, SA_STEP_CTAS_PER_SM)
+    route_step_kernel(const __grid_constant__ RouteStepArgs ra) {
+  const StepArgs& a = ra.st;
+  extern __shared__ unsigned char smem_raw[];
+  __shared__ uint32_t s_hist[512];
+  __shared__ uint32_t s_scan[32];
+  __shared__ uint32_t s_bc[8];
+  __shared__ int s_last, s_item, s_ntiles, s_count, s_ntok, s_flag;
+  unsigned char* base = reinterpret_cast<unsigned char*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  const int body = body_bytes(a.sel.kv.max_pages);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(base + body);
+  const sel::SelSmem S{base, bars, s_hist, s_scan, s_bc, &s_last};
+  const dec::Smem D{base, bars, reinterpret_cast<dec::TileRef*>(base + body + kBarBytes),
+                    reinterpret_cast<int*>(base + body + kBarBytes + kTileRefBytes), s_scan, &s_last,
+                    &s_ntiles};
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  if (lane == 0) {
+    for (int s = 0; s < kStages; ++s) mbar_init(bars + warp * kStages + s, 1);
+    fence_barrier_init();
+  }
+  if (threadIdx.x == 0) {
+    prefetch_tmap(&a.sel.tmap_meta);
+    prefetch_tmap(&a.dec.tmap_k);
+    prefetch_tmap(&a.dec.tmap_v);
+  }
+  __syncthreads();
+  grid_dep_wait();  // the previous kernel of the stream has completed (no global access before)
+  WarpState ws{0u, true, 0u, 0u};
+  const int units = a.sel.kv.B * a.sel.kv.Hkv;
+  const int n_pre = a.n_score + ra.n_base;
+  const int n_items = a.n_score + a.n_dec;
+  const uint32_t limit = a.flag_spin_limit ? a.flag_spin_limit : kFlagSpinLimit;
+  for (;;) {
+    if (threadIdx.x == 0) {
+      int item = (int)atomicAdd(&a.queue[0], 1u);
+      if (item >= a.n_score && item < n_items) {
+        int u, split;
+        dec::item_unit(a.dec, item - a.n_score, u, split);
+        const int ntok = a.dec.kv.seq_len[u / a.dec.kv.Hkv];
+        int cnt;
+        if (item < n_pre) {  // top-k window: the unit's list is written
+          cnt = wait_selected(a.sel.ws_count + u, a.sel.status, limit);
+          if (cnt > ra.route.k) cnt = ra.route.k;
+        } else {             // expansion window: the triggers are known
+          cnt = wait_count(ra.routed + 1, 1u, a.sel.status, limit) ? __ldcg(a.dec.count + u) : -1;
+        }
+        s_count = cnt;
+        s_ntok = ntok;
+        if (cnt < 0) item = n_items;  // gave up: this CTA stops taking work
+      }
+      s_item = item;
+    }
+    __syncthreads();
+    const int item = s_item;
+    if (item >= n_items) {
+      grid_dep_trigger();
+      break;
+    }
+    if (item < a.n_score) {
+      const int u = item / a.sel.splits;
+      sel::select_item<RULE, true, false, true>(a.sel, u, item % a.sel.splits, S, ws);
+      __syncthreads();
+      if (threadIdx.x == 0) {
+        const uint32_t prev = atom_add_acq_rel_u32(&a.sel.ws_count[u], 1u);
+        s_flag = prev == (uint32_t)(a.sel.splits - 1);
+      }
+      __syncthreads();
+      if (s_flag) {  // the unit's last scoring item: the router's selection
+        const int b = u / a.sel.kv.Hkv, g = u - b * a.sel.kv.Hkv;
+        int N, P;
+        sel::unit_geometry(a.sel, b, N, P);
+        fence_proxy_async();  // the ring becomes the selection's keys
+        rsel::route_select_tile(ra.route, b, g, P, base, s_hist, s_bc, s_scan);
+        __syncthreads();
+        if (threadIdx.x == 0) {
+          st_release_u32(&a.sel.ws_count[u], sel::kUnitSelected | (uint32_t)ra.route.kv_count[u]);
+          s_flag = atom_add_acq_rel_u32(ra.routed, 1u) == (uint32_t)(units - 1);
+        }
+        __syncthreads();
+        if (s_flag) {  // every unit selected: quantile, triggers, trimmed lists
+          rsel::route_finalize(ra.route, base);
+          __syncthreads();
+          if (threadIdx.x == 0) st_release_u32(ra.routed + 1, 1u);
+        }
+      }
+    } else {
+      int u, split;
+      dec::item_unit(a.dec, item - a.n_score, u, split);
+      dec::decode_item<false>(a.dec, u, split, D, ws, s_count, s_ntok);
+    }
+    fence_proxy_async();  // generic writes to the ring (keys, merge) before the next TMA writes
+    __syncthreads();
+  }
+  if (!ws.alive && lane == 0) {  // a wait timed out: let the copies in flight land (bounded)
+    uint64_t* wb = bars + warp * kStages;
+    for (uint32_t g = ws.drain_lo; g < ws.drain_hi; ++g)
+      mbar_wait(wb + g % kStages, (g / kStages) & 1u, nullptr);
+  }
+  // the last CTA out clears the unit flags, split counters and routed counters
+  if (threadIdx.x == 0) {
+    __threadfence();
+    s_last = atomicAdd(&a.queue[1], 1u) == gridDim.x - 1;
+  }
+  __syncthreads();
+  if (s_last) {
+    __threadfence();
+    for (int i = threadIdx.x; i < units; i += blockDim.x) {
+      a.sel.ws_count[i] = 0;
+      a.dec.ws_count[i] = 0;
+    }
+    if (threadIdx.x == 0) {
+      ra.routed[0] = 0;
+      ra.routed[1] = 0;
+      a.queue[0] = 0;
+      a.queue[1] = 0;
+    }
+  }
+}
+
 // Resident CTAs per SM of a step kernel for a shared-memory size (cached).
 int step_occupancy(const void* fn, size_t smem) {
   struct Entry {
@@ -390,6 +524,22 @@ cudaError_t launch_step_cluster(const StepArgs& a, int C, cudaStream_t st) {
   cfg.numAttrs = 2;
   if (a.sel.rule == 0) return cudaLaunchKernelEx(&cfg, step_cluster_kernel<0>, a);
   return cudaLaunchKernelEx(&cfg, step_cluster_kernel<1>, a);
+}
+
+cudaError_t launch_route_step(const RouteStepArgs& a, cudaStream_t st) {
+  const size_t smem = step_smem_bytes(a.st.sel.kv.max_pages, a.st.dec.max_sel, false);
+  const long long items = (long long)a.st.n_score + a.st.n_dec;
+  if (items > 0x7fffffffLL) return cudaErrorInvalidValue;
+  using Fn = void (*)(const RouteStepArgs);
+  const Fn f = a.st.sel.rule == 0 ? route_step_kernel<0> : route_step_kernel<1>;
+  cudaError_t e = set_smem_attr((const void*)f, smem);
+  if (e != cudaSuccess) return e;
+  int occ = step_occupancy((const void*)f, smem);
+  if (occ < 1) return cudaErrorInvalidConfiguration;
+  if (occ > SA_STEP_CTAS_PER_SM) occ = SA_STEP_CTAS_PER_SM;
+  long long grid = (long long)device_sm_count() * occ;
+  if (grid > items) grid = items;
+  return launch_pdl(f, (unsigned)grid, kThreads, smem, st, a);
 }
 
 cudaError_t launch_step(const StepArgs& a, cudaStream_t st) {

@@ -306,6 +306,27 @@ def sparse_attn_route_decode(kv: KvCache, meta: torch.Tensor, rule, q: torch.Ten
            "sparse_attn_route_decode")
 
 
+def sparse_attn_route_decode_step(kv: KvCache, meta: torch.Tensor, rule, q: torch.Tensor, k: int, rho: int,
+                                  quantile: float, tau: torch.Tensor | None, scale: float, kv_idx: torch.Tensor,
+                                  kv_count: torch.Tensor, sigma: torch.Tensor, sigma_bar: torch.Tensor,
+                                  triggered: torch.Tensor, tau_out: torch.Tensor | None, out: torch.Tensor,
+                                  lse: torch.Tensor | None, ws: torch.Tensor, stream=None) -> None:
+    """The router on the decode batch and the decode over its lists in one
+    launch (newest-page metadata refresh included): the outputs of
+    sparse_attn_route_decode plus out [B, Hq, 128] fp32 and lse [B, Hq]."""
+    if q.dtype != torch.bfloat16 or not q.is_contiguous():
+        raise ValueError("q must be contiguous bf16 [B, Hq, 128]")
+    if out.dtype != torch.float32 or not out.is_contiguous():
+        raise ValueError("out must be contiguous fp32")
+    _check(lib.sparse_attn_route_decode_step(C.byref(kv.desc), meta.data_ptr(), _rule(rule), q.data_ptr(),
+                                             q.shape[-2], int(k), int(rho), float(quantile), _ptr(tau),
+                                             float(scale), kv_idx.data_ptr(), kv_count.data_ptr(),
+                                             sigma.data_ptr(), sigma_bar.data_ptr(), triggered.data_ptr(),
+                                             _ptr(tau_out), out.data_ptr(), _ptr(lse), ws.data_ptr(),
+                                             ws.numel() * ws.element_size(), _stream(stream)),
+           "sparse_attn_route_decode_step")
+
+
 def sparse_attn_route(kv: KvCache, meta: torch.Tensor, rule, q: torch.Tensor, n_q_rows: int,
                       q_pos0: int, tile_rows: int, k: int, rho: int, quantile: float,
                       tau: torch.Tensor | None, kv_idx: torch.Tensor, kv_count: torch.Tensor,

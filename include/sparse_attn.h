@@ -333,6 +333,26 @@ sa_status sparse_attn_decode_step_wait_test(const sa_kv_desc* kv, void* meta, sa
                                             int32_t held_unit, uint32_t flag_spin_limit, void* ws,
                                             size_t ws_bytes, void* stream);
 
+/* The router applied to decode and the decode over its lists, in ONE launch
+ * ("Onzekerheidsgestuurde Selectie voor Blok-schaarse Aandacht",
+ * "Methodologie" steps 1-5 on one-row tiles; the same results as
+ * sparse_attn_route_decode followed by sparse_attn_decode over kv_idx /
+ * kv_count, after the newest page's metadata is refreshed as in
+ * sparse_attn_decode_step).  meta is read and its newest page rewritten.
+ * Outputs: kv_idx / kv_count / sigma / sigma_bar / triggered / tau_out as
+ * sparse_attn_route_decode (lists in rank order, -1 padded), out fp32
+ * [B][Hq][128] and lse (nullable) as sparse_attn_decode.  Every unit's top k
+ * pages are attended as soon as the unit is selected; the pages k .. rho*k-1
+ * of the triggered sequences once the batch's triggers are known.  Fixed
+ * pages only, B <= 1024, rho*k <= 1023; the workspace sized by
+ * sparse_attn_workspace_size with max_sel >= rho*k. */
+sa_status sparse_attn_route_decode_step(const sa_kv_desc* kv, void* meta, sa_score_rule rule,
+                                        const void* q, int32_t n_q_heads, int32_t k, int32_t rho,
+                                        float quantile, const float* tau, float scale, int32_t* kv_idx,
+                                        int32_t* kv_count, float* sigma, float* sigma_bar,
+                                        uint8_t* triggered, float* tau_out, float* out, float* lse,
+                                        void* ws, size_t ws_bytes, void* stream);
+
 /* Copy the workspace status word to *host_out (SA_OK if no device check
  * fired since the last init/clear) and clear it.  Synchronises `stream`. */
 sa_status sparse_attn_get_device_status(void* ws, sa_status* host_out, void* stream);

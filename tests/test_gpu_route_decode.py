@@ -135,3 +135,100 @@ def test_route_decode_rejects_bad_arguments(cuda_dev):
         sa.sparse_attn_route_decode(chunks, meta, "envelope", lay.q, 16, 2, 0.5, None, idx, cnt, sig, sb, tr,
                                     None, ws)
     assert e.value.status == sa.SA_ERR_UNSUPPORTED
+
+
+def _run_gpu_step(sa, lay, *, rule, ps, k, rho, quantile, tau, stale=True):
+    """The one-launch routed decode step, on metadata built for the cache as
+    it stood before its newest token (the step refreshes the newest page)."""
+    B, Hkv, cap, D = lay.k.shape
+    Hq = lay.q.shape[1]
+    dev = lay.k.device
+    kv = sa.KvCache(lay.k, lay.v, lay.seq_len, page_size=ps, max_pages=-(-cap // ps))
+    meta = kv.meta_buffer().fill_(0x5A)
+    prev = (lay.seq_len - 1).clamp(min=1).to(torch.int32) if stale else lay.seq_len
+    sa.sparse_attn_build_meta(sa.KvCache(lay.k, lay.v, prev, page_size=ps, max_pages=-(-cap // ps)), rule, 0,
+                              meta)
+    W = rho * k
+    ws = sa.make_workspace(kv, Hq, B, W)
+    kv_idx = torch.full((B, Hkv, W), -7, dtype=torch.int32, device=dev)
+    kv_count = torch.full((B, Hkv), -7, dtype=torch.int32, device=dev)
+    sigma = torch.full((B, Hkv), float("nan"), dtype=torch.float32, device=dev)
+    sbar = torch.full((B,), float("nan"), dtype=torch.float32, device=dev)
+    trig = torch.full((B,), 7, dtype=torch.uint8, device=dev)
+    tau_out = torch.full((1,), float("nan"), dtype=torch.float32, device=dev)
+    tau_t = None if tau is None else torch.tensor([tau], dtype=torch.float32, device=dev)
+    out = torch.full((B, Hq, 128), float("nan"), dtype=torch.float32, device=dev)
+    lse = torch.full((B, Hq), float("nan"), dtype=torch.float32, device=dev)
+    runs = []
+    for _ in range(2):  # twice on one workspace: the launch leaves its counters clean
+        sa.sparse_attn_route_decode_step(kv, meta, rule, lay.q, k, rho, quantile, tau_t, SCALE, kv_idx, kv_count,
+                                         sigma, sbar, trig, tau_out, out, lse, ws)
+        torch.cuda.synchronize()
+        runs.append(dict(kv_idx=kv_idx.cpu().numpy(), kv_count=kv_count.cpu().numpy(),
+                         sigma=sigma.cpu().numpy().astype(np.float64),
+                         sigma_bar=sbar.cpu().numpy().astype(np.float64),
+                         triggered=trig.cpu().numpy().astype(bool), tau=float(tau_out.item()),
+                         status=sa.sparse_attn_get_device_status(ws), out=out.cpu().clone(), lse=lse.cpu().clone()))
+    for key in ("kv_idx", "kv_count", "sigma", "triggered"):
+        assert np.array_equal(runs[0][key], runs[1][key]), key
+    assert torch.equal(runs[0]["out"], runs[1]["out"])
+    return runs[0]
+
+
+@pytest.mark.parametrize("rule", ["envelope", "centroid"])
+@pytest.mark.parametrize("ps,k,rho,quantile,tau", [
+    (16, 16, 2, 0.25, None),
+    (16, 16, 2, 0.5, 0.3),
+    (16, 12, 1, 0.25, None),
+    (64, 4, 3, 0.75, None),
+    (16, 16, 2, 0.0, None),
+])
+def test_route_decode_step_parity(cuda_dev, H, rule, ps, k, rho, quantile, tau):
+    """The one-launch routed decode step against the oracle (router rules,
+    attention over the listed pages) and against the separate calls: the
+    same lists, sigma and triggers exactly; outputs within 1e-5 (the step
+    splits the attention into the top-k and the expansion windows)."""
+    import block_sparse_kv_page_b200 as sa
+    rng = np.random.default_rng(ps * 31 + k)
+    B = 24
+    lens = [int(x) for x in rng.integers(200, 4000, size=B)]
+    lens[3] = 50
+    lay = DG.make_decode_layer(B=B, Hq=32, Hkv=4, seq_lens=lens, seed=801 + k, device=cuda_dev,
+                               cap=4000, key_scale="channel")
+    g_step = _run_gpu_step(sa, lay, rule=rule, ps=ps, k=k, rho=rho, quantile=quantile, tau=tau)
+    assert g_step["status"] == 0
+    ref = _oracle(H, lay, rule=rule, ps=ps, k=k, rho=rho, quantile=quantile, tau=tau)
+    H.compare(g_step, ref, k=k, rho=rho)
+    worst = _check_attention(H, lay, g_step, ps)
+    g_sep = _run_gpu(sa, lay, rule=rule, ps=ps, k=k, rho=rho, quantile=quantile, tau=tau)
+    for key in ("kv_idx", "kv_count", "triggered"):
+        assert np.array_equal(g_step[key], g_sep[key]), key
+    assert np.array_equal(g_step["sigma"], g_sep["sigma"]) and g_step["tau"] == g_sep["tau"]
+    assert float((g_step["out"] - g_sep["out"]).abs().max()) < 1e-5
+    print(f"\nstep {rule} ps={ps} k={k} rho={rho}: max-abs {worst:.2e}, triggered {int(g_step['triggered'].sum())}/{B}")
+
+
+@pytest.mark.parametrize("rule", ["envelope", "centroid"])
+def test_route_decode_step_48_layers(cuda_dev, H, rule):
+    """The benchmark's routed decode launch: 48 Qwen3-VL-shaped layers (29,504
+    tokens) as the batch, k = 256, rho = 2, quantile 0.25; every unit's list,
+    sigma, the triggers and the outputs against the separate calls, and the
+    attention of 12 sampled units against the oracle."""
+    import block_sparse_kv_page_b200 as sa
+    layers = [DG.workload2_layer(l, cuda_dev) for l in range(48)]
+    lay = DG.DecodeLayer(q=torch.cat([l.q for l in layers]), k=torch.cat([l.k for l in layers]),
+                         v=torch.cat([l.v for l in layers]), seq_len=torch.cat([l.seq_len for l in layers]))
+    del layers
+    kw = dict(rule=rule, ps=16, k=256, rho=2, quantile=0.25, tau=None)
+    g_step = _run_gpu_step(sa, lay, **kw)
+    g_sep = _run_gpu(sa, lay, **kw)
+    assert g_step["status"] == 0 and g_sep["status"] == 0
+    for key in ("kv_idx", "kv_count", "triggered"):
+        assert np.array_equal(g_step[key], g_sep[key]), key
+    assert int(g_step["triggered"].sum()) == 12
+    assert float((g_step["out"] - g_sep["out"]).abs().max()) < 1e-5
+    rng = np.random.default_rng(5)
+    for b in rng.choice(48, size=3, replace=False):
+        sub = DG.DecodeLayer(q=lay.q[b:b + 1], k=lay.k[b:b + 1], v=lay.v[b:b + 1], seq_len=lay.seq_len[b:b + 1])
+        one = {key: (val[b:b + 1] if key in ("kv_idx", "kv_count", "out") else val) for key, val in g_step.items()}
+        _check_attention(H, sub, one, 16)
