@@ -330,6 +330,20 @@ __global__ void __launch_bounds__(kThreads, 1) step_cluster_kernel(const __grid_
 // routed flag; an untriggered unit's are empty).  The last CTA of a unit
 // merges every window's partials in split order.  Waits only ever point to
 // items handed out earlier that never wait, so none can deadlock.
+// Decode item j of the routed step: the top-k windows of every unit first
+// (route_base_splits per unit), then the expansion windows.
+SA_DEV void route_item_unit(const RouteStepArgs& ra, const int j, int& u, int& split) {
+  const int sb = ra.st.dec.route_base_splits, se = ra.st.dec.splits - sb;
+  if (j < ra.n_base) {
+    u = j / sb;
+    split = j - u * sb;
+  } else {
+    const int x = j - ra.n_base;
+    u = x / se;
+    split = sb + (x - u * se);
+  }
+}
+
 template <int RULE>
 __global__ void __launch_bounds__(kThreads, SA_STEP_CTAS_PER_SM)
     route_step_kernel(const __grid_constant__ RouteStepArgs ra) {
@@ -369,7 +383,7 @@ __global__ void __launch_bounds__(kThreads, SA_STEP_CTAS_PER_SM)
       int item = (int)atomicAdd(&a.queue[0], 1u);
       if (item >= a.n_score && item < n_items) {
         int u, split;
-        dec::item_unit(a.dec, item - a.n_score, u, split);
+        route_item_unit(ra, item - a.n_score, u, split);
         const int ntok = a.dec.kv.seq_len[u / a.dec.kv.Hkv];
         int cnt;
         if (item < n_pre) {  // top-k window: the unit's list is written
@@ -419,7 +433,7 @@ __global__ void __launch_bounds__(kThreads, SA_STEP_CTAS_PER_SM)
       }
     } else {
       int u, split;
-      dec::item_unit(a.dec, item - a.n_score, u, split);
+      route_item_unit(ra, item - a.n_score, u, split);
       dec::decode_item<false>(a.dec, u, split, D, ws, s_count, s_ntok);
     }
     fence_proxy_async();  // generic writes to the ring (keys, merge) before the next TMA writes
