@@ -17,6 +17,7 @@
 //                            partials of decode -- after the scores in the
 //                            decode step --, router tables), not preserved
 //                            between calls
+#include <algorithm>
 #include <atomic>
 #include <cmath>
 #include <cstdint>
@@ -128,6 +129,19 @@ size_t route_decode_ws_bytes(long long units) {
 size_t select_scratch(const sa_kv_desc* kv, bool per_head = false, int n_q_heads = 0) {
   const size_t units = (size_t)kv->batch * (per_head ? n_q_heads : kv->n_kv_heads);
   return align256(units * score_stride(kv) * sizeof(float));
+}
+
+// Per-head decode step: the union of each KV head's G page sets, entries
+// int32 [B * Hkv][max_pages], head masks uint8 [B * Hkv][max_pages], counts
+// int32 [B * Hkv].
+size_t union_mask_off(const sa_kv_desc* kv) {
+  return align256((size_t)kv->batch * kv->n_kv_heads * kv->max_pages * 4);
+}
+size_t union_count_off(const sa_kv_desc* kv) {
+  return union_mask_off(kv) + align256((size_t)kv->batch * kv->n_kv_heads * kv->max_pages);
+}
+size_t union_scratch(const sa_kv_desc* kv) {
+  return union_count_off(kv) + align256((size_t)kv->batch * kv->n_kv_heads * 4);
 }
 
 // Split partials: one slot per work item (none when no unit is split).
@@ -415,9 +429,17 @@ size_t sparse_attn_workspace_size_per_head(const sa_kv_desc* kv, int32_t n_q_hea
   if (check_group(kv, n_q_heads, &G) != SA_OK) return 0;
   const long long units = (long long)kv->batch * n_q_heads;
   if (units > kMaxUnits) return 0;
-  const DecodePlan plan = decode_plan((int)units, max_tiles_per_unit(kv, max_sel), device_sm_count());
-  // the fused per-head step keeps the scores and the split partials at once
-  return kScratch + select_scratch(kv, true, n_q_heads) + decode_scratch(plan);
+  const int sm = device_sm_count();
+  // the separate per-head decode: partials per (sequence, query head)
+  const DecodePlan plan = decode_plan((int)units, max_tiles_per_unit(kv, max_sel), sm);
+  const size_t calls = decode_scratch(plan);
+  // the fused per-head step keeps the scores, the KV heads' unions and the
+  // split partials of the union decode at once
+  const long long kv_units = (long long)kv->batch * kv->n_kv_heads;
+  const int dec_sel = (int)std::min<long long>((long long)G * max_sel, kv->max_pages);
+  const DecodePlan up = decode_plan((int)kv_units, max_tiles_per_unit(kv, dec_sel), sm);
+  const size_t step = union_scratch(kv) + decode_scratch(up);
+  return kScratch + select_scratch(kv, true, n_q_heads) + (step > calls ? step : calls);
 }
 
 sa_status sparse_attn_workspace_init(void* ws, size_t ws_bytes, void* stream) {
@@ -561,39 +583,56 @@ static sa_status decode_step(const sa_kv_desc* kv, void* meta, sa_score_rule rul
   if (kv->page_size == 0 && max_sel > kMaxChunkSel) return SA_ERR_UNSUPPORTED;
   const long long units = (long long)kv->batch * (per_head ? n_q_heads : kv->n_kv_heads);
   const long long kv_units = (long long)kv->batch * kv->n_kv_heads;
-  // unit flags + split counters (+ per-head step: scoring counts per KV head)
-  if (2 * units + (per_head ? kv_units : 0) > kMaxUnits) return SA_ERR_UNSUPPORTED;
+  // unit flags + split counters (+ per-head step: scoring and selection counts per KV head)
+  if (2 * units + (per_head ? 2 * kv_units : 0) > kMaxUnits) return SA_ERR_UNSUPPORTED;
   const unsigned long long kv_rows = (unsigned long long)kv->batch * kv->n_kv_heads * kv->cap_tokens;
   if (kv_rows > 0x7fffffffULL) return SA_ERR_UNSUPPORTED;  // TMA row coordinates are int32
   const int sm = device_sm_count();
-  int plan_tiles = max_tiles_per_unit(kv, max_sel);
+  // per-head: the decode runs per (sequence, KV head) over the union of the
+  // G heads' sets (at most G * max_sel entries, and at most max_pages)
+  const int dec_sel = per_head ? (int)std::min<long long>((long long)G * max_sel, kv->max_pages) : max_sel;
+  int plan_tiles = max_tiles_per_unit(kv, dec_sel);
   if (budget->kind == SA_BUDGET_TOKENS) {  // the budget, not max_sel, bounds what is attended
-    const int t = token_budget_tiles(budget->token_budget);
-    if (t < plan_tiles) plan_tiles = t;
+    const long long t = (long long)token_budget_tiles(budget->token_budget) * (per_head ? G : 1);
+    if (t < plan_tiles) plan_tiles = (int)t;
   }
-  const DecodePlan plan = decode_plan((int)units, plan_tiles, sm);
+  const DecodePlan plan = decode_plan((int)kv_units, plan_tiles, sm);
   const size_t sel_bytes = select_scratch(kv, per_head, n_q_heads);
-  const size_t need = kScratch + sel_bytes + decode_scratch(plan);
+  const size_t union_bytes = per_head ? union_scratch(kv) : 0;
+  const size_t need = kScratch + sel_bytes + union_bytes + decode_scratch(plan);
   if ((s = check_ws(ws, ws_bytes, need)) != SA_OK) return s;
-  if (step_smem_bytes(kv->max_pages, max_sel, kv->page_size == 0) > 227 * 1024)
+  if (step_smem_bytes(kv->max_pages, per_head ? kv->max_pages : max_sel, kv->page_size == 0) > 227 * 1024)
     return SA_ERR_UNSUPPORTED;
 
   StepArgs a{};  // every field zero unless set below
   char* w = reinterpret_cast<char*>(ws);
+  // unit flags and split counters at w + 256, one per (sequence, KV head)
+  // (the per-head step flags the KV heads' unions, not the query heads)
+  uint32_t* flags = reinterpret_cast<uint32_t*>(w + 256);
+  char* union_base = w + kScratch + sel_bytes;
   if (!fill_select(&a.sel, kv, meta, rule, q, n_q_heads, G, budget, max_sel, sel_idx, sel_count,
                    nullptr, ws) ||
-      !fill_decode(&a.dec, kv, q, n_q_heads, G, scale, sel_idx, sel_count, max_sel,
-                   out_bf16 ? nullptr : static_cast<float*>(out), lse,
-                   reinterpret_cast<float*>(w + kScratch + sel_bytes),
-                   reinterpret_cast<uint32_t*>(w + 256) + units, reinterpret_cast<int*>(ws), plan))
+      !fill_decode(&a.dec, kv, q, n_q_heads, G, scale,
+                   per_head ? reinterpret_cast<int32_t*>(union_base) : sel_idx,
+                   per_head ? reinterpret_cast<int32_t*>(union_base + union_count_off(kv)) : sel_count,
+                   dec_sel, out_bf16 ? nullptr : static_cast<float*>(out), lse,
+                   reinterpret_cast<float*>(union_base + union_bytes), flags + kv_units,
+                   reinterpret_cast<int*>(ws), plan))
     return SA_ERR_CUDA;
   if (out_bf16) a.dec.out_bf16 = static_cast<__nv_bfloat16*>(out);
   if (per_head) {
     // scoring items per (sequence, KV head) write the G heads' rows; then one
-    // selection item per (sequence, query head)
+    // selection item per (sequence, query head); the decode per (sequence,
+    // KV head) over the union of its heads' sets, each head masked to its own
     a.sel.per_head = 1;
-    a.sel.kv_scored = reinterpret_cast<uint32_t*>(w + 256) + 2 * units;
-    a.dec.per_head = 1;
+    a.sel.kv_scored = flags + 2 * kv_units;
+    a.sel.kv_selected = flags + 3 * kv_units;
+    a.sel.union_idx = reinterpret_cast<int32_t*>(union_base);
+    a.sel.union_mask = reinterpret_cast<uint8_t*>(union_base + union_mask_off(kv));
+    a.sel.union_count = reinterpret_cast<int32_t*>(union_base + union_count_off(kv));
+    a.dec.mask = a.sel.union_mask;
+    a.dec.per_head = 0;
+    a.dec.max_sel = kv->max_pages;  // the union rows' stride
     a.n_sel = (int)units;
   }
   a.sel.meta_refresh = static_cast<unsigned char*>(meta);
@@ -617,7 +656,7 @@ static sa_status decode_step(const sa_kv_desc* kv, void* meta, sa_score_rule rul
     if (launch_step_cluster(c, C, (cudaStream_t)stream) == cudaSuccess) return SA_OK;
     cudaGetLastError();  // the cluster shape could not be launched here: use the persistent kernel
   }
-  const long long n_score = (per_head ? kv_units : units) * a.sel.splits, n_dec = plan.items;
+  const long long n_score = kv_units * a.sel.splits, n_dec = plan.items;
   if (n_score + a.n_sel + n_dec > 0x7fffffffLL) return SA_ERR_UNSUPPORTED;
   a.n_score = (int)n_score;
   a.n_dec = (int)n_dec;

@@ -73,13 +73,14 @@ static_assert(kDimsPerThread % 4 == 0, "merge writes float4");
 
 // Dynamic shared memory (offsets from a 1024-aligned base).
 constexpr int kOffBars = kRingBytes;
-constexpr int kOffTiles = kOffBars + kWarps * kStages * 8;
-constexpr int kOffPre = kOffTiles + kMaxItemTiles * 8;
-
 struct TileRef {
   int row;     // first tile row in the [B*Hkv*cap] row space (u * cap + token)
   int n;       // valid tokens (0 = empty tile)
+  int mask;    // the unit's query heads that attend the tile (bit j = head h0 + j)
 };
+
+constexpr int kOffTiles = kOffBars + kWarps * kStages * 8;
+constexpr int kOffPre = kOffTiles + kMaxItemTiles * (int)sizeof(TileRef);
 
 struct Smem {
   unsigned char* ring;   // [warp][stage][kTileBytes]
@@ -259,14 +260,17 @@ SA_DEV void decode_item(const DecodeArgs& a, const int u, const int split, const
   const long long row0 = (long long)um.kvu * a.kv.cap;
 
   // Token range of tile t of the unit (n = 0 for a skipped, invalid entry).
+  const uint8_t* mask_u = a.mask ? a.mask + (size_t)u * a.max_sel : nullptr;
   auto tile_ref = [&](int t) -> TileRef {
-    TileRef r{0, 0};
+    TileRef r{0, 0, 0xff};
     int start;
     if (ps > 0) {
       const int e = t / sub, part = t - e * sub;
       const int p = __ldcg(idx_u + e);
+      if (mask_u) r.mask = __ldcg(mask_u + e);
       if (p < 0 || p >= P) {
         flag_status(a.status, SA_ERR_DEVICE_CHECK);
+        r.n = 0;
         return r;
       }
       start = p * ps + part * 16;
@@ -278,6 +282,7 @@ SA_DEV void decode_item(const DecodeArgs& a, const int u, const int split, const
         if (pre[mid] <= t) lo = mid; else hi = mid - 1;
       }
       const int ch = __ldcg(idx_u + lo);
+      if (mask_u) r.mask = __ldcg(mask_u + lo);
       if (ch < 0 || ch >= P || off[ch] < 0) {
         flag_status(a.status, SA_ERR_DEVICE_CHECK);
         return r;
@@ -377,11 +382,13 @@ SA_DEV void decode_item(const DecodeArgs& a, const int u, const int split, const
         if (ks & 1) mma_bf16(s2, a0, a1, a2, a3, bq[2 * ks], bq[2 * ks + 1]);
         else        mma_bf16(s, a0, a1, a2, a3, bq[2 * ks], bq[2 * ks + 1]);
       }
+      // tokens gq / gq + 8 of the tile, heads 2c / 2c + 1 (those the tile's mask keeps)
       const bool v0 = gq < r.n, v1 = gq + 8 < r.n;
-      const float z0 = v0 ? (s[0] + s2[0]) * a.scale_log2 : ninf;
-      const float z1 = v0 ? (s[1] + s2[1]) * a.scale_log2 : ninf;
-      const float z2 = v1 ? (s[2] + s2[2]) * a.scale_log2 : ninf;
-      const float z3 = v1 ? (s[3] + s2[3]) * a.scale_log2 : ninf;
+      const bool k0 = (r.mask >> (2 * c)) & 1, k1 = (r.mask >> (2 * c + 1)) & 1;
+      const float z0 = v0 && k0 ? (s[0] + s2[0]) * a.scale_log2 : ninf;
+      const float z1 = v0 && k1 ? (s[1] + s2[1]) * a.scale_log2 : ninf;
+      const float z2 = v1 && k0 ? (s[2] + s2[2]) * a.scale_log2 : ninf;
+      const float z3 = v1 && k1 ? (s[3] + s2[3]) * a.scale_log2 : ninf;
       float mx0 = fmaxf(z0, z2), mx1 = fmaxf(z1, z3);
 #pragma unroll
       for (int o = 4; o < 32; o <<= 1) {

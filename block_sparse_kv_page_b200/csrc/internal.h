@@ -132,8 +132,14 @@ struct SelectArgs {
   int hold_flag_of;
   // per-query-head decode step: scoring items per (sequence, KV head) count
   // their completions here [B * Hkv]; the per-head selection items wait for
-  // the count to reach `splits`
+  // the count to reach `splits`, then count themselves in kv_selected; the
+  // last of a KV head's G builds the union of their page sets (union_idx /
+  // union_mask [B * Hkv][max_pages], union_count) for its decode items
   uint32_t* kv_scored;
+  uint32_t* kv_selected;
+  int32_t* union_idx;
+  uint8_t* union_mask;
+  int32_t* union_count;
 };
 cudaError_t launch_select(const SelectArgs& a, cudaStream_t st);
 
@@ -148,6 +154,7 @@ struct DecodeArgs {
   float scale_log2;           // scale * log2(e)
   const int32_t* idx;
   const int32_t* count;
+  const uint8_t* mask;        // nullable [units][max_sel]: bit j = query head h0 + j attends the entry
   int max_sel;
   float* out;
   __nv_bfloat16* out_bf16;    // non-null: the output goes here, rounded to bf16, instead of `out`

@@ -495,6 +495,49 @@ SA_DEV void select_unit_of(const SelectArgs& a, const int u, const SelSmem& S, c
   select_unit(a, u, b, N, P, S, sc_local);
 }
 
+// The union of the page sets that the G query heads of KV unit kvu selected
+// (rows b * Hq + g * G + j of sel_idx / sel_count, written earlier in the
+// launch and made visible to this CTA), with bit j of an entry's mask set
+// when head j kept the page: written to union_idx / union_mask in ascending
+// page order; returns the entry count (also stored in union_count).  Every
+// page is then streamed once for all the heads that kept it.  All threads
+// call it; `words` holds ceil(P / 4) words of shared memory.
+SA_DEV int build_union(const SelectArgs& a, const int kvu, const int P, uint32_t* words, uint32_t* scan) {
+  const int tid = threadIdx.x, nt = blockDim.x;
+  const int b = kvu / a.kv.Hkv, g = kvu - b * a.kv.Hkv;
+  const int nw = (P + 3) >> 2;
+  for (int i = tid; i < nw; i += nt) words[i] = 0u;
+  __syncthreads();
+  for (int j = 0; j < a.G; ++j) {
+    const int u = b * a.Hq + g * a.G + j;
+    const int n = min(__ldcg(a.sel_count + u), a.max_sel);
+    const int32_t* lst = a.sel_idx + (size_t)u * a.max_sel;
+    for (int e = tid; e < n; e += nt) {
+      const int p = __ldcg(lst + e);
+      if (p >= 0 && p < P) atomicOr(&words[p >> 2], (1u << j) << (8 * (p & 3)));
+    }
+  }
+  __syncthreads();
+  // compaction in page order: thread t takes pages [t per, (t + 1) per)
+  const int per = (P + nt - 1) / nt;
+  const int p0 = min(P, tid * per), p1 = min(P, p0 + per);
+  const uint8_t* m8 = reinterpret_cast<const uint8_t*>(words);
+  uint32_t cnt = 0;
+  for (int p = p0; p < p1; ++p) cnt += m8[p] ? 1u : 0u;
+  uint32_t total;
+  uint32_t pos = block_excl_scan(cnt, scan, total);
+  int32_t* uidx = a.union_idx + (size_t)kvu * a.kv.max_pages;
+  uint8_t* umask = a.union_mask + (size_t)kvu * a.kv.max_pages;
+  for (int p = p0; p < p1; ++p)
+    if (m8[p]) {
+      uidx[pos] = p;
+      umask[pos] = m8[p];
+      ++pos;
+    }
+  if (tid == 0) a.union_count[kvu] = (int)total;
+  return (int)total;
+}
+
 // FUSED (the decode step): refresh the newest page while scoring and publish
 // the unit's flag after selecting.
 // SCORE_ONLY: write the group scores and stop (no selection; the unit

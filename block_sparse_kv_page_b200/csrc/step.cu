@@ -93,9 +93,13 @@ SA_DEV bool wait_count(const uint32_t* count, uint32_t target, int* status, uint
 // Their scores still come from one scoring pass per (sequence, KV head)
 // (items [0, n_score) write the G heads' own score rows); items
 // [n_score, n_score + n_sel) are the per-head selections, each waiting
-// (bounded) until its KV head's scoring items are all done; the decode items
-// follow.  Every wait is on items handed out earlier that never wait on
-// later ones, so none can deadlock.
+// (bounded) until its KV head's scoring items are all done; the last of a KV
+// head's G selections builds the union of their page sets with a head mask
+// per page and publishes the KV head's flag.  The decode items follow, one
+// set per (sequence, KV head) over the union (a page is streamed once for
+// every head that kept it; each head attends only its own pages).  Every
+// wait is on items handed out earlier that never wait on later ones, so none
+// can deadlock.
 template <int RULE, bool PER_HEAD>
 __global__ void __launch_bounds__(kThreads, SA_STEP_CTAS_PER_SM)
     step_kernel(const __grid_constant__ StepArgs a) {
@@ -141,7 +145,7 @@ __global__ void __launch_bounds__(kThreads, SA_STEP_CTAS_PER_SM)
         dec::item_unit(a.dec, item - n_pre, u, split);
         // the sequence length is an input of the launch: its load (kept in a
         // register until after the wait) overlaps the acquire
-        const int ntok = a.dec.kv.seq_len[unit_map<PER_HEAD>(u, a.dec.kv.Hkv, a.dec.Hq, a.dec.G).b];
+        const int ntok = a.dec.kv.seq_len[u / a.dec.kv.Hkv];  // decode units: (sequence, KV head)
         const int cnt = wait_selected(a.sel.ws_count + u, a.sel.status, limit);  // acquire
         s_count = cnt;
         s_ntok = ntok;
@@ -161,17 +165,28 @@ __global__ void __launch_bounds__(kThreads, SA_STEP_CTAS_PER_SM)
       else
         sel::select_item<RULE, true, false>(a.sel, item / a.sel.splits, item % a.sel.splits, S, ws);
     } else if (PER_HEAD && item < n_pre) {
-      // one query head's selection from its score row; then its flag
-      const int u = item - a.n_score;
+      // one query head's selection from its score row; the KV head's last
+      // one builds the union of the G heads' sets and publishes its flag
+      const int u = item - a.n_score, b = u / a.sel.Hq;
+      const int kvu = b * a.sel.kv.Hkv + (u - b * a.sel.Hq) / a.sel.G;
       sel::select_unit_of(a.sel, u, S, nullptr, a.sel.Hq);
       __syncthreads();
-      if (threadIdx.x == 0 && a.sel.hold_flag_of != u + 1)
-        st_release_u32(&a.sel.ws_count[u], sel::kUnitSelected | (uint32_t)a.sel.sel_count[u]);
+      if (threadIdx.x == 0)
+        s_last = atom_add_acq_rel_u32(&a.sel.kv_selected[kvu], 1u) == (uint32_t)(a.sel.G - 1);
+      __syncthreads();
+      if (s_last) {
+        int N, P;
+        sel::unit_geometry(a.sel, b, N, P);
+        fence_proxy_async();  // the ring becomes the union's mask words
+        const int n = sel::build_union(a.sel, kvu, P, reinterpret_cast<uint32_t*>(base), s_scan);
+        __syncthreads();
+        if (threadIdx.x == 0) st_release_u32(&a.sel.ws_count[kvu], sel::kUnitSelected | (uint32_t)n);
+      }
     } else {
       int u, split;
       dec::item_unit(a.dec, item - n_pre, u, split);
       if (a.sel.k_new != nullptr && lane == 0) fence_proxy_async_global();  // appended rows, then TMA
-      dec::decode_item<PER_HEAD>(a.dec, u, split, D, ws, s_count, s_ntok);  // count from the unit's flag
+      dec::decode_item<false>(a.dec, u, split, D, ws, s_count, s_ntok);  // count from the unit's flag
     }
     fence_proxy_async();  // generic writes to the ring (keys, merge) before the next TMA writes
     __syncthreads();
@@ -189,13 +204,18 @@ __global__ void __launch_bounds__(kThreads, SA_STEP_CTAS_PER_SM)
   __syncthreads();
   if (s_last) {
     __threadfence();
-    const int units = a.sel.kv.B * (a.sel.per_head ? a.sel.Hq : a.sel.kv.Hkv);
+    // unit flags and split counters: one per (sequence, KV head) (per-head
+    // steps flag the KV heads' unions)
+    const int units = a.sel.kv.B * a.sel.kv.Hkv;
     for (int i = threadIdx.x; i < units; i += blockDim.x) {
       a.sel.ws_count[i] = 0;
       a.dec.ws_count[i] = 0;
     }
     if (PER_HEAD)
-      for (int i = threadIdx.x; i < a.sel.kv.B * a.sel.kv.Hkv; i += blockDim.x) a.sel.kv_scored[i] = 0;
+      for (int i = threadIdx.x; i < a.sel.kv.B * a.sel.kv.Hkv; i += blockDim.x) {
+        a.sel.kv_scored[i] = 0;
+        a.sel.kv_selected[i] = 0;
+      }
     if (threadIdx.x == 0) {
       a.queue[0] = 0;
       a.queue[1] = 0;

@@ -145,7 +145,9 @@ def test_step_parity(cuda_dev, R, rule, name):
 def test_step_per_head_parity(cuda_dev, R, rule, name):
     """The per-query-head step: every (sequence, query head) against the
     oracle run on that head alone, and against the separate per-head calls
-    (same page sets; outputs bit-identical except under a token budget)."""
+    (the same page sets bit for bit; outputs within 1e-5: the step decodes
+    each KV head's union of page sets once with per-head masks, the separate
+    call each head's own set)."""
     lay, ps, bd = _case(cuda_dev, name)
     s = R.run_step(lay, page_size=ps, rule=rule, budget=bd, scale=SCALE, stale=True, per_head=True)
     assert s["status"] == 0
@@ -154,7 +156,7 @@ def test_step_per_head_parity(cuda_dev, R, rule, name):
     assert st["max_out_err"] < 1e-4
     c = R.run_gpu(lay, page_size=ps, rule=rule, budget=bd, scale=SCALE, per_head=True)
     assert c["status"] == 0
-    _assert_same(s, c, lay, ps, f"{name}/{rule}/per-head", exact=bd["kind"] != "tokens")
+    _assert_same(s, c, lay, ps, f"{name}/{rule}/per-head", exact=False)
 
 
 @pytest.mark.parametrize("rule", ["envelope", "centroid"])
