@@ -6,35 +6,33 @@
 // entries are skipped.  Chunked-prefill rows attend causally: row r at
 // position q_pos0 + r sees only keys at positions <= its own.
 //
-// CTA = (tile, KV head, 128 query vectors), one CTA per SM; a query vector is
-// one (row, query head) pair of the tile and owns one TMEM lane.  The blocks
-// of the list run through a pipeline kDepth blocks deep: kDepth K/V stages in
-// shared memory and kDepth S/P buffers of 64 columns in tensor memory, with
-// the O accumulator (128 columns) beside them.  Warp-specialised, all waits
-// bounded:
-//   warp 4 (one thread)  streams each kept block (64 keys) of K and V by TMA
-//                        into stage i % kDepth (four 64-row x 128 B boxes),
-//                        once the PV of block i - kDepth has freed it;
-//   warp 5 (one thread)  issues S_i = Q K_i^T (M = 128 vectors, N = 64 keys,
-//                        K = 128 dims; K-major operands) kDepth - 1 blocks
-//                        ahead of the PVs, and O += [P_hi | P_lo] [V_i ; V_i]
-//                        (A = P read from tensor memory, N = 128 dims, K =
-//                        2 x 64 keys; V read MN-major) once P_i is written.
-//                        The MMAs run in issue order, so the S of block
-//                        i + kDepth - 1, written into the buffer of block
-//                        i - 1, follows the PV that read P_{i-1};
-//   warps 0-3            the softmax: thread = query vector (TMEM lane 32 w +
-//                        lane), its whole row of 64 keys: masks (causal,
-//                        cache end) only on the diagonal and cache-end blocks,
-//                        online softmax in the log2 domain against a
-//                        reference max, P split into a bf16 hi + lo pair
-//                        (error ~2^-17) stored over S as the PV's A operand.
-// With S computed kDepth - 1 blocks ahead, the softmax of block i + 1 starts
-// as soon as that of block i ends, and the tensor pipe holds the next blocks'
-// QKs and the PVs of the finished ones.  O stays in tensor memory; it is
-// rescaled in place only when a row's max grows past the reference by more
-// than 2^8.  Accumulation order per vector is the block order of the list, so
-// results do not depend on scheduling.
+// CTA = (tile, KV head, 256 query vectors) = two Q tiles of 128 vectors that
+// share every K/V block, one CTA per SM; a query vector is one (row, query
+// head) pair of the tile and owns one TMEM lane in its Q tile's columns.
+// Warp-specialised, all waits bounded:
+//   warp 8 (one thread)  streams each kept block (64 keys) of K and V by TMA
+//                        into a kStages ring (four 64-row x 128 B boxes);
+//   warp 9 + t (one thread) issues, for Q tile t and block i in order,
+//                        S = Q_t K_i^T (M = 128 vectors, N = 64 keys, K = 128
+//                        dims; K-major operands) into one of the tile's two
+//                        S/P buffers, then O_t += [P_hi | P_lo] . [V_{i-1} ;
+//                        V_{i-1}] (A = P read from tensor memory, N = 128
+//                        dims, K = 2 x 64 keys; V read MN-major) once
+//                        P_{i-1} is written; the tensor pipe interleaves the
+//                        two tiles' MMAs, so one tile's softmax and handoffs
+//                        overlap the other tile's MMAs;
+//   warps 0-3 / 4-7      the softmax of tile 0 / 1: thread = query vector
+//                        (TMEM lane 32 (warp % 4) + lane), its whole row of
+//                        64 keys: masks (causal, cache end) only on the
+//                        diagonal and cache-end blocks, online softmax in the
+//                        log2 domain against a reference max, P split into a
+//                        bf16 hi + lo pair (error ~2^-17) stored over S in
+//                        tensor memory as the PV MMA's A operand.
+// O stays in tensor memory; it is rescaled in place only when a row's max
+// grows past the reference by more than 2^8.  The MMAs of one issuing thread
+// run in issue order, so the S/P buffer of block i + 2 is written only after
+// the PV of block i has read it.  Accumulation order per vector is the block
+// order of the list, so results do not depend on scheduling.
 #include "common.cuh"
 #include "internal.h"
 #include "tcgen05.cuh"
@@ -43,30 +41,30 @@ namespace sa {
 namespace {
 
 constexpr int kBlk = 64;                       // keys per block
-constexpr int kSmWarps = 4;                    // softmax: one warp per TMEM lane quarter
-constexpr int kThreadsTc = 32 * (kSmWarps + 2);
+constexpr int kTiles = 2;                      // Q tiles of 128 vectors per CTA
+constexpr int kSmWarps = 4 * kTiles;           // softmax: one warp per TMEM lane quarter and tile
+constexpr int kThreadsTc = 32 * (kSmWarps + 1 + kTiles);
 constexpr int kProducerWarp = kSmWarps;
-constexpr int kMmaWarp = kSmWarps + 1;
-#ifndef SA_TA_DEPTH
-#define SA_TA_DEPTH 5
+constexpr int kMmaWarp0 = kSmWarps + 1;        // warp kMmaWarp0 + t issues tile t's MMAs
+#ifndef SA_TA_STAGES
+#define SA_TA_STAGES 3
 #endif
-constexpr int kDepth = SA_TA_DEPTH;            // blocks in flight: K/V stages and S/P buffers
+constexpr int kStages = SA_TA_STAGES;
 constexpr int kBox = kBlk * 128;               // 64 rows x 128 B
 constexpr int kStage = 4 * kBox;               // K lo | K hi | V lo | V hi = 32 KiB
-constexpr int kQChunk = 128 * 128;             // 128 vectors x 64 dims bf16
-constexpr int kQTile = 2 * kQChunk;            // 128 vectors x 128 dims bf16, two K chunks
+constexpr int kQTile = 2 * 128 * 128;          // 128 vectors x 128 dims bf16, two K chunks
 constexpr int kOffQ = 0;
-constexpr int kOffRing = kOffQ + kQTile;
-constexpr int kOffBars = kOffRing + kDepth * kStage;
-// per slot: kv full, kv empty, S full, P full, PV done; drain
-constexpr int kNumBars = 5 * kDepth + 1;
+constexpr int kOffRing = kOffQ + kTiles * kQTile;
+constexpr int kOffBars = kOffRing + kStages * kStage;
+// kv full/empty per stage; per tile and buffer: S full, P full, PV done; drain
+constexpr int kNumBars = 2 * kStages + 3 * kTiles * 2 + 1;
 constexpr int kOffList = kOffBars + kNumBars * 8 + 8;
-// tensor memory: S/P buffer b at columns [64 b, 64 b + 64) (64 fp32 S
-// columns; P's bf16 hi | lo pairs overwrite them), O at [384, 512)
-constexpr uint32_t kColO = 384;
-static_assert(64 * kDepth <= (int)kColO, "S/P buffers below the O accumulator");
+// tensor memory: tile t's two S/P buffers at columns [128 t, 128 t + 128) (64
+// fp32 columns each; P's bf16 hi | lo pairs overwrite them), its O
+// accumulator at [256 + 128 t, 256 + 128 t + 128)
+constexpr uint32_t kColSP = 0;
+constexpr uint32_t kColO = 256;
 static_assert(1024 + kOffList > 114 * 1024, "one CTA per SM: it allocates all 512 TMEM columns");
-static_assert(1024 + kOffList + 4096 <= 227 * 1024, "shared memory, with a list of up to 1023 blocks");
 
 // 2^x by the hardware approximation (relative error about 2^-22; 2^-inf = +0).
 SA_DEV float fast_exp2(float x) {
@@ -91,11 +89,11 @@ __global__ void __launch_bounds__(kThreadsTc, 1) tile_attn_tc_kernel(const __gri
   unsigned char* qs = base + kOffQ;
   unsigned char* ring = base + kOffRing;
   uint64_t* kv_full = reinterpret_cast<uint64_t*>(base + kOffBars);
-  uint64_t* kv_empty = kv_full + kDepth;
-  uint64_t* s_full = kv_empty + kDepth;
-  uint64_t* p_full = s_full + kDepth;
-  uint64_t* o_done = p_full + kDepth;  // the PV of the slot's block is done
-  uint64_t* drain = o_done + kDepth;
+  uint64_t* kv_empty = kv_full + kStages;
+  uint64_t* s_full = kv_empty + kStages;   // [tile][buffer]
+  uint64_t* p_full = s_full + 2 * kTiles;  // [tile][buffer]
+  uint64_t* o_full = p_full + 2 * kTiles;  // [tile][block parity]: PV of the block done
+  uint64_t* drain = o_full + 2 * kTiles;
   int* blist = reinterpret_cast<int*>(base + kOffList);
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -139,14 +137,16 @@ __global__ void __launch_bounds__(kThreadsTc, 1) tile_attn_tc_kernel(const __gri
   const float ninf = -__int_as_float(0x7f800000);
 
   if (tid == 0) {
-    for (int s = 0; s < kDepth; ++s) {
+    for (int s = 0; s < kStages; ++s) {
       mbar_init(kv_full + s, 1);
-      mbar_init(kv_empty + s, 1);  // the PV that read the stage commits
-      mbar_init(s_full + s, 1);
-      mbar_init(p_full + s, kSmWarps);
-      mbar_init(o_done + s, 1);
+      mbar_init(kv_empty + s, kTiles);  // each tile's MMA thread commits after its PV
     }
-    mbar_init(drain, 1);
+    for (int x = 0; x < 2 * kTiles; ++x) {
+      mbar_init(s_full + x, 1);
+      mbar_init(p_full + x, 4);  // the tile's four softmax warps
+      mbar_init(o_full + x, 1);
+    }
+    mbar_init(drain, kTiles);
     fence_barrier_init();
     prefetch_tmap(&a.tmap_k);
     prefetch_tmap(&a.tmap_v);
@@ -180,11 +180,11 @@ __global__ void __launch_bounds__(kThreadsTc, 1) tile_attn_tc_kernel(const __gri
   }
   const int nb = (int)nb_u;
 
-  // ---- the CTA's 128 query vectors: row vi of the K-major, 128B-swizzled Q
-  // (rows past V zero); 8 loads in flight per thread
+  // ---- the CTA's 256 query vectors: tile vi / 128, row vi % 128 of its
+  // K-major, 128B-swizzled Q (rows past V zero); 8 loads in flight per thread
   const __nv_bfloat16* Q = reinterpret_cast<const __nv_bfloat16*>(a.q);
-  const int v0 = mc * 128;
-  constexpr int kQPieces = 128 * 16;
+  const int v0 = mc * 128 * kTiles;
+  constexpr int kQPieces = 128 * kTiles * 16;
 #pragma unroll 1
   for (int b0 = 0; b0 < kQPieces; b0 += 8 * kThreadsTc) {
     uint4 rw[8];
@@ -201,7 +201,8 @@ __global__ void __launch_bounds__(kThreadsTc, 1) tile_attn_tc_kernel(const __gri
       const int x = b0 + i * kThreadsTc + tid;
       if (x >= kQPieces) continue;
       const int vi = x >> 4, d8 = x & 15;
-      *reinterpret_cast<uint4*>(qs + (d8 >> 3) * kQChunk + swz128(vi, d8 & 7)) = rw[i];
+      *reinterpret_cast<uint4*>(qs + (vi >> 7) * kQTile + (d8 >> 3) * (128 * 128) + swz128(vi & 127, d8 & 7)) =
+          rw[i];
     }
   }
   fence_proxy_async();  // generic writes (queries, list) before the async proxy reads them
@@ -212,13 +213,13 @@ __global__ void __launch_bounds__(kThreadsTc, 1) tile_attn_tc_kernel(const __gri
   int fail = 0;
 
   if (warp == kProducerWarp) {
-    // ---- TMA producer: block i -> stage i % kDepth (freed by the PV of block i - kDepth)
+    // ---- TMA producer: block i -> stage i % kStages (freed once both tiles' PV read it)
     if (lane == 0) {
       const long long rowbase = (long long)g * a.kv.cap;  // B == 1: unit = KV head
       int issued = 0;
       for (int i = 0; i < nb; ++i) {
-        const int s = i % kDepth;
-        if (i >= kDepth && !mbar_wait(kv_empty + s, ((i / kDepth) - 1) & 1u, a.status)) {
+        const int s = i % kStages;
+        if (i >= kStages && !mbar_wait(kv_empty + s, ((i / kStages) - 1) & 1u, a.status)) {
           fail = 1;
           break;
         }
@@ -232,85 +233,89 @@ __global__ void __launch_bounds__(kThreadsTc, 1) tile_attn_tc_kernel(const __gri
         issued = i + 1;
       }
       // every copy issued has landed before the CTA moves on (bounded)
-      for (int i = max(0, issued - kDepth); i < issued; ++i)
-        mbar_wait(kv_full + (i % kDepth), (i / kDepth) & 1u, nullptr);
+      for (int i = max(0, issued - kStages); i < issued; ++i)
+        mbar_wait(kv_full + (i % kStages), (i / kStages) & 1u, nullptr);
     }
-  } else if (warp == kMmaWarp) {
-    // ---- MMA issuer: the QKs of blocks 0 .. kDepth - 2 up front, then per
-    // block i: its PV once P_i is written, then the QK of block i + kDepth - 1
-    // (into the buffer of block i - 1, whose PV was issued before it)
+  } else if (warp >= kMmaWarp0) {
+    // ---- MMA issuer of tile tt, in order: QK of block i (its K/V stage
+    // landed; its S/P buffer was last read by the PV of block i - 2, issued
+    // before), then the PV of block i - 1 once P_{i-1} is written.  One thread
+    // per tile: an MMA issue returns about when the tensor pipe has taken the
+    // MMAs, so a single thread serving both tiles held each tile's PV behind
+    // the other tile's QKs; the pipe interleaves the two threads' MMAs.  A K/V
+    // stage is free once both tiles' PVs that read it are done.
+    const int tt = warp - kMmaWarp0;
     if (lane == 0) {
       const uint32_t idesc_s = tc::idesc_f32acc(tc::kFmtBF16, 128, kBlk);
       const uint32_t idesc_o = tc::idesc_f32acc(tc::kFmtBF16, 128, kHeadDim) | (1u << 16);  // V MN-major
-      auto qk = [&](int j) -> bool {
-        const int s = j % kDepth;
-        if (!mbar_wait(kv_full + s, (j / kDepth) & 1u, a.status)) return false;
+      const unsigned char* qt = qs + tt * kQTile;
+      auto pv = [&](int i) -> bool {
+        const int s = i % kStages, b = i & 1;
+        if (!mbar_wait(p_full + 2 * tt + b, (i >> 1) & 1u, a.status)) return false;
+        tc::fence_after_sync();
+        const unsigned char* vb = ring + s * kStage + 2 * kBox;
+#pragma unroll
+        for (int j = 0; j < 8; ++j)  // K = [P_hi keys 0-63 | P_lo keys 0-63], 16 per step
+          tc::mma_bf16_ts(tmem + kColO + 128u * tt, tmem + kColSP + 128u * tt + 64u * b + 8u * j,
+                          v_desc(vb + 16 * 128 * (j & 3)), idesc_o, i > 0 || j != 0);
+        tc::commit(o_full + 2 * tt + b);
+        tc::commit(kv_empty + s);
+        return true;
+      };
+      for (int i = 0; i < nb && !fail; ++i) {
+        const int s = i % kStages, b = i & 1;
+        if (!mbar_wait(kv_full + s, (i / kStages) & 1u, a.status)) {
+          fail = 1;
+          break;
+        }
         tc::fence_after_sync();
         const unsigned char* kb = ring + s * kStage;
 #pragma unroll
         for (int c = 0; c < 2; ++c)
 #pragma unroll
           for (int k = 0; k < 4; ++k)
-            tc::mma_bf16_ss(tmem + 64u * s, tc::smem_desc_sw128(qs + c * kQChunk + 32 * k),
+            tc::mma_bf16_ss(tmem + kColSP + 128u * tt + 64u * b, tc::smem_desc_sw128(qt + c * (128 * 128) + 32 * k),
                             tc::smem_desc_sw128(kb + c * kBox + 32 * k), idesc_s, (c | k) != 0);
-        tc::commit(s_full + s);
-        return true;
-      };
-      auto pv = [&](int i) -> bool {
-        const int s = i % kDepth;
-        if (!mbar_wait(p_full + s, (i / kDepth) & 1u, a.status)) return false;
-        tc::fence_after_sync();
-        const unsigned char* vb = ring + s * kStage + 2 * kBox;
-#pragma unroll
-        for (int j = 0; j < 8; ++j)  // K = [P_hi keys 0-63 | P_lo keys 0-63], 16 per step
-          tc::mma_bf16_ts(tmem + kColO, tmem + 64u * s + 8u * j, v_desc(vb + 16 * 128 * (j & 3)), idesc_o,
-                          i > 0 || j != 0);
-        tc::commit(o_done + s);
-        tc::commit(kv_empty + s);
-        return true;
-      };
-      for (int j = 0; j < min(nb, kDepth - 1) && !fail; ++j)
-        if (!qk(j)) fail = 1;
-      for (int i = 0; i < nb && !fail; ++i) {
-        if (!pv(i)) {
-          fail = 1;
-          break;
-        }
-        const int j = i + kDepth - 1;
-        if (j < nb && !qk(j)) fail = 1;
+        tc::commit(s_full + 2 * tt + b);
+        if (i > 0 && !pv(i - 1)) fail = 1;
       }
+      if (!fail && nb > 0 && !pv(nb - 1)) fail = 1;
       // every MMA issued has completed before TMEM is freed (bounded)
       tc::commit(drain);
       mbar_wait(drain, 0, nullptr);
     }
   } else {
-    // ---- softmax: TMEM lane r = 32 warp + lane is query vector v0 + r; the
-    // thread owns that vector's whole row
-    const int r = 32 * warp + lane;
-    const int v = v0 + r;
+    // ---- softmax of tile tt: TMEM lane r = 32 (warp % 4) + lane is query
+    // vector v0 + 128 tt + r; the thread owns that vector's whole row.
+    const int tt = warp >> 2, quarter = warp & 3;
+    const int r = 32 * quarter + lane;
+    const int v = v0 + 128 * tt + r;
     const bool vok = v < V;
     const int qpos = vok ? a.q_pos0 + row0 + v / G : -1;
-    const uint32_t lane_off = (uint32_t)(32 * warp) << 16;
-    const uint32_t sp_base = tmem + lane_off;
-    const uint32_t to = tmem + lane_off + kColO;
-    // PV of block j complete.  A slot's PV barrier never runs two phases
-    // ahead of a wait here: the PV of block j + kDepth needs P_{j + kDepth},
+    const uint32_t lane_off = (uint32_t)(32 * quarter) << 16;
+    const uint32_t sp_base = tmem + lane_off + kColSP + 128u * tt;
+    const uint32_t to = tmem + lane_off + kColO + 128u * tt;
+    uint64_t* s_full_t = s_full + 2 * tt;
+    uint64_t* p_full_t = p_full + 2 * tt;
+    uint64_t* o_full_t = o_full + 2 * tt;
+    // PV of block j complete.  A tile's PV barrier for one block parity never
+    // runs two phases ahead of a wait here: PV of block j + 2 needs P_{j+2},
     // which this thread writes later (or, after the loop, does not exist).
     auto wait_pv = [&](int j) -> bool {
-      const bool ok = mbar_wait(o_done + (j % kDepth), (j / kDepth) & 1u, a.status);
+      const bool ok = mbar_wait(o_full_t + (j & 1), (j >> 1) & 1u, a.status);
       return __all_sync(0xffffffffu, ok);
     };
     float mref = ninf, lh = 0.f;  // reference max (log2 units) and the row sum against it
     const float sl2 = a.scale_log2;
     for (int i = 0; i < nb; ++i) {
-      const int b = i % kDepth;
-      const bool ok = mbar_wait(s_full + b, (i / kDepth) & 1u, a.status);
+      const int b = i & 1;
+      const bool ok = mbar_wait(s_full_t + b, (i >> 1) & 1u, a.status);
       if (!__all_sync(0xffffffffu, ok)) {
         fail = 1;
         break;
       }
       tc::fence_after_sync();
-      const uint32_t ts = sp_base + 64u * b;  // S/P buffer of the block
+      const uint32_t ts = sp_base + 64u * b;
       uint32_t r0[16], r1[16], r2[16], r3[16];  // keys 0-15, 16-31, 32-47, 48-63
       tc::ld_32x32b_x16(ts, r0);
       tc::ld_32x32b_x16(ts + 16, r1);
@@ -391,9 +396,10 @@ __global__ void __launch_bounds__(kThreadsTc, 1) tile_attn_tc_kernel(const __gri
         tc::st_32x32b_x16(ts + 32 + 16 * h2, plo);
       }
       lh += (rq[0] + rq[1]) + (rq[2] + rq[3]);
-      // V rows past the cache end hold other data: zero them before PV reads them
+      // V rows past the cache end hold other data: zero them before PV reads
+      // them (each tile's warps do it, as each tile's PV waits only for its own)
       if (kb0 + kBlk > N) {
-        unsigned char* st = ring + b * kStage;
+        unsigned char* st = ring + (i % kStages) * kStage;
         for (int x = r; x < (kb0 + kBlk - N) * 16; x += 128) {
           const int row = (N - kb0) + (x >> 4), ch = x & 15;
           *reinterpret_cast<uint4*>(st + (2 + (ch >> 3)) * kBox + swz128(row, ch & 7)) = make_uint4(0u, 0u, 0u, 0u);
@@ -403,7 +409,7 @@ __global__ void __launch_bounds__(kThreadsTc, 1) tile_attn_tc_kernel(const __gri
       tc::wait_st();
       tc::fence_before_sync();  // P and the rescaled O before PV_i reads them
       __syncwarp();
-      if (lane == 0) mbar_arrive(p_full + b);
+      if (lane == 0) mbar_arrive(p_full_t + b);
     }
     // the row's output: PV of the last block (the earlier ones ran before it),
     // then O / l straight from tensor memory
@@ -454,7 +460,7 @@ cudaError_t launch_tile_attn_tc(const TileAttnArgs& a, cudaStream_t st) {
   return cudaGetLastError();
 }
 
-// CTAs per (tile, KV head): 128 query vectors each.
-int tile_attn_tc_mchunks(int vectors_per_tile) { return (vectors_per_tile + 127) / 128; }
+// CTAs per (tile, KV head): 256 query vectors each.
+int tile_attn_tc_mchunks(int vectors_per_tile) { return (vectors_per_tile + 128 * kTiles - 1) / (128 * kTiles); }
 
 }  // namespace sa
