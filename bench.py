@@ -1134,15 +1134,23 @@ def main():
         "selected_token_fraction": round(args.budget / N, 4),
         "per_kernel_ms": {k: round(v, 5) for k, v in kern.items()} if kern else None,
         "roofline": roof, "clocks": r["clocks"],
-        "e2e": {"value": r["job_tok_heads"] / (r["e2e_ms"] * 1e-3), "unit": UNIT,
-                "ms_per_step": round(r["e2e_ms"], 5), "h2d_bytes_per_step": r["h2d"],
-                "d2h_bytes_per_step": r["d2h"]},
+        # end to end through the public API: each step's inputs cross from
+        # pinned host memory in one copy, and the fp32 result reaches host
+        # memory -- written there by the step itself where the mode allows
+        # it (the same bits as a copy after the launch, which is reported
+        # beside it), else copied back after the launch
+        "e2e": ({"value": r["job_tok_heads"] / (r["e2e_zc"]["ms_per_step"] * 1e-3), "unit": UNIT,
+                 **r["e2e_zc"]} if r["e2e_zc"] is not None else
+                {"value": r["job_tok_heads"] / (r["e2e_ms"] * 1e-3), "unit": UNIT,
+                 "ms_per_step": round(r["e2e_ms"], 5), "h2d_bytes_per_step": r["h2d"],
+                 "d2h_bytes_per_step": r["d2h"]}),
+        "e2e_copy_out": {"value": r["job_tok_heads"] / (r["e2e_ms"] * 1e-3), "unit": UNIT,
+                         "ms_per_step": round(r["e2e_ms"], 5), "h2d_bytes_per_step": r["h2d"],
+                         "d2h_bytes_per_step": r["d2h"],
+                         "note": "the fp32 result copied to pinned host memory after the launch"},
         "e2e_bf16_out": None if r["e2e_bf16"] is None else {
             "value": r["job_tok_heads"] / (r["e2e_bf16"]["ms_per_step"] * 1e-3),
             "unit": UNIT, **r["e2e_bf16"]},
-        "e2e_host_written_out": None if r["e2e_zc"] is None else {
-            "value": r["job_tok_heads"] / (r["e2e_zc"]["ms_per_step"] * 1e-3),
-            "unit": UNIT, **r["e2e_zc"]},
         "gpu_launches": r["launches_per_step"] * args.steps,
         "cpu_baseline": cpu, "modes": r["extra"],
         "router": None if r["router"] is None else {
