@@ -206,3 +206,24 @@ def test_decode_static_rejects_tile_attention(lib, abi):
     r = lib.sparse_attn_decode_static(C.byref(d), 0x50000, 32, 3, 0, 1, 0.088, 0x60000, 0x70000, 16,
                                       0x80000, None, None, None)
     assert r == abi.SA_ERR_INVALID
+
+
+def test_route_decode_step_validation(lib, abi):
+    """The one-launch decode router validates on the host like the separate
+    router call: chunks unsupported, quantile in [0, 1], rho*k bounded, a
+    workspace that holds the scores, router tables and both windows' partials."""
+    ok = _desc(abi)
+
+    def call(desc=ok, k=8, rho=2, quantile=0.25, scale=0.088, ws_bytes=1 << 30, out=0x80000):
+        return lib.sparse_attn_route_decode_step(C.byref(desc), 0x40000, 0, 0x50000, 32, k, rho, quantile, None,
+                                                 scale, 0x60000, 0x70000, 0x90000, 0xa0000, 0xb0000, None, out,
+                                                 None, 0x100000, ws_bytes, None)
+    assert call(desc=_desc(abi, page_size=0, chunk_off=0x30000, n_chunks=0x30100)) == abi.SA_ERR_UNSUPPORTED
+    assert call(quantile=1.5) == abi.SA_ERR_INVALID
+    assert call(k=0) == abi.SA_ERR_INVALID
+    assert call(k=512, rho=2) == abi.SA_ERR_UNSUPPORTED           # rho * k > 1023
+    assert call(scale=float("nan")) == abi.SA_ERR_INVALID
+    assert call(out=0x80004) == abi.SA_ERR_INVALID                # misaligned output
+    need = lib.sparse_attn_workspace_size(C.byref(ok), 32, 1, 16)
+    assert need > 0
+    assert call(ws_bytes=need - 256) == abi.SA_ERR_WORKSPACE

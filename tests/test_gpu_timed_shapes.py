@@ -205,3 +205,26 @@ def test_needle_workload(cuda_dev, R, rule, seed_offset):
         c = int(sep["sel_count"][0, g])
         kept += len(set(pages) & set(sep["sel_idx"][0, g, :c].tolist()))
     print(f"\nneedles {rule} seed {seed_offset}: {kept} of 12 needle pages kept, {st}")
+
+
+# --------------------------------------------------------------------------- per-query-head launch
+@pytest.mark.slow
+@pytest.mark.parametrize("rule", ["envelope", "centroid"])
+def test_per_head_step_48_layers(cuda_dev, R, qwen3vl_48, rule):
+    """The per-query-head step in the benchmark's launch (48 stacked layers,
+    1,536 (layer, query head) units, top 256 pages each): page sets equal the
+    separate per-head calls' on every unit, outputs within 1e-5 of them, and
+    96 sampled units against the oracle applied to each head alone."""
+    lay = qwen3vl_48
+    bd = {"kind": "topk", "k": 256}
+    g = R.run_step(lay, page_size=16, rule=rule, budget=bd, scale=SCALE, stale=True, per_head=True)
+    assert g["status"] == 0
+    sep = R.run_gpu(lay, page_size=16, rule=rule, budget=bd, scale=SCALE, per_head=True)
+    assert sep["status"] == 0
+    assert torch.equal(g["sel_count"], sep["sel_count"]) and torch.equal(g["sel_idx"], sep["sel_idx"])
+    assert float((g["out"] - sep["out"]).abs().max()) < 1e-5
+    rng = np.random.default_rng(11)
+    units = [(int(b), int(h)) for b, h in zip(rng.integers(0, 48, 96), rng.integers(0, 32, 96))]
+    st = R.check_units_parallel(lay, [(g, rule, bd)], page_size=16, scale=SCALE, units=units, per_head=True)
+    assert st[0]["units"] == 96 and st[0]["max_out_err"] < 1e-4
+    print(f"\nper-head {rule}: {st[0]}")
