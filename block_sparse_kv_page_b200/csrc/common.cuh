@@ -142,31 +142,11 @@ SA_DEV uint32_t cluster_id_x() {
 SA_DEV void cluster_sync() {
   asm volatile("barrier.cluster.arrive.release.aligned;\nbarrier.cluster.wait.acquire.aligned;\n" ::: "memory");
 }
-// The two halves of cluster_sync, for work in between.
-SA_DEV void cluster_arrive() { asm volatile("barrier.cluster.arrive.release.aligned;\n" ::: "memory"); }
-SA_DEV void cluster_wait() { asm volatile("barrier.cluster.wait.acquire.aligned;\n" ::: "memory"); }
-// One-way signals between the CTAs of a cluster: an arrive (release at
-// cluster scope) on an mbarrier in the shared memory of CTA `rank`, and a
-// bounded wait (acquire at cluster scope) on one of this CTA's own.
-SA_DEV void mbar_arrive_cluster(const uint64_t* bar, uint32_t rank) {
-  uint32_t remote;
-  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;\n" : "=r"(remote) : "r"(smem_addr(bar)), "r"(rank));
-  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];\n" ::"r"(remote) : "memory");
-}
-SA_DEV bool mbar_wait_cluster(uint64_t* bar, uint32_t parity, int* status) {
-  for (uint32_t i = 0; i < kSpinLimit; ++i) {
-    uint32_t ok;
-    asm volatile(
-        "{\n .reg .pred p;\n mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n"
-        " selp.u32 %0, 1, 0, p;\n}\n"
-        : "=r"(ok)
-        : "r"(smem_addr(bar)), "r"(parity)
-        : "memory");
-    if (ok) return true;
-  }
-  flag_status(status, SA_ERR_TIMEOUT);
-  return false;
-}
+// The two halves of cluster_sync, for work in between: a relaxed arrive
+// (orders nothing; says "this CTA runs") and an acquire wait that the threads
+// of a warp may reach at different points.
+SA_DEV void cluster_arrive_relaxed() { asm volatile("barrier.cluster.arrive.relaxed.aligned;\n" ::: "memory"); }
+SA_DEV void cluster_wait() { asm volatile("barrier.cluster.wait.acquire;\n" ::: "memory"); }
 // Start moving the 128-byte line at p into L2 (no register written).
 SA_DEV void prefetch_l2(const void* p) { asm volatile("prefetch.global.L2 [%0];\n" ::"l"(p)); }
 SA_DEV void prefetch_tmap(const void* tmap) {

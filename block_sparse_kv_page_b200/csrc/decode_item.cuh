@@ -185,12 +185,10 @@ SA_DEV void merge_splits(const DecodeArgs& a, const float* base, const int split
 // part_dst (several splits only): write the split's partial to part_dst +
 // split * kPartStride (another CTA's shared memory, say) and return; the
 // caller merges (merge_splits) once every split's partial is there.
-// list (non-null): the unit's kept entries, already in this CTA's shared
-// memory (n_known must be given), instead of a.idx.
 template <bool PER_HEAD = false, int STAGES = kStages>
 SA_DEV void decode_item(const DecodeArgs& a, const int u, const int split, const Smem& sm,
                         WarpState& ws, const int n_known = -1, const int n_tok_known = -1,
-                        float* part_dst = nullptr, const int32_t* list = nullptr) {
+                        float* part_dst = nullptr) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int gq = lane >> 2, c = lane & 3;
   const UnitMap um = unit_map<PER_HEAD>(u, a.kv.Hkv, a.Hq, a.G);
@@ -204,9 +202,7 @@ SA_DEV void decode_item(const DecodeArgs& a, const int u, const int split, const
   int n_ent = n_known >= 0 ? n_known : __ldcg(a.count + u);  // L2: may be written earlier in the launch
   if (n_ent < 0 || n_ent > a.max_sel) bad = true;
   if (bad) n_ent = 0;
-  const int32_t* idx_u = list ? list : a.idx + (size_t)u * a.max_sel;
-  // an entry of the list: shared memory, or global memory written earlier in the launch
-  auto entry = [&](int e) -> int { return list ? list[e] : __ldcg(idx_u + e); };
+  const int32_t* idx_u = a.idx + (size_t)u * a.max_sel;
   const int ps = a.kv.page_size;
   const int sub = ps > 0 ? ps / 16 : 0;
   int P = 0;
@@ -223,7 +219,7 @@ SA_DEV void decode_item(const DecodeArgs& a, const int u, const int split, const
     const int e0 = min(n_ent, tid * per), e1 = min(n_ent, e0 + per);
     uint32_t loc = 0;
     for (int e = e0; e < e1; ++e) {
-      const int ch = entry(e);
+      const int ch = __ldcg(idx_u + e);
       int nt = 0;
       if (ch >= 0 && ch < P && off[ch] >= 0) nt = (max(0, min(off[ch + 1], N) - off[ch]) + 15) >> 4;
       pre[e] = nt;
@@ -270,7 +266,7 @@ SA_DEV void decode_item(const DecodeArgs& a, const int u, const int split, const
     int start;
     if (ps > 0) {
       const int e = t / sub, part = t - e * sub;
-      const int p = entry(e);
+      const int p = __ldcg(idx_u + e);
       if (mask_u) r.mask = __ldcg(mask_u + e);
       if (p < 0 || p >= P) {
         flag_status(a.status, SA_ERR_DEVICE_CHECK);
@@ -285,7 +281,7 @@ SA_DEV void decode_item(const DecodeArgs& a, const int u, const int split, const
         const int mid = (lo + hi + 1) >> 1;
         if (pre[mid] <= t) lo = mid; else hi = mid - 1;
       }
-      const int ch = entry(lo);
+      const int ch = __ldcg(idx_u + lo);
       if (mask_u) r.mask = __ldcg(mask_u + lo);
       if (ch < 0 || ch >= P || off[ch] < 0) {
         flag_status(a.status, SA_ERR_DEVICE_CHECK);

@@ -547,10 +547,18 @@ SA_DEV int build_union(const SelectArgs& a, const int kvu, const int P, uint32_t
 // HEAD_ROWS (with SCORE_ONLY, per (sequence, KV head) units): the G query
 // heads' own scores go to their rows b * Hq + h of the workspace (no group
 // max), and the item then counts itself done in a.kv_scored[u] (release).
-template <int RULE, bool FUSED, bool PER_HEAD = false, bool SCORE_ONLY = false, bool HEAD_ROWS = false>
+// CL_WAIT (a cluster launch whose CTAs arrived on the cluster barrier after
+// setting up): each thread waits on that barrier before its first store to
+// score_dst (another CTA's shared memory, which must be running), or at the
+// end if it stores none -- once the first tile is scored, so the wait
+// overlaps the first metadata load.
+template <int RULE, bool FUSED, bool PER_HEAD = false, bool SCORE_ONLY = false, bool HEAD_ROWS = false,
+          bool CL_WAIT = false>
 SA_DEV void select_item(const SelectArgs& a, const int u, const int split, const SelSmem& S,
                         WarpState& ws, float* score_dst = nullptr) {
   static_assert(!HEAD_ROWS || (SCORE_ONLY && !PER_HEAD), "head rows: score-only items of KV units");
+  static_assert(!CL_WAIT || (SCORE_ONLY && !HEAD_ROWS), "cluster wait: score-only items");
+  bool cl_waited = !CL_WAIT;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int gq = lane >> 2, c = lane & 3;
   const int Hkv = a.kv.Hkv;
@@ -754,6 +762,10 @@ SA_DEV void select_item(const SelectArgs& a, const int u, const int split, const
     mlo = fmaxf(mlo, __shfl_xor_sync(0xffffffffu, mlo, 2));
     mhi = fmaxf(mhi, __shfl_xor_sync(0xffffffffu, mhi, 1));
     mhi = fmaxf(mhi, __shfl_xor_sync(0xffffffffu, mhi, 2));
+    if (!cl_waited) {
+      cluster_wait();
+      cl_waited = true;
+    }
     if (c < 2) {
       const int page = t * 16 + gq + 8 * c;
       const float s = c == 0 ? mlo : mhi;
@@ -764,6 +776,7 @@ SA_DEV void select_item(const SelectArgs& a, const int u, const int split, const
     }
   }
   ws.gi += (uint32_t)n_it;
+  if (!cl_waited) cluster_wait();
   if (HEAD_ROWS) {
     __syncthreads();  // then one acq_rel increment publishes the CTA's score rows
     if (tid == 0) atom_add_acq_rel_u32(&a.kv_scored[u], 1u);

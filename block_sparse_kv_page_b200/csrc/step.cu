@@ -225,30 +225,28 @@ __global__ void __launch_bounds__(kThreads, SA_STEP_CTAS_PER_SM)
 
 // The decode step for few units (a single layer at batch 1, say): one
 // thread-block cluster of C CTAs per unit (sequence, KV head), one CTA per
-// SM, so the handoffs between stages are signals through distributed shared
-// memory instead of global item claims, flag polls and L2 round trips:
+// SM, so the handoffs between stages are cluster barriers and distributed
+// shared memory instead of global item claims, flag polls and L2 round trips:
 //  1. CTA r scores tile range r of C (the one holding the newest page also
-//     refreshes it), writes the group scores straight into the leader's
-//     (rank 0) shared memory, and signals the leader (a release arrive on
-//     the leader's mbarrier);
-//  2. the leader, once all C have arrived (acquire), selects the unit's
-//     pages from its shared memory, writes them out, copies the kept list
-//     and its count into every CTA's shared memory and signals each;
-//  3. CTA r runs decode splits r, r + C, ... from its local copy of the list
-//     with a deeper TMA ring (kClStages per warp: a split's tiles are all in
-//     flight at once).  With exactly C splits each CTA writes its partial
-//     into the leader's shared memory and signals it; the leader merges in
-//     split order.  With more, the splits merge through the workspace as in
-//     the persistent kernel.
-// A split cluster barrier (arrive after the barrier set-up, wait before the
-// first access to another CTA's shared memory) makes sure every CTA of the
-// cluster is running and its barriers are initialised.  The same item code
-// and splits as the separate calls and the same merge arithmetic, so results
-// are identical to them.
+//     refreshes it) and writes the group scores straight into the leader's
+//     (rank 0) shared memory -- after a cluster barrier that every CTA
+//     arrives on once its set-up is done and waits on only before its first
+//     such store, so the leader is known to run and the wait overlaps the
+//     first metadata load;
+//  2. cluster barrier; the leader selects the unit's pages from its shared
+//     memory and writes them out;
+//  3. cluster barrier; CTA r runs decode splits r, r + C, ... with a deeper
+//     TMA ring (kClStages per warp: a split's tiles are all in flight at
+//     once).  With exactly C splits each CTA writes its partial into the
+//     leader's shared memory and, after a last barrier, the leader merges
+//     them; with more, the splits merge through the workspace as in the
+//     persistent kernel.
+// The same item code and splits as the separate calls and the same merge
+// arithmetic, so results are identical to them.
 constexpr int kClStages = 4;  // decode ring depth per warp in the cluster kernel
 
 struct ClusterLayout {
-  int ring, bars_sel, bars_dec, bars_cl, tiles, pre, list, scores, parts, total;
+  int ring, bars_sel, bars_dec, tiles, pre, scores, parts, total;
 };
 __host__ __device__ inline ClusterLayout cluster_layout(int max_pages, int max_sel, bool chunks, int C,
                                                         bool local_merge) {
@@ -258,11 +256,9 @@ __host__ __device__ inline ClusterLayout cluster_layout(int max_pages, int max_s
   L.ring = 0;
   L.bars_sel = sel_body > dec_ring ? sel_body : dec_ring;
   L.bars_dec = L.bars_sel + kBarBytes;
-  L.bars_cl = L.bars_dec + dec::kWarps * kClStages * 8;    // scores in, list in, partials in; count word
-  L.tiles = L.bars_cl + 32;
+  L.tiles = L.bars_dec + dec::kWarps * kClStages * 8;
   L.pre = L.tiles + kTileRefBytes;
-  L.list = (L.pre + (chunks ? (max_sel + 1) * 4 : 0) + 15) & ~15;
-  L.scores = (L.list + max_sel * 4 + 15) & ~15;
+  L.scores = (L.pre + (chunks ? (max_sel + 1) * 4 : 0) + 15) & ~15;
   L.parts = (L.scores + ((max_pages + 3) & ~3) * 4 + 15) & ~15;
   L.total = L.parts + (local_merge ? C * dec::kPartStride * 4 : 0);
   return L;
@@ -284,11 +280,6 @@ __global__ void __launch_bounds__(kThreads, 1) step_cluster_kernel(const __grid_
                                           local_merge);
   uint64_t* bars_sel = reinterpret_cast<uint64_t*>(base + Lo.bars_sel);
   uint64_t* bars_dec = reinterpret_cast<uint64_t*>(base + Lo.bars_dec);
-  uint64_t* scores_in = reinterpret_cast<uint64_t*>(base + Lo.bars_cl);  // leader: C score arrivals
-  uint64_t* list_in = scores_in + 1;                                      // every CTA: the list is here
-  uint64_t* parts_in = scores_in + 2;                                     // leader: C partial arrivals
-  int* my_count = reinterpret_cast<int*>(scores_in + 3);
-  int32_t* my_list = reinterpret_cast<int32_t*>(base + Lo.list);
   float* my_scores = reinterpret_cast<float*>(base + Lo.scores);
   float* my_parts = reinterpret_cast<float*>(base + Lo.parts);
   const sel::SelSmem S{base, bars_sel, s_hist, s_scan, s_bc, &s_last};
@@ -301,59 +292,37 @@ __global__ void __launch_bounds__(kThreads, 1) step_cluster_kernel(const __grid_
   if (lane == 0) {
     for (int s = 0; s < kStages; ++s) mbar_init(bars_sel + warp * kStages + s, 1);
     for (int s = 0; s < kClStages; ++s) mbar_init(bars_dec + warp * kClStages + s, 1);
+    fence_barrier_init();
   }
   if (threadIdx.x == 0) {
-    mbar_init(scores_in, C);
-    mbar_init(list_in, 1);
-    mbar_init(parts_in, C);
     prefetch_tmap(&a.sel.tmap_meta);
     prefetch_tmap(&a.dec.tmap_k);
     prefetch_tmap(&a.dec.tmap_v);
   }
-  if (lane == 0) fence_barrier_init();
   __syncthreads();
-  cluster_arrive();    // this CTA runs and its barriers are set up (waited for before any remote access)
-  grid_dep_wait();     // the previous kernel of the stream has completed (no global access before)
-  grid_dep_trigger();  // the next kernel may be scheduled now; it waits for this one to complete
+  cluster_arrive_relaxed();  // this CTA runs (waited for before the first store to the leader)
+  grid_dep_wait();           // the previous kernel of the stream has completed (no global access before)
+  grid_dep_trigger();        // the next kernel may be scheduled now; it waits for this one to complete
   WarpState ws{0u, true, 0u, 0u};
-  // 1. scoring of tile range r of C (a.sel.splits == C): the metadata TMA and
-  // the MMAs run before the wait below; the scores go to the leader
-  cluster_wait();
-  sel::select_item<RULE, true, false, true>(a.sel, u, r, S, ws, lead_scores);
+  // 1. scoring of tile range r of C (a.sel.splits == C), scores to the leader
+  sel::select_item<RULE, true, false, true, false, true>(a.sel, u, r, S, ws, lead_scores);
   if (!ws.alive && lane == 0) {  // a wait timed out: let the copies in flight land (bounded)
     for (uint32_t g = ws.drain_lo; g < ws.drain_hi; ++g)
       mbar_wait(bars_sel + warp * kStages + g % kStages, (g / kStages) & 1u, nullptr);
   }
   fence_proxy_async();  // generic writes to the ring (the refresh patch) before it is reused
   __syncthreads();
-  if (threadIdx.x == 0) mbar_arrive_cluster(scores_in, 0);  // release: this CTA's scores
-  // 2. the leader selects, then hands the kept list to every CTA
-  int cnt = 0;
-  if (r == 0) {
-    mbar_wait_cluster(scores_in, 0, a.sel.status);  // bounded; a timeout is in the status word
-    sel::select_unit_of(a.sel, u, S, my_scores, a.sel.kv.Hkv);
-    __syncthreads();
-    cnt = min(__ldcg(a.sel.sel_count + u), a.dec.max_sel);
-    const int32_t* sel_u = a.sel.sel_idx + (size_t)u * a.sel.max_sel;
-    for (int rr = 0; rr < C; ++rr) {
-      int32_t* dst = cl.map_shared_rank(my_list, rr);
-      for (int e = threadIdx.x; e < cnt; e += blockDim.x) dst[e] = __ldcg(sel_u + e);
-      if (threadIdx.x == 0) *cl.map_shared_rank(my_count, rr) = cnt;
-    }
-    fence_proxy_async();  // the ring held the keys: generic writes before the decode TMA writes
-    __syncthreads();
-    if (threadIdx.x < C) mbar_arrive_cluster(list_in, threadIdx.x);
-    cluster_arrive();  // the leader's last access to another CTA's shared memory is done
-  }
-  if (!mbar_wait_cluster(list_in, 0, a.sel.status) && threadIdx.x == 0) *my_count = 0;
+  cluster_sync();       // every range's scores are in the leader's shared memory
+  // 2. the leader selects
+  if (r == 0) sel::select_unit_of(a.sel, u, S, my_scores, a.sel.kv.Hkv);
+  fence_proxy_async();  // the ring held the keys: generic writes before the decode TMA writes
   __syncthreads();
-  cnt = *my_count;
-  // 3. decode splits r, r + C, ... from the local copy of the list
+  cluster_sync();       // the selection is visible to every CTA of the cluster
+  // 3. decode splits r, r + C, ... (each reads the kept count and pages)
   if (a.sel.k_new != nullptr && lane == 0) fence_proxy_async_global();  // appended rows, then TMA
   WarpState wd{0u, ws.alive, 0u, 0u};
   for (int split = r; split < a.dec.splits; split += C) {
-    dec::decode_item<false, kClStages>(a.dec, u, split, D, wd, cnt, -1, local_merge ? lead_parts : nullptr,
-                                       my_list);
+    dec::decode_item<false, kClStages>(a.dec, u, split, D, wd, -1, -1, local_merge ? lead_parts : nullptr);
     fence_proxy_async();
     __syncthreads();
   }
@@ -361,22 +330,16 @@ __global__ void __launch_bounds__(kThreads, 1) step_cluster_kernel(const __grid_
     for (uint32_t g = wd.drain_lo; g < wd.drain_hi; ++g)
       mbar_wait(bars_dec + warp * kClStages + g % kClStages, (g / kClStages) & 1u, nullptr);
   }
-  if (local_merge && threadIdx.x == 0) mbar_arrive_cluster(parts_in, 0);  // release: this CTA's partial
-  // no CTA leaves while another may still access its shared memory: each
-  // arrives after its last remote access (the leader above, after handing out
-  // the list) and waits here, at its end
-  if (r != 0) cluster_arrive();
-  if (local_merge && r == 0) {
+  if (local_merge) {
+    cluster_sync();  // every split's partial is in the leader's shared memory
     const int h = threadIdx.x / dec::kThreadsPerHead;
     const int d0 = (threadIdx.x % dec::kThreadsPerHead) * dec::kDimsPerThread;
-    const bool ok = mbar_wait_cluster(parts_in, 0, a.sel.status);
-    if (ok && h < a.dec.G) {
+    if (r == 0 && h < a.dec.G) {
       const int b = u / a.dec.kv.Hkv, g = u - b * a.dec.kv.Hkv;
       dec::merge_splits<true>(a.dec, my_parts + h * dec::kPartHead, C,
                               (size_t)b * a.dec.Hq + (size_t)g * a.dec.G + h, d0);
     }
   }
-  cluster_wait();
 }
 
 // The router applied to decode in one launch (see RouteStepArgs).  Queue:
