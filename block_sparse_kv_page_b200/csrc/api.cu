@@ -120,10 +120,10 @@ int max_tiles_per_unit(const sa_kv_desc* kv, int max_sel) {
 // selecting CTA can read a row with 16-byte loads.
 int score_stride(const sa_kv_desc* kv) { return (kv->max_pages + 3) & ~3; }
 
-// Decode router scratch after the scores: lists [units][W], sigma (double)
-// and eligible counts per unit.
+// Decode router scratch after the scores: sigma (double) and eligible
+// counts per unit, and (routed decode step) the triggered units' list.
 size_t route_decode_ws_bytes(long long units) {
-  return align256((size_t)units * 8) + align256((size_t)units * 4);
+  return align256((size_t)units * 8) + align256((size_t)units * 4) + align256((size_t)units * 16);
 }
 
 size_t select_scratch(const sa_kv_desc* kv, bool per_head = false, int n_q_heads = 0) {
@@ -415,9 +415,10 @@ size_t sparse_attn_workspace_size(const sa_kv_desc* kv, int32_t n_q_heads, int32
     const long long ru = (long long)kv->batch * kv->n_kv_heads;
     size_t rd = select_scratch(kv) + route_decode_ws_bytes(ru);
     // the routed decode step adds split partials of its top-k and expansion
-    // windows, each at most the splits of a plain decode over max_sel
+    // windows, each at most the splits of a plain decode over max_sel, and
+    // one merged top-k partial per unit
     const DecodePlan rp = decode_plan((int)ru, max_tiles_per_unit(kv, max_sel), sm);
-    rd += decode_scratch(DecodePlan{2 * rp.splits, (int)ru, 2 * rp.splits, ru * 2 * rp.splits});
+    rd += decode_scratch(DecodePlan{2 * rp.splits, (int)ru, 2 * rp.splits, ru * (2 * rp.splits + 1)});
     if (rd > tail) tail = rd;
   }
   return kScratch + tail;
@@ -812,7 +813,7 @@ sa_status sparse_attn_route_decode(const sa_kv_desc* kv, const void* meta, sa_sc
   const size_t sel_bytes = select_scratch(kv);
   const size_t need = kScratch + sel_bytes + route_decode_ws_bytes(units);
   if ((s = check_ws(ws, ws_bytes, need)) != SA_OK) return s;
-  if (route_decode_smem_bytes(kv->max_pages, (int)W, k, kv->batch) > 227 * 1024) return SA_ERR_UNSUPPORTED;
+  if (route_decode_smem_bytes(kv->max_pages, (int)W, k, kv->batch, kv->n_kv_heads) > 227 * 1024) return SA_ERR_UNSUPPORTED;
   SelectArgs sa_{};  // every field zero unless set below
   if (!fill_select(&sa_, kv, meta, rule, q, n_q_heads, G, &dummy, (int)W, kv_idx, kv_count, nullptr, ws))
     return SA_ERR_CUDA;
@@ -881,7 +882,7 @@ sa_status sparse_attn_route_decode_step(const sa_kv_desc* kv, void* meta, sa_sco
   if (2 * units > kMaxUnits) return SA_ERR_UNSUPPORTED;  // unit flags + split counters
   const unsigned long long kv_rows = (unsigned long long)kv->batch * kv->n_kv_heads * kv->cap_tokens;
   if (kv_rows > 0x7fffffffULL) return SA_ERR_UNSUPPORTED;
-  if (route_decode_smem_bytes(kv->max_pages, (int)W, k, kv->batch) >
+  if (route_decode_smem_bytes(kv->max_pages, (int)W, k, kv->batch, kv->n_kv_heads) >
       (size_t)(kv->max_pages * 8 > 65536 ? kv->max_pages * 8 : 65536))
     return SA_ERR_UNSUPPORTED;  // the selection's keys and candidates live in the step's ring
   if (step_smem_bytes(kv->max_pages, (int)W, false) > 227 * 1024) return SA_ERR_UNSUPPORTED;
@@ -893,7 +894,9 @@ sa_status sparse_attn_route_decode_step(const sa_kv_desc* kv, void* meta, sa_sco
   DecodePlan plan{sb + se, (int)units, sb + se, units * (sb + se)};
   const size_t sel_bytes = select_scratch(kv);
   const size_t rt_bytes = route_decode_ws_bytes(units);
-  const size_t need = kScratch + sel_bytes + rt_bytes + decode_scratch(plan);
+  // partial slots: sb + se per unit and the unit's merged top-k window
+  const size_t need = kScratch + sel_bytes + rt_bytes +
+                      decode_scratch(DecodePlan{sb + se, (int)units, sb + se, units * (sb + se + 1)});
   if ((s = check_ws(ws, ws_bytes, need)) != SA_OK) return s;
 
   RouteStepArgs ra{};  // every field zero unless set below
@@ -937,6 +940,7 @@ sa_status sparse_attn_route_decode_step(const sa_kv_desc* kv, void* meta, sa_sco
   char* rbase = w + kScratch + sel_bytes;
   r.ws_sigma = reinterpret_cast<double*>(rbase);
   r.ws_elig = reinterpret_cast<int32_t*>(rbase + align256((size_t)units * 8));
+  r.trig_list = reinterpret_cast<int4*>(rbase + align256((size_t)units * 8) + align256((size_t)units * 4));
   r.status = reinterpret_cast<int*>(ws);
   ra.routed = reinterpret_cast<uint32_t*>(w + kQueueRouteStep);
   const long long n_score = units * a.sel.splits;

@@ -173,6 +173,19 @@ SA_DEV uint32_t atom_add_acq_rel_u32(uint32_t* p, uint32_t v) {
   return old;
 }
 
+// A GPU-scope fence, and the relaxed (strong) store and add that, after it,
+// publish what the fence ordered before them -- two signals for the cost of
+// one fence; the consumer of the add's count fences again to acquire.
+SA_DEV void fence_acq_rel_gpu() { asm volatile("fence.acq_rel.gpu;\n" ::: "memory"); }
+SA_DEV void st_relaxed_u32(uint32_t* p, uint32_t v) {
+  asm volatile("st.relaxed.gpu.global.u32 [%0], %1;\n" ::"l"(p), "r"(v) : "memory");
+}
+SA_DEV uint32_t atom_add_relaxed_u32(uint32_t* p, uint32_t v) {
+  uint32_t old;
+  asm volatile("atom.relaxed.gpu.global.add.u32 %0, [%1], %2;\n" : "=r"(old) : "l"(p), "r"(v) : "memory");
+  return old;
+}
+
 // GPU-scope acquire load / release store of a 32-bit flag in global memory.
 SA_DEV uint32_t ld_acquire_u32(const uint32_t* p) {
   uint32_t v;

@@ -129,9 +129,11 @@ SA_DEV void store_out(const DecodeArgs& a, size_t row, int d0, const float (&A)[
 // microsecond under full HBM load).  base = slot 0 of the unit, head h;
 // LOCAL: the partials are in (this CTA's) shared memory, else in global
 // memory written earlier in the launch.  The same arithmetic either way.
+// part_out (non-null, head h's row of a partial slot): the merged partial is
+// stored there too, unnormalised, like a split's.
 template <bool LOCAL>
 SA_DEV void merge_splits(const DecodeArgs& a, const float* base, const int splits, const size_t out_row,
-                         const int d0) {
+                         const int d0, float* part_out = nullptr) {
   const float ninf = -__int_as_float(0x7f800000);
   float MM = ninf, LL = 0.f, AA[kDimsPerThread];
 #pragma unroll
@@ -176,6 +178,67 @@ SA_DEV void merge_splits(const DecodeArgs& a, const float* base, const int split
   const float inv = LL > 0.f ? 1.f / LL : 0.f;
   store_out(a, out_row, d0, AA, inv);
   if (a.lse && d0 == 0) a.lse[out_row] = LL > 0.f ? MM * kLn2 + logf(LL) : ninf;
+  if (part_out != nullptr) {
+#pragma unroll
+    for (int x = 0; x < kDimsPerThread; x += 4)
+      *reinterpret_cast<float4*>(part_out + d0 + x) = make_float4(AA[x], AA[x + 1], AA[x + 2], AA[x + 3]);
+    if (d0 == 0) *reinterpret_cast<float2*>(part_out + kHeadDim) = make_float2(MM, LL);
+  }
+}
+
+// Routed lists (route_k > 0): a unit's top-k window runs in splits
+// [0, sb) and its expansion window, decoded only for a unit whose tile
+// triggered, in splits [sb, sb + se).  Partial slots per unit: sb + se + 1
+// ([0, sb) top-k splits, [sb] their merge, [sb + 1, ..) expansion splits).
+// One counter per unit: top-k splits add 1, expansion splits add 1 << 16,
+// the top-k merge adds 1 << 30.  The last top-k split merges its window and
+// writes the output (final unless the unit triggered) and the merged
+// partial; the final merge of a triggered unit (the top-k merge and the
+// expansion splits) falls to whichever of the last expansion split and the
+// top-k merge comes second in the counter's order.
+constexpr uint32_t kRouteExp = 1u << 16, kRouteBaseMerged = 1u << 30;
+SA_DEV int route_exp_count(uint32_t v) { return (int)((v >> 16) & 0x3fffu); }
+
+// Publish a routed split's partial and run the merges it falls to (see
+// kRouteExp).  The counter increments are acq_rel after a barrier: they
+// publish this CTA's partial and acquire the others'.
+SA_DEV void route_publish(const DecodeArgs& a, const int u, const int split, const int splits,
+                          const size_t slot0, const Smem& sm, const int h, const int G, const int d0,
+                          const size_t out_row, const float (&A)[kDimsPerThread], const float M, const float L) {
+  const int sb = a.route_base_splits, se = splits - sb;
+  const bool base = split < sb;
+  float* part = a.ws_part + (slot0 + (base ? split : split + 1)) * kPartStride;
+  if (h < G) {
+    float* dst = part + h * kPartHead;
+#pragma unroll
+    for (int x = 0; x < kDimsPerThread; x += 4)
+      *reinterpret_cast<float4*>(dst + d0 + x) = make_float4(A[x], A[x + 1], A[x + 2], A[x + 3]);
+    if (d0 == 0) *reinterpret_cast<float2*>(dst + kHeadDim) = make_float2(M, L);
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    const uint32_t prev = atom_add_acq_rel_u32(&a.ws_count[u], base ? 1u : kRouteExp);
+    // 1: merge the top-k window; 2: the final merge
+    *sm.last = base ? ((prev & 0xffffu) == (uint32_t)(sb - 1) ? 1 : 0)
+                    : (route_exp_count(prev) == se - 1 && (prev & kRouteBaseMerged) ? 2 : 0);
+  }
+  __syncthreads();
+  int what = *sm.last;
+  if (what == 1) {
+    if (h < G)
+      merge_splits<false>(a, a.ws_part + slot0 * kPartStride + h * kPartHead, sb, out_row, d0,
+                          se > 0 ? a.ws_part + (slot0 + sb) * kPartStride + h * kPartHead : nullptr);
+    if (se == 0) return;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      const uint32_t prev = atom_add_acq_rel_u32(&a.ws_count[u], kRouteBaseMerged);
+      *sm.last = route_exp_count(prev) == se ? 2 : 0;  // every expansion split already in
+    }
+    __syncthreads();
+    what = *sm.last;
+  }
+  if (what == 2 && h < G)
+    merge_splits<false>(a, a.ws_part + (slot0 + sb) * kPartStride + h * kPartHead, se + 1, out_row, d0);
 }
 
 // n_known >= 0: the unit's kept count, already read by the caller (the fused
@@ -240,8 +303,9 @@ SA_DEV void decode_item(const DecodeArgs& a, const int u, const int split, const
   // this unit's split count and first partial slot
   const bool coarse = u < a.fine_unit0;
   const int splits = coarse ? a.splits : a.splits_fine;
-  const size_t slot0 = coarse ? (size_t)u * a.splits
-                              : (size_t)a.fine_unit0 * a.splits + (size_t)(u - a.fine_unit0) * a.splits_fine;
+  const size_t slot0 = a.route_k > 0 ? (size_t)u * (a.splits + 1)
+                       : coarse ? (size_t)u * a.splits
+                                : (size_t)a.fine_unit0 * a.splits + (size_t)(u - a.fine_unit0) * a.splits_fine;
   int t_begin = (int)(((long long)T * split) / splits);
   int t_end = (int)(((long long)T * (split + 1)) / splits);
   if (a.route_k > 0) {  // routed lists: the top-k window, then the expansion window
@@ -495,6 +559,10 @@ SA_DEV void decode_item(const DecodeArgs& a, const int u, const int split, const
         *reinterpret_cast<float4*>(dst + d0 + x) = make_float4(A[x], A[x + 1], A[x + 2], A[x + 3]);
       if (d0 == 0) *reinterpret_cast<float2*>(dst + kHeadDim) = make_float2(M, L);
     }
+    return;
+  }
+  if (a.route_k > 0) {
+    route_publish(a, u, split, splits, slot0, sm, h, G, d0, out_row, A, M, L);
     return;
   }
   float* part = a.ws_part + (slot0 + split) * kPartStride;

@@ -210,6 +210,8 @@ struct RouteArgs {
   int32_t* ws_elig;           // [n_tiles][Hkv] eligible block counts
   uint32_t* ws_count;         // [n_tiles * Hkv] split counters (left zero)
   uint32_t* ws_final;         // [1] finalize counter (left zero)
+  int4* trig_list;            // routed decode step: the triggered (tile, KV head) pairs
+                              // {tile x Hkv + head, list count, sequence length, 0}; else null
   int* status;
 };
 // One decode step in one launch: newest-page metadata refresh, scoring,
@@ -264,7 +266,7 @@ int tile_attn_tc_mchunks(int vectors_per_tile);
 cudaError_t launch_route(const RouteArgs& a, cudaStream_t st);
 // Decode router tail: one CTA per (sequence, KV head) over dec_scores.
 cudaError_t launch_route_decode(const RouteArgs& a, cudaStream_t st);
-size_t route_decode_smem_bytes(int max_pages, int W, int k, int n_tiles);
+size_t route_decode_smem_bytes(int max_pages, int W, int k, int n_tiles, int Hkv);
 // Router scratch: keys, lists, sigma and eligible counts for n_tiles x Hkv.
 size_t route_ws_bytes(int n_tiles, int Hkv, int max_pages, int W);
 int route_splits(int vectors_per_tile);

@@ -602,18 +602,18 @@ size_t route_ws_bytes(int n_tiles, int Hkv, int max_pages, int W) {
   return al(tg * max_pages * 4) + al(tg * 8) + al(tg * 4);
 }
 
-size_t route_decode_smem_bytes(int max_pages, int W, int k, int n_tiles) {
+size_t route_decode_smem_bytes(int max_pages, int W, int k, int n_tiles, int Hkv) {
   int cap = W > k + 1 ? W : k + 1;
   if (cap > max_pages) cap = max_pages;
   int n2 = 1;
   while (n2 < cap) n2 <<= 1;
   const size_t sel = (((size_t)max_pages * 4 + 15) & ~(size_t)15) + (size_t)n2 * 8;
-  const size_t fin = (size_t)n_tiles * 16;
+  const size_t fin = finalize_smem_bytes(n_tiles, Hkv);
   return 16 + (sel > fin ? sel : fin);
 }
 
 cudaError_t launch_route_decode(const RouteArgs& a, cudaStream_t st) {
-  const size_t smem = route_decode_smem_bytes(a.kv.max_pages, a.W, a.k, a.n_tiles);
+  const size_t smem = route_decode_smem_bytes(a.kv.max_pages, a.W, a.k, a.n_tiles, a.kv.Hkv);
   const cudaError_t e = set_smem_attr((const void*)route_decode_kernel, smem);
   if (e != cudaSuccess) return e;
   return launch_pdl(route_decode_kernel, (unsigned)(a.n_tiles * a.kv.Hkv), kRdThreads, smem, st, a);

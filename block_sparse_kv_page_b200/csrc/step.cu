@@ -76,6 +76,20 @@ SA_DEV int wait_selected(const uint32_t* flag, int* status, uint32_t limit) {
   return -1;
 }
 
+// Wait until *flag is nonzero (acquire) and return it; 0 (and
+// SA_ERR_TIMEOUT) after `limit` polls.
+SA_DEV uint32_t wait_nonzero(const uint32_t* flag, int* status, uint32_t limit) {
+  uint32_t ns = 32;
+  for (uint32_t i = 0; i < limit; ++i) {
+    const uint32_t v = ld_acquire_u32(flag);
+    if (v != 0u) return v;
+    __nanosleep(ns);
+    if (ns < 256) ns <<= 1;
+  }
+  flag_status(status, SA_ERR_TIMEOUT);
+  return 0u;
+}
+
 // Wait until *count reaches `target` (acquire); false (and SA_ERR_TIMEOUT)
 // after `limit` polls.
 SA_DEV bool wait_count(const uint32_t* count, uint32_t target, int* status, uint32_t limit) {
@@ -348,26 +362,15 @@ __global__ void __launch_bounds__(kThreads, 1) step_cluster_kernel(const __grid_
 // max(rho k, k + 1) pages in rank order with sigma (the router's selection)
 // and publishes the unit's flag (with its list count); the CTA finishing the
 // last unit computes sigma_bar, the quantile threshold and the triggers,
-// trims the untriggered lists to k, and publishes the `routed` flag.  Then
-// [n_score, n_score + n_base) the top-k windows of the units' lists (each
-// waits for its unit's flag), then the expansion windows (each waits for the
-// routed flag; an untriggered unit's are empty).  The last CTA of a unit
-// merges every window's partials in split order.  Waits only ever point to
-// items handed out earlier that never wait, so none can deadlock.
-// Decode item j of the routed step: the top-k windows of every unit first
-// (route_base_splits per unit), then the expansion windows.
-SA_DEV void route_item_unit(const RouteStepArgs& ra, const int j, int& u, int& split) {
-  const int sb = ra.st.dec.route_base_splits, se = ra.st.dec.splits - sb;
-  if (j < ra.n_base) {
-    u = j / sb;
-    split = j - u * sb;
-  } else {
-    const int x = j - ra.n_base;
-    u = x / se;
-    split = sb + (x - u * se);
-  }
-}
-
+// trims the untriggered lists to k, lists the triggered units and publishes
+// the `routed` flag (1 + their number).  Then [n_score, n_score + n_base)
+// the top-k windows of the units' lists, unit by unit (each waits for its
+// unit's flag), then the expansion windows of the triggered units only (they
+// wait for the routed flag; the first item past them ends the CTA's work).
+// A unit's top-k windows merge when the last of them is done; a triggered
+// unit's expansion windows then merge onto that (decode_item.cuh,
+// kRouteExp).  Waits only ever point to items handed out earlier that never
+// wait, so none can deadlock.
 template <int RULE>
 __global__ void __launch_bounds__(kThreads, SA_STEP_CTAS_PER_SM)
     route_step_kernel(const __grid_constant__ RouteStepArgs ra) {
@@ -376,7 +379,7 @@ __global__ void __launch_bounds__(kThreads, SA_STEP_CTAS_PER_SM)
   __shared__ uint32_t s_hist[512];
   __shared__ uint32_t s_scan[32];
   __shared__ uint32_t s_bc[8];
-  __shared__ int s_last, s_item, s_ntiles, s_count, s_ntok, s_flag;
+  __shared__ int s_last, s_item, s_ntiles, s_count, s_ntok, s_flag, s_unit, s_split;
   unsigned char* base = reinterpret_cast<unsigned char*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   const int body = body_bytes(a.sel.kv.max_pages);
@@ -405,20 +408,30 @@ __global__ void __launch_bounds__(kThreads, SA_STEP_CTAS_PER_SM)
   for (;;) {
     if (threadIdx.x == 0) {
       int item = (int)atomicAdd(&a.queue[0], 1u);
-      if (item >= a.n_score && item < n_items) {
-        int u, split;
-        route_item_unit(ra, item - a.n_score, u, split);
-        const int ntok = a.dec.kv.seq_len[u / a.dec.kv.Hkv];
-        int cnt;
-        if (item < n_pre) {  // top-k window: the unit's list is written
-          cnt = wait_selected(a.sel.ws_count + u, a.sel.status, limit);
-          if (cnt > ra.route.k) cnt = ra.route.k;
-        } else {             // expansion window: the triggers are known
-          cnt = wait_count(ra.routed + 1, 1u, a.sel.status, limit) ? __ldcg(a.dec.count + u) : -1;
-        }
+      if (item >= a.n_score && item < n_pre) {  // top-k window: once the unit's list is written
+        const int sb = a.dec.route_base_splits;
+        const int u = (item - a.n_score) / sb;
+        const int ntok = a.dec.kv.seq_len[u / a.dec.kv.Hkv];  // overlaps the acquire
+        int cnt = wait_selected(a.sel.ws_count + u, a.sel.status, limit);
+        if (cnt > ra.route.k) cnt = ra.route.k;
+        s_unit = u;
+        s_split = item - a.n_score - u * sb;
         s_count = cnt;
         s_ntok = ntok;
         if (cnt < 0) item = n_items;  // gave up: this CTA stops taking work
+      } else if (item >= n_pre && item < n_items) {  // expansion window of the q-th triggered unit
+        const int sb = a.dec.route_base_splits, se = a.dec.splits - sb;
+        const int x = item - n_pre, q = x / se;
+        const uint32_t v = wait_nonzero(ra.routed + 1, a.sel.status, limit);  // 1 + triggered units
+        if (v == 0u || q >= (int)v - 1) {
+          item = n_items;  // timed out, or past the last triggered unit: no more work here
+        } else {
+          const int4 e = __ldcg(ra.route.trig_list + q);
+          s_unit = e.x;
+          s_split = sb + (x - q * se);
+          s_count = e.y;
+          s_ntok = e.z;
+        }
       }
       s_item = item;
     }
@@ -445,20 +458,22 @@ __global__ void __launch_bounds__(kThreads, SA_STEP_CTAS_PER_SM)
         rsel::route_select_tile(ra.route, b, g, P, base, s_hist, s_bc, s_scan);
         __syncthreads();
         if (threadIdx.x == 0) {
-          st_release_u32(&a.sel.ws_count[u], sel::kUnitSelected | (uint32_t)ra.route.kv_count[u]);
-          s_flag = atom_add_acq_rel_u32(ra.routed, 1u) == (uint32_t)(units - 1);
+          // one fence publishes the list, count and sigma through both signals
+          fence_acq_rel_gpu();
+          st_relaxed_u32(&a.sel.ws_count[u], sel::kUnitSelected | (uint32_t)ra.route.kv_count[u]);
+          s_flag = atom_add_relaxed_u32(ra.routed, 1u) == (uint32_t)(units - 1);
+          if (s_flag) fence_acq_rel_gpu();  // the last unit: acquire every unit's sigma and count
         }
         __syncthreads();
-        if (s_flag) {  // every unit selected: quantile, triggers, trimmed lists
-          rsel::route_finalize(ra.route, base);
-          __syncthreads();
-          if (threadIdx.x == 0) st_release_u32(ra.routed + 1, 1u);
+        if (s_flag) {  // every unit selected: quantile, triggers, the triggered units
+          double tau;
+          const int n_trig = rsel::route_triggers(ra.route, base, tau);
+          if (threadIdx.x == 0) st_release_u32(ra.routed + 1, 1u + (uint32_t)n_trig);
+          rsel::route_outputs(ra.route, base, tau);  // read by no decode item
         }
       }
     } else {
-      int u, split;
-      route_item_unit(ra, item - a.n_score, u, split);
-      dec::decode_item<false>(a.dec, u, split, D, ws, s_count, s_ntok);
+      dec::decode_item<false>(a.dec, s_unit, s_split, D, ws, s_count, s_ntok);
     }
     fence_proxy_async();  // generic writes to the ring (keys, merge) before the next TMA writes
     __syncthreads();
