@@ -414,11 +414,14 @@ size_t sparse_attn_workspace_size(const sa_kv_desc* kv, int32_t n_q_heads, int32
   if (kv->batch <= kMaxRouteTiles && kv->page_size > 0) {  // decode router: scores + router scratch
     const long long ru = (long long)kv->batch * kv->n_kv_heads;
     size_t rd = select_scratch(kv) + route_decode_ws_bytes(ru);
-    // the routed decode step adds split partials of its top-k and expansion
-    // windows, each at most the splits of a plain decode over max_sel, and
-    // one merged top-k partial per unit
+    // the routed decode step adds split partials of its top-k windows (at
+    // most the splits of a plain decode over max_sel), of its expansion
+    // windows (planned for as few as one row's units) and one merged top-k
+    // partial per unit
     const DecodePlan rp = decode_plan((int)ru, max_tiles_per_unit(kv, max_sel), sm);
-    rd += decode_scratch(DecodePlan{2 * rp.splits, (int)ru, 2 * rp.splits, ru * (2 * rp.splits + 1)});
+    const DecodePlan ep = decode_plan(kv->n_kv_heads, max_tiles_per_unit(kv, max_sel), sm);
+    const int rs = rp.splits + ep.splits;
+    rd += decode_scratch(DecodePlan{rs, (int)ru, rs, ru * (rs + 1)});
     if (rd > tail) tail = rd;
   }
   return kScratch + tail;
@@ -890,7 +893,16 @@ sa_status sparse_attn_route_decode_step(const sa_kv_desc* kv, void* meta, sa_sco
   const int sm = device_sm_count();
   const int sub = kv->page_size / 16;
   const int sb = decode_plan((int)units, k * sub, sm).splits;
-  const int se = W > k ? decode_plan((int)units, (int)(W - k) * sub, sm).splits : 0;
+  // expansion windows: split for the units expected to trigger (the rows
+  // below the q-quantile; every unit when the threshold is given), so the
+  // last items of the launch stay short
+  long long trig_units = units;
+  if (tau == nullptr) {
+    const long long rows = (long long)std::ceil((double)quantile * kv->batch);
+    trig_units = (rows < 1 ? 1 : rows) * kv->n_kv_heads;
+    if (trig_units > units) trig_units = units;
+  }
+  const int se = W > k ? decode_plan((int)trig_units, (int)(W - k) * sub, sm).splits : 0;
   DecodePlan plan{sb + se, (int)units, sb + se, units * (sb + se)};
   const size_t sel_bytes = select_scratch(kv);
   const size_t rt_bytes = route_decode_ws_bytes(units);
