@@ -193,6 +193,9 @@ SA_DEV void bitonic_sort_desc(unsigned long long* cand, const int n_sel) {
   }
 }
 
+SA_DEV void route_select_finish(const RouteArgs& a, const int tg, const int E, unsigned long long* cand,
+                                const int n_sel);
+
 // ---------------------------------------------------------------- selection for one (t, g)
 SA_DEV void route_select_tile(const RouteArgs& a, int t, int g, int E, unsigned char* smem,
                               uint32_t* hist, uint32_t* bc, uint32_t* scan) {
@@ -251,6 +254,16 @@ SA_DEV void route_select_tile(const RouteArgs& a, int t, int g, int E, unsigned 
     }
     n_sel = cap;
   }
+  route_select_finish(a, tg, E, cand, n_sel);
+}
+
+// The rest of a (tile, KV head)'s selection, from its n_sel candidates in
+// cand (composite keys, any order; the top max(rho k, k + 1) of its E
+// eligible blocks): rank order, sigma, the list as if the tile triggered
+// and its count.  All threads of the CTA call it.
+SA_DEV void route_select_finish(const RouteArgs& a, const int tg, const int E, unsigned long long* cand,
+                                const int n_sel) {
+  const int tid = threadIdx.x;
   // rank order: descending composite key = (score key, ~index); sorted runs
   // merged by rank when they fit the CTA's warps, else a bitonic sort
   __syncthreads();

@@ -216,10 +216,19 @@ SA_DEV uint32_t bin_slot(uint32_t b) {  // physical word of bin b in a 4096-bin 
   return (r << 5) | ((((w >> 2) ^ (r & 7u)) << 2) | (w & 3u));
 }
 
+// cand (non-null, shared memory past the first 36 KiB of S.ring): instead of
+// sel_idx and sel_count, the kept pages go to cand[0 .. kept) in page order
+// as composite keys (score key << 32 | ~page, the router's rank-order key).
+constexpr int kCandOffset = 36 * 1024;
+static_assert(2 * 4096 * 4 + 128 * 4 + 16 * 4 <= kCandOffset, "bins, row sums and warp totals stay below cand");
+SA_DEV unsigned long long cand_key(uint32_t key, int p) {
+  return ((unsigned long long)key << 32) | (0xffffffffu - (uint32_t)p);
+}
 template <int KPT, bool WEIGHTED>
 SA_DEV void select_unit_regs(const SelectArgs& a, const int u, const int N, const int P,
                              const uint32_t cap, const int forced_lo, const int forced_hi,
-                             const int32_t* off, const SelSmem& S, const float* sc_local) {
+                             const int32_t* off, const SelSmem& S, const float* sc_local,
+                             unsigned long long* cand = nullptr) {
   static_assert(KPT % 4 == 0 && KPT <= 32, "pages per thread");
   static_assert(kThreads == 128, "the register path maps 4096 bins onto 128 threads");
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -290,6 +299,12 @@ SA_DEV void select_unit_regs(const SelectArgs& a, const int u, const int N, cons
   }
   int32_t* sel_u = a.sel_idx + (size_t)u * a.max_sel;
   if (wall <= cap) {  // everything fits
+    if (cand != nullptr) {
+#pragma unroll
+      for (int i = 0; i < KPT; ++i)
+        if (valid >> i & 1u) cand[p0 + i] = cand_key(key[i], p0 + i);
+      return;
+    }
 #pragma unroll
     for (int i = 0; i < KPT; ++i)
       if ((valid >> i & 1u) && p0 + i < a.max_sel) sel_u[p0 + i] = p0 + i;
@@ -423,6 +438,12 @@ SA_DEV void select_unit_regs(const SelectArgs& a, const int u, const int N, cons
       if (k) keep |= 1u << i;
     }
     pos = block_excl_scan((uint32_t)__popc(keep), S.scan, total);
+  }
+  if (cand != nullptr) {
+#pragma unroll
+    for (int i = 0; i < KPT; ++i)
+      if (keep >> i & 1u) cand[pos++] = cand_key(key[i], p0 + i);
+    return;
   }
 #pragma unroll
   for (int i = 0; i < KPT; ++i)

@@ -48,6 +48,8 @@ static_assert(sel::kWarps == dec::kWarps, "one CTA shape for both item kinds");
 static_assert(sel::kStages == dec::kStages && sel::kTileBytes == dec::kTileBytes,
               "both item kinds use the same per-warp ring");
 
+static_assert(sel::kCandOffset + 16 * sel::kWarps * 32 * 8 <= sel::kRingBytes,
+              "the routed step's candidates (and their bitonic fallback) fit the ring");
 constexpr int kWarps = sel::kWarps;
 constexpr int kThreads = kWarps * 32;
 constexpr int kStages = sel::kStages;
@@ -455,7 +457,17 @@ __global__ void __launch_bounds__(kThreads, SA_STEP_CTAS_PER_SM)
         int N, P;
         sel::unit_geometry(a.sel, b, N, P);
         fence_proxy_async();  // the ring becomes the selection's keys
-        rsel::route_select_tile(ra.route, b, g, P, base, s_hist, s_bc, s_scan);
+        if (P <= 16 * kThreads) {
+          // the plain step's register selection finds the candidates (keys
+          // above the cut, then equal keys in page order), the router's code
+          // ranks them and computes sigma
+          const int cap = min(max(ra.route.W, ra.route.k + 1), P);
+          auto* cand = reinterpret_cast<unsigned long long*>(base + sel::kCandOffset);
+          sel::select_unit_regs<16, false>(a.sel, u, N, P, (uint32_t)cap, 0, P, nullptr, S, nullptr, cand);
+          rsel::route_select_finish(ra.route, u, P, cand, cap);
+        } else {
+          rsel::route_select_tile(ra.route, b, g, P, base, s_hist, s_bc, s_scan);
+        }
         __syncthreads();
         if (threadIdx.x == 0) {
           // one fence publishes the list, count and sigma through both signals
