@@ -113,6 +113,30 @@ def test_route_decode_parity(cuda_dev, H, rule, ps, k, rho, quantile, tau):
     print(f"\n{rule} ps={ps} k={k} rho={rho}: {stats}, triggered {int(g_res['triggered'].sum())}/{B}")
 
 
+@pytest.mark.parametrize("rule", ["envelope", "centroid"])
+@pytest.mark.parametrize("k,rho", [(96, 3), (128, 4)])
+def test_route_decode_long_lists_rank_order(cuda_dev, H, rule, k, rho):
+    """Lists of 288 and 512 entries (the rank order is built from three and
+    four sorted runs of 128 keys) through the separate calls and the
+    one-launch step, both against the oracle: sets and rank order with the
+    near-tie certificate, sigma, triggers, and the attention over the
+    lists."""
+    import block_sparse_kv_page_b200 as sa
+    rng = np.random.default_rng(977 + k)
+    B = 16
+    lens = [int(x) for x in rng.integers(5000, 8000, size=B)]
+    lens[5] = 1900  # 119 pages: one run
+    lay = DG.make_decode_layer(B=B, Hq=32, Hkv=4, seq_lens=lens, seed=907 + k, device=cuda_dev,
+                               cap=8000, key_scale="channel")
+    kw = dict(rule=rule, ps=16, k=k, rho=rho, quantile=0.25, tau=None)
+    ref = _oracle(H, lay, **kw)
+    for g_res in (_run_gpu(sa, lay, **kw), _run_gpu_step(sa, lay, **kw)):
+        assert g_res["status"] == 0
+        H.compare(g_res, ref, k=k, rho=rho)
+        assert g_res["triggered"].any()
+        _check_attention(H, lay, g_res, 16)
+
+
 def test_route_decode_rejects_bad_arguments(cuda_dev):
     import block_sparse_kv_page_b200 as sa
     lay = DG.make_decode_layer(B=2, Hq=32, Hkv=4, seq_lens=[300, 200], seed=811, device=cuda_dev)
