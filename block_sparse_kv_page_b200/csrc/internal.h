@@ -235,8 +235,9 @@ cudaError_t launch_step(const StepArgs& a, cudaStream_t st);
 struct RouteStepArgs {
   StepArgs st;                // sel: score-only scoring; dec: route_k/w set, idx/count = the lists
   RouteArgs route;            // dec_scores = the group scores; tiles = the sequences
-  uint32_t* routed;           // [2]: units selected so far, triggers published (flag)
-  int n_base;                 // decode items of the top-k windows (unit order), then the expansions
+  uint32_t* routed;           // [2]: units selected so far; 1 + the triggered units, once published
+  int n_base;                 // decode items of the top-k windows (unit order), then the
+                              // expansion windows of the triggered units (route.trig_list order)
 };
 cudaError_t launch_route_step(const RouteStepArgs& a, cudaStream_t st);
 // Few units: one cluster of C CTAs per unit (sel.splits must be C).

@@ -335,10 +335,12 @@ sa_status sparse_attn_decode_step_wait_test(const sa_kv_desc* kv, void* meta, sa
 
 /* The router applied to decode and the decode over its lists, in ONE launch
  * ("Onzekerheidsgestuurde Selectie voor Blok-schaarse Aandacht",
- * "Methodologie" steps 1-5 on one-row tiles; the same results as
- * sparse_attn_route_decode followed by sparse_attn_decode over kv_idx /
- * kv_count, after the newest page's metadata is refreshed as in
- * sparse_attn_decode_step).  meta is read and its newest page rewritten.
+ * "Methodologie" steps 1-5 on one-row tiles; what sparse_attn_route_decode
+ * followed by sparse_attn_decode over kv_idx / kv_count computes, after the
+ * newest page's metadata is refreshed as in sparse_attn_decode_step: the
+ * lists, sigma, sigma_bar, tau and triggers exactly, out and lse up to
+ * rounding, as the attention runs in a top-k and an expansion window merged
+ * in two steps).  meta is read and its newest page rewritten.
  * Outputs: kv_idx / kv_count / sigma / sigma_bar / triggered / tau_out as
  * sparse_attn_route_decode (lists in rank order, -1 padded), out fp32
  * [B][Hq][128] and lse (nullable) as sparse_attn_decode.  Every unit's top k
