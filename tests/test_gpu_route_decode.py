@@ -114,20 +114,23 @@ def test_route_decode_parity(cuda_dev, H, rule, ps, k, rho, quantile, tau):
 
 
 @pytest.mark.parametrize("rule", ["envelope", "centroid"])
-@pytest.mark.parametrize("k,rho", [(96, 3), (128, 4)])
+@pytest.mark.parametrize("k,rho", [(96, 3), (128, 4), (200, 3)])
 def test_route_decode_long_lists_rank_order(cuda_dev, H, rule, k, rho):
-    """Lists of 288 and 512 entries (the rank order is built from three and
-    four sorted runs of 128 keys) through the separate calls and the
+    """Lists of 288, 512 and 600 entries through the separate calls and the
     one-launch step, both against the oracle: sets and rank order with the
-    near-tie certificate, sigma, triggers, and the attention over the
-    lists."""
+    near-tie certificate, sigma, triggers, and the attention over the lists.
+    Up to 512 candidates the rank order is built from sorted runs of 128
+    keys (three or four runs here); 600 is past what the one-launch step's
+    four warps hold, so it takes the bitonic sort there (the separate call's
+    sixteen warps still merge runs)."""
     import block_sparse_kv_page_b200 as sa
     rng = np.random.default_rng(977 + k)
     B = 16
-    lens = [int(x) for x in rng.integers(5000, 8000, size=B)]
+    top = 8000 if rho * k <= 512 else 12000
+    lens = [int(x) for x in rng.integers(top - 3000, top, size=B)]
     lens[5] = 1900  # 119 pages: one run
     lay = DG.make_decode_layer(B=B, Hq=32, Hkv=4, seq_lens=lens, seed=907 + k, device=cuda_dev,
-                               cap=8000, key_scale="channel")
+                               cap=top, key_scale="channel")
     kw = dict(rule=rule, ps=16, k=k, rho=rho, quantile=0.25, tau=None)
     ref = _oracle(H, lay, **kw)
     for g_res in (_run_gpu(sa, lay, **kw), _run_gpu_step(sa, lay, **kw)):
