@@ -140,6 +140,29 @@ def test_route_decode_long_lists_rank_order(cuda_dev, H, rule, k, rho):
         _check_attention(H, lay, g_res, 16)
 
 
+@pytest.mark.parametrize("B,quantile,tau", [(1, 0.25, None), (2, 0.9, None), (3, 0.5, None), (3, 0.5, 1.5)])
+def test_route_decode_step_small_batches(cuda_dev, H, B, quantile, tau):
+    """The one-launch routed step on 1-3 sequences (the quantile over so few
+    rows, none or every row triggered, the expansion splits planned for
+    one row's units) against the oracle and the separate calls."""
+    import block_sparse_kv_page_b200 as sa
+    rng = np.random.default_rng(31 + B)
+    lens = [int(x) for x in rng.integers(900, 3000, size=B)]
+    lay = DG.make_decode_layer(B=B, Hq=32, Hkv=4, seq_lens=lens, seed=611 + B, device=cuda_dev,
+                               cap=3000, key_scale="channel")
+    kw = dict(rule="envelope", ps=16, k=24, rho=2, quantile=quantile, tau=tau)
+    ref = _oracle(H, lay, **kw)
+    g_step = _run_gpu_step(sa, lay, **kw)
+    g_sep = _run_gpu(sa, lay, **kw)
+    for g_res in (g_step, g_sep):
+        assert g_res["status"] == 0
+        H.compare(g_res, ref, k=24, rho=2)
+        _check_attention(H, lay, g_res, 16)
+    for key in ("kv_idx", "kv_count", "triggered"):
+        assert np.array_equal(g_step[key], g_sep[key]), key
+    assert float((g_step["out"] - g_sep["out"]).abs().max()) < 1e-5
+
+
 def test_route_decode_rejects_bad_arguments(cuda_dev):
     import block_sparse_kv_page_b200 as sa
     lay = DG.make_decode_layer(B=2, Hq=32, Hkv=4, seq_lens=[300, 200], seed=811, device=cuda_dev)
